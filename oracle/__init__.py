@@ -1,0 +1,183 @@
+"""Float64 CPU oracle for the selective scan -- TEST INFRASTRUCTURE ONLY.
+
+Only the tests, ``__graft_entry__.smoke()`` and the bench's CPU-baseline leg
+may import this package.  The CUDA library never calls it.  The arithmetic
+lives in ``ssm_oracle.c`` (plain loops in double precision); this module only
+compiles it with gcc, loads it with ctypes and converts arrays to float64.
+
+Functions (all return float64 numpy arrays):
+
+* ``s6(inp, reverse=False, ...)``      -- one direction (the per-step scan,
+  with skip term and SiLU gate)
+* ``bidir(inp, ...)``                  -- forward + reversed with separate
+  parameters, summed
+* ``ssd_seq(inp, ...)``                -- Mamba2 SSD as the sequential scan
+  with a scalar A per head
+* ``ssd_chunked(inp, chunk, ...)``     -- Mamba2 SSD in the chunked form
+  (matrix products inside chunks, state passed between chunks)
+
+``cols`` restricts the work to some columns (b*D + d for S6,
+(b*H + h)*P + p for SSD); other outputs are left at zero.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Sequence, Tuple
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ssm_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+_dp = ctypes.POINTER(ctypes.c_double)
+_ip = ctypes.POINTER(ctypes.c_int64)
+_i64 = ctypes.c_int64
+
+
+def build(force: bool = False) -> str:
+    """Compile ssm_oracle.c into liboracle.so (plain -O2, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fno-fast-math", "-fPIC", "-shared", "-fopenmp",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        lib.oracle_s6.argtypes = [_i64] * 4 + [_dp, _dp, _dp, ctypes.c_int, _dp, _dp, _dp, _dp, _dp,
+                                               ctypes.c_int, _dp, _dp, _ip, _i64, ctypes.c_int]
+        lib.oracle_bidir.argtypes = ([_i64] * 4 + [_dp, _dp, ctypes.c_int] + [_dp] * 7 + [_dp] * 7
+                                     + [_dp, _ip, _i64, ctypes.c_int])
+        lib.oracle_ssd_seq.argtypes = [_i64] * 5 + [_dp, _dp, _dp, ctypes.c_int, _dp, _dp, _dp, _dp,
+                                                    _dp, _dp, _dp, _ip, _i64, ctypes.c_int]
+        lib.oracle_ssd_chunked.argtypes = [_i64] * 6 + [_dp, _dp, _dp, ctypes.c_int, _dp, _dp, _dp,
+                                                        _dp, _dp, _dp, _dp, ctypes.c_int]
+        lib.oracle_max_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def max_threads() -> int:
+    return int(_load().oracle_max_threads())
+
+
+def _f64(a) -> Optional[np.ndarray]:
+    if a is None:
+        return None
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(_dp)
+
+
+def _cols(cols):
+    if cols is None:
+        return None, None, 0
+    c = np.ascontiguousarray(np.asarray(cols, dtype=np.int64))
+    return c, c.ctypes.data_as(_ip), len(c)
+
+
+def s6_arrays(x, delta, A, B, C, *, delta_bias=None, softplus=True, D=None, z=None,
+              reverse=False, cols=None, want_state=True, nthreads=1
+              ) -> Tuple[np.ndarray, Optional[np.ndarray]]:
+    """Single-direction S6 on raw arrays: returns (out (B,L,D), last_state (B,D,N))."""
+    x, delta, A, B, C = map(_f64, (x, delta, A, B, C))
+    delta_bias, D, z = map(_f64, (delta_bias, D, z))
+    Bsz, L, Dm = x.shape
+    N = A.shape[1]
+    out = np.zeros((Bsz, L, Dm))
+    st = np.zeros((Bsz, Dm, N)) if want_state else None
+    keep, cp, nc = _cols(cols)
+    _load().oracle_s6(Bsz, L, Dm, N, _ptr(x), _ptr(delta), _ptr(delta_bias), int(softplus),
+                      _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), int(reverse), _ptr(out),
+                      _ptr(st), cp, nc, int(nthreads))
+    return out, st
+
+
+def s6(inp, reverse=False, cols=None, softplus=True, nthreads=1):
+    """S6 on an ssm_gen.S6Inputs, forward-direction parameters."""
+    return s6_arrays(inp.x, inp.delta, inp.A_f, inp.B_f, inp.C_f, delta_bias=inp.dt_bias_f,
+                     softplus=softplus, D=inp.D_f, z=inp.z_f, reverse=reverse, cols=cols,
+                     nthreads=nthreads)
+
+
+def bidir_arrays(x, delta, fwd: dict, bwd: dict, *, softplus=True, cols=None, nthreads=1):
+    """Bidirectional scan on raw arrays.
+
+    fwd / bwd: dicts with keys delta_bias, A, B, C, D, z (delta_bias, D, z may
+    be None).  Returns (out, last_state_f, last_state_b).
+    """
+    x, delta = _f64(x), _f64(delta)
+    Bsz, L, Dm = x.shape
+    N = np.asarray(fwd["A"]).shape[1]
+    out = np.zeros((Bsz, L, Dm))
+    lf = np.zeros((Bsz, Dm, N))
+    lb = np.zeros((Bsz, Dm, N))
+    f = {k: _f64(fwd.get(k)) for k in ("delta_bias", "A", "B", "C", "D", "z")}
+    b = {k: _f64(bwd.get(k)) for k in ("delta_bias", "A", "B", "C", "D", "z")}
+    keep, cp, nc = _cols(cols)
+    _load().oracle_bidir(Bsz, L, Dm, N, _ptr(x), _ptr(delta), int(softplus),
+                         _ptr(f["delta_bias"]), _ptr(f["A"]), _ptr(f["B"]), _ptr(f["C"]),
+                         _ptr(f["D"]), _ptr(f["z"]), _ptr(lf),
+                         _ptr(b["delta_bias"]), _ptr(b["A"]), _ptr(b["B"]), _ptr(b["C"]),
+                         _ptr(b["D"]), _ptr(b["z"]), _ptr(lb),
+                         _ptr(out), cp, nc, int(nthreads))
+    return out, lf, lb
+
+
+def bidir(inp, cols=None, softplus=True, nthreads=1):
+    """Bidirectional scan on an ssm_gen.S6Inputs with bidir=True."""
+    fwd = dict(delta_bias=inp.dt_bias_f, A=inp.A_f, B=inp.B_f, C=inp.C_f, D=inp.D_f, z=inp.z_f)
+    bwd = dict(delta_bias=inp.dt_bias_b, A=inp.A_b, B=inp.B_b, C=inp.C_b, D=inp.D_b, z=inp.z_b)
+    return bidir_arrays(inp.x, inp.delta, fwd, bwd, softplus=softplus, cols=cols, nthreads=nthreads)
+
+
+def ssd_seq_arrays(x, delta, A, B, C, *, delta_bias=None, softplus=True, D=None, z=None,
+                   cols=None, nthreads=1):
+    """SSD by the sequential recurrence: returns (out (B,L,H,P), last_state (B,H,P,N))."""
+    x, delta, A, B, C = map(_f64, (x, delta, A, B, C))
+    delta_bias, D, z = map(_f64, (delta_bias, D, z))
+    Bsz, L, H, P = x.shape
+    N = B.shape[2]
+    out = np.zeros((Bsz, L, H, P))
+    st = np.zeros((Bsz, H, P, N))
+    keep, cp, nc = _cols(cols)
+    _load().oracle_ssd_seq(Bsz, L, H, P, N, _ptr(x), _ptr(delta), _ptr(delta_bias), int(softplus),
+                           _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(out), _ptr(st),
+                           cp, nc, int(nthreads))
+    return out, st
+
+
+def ssd_seq(inp, cols=None, softplus=True, nthreads=1):
+    return ssd_seq_arrays(inp.x, inp.delta, inp.A, inp.B, inp.C, delta_bias=inp.dt_bias,
+                          softplus=softplus, D=inp.D, z=inp.z, cols=cols, nthreads=nthreads)
+
+
+def ssd_chunked_arrays(x, delta, A, B, C, chunk, *, delta_bias=None, softplus=True, D=None,
+                       z=None, nthreads=1):
+    """SSD by the chunked form: returns (out (B,L,H,P), last_state (B,H,P,N))."""
+    x, delta, A, B, C = map(_f64, (x, delta, A, B, C))
+    delta_bias, D, z = map(_f64, (delta_bias, D, z))
+    Bsz, L, H, P = x.shape
+    N = B.shape[2]
+    out = np.zeros((Bsz, L, H, P))
+    st = np.zeros((Bsz, H, P, N))
+    _load().oracle_ssd_chunked(Bsz, L, H, P, N, int(chunk), _ptr(x), _ptr(delta),
+                               _ptr(delta_bias), int(softplus), _ptr(A), _ptr(B), _ptr(C),
+                               _ptr(D), _ptr(z), _ptr(out), _ptr(st), int(nthreads))
+    return out, st
+
+
+def ssd_chunked(inp, chunk=None, softplus=True, nthreads=1):
+    return ssd_chunked_arrays(inp.x, inp.delta, inp.A, inp.B, inp.C,
+                              inp.chunk if chunk is None else chunk, delta_bias=inp.dt_bias,
+                              softplus=softplus, D=inp.D, z=inp.z, nthreads=nthreads)

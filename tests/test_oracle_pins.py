@@ -1,0 +1,309 @@
+"""Pins for the float64 oracle, each independent of the oracle's own code.
+
+The pages print no numeric worked example for the scan, so the oracle is
+pinned by a hand-derived tiny case (tests/golden/s6_tiny.json), by closed
+forms evaluated by brute force, by the LTI convolution identity, by symmetry
+(reversal = flip, bidirectional = sum of directions), by the SSD chunked form
+against the sequential definition, and by special cases that reduce to
+textbook values.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import ssm_gen
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+RTOL = 1e-11
+
+
+def _softplus(v):
+    return np.logaddexp(0.0, v)
+
+
+def _silu(z):
+    return z * (1.0 / (1.0 + np.exp(-z)))
+
+
+def _rand_case(rng, Bz, L, Dm, N, gate=True):
+    x = rng.standard_normal((Bz, L, Dm))
+    delta = 0.5 * rng.standard_normal((Bz, L, Dm))
+    bias = rng.uniform(-4.0, 0.0, Dm)
+    A = -np.exp(rng.uniform(-1.0, 2.0, (Dm, N)))
+    B = rng.standard_normal((Bz, L, N))
+    C = rng.standard_normal((Bz, L, N))
+    D = rng.uniform(0.5, 1.5, Dm)
+    z = rng.standard_normal((Bz, L, Dm)) if gate else None
+    return x, delta, bias, A, B, C, D, z
+
+
+def _closed_form(x, delta, bias, A, B, C, D, z, reverse):
+    """y_t = sum_{s<=t} sum_n C_t[n] (prod_{s<k<=t} exp(dt_k A[d,n])) dt_s B_s[n] x_s
+    (+ D x_t, times silu(z_t)); for the reverse scan s >= t and the product
+    runs over t <= k < s.  Evaluated term by term."""
+    Bz, L, Dm = x.shape
+    N = A.shape[1]
+    dt = _softplus(delta + bias[None, None, :])
+    y = np.zeros_like(x)
+    for b in range(Bz):
+        for d in range(Dm):
+            for t in range(L):
+                acc = 0.0
+                srange = range(0, t + 1) if not reverse else range(t, L)
+                for s in srange:
+                    for n in range(N):
+                        if not reverse:
+                            ks = range(s + 1, t + 1)
+                        else:
+                            ks = range(t, s)
+                        decay = 1.0
+                        for k in ks:
+                            decay *= math.exp(dt[b, k, d] * A[d, n])
+                        acc += C[b, t, n] * decay * dt[b, s, d] * B[b, s, n] * x[b, s, d]
+                acc += D[d] * x[b, t, d]
+                if z is not None:
+                    acc *= _silu(z[b, t, d])
+                y[b, t, d] = acc
+    return y
+
+
+def _close(a, b, rtol=RTOL):
+    scale = max(np.max(np.abs(b)), 1e-300)
+    err = np.max(np.abs(a - b)) / scale
+    assert err < rtol, f"normwise error {err:.3e} > {rtol:.1e}"
+
+
+def test_hand_worked_example():
+    g = json.load(open(os.path.join(HERE, "golden", "s6_tiny.json")))
+    for case in g["cases"]:
+        x = np.array(case["x"], float).reshape(1, 3, 1)
+        delta = np.full((1, 3, 1), case["dt"])
+        A = np.array([[case["A"]]])
+        B = np.full((1, 3, 1), case["B"])
+        C = np.full((1, 3, 1), case["C"])
+        D = np.array([case["D"]])
+        y, st = oracle.s6_arrays(x, delta, A, B, C, softplus=False, D=D, z=None,
+                                 reverse=case["reverse"])
+        np.testing.assert_allclose(y.ravel(), case["y"], rtol=1e-14, atol=1e-14)
+        np.testing.assert_allclose(st.ravel(), [case["last_state"]], rtol=1e-14)
+
+
+@pytest.mark.parametrize("N", [1, 3, 16])
+@pytest.mark.parametrize("reverse", [False, True])
+def test_closed_form_brute_force(N, reverse):
+    rng = np.random.default_rng(100 + N + 7 * reverse)
+    Bz, L, Dm = 2, 9, 3
+    x, delta, bias, A, B, C, D, z = _rand_case(rng, Bz, L, Dm, N)
+    y, _ = oracle.s6_arrays(x, delta, A, B, C, delta_bias=bias, softplus=True, D=D, z=z,
+                            reverse=reverse)
+    ref = _closed_form(x, delta, bias, A, B, C, D, z, reverse)
+    _close(y, ref)
+
+
+def test_closed_form_longest_small_case():
+    rng = np.random.default_rng(7)
+    x, delta, bias, A, B, C, D, z = _rand_case(rng, 1, 16, 2, 4)
+    y, _ = oracle.s6_arrays(x, delta, A, B, C, delta_bias=bias, D=D, z=z)
+    _close(y, _closed_form(x, delta, bias, A, B, C, D, z, False))
+
+
+def test_lti_equals_convolution():
+    """Constant dt, B, C: the scan equals the causal convolution with
+    K_k = sum_n C[n] exp(dt A[n])^k dt B[n] (Mamba2 page, sec. 2.3 / 4.5)."""
+    rng = np.random.default_rng(11)
+    L, Dm, N = 64, 3, 8
+    x = rng.standard_normal((1, L, Dm))
+    dt = rng.uniform(0.01, 0.5, Dm)
+    delta = np.broadcast_to(dt, (1, L, Dm)).copy()
+    A = -np.exp(rng.uniform(-1.0, 1.5, (Dm, N)))
+    Bv = rng.standard_normal(N)
+    Cv = rng.standard_normal(N)
+    B = np.broadcast_to(Bv, (1, L, N)).copy()
+    C = np.broadcast_to(Cv, (1, L, N)).copy()
+    y, _ = oracle.s6_arrays(x, delta, A, B, C, softplus=False, D=None, z=None)
+    for d in range(Dm):
+        K = np.array([np.sum(Cv * np.exp(dt[d] * A[d]) ** k * dt[d] * Bv) for k in range(L)])
+        ref = np.convolve(x[0, :, d], K)[:L]
+        _close(y[0, :, d], ref, 1e-12)
+
+
+def test_reverse_is_flip():
+    rng = np.random.default_rng(12)
+    x, delta, bias, A, B, C, D, z = _rand_case(rng, 2, 23, 5, 16)
+    yr, sr = oracle.s6_arrays(x, delta, A, B, C, delta_bias=bias, D=D, z=z, reverse=True)
+    fl = lambda a: a[:, ::-1].copy()
+    yf, sf = oracle.s6_arrays(fl(x), fl(delta), A, fl(B), fl(C), delta_bias=bias, D=D, z=fl(z))
+    np.testing.assert_array_equal(yr, fl(yf))
+    np.testing.assert_array_equal(sr, sf)
+
+
+def test_bidir_is_sum_of_directions():
+    inp = ssm_gen.make_s6_inputs(2, 31, 8, 16, bidir=True, seed=3, random_A=True, random_D=True)
+    out, lf, lb = oracle.bidir(inp)
+    yf, sf = oracle.s6_arrays(inp.x, inp.delta, inp.A_f, inp.B_f, inp.C_f,
+                              delta_bias=inp.dt_bias_f, D=inp.D_f, z=inp.z_f)
+    yb, sb = oracle.s6_arrays(inp.x, inp.delta, inp.A_b, inp.B_b, inp.C_b,
+                              delta_bias=inp.dt_bias_b, D=inp.D_b, z=inp.z_b, reverse=True)
+    _close(out, yf + yb, 1e-15)
+    np.testing.assert_array_equal(lf, sf)
+    np.testing.assert_array_equal(lb, sb)
+
+
+def test_bidir_gate_after_sum_form():
+    """With z_f = z_b the per-direction gates equal the Vim form
+    silu(z) * (y_f + y_b) (Vim page, sec. 3.1: sum the directions, then gate)."""
+    inp = ssm_gen.make_s6_inputs(1, 17, 6, 16, bidir=True, seed=4, random_A=True)
+    inp.z_b = inp.z_f.copy()
+    out, _, _ = oracle.bidir(inp)
+    fwd = dict(delta_bias=inp.dt_bias_f, A=inp.A_f, B=inp.B_f, C=inp.C_f, D=inp.D_f, z=None)
+    bwd = dict(delta_bias=inp.dt_bias_b, A=inp.A_b, B=inp.B_b, C=inp.C_b, D=inp.D_b, z=None)
+    ungated, _, _ = oracle.bidir_arrays(inp.x, inp.delta, fwd, bwd)
+    _close(out, _silu(inp.z_f.astype(np.float64)) * ungated, 1e-14)
+
+
+def test_columns_subset_matches_full():
+    inp = ssm_gen.make_s6_inputs(3, 20, 7, 16, bidir=True, seed=5, random_A=True)
+    full, lf, lb = oracle.bidir(inp)
+    cols = [0, 5, 8, 20]
+    part, plf, plb = oracle.bidir(inp, cols=cols)
+    for c in cols:
+        b, d = divmod(c, 7)
+        np.testing.assert_array_equal(part[b, :, d], full[b, :, d])
+        np.testing.assert_array_equal(plf[b, d], lf[b, d])
+        np.testing.assert_array_equal(plb[b, d], lb[b, d])
+
+
+def test_threads_do_not_change_result():
+    inp = ssm_gen.make_s6_inputs(2, 40, 16, 16, bidir=True, seed=6)
+    a = oracle.bidir(inp, nthreads=1)
+    b = oracle.bidir(inp, nthreads=4)
+    for u, v in zip(a, b):
+        np.testing.assert_array_equal(u, v)
+
+
+# ---------------------------------------------------------------- special cases
+
+def test_zero_B_or_C_gives_skip_only():
+    rng = np.random.default_rng(13)
+    x, delta, bias, A, B, C, D, z = _rand_case(rng, 1, 12, 4, 16)
+    want = D[None, None, :] * x * _silu(z)
+    y, _ = oracle.s6_arrays(x, delta, A, np.zeros_like(B), C, delta_bias=bias, D=D, z=z)
+    _close(y, want, 1e-15)
+    y, _ = oracle.s6_arrays(x, delta, A, B, np.zeros_like(C), delta_bias=bias, D=D, z=z)
+    _close(y, want, 1e-15)
+
+
+def test_zero_dt_keeps_zero_state():
+    rng = np.random.default_rng(14)
+    x, delta, bias, A, B, C, D, z = _rand_case(rng, 1, 12, 4, 16)
+    y, st = oracle.s6_arrays(x, np.zeros_like(delta), A, B, C, softplus=False, D=D, z=z)
+    assert np.all(st == 0.0)
+    _close(y, D[None, None, :] * x * _silu(z), 1e-15)
+
+
+def test_N1_A0_is_prefix_sum():
+    rng = np.random.default_rng(15)
+    L = 30
+    x = rng.standard_normal((1, L, 1))
+    delta = rng.uniform(0.1, 1.0, (1, L, 1))
+    B = rng.standard_normal((1, L, 1))
+    C = rng.standard_normal((1, L, 1))
+    y, _ = oracle.s6_arrays(x, delta, np.zeros((1, 1)), B, C, softplus=False)
+    want = C[0, :, 0] * np.cumsum(delta[0, :, 0] * B[0, :, 0] * x[0, :, 0])
+    _close(y[0, :, 0], want, 1e-13)
+
+
+def test_zero_input_zero_output():
+    rng = np.random.default_rng(16)
+    x, delta, bias, A, B, C, D, z = _rand_case(rng, 1, 12, 4, 16)
+    y, st = oracle.s6_arrays(np.zeros_like(x), delta, A, B, C, delta_bias=bias, D=D, z=z)
+    assert np.all(y == 0.0) and np.all(st == 0.0)
+
+
+def test_L1_single_step():
+    rng = np.random.default_rng(17)
+    x, delta, bias, A, B, C, D, z = _rand_case(rng, 2, 1, 5, 16)
+    y, _ = oracle.s6_arrays(x, delta, A, B, C, delta_bias=bias, D=D, z=z)
+    dt = _softplus(delta + bias)
+    want = (np.einsum("bln,bln->bl", C, B)[..., None] * dt * x + D * x) * _silu(z)
+    _close(y, want, 1e-14)
+
+
+def test_softplus_and_silu_textbook_values():
+    one = np.ones((1, 1, 1))
+    # y = dt' * B * x * C with B = C = x = 1, A = 0: y = softplus(delta)
+    for v, want in [(0.0, math.log(2.0)), (50.0, 50.0), (-30.0, math.exp(-30.0)),
+                    (1.0, math.log1p(math.e))]:
+        y, _ = oracle.s6_arrays(one, np.full((1, 1, 1), v), np.zeros((1, 1)), one, one,
+                                softplus=True)
+        assert abs(y.item() - want) <= 1e-15 * max(1.0, abs(want)), (v, y.item(), want)
+    # gate: silu(0) = 0, silu(z) -> z for large z
+    y, _ = oracle.s6_arrays(one, one, np.zeros((1, 1)), one, one, softplus=False,
+                            z=np.zeros((1, 1, 1)))
+    assert y.item() == 0.0
+    y, _ = oracle.s6_arrays(one, one, np.zeros((1, 1)), one, one, softplus=False,
+                            z=np.full((1, 1, 1), 40.0))
+    assert abs(y.item() - 40.0) < 1e-12
+
+
+def test_empty_sequence():
+    x = np.zeros((2, 0, 3))
+    y, st = oracle.s6_arrays(x, x, np.zeros((3, 4)) - 1, np.zeros((2, 0, 4)),
+                             np.zeros((2, 0, 4)))
+    assert y.shape == (2, 0, 3) and np.all(st == 0)
+
+
+# ------------------------------------------------------------------------- SSD
+
+def _ssd_case(seed, Bz, L, H, P, N, random_D=True):
+    return ssm_gen.make_ssd_inputs(Bz, L, H, P, N, 8, dtype="f32", seed=seed, random_D=random_D)
+
+
+def test_ssd_seq_equals_s6_with_scalar_A():
+    inp = _ssd_case(21, 2, 19, 3, 4, 8)
+    y, st = oracle.ssd_seq(inp)
+    Bz, L, H, P = inp.x.shape
+    N = inp.B.shape[2]
+    x2 = inp.x.reshape(Bz, L, H * P)
+    d2 = np.repeat(inp.delta, P, axis=2)
+    A2 = np.repeat(np.broadcast_to(inp.A[:, None], (H, N)), P, axis=0)
+    y2, st2 = oracle.s6_arrays(x2, d2, A2, inp.B, inp.C, delta_bias=np.repeat(inp.dt_bias, P),
+                               D=np.repeat(inp.D, P), z=inp.z.reshape(Bz, L, H * P))
+    _close(y.reshape(Bz, L, H * P), y2, 1e-14)
+    _close(st.reshape(Bz, H * P, N), st2, 1e-14)
+
+
+@pytest.mark.parametrize("Q", [1, 8, 64])
+def test_ssd_chunked_equals_sequential(Q):
+    inp = _ssd_case(22, 2, 83, 3, 5, 16)  # 83 is not a multiple of 8 or 64
+    ys, ss = oracle.ssd_seq(inp)
+    yc, sc = oracle.ssd_chunked(inp, chunk=Q)
+    _close(yc, ys, 1e-11)
+    _close(sc, ss, 1e-11)
+
+
+def test_ssd_chunk1_is_recurrence_exactly_shaped():
+    """chunk = 1: every chunk is one step, the intra-chunk term is
+    C_t.B_t dt_t x_t and the carried state is the recurrence itself."""
+    inp = _ssd_case(23, 1, 10, 2, 3, 4)
+    ys, _ = oracle.ssd_seq(inp)
+    yc, _ = oracle.ssd_chunked(inp, chunk=1)
+    _close(yc, ys, 1e-13)
+
+
+def test_ssd_cols_subset():
+    inp = _ssd_case(24, 2, 30, 3, 4, 8)
+    full, fs = oracle.ssd_seq(inp)
+    cols = [0, 7, 13, 23]
+    part, ps = oracle.ssd_seq(inp, cols=cols)
+    P, H = 4, 3
+    for c in cols:
+        p = c % P
+        h = (c // P) % H
+        b = c // (P * H)
+        np.testing.assert_array_equal(part[b, :, h, p], full[b, :, h, p])
+        np.testing.assert_array_equal(ps[b, h, p], fs[b, h, p])
