@@ -1,0 +1,477 @@
+#!/usr/bin/env python
+"""Benchmark of the selective-scan hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config I] [--impl ours|reference]
+
+One step = one call of the hot path over one batch of the workload:
+config 1 (default) is the Vim-Small bidirectional scan, fp32, batch 64,
+L 197, d_inner 768, N 16 (bidir_scan_fwd); configs 0, 2, 3 are the other S6
+workloads and 4 the Mamba2 SSD workload.  Inputs are seeded synthetic
+tensors (ssm_gen) with the shapes and value distributions of those
+workloads.
+
+Timing: W untimed warm-up steps, then K timed steps.  Before every timed
+step a 512 MB buffer is written to flush the 126 MB L2; each step is
+bracketed by CUDA events on the launching stream, and the step times are
+summed (the flush is outside the events).  The timed region is bracketed by
+a barrier and torch.cuda.synchronize(); with N > 1 every rank runs its own
+batch (weak scaling, no collective on the data path) and the time is the
+max over ranks.  nvidia-smi samples SM clocks and throttle reasons during
+the timed region.
+
+Rank 0 prints one JSON line.  `--impl reference` times the float64 CPU
+oracle instead (bounded sample per step, all host cores).
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import ssm_gen  # noqa: E402
+
+METRIC = "scan elements/s (B·L·D·N) and HBM GB/s as % of B200 peak, per config"
+HBM_FALLBACK_GBS = 6650.0
+L2_FLUSH_BYTES = 512 << 20
+SMS = 148
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=1000)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--config", type=int, default=1)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args()
+
+
+# --------------------------------------------------------------- workload
+
+def workload_info(cfg: int):
+    w = dict(ssm_gen.WORKLOADS[cfg])
+    if w["kind"] == "s6":
+        ndir = 2 if w["bidir"] else 1
+        es = 4 if w["dtype"] == "f32" else 2
+        B, L, D, N = w["batch"], w["seqlen"], w["dim"], w["dstate"]
+        elems = B * L * D * N * ndir
+        io = B * L * D * es * (2 + ndir + 1)          # x, delta, z per direction, out
+        io += B * L * N * es * 2 * ndir               # B, C per direction
+        io += ndir * (D * N + 2 * D) * 4              # A, D, delta_bias
+        if w.get("last_state"):
+            io += ndir * B * D * N * 4
+        w.update(ndir=ndir, elems=elems, bytes=io)
+    else:
+        B, L, H, P, N = w["batch"], w["seqlen"], w["nheads"], w["headdim"], w["dstate"]
+        es = 2
+        elems = B * L * H * P * N
+        io = B * L * H * P * es * 3 + B * L * N * es * 2 + B * L * H * es + H * 12
+        w.update(ndir=1, elems=elems, bytes=io)
+    return w
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return {"hbm_gbs": HBM_FALLBACK_GBS, "bf16_tflops": 1590.0, "sm_max_mhz": 1965.0}, "fallback"
+
+
+def alu_peak_elems(sm_mhz: float) -> float:
+    """Element rate the SM pipes allow for the S6 inner step (one exp and four
+    FMA-pipe operations per element): exps split between the MUFU unit
+    (16/clk/SM) and an 8-operation FMA-pipe polynomial so that both pipes
+    (MUFU 16/clk/SM, FMA 128/clk/SM) finish together -> 64/3 elements per
+    clock per SM."""
+    return SMS * sm_mhz * 1e6 * (64.0 / 3.0)
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        loaded = [s for s in sm if mx and s > 0.5 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows),
+                "power_w_max": max((float(r[3]) for r in rows if r[3].replace(".", "").isdigit()),
+                                   default=None)}
+
+
+# ----------------------------------------------------------- device side
+
+class DeviceWorkload:
+    """Inputs resident in HBM plus the raw C-ABI call of one step."""
+
+    def __init__(self, cfg, seed, device):
+        import torch
+        import selective_state_space_24_b200 as ssm
+        self.torch, self.ssm, self.dev = torch, ssm, device
+        self.cfg = cfg
+        self.info = workload_info(cfg)
+        self.inp = ssm_gen.make_workload(cfg, seed=seed)
+        self.lib = ssm.load()
+        self.host = {}      # pinned host copies (for e2e)
+        self.d = {}         # device tensors
+        tdt = torch.float32 if self.inp.dtype == "f32" else torch.bfloat16
+        for k, v in vars(self.inp).items():
+            if isinstance(v, np.ndarray):
+                io = k in self.inp.io_tensors()
+                t = torch.from_numpy(np.ascontiguousarray(v, np.float32))
+                t = (t.to(tdt) if io else t).pin_memory()
+                self.host[k] = t
+                self.d[k] = t.to(device)
+        self.out = torch.empty_like(self.d["x"])
+        self.out_host = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
+        self.last = {}
+        if self.info["kind"] == "s6":
+            self.dims = ssm.ssm_dims(self.inp.batch, self.inp.seqlen, self.inp.dim, self.inp.dstate,
+                                     ssm.SSM_F32 if self.inp.dtype == "f32" else ssm.SSM_BF16)
+            if self.info.get("last_state"):
+                for s in ("f", "b"):
+                    self.last[s] = torch.empty((self.inp.batch, self.inp.dim, self.inp.dstate),
+                                               dtype=torch.float32, device=device)
+            if self.info["ndir"] == 2:
+                need = self.lib.bidir_scan_workspace_size(ctypes.byref(self.dims))
+            else:
+                need = self.lib.ssm_scan_workspace_size(ctypes.byref(self.dims))
+        else:
+            i = self.inp
+            self.dims = ssm.ssd_dims(i.batch, i.seqlen, i.nheads, i.headdim, i.dstate, i.chunk,
+                                     ssm.SSM_BF16)
+            need = self.lib.ssd_chunk_workspace_size(ctypes.byref(self.dims))
+        self.ws = torch.empty(max(int(need), 16), dtype=torch.uint8, device=device)
+        self.ws_bytes = int(need)
+        self.launches_per_step = self._launches()
+        self._bind()
+
+    def _launches(self):
+        if self.info["kind"] == "s6":
+            return 3 if self.ws_bytes > 0 else 1
+        return 1
+
+    def _bind(self):
+        d = self.d
+        p = lambda t: None if t is None else t.data_ptr()
+        if self.info["kind"] == "s6" and self.info["ndir"] == 2:
+            self.fwd = self.ssm.ssm_dir_params(p(d["dt_bias_f"]), p(d["A_f"]), p(d["B_f"]),
+                                               p(d["C_f"]), p(d["D_f"]), p(d.get("z_f")),
+                                               p(self.last.get("f")))
+            self.bwd = self.ssm.ssm_dir_params(p(d["dt_bias_b"]), p(d["A_b"]), p(d["B_b"]),
+                                               p(d["C_b"]), p(d["D_b"]), p(d.get("z_b")),
+                                               p(self.last.get("b")))
+
+    def step(self, stream_handle):
+        """One call of the hot path through the C ABI (inputs resident)."""
+        d, lib = self.d, self.lib
+        p = lambda t: None if t is None else t.data_ptr()
+        if self.info["kind"] == "s6" and self.info["ndir"] == 2:
+            st = lib.bidir_scan_fwd(ctypes.byref(self.dims), p(d["x"]), p(d["delta"]), 1,
+                                    ctypes.byref(self.fwd), ctypes.byref(self.bwd), p(self.out),
+                                    p(self.ws), self.ws_bytes, stream_handle)
+        elif self.info["kind"] == "s6":
+            st = lib.ssm_scan_fwd(ctypes.byref(self.dims), p(d["x"]), p(d["delta"]),
+                                  p(d["dt_bias_f"]), 1, p(d["A_f"]), p(d["B_f"]), p(d["C_f"]),
+                                  p(d["D_f"]), p(d.get("z_f")), 0, p(self.out), None, p(self.ws),
+                                  self.ws_bytes, stream_handle)
+        else:
+            st = lib.ssd_chunk_fwd(ctypes.byref(self.dims), p(d["x"]), p(d["delta"]),
+                                   p(d["dt_bias"]), 1, p(d["A"]), p(d["B"]), p(d["C"]), p(d["D"]),
+                                   p(d.get("z")), p(self.out), None, p(self.ws), self.ws_bytes,
+                                   stream_handle)
+        if st != 0:
+            raise RuntimeError(f"hot path returned {self.ssm.STATUS.get(st, st)}")
+
+    def e2e_step(self, stream_handle):
+        """Host buffers in, result out: H2D of every input from pinned memory,
+        the call, D2H of the output; returns (h2d bytes, d2h bytes)."""
+        hb = 0
+        for k, t in self.host.items():
+            self.d[k].copy_(t, non_blocking=True)
+            hb += t.numel() * t.element_size()
+        self.step(stream_handle)
+        self.out_host.copy_(self.out, non_blocking=True)
+        return hb, self.out.numel() * self.out.element_size()
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from selective_state_space_24_b200 import build as ssm_build
+    ssm_build.build()
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    info = workload_info(args.config)
+    wl = DeviceWorkload(args.config, seed=rank, device=device)
+    stream = torch.cuda.current_stream(device)
+    sh = stream.cuda_stream
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+
+    for _ in range(max(args.warmup, 3)):
+        flush.fill_(1.0)
+        wl.step(sh)
+    torch.cuda.synchronize()
+    assert torch.isfinite(wl.out.float()).all().item(), "non-finite output"
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_wall = time.perf_counter()
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        evs[i][0].record(stream)
+        wl.step(sh)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    wall = time.perf_counter() - t_wall
+    clocks = sampler.stop()
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    total_ms = float(sum(step_ms))
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    per_step_ms = total_ms / args.steps
+    value = info["elems"] * world * args.steps / (total_ms * 1e-3)
+
+    # roofline of the dominant kernel (the one launch of the step when the
+    # plan has a single segment; else the step is summary + carry + main)
+    peaks, peak_src = load_peaks()
+    kern_s = statistics.median(step_ms) * 1e-3
+    hbm_ach = info["bytes"] / kern_s / 1e9
+    alu_peak = alu_peak_elems(peaks.get("sm_max_mhz", 1965.0))
+    alu_ach = info["elems"] / kern_s
+    t_hbm = info["bytes"] / (peaks["hbm_gbs"] * 1e9)
+    t_alu = info["elems"] / alu_peak
+    if info["kind"] == "s6" and t_alu > t_hbm:
+        roof = {"bound": "alu", "achieved": alu_ach / 1e9, "peak": alu_peak / 1e9,
+                "unit": "Gelem/s", "frac": alu_ach / alu_peak, "traffic": None,
+                "hbm_achieved_gbs": hbm_ach, "hbm_peak_gbs": peaks["hbm_gbs"],
+                "hbm_frac": hbm_ach / peaks["hbm_gbs"], "peak_source": peak_src,
+                "algorithmic_bytes": info["bytes"], "kernel_ms_median": kern_s * 1e3}
+    else:
+        roof = {"bound": "hbm", "achieved": hbm_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": hbm_ach / peaks["hbm_gbs"], "traffic": None, "peak_source": peak_src,
+                "algorithmic_bytes": info["bytes"], "kernel_ms_median": kern_s * 1e3}
+
+    e2e = None
+    if not args.no_e2e:
+        ke = max(3, min(args.steps, 20))
+        for _ in range(2):
+            wl.e2e_step(sh)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        hb = db = 0
+        for _ in range(ke):
+            hb, db = wl.e2e_step(sh)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ems], dtype=torch.float64, device=device)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": info["elems"] * world * ke / (ems * 1e-3), "unit": "elements/s",
+               "h2d_bytes_per_step": hb, "d2h_bytes_per_step": db, "steps": ke,
+               "ms_per_step": ems / ke}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args.config, budget_s=10.0)
+
+    res = {
+        "metric": METRIC, "value": value, "unit": "elements/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32" if info["dtype"] == "f32" else "bf16 storage, f32 compute",
+        "data": "synthetic (seeded ssm_gen inputs with the workload's shapes and distributions)",
+        "config": {"workload": info["name"], "config_index": args.config,
+                   **{k: info[k] for k in ("batch", "seqlen", "dim", "dstate", "nheads", "headdim",
+                                           "chunk") if k in info},
+                   "directions": info["ndir"], "parallelism": f"dp{world} (independent batches)",
+                   "l2": "flushed before every timed step (512 MB write)",
+                   "algorithmic_bytes_per_step": info["bytes"],
+                   "elements_per_step": info["elems"]},
+        "hbm_gbs": info["bytes"] / (per_step_ms * 1e-3) / 1e9,
+        "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": wl.launches_per_step * args.steps,
+        "clocks": clocks, "wall_s_timed_region": wall,
+    }
+    return res
+
+
+# ------------------------------------------------------------ CPU oracle
+
+def _oracle_sample(cfg, frac_cols):
+    """Inputs and column sample for a bounded oracle run of workload cfg."""
+    inp = ssm_gen.make_workload(cfg, seed=0)
+    info = workload_info(cfg)
+    if info["kind"] == "s6":
+        ncols_all = inp.batch * inp.dim
+    else:
+        ncols_all = inp.batch * inp.nheads * inp.headdim
+    n = max(1, min(ncols_all, int(ncols_all * frac_cols)))
+    cols = np.random.default_rng(0).choice(ncols_all, n, replace=False)
+    return inp, info, cols, ncols_all
+
+
+def _oracle_call(inp, info, cols, threads):
+    import oracle
+    if info["kind"] == "s6":
+        if info["ndir"] == 2:
+            oracle.bidir(inp, cols=cols, nthreads=threads)
+        else:
+            oracle.s6(inp, cols=cols, nthreads=threads)
+    else:
+        oracle.ssd_seq(inp, cols=cols, nthreads=threads)
+
+
+def cpu_baseline(cfg, budget_s=10.0):
+    """The float64 oracle as it stands, on this host's cores, over a sample of
+    the workload's columns sized to about `budget_s` of CPU time."""
+    import oracle
+    threads = len(os.sched_getaffinity(0))
+    inp, info, cols, ncols_all = _oracle_sample(cfg, 1.0)
+    per_col = info["elems"] / ncols_all
+    probe = cols[: max(threads * 4, 16)]
+    t0 = time.perf_counter()
+    _oracle_call(inp, info, probe, threads)
+    dt = max(time.perf_counter() - t0, 1e-6)
+    n = int(min(len(cols), max(len(probe), len(probe) * budget_s / dt)))
+    sample = cols[:n]
+    t0 = time.perf_counter()
+    _oracle_call(inp, info, sample, threads)
+    el = time.perf_counter() - t0
+    return {"value": n * per_col / el, "unit": "elements/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n} of {ncols_all} (batch, channel) columns, whole sequence each, "
+                      f"{el:.1f} s, float64 C oracle with OpenMP",
+            "seconds": el}
+
+
+def run_reference(args):
+    threads = len(os.sched_getaffinity(0))
+    info = workload_info(args.config)
+    inp, _, cols, ncols_all = _oracle_sample(args.config, 1.0)
+    per_col = info["elems"] / ncols_all
+    probe = cols[: max(threads * 2, 8)]
+    t0 = time.perf_counter()
+    _oracle_call(inp, info, probe, threads)
+    dt = max(time.perf_counter() - t0, 1e-6)
+    # size each step so that warm-up + steps take about one minute in all
+    per_step_budget = 60.0 / max(1, args.steps + args.warmup)
+    n = int(min(len(cols), max(len(probe), len(probe) * per_step_budget / dt)))
+    sample = cols[:n]
+    for _ in range(args.warmup):
+        _oracle_call(inp, info, sample, threads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        _oracle_call(inp, info, sample, threads)
+    el = time.perf_counter() - t0
+    value = n * per_col * args.steps / el
+    samp = f"{n} of {ncols_all} (batch, channel) columns per step, whole sequence each"
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "elements/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": el * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": info["name"], "config_index": args.config},
+        "cpu_baseline": {"value": value, "unit": "elements/s", "cores": threads,
+                         "kind": "oracle", "sample": samp},
+        "e2e": {"value": value, "unit": "elements/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

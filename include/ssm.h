@@ -1,0 +1,190 @@
+/*
+ * ssm.h -- C ABI of libssm.so, a B200 (sm_100a) selective-scan library.
+ *
+ * Three operations:
+ *
+ *  ssm_scan_fwd    Mamba S6 selective scan, one direction.
+ *                  Defined by the discrete recurrence of the Mamba2 page
+ *                  ("手写简化版Mamba2", intelliparadigm.com) sec. 2.2 with the
+ *                  Bbar ~= dt*B approximation, the per-step scan of sec. 4.3
+ *                  and the D skip + SiLU gate of sec. 4.4:
+ *                    dt[b,t,d]  = softplus(delta[b,t,d] + delta_bias[d])
+ *                                 (plain delta + delta_bias if delta_softplus = 0)
+ *                    h[n]       = exp(dt * A[d,n]) * h[n] + dt * B[b,t,n] * x[b,t,d]
+ *                    out[b,t,d] = (sum_n C[b,t,n] h[n] + D[d] x[b,t,d]) * silu(z[b,t,d])
+ *                  h starts at zero; reverse = 1 runs t = L-1 .. 0.
+ *
+ *  bidir_scan_fwd  Vision-Mamba bidirectional scan (the Vim reproduction page,
+ *                  news.rkmt.cn, sec. 3.1-3.2): a forward scan and a reversed
+ *                  scan, each with its own delta_bias, A, B, C, D, z, on shared
+ *                  x and delta; out = forward result + reversed result, both at
+ *                  the original positions.  Both directions are computed in one
+ *                  launch over a single pass of HBM.
+ *
+ *  ssd_chunk_fwd   Mamba2 SSD (Mamba2 page sec. 3.1-3.2): the same recurrence
+ *                  with A a scalar per head, computed chunk by chunk -- matrix
+ *                  products (tensor cores) inside each chunk and the chunk state
+ *                  passed on between chunks.
+ *
+ * Conventions shared by all entry points
+ *  - Every tensor argument is a DEVICE pointer to a contiguous row-major array
+ *    (last index fastest) on the current CUDA device.  The caller owns all
+ *    memory, including the workspace; the library allocates nothing and keeps
+ *    no state between calls.
+ *  - x, delta, z, B, C and out have the element type dims->dtype (SSM_F32 or
+ *    SSM_BF16).  delta_bias, A, D and last_state are always float32.
+ *  - Every pointer must be 16-byte aligned; dim (S6) must be a multiple of 4
+ *    for SSM_F32 and of 8 for SSM_BF16.  Otherwise SSM_ERR_MISALIGNED.
+ *  - out must not overlap any input.  last_state is written, not accumulated.
+ *  - All arithmetic is float32 (the state, dt, exp(dt*A)); bf16 inputs are
+ *    widened exactly and the output is rounded to nearest even.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream) and thread-safe.  All arguments are validated before
+ *    anything is launched; on an error nothing is launched and the return
+ *    value says why.  SSM_ERR_CUDA means a launch failed (the CUDA error is
+ *    then sticky in the caller's context as usual).
+ *  - A zero batch, seqlen or dim is a valid empty call: the tensor pointers
+ *    may then be NULL, nothing is launched, and last_state (if given and of
+ *    non-zero size) is zero-filled.
+ */
+#ifndef SSM_B200_SSM_H
+#define SSM_B200_SSM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SSM_API __attribute__((visibility("default")))
+#else
+#define SSM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { SSM_F32 = 0, SSM_BF16 = 1 } ssm_dtype;
+
+typedef enum {
+    SSM_OK = 0,
+    SSM_ERR_INVALID_ARG = 1,         /* NULL required pointer, negative size, NULL dims */
+    SSM_ERR_UNSUPPORTED_SHAPE = 2,   /* dstate outside 1..16 (S6); SSD shape not supported */
+    SSM_ERR_MISALIGNED = 3,          /* pointer not 16-byte aligned / dim not a vector multiple */
+    SSM_ERR_UNSUPPORTED_DTYPE = 4,   /* dtype not SSM_F32 / SSM_BF16 (SSD: SSM_BF16 only) */
+    SSM_ERR_WORKSPACE_TOO_SMALL = 5, /* workspace_bytes < the *_workspace_size() value */
+    SSM_ERR_CUDA = 6,                /* a CUDA launch or runtime call failed */
+    SSM_ERR_DEVICE_TIMEOUT = 7       /* a bounded device-side wait gave up (see ssm_check_device) */
+} ssm_status;
+
+/* S6 problem size.  dtype is an ssm_dtype value. */
+typedef struct {
+    int64_t batch;   /* B */
+    int64_t seqlen;  /* L */
+    int64_t dim;     /* D, channels (d_inner) */
+    int64_t dstate;  /* N, 1..16 */
+    int32_t dtype;
+} ssm_dims;
+
+/* Parameters of one scan direction (bidir_scan_fwd). */
+typedef struct {
+    const float *delta_bias; /* (D) float32, or NULL for no bias              */
+    const float *A;          /* (D, N) float32, required                       */
+    const void *B;           /* (B, L, N) dtype, required; shared by channels  */
+    const void *C;           /* (B, L, N) dtype, required; shared by channels  */
+    const float *D;          /* (D) float32, or NULL for no skip term          */
+    const void *z;           /* (B, L, D) dtype, or NULL for no gate           */
+    float *last_state;       /* (B, D, N) float32 output, or NULL              */
+} ssm_dir_params;
+
+/*
+ * Bytes of device workspace ssm_scan_fwd needs for `dims` (0 if none).  The
+ * value depends only on dims.  Returns 0 for invalid dims.
+ */
+SSM_API size_t ssm_scan_workspace_size(const ssm_dims *dims);
+
+/*
+ * S6 scan, one direction.
+ *   x, delta   (B, L, D) dtype, required
+ *   delta_bias (D) float32 or NULL;  delta_softplus: 1 = apply softplus
+ *   A          (D, N) float32, required (any values; A < 0 keeps it stable)
+ *   B, C       (B, L, N) dtype, required
+ *   D          (D) float32 or NULL;  z (B, L, D) dtype or NULL
+ *   reverse    0 = t ascending, 1 = t descending (outputs stay at their t)
+ *   out        (B, L, D) dtype, written
+ *   last_state (B, D, N) float32 or NULL: the state after the last step
+ *              (after t = L-1 forward, after t = 0 reversed)
+ *   workspace  device scratch of at least ssm_scan_workspace_size(dims)
+ *              bytes (may be NULL when that size is 0); contents on entry
+ *              are ignored, contents on return are unspecified.
+ */
+SSM_API ssm_status ssm_scan_fwd(const ssm_dims *dims, const void *x, const void *delta,
+                        const float *delta_bias, int delta_softplus, const float *A,
+                        const void *B, const void *C, const float *D, const void *z,
+                        int reverse, void *out, float *last_state, void *workspace,
+                        size_t workspace_bytes, void *stream);
+
+/* Bytes of device workspace bidir_scan_fwd needs for `dims` (0 if none). */
+SSM_API size_t bidir_scan_workspace_size(const ssm_dims *dims);
+
+/*
+ * Vision-Mamba bidirectional scan:
+ *   out = S6(x, delta, fwd, reverse = 0) + S6(x, delta, bwd, reverse = 1)
+ * with x, delta (B, L, D) shared; fwd and bwd each as described for
+ * ssm_dir_params (their last_state fields are optional outputs).
+ * fwd and bwd must be non-NULL; out (B, L, D) dtype is written.
+ */
+SSM_API ssm_status bidir_scan_fwd(const ssm_dims *dims, const void *x, const void *delta,
+                          int delta_softplus, const ssm_dir_params *fwd,
+                          const ssm_dir_params *bwd, void *out, void *workspace,
+                          size_t workspace_bytes, void *stream);
+
+/* SSD problem size.  Supported: dtype SSM_BF16, headdim 64, dstate 128,
+ * chunk 64, seqlen any value >= 0 (a short last chunk is handled). */
+typedef struct {
+    int64_t batch;    /* B */
+    int64_t seqlen;   /* L */
+    int64_t nheads;   /* H */
+    int64_t headdim;  /* P */
+    int64_t dstate;   /* N */
+    int64_t chunk;    /* Q, tokens per chunk */
+    int32_t dtype;
+} ssd_dims;
+
+/* Bytes of device workspace ssd_chunk_fwd needs for `dims` (0 if none). */
+SSM_API size_t ssd_chunk_workspace_size(const ssd_dims *dims);
+
+/*
+ * Mamba2 SSD chunked scan (Mamba2 page sec. 3.2), equal to the sequential
+ * recurrence with A[d, n] = A[h] for every channel d = (h, p) of head h:
+ *   x, z       (B, L, H, P) dtype (z may be NULL: no gate)
+ *   delta      (B, L, H) dtype;  delta_bias (H) float32 or NULL
+ *   A          (H) float32;  D (H) float32 or NULL
+ *   B, C       (B, L, N) dtype, shared by all heads
+ *   out        (B, L, H, P) dtype, written
+ *   last_state (B, H, P, N) float32 or NULL
+ */
+SSM_API ssm_status ssd_chunk_fwd(const ssd_dims *dims, const void *x, const void *delta,
+                         const float *delta_bias, int delta_softplus, const float *A,
+                         const void *B, const void *C, const float *D, const void *z,
+                         void *out, float *last_state, void *workspace,
+                         size_t workspace_bytes, void *stream);
+
+/*
+ * Waits for `stream`, then reports (and clears) the library's device-side
+ * error word: SSM_ERR_DEVICE_TIMEOUT if a bounded wait inside a kernel gave
+ * up since the last check, SSM_ERR_CUDA if the stream reports a CUDA error,
+ * SSM_OK otherwise.  Blocking; meant for tests and debugging.
+ */
+SSM_API ssm_status ssm_check_device(void *stream);
+
+/* Static, human-readable name of a status code. */
+SSM_API const char *ssm_status_string(ssm_status status);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+SSM_API int ssm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSM_B200_SSM_H */

@@ -1,0 +1,229 @@
+"""Python binding of libssm.so, the sm_100a selective-scan library.
+
+Argument marshalling only: every step of the scan runs in the library's
+CUDA kernels.  PyTorch is used for device memory (tensors, the workspace)
+and streams.  If libssm.so is missing or fails to load, every entry point
+raises -- there is no fallback path.
+
+Entry points (names as in include/ssm.h):
+
+* ``ssm_scan_fwd(x, delta, A, B, C, ...)``  single-direction S6 scan
+* ``bidir_scan_fwd(x, delta, fwd, bwd, ...)``  Vision-Mamba bidirectional scan
+* ``ssd_chunk_fwd(x, delta, A, B, C, ...)``  Mamba2 SSD chunked scan
+
+Each also exists in raw form in ``capi`` (ctypes functions taking plain
+integers for pointers), which the tests use to check the boundary itself.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libssm.so")
+
+SSM_F32, SSM_BF16 = 0, 1
+STATUS = {
+    0: "SSM_OK", 1: "SSM_ERR_INVALID_ARG", 2: "SSM_ERR_UNSUPPORTED_SHAPE", 3: "SSM_ERR_MISALIGNED",
+    4: "SSM_ERR_UNSUPPORTED_DTYPE", 5: "SSM_ERR_WORKSPACE_TOO_SMALL", 6: "SSM_ERR_CUDA",
+    7: "SSM_ERR_DEVICE_TIMEOUT",
+}
+
+
+class SSMError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)}")
+
+
+class ssm_dims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64), ("dim", ctypes.c_int64),
+                ("dstate", ctypes.c_int64), ("dtype", ctypes.c_int32)]
+
+
+class ssd_dims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64), ("nheads", ctypes.c_int64),
+                ("headdim", ctypes.c_int64), ("dstate", ctypes.c_int64), ("chunk", ctypes.c_int64),
+                ("dtype", ctypes.c_int32)]
+
+
+class ssm_dir_params(ctypes.Structure):
+    _fields_ = [("delta_bias", ctypes.c_void_p), ("A", ctypes.c_void_p), ("B", ctypes.c_void_p),
+                ("C", ctypes.c_void_p), ("D", ctypes.c_void_p), ("z", ctypes.c_void_p),
+                ("last_state", ctypes.c_void_p)]
+
+
+_vp = ctypes.c_void_p
+_sz = ctypes.c_size_t
+_int = ctypes.c_int
+
+# exported name -> (restype, argtypes)
+SIGNATURES = {
+    "ssm_scan_workspace_size": (_sz, [ctypes.POINTER(ssm_dims)]),
+    "ssm_scan_fwd": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp, _vp,
+                            _int, _vp, _vp, _vp, _sz, _vp]),
+    "bidir_scan_workspace_size": (_sz, [ctypes.POINTER(ssm_dims)]),
+    "bidir_scan_fwd": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _int,
+                              ctypes.POINTER(ssm_dir_params), ctypes.POINTER(ssm_dir_params), _vp,
+                              _vp, _sz, _vp]),
+    "ssd_chunk_workspace_size": (_sz, [ctypes.POINTER(ssd_dims)]),
+    "ssd_chunk_fwd": (_int, [ctypes.POINTER(ssd_dims), _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp,
+                             _vp, _vp, _vp, _vp, _sz, _vp]),
+    "ssm_check_device": (_int, [_vp]),
+    "ssm_status_string": (ctypes.c_char_p, [_int]),
+    "ssm_version": (_int, []),
+}
+
+_capi = None
+
+
+def load(path: Optional[str] = None):
+    """Load libssm.so (once) and attach the signatures; raises if missing."""
+    global _capi
+    if _capi is not None and path is None:
+        return _capi
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise ImportError(f"{p} is missing: build it with "
+                          "`python -m selective_state_space_24_b200.build`")
+    lib = ctypes.CDLL(p)
+    for name, (res, args) in SIGNATURES.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    if path is None:
+        _capi = lib
+    return lib
+
+
+def capi():
+    return load()
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise SSMError(status, what)
+
+
+# ------------------------------------------------------------------ tensors
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.float32:
+        return SSM_F32
+    if t.dtype == torch.bfloat16:
+        return SSM_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _stream_handle(stream) -> Optional[int]:
+    torch = _torch()
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def workspace(nbytes: int, device):
+    """A device workspace of at least nbytes (None when 0)."""
+    if nbytes == 0:
+        return None
+    torch = _torch()
+    return torch.empty(int(nbytes), dtype=torch.uint8, device=device)
+
+
+@dataclass
+class DirParams:
+    """One direction's parameters for bidir_scan_fwd (tensors on the device)."""
+    A: object
+    B: object
+    C: object
+    delta_bias: object = None
+    D: object = None
+    z: object = None
+    last_state: object = None
+
+    def to_c(self) -> ssm_dir_params:
+        return ssm_dir_params(_ptr(self.delta_bias), _ptr(self.A), _ptr(self.B), _ptr(self.C),
+                              _ptr(self.D), _ptr(self.z), _ptr(self.last_state))
+
+
+def s6_dims(x, dstate: int) -> ssm_dims:
+    Bz, L, Dm = x.shape
+    return ssm_dims(Bz, L, Dm, dstate, _dtype_code(x))
+
+
+def ssm_scan_fwd(x, delta, A, B, C, *, delta_bias=None, delta_softplus=True, D=None, z=None,
+                 reverse=False, out=None, last_state=None, ws=None, stream=None):
+    """Single-direction S6 scan; returns out (B, L, D) in x's dtype."""
+    torch = _torch()
+    lib = capi()
+    dims = s6_dims(x, A.shape[1])
+    if out is None:
+        out = torch.empty_like(x)
+    need = lib.ssm_scan_workspace_size(ctypes.byref(dims))
+    if ws is None:
+        ws = workspace(need, x.device)
+    st = lib.ssm_scan_fwd(ctypes.byref(dims), _ptr(x), _ptr(delta), _ptr(delta_bias),
+                          int(bool(delta_softplus)), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+                          int(bool(reverse)), _ptr(out), _ptr(last_state), _ptr(ws),
+                          0 if ws is None else ws.numel(), _stream_handle(stream))
+    _check(st, "ssm_scan_fwd")
+    return out
+
+
+def bidir_scan_fwd(x, delta, fwd: DirParams, bwd: DirParams, *, delta_softplus=True, out=None,
+                   ws=None, stream=None):
+    """Vision-Mamba bidirectional scan; returns out (B, L, D) in x's dtype."""
+    torch = _torch()
+    lib = capi()
+    dims = s6_dims(x, fwd.A.shape[1])
+    if out is None:
+        out = torch.empty_like(x)
+    need = lib.bidir_scan_workspace_size(ctypes.byref(dims))
+    if ws is None:
+        ws = workspace(need, x.device)
+    f, b = fwd.to_c(), bwd.to_c()
+    st = lib.bidir_scan_fwd(ctypes.byref(dims), _ptr(x), _ptr(delta), int(bool(delta_softplus)),
+                            ctypes.byref(f), ctypes.byref(b), _ptr(out), _ptr(ws),
+                            0 if ws is None else ws.numel(), _stream_handle(stream))
+    _check(st, "bidir_scan_fwd")
+    return out
+
+
+def ssd_chunk_fwd(x, delta, A, B, C, *, chunk=64, delta_bias=None, delta_softplus=True, D=None,
+                  z=None, out=None, last_state=None, ws=None, stream=None):
+    """Mamba2 SSD chunked scan; returns out (B, L, H, P) in x's dtype."""
+    torch = _torch()
+    lib = capi()
+    Bz, L, H, P = x.shape
+    dims = ssd_dims(Bz, L, H, P, B.shape[2], chunk, _dtype_code(x))
+    if out is None:
+        out = torch.empty_like(x)
+    need = lib.ssd_chunk_workspace_size(ctypes.byref(dims))
+    if ws is None:
+        ws = workspace(need, x.device)
+    st = lib.ssd_chunk_fwd(ctypes.byref(dims), _ptr(x), _ptr(delta), _ptr(delta_bias),
+                           int(bool(delta_softplus)), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+                           _ptr(out), _ptr(last_state), _ptr(ws), 0 if ws is None else ws.numel(),
+                           _stream_handle(stream))
+    _check(st, "ssd_chunk_fwd")
+    return out
+
+
+def check_device(stream=None):
+    """Synchronise and raise if a kernel reported a device-side timeout."""
+    _check(capi().ssm_check_device(_stream_handle(stream)), "ssm_check_device")

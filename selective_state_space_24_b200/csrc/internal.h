@@ -1,0 +1,71 @@
+// internal.h -- launcher interface between the C-ABI shim and the kernels.
+// Not part of the public ABI (include/ssm.h is).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace ssm {
+
+// Parameters of one scan direction, device pointers.
+struct DirArgs {
+    const float *bias;   // (D) or nullptr
+    const float *A;      // (D, N)
+    const void *B;       // (Bsz, L, N)
+    const void *C;       // (Bsz, L, N)
+    const float *D;      // (D) or nullptr
+    const void *z;       // (Bsz, L, D) or nullptr
+    float *last_state;   // (Bsz, D, N) or nullptr
+};
+
+// One S6 call (single direction or bidirectional).
+//
+// The sequence is cut into S segments of T steps (the last one may be
+// shorter).  With S > 1 every segment first summarises itself (local end
+// state from a zero start plus the sum of dt), a carry pass composes those
+// summaries in scan order, and the main pass then rescans each segment from
+// its true entering state.  carry_h / carry_s are the caller's workspace.
+struct S6Args {
+    int Bsz, L, D, N;
+    int S, T;
+    int dtype;     // 0 = float32, 1 = bf16
+    int softplus;
+    int ndir;      // 1 or 2
+    int reverse;   // ndir == 1: 1 = the single direction runs t descending
+    const void *x;
+    const void *delta;
+    DirArgs dir[2];  // ndir == 2: dir[0] forward, dir[1] reversed
+    void *out;
+    float *carry_h;  // [ndir][Bsz][S][D][N]
+    float *carry_s;  // [ndir][Bsz][S][D]
+};
+
+struct S6Plan {
+    int S, T;
+    size_t workspace_bytes;
+};
+
+// Segment plan for a problem; depends on the sizes only.
+S6Plan plan_s6(int64_t Bsz, int64_t L, int64_t D, int64_t N, int ndir);
+
+cudaError_t launch_s6(const S6Args &a, cudaStream_t stream);
+
+// One SSD call.
+struct SSDArgs {
+    int Bsz, L, H, P, N, Q;
+    int softplus;
+    const void *x, *delta, *B, *C, *z;
+    const float *bias, *A, *D;
+    void *out;
+    float *last_state;
+    void *workspace;
+};
+
+size_t ssd_workspace_bytes(int64_t Bsz, int64_t L, int64_t H, int64_t P, int64_t N, int64_t Q);
+cudaError_t launch_ssd(const SSDArgs &a, cudaStream_t stream);
+
+// Device-side error word (bounded waits that gave up set it).
+cudaError_t read_and_clear_device_error(unsigned *value, cudaStream_t stream);
+
+}  // namespace ssm

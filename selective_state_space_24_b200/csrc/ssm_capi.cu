@@ -1,0 +1,272 @@
+// ssm_capi.cu -- the extern "C" boundary of libssm.so (declared in
+// include/ssm.h): argument validation, workspace sizing, dispatch.
+// Every check runs before anything is launched.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "../../include/ssm.h"
+#include "internal.h"
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool dtype_ok(int32_t dt) { return dt == SSM_F32 || dt == SSM_BF16; }
+
+// Common S6 shape / pointer checks.  Returns SSM_OK or the first failure.
+ssm_status check_s6_dims(const ssm_dims *d)
+{
+    if (!d)
+        return SSM_ERR_INVALID_ARG;
+    if (d->batch < 0 || d->seqlen < 0 || d->dim < 0 || d->dstate < 0)
+        return SSM_ERR_INVALID_ARG;
+    if (!dtype_ok(d->dtype))
+        return SSM_ERR_UNSUPPORTED_DTYPE;
+    if (d->dstate < 1 || d->dstate > 16)
+        return SSM_ERR_UNSUPPORTED_SHAPE;
+    // int32 indexing limits inside the kernels
+    if (d->batch > INT32_MAX || d->seqlen > INT32_MAX || d->dim > INT32_MAX)
+        return SSM_ERR_UNSUPPORTED_SHAPE;
+    const int64_t vec = d->dtype == SSM_F32 ? 4 : 8;
+    if (d->dim % vec != 0)
+        return SSM_ERR_MISALIGNED;
+    return SSM_OK;
+}
+
+ssm_status check_dir(const ssm_dir_params *p)
+{
+    if (!p || !p->A || !p->B || !p->C)
+        return SSM_ERR_INVALID_ARG;
+    const void *ptrs[] = {p->delta_bias, p->A, p->B, p->C, p->D, p->z, p->last_state};
+    for (const void *q : ptrs)
+        if (q && !aligned16(q))
+            return SSM_ERR_MISALIGNED;
+    return SSM_OK;
+}
+
+bool empty_s6(const ssm_dims *d) { return d->batch == 0 || d->seqlen == 0 || d->dim == 0; }
+
+ssm_status zero_state(float *st, const ssm_dims *d, cudaStream_t s)
+{
+    if (!st)
+        return SSM_OK;
+    const size_t n = (size_t)d->batch * d->dim * d->dstate;
+    if (n == 0)
+        return SSM_OK;
+    return cudaMemsetAsync(st, 0, n * sizeof(float), s) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+ssm::DirArgs dir_args(const ssm_dir_params &p)
+{
+    return ssm::DirArgs{p.delta_bias, p.A, p.B, p.C, p.D, p.z, p.last_state};
+}
+
+ssm_status run_s6(const ssm_dims *dims, const void *x, const void *delta, int softplus, int ndir,
+                  int reverse, const ssm_dir_params *dirs, void *out, void *ws, size_t ws_bytes,
+                  cudaStream_t stream)
+{
+    const ssm::S6Plan plan = ssm::plan_s6(dims->batch, dims->seqlen, dims->dim, dims->dstate, ndir);
+    if (plan.workspace_bytes > 0) {
+        if (!ws || ws_bytes < plan.workspace_bytes)
+            return SSM_ERR_WORKSPACE_TOO_SMALL;
+        if (!aligned16(ws))
+            return SSM_ERR_MISALIGNED;
+    }
+    ssm::S6Args a;
+    memset(&a, 0, sizeof(a));
+    a.Bsz = (int)dims->batch;
+    a.L = (int)dims->seqlen;
+    a.D = (int)dims->dim;
+    a.N = (int)dims->dstate;
+    a.S = plan.S;
+    a.T = plan.T;
+    a.dtype = dims->dtype == SSM_F32 ? 0 : 1;
+    a.softplus = softplus ? 1 : 0;
+    a.ndir = ndir;
+    a.reverse = reverse ? 1 : 0;
+    a.x = x;
+    a.delta = delta;
+    for (int i = 0; i < ndir; i++)
+        a.dir[i] = dir_args(dirs[i]);
+    a.out = out;
+    if (plan.S > 1) {
+        const size_t nh = (size_t)ndir * a.Bsz * a.S * a.D * a.N;
+        a.carry_h = static_cast<float *>(ws);
+        a.carry_s = static_cast<float *>(ws) + ((nh + 63) / 64) * 64;
+    }
+    return ssm::launch_s6(a, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t ssm_scan_workspace_size(const ssm_dims *dims)
+{
+    if (check_s6_dims(dims) != SSM_OK || empty_s6(dims))
+        return 0;
+    return ssm::plan_s6(dims->batch, dims->seqlen, dims->dim, dims->dstate, 1).workspace_bytes;
+}
+
+size_t bidir_scan_workspace_size(const ssm_dims *dims)
+{
+    if (check_s6_dims(dims) != SSM_OK || empty_s6(dims))
+        return 0;
+    return ssm::plan_s6(dims->batch, dims->seqlen, dims->dim, dims->dstate, 2).workspace_bytes;
+}
+
+ssm_status ssm_scan_fwd(const ssm_dims *dims, const void *x, const void *delta,
+                        const float *delta_bias, int delta_softplus, const float *A,
+                        const void *B, const void *C, const float *D, const void *z, int reverse,
+                        void *out, float *last_state, void *workspace, size_t workspace_bytes,
+                        void *stream)
+{
+    ssm_status s = check_s6_dims(dims);
+    if (s != SSM_OK)
+        return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (empty_s6(dims)) {
+        if (last_state && !aligned16(last_state))
+            return SSM_ERR_MISALIGNED;
+        return zero_state(last_state, dims, st);
+    }
+    if (!x || !delta || !out)
+        return SSM_ERR_INVALID_ARG;
+    ssm_dir_params p{delta_bias, A, B, C, D, z, last_state};
+    if ((s = check_dir(&p)) != SSM_OK)
+        return s;
+    if (!aligned16(x) || !aligned16(delta) || !aligned16(out))
+        return SSM_ERR_MISALIGNED;
+    return run_s6(dims, x, delta, delta_softplus, 1, reverse, &p, out, workspace, workspace_bytes, st);
+}
+
+ssm_status bidir_scan_fwd(const ssm_dims *dims, const void *x, const void *delta,
+                          int delta_softplus, const ssm_dir_params *fwd,
+                          const ssm_dir_params *bwd, void *out, void *workspace,
+                          size_t workspace_bytes, void *stream)
+{
+    ssm_status s = check_s6_dims(dims);
+    if (s != SSM_OK)
+        return s;
+    if (!fwd || !bwd)
+        return SSM_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (empty_s6(dims)) {
+        if ((fwd->last_state && !aligned16(fwd->last_state)) ||
+            (bwd->last_state && !aligned16(bwd->last_state)))
+            return SSM_ERR_MISALIGNED;
+        if ((s = zero_state(fwd->last_state, dims, st)) != SSM_OK)
+            return s;
+        return zero_state(bwd->last_state, dims, st);
+    }
+    if (!x || !delta || !out)
+        return SSM_ERR_INVALID_ARG;
+    if ((s = check_dir(fwd)) != SSM_OK || (s = check_dir(bwd)) != SSM_OK)
+        return s;
+    if (!aligned16(x) || !aligned16(delta) || !aligned16(out))
+        return SSM_ERR_MISALIGNED;
+    const ssm_dir_params dirs[2] = {*fwd, *bwd};
+    return run_s6(dims, x, delta, delta_softplus, 2, 0, dirs, out, workspace, workspace_bytes, st);
+}
+
+size_t ssd_chunk_workspace_size(const ssd_dims *d)
+{
+    if (!d || d->batch < 0 || d->seqlen < 0 || d->nheads < 0 || d->headdim < 0 || d->dstate < 0 ||
+        d->chunk <= 0)
+        return 0;
+    return ssm::ssd_workspace_bytes(d->batch, d->seqlen, d->nheads, d->headdim, d->dstate, d->chunk);
+}
+
+ssm_status ssd_chunk_fwd(const ssd_dims *dims, const void *x, const void *delta,
+                         const float *delta_bias, int delta_softplus, const float *A,
+                         const void *B, const void *C, const float *D, const void *z, void *out,
+                         float *last_state, void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (!dims)
+        return SSM_ERR_INVALID_ARG;
+    if (dims->batch < 0 || dims->seqlen < 0 || dims->nheads < 0 || dims->headdim < 0 ||
+        dims->dstate < 0 || dims->chunk < 0)
+        return SSM_ERR_INVALID_ARG;
+    if (dims->dtype != SSM_BF16)
+        return SSM_ERR_UNSUPPORTED_DTYPE;
+    if (dims->headdim != 64 || dims->dstate != 128 || dims->chunk != 64)
+        return SSM_ERR_UNSUPPORTED_SHAPE;
+    if (dims->batch > INT32_MAX || dims->seqlen > INT32_MAX || dims->nheads > INT32_MAX)
+        return SSM_ERR_UNSUPPORTED_SHAPE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (dims->batch == 0 || dims->nheads == 0)
+        return SSM_OK;
+    if (dims->seqlen > 0 && (!x || !delta || !A || !B || !C || !out))
+        return SSM_ERR_INVALID_ARG;
+    const void *ptrs[] = {x, delta, delta_bias, A, B, C, D, z, out, last_state};
+    for (const void *q : ptrs)
+        if (q && !aligned16(q))
+            return SSM_ERR_MISALIGNED;
+    if (dims->seqlen == 0) {
+        if (!last_state)
+            return SSM_OK;
+        const size_t n = (size_t)dims->batch * dims->nheads * dims->headdim * dims->dstate;
+        return cudaMemsetAsync(last_state, 0, n * sizeof(float), st) == cudaSuccess ? SSM_OK
+                                                                                    : SSM_ERR_CUDA;
+    }
+    const size_t need = ssm::ssd_workspace_bytes(dims->batch, dims->seqlen, dims->nheads,
+                                                 dims->headdim, dims->dstate, dims->chunk);
+    if (need > 0) {
+        if (!workspace || workspace_bytes < need)
+            return SSM_ERR_WORKSPACE_TOO_SMALL;
+        if (!aligned16(workspace))
+            return SSM_ERR_MISALIGNED;
+    }
+    ssm::SSDArgs a;
+    memset(&a, 0, sizeof(a));
+    a.Bsz = (int)dims->batch;
+    a.L = (int)dims->seqlen;
+    a.H = (int)dims->nheads;
+    a.P = (int)dims->headdim;
+    a.N = (int)dims->dstate;
+    a.Q = (int)dims->chunk;
+    a.softplus = delta_softplus ? 1 : 0;
+    a.x = x;
+    a.delta = delta;
+    a.B = B;
+    a.C = C;
+    a.z = z;
+    a.bias = delta_bias;
+    a.A = A;
+    a.D = D;
+    a.out = out;
+    a.last_state = last_state;
+    a.workspace = workspace;
+    const cudaError_t e = ssm::launch_ssd(a, st);
+    if (e == cudaErrorNotSupported)
+        return SSM_ERR_UNSUPPORTED_SHAPE;
+    return e == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+ssm_status ssm_check_device(void *stream)
+{
+    unsigned v = 0;
+    if (ssm::read_and_clear_device_error(&v, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return SSM_ERR_CUDA;
+    return v ? SSM_ERR_DEVICE_TIMEOUT : SSM_OK;
+}
+
+const char *ssm_status_string(ssm_status s)
+{
+    switch (s) {
+    case SSM_OK: return "SSM_OK";
+    case SSM_ERR_INVALID_ARG: return "SSM_ERR_INVALID_ARG: NULL required pointer or negative size";
+    case SSM_ERR_UNSUPPORTED_SHAPE: return "SSM_ERR_UNSUPPORTED_SHAPE: shape not supported";
+    case SSM_ERR_MISALIGNED: return "SSM_ERR_MISALIGNED: pointer or dim not aligned to 16 bytes";
+    case SSM_ERR_UNSUPPORTED_DTYPE: return "SSM_ERR_UNSUPPORTED_DTYPE: dtype not supported";
+    case SSM_ERR_WORKSPACE_TOO_SMALL: return "SSM_ERR_WORKSPACE_TOO_SMALL: workspace too small";
+    case SSM_ERR_CUDA: return "SSM_ERR_CUDA: a CUDA launch or runtime call failed";
+    case SSM_ERR_DEVICE_TIMEOUT: return "SSM_ERR_DEVICE_TIMEOUT: a device-side wait gave up";
+    }
+    return "unknown ssm_status";
+}
+
+int ssm_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,121 @@
+"""The C-ABI library on a machine without a GPU: it loads, exports every
+function include/ssm.h declares, and rejects bad arguments before launching
+anything (no call here reaches a kernel)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import selective_state_space_24_b200 as ssm
+from selective_state_space_24_b200 import build as ssm_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+FAKE = 0x7F0000000000  # 16-byte aligned stand-in address; never dereferenced here
+
+
+@pytest.fixture(scope="module")
+def lib():
+    ssm_build.build()
+    return ssm.load()
+
+
+def _declared_functions():
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if not h.endswith(".h"):
+            continue
+        txt = open(os.path.join(ROOT, "include", h)).read()
+        txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+        names += re.findall(r"^[A-Za-z_][\w\s\*]*?\b(\w+)\s*\([^;{]*\)\s*;", txt, flags=re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared_functions()
+    assert {"ssm_scan_fwd", "bidir_scan_fwd", "ssd_chunk_fwd"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+    assert set(names) == set(ssm.SIGNATURES), "binding and header disagree"
+
+
+def test_version_and_status_strings(lib):
+    assert lib.ssm_version() >= 100
+    for code in range(8):
+        assert lib.ssm_status_string(code).decode().startswith(ssm.STATUS[code])
+
+
+def _dims(B=2, L=8, D=16, N=16, dt=ssm.SSM_F32):
+    return ssm.ssm_dims(B, L, D, N, dt)
+
+
+def _scan(lib, dims, x=FAKE, delta=FAKE, A=FAKE, B=FAKE, C=FAKE, out=FAKE, ws=None, wsb=0,
+          z=None, last=None):
+    return lib.ssm_scan_fwd(ctypes.byref(dims) if dims is not None else None, x, delta, None, 1,
+                            A, B, C, None, z, 0, out, last, ws, wsb, None)
+
+
+def test_null_dims_and_pointers(lib):
+    assert _scan(lib, None) == 1
+    assert _scan(lib, _dims(), x=None) == 1
+    assert _scan(lib, _dims(), A=None) == 1
+    assert _scan(lib, _dims(), out=None) == 1
+    assert _scan(lib, _dims(B=-1)) == 1
+
+
+def test_shape_dtype_alignment(lib):
+    assert _scan(lib, _dims(N=17)) == 2
+    assert _scan(lib, _dims(N=0)) == 2
+    assert _scan(lib, _dims(dt=7)) == 4
+    assert _scan(lib, _dims(D=6)) == 3                       # f32 needs dim % 4 == 0
+    assert _scan(lib, _dims(D=12, dt=ssm.SSM_BF16)) == 3     # bf16 needs dim % 8 == 0
+    assert _scan(lib, _dims(), x=FAKE + 4) == 3
+    assert _scan(lib, _dims(), z=FAKE + 8) == 3
+
+
+def test_workspace_too_small(lib):
+    dims = _dims(B=1, L=4096, D=64, N=16)
+    need = lib.ssm_scan_workspace_size(ctypes.byref(dims))
+    assert need > 0
+    assert _scan(lib, dims, ws=None, wsb=0) == 5
+    assert _scan(lib, dims, ws=FAKE, wsb=need - 1) == 5
+    assert lib.ssm_scan_workspace_size(None) == 0
+
+
+def test_bidir_validation(lib):
+    dims = _dims()
+    good = ssm.ssm_dir_params(None, FAKE, FAKE, FAKE, None, None, None)
+    bad = ssm.ssm_dir_params(None, None, FAKE, FAKE, None, None, None)
+    mis = ssm.ssm_dir_params(None, FAKE, FAKE + 2, FAKE, None, None, None)
+    f = lambda fw, bw: lib.bidir_scan_fwd(ctypes.byref(dims), FAKE, FAKE, 1, fw, bw, FAKE, None,
+                                          0, None)
+    assert f(ctypes.byref(good), None) == 1
+    assert f(ctypes.byref(good), ctypes.byref(bad)) == 1
+    assert f(ctypes.byref(mis), ctypes.byref(good)) == 3
+
+
+def test_empty_problems_launch_nothing(lib):
+    # zero batch / seqlen with no last_state: valid, nothing to do
+    assert _scan(lib, _dims(B=0)) == 0
+    assert _scan(lib, _dims(L=0)) == 0
+    assert lib.ssm_scan_workspace_size(ctypes.byref(_dims(L=0))) == 0
+
+
+def test_ssd_validation(lib):
+    d = ssm.ssd_dims(1, 128, 2, 64, 128, 64, ssm.SSM_BF16)
+    call = lambda dims, x=FAKE: lib.ssd_chunk_fwd(ctypes.byref(dims), x, FAKE, None, 1, FAKE, FAKE,
+                                                  FAKE, None, None, FAKE, None, None, 0, None)
+    assert call(ssm.ssd_dims(1, 128, 2, 64, 128, 64, ssm.SSM_F32)) == 4
+    assert call(ssm.ssd_dims(1, 128, 2, 32, 128, 64, ssm.SSM_BF16)) == 2
+    assert call(d, x=None) == 1
+    assert call(d, x=FAKE + 2) == 3
+    assert call(ssm.ssd_dims(0, 128, 2, 64, 128, 64, ssm.SSM_BF16)) == 0
+
+
+def test_plan_is_deterministic(lib):
+    for dims in (_dims(64, 197, 768, 16), _dims(8, 1024, 768, 16, ssm.SSM_BF16),
+                 _dims(4, 16384, 192, 16, ssm.SSM_BF16)):
+        a = lib.bidir_scan_workspace_size(ctypes.byref(dims))
+        b = lib.bidir_scan_workspace_size(ctypes.byref(dims))
+        assert a == b
