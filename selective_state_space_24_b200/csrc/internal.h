@@ -39,15 +39,19 @@ struct S6Args {
     void *out;
     float *carry_h;  // [ndir][Bsz][S][D][N]
     float *carry_s;  // [ndir][Bsz][S][D]
+    float *stash;    // ndir == 2: fp32 (Bsz, L, D) parking space for the
+                     // first half of each direction's outputs (out itself
+                     // when out is fp32)
 };
 
 struct S6Plan {
     int S, T;
     size_t workspace_bytes;
+    size_t carry_h_off, carry_s_off, stash_off;  // byte offsets into the workspace
 };
 
-// Segment plan for a problem; depends on the sizes only.
-S6Plan plan_s6(int64_t Bsz, int64_t L, int64_t D, int64_t N, int ndir);
+// Segment plan for a problem; depends on the sizes and dtype only.
+S6Plan plan_s6(int64_t Bsz, int64_t L, int64_t D, int64_t N, int ndir, int dtype);
 
 cudaError_t launch_s6(const S6Args &a, cudaStream_t stream);
 

@@ -66,7 +66,9 @@ ssm_status run_s6(const ssm_dims *dims, const void *x, const void *delta, int so
                   int reverse, const ssm_dir_params *dirs, void *out, void *ws, size_t ws_bytes,
                   cudaStream_t stream)
 {
-    const ssm::S6Plan plan = ssm::plan_s6(dims->batch, dims->seqlen, dims->dim, dims->dstate, ndir);
+    const int dt = dims->dtype == SSM_F32 ? 0 : 1;
+    const ssm::S6Plan plan =
+        ssm::plan_s6(dims->batch, dims->seqlen, dims->dim, dims->dstate, ndir, dt);
     if (plan.workspace_bytes > 0) {
         if (!ws || ws_bytes < plan.workspace_bytes)
             return SSM_ERR_WORKSPACE_TOO_SMALL;
@@ -81,7 +83,7 @@ ssm_status run_s6(const ssm_dims *dims, const void *x, const void *delta, int so
     a.N = (int)dims->dstate;
     a.S = plan.S;
     a.T = plan.T;
-    a.dtype = dims->dtype == SSM_F32 ? 0 : 1;
+    a.dtype = dt;
     a.softplus = softplus ? 1 : 0;
     a.ndir = ndir;
     a.reverse = reverse ? 1 : 0;
@@ -90,11 +92,13 @@ ssm_status run_s6(const ssm_dims *dims, const void *x, const void *delta, int so
     for (int i = 0; i < ndir; i++)
         a.dir[i] = dir_args(dirs[i]);
     a.out = out;
+    char *w = static_cast<char *>(ws);
     if (plan.S > 1) {
-        const size_t nh = (size_t)ndir * a.Bsz * a.S * a.D * a.N;
-        a.carry_h = static_cast<float *>(ws);
-        a.carry_s = static_cast<float *>(ws) + ((nh + 63) / 64) * 64;
+        a.carry_h = reinterpret_cast<float *>(w + plan.carry_h_off);
+        a.carry_s = reinterpret_cast<float *>(w + plan.carry_s_off);
     }
+    if (ndir == 2)
+        a.stash = dt == 0 ? static_cast<float *>(out) : reinterpret_cast<float *>(w + plan.stash_off);
     return ssm::launch_s6(a, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
@@ -106,14 +110,16 @@ size_t ssm_scan_workspace_size(const ssm_dims *dims)
 {
     if (check_s6_dims(dims) != SSM_OK || empty_s6(dims))
         return 0;
-    return ssm::plan_s6(dims->batch, dims->seqlen, dims->dim, dims->dstate, 1).workspace_bytes;
+    return ssm::plan_s6(dims->batch, dims->seqlen, dims->dim, dims->dstate, 1,
+                        dims->dtype == SSM_F32 ? 0 : 1).workspace_bytes;
 }
 
 size_t bidir_scan_workspace_size(const ssm_dims *dims)
 {
     if (check_s6_dims(dims) != SSM_OK || empty_s6(dims))
         return 0;
-    return ssm::plan_s6(dims->batch, dims->seqlen, dims->dim, dims->dstate, 2).workspace_bytes;
+    return ssm::plan_s6(dims->batch, dims->seqlen, dims->dim, dims->dstate, 2,
+                        dims->dtype == SSM_F32 ? 0 : 1).workspace_bytes;
 }
 
 ssm_status ssm_scan_fwd(const ssm_dims *dims, const void *x, const void *delta,
