@@ -131,7 +131,8 @@ SSM_API size_t bidir_scan_workspace_size(const ssm_dims *dims);
  *   out = S6(x, delta, fwd, reverse = 0) + S6(x, delta, bwd, reverse = 1)
  * with x, delta (B, L, D) shared; fwd and bwd each as described for
  * ssm_dir_params (their last_state fields are optional outputs).
- * fwd and bwd must be non-NULL; out (B, L, D) dtype is written.
+ * fwd and bwd must be non-NULL, and either both or neither have a gate z
+ * (SSM_ERR_INVALID_ARG otherwise); out (B, L, D) dtype is written.
  */
 SSM_API ssm_status bidir_scan_fwd(const ssm_dims *dims, const void *x, const void *delta,
                           int delta_softplus, const ssm_dir_params *fwd,

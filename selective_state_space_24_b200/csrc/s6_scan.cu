@@ -10,22 +10,23 @@
 // parameter set, the two results summed.
 //
 // Work decomposition
-//   * One thread owns one (b, d, direction) column and keeps its N states in
-//     fp32 registers; the h sequence never leaves the SM (the pages' fusion
-//     rule: never materialise (B, L, D, N)).
-//   * Lanes of a warp own 32 consecutive channels, so every x / delta / z
-//     access of a warp is one contiguous row segment, prefetched one step
-//     ahead.  B[t] and C[t] are the same for every lane: each warp stages
-//     them for 16 steps at a time in shared memory as fp32 (zero-padded to
-//     the template state count) and reads them back as broadcast 16-byte
-//     loads.
-//   * Bidirectional: a CTA is a warp pair over the same 32 channels, the
+//   * One thread owns two adjacent channels of one (b, direction) and keeps
+//     their 2 x N states in fp32 registers; the h sequence never leaves the
+//     SM (the pages' fusion rule: never materialise (B, L, D, N)).  The state
+//     update runs on packed f32x2 FMA/MUL instructions (two states per
+//     instruction).
+//   * A warp owns 64 consecutive channels, so every x / delta / z access of a
+//     warp is one contiguous row segment.  Those rows arrive by cp.async in a
+//     per-warp shared-memory ring 4 to 8 steps ahead of use.  B[t] and C[t]
+//     are the same for every lane: each warp stages them 16 steps at a time
+//     in shared memory as fp32 (zero-padded to the template state count) and
+//     reads them back as broadcast 16-byte loads.
+//   * Bidirectional: a CTA is a warp pair over the same 64 channels, the
 //     forward warp walking its segment upward, the reversed warp downward.
 //     Each parks the first half of its outputs in an fp32 stash (the output
 //     itself for fp32, the workspace for bf16), the pair meets at one named
 //     barrier, and in the second half each adds the other direction's parked
-//     value and writes the final sum.  x and delta are read by both warps;
-//     the second read is served by L1/L2.
+//     value and writes the final sum, so out is written once.
 //   * Long sequences are cut into S segments (the chunked scan with
 //     state hand-off of the Mamba2 page sec. 3.2): a summary kernel computes
 //     each segment's local end state and sum of dt, a carry kernel composes
@@ -33,9 +34,9 @@
 //     rescans every segment from its true entering state.
 //   * exp(dt A) is 2^(dt A log2 e).  The first NS - NPOLY states use the MUFU
 //     ex2.approx instruction, the last NPOLY states a degree-5 polynomial on
-//     the FMA pipe (Cody-Waite style split into integer and fraction,
-//     minimax coefficients fitted by fit_exp2_poly.py), so that the MUFU and
-//     FMA pipes share the work.
+//     the FMA pipe (integer / fraction split of the exponent, minimax
+//     coefficients fitted by fit_exp2_poly.py), so that the MUFU and FMA
+//     pipes share the work.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -47,8 +48,18 @@ namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr int kTC = 16;        // steps per B/C staging chunk
-constexpr int kWarps = 2;      // warps per CTA
+constexpr int kWarps = 2;   // warps per CTA
+constexpr int kCh = 64;     // channels per warp (2 per lane)
+constexpr int kTC = 16;     // steps per B/C staging chunk
+constexpr int kSub = 4;     // steps per cp.async group
+constexpr int kStages = 2;  // cp.async groups in the ring
+constexpr int kSlots = kSub * kStages;
+#ifndef SSM_S6_MINB
+#define SSM_S6_MINB 6
+#endif
+constexpr int kMinBlocks = SSM_S6_MINB;   // CTAs per SM the register budget is sized for
+
+// ------------------------------------------------------------ math helpers
 
 __device__ __forceinline__ float ex2_mufu(float v)
 {
@@ -71,23 +82,26 @@ __device__ __forceinline__ float rcp_mufu(float v)
     return r;
 }
 
-// 2^v on the FMA pipe: v = j + f with j = rint(v), |f| <= 1/2; 2^f by a
-// degree-5 minimax polynomial (relative error 2.1e-7 in fp32); 2^j added to
-// the exponent field.  v is clamped to [-126, 127] so the exponent stays in
-// range.
-__device__ __forceinline__ float ex2_poly(float v)
+// 2^v for two values on the FMA pipe: v = j + f with j = rint(v), |f| <= 1/2;
+// 2^f by a degree-5 minimax polynomial (relative error 2.1e-7 in fp32); 2^j
+// added to the exponent field.  v is clamped to [-126, 127] so the exponent
+// stays in range.
+__device__ __forceinline__ float2 ex2_poly2(float2 v)
 {
-    v = fminf(fmaxf(v, -126.f), 127.f);
     const float kMagic = 12582912.f;  // 1.5 * 2^23: v + kMagic rounds v to an integer
-    const float t = v + kMagic;
-    const float f = v - (t - kMagic);
-    float p = 1.327647245e-03f;
-    p = fmaf(p, f, 9.675540961e-03f);
-    p = fmaf(p, f, 5.550713092e-02f);
-    p = fmaf(p, f, 2.402212024e-01f);
-    p = fmaf(p, f, 6.931469440e-01f);
-    p = fmaf(p, f, 1.000000119e+00f);
-    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+    v.x = fminf(fmaxf(v.x, -126.f), 127.f);
+    v.y = fminf(fmaxf(v.y, -126.f), 127.f);
+    const float2 t = __fadd2_rn(v, make_float2(kMagic, kMagic));
+    const float2 j = __fadd2_rn(t, make_float2(-kMagic, -kMagic));
+    const float2 f = __fadd2_rn(v, make_float2(-j.x, -j.y));
+    float2 p = make_float2(1.327647245e-03f, 1.327647245e-03f);
+    p = __ffma2_rn(p, f, make_float2(9.675540961e-03f, 9.675540961e-03f));
+    p = __ffma2_rn(p, f, make_float2(5.550713092e-02f, 5.550713092e-02f));
+    p = __ffma2_rn(p, f, make_float2(2.402212024e-01f, 2.402212024e-01f));
+    p = __ffma2_rn(p, f, make_float2(6.931469440e-01f, 6.931469440e-01f));
+    p = __ffma2_rn(p, f, make_float2(1.000000119e+00f, 1.000000119e+00f));
+    return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                       __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
 // softplus(v) = max(v, 0) + log1p(e), e = exp(-|v|) in (0, 1].  log1p(e) is
@@ -104,19 +118,28 @@ __device__ __forceinline__ float softplus_f(float v)
 
 __device__ __forceinline__ float silu_f(float z) { return z * rcp_mufu(1.f + ex2_mufu(-z * kLog2e)); }
 
+// ----------------------------------------------------- storage-type helpers
+
 template <typename T> struct IO;
 template <> struct IO<float> {
-    static __device__ __forceinline__ float ld(const float *p, size_t i) { return __ldg(p + i); }
-    static __device__ __forceinline__ void st(float *p, size_t i, float v) { p[i] = v; }
+    // two adjacent channels
+    static __device__ __forceinline__ float2 ld2(const void *p) { return *reinterpret_cast<const float2 *>(p); }
+    static __device__ __forceinline__ void st2(float *p, float2 v) { *reinterpret_cast<float2 *>(p) = v; }
+    static __device__ __forceinline__ float ld1(const float *p, size_t i) { return __ldg(p + i); }
 };
 template <> struct IO<__nv_bfloat16> {
-    static __device__ __forceinline__ float ld(const __nv_bfloat16 *p, size_t i)
+    static __device__ __forceinline__ float2 ld2(const void *p)
+    {
+        const uint32_t u = *reinterpret_cast<const uint32_t *>(p);
+        return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+    }
+    static __device__ __forceinline__ void st2(__nv_bfloat16 *p, float2 v)
+    {
+        *reinterpret_cast<__nv_bfloat162 *>(p) = __floats2bfloat162_rn(v.x, v.y);
+    }
+    static __device__ __forceinline__ float ld1(const __nv_bfloat16 *p, size_t i)
     {
         return __bfloat162float(__ldg(p + i));
-    }
-    static __device__ __forceinline__ void st(__nv_bfloat16 *p, size_t i, float v)
-    {
-        p[i] = __float2bfloat16_rn(v);
     }
 };
 
@@ -124,6 +147,16 @@ __device__ __forceinline__ bool first_in_order(int seg, int S, bool rev) { retur
 __device__ __forceinline__ bool last_in_order(int seg, int S, bool rev) { return rev ? seg == 0 : seg == S - 1; }
 
 __device__ __forceinline__ void pair_barrier() { asm volatile("bar.sync 1, 64;" ::: "memory"); }
+
+template <int BYTES>
+__device__ __forceinline__ void cp_async(void *smem, const void *gmem)
+{
+    const unsigned sa = (unsigned)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"(sa), "l"(gmem), "n"(BYTES) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int K> __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(K) : "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // Per-warp staging of B[t], C[t] for kTC steps.  Row i of a chunk holds
 // B (NS floats) then C (NS floats) of time t(i); lane l fills half l & 1
@@ -168,7 +201,7 @@ struct BCStage {
 #pragma unroll
                 for (int n = 0; n < NS; n++)
                     if (n < N)
-                        v[n] = IO<T>::ld(row, n);
+                        v[n] = IO<T>::ld1(row, n);
             }
         }
     }
@@ -182,37 +215,33 @@ struct BCStage {
     }
 };
 
-__device__ __forceinline__ void cp_async4(void *smem, const void *gmem)
-{
-    const unsigned sa = (unsigned)__cvta_generic_to_shared(smem);
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(sa), "l"(gmem) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int K> __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(K) : "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+template <bool V> struct PhaseTag {
+    static constexpr bool value = V;
+};
 
-__device__ __forceinline__ float bf16_bits_to_f(unsigned short u) { return __uint_as_float((unsigned)u << 16); }
+// Shared memory of one warp: the x / delta / z / stash ring and the B/C rows.
+template <typename T, int NS>
+struct WarpSmem {
+    static constexpr int kRowB = kCh * (int)sizeof(T);   // one x, delta or z row
+    static constexpr int kStashB = kCh * 4;              // one fp32 stash row
+    static constexpr int kSlotB = 3 * kRowB + kStashB;
+    char ring[kSlots * kSlotB];
+    float bc[2 * kTC * 2 * NS];
+};
 
-// Per-warp ring of kStages stages x kSub steps; each step slot holds four
-// 128-byte rows: x, delta, z (the warp's 32 channels in the storage dtype)
-// and the fp32 stash row.  Rows arrive by cp.async, kStages - 1 stages
-// (12 steps) ahead of use.
-constexpr int kSub = 4;
-constexpr int kStages = 4;
-constexpr int kRowB = 128;
-constexpr int kSlotB = 4 * kRowB;
-constexpr int kRingB = kStages * kSub * kSlotB;
-
-// One warp's scan over one segment of one column per lane.
+// One warp's scan over one segment, two channels per lane.
 //   SUMMARY: local end state from the given h, plus the sum of dt; no output.
 //   otherwise: outputs; BIDIR adds the midpoint exchange with the partner warp.
-template <typename T, int NS, int NPOLY, bool SUMMARY, bool BIDIR>
-__device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P, float *sbc,
-                                             char *ring, int b, int dbase, bool active, int s0,
-                                             int s1, bool rev, float (&h)[NS], float &sdt)
+template <typename T, int NS, int NPOLY, bool SUMMARY, bool BIDIR, bool GATE, bool SOFTPLUS>
+__device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P,
+                                             WarpSmem<T, NS> &sm, int b, int dbase, bool active,
+                                             int s0, int s1, bool rev, float2 (&h)[2][NS / 2],
+                                             float2 &sdt)
 {
+    using WS = WarpSmem<T, NS>;
+    static_assert(NPOLY % 2 == 0 && NPOLY <= NS, "NPOLY counts state pairs");
     const int lane = threadIdx.x & 31;
-    const int d = dbase + lane;
+    const int d = dbase + 2 * lane;
     const int N = a.N;
     const int Tn = s1 - s0;
     const size_t rowbase = (size_t)b * a.L;
@@ -221,41 +250,39 @@ __device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P, 
     const T *zp = static_cast<const T *>(P.z);
     T *out = static_cast<T *>(a.out);
     float *stash = a.stash;
-    const bool gate = zp != nullptr;
-    constexpr bool kF32 = sizeof(T) == 4;
 
-    float Al2[NS];
+    // A log2(e) for both channels, as pairs of states
+    float2 Ap[2][NS / 2];
 #pragma unroll
-    for (int n = 0; n < NS; n++)
-        Al2[n] = (active && n < N) ? P.A[(size_t)d * N + n] * kLog2e : 0.f;
-    const float bias = (active && P.bias) ? P.bias[d] : 0.f;
-    const float Dd = (active && P.D) ? P.D[d] : 0.f;
+    for (int c = 0; c < 2; c++)
+#pragma unroll
+        for (int k = 0; k < NS / 2; k++) {
+            const int n = 2 * k;
+            const float *Ar = P.A + (size_t)(d + c) * N;
+            Ap[c][k] = make_float2((active && n < N) ? Ar[n] * kLog2e : 0.f,
+                                   (active && n + 1 < N) ? Ar[n + 1] * kLog2e : 0.f);
+        }
+    const float2 bias = (active && P.bias) ? make_float2(P.bias[d], P.bias[d + 1]) : make_float2(0.f, 0.f);
+    const float2 Dd = (active && P.D) ? make_float2(P.D[d], P.D[d + 1]) : make_float2(0.f, 0.f);
 
     // midpoint of the pair exchange (see file comment)
-    const int M = rev ? Tn / 2 : (Tn + 1) / 2;
+    const int M = BIDIR ? (rev ? Tn / 2 : (Tn + 1) / 2) : Tn;
     auto tpos = [&](int i) { return rev ? s1 - 1 - i : s0 + i; };
-    const int w = lane & 15;                    // bf16 rows: 16 words of 2 channels
-    const bool wok = 2 * w < a.D - dbase;
+    auto slot_of = [&](int i) { return sm.ring + (i % kSlots) * WS::kSlotB; };
 
-    // copy x / delta / z (and the stash when allowed) of step i into its slot
+    // copy x / delta / z (and the stash row when allowed) of step i
     auto issue_step = [&](int i, bool with_stash) {
-        const int t = tpos(i);
-        char *slot = ring + ((i / kSub) % kStages) * kSub * kSlotB + (i % kSub) * kSlotB;
-        const size_t ro = (rowbase + t) * a.D + dbase;
-        if (kF32) {
-            if (active) {
-                cp_async4(slot + lane * 4, x + ro + lane);
-                cp_async4(slot + kRowB + lane * 4, dl + ro + lane);
-                if (!SUMMARY && gate)
-                    cp_async4(slot + 2 * kRowB + lane * 4, zp + ro + lane);
-            }
-        } else if (wok) {
-            cp_async4(slot + (lane >> 4) * kRowB + w * 4, (lane < 16 ? x : dl) + ro + 2 * w);
-            if (!SUMMARY && gate && lane < 16)
-                cp_async4(slot + 2 * kRowB + w * 4, zp + ro + 2 * w);
+        char *slot = slot_of(i);
+        const size_t ro = (rowbase + tpos(i)) * a.D + d;
+        if (active) {
+            constexpr int E = 2 * (int)sizeof(T);
+            cp_async<E>(slot + lane * E, x + ro);
+            cp_async<E>(slot + WS::kRowB + lane * E, dl + ro);
+            if (!SUMMARY && GATE)
+                cp_async<E>(slot + 2 * WS::kRowB + lane * E, zp + ro);
+            if (BIDIR && with_stash)
+                cp_async<8>(slot + 3 * WS::kRowB + lane * 8, stash + ro);
         }
-        if (BIDIR && with_stash && i >= M && active)
-            cp_async4(slot + 3 * kRowB + lane * 4, stash + ro + lane);
     };
     auto issue_chunk = [&](int c, bool with_stash) {
 #pragma unroll
@@ -268,160 +295,219 @@ __device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P, 
     };
 
     BCStage<T, NS> stg;
-    stg.load(static_cast<const T *>(P.B), static_cast<const T *>(P.C), N, rowbase, s0, s1, rev, 0,
-             lane);
-    stg.store(sbc, lane);
-    constexpr int kSubPerTC = kTC / kSub;
-    const int nbc = (Tn + kTC - 1) / kTC;
-    const int nchunks = (Tn + kSub - 1) / kSub;
-    bool stash_ok = false;
+    const T *Bm = static_cast<const T *>(P.B);
+    const T *Cm = static_cast<const T *>(P.C);
+    stg.load(Bm, Cm, N, rowbase, s0, s1, rev, 0, lane);
+    stg.store(sm.bc, lane);
+    stg.load(Bm, Cm, N, rowbase, s0, s1, rev, kTC, lane);
 #pragma unroll
     for (int c = 0; c < kStages - 1; c++)
         issue_chunk(c, false);
     __syncwarp();
 
-    for (int c = 0; c < nchunks; c++) {
-        issue_chunk(c + kStages - 1, stash_ok);
+    bool with_stash = false;
+    // chunk management at a group-aligned step: refill the stage consumed
+    // last, wait for the one holding step i, rotate the B/C staging
+    auto chunk_mgmt = [&](int i) {
+        __syncwarp();
+        issue_chunk(i / kSub + kStages - 1, with_stash);
         cp_async_wait<kStages - 1>();
+        if ((i & (kTC - 1)) == 0 && i > 0) {
+            stg.store(sm.bc + ((i / kTC) & 1) * kTC * 2 * NS, lane);
+            stg.load(Bm, Cm, N, rowbase, s0, s1, rev, i + kTC, lane);
+        }
         __syncwarp();
-        const int kb = c / kSubPerTC;
-        if (c % kSubPerTC == 0 && kb + 1 < nbc)
-            stg.load(static_cast<const T *>(P.B), static_cast<const T *>(P.C), N, rowbase, s0, s1,
-                     rev, (kb + 1) * kTC, lane);
-        const float *cur = sbc + (kb & 1) * kTC * 2 * NS + (c % kSubPerTC) * kSub * 2 * NS;
-        const char *stage = ring + (c % kStages) * kSub * kSlotB;
+    };
+    // Step stages.  load_dt: operands from the ring and dt (independent of h);
+    // recur: the state update and readout (the only part that depends on the
+    // previous step); finish: skip term, gate, store.
+    struct StepIn {
+        float2 xv, zv, dt;
+    };
+    auto load_dt = [&](int i) {
+        const char *slot = slot_of(i);
+        StepIn o;
+        o.xv = IO<T>::ld2(slot + lane * 2 * sizeof(T));
+        const float2 dv = IO<T>::ld2(slot + WS::kRowB + lane * 2 * sizeof(T));
+        o.zv = make_float2(0.f, 0.f);
+        if (!SUMMARY && GATE)
+            o.zv = IO<T>::ld2(slot + 2 * WS::kRowB + lane * 2 * sizeof(T));
+        o.dt = make_float2(dv.x + bias.x, dv.y + bias.y);
+        if (SOFTPLUS)
+            o.dt = make_float2(softplus_f(o.dt.x), softplus_f(o.dt.y));
+        if (!SUMMARY && GATE)
+            o.zv = make_float2(silu_f(o.zv.x), silu_f(o.zv.y));   // zv now holds the gate
+        return o;
+    };
+    auto recur = [&](int i, const StepIn &in) {
+        const float2 dtc[2] = {make_float2(in.dt.x, in.dt.x), make_float2(in.dt.y, in.dt.y)};
+        const float2 dtx[2] = {make_float2(in.dt.x * in.xv.x, in.dt.x * in.xv.x),
+                               make_float2(in.dt.y * in.xv.y, in.dt.y * in.xv.y)};
+        const float4 *row = reinterpret_cast<const float4 *>(sm.bc + (i & (2 * kTC - 1)) * 2 * NS);
+        float2 ya[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        float2 yb[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        if (SUMMARY)
+            sdt = __fadd2_rn(sdt, in.dt);
 #pragma unroll
-        for (int j = 0; j < kSub; j++) {
-            const int i = c * kSub + j;
-            if (i >= Tn)
-                break;
-            if (BIDIR && i == M) {
-                pair_barrier();
-                stash_ok = true;
-                // steps already in flight were issued without their stash rows
-                const int fr = min(Tn, (c + kStages) * kSub);
-                for (int ii = M; ii < fr; ii++) {
-                    char *slot = ring + ((ii / kSub) % kStages) * kSub * kSlotB + (ii % kSub) * kSlotB;
-                    if (active)
-                        cp_async4(slot + 3 * kRowB + lane * 4,
-                                  stash + (rowbase + tpos(ii)) * a.D + d);
-                }
-                cp_async_wait_all();
-                __syncwarp();
-            }
-            const char *slot = stage + j * kSlotB;
-            float xv, dv, zv = 0.f;
-            if (kF32) {
-                xv = *reinterpret_cast<const float *>(slot + lane * 4);
-                dv = *reinterpret_cast<const float *>(slot + kRowB + lane * 4);
-                if (!SUMMARY && gate)
-                    zv = *reinterpret_cast<const float *>(slot + 2 * kRowB + lane * 4);
-            } else {
-                xv = bf16_bits_to_f(*reinterpret_cast<const unsigned short *>(slot + lane * 2));
-                dv = bf16_bits_to_f(*reinterpret_cast<const unsigned short *>(slot + kRowB + lane * 2));
-                if (!SUMMARY && gate)
-                    zv = bf16_bits_to_f(
-                        *reinterpret_cast<const unsigned short *>(slot + 2 * kRowB + lane * 2));
-            }
-            float dt = dv + bias;
-            if (a.softplus)
-                dt = softplus_f(dt);
-            const float dtx = dt * xv;
-            const float4 *row = reinterpret_cast<const float4 *>(cur + j * 2 * NS);
-            if (SUMMARY) {
-                sdt += dt;
+        for (int q = 0; q < NS / 4; q++) {
+            const float4 bq = row[q];
+            float4 cq = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (!SUMMARY)
+                cq = row[NS / 4 + q];
+            const float2 bp[2] = {make_float2(bq.x, bq.y), make_float2(bq.z, bq.w)};
+            const float2 cp[2] = {make_float2(cq.x, cq.y), make_float2(cq.z, cq.w)};
 #pragma unroll
-                for (int q = 0; q < NS / 4; q++) {
-                    const float4 bq = row[q];
-                    const float bb[4] = {bq.x, bq.y, bq.z, bq.w};
+            for (int r = 0; r < 2; r++) {
+                const int k = 2 * q + r;   // state pair index
 #pragma unroll
-                    for (int r = 0; r < 4; r++) {
-                        const int n = 4 * q + r;
-                        const float e = n < NS - NPOLY ? ex2_mufu(dt * Al2[n]) : ex2_poly(dt * Al2[n]);
-                        h[n] = fmaf(e, h[n], dtx * bb[r]);
+                for (int c = 0; c < 2; c++) {
+                    const float2 v = __fmul2_rn(dtc[c], Ap[c][k]);
+                    float2 e;
+                    if (2 * k < NS - NPOLY) {
+                        e.x = ex2_mufu(v.x);
+                        e.y = ex2_mufu(v.y);
+                    } else {
+                        e = ex2_poly2(v);
                     }
-                }
-            } else {
-                float y0 = 0.f, y1 = 0.f;
-#pragma unroll
-                for (int q = 0; q < NS / 4; q++) {
-                    const float4 bq = row[q];
-                    const float4 cq = row[NS / 4 + q];
-                    const float bb[4] = {bq.x, bq.y, bq.z, bq.w};
-                    const float cc[4] = {cq.x, cq.y, cq.z, cq.w};
-#pragma unroll
-                    for (int r = 0; r < 4; r++) {
-                        const int n = 4 * q + r;
-                        const float e = n < NS - NPOLY ? ex2_mufu(dt * Al2[n]) : ex2_poly(dt * Al2[n]);
-                        h[n] = fmaf(e, h[n], dtx * bb[r]);
-                        if (r & 1)
-                            y1 = fmaf(cc[r], h[n], y1);
+                    h[c][k] = __ffma2_rn(e, h[c][k], __fmul2_rn(dtx[c], bp[r]));
+                    if (!SUMMARY) {
+                        if (r == 0)
+                            ya[c] = __ffma2_rn(cp[r], h[c][k], ya[c]);
                         else
-                            y0 = fmaf(cc[r], h[n], y0);
+                            yb[c] = __ffma2_rn(cp[r], h[c][k], yb[c]);
                     }
-                }
-                float y = fmaf(Dd, xv, y0 + y1);
-                if (gate)
-                    y *= silu_f(zv);
-                if (active) {
-                    const size_t io = (rowbase + tpos(i)) * a.D + d;
-                    if (!BIDIR)
-                        IO<T>::st(out, io, y);
-                    else if (i < M)
-                        stash[io] = y;
-                    else
-                        IO<T>::st(out, io, y + *reinterpret_cast<const float *>(slot + 3 * kRowB + lane * 4));
                 }
             }
         }
-        __syncwarp();
-        if (c % kSubPerTC == kSubPerTC - 1 && kb + 1 < nbc) {
-            stg.store(sbc + ((kb + 1) & 1) * kTC * 2 * NS, lane);
-            __syncwarp();
+        const float2 s0v = __fadd2_rn(ya[0], yb[0]);
+        const float2 s1v = __fadd2_rn(ya[1], yb[1]);
+        return make_float2(s0v.x + s0v.y, s1v.x + s1v.y);
+    };
+    auto finish = [&](int i, const StepIn &in, float2 ys, auto phase2_tag) {
+        constexpr bool kPhase2 = decltype(phase2_tag)::value;
+        if (SUMMARY)
+            return;
+        float2 y = make_float2(fmaf(Dd.x, in.xv.x, ys.x), fmaf(Dd.y, in.xv.y, ys.y));
+        if (GATE) {
+            y.x *= in.zv.x;
+            y.y *= in.zv.y;
         }
+        if (active) {
+            const size_t io = (rowbase + tpos(i)) * a.D + d;
+            if (!BIDIR) {
+                IO<T>::st2(out + io, y);
+            } else if (!kPhase2) {
+                *reinterpret_cast<float2 *>(stash + io) = y;
+            } else {
+                const float2 o = *reinterpret_cast<const float2 *>(slot_of(i) + 3 * WS::kRowB + lane * 8);
+                IO<T>::st2(out + io, make_float2(y.x + o.x, y.y + o.y));
+            }
+        }
+    };
+    auto step = [&](int i, auto phase2_tag) {
+        const StepIn in = load_dt(i);
+        finish(i, in, recur(i, in), phase2_tag);
+    };
+    // a full group of kSub steps: all operands and dt first, then the
+    // recurrences back to back, then the epilogues
+    auto group = [&](int i, auto phase2_tag) {
+        StepIn in[kSub];
+        float2 ys[kSub];
+#pragma unroll
+        for (int j = 0; j < kSub; j++)
+            in[j] = load_dt(i + j);
+#pragma unroll
+        for (int j = 0; j < kSub; j++)
+            ys[j] = recur(i + j, in[j]);
+#pragma unroll
+        for (int j = 0; j < kSub; j++)
+            finish(i + j, in[j], ys[j], phase2_tag);
+    };
+    // steps [i0, i1): unaligned head one by one, then straight-line groups of
+    // kSub steps (so consecutive steps' independent work can interleave),
+    // then the tail
+    auto run = [&](int i0, int i1, auto phase2_tag) {
+        int i = i0;
+        for (; i < i1 && (i & (kSub - 1)) != 0; i++)
+            step(i, phase2_tag);
+        for (; i + kSub <= i1; i += kSub) {
+            chunk_mgmt(i);
+            group(i, phase2_tag);
+        }
+        if (i < i1) {
+            chunk_mgmt(i);
+            for (; i < i1; i++)
+                step(i, phase2_tag);
+        }
+    };
+
+    run(0, M, PhaseTag<false>{});
+    if (BIDIR) {
+        pair_barrier();
+        with_stash = true;
+        // steps already in flight were issued without their stash rows
+        const int issued = min(Tn, ((M + kSub - 1) / kSub + kStages - 1) * kSub);
+        for (int i = M; i < issued; i++)
+            if (active)
+                cp_async<8>(slot_of(i) + 3 * WS::kRowB + lane * 8,
+                            stash + (rowbase + tpos(i)) * a.D + d);
+        cp_async_wait_all();
+        __syncwarp();
+        run(M, Tn, PhaseTag<true>{});
     }
     cp_async_wait_all();
-    if (BIDIR && M == Tn)
-        pair_barrier();
 }
 
+template <typename T, int NS>
+constexpr int smem_bytes() { return kWarps * (int)sizeof(WarpSmem<T, NS>); }
+
 // ---------------------------------------------------------------- summary
-template <typename T, int NS, int NPOLY>
-__global__ void __launch_bounds__(64, 8) s6_summary_kernel(const S6Args a)
+template <typename T, int NS, int NPOLY, bool SOFTPLUS>
+__global__ void __launch_bounds__(64, kMinBlocks) s6_summary_kernel(const S6Args a)
 {
-    __shared__ __align__(16) float sbc[kWarps][2 * kTC * 2 * NS];
-    __shared__ __align__(16) char ring[kWarps][kRingB];
+    extern __shared__ __align__(16) char smem_raw[];
+    WarpSmem<T, NS> *sm = reinterpret_cast<WarpSmem<T, NS> *>(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int dbase = (blockIdx.x * kWarps + warp) * 32;
-    const int d = dbase + lane;
+    const int dbase = (blockIdx.x * kWarps + warp) * kCh;
+    const int d = dbase + 2 * lane;
     const int seg = blockIdx.y;
     const int dsel = blockIdx.z % a.ndir;
     const int b = blockIdx.z / a.ndir;
     const bool rev = a.ndir == 2 ? dsel == 1 : a.reverse != 0;
-    if (last_in_order(seg, a.S, rev) || (blockIdx.x * kWarps + warp) * 32 >= a.D)
+    if (last_in_order(seg, a.S, rev) || dbase >= a.D)
         return;
     const bool active = d < a.D;
     const int s0 = seg * a.T, s1 = min(a.L, s0 + a.T);
-    float h[NS];
+    float2 h[2][NS / 2];
 #pragma unroll
-    for (int n = 0; n < NS; n++)
-        h[n] = 0.f;
-    float sdt = 0.f;
-    scan_segment<T, NS, NPOLY, true, false>(a, a.dir[dsel], sbc[warp], ring[warp], b, dbase,
-                                            active, s0, s1, rev, h, sdt);
+    for (int c = 0; c < 2; c++)
+#pragma unroll
+        for (int k = 0; k < NS / 2; k++)
+            h[c][k] = make_float2(0.f, 0.f);
+    float2 sdt = make_float2(0.f, 0.f);
+    scan_segment<T, NS, NPOLY, true, false, false, SOFTPLUS>(a, a.dir[dsel], sm[warp], b, dbase,
+                                                             active, s0, s1, rev, h, sdt);
     if (!active)
         return;
-    const size_t ci = (((size_t)dsel * a.Bsz + b) * a.S + seg) * a.D + d;
+    const float sd[2] = {sdt.x, sdt.y};
 #pragma unroll
-    for (int n = 0; n < NS; n++)
-        if (n < a.N)
-            a.carry_h[ci * a.N + n] = h[n];
-    a.carry_s[ci] = sdt;
+    for (int c = 0; c < 2; c++) {
+        const size_t ci = (((size_t)dsel * a.Bsz + b) * a.S + seg) * a.D + d + c;
+#pragma unroll
+        for (int k = 0; k < NS / 2; k++) {
+            if (2 * k < a.N)
+                a.carry_h[ci * a.N + 2 * k] = h[c][k].x;
+            if (2 * k + 1 < a.N)
+                a.carry_h[ci * a.N + 2 * k + 1] = h[c][k].y;
+        }
+        a.carry_s[ci] = sd[c];
+    }
 }
 
 // ------------------------------------------------------------------ carry
 // Per (direction, b, d, n): walk the segments in scan order, replace each
-// summary by the state entering that segment.
+// summary by the state entering that segment.  Summaries are fetched 16
+// segments at a time ahead of the dependent chain.
 __global__ void s6_carry_kernel(const S6Args a)
 {
     const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -434,70 +520,113 @@ __global__ void s6_carry_kernel(const S6Args a)
     const int dsel = idx / ((size_t)a.N * a.D * a.Bsz);
     const bool rev = a.ndir == 2 ? dsel == 1 : a.reverse != 0;
     const float Al2 = a.dir[dsel].A[(size_t)d * a.N + n] * kLog2e;
+    const size_t cbase = ((size_t)dsel * a.Bsz + b) * a.S;   // segment index base
+    constexpr int kBatch = 16;
     float hin = 0.f;
-    for (int k = 0; k < a.S; k++) {
-        const int seg = rev ? a.S - 1 - k : k;
-        const size_t ci = (((size_t)dsel * a.Bsz + b) * a.S + seg) * a.D + d;
-        if (k == a.S - 1) {
-            a.carry_h[ci * a.N + n] = hin;
-            break;
+    for (int k0 = 0; k0 < a.S; k0 += kBatch) {
+        float hl[kBatch], sd[kBatch];
+#pragma unroll
+        for (int j = 0; j < kBatch; j++) {
+            const int k = k0 + j;
+            hl[j] = 0.f;
+            sd[j] = 0.f;
+            if (k < a.S - 1) {   // the last segment in scan order has no summary
+                const int seg = rev ? a.S - 1 - k : k;
+                const size_t ci = (cbase + seg) * a.D + d;
+                hl[j] = a.carry_h[ci * a.N + n];
+                sd[j] = a.carry_s[ci];
+            }
         }
-        const float hl = a.carry_h[ci * a.N + n];
-        const float s = a.carry_s[ci];
-        a.carry_h[ci * a.N + n] = hin;
-        hin = fmaf(ex2_mufu(Al2 * s), hin, hl);
+#pragma unroll
+        for (int j = 0; j < kBatch; j++) {
+            const int k = k0 + j;
+            if (k < a.S) {
+                const int seg = rev ? a.S - 1 - k : k;
+                a.carry_h[((cbase + seg) * a.D + d) * a.N + n] = hin;
+                hin = fmaf(ex2_mufu(Al2 * sd[j]), hin, hl[j]);
+            }
+        }
     }
 }
 
 // ------------------------------------------------------------------- main
-template <typename T, int NS, int NPOLY, bool BIDIR>
-__global__ void __launch_bounds__(64, 8) s6_main_kernel(const S6Args a)
+template <typename T, int NS, int NPOLY, bool BIDIR, bool GATE, bool SOFTPLUS>
+__global__ void __launch_bounds__(64, kMinBlocks) s6_main_kernel(const S6Args a)
 {
-    __shared__ __align__(16) float sbc[kWarps][2 * kTC * 2 * NS];
-    __shared__ __align__(16) char ring[kWarps][kRingB];
+    extern __shared__ __align__(16) char smem_raw[];
+    WarpSmem<T, NS> *sm = reinterpret_cast<WarpSmem<T, NS> *>(smem_raw);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int dsel = BIDIR ? warp : 0;
-    const int dbase = BIDIR ? blockIdx.x * 32 : (blockIdx.x * kWarps + warp) * 32;
-    const int d = dbase + lane;
+    const int dbase = BIDIR ? blockIdx.x * kCh : (blockIdx.x * kWarps + warp) * kCh;
+    const int d = dbase + 2 * lane;
     const bool active = d < a.D;
     const int seg = blockIdx.y, b = blockIdx.z;
     const int s0 = seg * a.T, s1 = min(a.L, s0 + a.T);
     const bool rev = BIDIR ? dsel == 1 : a.reverse != 0;
     const DirArgs &P = a.dir[dsel];
-    if (!BIDIR && (blockIdx.x * kWarps + warp) * 32 >= a.D)
+    if (!BIDIR && dbase >= a.D)
         return;   // whole warp past the channels (never with a barrier partner)
-    float h[NS];
+    float2 h[2][NS / 2];
     const bool has_carry = a.S > 1 && !first_in_order(seg, a.S, rev);
-    const size_t ci = (((size_t)dsel * a.Bsz + b) * a.S + seg) * a.D + d;
 #pragma unroll
-    for (int n = 0; n < NS; n++)
-        h[n] = (active && n < a.N && has_carry) ? a.carry_h[ci * a.N + n] : 0.f;
-    float sdt = 0.f;
-    scan_segment<T, NS, NPOLY, false, BIDIR>(a, P, sbc[warp], ring[warp], b, dbase, active, s0, s1,
-                                             rev, h, sdt);
+    for (int c = 0; c < 2; c++) {
+        const size_t ci = (((size_t)dsel * a.Bsz + b) * a.S + seg) * a.D + d + c;
+#pragma unroll
+        for (int k = 0; k < NS / 2; k++) {
+            h[c][k].x = (active && has_carry && 2 * k < a.N) ? a.carry_h[ci * a.N + 2 * k] : 0.f;
+            h[c][k].y = (active && has_carry && 2 * k + 1 < a.N) ? a.carry_h[ci * a.N + 2 * k + 1] : 0.f;
+        }
+    }
+    float2 sdt = make_float2(0.f, 0.f);
+    scan_segment<T, NS, NPOLY, false, BIDIR, GATE, SOFTPLUS>(a, P, sm[warp], b, dbase, active, s0,
+                                                             s1, rev, h, sdt);
     if (active && P.last_state && last_in_order(seg, a.S, rev)) {
 #pragma unroll
-        for (int n = 0; n < NS; n++)
-            if (n < a.N)
-                P.last_state[((size_t)b * a.D + d) * a.N + n] = h[n];
+        for (int c = 0; c < 2; c++) {
+            float *ls = P.last_state + ((size_t)b * a.D + d + c) * a.N;
+#pragma unroll
+            for (int k = 0; k < NS / 2; k++) {
+                if (2 * k < a.N)
+                    ls[2 * k] = h[c][k].x;
+                if (2 * k + 1 < a.N)
+                    ls[2 * k + 1] = h[c][k].y;
+            }
+        }
     }
 }
 
-template <typename T, int NS, int NPOLY>
+template <typename KernelT>
+cudaError_t set_smem(KernelT k, int bytes)
+{
+    return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+template <typename T, int NS, int NPOLY, bool GATE, bool SOFTPLUS>
 cudaError_t launch_typed(const S6Args &a, cudaStream_t st)
 {
+    constexpr int smem = smem_bytes<T, NS>();
+    cudaError_t e;
     if (a.S > 1) {
-        dim3 g1((a.D + 63) / 64, a.S, a.Bsz * a.ndir);
-        s6_summary_kernel<T, NS, NPOLY><<<g1, 64, 0, st>>>(a);
+        auto ks = s6_summary_kernel<T, NS, NPOLY, SOFTPLUS>;
+        if ((e = set_smem(ks, smem)) != cudaSuccess)
+            return e;
+        dim3 g1((a.D + kWarps * kCh - 1) / (kWarps * kCh), a.S, a.Bsz * a.ndir);
+        ks<<<g1, 64, smem, st>>>(a);
         const size_t tot = (size_t)a.ndir * a.Bsz * a.D * a.N;
         s6_carry_kernel<<<(unsigned)((tot + 255) / 256), 256, 0, st>>>(a);
     }
     if (a.ndir == 2) {
-        dim3 g((a.D + 31) / 32, a.S, a.Bsz);
-        s6_main_kernel<T, NS, NPOLY, true><<<g, 64, 0, st>>>(a);
+        auto km = s6_main_kernel<T, NS, NPOLY, true, GATE, SOFTPLUS>;
+        if ((e = set_smem(km, smem)) != cudaSuccess)
+            return e;
+        dim3 g((a.D + kCh - 1) / kCh, a.S, a.Bsz);
+        km<<<g, 64, smem, st>>>(a);
     } else {
-        dim3 g((a.D + 63) / 64, a.S, a.Bsz);
-        s6_main_kernel<T, NS, NPOLY, false><<<g, 64, 0, st>>>(a);
+        auto km = s6_main_kernel<T, NS, NPOLY, false, GATE, SOFTPLUS>;
+        if ((e = set_smem(km, smem)) != cudaSuccess)
+            return e;
+        dim3 g((a.D + kWarps * kCh - 1) / (kWarps * kCh), a.S, a.Bsz);
+        km<<<g, 64, smem, st>>>(a);
     }
     return cudaGetLastError();
 }
@@ -506,29 +635,40 @@ cudaError_t launch_typed(const S6Args &a, cudaStream_t st)
 #define SSM_S6_NPOLY 0
 #endif
 
+template <typename T, int NS, int NPOLY>
+cudaError_t launch_flags(const S6Args &a, cudaStream_t st)
+{
+    const bool gate = a.dir[0].z != nullptr;
+    if (gate)
+        return a.softplus ? launch_typed<T, NS, NPOLY, true, true>(a, st)
+                          : launch_typed<T, NS, NPOLY, true, false>(a, st);
+    return a.softplus ? launch_typed<T, NS, NPOLY, false, true>(a, st)
+                      : launch_typed<T, NS, NPOLY, false, false>(a, st);
+}
+
 template <typename T>
 cudaError_t launch_ns(const S6Args &a, cudaStream_t st)
 {
     if (a.N <= 4)
-        return launch_typed<T, 4, 0>(a, st);
+        return launch_flags<T, 4, 0>(a, st);
     if (a.N <= 8)
-        return launch_typed<T, 8, 0>(a, st);
-    return launch_typed<T, 16, SSM_S6_NPOLY>(a, st);
+        return launch_flags<T, 8, 0>(a, st);
+    return launch_flags<T, 16, SSM_S6_NPOLY>(a, st);
 }
 
 }  // namespace
 
 S6Plan plan_s6(int64_t Bsz, int64_t L, int64_t D, int64_t N, int ndir, int dtype)
 {
-    S6Plan p{1, (int)L, 0, 0};
+    S6Plan p{1, (int)L, 0, 0, 0, 0};
     if (L <= 0)
         return p;
     const int64_t kMinT = 16;
-    const int64_t kTargetThreads = 148 * 512;
-    const int64_t cols = (int64_t)ndir * Bsz * D;
+    const int64_t kTargetThreads = 148 * 320;
+    const int64_t threads = (int64_t)ndir * Bsz * ((D + 1) / 2);
     int64_t S = 1;
-    if (cols > 0 && cols < kTargetThreads)
-        S = (kTargetThreads + cols - 1) / cols;
+    if (threads > 0 && threads < kTargetThreads)
+        S = (kTargetThreads + threads - 1) / threads;
     const int64_t smax = (L + kMinT - 1) / kMinT;
     if (S > smax)
         S = smax;

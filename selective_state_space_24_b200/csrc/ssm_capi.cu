@@ -170,6 +170,8 @@ ssm_status bidir_scan_fwd(const ssm_dims *dims, const void *x, const void *delta
         return SSM_ERR_INVALID_ARG;
     if ((s = check_dir(fwd)) != SSM_OK || (s = check_dir(bwd)) != SSM_OK)
         return s;
+    if ((fwd->z == nullptr) != (bwd->z == nullptr))
+        return SSM_ERR_INVALID_ARG;   // both directions gated, or neither
     if (!aligned16(x) || !aligned16(delta) || !aligned16(out))
         return SSM_ERR_MISALIGNED;
     const ssm_dir_params dirs[2] = {*fwd, *bwd};

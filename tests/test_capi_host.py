@@ -93,6 +93,8 @@ def test_bidir_validation(lib):
     assert f(ctypes.byref(good), None) == 1
     assert f(ctypes.byref(good), ctypes.byref(bad)) == 1
     assert f(ctypes.byref(mis), ctypes.byref(good)) == 3
+    gated = ssm.ssm_dir_params(None, FAKE, FAKE, FAKE, None, FAKE, None)
+    assert f(ctypes.byref(gated), ctypes.byref(good)) == 1   # one direction gated only
 
 
 def test_empty_problems_launch_nothing(lib):
