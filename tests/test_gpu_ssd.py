@@ -1,0 +1,97 @@
+"""GPU parity of the Mamba2 SSD chunked scan (tcgen05 path) against the
+float64 oracle, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import ssm_gen
+import selective_state_space_24_b200 as ssm
+from gpu_util import TOL, dev, f32dev, host, rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib(cuda_device):
+    ssm.load()
+
+
+def run_ssd(inp, last_state=True, gate=True, D=True, bias=True):
+    x = dev(inp.x, "bf16")
+    delta = dev(inp.delta, "bf16")
+    ls = None
+    if last_state:
+        ls = torch.full((inp.batch, inp.nheads, inp.headdim, inp.dstate), 7.0, device="cuda")
+    out = ssm.ssd_chunk_fwd(x, delta, f32dev(inp.A), dev(inp.B, "bf16"), dev(inp.C, "bf16"),
+                            chunk=inp.chunk, delta_bias=f32dev(inp.dt_bias) if bias else None,
+                            D=f32dev(inp.D) if D else None,
+                            z=dev(inp.z, "bf16") if gate else None, last_state=ls)
+    torch.cuda.synchronize()
+    ssm.check_device()
+    return out, ls
+
+
+def _ref(inp, cols=None, gate=True, D=True, bias=True):
+    return oracle.ssd_seq_arrays(inp.x, inp.delta, inp.A, inp.B, inp.C,
+                                 delta_bias=inp.dt_bias if bias else None, softplus=True,
+                                 D=inp.D if D else None, z=inp.z if gate else None, cols=cols,
+                                 nthreads=8)
+
+
+@pytest.mark.parametrize("L", [1, 63, 64, 65, 200, 333])
+def test_ssd_small_full_compare(L):
+    inp = ssm_gen.make_ssd_inputs(2, L, 3, 64, 128, 64, dtype="bf16", seed=L, random_D=True)
+    out, ls = run_ssd(inp)
+    ref, rls = _ref(inp)
+    e = rel_err(host(out), ref)
+    es = rel_err(ls.cpu().numpy(), rls)
+    assert e <= TOL["bf16"], f"out rel err {e:.3e}"
+    assert es <= TOL["bf16"], f"last_state rel err {es:.3e}"
+
+
+def test_ssd_matches_chunked_oracle_form():
+    inp = ssm_gen.make_ssd_inputs(1, 256, 2, 64, 128, 64, dtype="bf16", seed=5)
+    out, _ = run_ssd(inp, last_state=False)
+    refc, _ = oracle.ssd_chunked(inp, chunk=64, nthreads=8)
+    assert rel_err(host(out), refc) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("gate,D,bias", [(False, True, True), (True, False, True), (True, True, False)])
+def test_ssd_optional_inputs(gate, D, bias):
+    inp = ssm_gen.make_ssd_inputs(1, 150, 2, 64, 128, 64, dtype="bf16", seed=9, random_D=True)
+    out, ls = run_ssd(inp, gate=gate, D=D, bias=bias)
+    ref, rls = _ref(inp, gate=gate, D=D, bias=bias)
+    assert rel_err(host(out), ref) <= TOL["bf16"]
+    assert rel_err(ls.cpu().numpy(), rls) <= TOL["bf16"]
+
+
+def test_ssd_full_size_sampled():
+    """Mamba2 SSD workload: B 4, L 8192, 32 heads x 64, N 128, chunk 64;
+    64 sampled (b, h, p) columns over the whole sequence, plus their last state."""
+    inp = ssm_gen.make_workload(4)
+    out, ls = run_ssd(inp)
+    rng = np.random.default_rng(3)
+    P, H = inp.headdim, inp.nheads
+    cols = rng.choice(inp.batch * H * P, 64, replace=False)
+    ref, rls = _ref(inp, cols=cols)
+    g = host(out)
+    p = cols % P
+    h = (cols // P) % H
+    b = cols // (P * H)
+    assert rel_err(g[b, :, h, p], ref[b, :, h, p]) <= TOL["bf16"]
+    assert rel_err(ls.cpu().numpy()[b, h, p], rls[b, h, p]) <= TOL["bf16"]
+
+
+def test_ssd_deterministic():
+    inp = ssm_gen.make_ssd_inputs(2, 512, 4, 64, 128, 64, dtype="bf16", seed=11)
+    a, _ = run_ssd(inp)
+    b, _ = run_ssd(inp)
+    assert torch.equal(a, b)
+
+
+def test_ssd_unsupported_shape_rejected():
+    inp = ssm_gen.make_ssd_inputs(1, 64, 2, 32, 128, 64, dtype="bf16", seed=1)
+    with pytest.raises(ssm.SSMError):
+        ssm.ssd_chunk_fwd(dev(inp.x, "bf16"), dev(inp.delta, "bf16"), f32dev(inp.A),
+                          dev(inp.B, "bf16"), dev(inp.C, "bf16"))
