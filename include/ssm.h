@@ -123,6 +123,33 @@ SSM_API ssm_status ssm_scan_fwd(const ssm_dims *dims, const void *x, const void 
                         int reverse, void *out, float *last_state, void *workspace,
                         size_t workspace_bytes, void *stream);
 
+/* Bytes of the scratch array that ssm_scan_fwd_noalloc draws from. */
+#define SSM_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+/*
+ * ssm_scan_fwd for callers that cannot allocate device memory when they run
+ * the scan -- for example a plugin inside an inference engine that receives
+ * only its tensors and a stream at enqueue time, or a serving loop that
+ * allows no allocation after start-up.  The pages have no counterpart to
+ * this entry point; it is a convenience of this library.
+ *
+ * Arguments and results are those of ssm_scan_fwd without the workspace.
+ * The scratch comes from one array of SSM_NOALLOC_SCRATCH_BYTES that the
+ * library keeps on every GPU that loads it, until the process exits.  A
+ * problem that needs more (ssm_scan_workspace_size(dims) larger than
+ * SSM_NOALLOC_SCRATCH_BYTES) returns SSM_ERR_WORKSPACE_TOO_SMALL before
+ * anything runs.  The first call on each device looks up the array's device
+ * address with a CUDA runtime call; make that first call before any stream
+ * capture.  All calls share the array: nothing in it needs to start at zero,
+ * but calls whose kernels overlap on the GPU (other streams, other host
+ * threads) race on it.  Allocates nothing.
+ */
+SSM_API ssm_status ssm_scan_fwd_noalloc(const ssm_dims *dims, const void *x, const void *delta,
+                                        const float *delta_bias, int delta_softplus,
+                                        const float *A, const void *B, const void *C,
+                                        const float *D, const void *z, int reverse, void *out,
+                                        float *last_state, void *stream);
+
 /* Bytes of device workspace bidir_scan_fwd needs for `dims` (0 if none). */
 SSM_API size_t bidir_scan_workspace_size(const ssm_dims *dims);
 

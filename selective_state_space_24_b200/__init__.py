@@ -64,6 +64,8 @@ SIGNATURES = {
     "ssm_scan_workspace_size": (_sz, [ctypes.POINTER(ssm_dims)]),
     "ssm_scan_fwd": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp, _vp,
                             _int, _vp, _vp, _vp, _sz, _vp]),
+    "ssm_scan_fwd_noalloc": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp,
+                                    _vp, _int, _vp, _vp, _vp]),
     "bidir_scan_workspace_size": (_sz, [ctypes.POINTER(ssm_dims)]),
     "bidir_scan_fwd": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _int,
                               ctypes.POINTER(ssm_dir_params), ctypes.POINTER(ssm_dir_params), _vp,
@@ -182,6 +184,25 @@ def ssm_scan_fwd(x, delta, A, B, C, *, delta_bias=None, delta_softplus=True, D=N
                           int(bool(reverse)), _ptr(out), _ptr(last_state), _ptr(ws),
                           0 if ws is None else ws.numel(), _stream_handle(stream))
     _check(st, "ssm_scan_fwd")
+    return out
+
+
+def ssm_scan_fwd_noalloc(x, delta, A, B, C, *, delta_bias=None, delta_softplus=True, D=None,
+                         z=None, reverse=False, out=None, last_state=None, stream=None):
+    """ssm_scan_fwd without a workspace: the library's own scratch array is
+    used, for callers that cannot allocate device memory when they run the
+    scan.  Problems needing more than SSM_NOALLOC_SCRATCH_BYTES of scratch
+    raise SSMError (SSM_ERR_WORKSPACE_TOO_SMALL)."""
+    torch = _torch()
+    lib = capi()
+    dims = s6_dims(x, A.shape[1])
+    if out is None:
+        out = torch.empty_like(x)
+    st = lib.ssm_scan_fwd_noalloc(ctypes.byref(dims), _ptr(x), _ptr(delta), _ptr(delta_bias),
+                                  int(bool(delta_softplus)), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                  _ptr(z), int(bool(reverse)), _ptr(out), _ptr(last_state),
+                                  _stream_handle(stream))
+    _check(st, "ssm_scan_fwd_noalloc")
     return out
 
 
