@@ -101,6 +101,29 @@ def alu_peak_elems(sm_mhz: float) -> float:
     return SMS * sm_mhz * 1e6 * (64.0 / 3.0)
 
 
+# ------------------------------------------------------- multi-rank helpers
+
+def rank_seed(rank: int) -> int:
+    """Each rank scans its own batch (weak scaling): rank r draws seed r."""
+    return rank
+
+
+def max_over_ranks(ms: float, world: int, device=None) -> float:
+    """The job's time: the max of a per-rank device time over all ranks."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank_step: float, world: int, steps: int, job_ms: float) -> float:
+    """Units all ranks processed per second of job time."""
+    return units_per_rank_step * world * steps / (job_ms * 1e-3)
+
+
 # ----------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -258,7 +281,7 @@ def run_ours(args, rank, world, local_rank):
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
     info = workload_info(args.config)
-    wl = DeviceWorkload(args.config, seed=rank, device=device)
+    wl = DeviceWorkload(args.config, seed=rank_seed(rank), device=device)
     stream = torch.cuda.current_stream(device)
     sh = stream.cuda_stream
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
@@ -288,13 +311,9 @@ def run_ours(args, rank, world, local_rank):
     wall = time.perf_counter() - t_wall
     clocks = sampler.stop()
     step_ms = [a.elapsed_time(b) for a, b in evs]
-    total_ms = float(sum(step_ms))
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(float(sum(step_ms)), world, device)
     per_step_ms = total_ms / args.steps
-    value = info["elems"] * world * args.steps / (total_ms * 1e-3)
+    value = job_throughput(info["elems"], world, args.steps, total_ms)
 
     # roofline of the dominant kernel (the one launch of the step when the
     # plan has a single segment; else the step is summary + carry + main)
@@ -331,12 +350,8 @@ def run_ours(args, rank, world, local_rank):
             hb, db = wl.e2e_step(sh)
         e1.record(stream)
         torch.cuda.synchronize()
-        ems = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ems], dtype=torch.float64, device=device)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = {"value": info["elems"] * world * ke / (ems * 1e-3), "unit": "elements/s",
+        ems = max_over_ranks(e0.elapsed_time(e1), world, device)
+        e2e = {"value": job_throughput(info["elems"], world, ke, ems), "unit": "elements/s",
                "h2d_bytes_per_step": hb, "d2h_bytes_per_step": db, "steps": ke,
                "ms_per_step": ems / ke}
 
@@ -393,23 +408,29 @@ def _oracle_call(inp, info, cols, threads):
 
 def cpu_baseline(cfg, budget_s=10.0):
     """The float64 oracle as it stands, on this host's cores, over a sample of
-    the workload's columns sized to about `budget_s` of CPU time."""
-    import oracle
+    the workload's columns sized to about `budget_s` seconds (the whole
+    workload, repeated, when one pass is shorter)."""
     threads = len(os.sched_getaffinity(0))
     inp, info, cols, ncols_all = _oracle_sample(cfg, 1.0)
     per_col = info["elems"] / ncols_all
-    probe = cols[: max(threads * 4, 16)]
+    _oracle_call(inp, info, cols[: threads * 4], threads)        # warm the thread pool
+    probe = cols[: max(threads * 16, ncols_all // 16)]
     t0 = time.perf_counter()
     _oracle_call(inp, info, probe, threads)
-    dt = max(time.perf_counter() - t0, 1e-6)
-    n = int(min(len(cols), max(len(probe), len(probe) * budget_s / dt)))
-    sample = cols[:n]
+    per_col_s = max(time.perf_counter() - t0, 1e-6) / len(probe)
+    if per_col_s * ncols_all <= budget_s:
+        reps = max(1, int(budget_s / (per_col_s * ncols_all)))
+        sample, what = cols, f"the whole workload ({ncols_all} columns) x {reps}"
+    else:
+        reps = 1
+        sample = cols[: max(len(probe), int(budget_s / per_col_s))]
+        what = f"{len(sample)} of {ncols_all} (batch, channel) columns, whole sequence each"
     t0 = time.perf_counter()
-    _oracle_call(inp, info, sample, threads)
+    for _ in range(reps):
+        _oracle_call(inp, info, sample, threads)
     el = time.perf_counter() - t0
-    return {"value": n * per_col / el, "unit": "elements/s", "cores": threads, "kind": "oracle",
-            "sample": f"{n} of {ncols_all} (batch, channel) columns, whole sequence each, "
-                      f"{el:.1f} s, float64 C oracle with OpenMP",
+    return {"value": len(sample) * reps * per_col / el, "unit": "elements/s", "cores": threads,
+            "kind": "oracle", "sample": f"{what}, {el:.1f} s, float64 C oracle, OpenMP",
             "seconds": el}
 
 
