@@ -1,17 +1,19 @@
-"""Fits the polynomial that ex2_poly2 in s6_scan.cu uses for 2^f, |f| <= 1/2.
+"""Fits the polynomials s6_scan.cu uses:
+
+* 2^f for |f| <= 1/2 (ex2_poly2): degree 5, 2.1e-7 relative error in fp32,
+  the class of the MUFU ex2.approx instruction;
+* log1p(e) / e for e in [0, 1] (softplus_f): degree 7, 3.4e-7 relative.
 
 Remez exchange on the relative error, then the coefficients are rounded to
-float32 and the error of float32 Horner evaluation is re-measured.  Degree 5
-gives 2.1e-7 relative error, the class of the MUFU ex2.approx instruction.
+float32 and the error of float32 Horner evaluation is re-measured.
 
-    python fit_exp2_poly.py
+    python fit_polys.py
 """
 import numpy as np
-def remez(deg, a=-0.5, b=0.5, iters=30):
+def remez(deg, a=-0.5, b=0.5, iters=30, f=lambda t: np.exp2(t)):
     n = deg + 2
     k = np.arange(n)
     x = 0.5*(a+b) + 0.5*(b-a)*np.cos(np.pi*k/(n-1))[::-1]
-    f = lambda t: np.exp2(t)
     for _ in range(iters):
         # solve p(x_i) + (-1)^i E f(x_i) = f(x_i)   (relative error)
         M = np.zeros((n, n)); 
@@ -47,4 +49,18 @@ for deg in (4,5,6):
         p = (p.astype(np.float64)*t.astype(np.float64) + np.float64(ci)).astype(np.float32)
     e32 = np.max(np.abs(p.astype(np.float64)/np.exp2(t.astype(np.float64)) - 1))
     print(deg, 'minimax rel err %.3e, fp32 coeffs+Horner %.3e' % (e, e32))
+    print('   coeffs (c0..cdeg):', ', '.join('%.9ef' % v for v in c32))
+
+# log1p(e) / e on [0, 1]
+g = lambda e: np.where(e == 0, 1.0, np.log1p(e) / np.where(e == 0, 1, e))
+for deg in (7,):
+    c, e = remez(deg, 0.0, 1.0, 40, g)
+    c32 = c.astype(np.float32)
+    t = np.linspace(0, 1, 200001).astype(np.float32)
+    p = np.float32(c32[-1])
+    for ci in c32[-2::-1]:
+        p = (p.astype(np.float64)*t.astype(np.float64) + np.float64(ci)).astype(np.float32)
+    val = (p.astype(np.float64)*t).astype(np.float32)
+    ref = np.log1p(t.astype(np.float64)); m = ref > 0
+    print('log1p', deg, 'minimax rel err %.3e, fp32 %.3e' % (e, np.max(np.abs(val[m]/ref[m]-1))))
     print('   coeffs (c0..cdeg):', ', '.join('%.9ef' % v for v in c32))

@@ -47,7 +47,6 @@ namespace ssm {
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kWarps = 2;   // warps per CTA
 constexpr int kCh = 64;     // channels per warp (2 per lane)
 constexpr int kTC = 16;     // steps per B/C staging chunk
@@ -65,13 +64,6 @@ __device__ __forceinline__ float ex2_mufu(float v)
 {
     float r;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
-    return r;
-}
-
-__device__ __forceinline__ float lg2_mufu(float v)
-{
-    float r;
-    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
     return r;
 }
 
@@ -104,19 +96,36 @@ __device__ __forceinline__ float2 ex2_poly2(float2 v)
                        __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
-// softplus(v) = max(v, 0) + log1p(e), e = exp(-|v|) in (0, 1].  log1p(e) is
-// a 6-term series for e < 1/16 (truncation < 1e-8 relative) and
-// lg2(1 + e) ln 2 otherwise.
+// softplus(v) = max(v, 0) + log1p(e), e = exp(-|v|) in (0, 1], with
+// log1p(e) = e q(e) and q a degree-7 minimax polynomial for log1p(e) / e on
+// [0, 1] (relative error 3.4e-7 in fp32; coefficients from fit_polys.py).
 __device__ __forceinline__ float softplus_f(float v)
 {
     const float e = ex2_mufu(-fabsf(v) * kLog2e);
-    const float s = e * fmaf(e, fmaf(e, fmaf(e, fmaf(e, fmaf(e, -1.f / 6.f, 0.2f), -0.25f),
-                                              1.f / 3.f), -0.5f), 1.f);
-    const float g = lg2_mufu(1.f + e) * kLn2;
-    return fmaxf(v, 0.f) + (e < 0.0625f ? s : g);
+    float q = -8.539208211e-03f;
+    q = fmaf(q, e, 4.408963397e-02f);
+    q = fmaf(q, e, -1.076817140e-01f);
+    q = fmaf(q, e, 1.774524152e-01f);
+    q = fmaf(q, e, -2.449546307e-01f);
+    q = fmaf(q, e, 3.327547908e-01f);
+    q = fmaf(q, e, -4.999740422e-01f);
+    q = fmaf(q, e, 9.999998212e-01f);
+    return fmaf(e, q, fmaxf(v, 0.f));
 }
 
-__device__ __forceinline__ float silu_f(float z) { return z * rcp_mufu(1.f + ex2_mufu(-z * kLog2e)); }
+// silu(z) = z sigmoid(z).  fp32 data: z / (1 + 2^(-z log2 e)) with the MUFU
+// reciprocal.  bf16 data: z (1 + tanh(z / 2)) / 2 with the single MUFU
+// tanh.approx (relative error 2^-11, below the bf16 output rounding).
+template <typename T>
+__device__ __forceinline__ float silu_f(float z)
+{
+    if (sizeof(T) == 2) {
+        float t;
+        asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * z));
+        return 0.5f * z * (1.f + t);
+    }
+    return z * rcp_mufu(1.f + ex2_mufu(-z * kLog2e));
+}
 
 // ----------------------------------------------------- storage-type helpers
 
@@ -336,7 +345,7 @@ __device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P,
         if (SOFTPLUS)
             o.dt = make_float2(softplus_f(o.dt.x), softplus_f(o.dt.y));
         if (!SUMMARY && GATE)
-            o.zv = make_float2(silu_f(o.zv.x), silu_f(o.zv.y));   // zv now holds the gate
+            o.zv = make_float2(silu_f<T>(o.zv.x), silu_f<T>(o.zv.y));   // zv now holds the gate
         return o;
     };
     auto recur = [&](int i, const StepIn &in) {

@@ -23,13 +23,22 @@
 // lo accumulated), so they carry about 16 mantissa bits instead of 8; the
 // loaded operands X, B, C are exact in bf16.
 //
-// One CTA of 128 threads owns one (b, h) and walks its chunks in order.  TMA
-// brings each chunk's X, Z (64 x 64 bf16 tiles) and B, C (64 x 128) into a
-// two-stage shared-memory ring with 128-byte swizzle, which is directly the
-// layout the tensor core reads (C and B as K-major operands of C B^T, B as
-// an MN-major operand of B^T W, X as an MN-major operand of M X).  Thread 0
-// issues the TMA loads and the MMAs; completion is tracked by mbarriers with
-// bounded waits that set the library's error word if they give up.
+// One CTA owns one (b, h) and walks its chunks in order.  It has four
+// warpgroups of math threads -- warpgroup g owns columns [16 g, 16 g + 16) of
+// every 64-wide row --, one warp whose lane 0 issues the tensor-core MMAs
+// when the math threads signal (mbarriers) that the operands are written, and
+// one warp that computes dt and its cumulative sum up to three chunks ahead.
+// The loop is software-pipelined: while the math threads build chunk c's
+// decay matrix, update the state and write chunk c's outputs, the tensor core
+// runs chunk c + 1's first products (W and the Yo accumulator are
+// double-buffered by chunk parity, dt / cs triple-buffered).  The hi and lo
+// halves of S_in and of W sit side by side as one N = 128 operand, so each
+// of those products is one MMA per K-step.  TMA brings each chunk's X, Z
+// (64 x 64 bf16) and B, C (64 x 128) tiles into a three-stage shared-memory
+// ring with the 128-byte swizzle, which is directly the layout the tensor
+// core reads (C and B as K-major operands of C B^T, B as an MN-major operand
+// of B^T W, X as an MN-major operand of M X).  Every mbarrier wait is bounded
+// and sets the library's error word if it gives up.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -47,7 +56,11 @@ namespace {
 constexpr int kQ = 64;          // chunk length
 constexpr int kP = 64;          // head dim
 constexpr int kN = 128;         // state size
-constexpr int kThreads = 128;
+constexpr int kMath = 512;      // four warpgroups; warpgroup g owns columns [16 g, 16 g + 16)
+constexpr int kThreads = kMath + 64;   // + one warp that issues the MMAs, one that computes dt
+constexpr int kMmaWarp = kMath / 32, kDtWarp = kMath / 32 + 1;
+constexpr int kDtBufs = 3;             // dt / cs buffers, one per TMA stage
+static_assert(kDtBufs == 3, "the dt buffers are recycled with the TMA stages");
 constexpr float kLog2e = 1.4426950408889634f;
 
 // shared-memory plan (byte offsets from a 1024-aligned base)
@@ -58,15 +71,19 @@ constexpr int kStageZ = kTileX;
 constexpr int kStageB = 2 * kTileX;            // two halves (n 0..63, 64..127)
 constexpr int kStageC = 2 * kTileX + 2 * kTileBC;
 constexpr int kStageBytes = 2 * kTileX + 4 * kTileBC;   // 48 KB
-constexpr int kOffW = 2 * kStageBytes;                  // W hi, lo: 2 x 8 KB, rows j, MN-major
-constexpr int kOffM = kOffW + 2 * kTileX;               // M hi, lo: 2 x 8 KB, rows i, K-major
-constexpr int kOffS = kOffM + 2 * kTileX;               // S_in [buffer][hi, lo]: 4 x 16 KB, rows n, MN-major
+constexpr int kStages = 3;                              // TMA ring depth
+constexpr int kOffW = kStages * kStageBytes;            // W [buffer][hi, lo]: 4 x 8 KB, rows j, MN-major
+constexpr int kOffM = kOffW + 4 * kTileX;               // M [hi, lo]: 2 x 8 KB, rows i, K-major
 constexpr int kSBytes = kN * 128;
-constexpr int kOffVec = kOffS + 4 * kSBytes;            // cs[64], dt[64], warp sums
-constexpr int kSmemBytes = kOffVec + 3 * 64 * 4 + 1024; // + alignment slack
+constexpr int kOffS = kOffM + 2 * kTileX;               // S_in [hi, lo]: 2 x 16 KB, rows n, MN-major
+constexpr int kOffVec = kOffS + 2 * kSBytes;            // cs[kDtBufs][64], dt[kDtBufs][64]
+constexpr int kSmemBytes = kOffVec + 2 * kDtBufs * 64 * 4 + 1024; // + alignment slack
 
-// TMEM columns
-constexpr uint32_t kColG = 0, kColYo = 64, kColYd = 128, kColDS = 192, kTmemCols = 256;
+// TMEM columns.  dS and Yo hold the hi and lo halves side by side
+// (N = 128: columns [0, 64) from the hi operand, [64, 128) from lo); Yo is
+// double-buffered by chunk parity because chunk c's outputs read it after
+// chunk c + 1's first products were issued.
+constexpr uint32_t kColG = 0, kColDS = 64, kColYo = 192, kColYd = 448, kTmemCols = 512;
 
 constexpr long kWaitLimit = 1l << 26;
 
@@ -148,43 +165,37 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, i
         : "memory");
 }
 
-// 32 columns of one M = 64 accumulator row: threads t < 16 of warp w get row
-// 16 w + t, columns [col, col + 32); threads t >= 16 the same row, columns
-// [col + 32, col + 64).
-__device__ __forceinline__ void tmem_ld_half_row(uint32_t taddr, float (&v)[32])
+
+// 8 columns of one M = 64 accumulator row: threads t < 16 of warp w get row
+// 16 (w mod 4) + t, columns [col, col + 8); threads t >= 16 the same row,
+// columns [col + 8, col + 16).
+__device__ __forceinline__ void tmem_ld_eighth_row(uint32_t taddr, float (&v)[8])
 {
-    uint32_t r[32];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32], 32;"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
+    uint32_t r[8];
+    asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8], 8;"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-    for (int k = 0; k < 32; k++)
+    for (int k = 0; k < 8; k++)
         v[k] = __uint_as_float(r[k]);
 }
 
-// 32 consecutive columns of this thread's lane (an M = 128 accumulator row)
-__device__ __forceinline__ void tmem_ld_row32(uint32_t taddr, float *v)
+// 16 consecutive columns of this thread's lane (an M = 128 accumulator row)
+__device__ __forceinline__ void tmem_ld_row16(uint32_t taddr, float *v)
 {
-    uint32_t r[32];
+    uint32_t r[16];
     asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr));
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-    for (int k = 0; k < 32; k++)
+    for (int k = 0; k < 16; k++)
         v[k] = __uint_as_float(r[k]);
 }
+
 
 __device__ __forceinline__ float ex2f(float v)
 {
@@ -231,6 +242,11 @@ __device__ __forceinline__ float2 unpack_bf16(uint32_t u)
     return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 struct SSDKernelArgs {
     int Bsz, L, H, nchunks;
     int softplus;
@@ -246,29 +262,43 @@ __global__ void __launch_bounds__(kThreads, 1)
                      const __grid_constant__ CUtensorMap mapB, const __grid_constant__ CUtensorMap mapC,
                      const SSDKernelArgs args)
 {
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ __align__(8) uint64_t bar_tma[2];
-    __shared__ __align__(8) uint64_t bar_mma1, bar_mma2;
+    __shared__ __align__(8) uint64_t bar_tma[kStages];
+    __shared__ __align__(8) uint64_t bar_mma1[2];
+    __shared__ __align__(8) uint64_t bar_mma2;
+    __shared__ __align__(8) uint64_t bar_mready;  // math threads: M(c) written
+    __shared__ __align__(8) uint64_t bar_sready;  // math threads: S_in(c + 1), W(c + 1) written
+    __shared__ __align__(8) uint64_t bar_dt_full[kDtBufs];    // dt warp: dt / cs of a chunk written
+    __shared__ __align__(8) uint64_t bar_free[kDtBufs];       // math threads: done with a chunk's stage and dt
     __shared__ uint32_t tmem_base_sh;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int wq = warp & 3;      // TMEM lane quadrant of this warp
+    const int g = warp >> 2;      // warpgroup: column quarter
     const int bh = blockIdx.x;
     const int b = bh / args.H, h = bh % args.H;
     const int L = args.L;
-    float *cs_s = reinterpret_cast<float *>(sm + kOffVec);
-    float *dt_s = cs_s + 64;
-    float *wsum = dt_s + 64;
+    const int nch = args.nchunks;
+    float *cs_s = reinterpret_cast<float *>(sm + kOffVec);   // [kDtBufs][64], buffer c % kDtBufs
+    float *dt_s = cs_s + kDtBufs * 64;                        // [kDtBufs][64]
 
     const float bias = args.bias ? args.bias[h] : 0.f;
     const float Ah = args.A[h] * kLog2e;   // exponents are taken base 2
     const float Dh = args.D ? args.D[h] : 0.f;
 
     if (tid == 0) {
-        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bar_tma[0])));
-        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bar_tma[1])));
-        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bar_mma1)));
+        for (int k = 0; k < kStages; k++)
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bar_tma[k])));
+        for (int k = 0; k < 2; k++)
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bar_mma1[k])));
         asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bar_mma2)));
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(&bar_mready)), "r"(kMath));
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(&bar_sready)), "r"(kMath));
+        for (int k = 0; k < kDtBufs; k++) {
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 32;" ::"r"(smem_u32(&bar_dt_full[k])));
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(&bar_free[k])), "r"(kMath));
+        }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 0) {
@@ -276,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                      "r"(kTmemCols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
-    // zero S_in buffer 0 (the state entering chunk 0)
+    // zero S_in (hi and lo): the state entering chunk 0
     for (int k = tid; k < 2 * kSBytes / 16; k += kThreads)
         reinterpret_cast<uint4 *>(sm + kOffS)[k] = make_uint4(0, 0, 0, 0);
     fence_async_smem();
@@ -284,11 +314,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tb = tmem_base_sh;
-    const uint32_t tw = tb + ((uint32_t)(warp * 32) << 16);   // this warp's TMEM lanes
+    const uint32_t tw = tb + ((uint32_t)(wq * 32) << 16);   // this warp's TMEM lanes
 
     auto issue_tma = [&](int c) {
-        uint8_t *st = sm + (c & 1) * kStageBytes;
-        uint64_t *bar = &bar_tma[c & 1];
+        uint8_t *st = sm + (c % kStages) * kStageBytes;
+        uint64_t *bar = &bar_tma[c % kStages];
         const uint32_t bytes = args.has_z ? kStageBytes : kStageBytes - kTileX;
         asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                      : "memory");
@@ -301,236 +331,271 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(st + kStageC, &mapC, 0, t0, b, bar);
         tma_load_3d(st + kStageC + kTileBC, &mapC, 64, t0, b, bar);
     };
-    if (tid == 0) {
-        issue_tma(0);
-        if (args.nchunks > 1)
-            issue_tma(1);
-    }
 
-    // delta for the first chunk (threads 0..63 hold one step each)
-    auto load_delta = [&](int c) {
-        const int t = c * kQ + tid;
-        return (tid < kQ && t < L) ? __bfloat162float(args.delta[((size_t)b * L + t) * args.H + h]) : 0.f;
+    // raw delta of steps 2 lane, 2 lane + 1 of chunk c (dt warp)
+    auto load_delta2 = [&](int c) {
+        const int t = c * kQ + 2 * lane;
+        float2 d = make_float2(0.f, 0.f);
+        if (c < nch && t < L)
+            d.x = __bfloat162float(args.delta[((size_t)b * L + t) * args.H + h]);
+        if (c < nch && t + 1 < L)
+            d.y = __bfloat162float(args.delta[((size_t)b * L + t + 1) * args.H + h]);
+        return d;
     };
-    float dnext = load_delta(0);
-
-    // S: this thread's row n = tid, 64 columns p, fp32
-    float S[kP];
-#pragma unroll
-    for (int p = 0; p < kP; p++)
-        S[p] = 0.f;
-
-    const uint32_t idG = idesc_bf16(64, 64, 0, 0);    // C (K-major) x B (K-major)
-    const uint32_t idDS = idesc_bf16(128, 64, 1, 1);  // B^T (MN-major) x W (MN-major)
-    const uint32_t idYo = idesc_bf16(64, 64, 0, 1);   // C (K-major) x S_in (MN-major)
-    const uint32_t idYd = idesc_bf16(64, 64, 0, 1);   // M (K-major) x X (MN-major)
-
-    const int row_i = 16 * warp + (lane & 15);   // M = 64 accumulator row of this thread
-    const int hh = lane >> 4;                    // which 32-column half
-
-    for (int c = 0; c < args.nchunks; c++) {
-        uint8_t *st = sm + (c & 1) * kStageBytes;
-        const int t0 = c * kQ;
-        // ---- dt and the inclusive cumulative sum of dt A inside the chunk
-        float dt = 0.f;
-        if (tid < kQ && t0 + tid < L) {
-            dt = dnext + bias;
+    // dt and the inclusive cumulative sum of dt A (base-2 units) of chunk c
+    // into buffer c % kDtBufs; one warp, two steps per lane
+    auto chunk_dt = [&](int c, float2 draw) {
+        const int t = c * kQ + 2 * lane;
+        float d0 = 0.f, d1 = 0.f;
+        if (t < L) {
+            d0 = draw.x + bias;
             if (args.softplus)
-                dt = softplus_f(dt);
+                d0 = softplus_f(d0);
         }
-        if (c + 1 < args.nchunks)
-            dnext = load_delta(c + 1);
-        float a = dt * Ah;
+        if (t + 1 < L) {
+            d1 = draw.y + bias;
+            if (args.softplus)
+                d1 = softplus_f(d1);
+        }
+        const float a0 = d0 * Ah, a1 = d1 * Ah;
+        float incl = a0 + a1;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const float v = __shfl_up_sync(0xffffffffu, a, o);
+            const float v = __shfl_up_sync(0xffffffffu, incl, o);
             if (lane >= o)
-                a += v;
+                incl += v;
         }
-        if (lane == 31 && warp < 2)
-            wsum[warp] = a;
-        __syncthreads();
-        if (warp == 1)
-            a += wsum[0];
-        if (tid < kQ) {
-            cs_s[tid] = a;
-            dt_s[tid] = dt;
-        }
-        __syncthreads();
-        const float cs_end = cs_s[kQ - 1];
+        float *cs = cs_s + (c % kDtBufs) * 64, *dtv = dt_s + (c % kDtBufs) * 64;
+        *reinterpret_cast<float2 *>(cs + 2 * lane) = make_float2(incl - a1, incl);
+        *reinterpret_cast<float2 *>(dtv + 2 * lane) = make_float2(d0, d1);
+    };
 
-        // ---- wait for this chunk's tiles
-        const bool ok_tma = mbar_wait(&bar_tma[c & 1], (c >> 1) & 1);
-        (void)ok_tma;
-
-        // ---- W = exp(cs_end - cs_j) dt_j X[j, :], rows j, same swizzled layout as X
-        {
-            const int j = tid >> 1, half = tid & 1;
-            const float wj = ex2f(cs_end - cs_s[j]) * dt_s[j];
+    // W(c) = exp(cs_end - cs_j) dt_j X[j, :] as bf16 hi + lo, rows j, X's swizzled layout
+    auto build_w = [&](int c) {
+        const uint8_t *st = sm + (c % kStages) * kStageBytes;
+        const float *cs = cs_s + (c % kDtBufs) * 64, *dtv = dt_s + (c % kDtBufs) * 64;
+        uint8_t *wb = sm + kOffW + (c & 1) * 2 * kTileX;
+        const int j = tid >> 3, q = tid & 7;
+        const float wj = ex2f(cs[kQ - 1] - cs[j]) * dtv[j];
+        const uint4 xv = *reinterpret_cast<const uint4 *>(st + kStageX + sw_chunk(j, q));
+        const uint32_t u[4] = {xv.x, xv.y, xv.z, xv.w};
+        uint32_t o[4], ol[4];
 #pragma unroll
-            for (int q4 = 0; q4 < 4; q4++) {
-                const int q = 4 * half + q4;
-                const uint4 xv = *reinterpret_cast<const uint4 *>(st + kStageX + sw_chunk(j, q));
-                const uint32_t u[4] = {xv.x, xv.y, xv.z, xv.w};
+        for (int k = 0; k < 4; k++) {
+            const float2 f = unpack_bf16(u[k]);
+            split_bf16(f.x * wj, f.y * wj, o[k], ol[k]);
+        }
+        *reinterpret_cast<uint4 *>(wb + sw_chunk(j, q)) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4 *>(wb + kTileX + sw_chunk(j, q)) = make_uint4(ol[0], ol[1], ol[2], ol[3]);
+    };
+
+    const uint32_t idG = idesc_bf16(64, 64, 0, 0);    // C (K-major) x B (K-major)
+    const uint32_t idDS = idesc_bf16(128, 128, 1, 1); // B^T (MN-major) x [W_hi | W_lo] (MN-major)
+    const uint32_t idYo = idesc_bf16(64, 128, 0, 1);  // C (K-major) x [S_hi | S_lo] (MN-major)
+    const uint32_t idYd = idesc_bf16(64, 64, 0, 1);   // M (K-major) x X (MN-major)
+
+    // first MMA group of chunk c: G = C B^T, Yo = C [S_hi | S_lo] (buffer c & 1),
+    // dS = B^T [W_hi | W_lo]
+    auto issue_group1 = [&](int c) {
+        const uint8_t *st = sm + (c % kStages) * kStageBytes;
+        const uint32_t sC = smem_u32(st + kStageC), sB = smem_u32(st + kStageB);
+        const uint32_t sS = smem_u32(sm + kOffS);
+        const uint32_t sW = smem_u32(sm + kOffW + (c & 1) * 2 * kTileX);
+#pragma unroll
+        for (int kk = 0; kk < 8; kk++) {   // K = n, 8 steps of 16; two 64-wide atoms
+            const uint32_t off = (kk >> 2) * kTileBC + (kk & 3) * 32;
+            umma(tb + kColG, desc_sw128(sC + off, 16, 1024), desc_sw128(sB + off, 16, 1024), idG, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 8; kk++) {   // K = n; S rows n (MN-major), hi and lo blocks 16 KB apart
+            const uint32_t offc = (kk >> 2) * kTileBC + (kk & 3) * 32;
+            umma(tb + kColYo + (uint32_t)(c & 1) * 128, desc_sw128(sC + offc, 16, 1024),
+                 desc_sw128(sS + kk * 2048, kSBytes, 1024), idYo, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 4; kk++)     // K = j (rows); B^T: two MN atoms of 64 n, 8 KB apart;
+            umma(tb + kColDS, desc_sw128(sB + kk * 2048, kTileBC, 1024),      // W hi and lo 8 KB apart
+                 desc_sw128(sW + kk * 2048, kTileX, 1024), idDS, kk > 0);
+        umma_commit(&bar_mma1[c & 1]);
+    };
+
+    // S: this thread's row n (= its TMEM lane), columns [16 g, 16 g + 16), fp32
+    const int row_n = wq * 32 + lane;
+    float S[16];
+#pragma unroll
+    for (int p = 0; p < 16; p++)
+        S[p] = 0.f;
+
+    const int row_i = 16 * wq + (lane & 15);   // M = 64 accumulator row of this thread
+    const int c8 = 16 * g + 8 * (lane >> 4);   // first of this thread's 8 columns
+
+    if (warp == kDtWarp) {
+        // ---- the dt warp: for every chunk k, once the math threads are done
+        // with chunk k - kStages (its stage and dt buffer), issue chunk k's TMA
+        // loads (lane 0) and compute dt and the cumulative sum of dt A
+        float2 draw = load_delta2(0);
+        for (int k = 0; k < nch; k++) {
+            const float2 dnext = load_delta2(k + 1);
+            if (k >= kStages)
+                mbar_wait(&bar_free[k % kStages], ((k / kStages) - 1) & 1);
+            if (lane == 0)
+                issue_tma(k);
+            __syncwarp();
+            chunk_dt(k, draw);
+            mbar_arrive(&bar_dt_full[k % kDtBufs]);
+            draw = dnext;
+        }
+    } else if (warp == kMmaWarp) {
+        // ---- the MMA warp: wait until the math threads have written the
+        // operands, then issue; lane 0 issues, the warp stays converged
+        bool ok = mbar_wait(&bar_sready, 0);   // W(0) written
+        if (lane == 0) {
+            tc_fence_after();
+            issue_group1(0);
+        }
+        __syncwarp();
+        for (int c = 0; c < nch && ok; c++) {
+            ok = mbar_wait(&bar_mready, c & 1);   // M(c) written
+            if (lane == 0) {
+                tc_fence_after();
+                const uint8_t *st = sm + (c % kStages) * kStageBytes;
+                const uint32_t sM = smem_u32(sm + kOffM), sX = smem_u32(st + kStageX);
+#pragma unroll
+                for (int part = 0; part < 2; part++)   // M hi, then lo
+#pragma unroll
+                    for (int kk = 0; kk < 4; kk++)
+                        umma(tb + kColYd, desc_sw128(sM + part * kTileX + kk * 32, 16, 1024),
+                             desc_sw128(sX + kk * 2048, 8192, 1024), idYd, part + kk > 0);
+                umma_commit(&bar_mma2);
+            }
+            __syncwarp();
+            ok = ok && mbar_wait(&bar_sready, (c + 1) & 1);   // S_in(c + 1), W(c + 1) written
+            if (lane == 0 && c + 1 < nch) {
+                tc_fence_after();
+                issue_group1(c + 1);
+            }
+            __syncwarp();
+        }
+    } else {
+        // ---- math threads.  Prologue: W(0)
+        mbar_wait(&bar_dt_full[0], 0);
+        mbar_wait(&bar_tma[0], 0);
+        build_w(0);
+        fence_async_smem();
+        tc_fence_before();
+        mbar_arrive(&bar_sready);
+
+        for (int c = 0; c < nch; c++) {
+            const uint8_t *st = sm + (c % kStages) * kStageBytes;
+            const float *cs = cs_s + (c % kDtBufs) * 64, *dtv = dt_s + (c % kDtBufs) * 64;
+            const int t0 = c * kQ;
+            // ---- 1. next chunk's W
+            if (c + 1 < nch) {
+                mbar_wait(&bar_dt_full[(c + 1) % kDtBufs], ((c + 1) / kDtBufs) & 1);
+                mbar_wait(&bar_tma[(c + 1) % kStages], ((c + 1) / kStages) & 1);
+                build_w(c + 1);
+            }
+            // ---- 2. this chunk's first MMA group is done
+            mbar_wait(&bar_mma1[c & 1], (c >> 1) & 1);
+            tc_fence_after();
+            const uint32_t buf = (uint32_t)(c & 1) * 64;
+            // ---- 3. masked decay matrix M (bf16 hi + lo, K-major rows i) from G; hand it over
+            {
+                float gv[8];
+                tmem_ld_eighth_row(tw + kColG + 16 * g, gv);
+                const float csi = cs[row_i];
                 uint32_t o[4], ol[4];
 #pragma unroll
-                for (int k = 0; k < 4; k++) {
-                    const float2 f = unpack_bf16(u[k]);
-                    split_bf16(f.x * wj, f.y * wj, o[k], ol[k]);
+                for (int k = 0; k < 8; k += 2) {
+                    const int j0 = c8 + k;
+                    const float m0 = (j0 <= row_i) ? gv[k] * ex2f(csi - cs[j0]) * dtv[j0] : 0.f;
+                    const float m1 = (j0 + 1 <= row_i) ? gv[k + 1] * ex2f(csi - cs[j0 + 1]) * dtv[j0 + 1] : 0.f;
+                    split_bf16(m0, m1, o[k >> 1], ol[k >> 1]);
                 }
-                *reinterpret_cast<uint4 *>(sm + kOffW + sw_chunk(j, q)) = make_uint4(o[0], o[1], o[2], o[3]);
-                *reinterpret_cast<uint4 *>(sm + kOffW + kTileX + sw_chunk(j, q)) = make_uint4(ol[0], ol[1], ol[2], ol[3]);
+                const int q = c8 >> 3;
+                *reinterpret_cast<uint4 *>(sm + kOffM + sw_chunk(row_i, q)) = make_uint4(o[0], o[1], o[2], o[3]);
+                *reinterpret_cast<uint4 *>(sm + kOffM + kTileX + sw_chunk(row_i, q)) =
+                    make_uint4(ol[0], ol[1], ol[2], ol[3]);
             }
-        }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-
-        // ---- first MMA group: G = C B^T, Yo = C S_in, dS = B^T W
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t sC = smem_u32(st + kStageC), sB = smem_u32(st + kStageB);
-            const uint32_t sS = smem_u32(sm + kOffS + (c & 1) * 2 * kSBytes), sW = smem_u32(sm + kOffW);
+            fence_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bar_mready);
+            // ---- 4. state update S = exp(cs_end) S + dS; bf16 hi + lo copy for the next chunk
+            {
+                const float decay = ex2f(cs[kQ - 1]);
+                float ds[16], dl[16];
+                tmem_ld_row16(tw + kColDS + 16 * g, ds);
+                tmem_ld_row16(tw + kColDS + 64 + 16 * g, dl);
 #pragma unroll
-            for (int kk = 0; kk < 8; kk++) {   // K = n, 8 steps of 16; two 64-wide atoms
-                const uint32_t off = (kk >> 2) * kTileBC + (kk & 3) * 32;
-                umma(tb + kColG, desc_sw128(sC + off, 16, 1024), desc_sw128(sB + off, 16, 1024), idG, kk > 0);
-            }
+                for (int k = 0; k < 16; k++)
+                    S[k] = fmaf(decay, S[k], ds[k] + dl[k]);
+                if (c + 1 < nch) {
+                    // single buffer: this chunk's C S_in finished before step 2
+                    uint8_t *sn = sm + kOffS;
 #pragma unroll
-            for (int part = 0; part < 2; part++)   // S_in hi, then lo
+                    for (int q2 = 0; q2 < 2; q2++) {
+                        uint32_t hi[4], lo[4];
 #pragma unroll
-                for (int kk = 0; kk < 8; kk++) {   // K = n; S_in rows n (MN-major, 8 rows per 1 KB)
-                    const uint32_t offc = (kk >> 2) * kTileBC + (kk & 3) * 32;
-                    umma(tb + kColYo, desc_sw128(sC + offc, 16, 1024),
-                         desc_sw128(sS + part * kSBytes + kk * 2048, 8192, 1024), idYo, part + kk > 0);
-                }
-#pragma unroll
-            for (int part = 0; part < 2; part++)   // W hi, then lo
-#pragma unroll
-                for (int kk = 0; kk < 4; kk++)     // K = j (rows); B^T: two MN atoms of 64 n, 8 KB apart
-                    umma(tb + kColDS, desc_sw128(sB + kk * 2048, kTileBC, 1024),
-                         desc_sw128(sW + part * kTileX + kk * 2048, 8192, 1024), idDS, part + kk > 0);
-            umma_commit(&bar_mma1);
-        }
-        __syncwarp();
-        mbar_wait(&bar_mma1, c & 1);
-        tc_fence_after();
-
-        // ---- masked decay matrix M (bf16, K-major rows i) from G
-        {
-            float g[32];
-            tmem_ld_half_row(tw + kColG, g);
-            const float csi = cs_s[row_i];
-            uint32_t o[16], ol[16];
-#pragma unroll
-            for (int k = 0; k < 32; k += 2) {
-                const int j0 = 32 * hh + k;
-                const float m0 = (j0 <= row_i) ? g[k] * ex2f(csi - cs_s[j0]) * dt_s[j0] : 0.f;
-                const float m1 = (j0 + 1 <= row_i) ? g[k + 1] * ex2f(csi - cs_s[j0 + 1]) * dt_s[j0 + 1] : 0.f;
-                split_bf16(m0, m1, o[k >> 1], ol[k >> 1]);
-            }
-#pragma unroll
-            for (int q4 = 0; q4 < 4; q4++) {
-                *reinterpret_cast<uint4 *>(sm + kOffM + sw_chunk(row_i, 4 * hh + q4)) =
-                    make_uint4(o[4 * q4], o[4 * q4 + 1], o[4 * q4 + 2], o[4 * q4 + 3]);
-                *reinterpret_cast<uint4 *>(sm + kOffM + kTileX + sw_chunk(row_i, 4 * hh + q4)) =
-                    make_uint4(ol[4 * q4], ol[4 * q4 + 1], ol[4 * q4 + 2], ol[4 * q4 + 3]);
-            }
-        }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t sM = smem_u32(sm + kOffM), sX = smem_u32(st + kStageX);
-#pragma unroll
-            for (int part = 0; part < 2; part++)   // M hi, then lo
-#pragma unroll
-                for (int kk = 0; kk < 4; kk++)
-                    umma(tb + kColYd, desc_sw128(sM + part * kTileX + kk * 32, 16, 1024),
-                         desc_sw128(sX + kk * 2048, 8192, 1024), idYd, part + kk > 0);
-            umma_commit(&bar_mma2);
-        }
-        __syncwarp();
-
-        // ---- state update S = exp(cs_end) S + dS, row n = tid; bf16 copy for the next chunk
-        {
-            const float decay = ex2f(cs_end);
-            float ds[32];
-#pragma unroll
-            for (int half = 0; half < 2; half++) {
-                tmem_ld_row32(tw + kColDS + 32 * half, ds);
-#pragma unroll
-                for (int k = 0; k < 32; k++)
-                    S[32 * half + k] = fmaf(decay, S[32 * half + k], ds[k]);
-            }
-            if (c + 1 < args.nchunks) {
-                uint8_t *sn = sm + kOffS + ((c + 1) & 1) * 2 * kSBytes;
-#pragma unroll
-                for (int q = 0; q < 8; q++) {
-                    uint32_t hi[4], lo[4];
-#pragma unroll
-                    for (int k = 0; k < 4; k++)
-                        split_bf16(S[8 * q + 2 * k], S[8 * q + 2 * k + 1], hi[k], lo[k]);
-                    *reinterpret_cast<uint4 *>(sn + sw_chunk(tid, q)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                    *reinterpret_cast<uint4 *>(sn + kSBytes + sw_chunk(tid, q)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                        for (int k = 0; k < 4; k++)
+                            split_bf16(S[8 * q2 + 2 * k], S[8 * q2 + 2 * k + 1], hi[k], lo[k]);
+                        const int q = 2 * g + q2;
+                        *reinterpret_cast<uint4 *>(sn + sw_chunk(row_n, q)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                        *reinterpret_cast<uint4 *>(sn + kSBytes + sw_chunk(row_n, q)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                    }
                 }
             }
-        }
-
-        // ---- outputs: y = (Yd + exp(cs_i) Yo + D x) silu(z), row i, 32 columns
-        {
-            float yo[32], yd[32];
-            tmem_ld_half_row(tw + kColYo, yo);
-            mbar_wait(&bar_mma2, c & 1);
-            tc_fence_after();
-            tmem_ld_half_row(tw + kColYd, yd);
-            const float ei = ex2f(cs_s[row_i]);
-            const int t = t0 + row_i;
-            uint32_t o[16];
+            // ---- 5. hand S_in(c + 1), W(c + 1) to the MMA warp
+            fence_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bar_sready);
+            // ---- 6. outputs: y = (Yd + exp(cs_i) Yo + D x) silu(z), row i, 8 columns
+            {
+                float yo[8], yl[8], yd[8];
+                tmem_ld_eighth_row(tw + kColYo + 2 * buf + 16 * g, yo);
+                tmem_ld_eighth_row(tw + kColYo + 2 * buf + 64 + 16 * g, yl);
 #pragma unroll
-            for (int q4 = 0; q4 < 4; q4++) {
-                const int q = 4 * hh + q4;
+                for (int k = 0; k < 8; k++)
+                    yo[k] += yl[k];
+                mbar_wait(&bar_mma2, c & 1);
+                tc_fence_after();
+                tmem_ld_eighth_row(tw + kColYd + 16 * g, yd);
+                const float ei = ex2f(cs[row_i]);
+                const int t = t0 + row_i;
+                const int q = c8 >> 3;
                 const uint4 xv = *reinterpret_cast<const uint4 *>(st + kStageX + sw_chunk(row_i, q));
                 uint4 zv = make_uint4(0, 0, 0, 0);
                 if (args.has_z)
                     zv = *reinterpret_cast<const uint4 *>(st + kStageZ + sw_chunk(row_i, q));
                 const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w};
                 const uint32_t zu[4] = {zv.x, zv.y, zv.z, zv.w};
+                uint32_t o[4];
 #pragma unroll
                 for (int k = 0; k < 4; k++) {
-                    const int col = 8 * q4 + 2 * k;   // column within this half
                     const float2 xf = unpack_bf16(xu[k]);
-                    float y0 = fmaf(ei, yo[col], yd[col]) + Dh * xf.x;
-                    float y1 = fmaf(ei, yo[col + 1], yd[col + 1]) + Dh * xf.y;
+                    float y0 = fmaf(ei, yo[2 * k], yd[2 * k]) + Dh * xf.x;
+                    float y1 = fmaf(ei, yo[2 * k + 1], yd[2 * k + 1]) + Dh * xf.y;
                     if (args.has_z) {
                         const float2 zf = unpack_bf16(zu[k]);
                         y0 *= silu_f(zf.x);
                         y1 *= silu_f(zf.y);
                     }
-                    o[4 * q4 + k] = pack_bf16(y0, y1);
+                    o[k] = pack_bf16(y0, y1);
                 }
+                if (t < L)
+                    *reinterpret_cast<uint4 *>(args.out + (((size_t)b * L + t) * args.H + h) * kP + c8) =
+                        make_uint4(o[0], o[1], o[2], o[3]);
             }
-            if (t < L) {
-                uint4 *dst = reinterpret_cast<uint4 *>(args.out + (((size_t)b * L + t) * args.H + h) * kP + 32 * hh);
-#pragma unroll
-                for (int q4 = 0; q4 < 4; q4++)
-                    dst[q4] = make_uint4(o[4 * q4], o[4 * q4 + 1], o[4 * q4 + 2], o[4 * q4 + 3]);
-            }
+            // ---- 7. hand chunk c's stage and dt buffer back to the dt warp
+            fence_async_smem();
+            mbar_arrive(&bar_free[c % kStages]);
         }
-        // ---- release this stage; prefetch chunk c + 2 into it
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0 && c + 2 < args.nchunks)
-            issue_tma(c + 2);
     }
 
-    if (args.last_state) {
+    if (args.last_state && tid < kMath) {
         float *ls = args.last_state + (size_t)bh * kP * kN;
 #pragma unroll
-        for (int p = 0; p < kP; p++)
-            ls[(size_t)p * kN + tid] = S[p];
+        for (int k = 0; k < 16; k++)
+            ls[(size_t)(16 * g + k) * kN + row_n] = S[k];
     }
     tc_fence_before();
     __syncthreads();
