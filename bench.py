@@ -45,6 +45,10 @@ METRIC = "scan elements/s (B·L·D·N) and HBM GB/s as % of B200 peak, per confi
 HBM_FALLBACK_GBS = 6650.0
 L2_FLUSH_BYTES = 512 << 20
 SMS = 148
+# DRAM bytes (read + write) per launch of the dominant kernel, from one ncu
+# capture of the current kernels (profiles/s6_main_vim_small_bidir_fp32.md,
+# profiles/ssd_chunk_mamba2_bf16.md); None where no capture matches them.
+NCU_TRAFFIC = {1: 273.28e6, 4: 397.21e6}
 
 
 def parse():
@@ -326,13 +330,14 @@ def run_ours(args, rank, world, local_rank):
     t_alu = info["elems"] / alu_peak
     if info["kind"] == "s6" and t_alu > t_hbm:
         roof = {"bound": "alu", "achieved": alu_ach / 1e9, "peak": alu_peak / 1e9,
-                "unit": "Gelem/s", "frac": alu_ach / alu_peak, "traffic": None,
+                "unit": "Gelem/s", "frac": alu_ach / alu_peak, "traffic": NCU_TRAFFIC.get(args.config),
                 "hbm_achieved_gbs": hbm_ach, "hbm_peak_gbs": peaks["hbm_gbs"],
                 "hbm_frac": hbm_ach / peaks["hbm_gbs"], "peak_source": peak_src,
                 "algorithmic_bytes": info["bytes"], "kernel_ms_median": kern_s * 1e3}
     else:
         roof = {"bound": "hbm", "achieved": hbm_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": hbm_ach / peaks["hbm_gbs"], "traffic": None, "peak_source": peak_src,
+                "frac": hbm_ach / peaks["hbm_gbs"], "traffic": NCU_TRAFFIC.get(args.config),
+                "peak_source": peak_src,
                 "algorithmic_bytes": info["bytes"], "kernel_ms_median": kern_s * 1e3}
 
     e2e = None
