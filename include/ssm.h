@@ -166,6 +166,22 @@ SSM_API ssm_status bidir_scan_fwd(const ssm_dims *dims, const void *x, const voi
                           const ssm_dir_params *bwd, void *out, void *workspace,
                           size_t workspace_bytes, void *stream);
 
+/*
+ * How ssm_scan_fwd (bidirectional = 0) or bidir_scan_fwd (bidirectional = 1)
+ * runs a problem of these sizes.  The pages have no counterpart: this is a
+ * query of the library's own launch plan, for callers sizing work and for
+ * tests.
+ *   segments           (out, may be NULL) the number of pieces the sequence
+ *                      is cut into for parallelism (1: one pass; more: the
+ *                      chunked scan with state hand-off of the Mamba2 page,
+ *                      sec. 3.2, run as summary, carry and main passes)
+ *   channels_per_lane  (out, may be NULL) 1 or 2: channels one GPU thread owns
+ * Host-only, makes no CUDA call.  Returns the status the scan entry points
+ * give for invalid dims; an empty problem reports 1 segment.
+ */
+SSM_API ssm_status ssm_scan_plan(const ssm_dims *dims, int bidirectional, int *segments,
+                                 int *channels_per_lane);
+
 /* SSD problem size.  Supported: dtype SSM_BF16, headdim 64, dstate 128,
  * chunk 64, seqlen any value >= 0 (a short last chunk is handled). */
 typedef struct {

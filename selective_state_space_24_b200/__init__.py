@@ -73,6 +73,8 @@ SIGNATURES = {
     "ssd_chunk_workspace_size": (_sz, [ctypes.POINTER(ssd_dims)]),
     "ssd_chunk_fwd": (_int, [ctypes.POINTER(ssd_dims), _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp,
                              _vp, _vp, _vp, _vp, _sz, _vp]),
+    "ssm_scan_plan": (_int, [ctypes.POINTER(ssm_dims), _int, ctypes.POINTER(_int),
+                             ctypes.POINTER(_int)]),
     "ssm_check_device": (_int, [_vp]),
     "ssm_status_string": (ctypes.c_char_p, [_int]),
     "ssm_version": (_int, []),
@@ -243,6 +245,16 @@ def ssd_chunk_fwd(x, delta, A, B, C, *, chunk=64, delta_bias=None, delta_softplu
                            _stream_handle(stream))
     _check(st, "ssd_chunk_fwd")
     return out
+
+
+def scan_plan(batch, seqlen, dim, dstate, dtype=SSM_F32, bidirectional=False):
+    """(segments, channels_per_lane) the library uses for an S6 problem."""
+    lib = capi()
+    dims = ssm_dims(batch, seqlen, dim, dstate, dtype)
+    seg, cpl = _int(0), _int(0)
+    _check(lib.ssm_scan_plan(ctypes.byref(dims), int(bool(bidirectional)), ctypes.byref(seg),
+                             ctypes.byref(cpl)), "ssm_scan_plan")
+    return seg.value, cpl.value
 
 
 def check_device(stream=None):

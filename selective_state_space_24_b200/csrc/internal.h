@@ -29,6 +29,7 @@ struct DirArgs {
 struct S6Args {
     int Bsz, L, D, N;
     int S, T;
+    int cpl;       // channels per lane: 1 or 2
     int dtype;     // 0 = float32, 1 = bf16
     int softplus;
     int ndir;      // 1 or 2
@@ -46,11 +47,13 @@ struct S6Args {
 
 struct S6Plan {
     int S, T;
+    int cpl;   // channels per lane
     size_t workspace_bytes;
     size_t carry_h_off, carry_s_off, stash_off;  // byte offsets into the workspace
 };
 
-// Segment plan for a problem; depends on the sizes and dtype only.
+// Segment plan and lane mapping for a problem; depends on the sizes and
+// dtype only.
 S6Plan plan_s6(int64_t Bsz, int64_t L, int64_t D, int64_t N, int ndir, int dtype);
 
 cudaError_t launch_s6(const S6Args &a, cudaStream_t stream);

@@ -109,6 +109,7 @@ extern "C" SSM_API ssm_status ssm_scan_fwd_noalloc(const ssm_dims *dims, const v
     a.N = (int)dims->dstate;
     a.S = plan.S;
     a.T = plan.T;
+    a.cpl = plan.cpl;
     a.dtype = dt;
     a.softplus = delta_softplus ? 1 : 0;
     a.ndir = 1;

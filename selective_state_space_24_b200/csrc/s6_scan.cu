@@ -10,18 +10,21 @@
 // parameter set, the two results summed.
 //
 // Work decomposition
-//   * One thread owns two adjacent channels of one (b, direction) and keeps
-//     their 2 x N states in fp32 registers; the h sequence never leaves the
-//     SM (the pages' fusion rule: never materialise (B, L, D, N)).  The state
-//     update runs on packed f32x2 FMA/MUL instructions (two states per
-//     instruction).
-//   * A warp owns 64 consecutive channels, so every x / delta / z access of a
-//     warp is one contiguous row segment.  Those rows arrive by cp.async in a
-//     per-warp shared-memory ring 4 to 8 steps ahead of use.  B[t] and C[t]
+//   * One thread owns one or two adjacent channels (CPL) of one (b,
+//     direction) and keeps their CPL x N states in fp32 registers; the h
+//     sequence never leaves the SM (the pages' fusion rule: never
+//     materialise (B, L, D, N)).  The state update runs on packed f32x2
+//     FMA/MUL instructions (two states per instruction).  Two channels per
+//     lane give each thread more independent work; one channel per lane
+//     gives twice the threads when the problem is small.
+//   * A warp owns 32 CPL consecutive channels, so every x / delta / z access
+//     of a warp is one contiguous row segment.  Those rows arrive by 16-byte
+//     cp.async copies in a per-warp shared-memory ring 4 to 8 steps ahead of
+//     use.  B[t] and C[t]
 //     are the same for every lane: each warp stages them 16 steps at a time
 //     in shared memory as fp32 (zero-padded to the template state count) and
 //     reads them back as broadcast 16-byte loads.
-//   * Bidirectional: a CTA is a warp pair over the same 64 channels, the
+//   * Bidirectional: a CTA is a warp pair over the same channels, the
 //     forward warp walking its segment upward, the reversed warp downward.
 //     Each parks the first half of its outputs in an fp32 stash (the output
 //     itself for fp32, the workspace for bf16), the pair meets at one named
@@ -48,7 +51,6 @@ namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kWarps = 2;   // warps per CTA
-constexpr int kCh = 64;     // channels per warp (2 per lane)
 constexpr int kTC = 16;     // steps per B/C staging chunk
 constexpr int kSub = 4;     // steps per cp.async group
 constexpr int kStages = 2;  // cp.async groups in the ring
@@ -56,7 +58,32 @@ constexpr int kSlots = kSub * kStages;
 #ifndef SSM_S6_MINB
 #define SSM_S6_MINB 6
 #endif
-constexpr int kMinBlocks = SSM_S6_MINB;   // CTAs per SM the register budget is sized for
+#ifndef SSM_S6_MINB1
+#define SSM_S6_MINB1 8
+#endif
+// Tuning knobs (compile-time): channels per lane (0 = by problem size), the
+// thread count below which one channel per lane is used, the target thread
+// counts that decide the number of segments, and how many state pairs the
+// summary pass evaluates on the FMA pipe.
+#ifndef SSM_S6_CPL
+#define SSM_S6_CPL 0
+#endif
+#ifndef SSM_S6_CPL1_BELOW
+#define SSM_S6_CPL1_BELOW (148 * 128)
+#endif
+#ifndef SSM_S6_TARGET1
+#define SSM_S6_TARGET1 (148 * 640)
+#endif
+#ifndef SSM_S6_TARGET2
+#define SSM_S6_TARGET2 (148 * 320)
+#endif
+#ifndef SSM_S6_SUM_NPOLY_N
+#define SSM_S6_SUM_NPOLY_N 0
+#endif
+#define SSM_S6_SUM_NPOLY(NS) ((NS) == 16 ? SSM_S6_SUM_NPOLY_N : 0)
+
+// CTAs per SM the register budget is sized for, by channels per lane
+template <int CPL> constexpr int min_blocks() { return CPL == 2 ? SSM_S6_MINB : SSM_S6_MINB1; }
 
 // ------------------------------------------------------------ math helpers
 
@@ -129,39 +156,68 @@ __device__ __forceinline__ float silu_f(float z)
 
 // ----------------------------------------------------- storage-type helpers
 
-template <typename T> struct IO;
-template <> struct IO<float> {
-    // two adjacent channels
-    static __device__ __forceinline__ float2 ld2(const void *p) { return *reinterpret_cast<const float2 *>(p); }
-    static __device__ __forceinline__ void st2(float *p, float2 v) { *reinterpret_cast<float2 *>(p) = v; }
-    static __device__ __forceinline__ float ld1(const float *p, size_t i) { return __ldg(p + i); }
+// CPL adjacent channels of one lane: loads from the staging ring (shared
+// memory) and stores to the output.
+template <typename T, int CPL> struct IO;
+template <> struct IO<float, 2> {
+    static __device__ __forceinline__ void ld(const void *p, float (&v)[2])
+    {
+        const float2 u = *reinterpret_cast<const float2 *>(p);
+        v[0] = u.x;
+        v[1] = u.y;
+    }
+    static __device__ __forceinline__ void st(float *p, const float (&v)[2])
+    {
+        *reinterpret_cast<float2 *>(p) = make_float2(v[0], v[1]);
+    }
 };
-template <> struct IO<__nv_bfloat16> {
-    static __device__ __forceinline__ float2 ld2(const void *p)
+template <> struct IO<float, 1> {
+    static __device__ __forceinline__ void ld(const void *p, float (&v)[1])
+    {
+        v[0] = *reinterpret_cast<const float *>(p);
+    }
+    static __device__ __forceinline__ void st(float *p, const float (&v)[1]) { *p = v[0]; }
+};
+template <> struct IO<__nv_bfloat16, 2> {
+    static __device__ __forceinline__ void ld(const void *p, float (&v)[2])
     {
         const uint32_t u = *reinterpret_cast<const uint32_t *>(p);
-        return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+        v[0] = __uint_as_float(u << 16);
+        v[1] = __uint_as_float(u & 0xffff0000u);
     }
-    static __device__ __forceinline__ void st2(__nv_bfloat16 *p, float2 v)
+    static __device__ __forceinline__ void st(__nv_bfloat16 *p, const float (&v)[2])
     {
-        *reinterpret_cast<__nv_bfloat162 *>(p) = __floats2bfloat162_rn(v.x, v.y);
-    }
-    static __device__ __forceinline__ float ld1(const __nv_bfloat16 *p, size_t i)
-    {
-        return __bfloat162float(__ldg(p + i));
+        *reinterpret_cast<__nv_bfloat162 *>(p) = __floats2bfloat162_rn(v[0], v[1]);
     }
 };
+template <> struct IO<__nv_bfloat16, 1> {
+    static __device__ __forceinline__ void ld(const void *p, float (&v)[1])
+    {
+        v[0] = __uint_as_float((uint32_t)*reinterpret_cast<const unsigned short *>(p) << 16);
+    }
+    static __device__ __forceinline__ void st(__nv_bfloat16 *p, const float (&v)[1])
+    {
+        *p = __float2bfloat16_rn(v[0]);
+    }
+};
+
+template <typename T>
+__device__ __forceinline__ float ld1(const T *p, size_t i);
+template <> __device__ __forceinline__ float ld1<float>(const float *p, size_t i) { return __ldg(p + i); }
+template <> __device__ __forceinline__ float ld1<__nv_bfloat16>(const __nv_bfloat16 *p, size_t i)
+{
+    return __bfloat162float(__ldg(p + i));
+}
 
 __device__ __forceinline__ bool first_in_order(int seg, int S, bool rev) { return rev ? seg == S - 1 : seg == 0; }
 __device__ __forceinline__ bool last_in_order(int seg, int S, bool rev) { return rev ? seg == 0 : seg == S - 1; }
 
 __device__ __forceinline__ void pair_barrier() { asm volatile("bar.sync 1, 64;" ::: "memory"); }
 
-template <int BYTES>
-__device__ __forceinline__ void cp_async(void *smem, const void *gmem)
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem)
 {
     const unsigned sa = (unsigned)__cvta_generic_to_shared(smem);
-    asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"(sa), "l"(gmem), "n"(BYTES) : "memory");
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int K> __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(K) : "memory"); }
@@ -210,7 +266,7 @@ struct BCStage {
 #pragma unroll
                 for (int n = 0; n < NS; n++)
                     if (n < N)
-                        v[n] = IO<T>::ld1(row, n);
+                        v[n] = ld1<T>(row, n);
             }
         }
     }
@@ -229,8 +285,10 @@ template <bool V> struct PhaseTag {
 };
 
 // Shared memory of one warp: the x / delta / z / stash ring and the B/C rows.
-template <typename T, int NS>
+// A warp owns 32 * CPL consecutive channels; one ring slot holds one step.
+template <typename T, int NS, int CPL>
 struct WarpSmem {
+    static constexpr int kCh = 32 * CPL;                  // channels per warp
     static constexpr int kRowB = kCh * (int)sizeof(T);   // one x, delta or z row
     static constexpr int kStashB = kCh * 4;              // one fp32 stash row
     static constexpr int kSlotB = 3 * kRowB + kStashB;
@@ -238,19 +296,33 @@ struct WarpSmem {
     float bc[2 * kTC * 2 * NS];
 };
 
-// One warp's scan over one segment, two channels per lane.
+// Copies of whole rows into the ring, 16 bytes per lane: ROWB / 16 lanes
+// cover one step's row, so one pass of the warp moves 512 / ROWB steps.
+// Every 16-byte piece lies entirely inside or entirely past the channel
+// range (D is a multiple of 16 / sizeof(element), the warp's first channel
+// a multiple of 32).
+template <int ROWB>
+struct RowCopy {
+    static constexpr int kLanesPerRow = ROWB / 16;
+    static constexpr int kRowsPerPass = 32 / kLanesPerRow;
+    static_assert(ROWB % 16 == 0 && kLanesPerRow <= 32, "row must be whole 16-byte pieces");
+};
+
+// One warp's scan over one segment, CPL adjacent channels per lane.
 //   SUMMARY: local end state from the given h, plus the sum of dt; no output.
 //   otherwise: outputs; BIDIR adds the midpoint exchange with the partner warp.
-template <typename T, int NS, int NPOLY, bool SUMMARY, bool BIDIR, bool GATE, bool SOFTPLUS>
+template <typename T, int NS, int CPL, int NPOLY, bool SUMMARY, bool BIDIR, bool GATE, bool SOFTPLUS>
 __device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P,
-                                             WarpSmem<T, NS> &sm, int b, int dbase, bool active,
-                                             int s0, int s1, bool rev, float2 (&h)[2][NS / 2],
-                                             float2 &sdt)
+                                             WarpSmem<T, NS, CPL> &sm, int b, int dbase, bool active,
+                                             int s0, int s1, bool rev, float2 (&h)[CPL][NS / 2],
+                                             float (&sdt)[CPL])
 {
-    using WS = WarpSmem<T, NS>;
+    using WS = WarpSmem<T, NS, CPL>;
+    using RC = RowCopy<WS::kRowB>;
+    using RS = RowCopy<WS::kStashB>;
     static_assert(NPOLY % 2 == 0 && NPOLY <= NS, "NPOLY counts state pairs");
     const int lane = threadIdx.x & 31;
-    const int d = dbase + 2 * lane;
+    const int d = dbase + CPL * lane;
     const int N = a.N;
     const int Tn = s1 - s0;
     const size_t rowbase = (size_t)b * a.L;
@@ -260,46 +332,56 @@ __device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P,
     T *out = static_cast<T *>(a.out);
     float *stash = a.stash;
 
-    // A log2(e) for both channels, as pairs of states
-    float2 Ap[2][NS / 2];
+    // A log2(e) per channel, as pairs of states
+    float2 Ap[CPL][NS / 2];
+    float bias[CPL], Dd[CPL];
 #pragma unroll
-    for (int c = 0; c < 2; c++)
+    for (int c = 0; c < CPL; c++) {
+        const float *Ar = P.A + (size_t)(d + c) * N;
 #pragma unroll
         for (int k = 0; k < NS / 2; k++) {
             const int n = 2 * k;
-            const float *Ar = P.A + (size_t)(d + c) * N;
             Ap[c][k] = make_float2((active && n < N) ? Ar[n] * kLog2e : 0.f,
                                    (active && n + 1 < N) ? Ar[n + 1] * kLog2e : 0.f);
         }
-    const float2 bias = (active && P.bias) ? make_float2(P.bias[d], P.bias[d + 1]) : make_float2(0.f, 0.f);
-    const float2 Dd = (active && P.D) ? make_float2(P.D[d], P.D[d + 1]) : make_float2(0.f, 0.f);
+        bias[c] = (active && P.bias) ? P.bias[d + c] : 0.f;
+        Dd[c] = (active && P.D) ? P.D[d + c] : 0.f;
+    }
 
     // midpoint of the pair exchange (see file comment)
     const int M = BIDIR ? (rev ? Tn / 2 : (Tn + 1) / 2) : Tn;
     auto tpos = [&](int i) { return rev ? s1 - 1 - i : s0 + i; };
     auto slot_of = [&](int i) { return sm.ring + (i % kSlots) * WS::kSlotB; };
 
-    // copy x / delta / z (and the stash row when allowed) of step i
-    auto issue_step = [&](int i, bool with_stash) {
-        char *slot = slot_of(i);
-        const size_t ro = (rowbase + tpos(i)) * a.D + d;
-        if (active) {
-            constexpr int E = 2 * (int)sizeof(T);
-            cp_async<E>(slot + lane * E, x + ro);
-            cp_async<E>(slot + WS::kRowB + lane * E, dl + ro);
-            if (!SUMMARY && GATE)
-                cp_async<E>(slot + 2 * WS::kRowB + lane * E, zp + ro);
-            if (BIDIR && with_stash)
-                cp_async<8>(slot + 3 * WS::kRowB + lane * 8, stash + ro);
-        }
+    // this lane's 16-byte piece of a row and of a stash row
+    const int pc = lane % RC::kLanesPerRow, pr = lane / RC::kLanesPerRow;
+    const int spc = lane % RS::kLanesPerRow, spr = lane / RS::kLanesPerRow;
+    const bool pc_on = dbase + pc * (16 / (int)sizeof(T)) < a.D;
+    const bool spc_on = dbase + spc * 4 < a.D;
+    // stash rows of steps [i0, i1)
+    auto issue_stash = [&](int i0, int i1) {
+        for (int i = i0 + spr; i < i1; i += RS::kRowsPerPass)
+            if (spc_on)
+                cp_async16(slot_of(i) + 3 * WS::kRowB + spc * 16,
+                           stash + (rowbase + tpos(i)) * a.D + dbase + spc * 4);
     };
+    // x / delta / z (and stash when allowed) rows of group c
     auto issue_chunk = [&](int c, bool with_stash) {
+        const int i0 = c * kSub, i1 = min(Tn, i0 + kSub);
 #pragma unroll
-        for (int j = 0; j < kSub; j++) {
-            const int i = c * kSub + j;
-            if (i < Tn)
-                issue_step(i, with_stash);
+        for (int p = 0; p < (kSub + RC::kRowsPerPass - 1) / RC::kRowsPerPass; p++) {
+            const int i = i0 + p * RC::kRowsPerPass + pr;
+            if (i < i1 && pc_on) {
+                char *slot = slot_of(i) + pc * 16;
+                const size_t ro = (rowbase + tpos(i)) * a.D + dbase + pc * (16 / (int)sizeof(T));
+                cp_async16(slot, x + ro);
+                cp_async16(slot + WS::kRowB, dl + ro);
+                if (!SUMMARY && GATE)
+                    cp_async16(slot + 2 * WS::kRowB, zp + ro);
+            }
         }
+        if (BIDIR && with_stash)
+            issue_stash(i0, i1);
         cp_async_commit();
     };
 
@@ -331,32 +413,45 @@ __device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P,
     // recur: the state update and readout (the only part that depends on the
     // previous step); finish: skip term, gate, store.
     struct StepIn {
-        float2 xv, zv, dt;
+        float xv[CPL], zv[CPL], dt[CPL];
     };
     auto load_dt = [&](int i) {
-        const char *slot = slot_of(i);
+        const char *slot = slot_of(i) + lane * CPL * (int)sizeof(T);
         StepIn o;
-        o.xv = IO<T>::ld2(slot + lane * 2 * sizeof(T));
-        const float2 dv = IO<T>::ld2(slot + WS::kRowB + lane * 2 * sizeof(T));
-        o.zv = make_float2(0.f, 0.f);
+        float dv[CPL];
+        IO<T, CPL>::ld(slot, o.xv);
+        IO<T, CPL>::ld(slot + WS::kRowB, dv);
         if (!SUMMARY && GATE)
-            o.zv = IO<T>::ld2(slot + 2 * WS::kRowB + lane * 2 * sizeof(T));
-        o.dt = make_float2(dv.x + bias.x, dv.y + bias.y);
-        if (SOFTPLUS)
-            o.dt = make_float2(softplus_f(o.dt.x), softplus_f(o.dt.y));
-        if (!SUMMARY && GATE)
-            o.zv = make_float2(silu_f<T>(o.zv.x), silu_f<T>(o.zv.y));   // zv now holds the gate
+            IO<T, CPL>::ld(slot + 2 * WS::kRowB, o.zv);
+#pragma unroll
+        for (int c = 0; c < CPL; c++) {
+            o.dt[c] = dv[c] + bias[c];
+            if (SOFTPLUS)
+                o.dt[c] = softplus_f(o.dt[c]);
+            o.zv[c] = (!SUMMARY && GATE) ? silu_f<T>(o.zv[c]) : 0.f;   // zv now holds the gate
+        }
         return o;
     };
+    struct StepOut {
+        float y[CPL];
+    };
     auto recur = [&](int i, const StepIn &in) {
-        const float2 dtc[2] = {make_float2(in.dt.x, in.dt.x), make_float2(in.dt.y, in.dt.y)};
-        const float2 dtx[2] = {make_float2(in.dt.x * in.xv.x, in.dt.x * in.xv.x),
-                               make_float2(in.dt.y * in.xv.y, in.dt.y * in.xv.y)};
+        float2 dtc[CPL], dtx[CPL];
+#pragma unroll
+        for (int c = 0; c < CPL; c++) {
+            dtc[c] = make_float2(in.dt[c], in.dt[c]);
+            const float u = in.dt[c] * in.xv[c];
+            dtx[c] = make_float2(u, u);
+        }
         const float4 *row = reinterpret_cast<const float4 *>(sm.bc + (i & (2 * kTC - 1)) * 2 * NS);
-        float2 ya[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        float2 yb[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        if (SUMMARY)
-            sdt = __fadd2_rn(sdt, in.dt);
+        float2 ya[CPL], yb[CPL];
+#pragma unroll
+        for (int c = 0; c < CPL; c++) {
+            ya[c] = make_float2(0.f, 0.f);
+            yb[c] = make_float2(0.f, 0.f);
+            if (SUMMARY)
+                sdt[c] += in.dt[c];
+        }
 #pragma unroll
         for (int q = 0; q < NS / 4; q++) {
             const float4 bq = row[q];
@@ -369,7 +464,7 @@ __device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P,
             for (int r = 0; r < 2; r++) {
                 const int k = 2 * q + r;   // state pair index
 #pragma unroll
-                for (int c = 0; c < 2; c++) {
+                for (int c = 0; c < CPL; c++) {
                     const float2 v = __fmul2_rn(dtc[c], Ap[c][k]);
                     float2 e;
                     if (2 * k < NS - NPOLY) {
@@ -388,28 +483,36 @@ __device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P,
                 }
             }
         }
-        const float2 s0v = __fadd2_rn(ya[0], yb[0]);
-        const float2 s1v = __fadd2_rn(ya[1], yb[1]);
-        return make_float2(s0v.x + s0v.y, s1v.x + s1v.y);
-    };
-    auto finish = [&](int i, const StepIn &in, float2 ys, auto phase2_tag) {
-        constexpr bool kPhase2 = decltype(phase2_tag)::value;
-        if (SUMMARY)
-            return;
-        float2 y = make_float2(fmaf(Dd.x, in.xv.x, ys.x), fmaf(Dd.y, in.xv.y, ys.y));
-        if (GATE) {
-            y.x *= in.zv.x;
-            y.y *= in.zv.y;
+        StepOut o;
+#pragma unroll
+        for (int c = 0; c < CPL; c++) {
+            const float2 sv = __fadd2_rn(ya[c], yb[c]);
+            o.y[c] = sv.x + sv.y;
         }
-        if (active) {
+        return o;
+    };
+    auto finish = [&](int i, const StepIn &in, const StepOut &ys, auto phase2_tag) {
+        constexpr bool kPhase2 = decltype(phase2_tag)::value;
+        float y[CPL];
+#pragma unroll
+        for (int c = 0; c < CPL; c++) {
+            y[c] = fmaf(Dd[c], in.xv[c], ys.y[c]);
+            if (GATE)
+                y[c] *= in.zv[c];
+        }
+        if (!SUMMARY && active) {
             const size_t io = (rowbase + tpos(i)) * a.D + d;
             if (!BIDIR) {
-                IO<T>::st2(out + io, y);
+                IO<T, CPL>::st(out + io, y);
             } else if (!kPhase2) {
-                *reinterpret_cast<float2 *>(stash + io) = y;
+                IO<float, CPL>::st(stash + io, y);
             } else {
-                const float2 o = *reinterpret_cast<const float2 *>(slot_of(i) + 3 * WS::kRowB + lane * 8);
-                IO<T>::st2(out + io, make_float2(y.x + o.x, y.y + o.y));
+                float o[CPL];
+                IO<float, CPL>::ld(slot_of(i) + 3 * WS::kRowB + lane * CPL * 4, o);
+#pragma unroll
+                for (int c = 0; c < CPL; c++)
+                    y[c] += o[c];
+                IO<T, CPL>::st(out + io, y);
             }
         }
     };
@@ -421,7 +524,7 @@ __device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P,
     // recurrences back to back, then the epilogues
     auto group = [&](int i, auto phase2_tag) {
         StepIn in[kSub];
-        float2 ys[kSub];
+        StepOut ys[kSub];
 #pragma unroll
         for (int j = 0; j < kSub; j++)
             in[j] = load_dt(i + j);
@@ -456,10 +559,7 @@ __device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P,
         with_stash = true;
         // steps already in flight were issued without their stash rows
         const int issued = min(Tn, ((M + kSub - 1) / kSub + kStages - 1) * kSub);
-        for (int i = M; i < issued; i++)
-            if (active)
-                cp_async<8>(slot_of(i) + 3 * WS::kRowB + lane * 8,
-                            stash + (rowbase + tpos(i)) * a.D + d);
+        issue_stash(M, issued);
         cp_async_wait_all();
         __syncwarp();
         run(M, Tn, PhaseTag<true>{});
@@ -467,18 +567,19 @@ __device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P,
     cp_async_wait_all();
 }
 
-template <typename T, int NS>
-constexpr int smem_bytes() { return kWarps * (int)sizeof(WarpSmem<T, NS>); }
+template <typename T, int NS, int CPL>
+constexpr int smem_bytes() { return kWarps * (int)sizeof(WarpSmem<T, NS, CPL>); }
 
 // ---------------------------------------------------------------- summary
-template <typename T, int NS, int NPOLY, bool SOFTPLUS>
-__global__ void __launch_bounds__(64, kMinBlocks) s6_summary_kernel(const S6Args a)
+template <typename T, int NS, int CPL, int NPOLY, bool SOFTPLUS>
+__global__ void __launch_bounds__(64, min_blocks<CPL>()) s6_summary_kernel(const S6Args a)
 {
     extern __shared__ __align__(16) char smem_raw[];
-    WarpSmem<T, NS> *sm = reinterpret_cast<WarpSmem<T, NS> *>(smem_raw);
+    WarpSmem<T, NS, CPL> *sm = reinterpret_cast<WarpSmem<T, NS, CPL> *>(smem_raw);
+    constexpr int kCh = 32 * CPL;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int dbase = (blockIdx.x * kWarps + warp) * kCh;
-    const int d = dbase + 2 * lane;
+    const int d = dbase + CPL * lane;
     const int seg = blockIdx.y;
     const int dsel = blockIdx.z % a.ndir;
     const int b = blockIdx.z / a.ndir;
@@ -487,20 +588,21 @@ __global__ void __launch_bounds__(64, kMinBlocks) s6_summary_kernel(const S6Args
         return;
     const bool active = d < a.D;
     const int s0 = seg * a.T, s1 = min(a.L, s0 + a.T);
-    float2 h[2][NS / 2];
+    float2 h[CPL][NS / 2];
+    float sdt[CPL];
 #pragma unroll
-    for (int c = 0; c < 2; c++)
+    for (int c = 0; c < CPL; c++) {
+        sdt[c] = 0.f;
 #pragma unroll
         for (int k = 0; k < NS / 2; k++)
             h[c][k] = make_float2(0.f, 0.f);
-    float2 sdt = make_float2(0.f, 0.f);
-    scan_segment<T, NS, NPOLY, true, false, false, SOFTPLUS>(a, a.dir[dsel], sm[warp], b, dbase,
-                                                             active, s0, s1, rev, h, sdt);
+    }
+    scan_segment<T, NS, CPL, NPOLY, true, false, false, SOFTPLUS>(a, a.dir[dsel], sm[warp], b, dbase,
+                                                                  active, s0, s1, rev, h, sdt);
     if (!active)
         return;
-    const float sd[2] = {sdt.x, sdt.y};
 #pragma unroll
-    for (int c = 0; c < 2; c++) {
+    for (int c = 0; c < CPL; c++) {
         const size_t ci = (((size_t)dsel * a.Bsz + b) * a.S + seg) * a.D + d + c;
 #pragma unroll
         for (int k = 0; k < NS / 2; k++) {
@@ -509,7 +611,7 @@ __global__ void __launch_bounds__(64, kMinBlocks) s6_summary_kernel(const S6Args
             if (2 * k + 1 < a.N)
                 a.carry_h[ci * a.N + 2 * k + 1] = h[c][k].y;
         }
-        a.carry_s[ci] = sd[c];
+        a.carry_s[ci] = sdt[c];
     }
 }
 
@@ -559,15 +661,16 @@ __global__ void s6_carry_kernel(const S6Args a)
 }
 
 // ------------------------------------------------------------------- main
-template <typename T, int NS, int NPOLY, bool BIDIR, bool GATE, bool SOFTPLUS>
-__global__ void __launch_bounds__(64, kMinBlocks) s6_main_kernel(const S6Args a)
+template <typename T, int NS, int CPL, int NPOLY, bool BIDIR, bool GATE, bool SOFTPLUS>
+__global__ void __launch_bounds__(64, min_blocks<CPL>()) s6_main_kernel(const S6Args a)
 {
     extern __shared__ __align__(16) char smem_raw[];
-    WarpSmem<T, NS> *sm = reinterpret_cast<WarpSmem<T, NS> *>(smem_raw);
+    WarpSmem<T, NS, CPL> *sm = reinterpret_cast<WarpSmem<T, NS, CPL> *>(smem_raw);
+    constexpr int kCh = 32 * CPL;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int dsel = BIDIR ? warp : 0;
     const int dbase = BIDIR ? blockIdx.x * kCh : (blockIdx.x * kWarps + warp) * kCh;
-    const int d = dbase + 2 * lane;
+    const int d = dbase + CPL * lane;
     const bool active = d < a.D;
     const int seg = blockIdx.y, b = blockIdx.z;
     const int s0 = seg * a.T, s1 = min(a.L, s0 + a.T);
@@ -575,10 +678,12 @@ __global__ void __launch_bounds__(64, kMinBlocks) s6_main_kernel(const S6Args a)
     const DirArgs &P = a.dir[dsel];
     if (!BIDIR && dbase >= a.D)
         return;   // whole warp past the channels (never with a barrier partner)
-    float2 h[2][NS / 2];
+    float2 h[CPL][NS / 2];
+    float sdt[CPL];
     const bool has_carry = a.S > 1 && !first_in_order(seg, a.S, rev);
 #pragma unroll
-    for (int c = 0; c < 2; c++) {
+    for (int c = 0; c < CPL; c++) {
+        sdt[c] = 0.f;
         const size_t ci = (((size_t)dsel * a.Bsz + b) * a.S + seg) * a.D + d + c;
 #pragma unroll
         for (int k = 0; k < NS / 2; k++) {
@@ -586,12 +691,11 @@ __global__ void __launch_bounds__(64, kMinBlocks) s6_main_kernel(const S6Args a)
             h[c][k].y = (active && has_carry && 2 * k + 1 < a.N) ? a.carry_h[ci * a.N + 2 * k + 1] : 0.f;
         }
     }
-    float2 sdt = make_float2(0.f, 0.f);
-    scan_segment<T, NS, NPOLY, false, BIDIR, GATE, SOFTPLUS>(a, P, sm[warp], b, dbase, active, s0,
-                                                             s1, rev, h, sdt);
+    scan_segment<T, NS, CPL, NPOLY, false, BIDIR, GATE, SOFTPLUS>(a, P, sm[warp], b, dbase, active,
+                                                                  s0, s1, rev, h, sdt);
     if (active && P.last_state && last_in_order(seg, a.S, rev)) {
 #pragma unroll
-        for (int c = 0; c < 2; c++) {
+        for (int c = 0; c < CPL; c++) {
             float *ls = P.last_state + ((size_t)b * a.D + d + c) * a.N;
 #pragma unroll
             for (int k = 0; k < NS / 2; k++) {
@@ -610,13 +714,14 @@ cudaError_t set_smem(KernelT k, int bytes)
     return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
-template <typename T, int NS, int NPOLY, bool GATE, bool SOFTPLUS>
+template <typename T, int NS, int CPL, int NPOLY, bool GATE, bool SOFTPLUS>
 cudaError_t launch_typed(const S6Args &a, cudaStream_t st)
 {
-    constexpr int smem = smem_bytes<T, NS>();
+    constexpr int smem = smem_bytes<T, NS, CPL>();
+    constexpr int kCh = 32 * CPL;
     cudaError_t e;
     if (a.S > 1) {
-        auto ks = s6_summary_kernel<T, NS, NPOLY, SOFTPLUS>;
+        auto ks = s6_summary_kernel<T, NS, CPL, SSM_S6_SUM_NPOLY(NS), SOFTPLUS>;
         if ((e = set_smem(ks, smem)) != cudaSuccess)
             return e;
         dim3 g1((a.D + kWarps * kCh - 1) / (kWarps * kCh), a.S, a.Bsz * a.ndir);
@@ -625,19 +730,26 @@ cudaError_t launch_typed(const S6Args &a, cudaStream_t st)
         s6_carry_kernel<<<(unsigned)((tot + 255) / 256), 256, 0, st>>>(a);
     }
     if (a.ndir == 2) {
-        auto km = s6_main_kernel<T, NS, NPOLY, true, GATE, SOFTPLUS>;
+        auto km = s6_main_kernel<T, NS, CPL, NPOLY, true, GATE, SOFTPLUS>;
         if ((e = set_smem(km, smem)) != cudaSuccess)
             return e;
         dim3 g((a.D + kCh - 1) / kCh, a.S, a.Bsz);
         km<<<g, 64, smem, st>>>(a);
     } else {
-        auto km = s6_main_kernel<T, NS, NPOLY, false, GATE, SOFTPLUS>;
+        auto km = s6_main_kernel<T, NS, CPL, NPOLY, false, GATE, SOFTPLUS>;
         if ((e = set_smem(km, smem)) != cudaSuccess)
             return e;
         dim3 g((a.D + kWarps * kCh - 1) / (kWarps * kCh), a.S, a.Bsz);
         km<<<g, 64, smem, st>>>(a);
     }
     return cudaGetLastError();
+}
+
+template <typename T, int NS, int NPOLY, bool GATE, bool SOFTPLUS>
+cudaError_t launch_cpl(const S6Args &a, cudaStream_t st)
+{
+    return a.cpl == 1 ? launch_typed<T, NS, 1, NPOLY, GATE, SOFTPLUS>(a, st)
+                      : launch_typed<T, NS, 2, NPOLY, GATE, SOFTPLUS>(a, st);
 }
 
 #ifndef SSM_S6_NPOLY
@@ -649,10 +761,10 @@ cudaError_t launch_flags(const S6Args &a, cudaStream_t st)
 {
     const bool gate = a.dir[0].z != nullptr;
     if (gate)
-        return a.softplus ? launch_typed<T, NS, NPOLY, true, true>(a, st)
-                          : launch_typed<T, NS, NPOLY, true, false>(a, st);
-    return a.softplus ? launch_typed<T, NS, NPOLY, false, true>(a, st)
-                      : launch_typed<T, NS, NPOLY, false, false>(a, st);
+        return a.softplus ? launch_cpl<T, NS, NPOLY, true, true>(a, st)
+                          : launch_cpl<T, NS, NPOLY, true, false>(a, st);
+    return a.softplus ? launch_cpl<T, NS, NPOLY, false, true>(a, st)
+                      : launch_cpl<T, NS, NPOLY, false, false>(a, st);
 }
 
 template <typename T>
@@ -669,12 +781,16 @@ cudaError_t launch_ns(const S6Args &a, cudaStream_t st)
 
 S6Plan plan_s6(int64_t Bsz, int64_t L, int64_t D, int64_t N, int ndir, int dtype)
 {
-    S6Plan p{1, (int)L, 0, 0, 0, 0};
+    S6Plan p{1, (int)L, 2, 0, 0, 0, 0};
     if (L <= 0)
         return p;
+    // Channels per lane: two give each thread more independent work, one
+    // gives twice the threads (and fewer segments) when the problem is small.
+    const int64_t lanes2 = (int64_t)ndir * Bsz * ((D + 1) / 2);
+    p.cpl = SSM_S6_CPL != 0 ? SSM_S6_CPL : (lanes2 < SSM_S6_CPL1_BELOW ? 1 : 2);
     const int64_t kMinT = 16;
-    const int64_t kTargetThreads = 148 * 320;
-    const int64_t threads = (int64_t)ndir * Bsz * ((D + 1) / 2);
+    const int64_t kTargetThreads = p.cpl == 1 ? SSM_S6_TARGET1 : SSM_S6_TARGET2;
+    const int64_t threads = (int64_t)ndir * Bsz * ((D + p.cpl - 1) / p.cpl);
     int64_t S = 1;
     if (threads > 0 && threads < kTargetThreads)
         S = (kTargetThreads + threads - 1) / threads;

@@ -83,6 +83,7 @@ ssm_status run_s6(const ssm_dims *dims, const void *x, const void *delta, int so
     a.N = (int)dims->dstate;
     a.S = plan.S;
     a.T = plan.T;
+    a.cpl = plan.cpl;
     a.dtype = dt;
     a.softplus = softplus ? 1 : 0;
     a.ndir = ndir;
@@ -120,6 +121,23 @@ size_t bidir_scan_workspace_size(const ssm_dims *dims)
         return 0;
     return ssm::plan_s6(dims->batch, dims->seqlen, dims->dim, dims->dstate, 2,
                         dims->dtype == SSM_F32 ? 0 : 1).workspace_bytes;
+}
+
+ssm_status ssm_scan_plan(const ssm_dims *dims, int bidirectional, int *segments,
+                         int *channels_per_lane)
+{
+    const ssm_status st = check_s6_dims(dims);
+    if (st != SSM_OK)
+        return st;
+    ssm::S6Plan plan{1, 0, 2, 0, 0, 0, 0};
+    if (!empty_s6(dims))
+        plan = ssm::plan_s6(dims->batch, dims->seqlen, dims->dim, dims->dstate,
+                            bidirectional ? 2 : 1, dims->dtype == SSM_F32 ? 0 : 1);
+    if (segments)
+        *segments = plan.S;
+    if (channels_per_lane)
+        *channels_per_lane = plan.cpl;
+    return SSM_OK;
 }
 
 ssm_status ssm_scan_fwd(const ssm_dims *dims, const void *x, const void *delta,

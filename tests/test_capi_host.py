@@ -121,3 +121,29 @@ def test_plan_is_deterministic(lib):
         a = lib.bidir_scan_workspace_size(ctypes.byref(dims))
         b = lib.bidir_scan_workspace_size(ctypes.byref(dims))
         assert a == b
+
+
+def test_scan_plan(lib):
+    """The launch-plan query: segment count and channels per lane for the
+    workloads' sizes, the bounds the plan keeps, and its argument checks."""
+    # Vim-Small bidirectional: enough channels for one pass, two per lane
+    assert ssm.scan_plan(64, 197, 768, 16, bidirectional=True) == (1, 2)
+    # the bf16 workloads have few channels: one per lane, several segments
+    for b, L, D in ((8, 1024, 768), (4, 16384, 192)):
+        seg, cpl = ssm.scan_plan(b, L, D, 16, ssm.SSM_BF16, bidirectional=True)
+        assert cpl == 1 and 1 < seg <= (L + 15) // 16
+    # segments never shorter than 16 steps, never more than the steps
+    for L in (1, 15, 16, 17, 100):
+        seg, _ = ssm.scan_plan(1, L, 32, 16)
+        assert 1 <= seg <= max(1, (L + 15) // 16)
+    assert ssm.scan_plan(0, 10, 32, 16)[0] == 1      # empty problem
+    assert ssm.scan_plan(2, 0, 32, 16)[0] == 1
+    # the plan's segment count matches the workspace the scan asks for
+    dims = _dims(2, 4096, 64, 16)
+    seg, _ = ssm.scan_plan(2, 4096, 64, 16)
+    assert seg > 1 and lib.ssm_scan_workspace_size(ctypes.byref(dims)) > 0
+    with pytest.raises(ssm.SSMError):
+        ssm.scan_plan(1, 10, 32, 17)                 # N > 16
+    with pytest.raises(ssm.SSMError):
+        ssm.scan_plan(1, 10, 30, 16)                 # D not a multiple of 4
+    assert lib.ssm_scan_plan(None, 0, None, None) == 1

@@ -93,6 +93,40 @@ def test_long_row_bidir_bf16_full_size_sampled():
     _check_bidir(inp, last_state=True, cols=cols)
 
 
+# ------------------------------------------------- both lane mappings
+
+@pytest.mark.parametrize("batch,L,D,bidir,dtype,cpl", [
+    (32, 300, 768, True, "f32", 2),    # two channels per lane, two segments
+    (64, 100, 768, False, "f32", 2),   # single direction, two per lane, two segments
+    (2, 300, 96, True, "bf16", 1),     # one per lane, 16-step segments, 3 warps of channels
+    (3, 500, 40, False, "f32", 1),     # one per lane, a warp only partly inside D
+])
+def test_lane_mappings(batch, L, D, bidir, dtype, cpl):
+    """Both thread layouts (one or two channels per lane), with and without
+    segments, against the oracle on sampled columns (reversed for the
+    single-direction cases)."""
+    code = ssm.SSM_F32 if dtype == "f32" else ssm.SSM_BF16
+    seg, got = ssm.scan_plan(batch, L, D, 16, code, bidirectional=bidir)
+    assert got == cpl and seg > 1
+    inp = ssm_gen.make_s6_inputs(batch, L, D, 16, dtype=dtype, bidir=bidir, seed=L + D,
+                                 random_A=True, random_D=True)
+    rng = np.random.default_rng(L)
+    cols = rng.choice(batch * D, min(48, batch * D), replace=False)
+    b, d = np.divmod(cols, D)
+    tol = TOL[dtype]
+    if bidir:
+        out, lf, lb = run_bidir(inp, last_state=True)
+        ref, rlf, rlb = oracle.bidir(inp, cols=cols, nthreads=8)
+        assert rel_err(host(out)[b, :, d], ref[b, :, d]) <= tol
+        assert rel_err(lf.cpu().numpy()[b, d], rlf[b, d]) <= tol
+        assert rel_err(lb.cpu().numpy()[b, d], rlb[b, d]) <= tol
+    else:
+        out, st = run_s6(inp, reverse=True)
+        ref, rst = oracle.s6(inp, reverse=True, cols=cols, nthreads=8)
+        assert rel_err(host(out)[b, :, d], ref[b, :, d]) <= tol
+        assert rel_err(st.cpu().numpy()[b, d], rst[b, d]) <= tol
+
+
 # ------------------------------------------------------------ ragged / edges
 
 @pytest.mark.parametrize("L", [1, 2, 3, 17, 255, 256, 257, 1000, 4099])
