@@ -52,9 +52,26 @@ namespace {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kWarps = 2;   // warps per CTA
 constexpr int kTC = 16;     // steps per B/C staging chunk
-constexpr int kSub = 4;     // steps per cp.async group
-constexpr int kStages = 2;  // cp.async groups in the ring
-constexpr int kSlots = kSub * kStages;
+// cp.async ring: steps per group and groups in flight, by channels per lane
+// (two channels per lane hold more registers, so shorter groups).
+#ifndef SSM_S6_KSUB2
+#define SSM_S6_KSUB2 2
+#endif
+#ifndef SSM_S6_KSTAGES2
+#define SSM_S6_KSTAGES2 4
+#endif
+#ifndef SSM_S6_KSUB1
+#define SSM_S6_KSUB1 4
+#endif
+#ifndef SSM_S6_KSTAGES1
+#define SSM_S6_KSTAGES1 2
+#endif
+template <int CPL> struct Ring {
+    static constexpr int kSub = CPL == 2 ? SSM_S6_KSUB2 : SSM_S6_KSUB1;        // steps per group
+    static constexpr int kStages = CPL == 2 ? SSM_S6_KSTAGES2 : SSM_S6_KSTAGES1;  // groups in the ring
+    static constexpr int kSlots = kSub * kStages;
+    static_assert(kTC % kSub == 0, "B/C staging rotates on group boundaries");
+};
 #ifndef SSM_S6_MINB
 #define SSM_S6_MINB 6
 #endif
@@ -99,6 +116,30 @@ __device__ __forceinline__ float rcp_mufu(float v)
     float r;
     asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
     return r;
+}
+
+// Pairwise multiply / fused multiply-add on two states at once: the packed
+// f32x2 instructions of sm_100, or two scalar instructions (SSM_S6_SCALAR).
+#ifndef SSM_S6_SCALAR
+#define SSM_S6_SCALAR 0
+#endif
+__device__ __forceinline__ float2 mul2(float2 a, float2 b)
+{
+    if (SSM_S6_SCALAR)
+        return make_float2(a.x * b.x, a.y * b.y);
+    return __fmul2_rn(a, b);
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c)
+{
+    if (SSM_S6_SCALAR)
+        return make_float2(fmaf(a.x, b.x, c.x), fmaf(a.y, b.y, c.y));
+    return __ffma2_rn(a, b, c);
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b)
+{
+    if (SSM_S6_SCALAR)
+        return make_float2(a.x + b.x, a.y + b.y);
+    return __fadd2_rn(a, b);
 }
 
 // 2^v for two values on the FMA pipe: v = j + f with j = rint(v), |f| <= 1/2;
@@ -292,7 +333,7 @@ struct WarpSmem {
     static constexpr int kRowB = kCh * (int)sizeof(T);   // one x, delta or z row
     static constexpr int kStashB = kCh * 4;              // one fp32 stash row
     static constexpr int kSlotB = 3 * kRowB + kStashB;
-    char ring[kSlots * kSlotB];
+    char ring[Ring<CPL>::kSlots * kSlotB];
     float bc[2 * kTC * 2 * NS];
 };
 
@@ -320,6 +361,7 @@ __device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P,
     using WS = WarpSmem<T, NS, CPL>;
     using RC = RowCopy<WS::kRowB>;
     using RS = RowCopy<WS::kStashB>;
+    constexpr int kSub = Ring<CPL>::kSub, kStages = Ring<CPL>::kStages, kSlots = Ring<CPL>::kSlots;
     static_assert(NPOLY % 2 == 0 && NPOLY <= NS, "NPOLY counts state pairs");
     const int lane = threadIdx.x & 31;
     const int d = dbase + CPL * lane;
@@ -465,7 +507,7 @@ __device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P,
                 const int k = 2 * q + r;   // state pair index
 #pragma unroll
                 for (int c = 0; c < CPL; c++) {
-                    const float2 v = __fmul2_rn(dtc[c], Ap[c][k]);
+                    const float2 v = mul2(dtc[c], Ap[c][k]);
                     float2 e;
                     if (2 * k < NS - NPOLY) {
                         e.x = ex2_mufu(v.x);
@@ -473,12 +515,12 @@ __device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P,
                     } else {
                         e = ex2_poly2(v);
                     }
-                    h[c][k] = __ffma2_rn(e, h[c][k], __fmul2_rn(dtx[c], bp[r]));
+                    h[c][k] = fma2(e, h[c][k], mul2(dtx[c], bp[r]));
                     if (!SUMMARY) {
                         if (r == 0)
-                            ya[c] = __ffma2_rn(cp[r], h[c][k], ya[c]);
+                            ya[c] = fma2(cp[r], h[c][k], ya[c]);
                         else
-                            yb[c] = __ffma2_rn(cp[r], h[c][k], yb[c]);
+                            yb[c] = fma2(cp[r], h[c][k], yb[c]);
                     }
                 }
             }
@@ -486,7 +528,7 @@ __device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P,
         StepOut o;
 #pragma unroll
         for (int c = 0; c < CPL; c++) {
-            const float2 sv = __fadd2_rn(ya[c], yb[c]);
+            const float2 sv = add2(ya[c], yb[c]);
             o.y[c] = sv.x + sv.y;
         }
         return o;

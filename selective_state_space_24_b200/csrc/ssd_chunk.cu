@@ -85,7 +85,7 @@ constexpr int kSmemBytes = kOffVec + 2 * kDtBufs * 64 * 4 + 1024; // + alignment
 // chunk c + 1's first products were issued.
 constexpr uint32_t kColG = 0, kColDS = 64, kColYo = 192, kColYd = 448, kTmemCols = 512;
 
-constexpr long kWaitLimit = 1l << 26;
+constexpr long kWaitLimit = 1l << 20;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
@@ -128,20 +128,38 @@ __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence:
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-// Bounded wait on an mbarrier phase; on giving up, flag the error and return
-// false (the caller carries on so that every thread still meets every barrier).
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
+// Bounded wait on an mbarrier phase (with SSM_SSD_SUSPEND_NS > 0 each
+// try_wait may suspend the thread for up to that long; it resumes when the
+// phase completes).  On
+// giving up, a thread flags the library's error word and its CTA's abort
+// word and returns false; every later wait in the CTA then gives up at once,
+// so the kernel still ends promptly (with wrong values, reported by
+// ssm_check_device) and every thread still meets every barrier.
+#ifndef SSM_SSD_SUSPEND_NS
+#define SSM_SSD_SUSPEND_NS 0
+#endif
+constexpr uint32_t kSuspendNs = SSM_SSD_SUSPEND_NS;
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort)
 {
     const uint32_t a = smem_u32(bar);
     for (long it = 0; it < kWaitLimit; it++) {
         uint32_t ok;
-        asm volatile("{.reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p;}"
-                     : "=r"(ok)
-                     : "r"(a), "r"(parity)
-                     : "memory");
+        if (kSuspendNs)
+            asm volatile("{.reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p;}"
+                         : "=r"(ok)
+                         : "r"(a), "r"(parity), "r"(kSuspendNs)
+                         : "memory");
+        else
+            asm volatile("{.reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p;}"
+                         : "=r"(ok)
+                         : "r"(a), "r"(parity)
+                         : "memory");
         if (ok)
             return true;
+        if ((it & 255) == 255 && *abort)
+            return false;
     }
+    *abort = 1;
     atomicExch(&g_device_error, 1u);
     return false;
 }
@@ -166,34 +184,38 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, i
 }
 
 
+// TMEM loads.  They are asynchronous: the registers are valid only after
+// tmem_wait_ld(), so several loads can be in flight behind one wait.
+//
 // 8 columns of one M = 64 accumulator row: threads t < 16 of warp w get row
 // 16 (w mod 4) + t, columns [col, col + 8); threads t >= 16 the same row,
 // columns [col + 8, col + 16).
-__device__ __forceinline__ void tmem_ld_eighth_row(uint32_t taddr, float (&v)[8])
+__device__ __forceinline__ void tmem_ld_eighth_row(uint32_t taddr, uint32_t (&r)[8])
 {
-    uint32_t r[8];
     asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8], 8;"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
                  : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int k = 0; k < 8; k++)
-        v[k] = __uint_as_float(r[k]);
 }
 
 // 16 consecutive columns of this thread's lane (an M = 128 accumulator row)
-__device__ __forceinline__ void tmem_ld_row16(uint32_t taddr, float *v)
+__device__ __forceinline__ void tmem_ld_row16(uint32_t taddr, uint32_t (&r)[16])
 {
-    uint32_t r[16];
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr));
+}
+
+// Wait for this thread's TMEM loads.  The registers pass through an empty
+// asm so that no use of them is scheduled above the wait.
+template <int K>
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[K])
+{
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-    for (int k = 0; k < 16; k++)
-        v[k] = __uint_as_float(r[k]);
+    for (int k = 0; k < K; k++)
+        asm volatile("" : "+r"(r[k]));
 }
 
 
@@ -265,10 +287,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ __align__(8) uint64_t bar_tma[kStages];
-    __shared__ __align__(8) uint64_t bar_mma1[2];
-    __shared__ __align__(8) uint64_t bar_mma2;
-    __shared__ __align__(8) uint64_t bar_mready;  // math threads: M(c) written
-    __shared__ __align__(8) uint64_t bar_sready;  // math threads: S_in(c + 1), W(c + 1) written
+    __shared__ __align__(8) uint64_t bar_g;       // tensor core: G(c) done
+    __shared__ __align__(8) uint64_t bar_ds;      // tensor core: dS(c) done (and Yo(c) before it)
+    __shared__ __align__(8) uint64_t bar_mma2;    // tensor core: Yd(c) done
+    __shared__ __align__(8) uint64_t bar_mready;  // math threads: M(c) written, G(c) read
+    __shared__ __align__(8) uint64_t bar_sready;  // math threads: W(c + 1), S_in(c + 1) written, dS(c) read
+    __shared__ volatile int abort_sh;
     __shared__ __align__(8) uint64_t bar_dt_full[kDtBufs];    // dt warp: dt / cs of a chunk written
     __shared__ __align__(8) uint64_t bar_free[kDtBufs];       // math threads: done with a chunk's stage and dt
     __shared__ uint32_t tmem_base_sh;
@@ -290,8 +314,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
         for (int k = 0; k < kStages; k++)
             asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bar_tma[k])));
-        for (int k = 0; k < 2; k++)
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bar_mma1[k])));
+        abort_sh = 0;
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bar_g)));
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bar_ds)));
         asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bar_mma2)));
         asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(&bar_mready)), "r"(kMath));
         asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(&bar_sready)), "r"(kMath));
@@ -315,6 +340,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tb = tmem_base_sh;
     const uint32_t tw = tb + ((uint32_t)(wq * 32) << 16);   // this warp's TMEM lanes
+    volatile int *abort = &abort_sh;
+    auto wait = [&](uint64_t *bar, uint32_t parity) { return mbar_wait(bar, parity, abort); };
 
     auto issue_tma = [&](int c) {
         uint8_t *st = sm + (c % kStages) * kStageBytes;
@@ -370,20 +397,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         *reinterpret_cast<float2 *>(dtv + 2 * lane) = make_float2(d0, d1);
     };
 
-    // W(c) = exp(cs_end - cs_j) dt_j X[j, :] as bf16 hi + lo, rows j, X's swizzled layout
-    auto build_w = [&](int c) {
+    // W(c) = exp(cs_end - cs_j) dt_j X[j, :] as bf16 hi + lo, rows j, X's
+    // swizzled layout, into buffer c & 1: this thread's 16-byte piece (row
+    // j = tid / 8, piece tid mod 8).  Split in two so the loads can be issued
+    // early and the rest interleaved with other work.
+    struct WIn {
+        uint4 xv;
+        float wj;
+    };
+    auto w_load = [&](int c) {
         const uint8_t *st = sm + (c % kStages) * kStageBytes;
         const float *cs = cs_s + (c % kDtBufs) * 64, *dtv = dt_s + (c % kDtBufs) * 64;
+        const int j = tid >> 3, q = tid & 7;
+        WIn w;
+        w.wj = ex2f(cs[kQ - 1] - cs[j]) * dtv[j];
+        w.xv = *reinterpret_cast<const uint4 *>(st + kStageX + sw_chunk(j, q));
+        return w;
+    };
+    auto w_store = [&](int c, const WIn &w) {
         uint8_t *wb = sm + kOffW + (c & 1) * 2 * kTileX;
         const int j = tid >> 3, q = tid & 7;
-        const float wj = ex2f(cs[kQ - 1] - cs[j]) * dtv[j];
-        const uint4 xv = *reinterpret_cast<const uint4 *>(st + kStageX + sw_chunk(j, q));
-        const uint32_t u[4] = {xv.x, xv.y, xv.z, xv.w};
+        const uint32_t u[4] = {w.xv.x, w.xv.y, w.xv.z, w.xv.w};
         uint32_t o[4], ol[4];
 #pragma unroll
         for (int k = 0; k < 4; k++) {
             const float2 f = unpack_bf16(u[k]);
-            split_bf16(f.x * wj, f.y * wj, o[k], ol[k]);
+            split_bf16(f.x * w.wj, f.y * w.wj, o[k], ol[k]);
         }
         *reinterpret_cast<uint4 *>(wb + sw_chunk(j, q)) = make_uint4(o[0], o[1], o[2], o[3]);
         *reinterpret_cast<uint4 *>(wb + kTileX + sw_chunk(j, q)) = make_uint4(ol[0], ol[1], ol[2], ol[3]);
@@ -394,29 +433,48 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t idYo = idesc_bf16(64, 128, 0, 1);  // C (K-major) x [S_hi | S_lo] (MN-major)
     const uint32_t idYd = idesc_bf16(64, 64, 0, 1);   // M (K-major) x X (MN-major)
 
-    // first MMA group of chunk c: G = C B^T, Yo = C [S_hi | S_lo] (buffer c & 1),
-    // dS = B^T [W_hi | W_lo]
-    auto issue_group1 = [&](int c) {
+    // G = C B^T (committed on its own, so the decay matrix can start), then
+    // Yo = C [S_hi | S_lo] into buffer c & 1 (no commit: dS(c), issued after
+    // it, covers it)
+    auto issue_G_Yo = [&](int c) {
         const uint8_t *st = sm + (c % kStages) * kStageBytes;
         const uint32_t sC = smem_u32(st + kStageC), sB = smem_u32(st + kStageB);
         const uint32_t sS = smem_u32(sm + kOffS);
-        const uint32_t sW = smem_u32(sm + kOffW + (c & 1) * 2 * kTileX);
 #pragma unroll
         for (int kk = 0; kk < 8; kk++) {   // K = n, 8 steps of 16; two 64-wide atoms
             const uint32_t off = (kk >> 2) * kTileBC + (kk & 3) * 32;
             umma(tb + kColG, desc_sw128(sC + off, 16, 1024), desc_sw128(sB + off, 16, 1024), idG, kk > 0);
         }
+        umma_commit(&bar_g);
 #pragma unroll
         for (int kk = 0; kk < 8; kk++) {   // K = n; S rows n (MN-major), hi and lo blocks 16 KB apart
             const uint32_t offc = (kk >> 2) * kTileBC + (kk & 3) * 32;
             umma(tb + kColYo + (uint32_t)(c & 1) * 128, desc_sw128(sC + offc, 16, 1024),
                  desc_sw128(sS + kk * 2048, kSBytes, 1024), idYo, kk > 0);
         }
+    };
+    // dS = B^T [W_hi | W_lo]
+    auto issue_dS = [&](int c) {
+        const uint8_t *st = sm + (c % kStages) * kStageBytes;
+        const uint32_t sB = smem_u32(st + kStageB);
+        const uint32_t sW = smem_u32(sm + kOffW + (c & 1) * 2 * kTileX);
 #pragma unroll
         for (int kk = 0; kk < 4; kk++)     // K = j (rows); B^T: two MN atoms of 64 n, 8 KB apart;
             umma(tb + kColDS, desc_sw128(sB + kk * 2048, kTileBC, 1024),      // W hi and lo 8 KB apart
                  desc_sw128(sW + kk * 2048, kTileX, 1024), idDS, kk > 0);
-        umma_commit(&bar_mma1[c & 1]);
+        umma_commit(&bar_ds);
+    };
+    // Yd = [M_hi, then M_lo] X
+    auto issue_Yd = [&](int c) {
+        const uint8_t *st = sm + (c % kStages) * kStageBytes;
+        const uint32_t sM = smem_u32(sm + kOffM), sX = smem_u32(st + kStageX);
+#pragma unroll
+        for (int part = 0; part < 2; part++)
+#pragma unroll
+            for (int kk = 0; kk < 4; kk++)
+                umma(tb + kColYd, desc_sw128(sM + part * kTileX + kk * 32, 16, 1024),
+                     desc_sw128(sX + kk * 2048, 8192, 1024), idYd, part + kk > 0);
+        umma_commit(&bar_mma2);
     };
 
     // S: this thread's row n (= its TMEM lane), columns [16 g, 16 g + 16), fp32
@@ -437,7 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = 0; k < nch; k++) {
             const float2 dnext = load_delta2(k + 1);
             if (k >= kStages)
-                mbar_wait(&bar_free[k % kStages], ((k / kStages) - 1) & 1);
+                wait(&bar_free[k % kStages], ((k / kStages) - 1) & 1);
             if (lane == 0)
                 issue_tma(k);
             __syncwarp();
@@ -446,41 +504,38 @@ __global__ void __launch_bounds__(kThreads, 1)
             draw = dnext;
         }
     } else if (warp == kMmaWarp) {
-        // ---- the MMA warp: wait until the math threads have written the
-        // operands, then issue; lane 0 issues, the warp stays converged
-        bool ok = mbar_wait(&bar_sready, 0);   // W(0) written
-        if (lane == 0) {
-            tc_fence_after();
-            issue_group1(0);
-        }
-        __syncwarp();
-        for (int c = 0; c < nch && ok; c++) {
-            ok = mbar_wait(&bar_mready, c & 1);   // M(c) written
+        // ---- the MMA warp: lane 0 issues each product once its operands are
+        // written and its accumulator read; the warp stays converged.
+        // Per chunk c: Yd(c) once M(c) is written; G, Yo and dS of chunk
+        // c + 1 once W(c + 1) and S_in(c + 1) are.
+        auto lane0 = [&](auto fn) {
             if (lane == 0) {
                 tc_fence_after();
-                const uint8_t *st = sm + (c % kStages) * kStageBytes;
-                const uint32_t sM = smem_u32(sm + kOffM), sX = smem_u32(st + kStageX);
-#pragma unroll
-                for (int part = 0; part < 2; part++)   // M hi, then lo
-#pragma unroll
-                    for (int kk = 0; kk < 4; kk++)
-                        umma(tb + kColYd, desc_sw128(sM + part * kTileX + kk * 32, 16, 1024),
-                             desc_sw128(sX + kk * 2048, 8192, 1024), idYd, part + kk > 0);
-                umma_commit(&bar_mma2);
+                fn();
             }
             __syncwarp();
-            ok = ok && mbar_wait(&bar_sready, (c + 1) & 1);   // S_in(c + 1), W(c + 1) written
-            if (lane == 0 && c + 1 < nch) {
-                tc_fence_after();
-                issue_group1(c + 1);
+        };
+        bool ok = wait(&bar_sready, 0);   // W(0) written (its TMA landed); S_in(0) is zero
+        lane0([&] {
+            issue_G_Yo(0);
+            issue_dS(0);
+        });
+        for (int c = 0; c < nch && ok; c++) {
+            ok = wait(&bar_mready, c & 1);   // M(c) written, G(c) read
+            lane0([&] { issue_Yd(c); });
+            if (c + 1 < nch) {
+                ok = ok && wait(&bar_sready, (c + 1) & 1);   // W(c + 1), S_in(c + 1) written, dS(c) read
+                lane0([&] {
+                    issue_G_Yo(c + 1);
+                    issue_dS(c + 1);
+                });
             }
-            __syncwarp();
         }
     } else {
         // ---- math threads.  Prologue: W(0)
-        mbar_wait(&bar_dt_full[0], 0);
-        mbar_wait(&bar_tma[0], 0);
-        build_w(0);
+        wait(&bar_dt_full[0], 0);
+        wait(&bar_tma[0], 0);
+        w_store(0, w_load(0));
         fence_async_smem();
         tc_fence_before();
         mbar_arrive(&bar_sready);
@@ -489,29 +544,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint8_t *st = sm + (c % kStages) * kStageBytes;
             const float *cs = cs_s + (c % kDtBufs) * 64, *dtv = dt_s + (c % kDtBufs) * 64;
             const int t0 = c * kQ;
-            // ---- 1. next chunk's W
-            if (c + 1 < nch) {
-                mbar_wait(&bar_dt_full[(c + 1) % kDtBufs], ((c + 1) / kDtBufs) & 1);
-                mbar_wait(&bar_tma[(c + 1) % kStages], ((c + 1) / kStages) & 1);
-                build_w(c + 1);
-            }
-            // ---- 2. this chunk's first MMA group is done
-            mbar_wait(&bar_mma1[c & 1], (c >> 1) & 1);
-            tc_fence_after();
             const uint32_t buf = (uint32_t)(c & 1) * 64;
-            // ---- 3. masked decay matrix M (bf16 hi + lo, K-major rows i) from G; hand it over
+            // ---- 1. masked decay matrix M (bf16 hi + lo, K-major rows i) from G; hand it over
+            wait(&bar_g, c & 1);
+            tc_fence_after();
             {
-                float gv[8];
-                tmem_ld_eighth_row(tw + kColG + 16 * g, gv);
+                uint32_t gr[8];
+                tmem_ld_eighth_row(tw + kColG + 16 * g, gr);
                 const float csi = cs[row_i];
+                float e[8];
+#pragma unroll
+                for (int k = 0; k < 8; k++) {
+                    const int j = c8 + k;
+                    e[k] = (j <= row_i) ? ex2f(csi - cs[j]) * dtv[j] : 0.f;
+                }
+                tmem_wait_ld(gr);
                 uint32_t o[4], ol[4];
 #pragma unroll
-                for (int k = 0; k < 8; k += 2) {
-                    const int j0 = c8 + k;
-                    const float m0 = (j0 <= row_i) ? gv[k] * ex2f(csi - cs[j0]) * dtv[j0] : 0.f;
-                    const float m1 = (j0 + 1 <= row_i) ? gv[k + 1] * ex2f(csi - cs[j0 + 1]) * dtv[j0 + 1] : 0.f;
-                    split_bf16(m0, m1, o[k >> 1], ol[k >> 1]);
-                }
+                for (int k = 0; k < 8; k += 2)
+                    split_bf16(__uint_as_float(gr[k]) * e[k], __uint_as_float(gr[k + 1]) * e[k + 1], o[k >> 1],
+                               ol[k >> 1]);
                 const int q = c8 >> 3;
                 *reinterpret_cast<uint4 *>(sm + kOffM + sw_chunk(row_i, q)) = make_uint4(o[0], o[1], o[2], o[3]);
                 *reinterpret_cast<uint4 *>(sm + kOffM + kTileX + sw_chunk(row_i, q)) =
@@ -520,17 +572,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             fence_async_smem();
             tc_fence_before();
             mbar_arrive(&bar_mready);
-            // ---- 4. state update S = exp(cs_end) S + dS; bf16 hi + lo copy for the next chunk
+            // ---- 2. next chunk's W (the tensor core meanwhile finishes Yo(c), dS(c), Yd(c))
+            if (c + 1 < nch) {
+                wait(&bar_dt_full[(c + 1) % kDtBufs], ((c + 1) / kDtBufs) & 1);
+                wait(&bar_tma[(c + 1) % kStages], ((c + 1) / kStages) & 1);
+                w_store(c + 1, w_load(c + 1));
+            }
+            // ---- 3. state update S = exp(cs_end) S + dS; bf16 hi + lo copy S_in(c + 1); hand
+            // S_in(c + 1) and W(c + 1) over
+            wait(&bar_ds, c & 1);   // dS(c) done, and Yo(c) before it (S_in(c) is free)
+            tc_fence_after();
             {
                 const float decay = ex2f(cs[kQ - 1]);
-                float ds[16], dl[16];
+                uint32_t ds[16], dl[16];
                 tmem_ld_row16(tw + kColDS + 16 * g, ds);
                 tmem_ld_row16(tw + kColDS + 64 + 16 * g, dl);
+                tmem_wait_ld(ds);
+                tmem_wait_ld(dl);
 #pragma unroll
                 for (int k = 0; k < 16; k++)
-                    S[k] = fmaf(decay, S[k], ds[k] + dl[k]);
+                    S[k] = fmaf(decay, S[k], __uint_as_float(ds[k]) + __uint_as_float(dl[k]));
                 if (c + 1 < nch) {
-                    // single buffer: this chunk's C S_in finished before step 2
                     uint8_t *sn = sm + kOffS;
 #pragma unroll
                     for (int q2 = 0; q2 < 2; q2++) {
@@ -544,36 +606,37 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            // ---- 5. hand S_in(c + 1), W(c + 1) to the MMA warp
             fence_async_smem();
             tc_fence_before();
             mbar_arrive(&bar_sready);
-            // ---- 6. outputs: y = (Yd + exp(cs_i) Yo + D x) silu(z), row i, 8 columns
+            // ---- 4. outputs of chunk c: y = (Yd + exp(cs_i) Yo + D x) silu(z), row i, 8 columns
             {
-                float yo[8], yl[8], yd[8];
-                tmem_ld_eighth_row(tw + kColYo + 2 * buf + 16 * g, yo);
-                tmem_ld_eighth_row(tw + kColYo + 2 * buf + 64 + 16 * g, yl);
-#pragma unroll
-                for (int k = 0; k < 8; k++)
-                    yo[k] += yl[k];
-                mbar_wait(&bar_mma2, c & 1);
-                tc_fence_after();
-                tmem_ld_eighth_row(tw + kColYd + 16 * g, yd);
-                const float ei = ex2f(cs[row_i]);
-                const int t = t0 + row_i;
                 const int q = c8 >> 3;
                 const uint4 xv = *reinterpret_cast<const uint4 *>(st + kStageX + sw_chunk(row_i, q));
                 uint4 zv = make_uint4(0, 0, 0, 0);
                 if (args.has_z)
                     zv = *reinterpret_cast<const uint4 *>(st + kStageZ + sw_chunk(row_i, q));
+                const float ei = ex2f(cs[row_i]);
+                wait(&bar_mma2, c & 1);   // Yd(c) done
+                tc_fence_after();
+                uint32_t yo[8], yl[8], yd[8];
+                tmem_ld_eighth_row(tw + kColYo + 2 * buf + 16 * g, yo);
+                tmem_ld_eighth_row(tw + kColYo + 2 * buf + 64 + 16 * g, yl);
+                tmem_ld_eighth_row(tw + kColYd + 16 * g, yd);
+                tmem_wait_ld(yo);
+                tmem_wait_ld(yl);
+                tmem_wait_ld(yd);
+                const int t = t0 + row_i;
                 const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w};
                 const uint32_t zu[4] = {zv.x, zv.y, zv.z, zv.w};
                 uint32_t o[4];
 #pragma unroll
                 for (int k = 0; k < 4; k++) {
                     const float2 xf = unpack_bf16(xu[k]);
-                    float y0 = fmaf(ei, yo[2 * k], yd[2 * k]) + Dh * xf.x;
-                    float y1 = fmaf(ei, yo[2 * k + 1], yd[2 * k + 1]) + Dh * xf.y;
+                    const float yo0 = __uint_as_float(yo[2 * k]) + __uint_as_float(yl[2 * k]);
+                    const float yo1 = __uint_as_float(yo[2 * k + 1]) + __uint_as_float(yl[2 * k + 1]);
+                    float y0 = fmaf(ei, yo0, __uint_as_float(yd[2 * k])) + Dh * xf.x;
+                    float y1 = fmaf(ei, yo1, __uint_as_float(yd[2 * k + 1])) + Dh * xf.y;
                     if (args.has_z) {
                         const float2 zf = unpack_bf16(zu[k]);
                         y0 *= silu_f(zf.x);
@@ -585,8 +648,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     *reinterpret_cast<uint4 *>(args.out + (((size_t)b * L + t) * args.H + h) * kP + c8) =
                         make_uint4(o[0], o[1], o[2], o[3]);
             }
-            // ---- 7. hand chunk c's stage and dt buffer back to the dt warp
-            fence_async_smem();
+            // ---- 5. hand chunk c's stage and dt buffer back to the dt warp
             mbar_arrive(&bar_free[c % kStages]);
         }
     }
