@@ -54,6 +54,8 @@ def _load():
         lib = ctypes.CDLL(build())
         lib.oracle_s6.argtypes = [_i64] * 4 + [_dp, _dp, _dp, ctypes.c_int, _dp, _dp, _dp, _dp, _dp,
                                                ctypes.c_int, _dp, _dp, _ip, _i64, ctypes.c_int]
+        lib.oracle_s6_state.argtypes = ([_i64] * 4 + [_dp, _dp, _dp, ctypes.c_int, _dp, _dp, _dp, _dp, _dp,
+                                         ctypes.c_int, _dp, _dp, _dp, _dp, _i64, ctypes.c_int])
         lib.oracle_bidir.argtypes = ([_i64] * 4 + [_dp, _dp, ctypes.c_int] + [_dp] * 7 + [_dp] * 7
                                      + [_dp, _ip, _i64, ctypes.c_int])
         lib.oracle_ssd_seq.argtypes = [_i64] * 5 + [_dp, _dp, _dp, ctypes.c_int, _dp, _dp, _dp, _dp,
@@ -87,20 +89,39 @@ def _cols(cols):
 
 
 def s6_arrays(x, delta, A, B, C, *, delta_bias=None, softplus=True, D=None, z=None,
-              reverse=False, cols=None, want_state=True, nthreads=1
+              reverse=False, cols=None, want_state=True, nthreads=1, initial_state=None
               ) -> Tuple[np.ndarray, Optional[np.ndarray]]:
-    """Single-direction S6 on raw arrays: returns (out (B,L,D), last_state (B,D,N))."""
+    """Single-direction S6 on raw arrays: returns (out (B,L,D), last_state (B,D,N)).
+
+    initial_state (B, D, N): the state before the first step (None = zero)."""
     x, delta, A, B, C = map(_f64, (x, delta, A, B, C))
-    delta_bias, D, z = map(_f64, (delta_bias, D, z))
+    delta_bias, D, z, h0 = map(_f64, (delta_bias, D, z, initial_state))
     Bsz, L, Dm = x.shape
     N = A.shape[1]
     out = np.zeros((Bsz, L, Dm))
     st = np.zeros((Bsz, Dm, N)) if want_state else None
     keep, cp, nc = _cols(cols)
-    _load().oracle_s6(Bsz, L, Dm, N, _ptr(x), _ptr(delta), _ptr(delta_bias), int(softplus),
-                      _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), int(reverse), _ptr(out),
-                      _ptr(st), cp, nc, int(nthreads))
+    if h0 is None:
+        _load().oracle_s6(Bsz, L, Dm, N, _ptr(x), _ptr(delta), _ptr(delta_bias), int(softplus),
+                          _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), int(reverse), _ptr(out),
+                          _ptr(st), cp, nc, int(nthreads))
+    else:
+        assert h0.shape == (Bsz, Dm, N)
+        _load().oracle_s6_state(Bsz, L, Dm, N, _ptr(x), _ptr(delta), _ptr(delta_bias),
+                                int(softplus), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+                                int(reverse), _ptr(h0), _ptr(out), _ptr(st), cp, nc, int(nthreads))
     return out, st
+
+
+def step_arrays(x, delta, A, B, C, state, *, delta_bias=None, softplus=True, D=None, z=None):
+    """One time step of S6 for every (b, d) from a stored state -- the
+    recurrent (decode) form: x, delta, z (B, D); B, C (B, N); state (B, D, N).
+    Returns (y (B, D), new state (B, D, N)).  It is s6_arrays on a length-1
+    sequence started from `state`."""
+    add_t = lambda a: None if a is None else np.asarray(a)[:, None, ...]
+    out, st = s6_arrays(add_t(x), add_t(delta), A, add_t(B), add_t(C), delta_bias=delta_bias,
+                        softplus=softplus, D=D, z=add_t(z), initial_state=state)
+    return out[:, 0, :], st
 
 
 def s6(inp, reverse=False, cols=None, softplus=True, nthreads=1):

@@ -61,16 +61,18 @@ static double dt_of(double delta, const double *bias, int64_t d, int softplus)
 
 /*
  * One S6 column (batch b, channel d): the recurrence of sec. 4.3 with the
- * skip term and gate of sec. 4.4.  Writes y[t] for t in [0, L) and the final
- * state (N values) to hlast if non-NULL.
+ * skip term and gate of sec. 4.4.  The state starts at h0 (N values) or, if
+ * h0 is NULL, at zero as in sec. 4.3.  Writes y[t] for t in [0, L) and the
+ * final state (N values) to hlast if non-NULL.
  */
 static void s6_column(int64_t b, int64_t d, int64_t L, int64_t D, int64_t N,
                       const double *x, const double *delta, const double *bias, int softplus,
                       const double *A, const double *Bm, const double *Cm, const double *Dv,
-                      const double *z, int reverse, double *y, double *hlast, double *h)
+                      const double *z, int reverse, double *y, double *hlast, double *h,
+                      const double *h0)
 {
     for (int64_t n = 0; n < N; n++)
-        h[n] = 0.0;
+        h[n] = h0 ? h0[n] : 0.0;
     for (int64_t step = 0; step < L; step++) {
         int64_t t = reverse ? (L - 1 - step) : step;
         int64_t i = (b * L + t) * D + d;            /* (b, t, d) */
@@ -96,7 +98,8 @@ static void s6_column(int64_t b, int64_t d, int64_t L, int64_t D, int64_t N,
 /*
  * Single-direction S6.  x, delta, z: (Bsz, L, D); A: (D, N); Bm, Cm:
  * (Bsz, L, N); delta_bias, Dv: (D) or NULL; z NULL disables the gate.
- * out: (Bsz, L, D); last_state: (Bsz, D, N) or NULL.
+ * out: (Bsz, L, D); last_state: (Bsz, D, N) or NULL; initial_state:
+ * (Bsz, D, N), the state before the first step, or NULL for zero.
  * cols: list of column ids b*D + d to compute (NULL = every column); only
  * those columns of out / last_state are written.  If accumulate is set the
  * column's output is added to out instead of stored.
@@ -105,7 +108,8 @@ static void s6_run(int64_t Bsz, int64_t L, int64_t D, int64_t N,
                    const double *x, const double *delta, const double *delta_bias, int softplus,
                    const double *A, const double *Bm, const double *Cm, const double *Dv,
                    const double *z, int reverse, double *out, double *last_state,
-                   const int64_t *cols, int64_t ncols, int nthreads, int accumulate)
+                   const double *initial_state, const int64_t *cols, int64_t ncols, int nthreads,
+                   int accumulate)
 {
     int64_t total = cols ? ncols : Bsz * D;
 #ifdef _OPENMP
@@ -123,8 +127,9 @@ static void s6_run(int64_t Bsz, int64_t L, int64_t D, int64_t N,
             int64_t col = cols ? cols[k] : k;
             int64_t b = col / D, d = col % D;
             double *hl = last_state ? last_state + (b * D + d) * N : NULL;
+            const double *h0 = initial_state ? initial_state + (b * D + d) * N : NULL;
             s6_column(b, d, L, D, N, x, delta, delta_bias, softplus, A, Bm, Cm, Dv, z,
-                      reverse, y, hl, h);
+                      reverse, y, hl, h, h0);
             for (int64_t t = 0; t < L; t++) {
                 int64_t i = (b * L + t) * D + d;
                 out[i] = accumulate ? out[i] + y[t] : y[t];
@@ -142,7 +147,24 @@ void oracle_s6(int64_t Bsz, int64_t L, int64_t D, int64_t N,
                const int64_t *cols, int64_t ncols, int nthreads)
 {
     s6_run(Bsz, L, D, N, x, delta, delta_bias, softplus, A, Bm, Cm, Dv, z, reverse, out,
-           last_state, cols, ncols, nthreads, 0);
+           last_state, NULL, cols, ncols, nthreads, 0);
+}
+
+/*
+ * oracle_s6 from a given state: initial_state (Bsz, D, N) is h before the
+ * first step (before t = 0, or before t = L-1 reversed).  The recurrence
+ * of sec. 4.3 depends only on the previous h, which is what lets a long
+ * sequence run in pieces and lets inference run one step at a time from a
+ * stored state (sec. 5.2).
+ */
+void oracle_s6_state(int64_t Bsz, int64_t L, int64_t D, int64_t N,
+                     const double *x, const double *delta, const double *delta_bias, int softplus,
+                     const double *A, const double *Bm, const double *Cm, const double *Dv,
+                     const double *z, int reverse, const double *initial_state, double *out,
+                     double *last_state, const int64_t *cols, int64_t ncols, int nthreads)
+{
+    s6_run(Bsz, L, D, N, x, delta, delta_bias, softplus, A, Bm, Cm, Dv, z, reverse, out,
+           last_state, initial_state, cols, ncols, nthreads, 0);
 }
 
 /*
@@ -160,9 +182,9 @@ void oracle_bidir(int64_t Bsz, int64_t L, int64_t D, int64_t N,
                   double *out, const int64_t *cols, int64_t ncols, int nthreads)
 {
     s6_run(Bsz, L, D, N, x, delta, bias_f, softplus, A_f, B_f, C_f, D_f, z_f, 0, out, last_f,
-           cols, ncols, nthreads, 0);
+           NULL, cols, ncols, nthreads, 0);
     s6_run(Bsz, L, D, N, x, delta, bias_b, softplus, A_b, B_b, C_b, D_b, z_b, 1, out, last_b,
-           cols, ncols, nthreads, 1);
+           NULL, cols, ncols, nthreads, 1);
 }
 
 /*

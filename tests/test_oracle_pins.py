@@ -307,3 +307,90 @@ def test_ssd_cols_subset():
         b = c // (P * H)
         np.testing.assert_array_equal(part[b, :, h, p], full[b, :, h, p])
         np.testing.assert_array_equal(ps[b, h, p], fs[b, h, p])
+
+
+# ------------------------------------------------ scans from a given state
+
+def _closed_form_h0(x, delta, bias, A, B, C, D, z, h0, reverse):
+    """The closed form with a state h0 before the first step: every output
+    gains sum_n C_t[n] (prod over the steps taken so far of exp(dt_k A[d,n]))
+    h0[n], the prior decayed through all steps up to and including t."""
+    Bz, L, Dm = x.shape
+    N = A.shape[1]
+    dt = _softplus(delta + bias[None, None, :])
+    y = _closed_form(x, delta, bias, A, B, C, D, None, reverse)
+    for b in range(Bz):
+        for d in range(Dm):
+            for t in range(L):
+                ks = range(0, t + 1) if not reverse else range(t, L)
+                prior = 0.0
+                for n in range(N):
+                    decay = 1.0
+                    for k in ks:
+                        decay *= math.exp(dt[b, k, d] * A[d, n])
+                    prior += C[b, t, n] * decay * h0[b, d, n]
+                y[b, t, d] += prior
+                if z is not None:
+                    y[b, t, d] *= _silu(z[b, t, d])
+    return y
+
+
+@pytest.mark.parametrize("reverse", [False, True])
+def test_initial_state_closed_form(reverse):
+    rng = np.random.default_rng(300 + reverse)
+    x, delta, bias, A, B, C, D, z = _rand_case(rng, 2, 7, 3, 4)
+    h0 = rng.standard_normal((2, 3, 4))
+    y, _ = oracle.s6_arrays(x, delta, A, B, C, delta_bias=bias, D=D, z=z, reverse=reverse,
+                            initial_state=h0)
+    _close(y, _closed_form_h0(x, delta, bias, A, B, C, D, z, h0, reverse))
+
+
+@pytest.mark.parametrize("reverse", [False, True])
+def test_initial_state_chains_pieces(reverse):
+    """Running [0, L) in one go equals running it in pieces, each piece
+    started from the state the previous piece ended with (reversed: the
+    pieces are taken from the end)."""
+    rng = np.random.default_rng(310 + reverse)
+    Bz, L, Dm, N = 2, 23, 3, 5
+    x, delta, bias, A, B, C, D, z = _rand_case(rng, Bz, L, Dm, N)
+    whole, st_whole = oracle.s6_arrays(x, delta, A, B, C, delta_bias=bias, D=D, z=z,
+                                       reverse=reverse)
+    cuts = [0, 6, 7, 15, L]
+    pieces = list(zip(cuts[:-1], cuts[1:]))
+    if reverse:
+        pieces = pieces[::-1]
+    out = np.zeros_like(whole)
+    st = None
+    for a, e in pieces:
+        sl = slice(a, e)
+        o, st = oracle.s6_arrays(x[:, sl], delta[:, sl], A, B[:, sl], C[:, sl], delta_bias=bias,
+                                 D=D, z=z[:, sl], reverse=reverse, initial_state=st)
+        out[:, sl] = o
+    _close(out, whole)
+    _close(st, st_whole)
+
+
+def test_initial_state_zero_input_decays_prior():
+    """x = 0: the state is the prior decayed step by step, h_t = exp(A sum dt) h0."""
+    rng = np.random.default_rng(320)
+    _, delta, bias, A, B, C, D, _ = _rand_case(rng, 1, 9, 2, 3, gate=False)
+    x = np.zeros((1, 9, 2))
+    h0 = rng.standard_normal((1, 2, 3))
+    _, st = oracle.s6_arrays(x, delta, A, B, C, delta_bias=bias, D=D, initial_state=h0)
+    dt_sum = _softplus(delta + bias[None, None, :]).sum(axis=1)          # (1, D)
+    _close(st, np.exp(dt_sum[:, :, None] * A[None]) * h0)
+
+
+def test_step_is_one_step_scan():
+    """The decode step equals a length-1 scan from the stored state, and L
+    steps in a row equal the scan of the L-step sequence."""
+    rng = np.random.default_rng(330)
+    Bz, L, Dm, N = 2, 5, 3, 4
+    x, delta, bias, A, B, C, D, z = _rand_case(rng, Bz, L, Dm, N)
+    whole, st_whole = oracle.s6_arrays(x, delta, A, B, C, delta_bias=bias, D=D, z=z)
+    st = np.zeros((Bz, Dm, N))
+    for t in range(L):
+        y, st = oracle.step_arrays(x[:, t], delta[:, t], A, B[:, t], C[:, t], st, delta_bias=bias,
+                                   D=D, z=z[:, t])
+        _close(y, whole[:, t])
+    _close(st, st_whole)
