@@ -123,6 +123,44 @@ SSM_API ssm_status ssm_scan_fwd(const ssm_dims *dims, const void *x, const void 
                         int reverse, void *out, float *last_state, void *workspace,
                         size_t workspace_bytes, void *stream);
 
+/*
+ * ssm_scan_fwd started from a given state.  The recurrence depends only on
+ * the previous h (Mamba2 page, sec. 4.3; sec. 5.2 for inference from a
+ * stored state), so a long sequence can run in pieces, each piece's
+ * last_state handed to the next as its initial_state.
+ *   initial_state  (B, D, N) float32 or NULL (zero): h before the first step
+ *                  (before t = 0, or before t = L-1 when reversed).  It may
+ *                  be the same buffer as last_state (updated in place).
+ * Other arguments, workspace and errors as for ssm_scan_fwd.  With L = 0 the
+ * last state is the initial state.
+ */
+SSM_API ssm_status ssm_scan_fwd_state(const ssm_dims *dims, const void *x, const void *delta,
+                                      const float *delta_bias, int delta_softplus, const float *A,
+                                      const void *B, const void *C, const float *D, const void *z,
+                                      int reverse, const float *initial_state, void *out,
+                                      float *last_state, void *workspace, size_t workspace_bytes,
+                                      void *stream);
+
+/*
+ * One decode step for every (batch, channel): the recurrent inference form
+ * of the Mamba2 page, sec. 5.2 -- the scan's step of sec. 4.3 - 4.4 applied
+ * once to a stored state:
+ *   dt = softplus(delta + bias);  state = exp(dt A) state + dt B x;
+ *   out = (C state + D x) silu(z)
+ * dims: seqlen must be 1 (SSM_ERR_UNSUPPORTED_SHAPE otherwise); batch, dim,
+ *   dstate and dtype as for ssm_scan_fwd.
+ *   x, delta, z  (B, D) dtype (z may be NULL: no gate)
+ *   B, C         (B, N) dtype
+ *   A (D, N), delta_bias (D) or NULL, D (D) or NULL: float32
+ *   state        (B, D, N) float32, read and written in place
+ *   out          (B, D) dtype, written
+ * No workspace.  All pointers 16-byte aligned; asynchronous on stream.
+ */
+SSM_API ssm_status ssm_step(const ssm_dims *dims, const void *x, const void *delta,
+                            const float *delta_bias, int delta_softplus, const float *A,
+                            const void *B, const void *C, const float *D, const void *z,
+                            float *state, void *out, void *stream);
+
 /* Bytes of the scratch array that ssm_scan_fwd_noalloc draws from. */
 #define SSM_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
 

@@ -8,6 +8,8 @@ raises -- there is no fallback path.
 Entry points (names as in include/ssm.h):
 
 * ``ssm_scan_fwd(x, delta, A, B, C, ...)``  single-direction S6 scan
+* ``ssm_scan_fwd_state(...)``  the same from a given initial state
+* ``ssm_step(x, delta, A, B, C, state, ...)``  one decode step, state in place
 * ``bidir_scan_fwd(x, delta, fwd, bwd, ...)``  Vision-Mamba bidirectional scan
 * ``ssd_chunk_fwd(x, delta, A, B, C, ...)``  Mamba2 SSD chunked scan
 
@@ -64,6 +66,10 @@ SIGNATURES = {
     "ssm_scan_workspace_size": (_sz, [ctypes.POINTER(ssm_dims)]),
     "ssm_scan_fwd": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp, _vp,
                             _int, _vp, _vp, _vp, _sz, _vp]),
+    "ssm_scan_fwd_state": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp,
+                                  _vp, _int, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "ssm_step": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp, _vp, _vp,
+                        _vp, _vp]),
     "ssm_scan_fwd_noalloc": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp,
                                     _vp, _int, _vp, _vp, _vp]),
     "bidir_scan_workspace_size": (_sz, [ctypes.POINTER(ssm_dims)]),
@@ -186,6 +192,45 @@ def ssm_scan_fwd(x, delta, A, B, C, *, delta_bias=None, delta_softplus=True, D=N
                           int(bool(reverse)), _ptr(out), _ptr(last_state), _ptr(ws),
                           0 if ws is None else ws.numel(), _stream_handle(stream))
     _check(st, "ssm_scan_fwd")
+    return out
+
+
+def ssm_scan_fwd_state(x, delta, A, B, C, *, initial_state=None, delta_bias=None,
+                       delta_softplus=True, D=None, z=None, reverse=False, out=None,
+                       last_state=None, ws=None, stream=None):
+    """ssm_scan_fwd from a given state (initial_state (B, D, N) float32, None
+    for zero); last_state may be the same tensor as initial_state."""
+    torch = _torch()
+    lib = capi()
+    dims = s6_dims(x, A.shape[1])
+    if out is None:
+        out = torch.empty_like(x)
+    need = lib.ssm_scan_workspace_size(ctypes.byref(dims))
+    if ws is None:
+        ws = workspace(need, x.device)
+    st = lib.ssm_scan_fwd_state(ctypes.byref(dims), _ptr(x), _ptr(delta), _ptr(delta_bias),
+                                int(bool(delta_softplus)), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                _ptr(z), int(bool(reverse)), _ptr(initial_state), _ptr(out),
+                                _ptr(last_state), _ptr(ws), 0 if ws is None else ws.numel(),
+                                _stream_handle(stream))
+    _check(st, "ssm_scan_fwd_state")
+    return out
+
+
+def ssm_step(x, delta, A, B, C, state, *, delta_bias=None, delta_softplus=True, D=None, z=None,
+             out=None, stream=None):
+    """One decode step: x, delta, z (B, D); B, C (B, N); state (B, D, N)
+    float32 updated in place.  Returns out (B, D) in x's dtype."""
+    torch = _torch()
+    lib = capi()
+    Bz, Dm = x.shape
+    dims = ssm_dims(Bz, 1, Dm, A.shape[1], _dtype_code(x))
+    if out is None:
+        out = torch.empty_like(x)
+    st = lib.ssm_step(ctypes.byref(dims), _ptr(x), _ptr(delta), _ptr(delta_bias),
+                      int(bool(delta_softplus)), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+                      _ptr(state), _ptr(out), _stream_handle(stream))
+    _check(st, "ssm_step")
     return out
 
 

@@ -17,6 +17,7 @@ struct DirArgs {
     const float *D;      // (D) or nullptr
     const void *z;       // (Bsz, L, D) or nullptr
     float *last_state;   // (Bsz, D, N) or nullptr
+    const float *init;   // (Bsz, D, N) state before the first step, or nullptr (zero)
 };
 
 // One S6 call (single direction or bidirectional).
@@ -24,8 +25,10 @@ struct DirArgs {
 // The sequence is cut into S segments of T steps (the last one may be
 // shorter).  With S > 1 every segment first summarises itself (local end
 // state from a zero start plus the sum of dt), a carry pass composes those
-// summaries in scan order, and the main pass then rescans each segment from
-// its true entering state.  carry_h / carry_s are the caller's workspace.
+// summaries in scan order, starting from the direction's initial state, and
+// the main pass then rescans each segment from its true entering state.
+// carry_h / carry_s are the caller's workspace.  With S > 1 only the carry
+// pass reads the initial state, so it may share a buffer with last_state.
 struct S6Args {
     int Bsz, L, D, N;
     int S, T;
@@ -57,6 +60,18 @@ struct S6Plan {
 S6Plan plan_s6(int64_t Bsz, int64_t L, int64_t D, int64_t N, int ndir, int dtype);
 
 cudaError_t launch_s6(const S6Args &a, cudaStream_t stream);
+
+// One decode step of S6 for every (batch, channel), state updated in place.
+struct StepArgs {
+    int Bsz, D, N;
+    int dtype;     // 0 = float32, 1 = bf16
+    int softplus;
+    const void *x, *delta, *B, *C, *z;   // x, delta, z (Bsz, D); B, C (Bsz, N)
+    const float *bias, *A, *Dskip;       // (D), (D, N), (D)
+    float *state;                        // (Bsz, D, N) in and out
+    void *out;                           // (Bsz, D)
+};
+cudaError_t launch_step(const StepArgs &a, cudaStream_t stream);
 
 // One SSD call.
 struct SSDArgs {

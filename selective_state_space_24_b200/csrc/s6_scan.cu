@@ -45,11 +45,11 @@
 #include <stdint.h>
 
 #include "internal.h"
+#include "s6_math.cuh"
 
 namespace ssm {
 namespace {
 
-constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kWarps = 2;   // warps per CTA
 constexpr int kTC = 16;     // steps per B/C staging chunk
 // cp.async ring: steps per group and groups in flight, by channels per lane
@@ -104,20 +104,6 @@ template <int CPL> constexpr int min_blocks() { return CPL == 2 ? SSM_S6_MINB : 
 
 // ------------------------------------------------------------ math helpers
 
-__device__ __forceinline__ float ex2_mufu(float v)
-{
-    float r;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
-    return r;
-}
-
-__device__ __forceinline__ float rcp_mufu(float v)
-{
-    float r;
-    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
-    return r;
-}
-
 // Pairwise multiply / fused multiply-add on two states at once: the packed
 // f32x2 instructions of sm_100, or two scalar instructions (SSM_S6_SCALAR).
 #ifndef SSM_S6_SCALAR
@@ -162,37 +148,6 @@ __device__ __forceinline__ float2 ex2_poly2(float2 v)
     p = __ffma2_rn(p, f, make_float2(1.000000119e+00f, 1.000000119e+00f));
     return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
                        __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
-}
-
-// softplus(v) = max(v, 0) + log1p(e), e = exp(-|v|) in (0, 1], with
-// log1p(e) = e q(e) and q a degree-7 minimax polynomial for log1p(e) / e on
-// [0, 1] (relative error 3.4e-7 in fp32; coefficients from fit_polys.py).
-__device__ __forceinline__ float softplus_f(float v)
-{
-    const float e = ex2_mufu(-fabsf(v) * kLog2e);
-    float q = -8.539208211e-03f;
-    q = fmaf(q, e, 4.408963397e-02f);
-    q = fmaf(q, e, -1.076817140e-01f);
-    q = fmaf(q, e, 1.774524152e-01f);
-    q = fmaf(q, e, -2.449546307e-01f);
-    q = fmaf(q, e, 3.327547908e-01f);
-    q = fmaf(q, e, -4.999740422e-01f);
-    q = fmaf(q, e, 9.999998212e-01f);
-    return fmaf(e, q, fmaxf(v, 0.f));
-}
-
-// silu(z) = z sigmoid(z).  fp32 data: z / (1 + 2^(-z log2 e)) with the MUFU
-// reciprocal.  bf16 data: z (1 + tanh(z / 2)) / 2 with the single MUFU
-// tanh.approx (relative error 2^-11, below the bf16 output rounding).
-template <typename T>
-__device__ __forceinline__ float silu_f(float z)
-{
-    if (sizeof(T) == 2) {
-        float t;
-        asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * z));
-        return 0.5f * z * (1.f + t);
-    }
-    return z * rcp_mufu(1.f + ex2_mufu(-z * kLog2e));
 }
 
 // ----------------------------------------------------- storage-type helpers
@@ -658,7 +613,8 @@ __global__ void __launch_bounds__(64, min_blocks<CPL>()) s6_summary_kernel(const
 }
 
 // ------------------------------------------------------------------ carry
-// Per (direction, b, d, n): walk the segments in scan order, replace each
+// Per (direction, b, d, n): walk the segments in scan order from the initial
+// state (or zero), replace each
 // summary by the state entering that segment.  Summaries are fetched 16
 // segments at a time ahead of the dependent chain.
 __global__ void s6_carry_kernel(const S6Args a)
@@ -675,7 +631,8 @@ __global__ void s6_carry_kernel(const S6Args a)
     const float Al2 = a.dir[dsel].A[(size_t)d * a.N + n] * kLog2e;
     const size_t cbase = ((size_t)dsel * a.Bsz + b) * a.S;   // segment index base
     constexpr int kBatch = 16;
-    float hin = 0.f;
+    const float *init = a.dir[dsel].init;
+    float hin = init ? init[((size_t)b * a.D + d) * a.N + n] : 0.f;
     for (int k0 = 0; k0 < a.S; k0 += kBatch) {
         float hl[kBatch], sd[kBatch];
 #pragma unroll
@@ -722,15 +679,21 @@ __global__ void __launch_bounds__(64, min_blocks<CPL>()) s6_main_kernel(const S6
         return;   // whole warp past the channels (never with a barrier partner)
     float2 h[CPL][NS / 2];
     float sdt[CPL];
-    const bool has_carry = a.S > 1 && !first_in_order(seg, a.S, rev);
+    // the entering state: with segments, the carry pass wrote it for every
+    // segment (the first one's is the initial state); otherwise the initial
+    // state itself, or zero
+    const bool has_carry = a.S > 1;
+    const float *init = P.init;
 #pragma unroll
     for (int c = 0; c < CPL; c++) {
         sdt[c] = 0.f;
         const size_t ci = (((size_t)dsel * a.Bsz + b) * a.S + seg) * a.D + d + c;
 #pragma unroll
         for (int k = 0; k < NS / 2; k++) {
-            h[c][k].x = (active && has_carry && 2 * k < a.N) ? a.carry_h[ci * a.N + 2 * k] : 0.f;
-            h[c][k].y = (active && has_carry && 2 * k + 1 < a.N) ? a.carry_h[ci * a.N + 2 * k + 1] : 0.f;
+            const float *src = has_carry ? a.carry_h + ci * a.N
+                                         : (init ? init + ((size_t)b * a.D + d + c) * a.N : nullptr);
+            h[c][k].x = (active && src && 2 * k < a.N) ? src[2 * k] : 0.f;
+            h[c][k].y = (active && src && 2 * k + 1 < a.N) ? src[2 * k + 1] : 0.f;
         }
     }
     scan_segment<T, NS, CPL, NPOLY, false, BIDIR, GATE, SOFTPLUS>(a, P, sm[warp], b, dbase, active,

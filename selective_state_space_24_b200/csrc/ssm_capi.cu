@@ -64,7 +64,7 @@ ssm::DirArgs dir_args(const ssm_dir_params &p)
 
 ssm_status run_s6(const ssm_dims *dims, const void *x, const void *delta, int softplus, int ndir,
                   int reverse, const ssm_dir_params *dirs, void *out, void *ws, size_t ws_bytes,
-                  cudaStream_t stream)
+                  cudaStream_t stream, const float *initial_state = nullptr)
 {
     const int dt = dims->dtype == SSM_F32 ? 0 : 1;
     const ssm::S6Plan plan =
@@ -92,6 +92,7 @@ ssm_status run_s6(const ssm_dims *dims, const void *x, const void *delta, int so
     a.delta = delta;
     for (int i = 0; i < ndir; i++)
         a.dir[i] = dir_args(dirs[i]);
+    a.dir[0].init = initial_state;   // single direction only
     a.out = out;
     char *w = static_cast<char *>(ws);
     if (plan.S > 1) {
@@ -140,19 +141,29 @@ ssm_status ssm_scan_plan(const ssm_dims *dims, int bidirectional, int *segments,
     return SSM_OK;
 }
 
-ssm_status ssm_scan_fwd(const ssm_dims *dims, const void *x, const void *delta,
-                        const float *delta_bias, int delta_softplus, const float *A,
-                        const void *B, const void *C, const float *D, const void *z, int reverse,
-                        void *out, float *last_state, void *workspace, size_t workspace_bytes,
-                        void *stream)
+ssm_status ssm_scan_fwd_state(const ssm_dims *dims, const void *x, const void *delta,
+                              const float *delta_bias, int delta_softplus, const float *A,
+                              const void *B, const void *C, const float *D, const void *z,
+                              int reverse, const float *initial_state, void *out, float *last_state,
+                              void *workspace, size_t workspace_bytes, void *stream)
 {
     ssm_status s = check_s6_dims(dims);
     if (s != SSM_OK)
         return s;
+    if ((initial_state && !aligned16(initial_state)) || (last_state && !aligned16(last_state)))
+        return SSM_ERR_MISALIGNED;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (empty_s6(dims)) {
-        if (last_state && !aligned16(last_state))
-            return SSM_ERR_MISALIGNED;
+        // no step taken: the last state is the initial state (or zero)
+        const size_t n = (size_t)dims->batch * dims->dim * dims->dstate;
+        if (last_state && initial_state && dims->seqlen == 0 && n > 0) {
+            if (last_state == initial_state)
+                return SSM_OK;
+            return cudaMemcpyAsync(last_state, initial_state, n * sizeof(float), cudaMemcpyDeviceToDevice,
+                                   st) == cudaSuccess
+                       ? SSM_OK
+                       : SSM_ERR_CUDA;
+        }
         return zero_state(last_state, dims, st);
     }
     if (!x || !delta || !out)
@@ -162,7 +173,54 @@ ssm_status ssm_scan_fwd(const ssm_dims *dims, const void *x, const void *delta,
         return s;
     if (!aligned16(x) || !aligned16(delta) || !aligned16(out))
         return SSM_ERR_MISALIGNED;
-    return run_s6(dims, x, delta, delta_softplus, 1, reverse, &p, out, workspace, workspace_bytes, st);
+    return run_s6(dims, x, delta, delta_softplus, 1, reverse, &p, out, workspace, workspace_bytes, st,
+                  initial_state);
+}
+
+ssm_status ssm_scan_fwd(const ssm_dims *dims, const void *x, const void *delta,
+                        const float *delta_bias, int delta_softplus, const float *A,
+                        const void *B, const void *C, const float *D, const void *z, int reverse,
+                        void *out, float *last_state, void *workspace, size_t workspace_bytes,
+                        void *stream)
+{
+    return ssm_scan_fwd_state(dims, x, delta, delta_bias, delta_softplus, A, B, C, D, z, reverse, nullptr,
+                              out, last_state, workspace, workspace_bytes, stream);
+}
+
+ssm_status ssm_step(const ssm_dims *dims, const void *x, const void *delta, const float *delta_bias,
+                    int delta_softplus, const float *A, const void *B, const void *C, const float *D,
+                    const void *z, float *state, void *out, void *stream)
+{
+    ssm_status s = check_s6_dims(dims);
+    if (s != SSM_OK)
+        return s;
+    if (dims->seqlen != 1)
+        return SSM_ERR_UNSUPPORTED_SHAPE;
+    if (dims->batch == 0 || dims->dim == 0)
+        return SSM_OK;
+    if (!x || !delta || !A || !B || !C || !state || !out)
+        return SSM_ERR_INVALID_ARG;
+    const void *ptrs[] = {x, delta, delta_bias, A, B, C, D, z, state, out};
+    for (const void *q : ptrs)
+        if (q && !aligned16(q))
+            return SSM_ERR_MISALIGNED;
+    ssm::StepArgs a;
+    a.Bsz = (int)dims->batch;
+    a.D = (int)dims->dim;
+    a.N = (int)dims->dstate;
+    a.dtype = dims->dtype == SSM_F32 ? 0 : 1;
+    a.softplus = delta_softplus ? 1 : 0;
+    a.x = x;
+    a.delta = delta;
+    a.B = B;
+    a.C = C;
+    a.z = z;
+    a.bias = delta_bias;
+    a.A = A;
+    a.Dskip = D;
+    a.state = state;
+    a.out = out;
+    return ssm::launch_step(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
 ssm_status bidir_scan_fwd(const ssm_dims *dims, const void *x, const void *delta,

@@ -147,3 +147,25 @@ def test_scan_plan(lib):
     with pytest.raises(ssm.SSMError):
         ssm.scan_plan(1, 10, 30, 16)                 # D not a multiple of 4
     assert lib.ssm_scan_plan(None, 0, None, None) == 1
+
+
+def test_state_and_step_validation(lib):
+    """ssm_scan_fwd_state and ssm_step reject bad arguments before launching."""
+    dims = _dims(2, 8, 16, 16)
+    # misaligned initial state
+    st = lib.ssm_scan_fwd_state(ctypes.byref(dims), FAKE, FAKE, None, 1, FAKE, FAKE, FAKE, None, None,
+                                0, FAKE + 4, FAKE, None, None, 0, None)
+    assert st == 3
+    # a step is one time step
+    st = lib.ssm_step(ctypes.byref(dims), FAKE, FAKE, None, 1, FAKE, FAKE, FAKE, None, None, FAKE,
+                      FAKE, None)
+    assert st == 2
+    one = _dims(2, 1, 16, 16)
+    assert lib.ssm_step(ctypes.byref(one), FAKE, FAKE, None, 1, FAKE, FAKE, FAKE, None, None, None,
+                        FAKE, None) == 1          # no state
+    assert lib.ssm_step(ctypes.byref(one), FAKE, FAKE, None, 1, FAKE, FAKE, FAKE, None, None, FAKE,
+                        FAKE + 8, None) == 3      # misaligned out
+    assert lib.ssm_step(None, FAKE, FAKE, None, 1, FAKE, FAKE, FAKE, None, None, FAKE, FAKE, None) == 1
+    empty = _dims(0, 1, 16, 16)
+    assert lib.ssm_step(ctypes.byref(empty), None, None, None, 1, None, None, None, None, None, None,
+                        None, None) == 0
