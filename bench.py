@@ -48,7 +48,7 @@ SMS = 148
 # DRAM bytes (read + write) per launch of the dominant kernel, from one ncu
 # capture of the current kernels (profiles/s6_main_vim_small_bidir_fp32.md,
 # profiles/ssd_chunk_mamba2_bf16.md); None where no capture matches them.
-NCU_TRAFFIC = {1: 273.28e6, 4: 397.21e6}
+NCU_TRAFFIC = {1: 273.17e6, 4: 398.97e6}
 
 
 def parse():
@@ -60,6 +60,9 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--op", default="scan", choices=["scan", "step"],
+                   help="scan: the workload's scan (default); step: one decode step of a "
+                        "batch-512 x 1536-channel x 16-state fp32 state (ssm_step)")
     return p.parse_args()
 
 
@@ -385,6 +388,80 @@ def run_ours(args, rank, world, local_rank):
     return res
 
 
+# ------------------------------------------------------- decode step
+
+STEP_WORKLOAD = {"batch": 512, "dim": 1536, "dstate": 16}
+
+
+def run_step(args):
+    """One decode step (ssm_step) of a (512, 1536, 16) fp32 state with fp32
+    activations, timed like the scan: inputs resident, L2 flushed before
+    every step, CUDA events on the launching stream.  HBM-bound: the state
+    is read and written once."""
+    import ctypes
+    import torch
+    from selective_state_space_24_b200 import build as ssm_build
+    import selective_state_space_24_b200 as ssm
+    ssm_build.build()
+    lib = ssm.load()
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    Bz, Dm, N = STEP_WORKLOAD["batch"], STEP_WORKLOAD["dim"], STEP_WORKLOAD["dstate"]
+    inp = ssm_gen.make_s6_inputs(Bz, 1, Dm, N, dtype="f32", seed=0)
+    f = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device)
+    x, delta, z = f(inp.x[:, 0]), f(inp.delta[:, 0]), f(inp.z_f[:, 0])
+    Bm, Cm = f(inp.B_f[:, 0]), f(inp.C_f[:, 0])
+    A, bias, Dv = f(inp.A_f), f(inp.dt_bias_f), f(inp.D_f)
+    state = torch.zeros((Bz, Dm, N), device=device)
+    out = torch.empty_like(x)
+    dims = ssm.ssm_dims(Bz, 1, Dm, N, ssm.SSM_F32)
+    p = lambda t: t.data_ptr()
+    stream = torch.cuda.current_stream(device)
+    sh = stream.cuda_stream
+
+    def step():
+        st = lib.ssm_step(ctypes.byref(dims), p(x), p(delta), p(bias), 1, p(A), p(Bm), p(Cm), p(Dv),
+                          p(z), p(state), p(out), sh)
+        if st != 0:
+            raise RuntimeError(f"ssm_step returned {ssm.STATUS.get(st, st)}")
+
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    for _ in range(max(args.warmup, 3)):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    sampler = ClockSampler(0)
+    sampler.start()
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = [a.elapsed_time(b) for a, b in evs]
+    med = statistics.median(ms)
+    elems = Bz * Dm * N
+    nbytes = 2 * elems * 4 + 4 * Bz * Dm * 4 + 2 * Bz * N * 4 + Dm * N * 4 + 2 * Dm * 4
+    peaks, peak_src = load_peaks()
+    hbm = nbytes / (med * 1e-3) / 1e9
+    return {
+        "metric": "decode step: state elements/s (B·D·N) and HBM GB/s", "value": elems / (med * 1e-3),
+        "unit": "elements/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": sum(ms) / len(ms), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded ssm_gen inputs)",
+        "config": {"workload": "decode_step_b512_d1536_n16_fp32", **STEP_WORKLOAD,
+                   "l2": "flushed before every timed step (512 MB write)",
+                   "algorithmic_bytes_per_step": nbytes},
+        "roofline": {"bound": "hbm", "achieved": hbm, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": hbm / peaks["hbm_gbs"], "traffic": None, "peak_source": peak_src,
+                     "kernel_ms_median": med},
+        "gpu_launches": args.steps, "clocks": clocks,
+    }
+
+
 # ------------------------------------------------------------ CPU oracle
 
 def _oracle_sample(cfg, frac_cols):
@@ -481,6 +558,10 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
+        return
+    if args.op == "step":
+        if rank == 0:
+            print(json.dumps(run_step(args)), flush=True)
         return
     if world > 1:
         import datetime

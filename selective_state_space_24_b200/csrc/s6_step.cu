@@ -6,10 +6,9 @@
 //     dt = softplus(delta + bias),  h = exp(dt A) h + dt B x,
 //     y  = (C h + D x) silu(z).
 //
-// One thread per (b, d) keeps the N <= 16 states of its row in registers.
-// The state is the only large operand (B D N float32 read and written once),
-// so the kernel is HBM-bound: consecutive threads own consecutive rows, and
-// a row is read and written as 16-byte vectors when N is a multiple of 4.
+// The state is the only large operand (B D N float32 read and written
+// once), so the kernel is HBM-bound; four lanes share one (b, d) row, each
+// holding a quarter of its N <= 16 states in registers.
 // The transcendentals take the same forms as in the scan kernels
 // (s6_math.cuh), with A scaled by log2(e) before the product with dt.
 #include <cuda_bf16.h>
@@ -31,76 +30,98 @@ template <> __device__ __forceinline__ float ldv<__nv_bfloat16>(const __nv_bfloa
 __device__ __forceinline__ void stv(float *p, size_t i, float v) { p[i] = v; }
 __device__ __forceinline__ void stv(__nv_bfloat16 *p, size_t i, float v) { p[i] = __float2bfloat16_rn(v); }
 
+// Four lanes share one (b, d) row: lane part p owns states [p K, p K + K),
+// K = NS / 4, so a warp's state loads and stores cover 8 whole rows
+// (8 x 4 N bytes) contiguously.  The readout is summed over the four lanes
+// with two shuffles.
 template <typename T, int NS, bool VEC>
 __global__ void __launch_bounds__(256) s6_step_kernel(const StepArgs a)
 {
-    const size_t row = (size_t)blockIdx.x * blockDim.x + threadIdx.x;   // b * D + d
-    if (row >= (size_t)a.Bsz * a.D)
-        return;
+    constexpr int K = NS / 4;
+    const size_t tid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const size_t row = tid >> 2;   // b * D + d
+    const int part = (int)(tid & 3);
+    const bool live = row < (size_t)a.Bsz * a.D;   // whole groups of 4 agree
     const int N = a.N;
-    const int d = (int)(row % a.D);
-    const size_t b = row / a.D;
+    const int d = live ? (int)(row % a.D) : 0;
+    const size_t b = live ? row / a.D : 0;
     const T *x = static_cast<const T *>(a.x), *dl = static_cast<const T *>(a.delta);
     const T *Bm = static_cast<const T *>(a.B), *Cm = static_cast<const T *>(a.C);
     const T *z = static_cast<const T *>(a.z);
 
-    const float xv = ldv(x, row);
-    float dt = ldv(dl, row) + (a.bias ? a.bias[d] : 0.f);
-    if (a.softplus)
-        dt = softplus_f(dt);
-    const float dtx = dt * xv;
-
-    float h[NS], Av[NS];
-    float *st = a.state + row * N;
-    const float *Ar = a.A + (size_t)d * N;
-    if (VEC) {   // N == NS, a multiple of 4: 16-byte rows
+    float y = 0.f, xv = 0.f;
+    if (live) {
+        xv = ldv(x, row);
+        float dt = ldv(dl, row) + (a.bias ? a.bias[d] : 0.f);
+        if (a.softplus)
+            dt = softplus_f(dt);
+        const float dtx = dt * xv;
+        float h[K], Av[K];
+        float *st = a.state + row * N + part * K;
+        const float *Ar = a.A + (size_t)d * N + part * K;
+        if (VEC) {   // N == NS: this lane's K states are one aligned vector
+            if (K == 4) {
+                const float4 hv = *reinterpret_cast<const float4 *>(st);
+                const float4 av = __ldg(reinterpret_cast<const float4 *>(Ar));
+                h[0] = hv.x, h[1] = hv.y, h[2] = hv.z, h[3] = hv.w;
+                Av[0] = av.x, Av[1] = av.y, Av[2] = av.z, Av[3] = av.w;
+            } else if (K == 2) {
+                const float2 hv = *reinterpret_cast<const float2 *>(st);
+                const float2 av = __ldg(reinterpret_cast<const float2 *>(Ar));
+                h[0] = hv.x, h[1] = hv.y;
+                Av[0] = av.x, Av[1] = av.y;
+            } else {
+                h[0] = st[0];
+                Av[0] = __ldg(Ar);
+            }
+        } else {
 #pragma unroll
-        for (int q = 0; q < NS / 4; q++) {
-            const float4 hv = reinterpret_cast<const float4 *>(st)[q];
-            const float4 av = __ldg(reinterpret_cast<const float4 *>(Ar) + q);
-            h[4 * q] = hv.x, h[4 * q + 1] = hv.y, h[4 * q + 2] = hv.z, h[4 * q + 3] = hv.w;
-            Av[4 * q] = av.x * kLog2e, Av[4 * q + 1] = av.y * kLog2e;
-            Av[4 * q + 2] = av.z * kLog2e, Av[4 * q + 3] = av.w * kLog2e;
+            for (int k = 0; k < K; k++) {
+                const bool in = part * K + k < N;
+                h[k] = in ? st[k] : 0.f;
+                Av[k] = in ? Ar[k] : 0.f;
+            }
         }
-    } else {
 #pragma unroll
-        for (int n = 0; n < NS; n++) {
-            h[n] = n < N ? st[n] : 0.f;
-            Av[n] = n < N ? Ar[n] * kLog2e : 0.f;
+        for (int k = 0; k < K; k++) {
+            const int n = part * K + k;
+            if (VEC || n < N) {
+                const float e = ex2_mufu(dt * (Av[k] * kLog2e));
+                h[k] = fmaf(e, h[k], dtx * ldv(Bm, b * N + n));
+                y = fmaf(ldv(Cm, b * N + n), h[k], y);
+            }
+        }
+        if (VEC) {
+            if (K == 4)
+                *reinterpret_cast<float4 *>(st) = make_float4(h[0], h[1], h[2], h[3]);
+            else if (K == 2)
+                *reinterpret_cast<float2 *>(st) = make_float2(h[0], h[1]);
+            else
+                st[0] = h[0];
+        } else {
+#pragma unroll
+            for (int k = 0; k < K; k++)
+                if (part * K + k < N)
+                    st[k] = h[k];
         }
     }
-    float y = 0.f;
-#pragma unroll
-    for (int n = 0; n < NS; n++) {
-        if (n < N) {
-            const float e = ex2_mufu(dt * Av[n]);
-            h[n] = fmaf(e, h[n], dtx * ldv(Bm, b * N + n));
-            y = fmaf(ldv(Cm, b * N + n), h[n], y);
-        }
+    y += __shfl_xor_sync(0xffffffffu, y, 1);
+    y += __shfl_xor_sync(0xffffffffu, y, 2);
+    if (live && part == 0) {
+        if (a.Dskip)
+            y = fmaf(a.Dskip[d], xv, y);
+        if (z)
+            y *= silu_f<T>(ldv(z, row));
+        stv(static_cast<T *>(a.out), row, y);
     }
-    if (VEC) {
-#pragma unroll
-        for (int q = 0; q < NS / 4; q++)
-            reinterpret_cast<float4 *>(st)[q] = make_float4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
-    } else {
-#pragma unroll
-        for (int n = 0; n < NS; n++)
-            if (n < N)
-                st[n] = h[n];
-    }
-    if (a.Dskip)
-        y = fmaf(a.Dskip[d], xv, y);
-    if (z)
-        y *= silu_f<T>(ldv(z, row));
-    stv(static_cast<T *>(a.out), row, y);
 }
 
 template <typename T, int NS>
 cudaError_t launch_ns(const StepArgs &a, cudaStream_t st)
 {
-    const size_t rows = (size_t)a.Bsz * a.D;
-    const unsigned grid = (unsigned)((rows + 255) / 256);
-    if (a.N == NS && NS % 4 == 0)
+    const size_t threads = (size_t)a.Bsz * a.D * 4;
+    const unsigned grid = (unsigned)((threads + 255) / 256);
+    if (a.N == NS)
         s6_step_kernel<T, NS, true><<<grid, 256, 0, st>>>(a);
     else
         s6_step_kernel<T, NS, false><<<grid, 256, 0, st>>>(a);
