@@ -38,7 +38,7 @@
 //   * exp(dt A) is 2^(dt A log2 e).  The first NS - NPOLY states use the MUFU
 //     ex2.approx instruction, the last NPOLY states a degree-5 polynomial on
 //     the FMA pipe (integer / fraction split of the exponent, minimax
-//     coefficients fitted by fit_exp2_poly.py), so that the MUFU and FMA
+//     coefficients fitted by fit_polys.py), so that the MUFU and FMA
 //     pipes share the work.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>

@@ -27,10 +27,13 @@
 // warpgroups of math threads -- warpgroup g owns columns [16 g, 16 g + 16) of
 // every 64-wide row --, one warp whose lane 0 issues the tensor-core MMAs
 // when the math threads signal (mbarriers) that the operands are written, and
-// one warp that computes dt and its cumulative sum up to three chunks ahead.
-// The loop is software-pipelined: while the math threads build chunk c's
-// decay matrix, update the state and write chunk c's outputs, the tensor core
-// runs chunk c + 1's first products (W and the Yo accumulator are
+// one warp that issues the TMA loads and computes dt and its cumulative sum
+// up to three chunks ahead.  Per chunk c the math threads build the decay
+// matrix M(c) as soon as G(c) is done (G has its own commit), then the next
+// chunk's W(c + 1) while the tensor core finishes Yo(c), dS(c) and Yd(c),
+// then update the state and write S_in(c + 1), then chunk c's outputs; the
+// MMA warp issues Yd(c) once M(c) is written and chunk c + 1's G, Yo and dS
+// once W(c + 1) and S_in(c + 1) are (W and the Yo accumulator are
 // double-buffered by chunk parity, dt / cs triple-buffered).  The hi and lo
 // halves of S_in and of W sit side by side as one N = 128 operand, so each
 // of those products is one MMA per K-step.  TMA brings each chunk's X, Z
