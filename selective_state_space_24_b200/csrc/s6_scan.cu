@@ -79,14 +79,17 @@ template <int CPL> struct Ring {
 #define SSM_S6_MINB1 8
 #endif
 // Tuning knobs (compile-time): channels per lane (0 = by problem size), the
-// thread count below which one channel per lane is used, the target thread
-// counts that decide the number of segments, and how many state pairs the
-// summary pass evaluates on the FMA pipe.
+// thread count below which one channel per lane is used, the waves of
+// resident CTAs the segments fill (0: use the target thread counts instead),
+// and how many state pairs the summary pass evaluates on the FMA pipe.
 #ifndef SSM_S6_CPL
 #define SSM_S6_CPL 0
 #endif
 #ifndef SSM_S6_CPL1_BELOW
 #define SSM_S6_CPL1_BELOW (148 * 128)
+#endif
+#ifndef SSM_S6_WAVES
+#define SSM_S6_WAVES 1
 #endif
 #ifndef SSM_S6_TARGET1
 #define SSM_S6_TARGET1 (148 * 640)
@@ -794,11 +797,22 @@ S6Plan plan_s6(int64_t Bsz, int64_t L, int64_t D, int64_t N, int ndir, int dtype
     const int64_t lanes2 = (int64_t)ndir * Bsz * ((D + 1) / 2);
     p.cpl = SSM_S6_CPL != 0 ? SSM_S6_CPL : (lanes2 < SSM_S6_CPL1_BELOW ? 1 : 2);
     const int64_t kMinT = 16;
-    const int64_t kTargetThreads = p.cpl == 1 ? SSM_S6_TARGET1 : SSM_S6_TARGET2;
-    const int64_t threads = (int64_t)ndir * Bsz * ((D + p.cpl - 1) / p.cpl);
     int64_t S = 1;
-    if (threads > 0 && threads < kTargetThreads)
-        S = (kTargetThreads + threads - 1) / threads;
+    if (SSM_S6_WAVES > 0) {
+        // Segments: as many as fill SSM_S6_WAVES waves of the main kernel's
+        // resident CTAs (148 SMs x CTAs per SM for this lane mapping) -- a
+        // CTA count just past a wave boundary costs a whole extra wave.
+        const int64_t ch_per_cta = (ndir == 2 ? 32 : 64) * p.cpl;
+        const int64_t ctas_per_seg = (D + ch_per_cta - 1) / ch_per_cta * Bsz;
+        const int64_t slots = (int64_t)148 * (p.cpl == 2 ? SSM_S6_MINB : SSM_S6_MINB1) * SSM_S6_WAVES;
+        if (ctas_per_seg > 0)
+            S = slots / ctas_per_seg;
+    } else {
+        const int64_t kTargetThreads = p.cpl == 1 ? SSM_S6_TARGET1 : SSM_S6_TARGET2;
+        const int64_t threads = (int64_t)ndir * Bsz * ((D + p.cpl - 1) / p.cpl);
+        if (threads > 0 && threads < kTargetThreads)
+            S = (kTargetThreads + threads - 1) / threads;
+    }
     const int64_t smax = (L + kMinT - 1) / kMinT;
     if (S > smax)
         S = smax;
