@@ -56,6 +56,9 @@ def _load():
                                                ctypes.c_int, _dp, _dp, _ip, _i64, ctypes.c_int]
         lib.oracle_s6_state.argtypes = ([_i64] * 4 + [_dp, _dp, _dp, ctypes.c_int, _dp, _dp, _dp, _dp, _dp,
                                          ctypes.c_int, _dp, _dp, _dp, _dp, _i64, ctypes.c_int])
+        lib.oracle_s6_masked.argtypes = ([_i64] * 4 + [_dp, _dp, _dp, ctypes.c_int, _dp, _dp, _dp, _dp, _dp,
+                                          ctypes.c_int, ctypes.c_void_p, _dp, _dp, _ip, _i64,
+                                          ctypes.c_int])
         lib.oracle_bidir.argtypes = ([_i64] * 4 + [_dp, _dp, ctypes.c_int] + [_dp] * 7 + [_dp] * 7
                                      + [_dp, _ip, _i64, ctypes.c_int])
         lib.oracle_ssd_seq.argtypes = [_i64] * 5 + [_dp, _dp, _dp, ctypes.c_int, _dp, _dp, _dp, _dp,
@@ -111,6 +114,58 @@ def s6_arrays(x, delta, A, B, C, *, delta_bias=None, softplus=True, D=None, z=No
                                 int(softplus), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
                                 int(reverse), _ptr(h0), _ptr(out), _ptr(st), cp, nc, int(nthreads))
     return out, st
+
+
+def s6_ordered_arrays(x, delta, A, B, C, *, order=None, mask=None, delta_bias=None, softplus=True,
+                      D=None, z=None, reverse=False, cols=None, nthreads=1
+                      ) -> Tuple[np.ndarray, np.ndarray]:
+    """Single-direction S6 along a given order of the L positions, with an
+    optional token mask.
+
+    order (L,): a permutation of 0..L-1; step i visits position order[i]
+    (reversed: order[L-1-i]) -- the row, column, cross and spiral scans of
+    the Samba (sec. 3.1) and Mamba-YOLO (sec. 1.2, 4.4) pages.  mask (B, L),
+    indexed by position: 0 bypasses the token (Samba page, sec. 2) -- the
+    state passes through unchanged and its output is 0.
+    Defined as the scan of the inputs gathered in that order, outputs
+    scattered back to their positions."""
+    x, delta, A, B, C = map(_f64, (x, delta, A, B, C))
+    delta_bias, D, z = map(_f64, (delta_bias, D, z))
+    Bsz, L, Dm = x.shape
+    N = A.shape[1]
+    o = np.arange(L) if order is None else np.asarray(order, dtype=np.int64)
+    assert sorted(o.tolist()) == list(range(L)), "order must be a permutation"
+    g = lambda a: None if a is None else np.ascontiguousarray(np.take(a, o, axis=1))
+    xg, dg, zg, Bg, Cg = g(x), g(delta), g(z), g(B), g(C)
+    outg = np.zeros((Bsz, L, Dm))
+    st = np.zeros((Bsz, Dm, N))
+    keep, cp, nc = _cols(cols)
+    if mask is None:
+        _load().oracle_s6(Bsz, L, Dm, N, _ptr(xg), _ptr(dg), _ptr(delta_bias), int(softplus),
+                          _ptr(A), _ptr(Bg), _ptr(Cg), _ptr(D), _ptr(zg), int(reverse), _ptr(outg),
+                          _ptr(st), cp, nc, int(nthreads))
+    else:
+        mg = np.ascontiguousarray(np.take(np.asarray(mask, dtype=np.uint8), o, axis=1))
+        _load().oracle_s6_masked(Bsz, L, Dm, N, _ptr(xg), _ptr(dg), _ptr(delta_bias), int(softplus),
+                                 _ptr(A), _ptr(Bg), _ptr(Cg), _ptr(D), _ptr(zg), int(reverse),
+                                 mg.ctypes.data_as(ctypes.c_void_p), _ptr(outg), _ptr(st), cp, nc,
+                                 int(nthreads))
+    out = np.zeros_like(outg)
+    out[:, o] = outg
+    return out, st
+
+
+def bidir_ordered_arrays(x, delta, fwd: dict, bwd: dict, *, order=None, mask=None, softplus=True,
+                         cols=None, nthreads=1):
+    """Bidirectional scan along an order (Vim page sec. 3.2 on the ordered
+    sequence): the forward parameters scan the order, the backward ones scan
+    it reversed, the two outputs are summed.  Returns (out, last_f, last_b)."""
+    kw = dict(order=order, mask=mask, softplus=softplus, cols=cols, nthreads=nthreads)
+    of, lf = s6_ordered_arrays(x, delta, fwd["A"], fwd["B"], fwd["C"], delta_bias=fwd.get("delta_bias"),
+                               D=fwd.get("D"), z=fwd.get("z"), reverse=False, **kw)
+    ob, lb = s6_ordered_arrays(x, delta, bwd["A"], bwd["B"], bwd["C"], delta_bias=bwd.get("delta_bias"),
+                               D=bwd.get("D"), z=bwd.get("z"), reverse=True, **kw)
+    return of + ob, lf, lb
 
 
 def step_arrays(x, delta, A, B, C, state, *, delta_bias=None, softplus=True, D=None, z=None):

@@ -62,20 +62,27 @@ static double dt_of(double delta, const double *bias, int64_t d, int softplus)
 /*
  * One S6 column (batch b, channel d): the recurrence of sec. 4.3 with the
  * skip term and gate of sec. 4.4.  The state starts at h0 (N values) or, if
- * h0 is NULL, at zero as in sec. 4.3.  Writes y[t] for t in [0, L) and the
- * final state (N values) to hlast if non-NULL.
+ * h0 is NULL, at zero as in sec. 4.3.  mask (Bsz, L) or NULL: a token with
+ * mask 0 is bypassed (Samba page, sec. 2: the state is not updated and the
+ * computation is skipped) -- h passes through unchanged and y[t] = 0.
+ * Writes y[t] for t in [0, L) and the final state (N values) to hlast if
+ * non-NULL.
  */
 static void s6_column(int64_t b, int64_t d, int64_t L, int64_t D, int64_t N,
                       const double *x, const double *delta, const double *bias, int softplus,
                       const double *A, const double *Bm, const double *Cm, const double *Dv,
                       const double *z, int reverse, double *y, double *hlast, double *h,
-                      const double *h0)
+                      const double *h0, const unsigned char *mask)
 {
     for (int64_t n = 0; n < N; n++)
         h[n] = h0 ? h0[n] : 0.0;
     for (int64_t step = 0; step < L; step++) {
         int64_t t = reverse ? (L - 1 - step) : step;
         int64_t i = (b * L + t) * D + d;            /* (b, t, d) */
+        if (mask && !mask[b * L + t]) {
+            y[t] = 0.0;
+            continue;
+        }
         double dt = dt_of(delta[i], bias, d, softplus);
         double acc = 0.0;
         for (int64_t n = 0; n < N; n++) {
@@ -99,7 +106,8 @@ static void s6_column(int64_t b, int64_t d, int64_t L, int64_t D, int64_t N,
  * Single-direction S6.  x, delta, z: (Bsz, L, D); A: (D, N); Bm, Cm:
  * (Bsz, L, N); delta_bias, Dv: (D) or NULL; z NULL disables the gate.
  * out: (Bsz, L, D); last_state: (Bsz, D, N) or NULL; initial_state:
- * (Bsz, D, N), the state before the first step, or NULL for zero.
+ * (Bsz, D, N), the state before the first step, or NULL for zero; mask:
+ * (Bsz, L) bytes or NULL (see s6_column).
  * cols: list of column ids b*D + d to compute (NULL = every column); only
  * those columns of out / last_state are written.  If accumulate is set the
  * column's output is added to out instead of stored.
@@ -108,8 +116,8 @@ static void s6_run(int64_t Bsz, int64_t L, int64_t D, int64_t N,
                    const double *x, const double *delta, const double *delta_bias, int softplus,
                    const double *A, const double *Bm, const double *Cm, const double *Dv,
                    const double *z, int reverse, double *out, double *last_state,
-                   const double *initial_state, const int64_t *cols, int64_t ncols, int nthreads,
-                   int accumulate)
+                   const double *initial_state, const unsigned char *mask, const int64_t *cols,
+                   int64_t ncols, int nthreads, int accumulate)
 {
     int64_t total = cols ? ncols : Bsz * D;
 #ifdef _OPENMP
@@ -129,7 +137,7 @@ static void s6_run(int64_t Bsz, int64_t L, int64_t D, int64_t N,
             double *hl = last_state ? last_state + (b * D + d) * N : NULL;
             const double *h0 = initial_state ? initial_state + (b * D + d) * N : NULL;
             s6_column(b, d, L, D, N, x, delta, delta_bias, softplus, A, Bm, Cm, Dv, z,
-                      reverse, y, hl, h, h0);
+                      reverse, y, hl, h, h0, mask);
             for (int64_t t = 0; t < L; t++) {
                 int64_t i = (b * L + t) * D + d;
                 out[i] = accumulate ? out[i] + y[t] : y[t];
@@ -147,7 +155,7 @@ void oracle_s6(int64_t Bsz, int64_t L, int64_t D, int64_t N,
                const int64_t *cols, int64_t ncols, int nthreads)
 {
     s6_run(Bsz, L, D, N, x, delta, delta_bias, softplus, A, Bm, Cm, Dv, z, reverse, out,
-           last_state, NULL, cols, ncols, nthreads, 0);
+           last_state, NULL, NULL, cols, ncols, nthreads, 0);
 }
 
 /*
@@ -164,7 +172,24 @@ void oracle_s6_state(int64_t Bsz, int64_t L, int64_t D, int64_t N,
                      double *last_state, const int64_t *cols, int64_t ncols, int nthreads)
 {
     s6_run(Bsz, L, D, N, x, delta, delta_bias, softplus, A, Bm, Cm, Dv, z, reverse, out,
-           last_state, initial_state, cols, ncols, nthreads, 0);
+           last_state, initial_state, NULL, cols, ncols, nthreads, 0);
+}
+
+/*
+ * oracle_s6 with a token mask (Bsz, L): masked tokens are bypassed (Samba
+ * page, sec. 2) -- the state passes through unchanged and the output is 0.
+ * A scan along another order of the positions (Samba page sec. 3.1, the
+ * Mamba-YOLO page sec. 1.2 / 4.4) is this scan on inputs gathered in that
+ * order, its outputs scattered back (done by the Python wrapper).
+ */
+void oracle_s6_masked(int64_t Bsz, int64_t L, int64_t D, int64_t N,
+                      const double *x, const double *delta, const double *delta_bias, int softplus,
+                      const double *A, const double *Bm, const double *Cm, const double *Dv,
+                      const double *z, int reverse, const unsigned char *mask, double *out,
+                      double *last_state, const int64_t *cols, int64_t ncols, int nthreads)
+{
+    s6_run(Bsz, L, D, N, x, delta, delta_bias, softplus, A, Bm, Cm, Dv, z, reverse, out,
+           last_state, NULL, mask, cols, ncols, nthreads, 0);
 }
 
 /*
@@ -182,9 +207,9 @@ void oracle_bidir(int64_t Bsz, int64_t L, int64_t D, int64_t N,
                   double *out, const int64_t *cols, int64_t ncols, int nthreads)
 {
     s6_run(Bsz, L, D, N, x, delta, bias_f, softplus, A_f, B_f, C_f, D_f, z_f, 0, out, last_f,
-           NULL, cols, ncols, nthreads, 0);
+           NULL, NULL, cols, ncols, nthreads, 0);
     s6_run(Bsz, L, D, N, x, delta, bias_b, softplus, A_b, B_b, C_b, D_b, z_b, 1, out, last_b,
-           NULL, cols, ncols, nthreads, 1);
+           NULL, NULL, cols, ncols, nthreads, 1);
 }
 
 /*

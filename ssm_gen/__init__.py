@@ -239,3 +239,51 @@ def make_workload(idx: int, seed: int = 0, **overrides):
                               dtype=w["dtype"], bidir=w["bidir"], seed=seed)
     return make_ssd_inputs(w["batch"], w["seqlen"], w["nheads"], w["headdim"],
                            w["dstate"], w["chunk"], dtype=w["dtype"], seed=seed)
+
+
+# ------------------------------------------------------------ scan orders
+# Visiting orders of an H x W grid flattened row-major (position r * W + c),
+# and token masks: inputs of the ordered / masked scans, no scan arithmetic.
+
+def order_rows(H: int, W: int) -> np.ndarray:
+    """Row by row, left to right (the plain flattened order)."""
+    return np.arange(H * W, dtype=np.int32)
+
+
+def order_cols(H: int, W: int) -> np.ndarray:
+    """Column by column, top to bottom."""
+    return np.array([r * W + c for c in range(W) for r in range(H)], dtype=np.int32)
+
+
+def order_spiral(H: int, W: int) -> np.ndarray:
+    """Square spiral from the centre cell outward, clockwise (right, down,
+    left, up with run lengths 1, 1, 2, 2, 3, 3, ...), cells outside the grid
+    skipped, until every cell is visited."""
+    r, c = (H - 1) // 2, (W - 1) // 2
+    seen = np.zeros((H, W), dtype=bool)
+    out = []
+    moves = [(0, 1), (1, 0), (0, -1), (-1, 0)]
+    run, k = 1, 0
+    if H * W:
+        out.append(r * W + c)
+        seen[r, c] = True
+    while len(out) < H * W:
+        for _ in range(2):
+            dr, dc = moves[k % 4]
+            for _ in range(run):
+                r, c = r + dr, c + dc
+                if 0 <= r < H and 0 <= c < W and not seen[r, c]:
+                    seen[r, c] = True
+                    out.append(r * W + c)
+            k += 1
+        run += 1
+    return np.array(out, dtype=np.int32)
+
+
+def order_random(L: int, seed: int = 0) -> np.ndarray:
+    return np.random.default_rng(seed).permutation(L).astype(np.int32)
+
+
+def token_mask(batch: int, L: int, keep: float, seed: int = 0) -> np.ndarray:
+    """(batch, L) uint8, 1 = keep, each token kept with probability keep."""
+    return (np.random.default_rng(seed).random((batch, L)) < keep).astype(np.uint8)

@@ -394,3 +394,92 @@ def test_step_is_one_step_scan():
                                    D=D, z=z[:, t])
         _close(y, whole[:, t])
     _close(st, st_whole)
+
+
+# ------------------------------------------------ scan orders and token masks
+
+@pytest.mark.parametrize("reverse", [False, True])
+def test_identity_order_is_plain_scan(reverse):
+    rng = np.random.default_rng(400 + reverse)
+    x, delta, bias, A, B, C, D, z = _rand_case(rng, 2, 11, 3, 4)
+    y, st = oracle.s6_ordered_arrays(x, delta, A, B, C, order=np.arange(11), delta_bias=bias, D=D, z=z,
+                                     reverse=reverse)
+    y0, st0 = oracle.s6_arrays(x, delta, A, B, C, delta_bias=bias, D=D, z=z, reverse=reverse)
+    _close(y, y0)
+    _close(st, st0)
+
+
+def test_reversed_order_is_reverse_scan():
+    rng = np.random.default_rng(410)
+    x, delta, bias, A, B, C, D, z = _rand_case(rng, 2, 13, 3, 4)
+    y, st = oracle.s6_ordered_arrays(x, delta, A, B, C, order=np.arange(13)[::-1].copy(),
+                                     delta_bias=bias, D=D, z=z)
+    y0, st0 = oracle.s6_arrays(x, delta, A, B, C, delta_bias=bias, D=D, z=z, reverse=True)
+    _close(y, y0)
+    _close(st, st0)
+
+
+@pytest.mark.parametrize("reverse", [False, True])
+def test_column_order_is_transposed_grid(reverse):
+    """The column-major scan of an H x W grid equals the row scan of the
+    transposed grid, transposed back (reshape / transpose, no index array)."""
+    rng = np.random.default_rng(420 + reverse)
+    H, W, Bz, Dm, N = 3, 5, 2, 3, 4
+    x, delta, bias, A, B, C, D, z = _rand_case(rng, Bz, H * W, Dm, N)
+    y, st = oracle.s6_ordered_arrays(x, delta, A, B, C, order=ssm_gen.order_cols(H, W),
+                                     delta_bias=bias, D=D, z=z, reverse=reverse)
+    tr = lambda a: a.reshape(Bz, H, W, -1).transpose(0, 2, 1, 3).reshape(Bz, H * W, -1)
+    yt, stt = oracle.s6_arrays(tr(x), tr(delta), A, tr(B), tr(C), delta_bias=bias, D=D, z=tr(z),
+                               reverse=reverse)
+    back = yt.reshape(Bz, W, H, Dm).transpose(0, 2, 1, 3).reshape(Bz, H * W, Dm)
+    _close(y, back)
+    _close(st, stt)
+
+
+@pytest.mark.parametrize("reverse", [False, True])
+def test_masked_token_is_deleted_token(reverse):
+    """Masking one position equals scanning the sequence with that token
+    removed; the masked position's output is 0."""
+    rng = np.random.default_rng(430 + reverse)
+    x, delta, bias, A, B, C, D, z = _rand_case(rng, 1, 12, 3, 4)
+    p = 5
+    mask = np.ones((1, 12), dtype=np.uint8)
+    mask[0, p] = 0
+    order = ssm_gen.order_random(12, seed=3)
+    y, st = oracle.s6_ordered_arrays(x, delta, A, B, C, order=order, mask=mask, delta_bias=bias, D=D,
+                                     z=z, reverse=reverse)
+    keep = [q for q in order.tolist() if q != p]      # the visiting order without p
+    g = lambda a: a[:, keep]
+    yk, stk = oracle.s6_arrays(g(x), g(delta), A, g(B), g(C), delta_bias=bias, D=D, z=g(z),
+                               reverse=reverse)
+    assert np.all(y[:, p] == 0.0)
+    _close(y[:, keep], yk)
+    _close(st, stk)
+
+
+def test_all_masked_gives_zero():
+    rng = np.random.default_rng(440)
+    x, delta, bias, A, B, C, D, z = _rand_case(rng, 2, 6, 3, 4)
+    y, st = oracle.s6_ordered_arrays(x, delta, A, B, C, mask=np.zeros((2, 6), np.uint8),
+                                     delta_bias=bias, D=D, z=z)
+    assert np.all(y == 0.0) and np.all(st == 0.0)
+
+
+def test_bidir_ordered_identity_matches_bidir():
+    rng = np.random.default_rng(450)
+    x, delta, bias, A, B, C, D, z = _rand_case(rng, 2, 9, 3, 4)
+    _, _, bias2, A2, B2, C2, D2, z2 = _rand_case(rng, 2, 9, 3, 4)
+    f = dict(delta_bias=bias, A=A, B=B, C=C, D=D, z=z)
+    b = dict(delta_bias=bias2, A=A2, B=B2, C=C2, D=D2, z=z2)
+    y, lf, lb = oracle.bidir_ordered_arrays(x, delta, f, b)
+    y0, lf0, lb0 = oracle.bidir_arrays(x, delta, f, b)
+    _close(y, y0)
+    _close(lf, lf0)
+    _close(lb, lb0)
+
+
+def test_spiral_order_is_a_permutation_from_the_centre():
+    for H, W in [(1, 1), (3, 3), (4, 5), (6, 2), (14, 14)]:
+        o = ssm_gen.order_spiral(H, W)
+        assert sorted(o.tolist()) == list(range(H * W))
+        assert o[0] == ((H - 1) // 2) * W + (W - 1) // 2
