@@ -220,6 +220,38 @@ SSM_API ssm_status bidir_scan_fwd(const ssm_dims *dims, const void *x, const voi
 SSM_API ssm_status ssm_scan_plan(const ssm_dims *dims, int bidirectional, int *segments,
                                  int *channels_per_lane);
 
+/*
+ * S6 along a given order of the positions, with an optional token mask:
+ * the row, column, cross (several orders, summed by the caller) and
+ * centre-out spiral scans of the Samba (sec. 3.1) and Mamba-YOLO
+ * (sec. 1.2, 4.4) pages, and the masked-token bypass of the Samba page's
+ * pyramid-mask module (sec. 2).
+ *   order  (L) int32, 4-byte aligned, a permutation of 0..L-1 shared by the
+ *          batch, or NULL (0..L-1): step i reads and writes position
+ *          order[i] (order[L-1-i] when reversed).  An entry outside [0, L)
+ *          is treated as its own step index and makes ssm_check_device
+ *          return SSM_ERR_INVALID_ARG; repeated entries give unspecified
+ *          results.
+ *   mask   (B, L) bytes indexed by position, or NULL: 0 bypasses the token
+ *          -- the state passes through unchanged and out at that position
+ *          is 0 (for the bidirectional form, in both directions).
+ * Other arguments, workspace and errors as for ssm_scan_fwd.
+ */
+SSM_API ssm_status ssm_scan_fwd_ordered(const ssm_dims *dims, const void *x, const void *delta,
+                                        const float *delta_bias, int delta_softplus, const float *A,
+                                        const void *B, const void *C, const float *D, const void *z,
+                                        int reverse, const int32_t *order, const unsigned char *mask,
+                                        void *out, float *last_state, void *workspace,
+                                        size_t workspace_bytes, void *stream);
+
+/* bidir_scan_fwd along an order (the forward parameters scan it, the
+ * backward ones scan it reversed), with the token mask above. */
+SSM_API ssm_status bidir_scan_fwd_ordered(const ssm_dims *dims, const void *x, const void *delta,
+                                          int delta_softplus, const ssm_dir_params *fwd,
+                                          const ssm_dir_params *bwd, const int32_t *order,
+                                          const unsigned char *mask, void *out, void *workspace,
+                                          size_t workspace_bytes, void *stream);
+
 /* SSD problem size.  Supported: dtype SSM_BF16, headdim 64, dstate 128,
  * chunk 64, seqlen any value >= 0 (a short last chunk is handled). */
 typedef struct {
@@ -253,8 +285,9 @@ SSM_API ssm_status ssd_chunk_fwd(const ssd_dims *dims, const void *x, const void
 
 /*
  * Waits for `stream`, then reports (and clears) the library's device-side
- * error word: SSM_ERR_DEVICE_TIMEOUT if a bounded wait inside a kernel gave
- * up since the last check, SSM_ERR_CUDA if the stream reports a CUDA error,
+ * error words: SSM_ERR_DEVICE_TIMEOUT if a bounded wait inside a kernel gave
+ * up since the last check, SSM_ERR_INVALID_ARG if a scan order held an
+ * index outside [0, L), SSM_ERR_CUDA if the stream reports a CUDA error,
  * SSM_OK otherwise.  Blocking; meant for tests and debugging.
  */
 SSM_API ssm_status ssm_check_device(void *stream);

@@ -10,6 +10,8 @@ Entry points (names as in include/ssm.h):
 * ``ssm_scan_fwd(x, delta, A, B, C, ...)``  single-direction S6 scan
 * ``ssm_scan_fwd_state(...)``  the same from a given initial state
 * ``ssm_step(x, delta, A, B, C, state, ...)``  one decode step, state in place
+* ``ssm_scan_fwd_ordered`` / ``bidir_scan_fwd_ordered``  scans along a given
+  order of the positions, with an optional token mask
 * ``bidir_scan_fwd(x, delta, fwd, bwd, ...)``  Vision-Mamba bidirectional scan
 * ``ssd_chunk_fwd(x, delta, A, B, C, ...)``  Mamba2 SSD chunked scan
 
@@ -68,6 +70,11 @@ SIGNATURES = {
                             _int, _vp, _vp, _vp, _sz, _vp]),
     "ssm_scan_fwd_state": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp,
                                   _vp, _int, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "ssm_scan_fwd_ordered": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp,
+                                    _vp, _int, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "bidir_scan_fwd_ordered": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _int,
+                                      ctypes.POINTER(ssm_dir_params), ctypes.POINTER(ssm_dir_params),
+                                      _vp, _vp, _vp, _vp, _sz, _vp]),
     "ssm_step": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp, _vp, _vp,
                         _vp, _vp]),
     "ssm_scan_fwd_noalloc": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp,
@@ -214,6 +221,48 @@ def ssm_scan_fwd_state(x, delta, A, B, C, *, initial_state=None, delta_bias=None
                                 _ptr(last_state), _ptr(ws), 0 if ws is None else ws.numel(),
                                 _stream_handle(stream))
     _check(st, "ssm_scan_fwd_state")
+    return out
+
+
+def ssm_scan_fwd_ordered(x, delta, A, B, C, *, order=None, mask=None, delta_bias=None,
+                         delta_softplus=True, D=None, z=None, reverse=False, out=None,
+                         last_state=None, ws=None, stream=None):
+    """S6 along `order` (L) int32 (None = 0..L-1) with an optional token
+    mask (B, L) uint8 (0 = bypass the token)."""
+    torch = _torch()
+    lib = capi()
+    dims = s6_dims(x, A.shape[1])
+    if out is None:
+        out = torch.empty_like(x)
+    need = lib.ssm_scan_workspace_size(ctypes.byref(dims))
+    if ws is None:
+        ws = workspace(need, x.device)
+    st = lib.ssm_scan_fwd_ordered(ctypes.byref(dims), _ptr(x), _ptr(delta), _ptr(delta_bias),
+                                  int(bool(delta_softplus)), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                  _ptr(z), int(bool(reverse)), _ptr(order), _ptr(mask), _ptr(out),
+                                  _ptr(last_state), _ptr(ws), 0 if ws is None else ws.numel(),
+                                  _stream_handle(stream))
+    _check(st, "ssm_scan_fwd_ordered")
+    return out
+
+
+def bidir_scan_fwd_ordered(x, delta, fwd: DirParams, bwd: DirParams, *, order=None, mask=None,
+                           delta_softplus=True, out=None, ws=None, stream=None):
+    """bidir_scan_fwd along `order`, with an optional token mask."""
+    torch = _torch()
+    lib = capi()
+    dims = s6_dims(x, fwd.A.shape[1])
+    if out is None:
+        out = torch.empty_like(x)
+    need = lib.bidir_scan_workspace_size(ctypes.byref(dims))
+    if ws is None:
+        ws = workspace(need, x.device)
+    f, b = fwd.to_c(), bwd.to_c()
+    st = lib.bidir_scan_fwd_ordered(ctypes.byref(dims), _ptr(x), _ptr(delta), int(bool(delta_softplus)),
+                                    ctypes.byref(f), ctypes.byref(b), _ptr(order), _ptr(mask),
+                                    _ptr(out), _ptr(ws), 0 if ws is None else ws.numel(),
+                                    _stream_handle(stream))
+    _check(st, "bidir_scan_fwd_ordered")
     return out
 
 

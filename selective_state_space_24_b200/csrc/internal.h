@@ -46,6 +46,8 @@ struct S6Args {
     float *stash;    // ndir == 2: fp32 (Bsz, L, D) parking space for the
                      // first half of each direction's outputs (out itself
                      // when out is fp32)
+    const int *order;            // (L) visiting order of the positions, or nullptr (0..L-1)
+    const unsigned char *mask;   // (Bsz, L) by position, 0 = bypass the token, or nullptr
 };
 
 struct S6Plan {
@@ -87,7 +89,9 @@ struct SSDArgs {
 size_t ssd_workspace_bytes(int64_t Bsz, int64_t L, int64_t H, int64_t P, int64_t N, int64_t Q);
 cudaError_t launch_ssd(const SSDArgs &a, cudaStream_t stream);
 
-// Device-side error word (bounded waits that gave up set it).
+// Device-side error words: the SSD kernel's (bounded waits that gave up)
+// and the S6 kernels' (an out-of-range entry of a scan order).
 cudaError_t read_and_clear_device_error(unsigned *value, cudaStream_t stream);
+cudaError_t read_and_clear_s6_error(unsigned *value, cudaStream_t stream);
 
 }  // namespace ssm

@@ -48,6 +48,11 @@
 #include "s6_math.cuh"
 
 namespace ssm {
+
+// Set when a scan order holds an index outside [0, L) (the entry is then
+// treated as its own scan index, so nothing is accessed out of bounds).
+__device__ unsigned g_s6_error;
+
 namespace {
 
 constexpr int kWarps = 2;   // warps per CTA
@@ -209,6 +214,18 @@ template <> __device__ __forceinline__ float ld1<__nv_bfloat16>(const __nv_bfloa
 }
 
 __device__ __forceinline__ bool first_in_order(int seg, int S, bool rev) { return rev ? seg == S - 1 : seg == 0; }
+
+// Position visited at scan index t: order[t], or t itself without an order.
+__device__ __forceinline__ int position(int t, const int *order, int L)
+{
+    if (!order)
+        return t;
+    const int p = __ldg(order + t);
+    if ((unsigned)p < (unsigned)L)
+        return p;
+    atomicOr(&g_s6_error, 1u);
+    return t;
+}
 __device__ __forceinline__ bool last_in_order(int seg, int S, bool rev) { return rev ? seg == 0 : seg == S - 1; }
 
 __device__ __forceinline__ void pair_barrier() { asm volatile("bar.sync 1, 64;" ::: "memory"); }
@@ -230,7 +247,7 @@ struct BCStage {
     float v[NS];
 
     __device__ __forceinline__ void load(const T *Bm, const T *Cm, int N, size_t rowbase, int s0,
-                                         int s1, bool rev, int i0, int lane)
+                                         int s1, bool rev, int i0, int lane, const int *order, int L)
     {
         const int i = i0 + (lane >> 1);
         const int Tn = s1 - s0;
@@ -239,7 +256,7 @@ struct BCStage {
         for (int n = 0; n < NS; n++)
             v[n] = 0.f;
         if (i < Tn) {
-            const int t = rev ? s1 - 1 - i : s0 + i;
+            const int t = position(rev ? s1 - 1 - i : s0 + i, order, L);
             const T *row = src + (rowbase + t) * N;
             if (N == NS && sizeof(T) == 4 && NS % 4 == 0) {
 #pragma unroll
@@ -310,7 +327,8 @@ struct RowCopy {
 // One warp's scan over one segment, CPL adjacent channels per lane.
 //   SUMMARY: local end state from the given h, plus the sum of dt; no output.
 //   otherwise: outputs; BIDIR adds the midpoint exchange with the partner warp.
-template <typename T, int NS, int CPL, int NPOLY, bool SUMMARY, bool BIDIR, bool GATE, bool SOFTPLUS>
+template <typename T, int NS, int CPL, int NPOLY, bool SUMMARY, bool BIDIR, bool GATE, bool SOFTPLUS,
+          bool ORD>
 __device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P,
                                              WarpSmem<T, NS, CPL> &sm, int b, int dbase, bool active,
                                              int s0, int s1, bool rev, float2 (&h)[CPL][NS / 2],
@@ -350,7 +368,11 @@ __device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P,
 
     // midpoint of the pair exchange (see file comment)
     const int M = BIDIR ? (rev ? Tn / 2 : (Tn + 1) / 2) : Tn;
-    auto tpos = [&](int i) { return rev ? s1 - 1 - i : s0 + i; };
+    // position of step i (the scan index, mapped through the order if any)
+    // (ORD: the kernel was launched with an order and / or a token mask)
+    const int *order = ORD ? a.order : nullptr;
+    const unsigned char *tmask = ORD ? a.mask : nullptr;
+    auto tpos = [&](int i) { return position(rev ? s1 - 1 - i : s0 + i, order, a.L); };
     auto slot_of = [&](int i) { return sm.ring + (i % kSlots) * WS::kSlotB; };
 
     // this lane's 16-byte piece of a row and of a stash row
@@ -388,9 +410,9 @@ __device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P,
     BCStage<T, NS> stg;
     const T *Bm = static_cast<const T *>(P.B);
     const T *Cm = static_cast<const T *>(P.C);
-    stg.load(Bm, Cm, N, rowbase, s0, s1, rev, 0, lane);
+    stg.load(Bm, Cm, N, rowbase, s0, s1, rev, 0, lane, order, a.L);
     stg.store(sm.bc, lane);
-    stg.load(Bm, Cm, N, rowbase, s0, s1, rev, kTC, lane);
+    stg.load(Bm, Cm, N, rowbase, s0, s1, rev, kTC, lane, order, a.L);
 #pragma unroll
     for (int c = 0; c < kStages - 1; c++)
         issue_chunk(c, false);
@@ -405,7 +427,7 @@ __device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P,
         cp_async_wait<kStages - 1>();
         if ((i & (kTC - 1)) == 0 && i > 0) {
             stg.store(sm.bc + ((i / kTC) & 1) * kTC * 2 * NS, lane);
-            stg.load(Bm, Cm, N, rowbase, s0, s1, rev, i + kTC, lane);
+            stg.load(Bm, Cm, N, rowbase, s0, s1, rev, i + kTC, lane, order, a.L);
         }
         __syncwarp();
     };
@@ -414,10 +436,12 @@ __device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P,
     // previous step); finish: skip term, gate, store.
     struct StepIn {
         float xv[CPL], zv[CPL], dt[CPL];
+        bool keep;   // false: the token is masked (bypassed)
     };
     auto load_dt = [&](int i) {
         const char *slot = slot_of(i) + lane * CPL * (int)sizeof(T);
         StepIn o;
+        o.keep = !ORD || !tmask || tmask[rowbase + tpos(i)] != 0;
         float dv[CPL];
         IO<T, CPL>::ld(slot, o.xv);
         IO<T, CPL>::ld(slot + WS::kRowB, dv);
@@ -428,6 +452,8 @@ __device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P,
             o.dt[c] = dv[c] + bias[c];
             if (SOFTPLUS)
                 o.dt[c] = softplus_f(o.dt[c]);
+            if (ORD && !o.keep)
+                o.dt[c] = 0.f;   // exp(0 A) = 1 and dt B x = 0: the state passes through
             o.zv[c] = (!SUMMARY && GATE) ? silu_f<T>(o.zv[c]) : 0.f;   // zv now holds the gate
         }
         return o;
@@ -499,6 +525,8 @@ __device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P,
             y[c] = fmaf(Dd[c], in.xv[c], ys.y[c]);
             if (GATE)
                 y[c] *= in.zv[c];
+            if (ORD && !in.keep)
+                y[c] = 0.f;
         }
         if (!SUMMARY && active) {
             const size_t io = (rowbase + tpos(i)) * a.D + d;
@@ -571,7 +599,7 @@ template <typename T, int NS, int CPL>
 constexpr int smem_bytes() { return kWarps * (int)sizeof(WarpSmem<T, NS, CPL>); }
 
 // ---------------------------------------------------------------- summary
-template <typename T, int NS, int CPL, int NPOLY, bool SOFTPLUS>
+template <typename T, int NS, int CPL, int NPOLY, bool SOFTPLUS, bool ORD>
 __global__ void __launch_bounds__(64, min_blocks<CPL>()) s6_summary_kernel(const S6Args a)
 {
     extern __shared__ __align__(16) char smem_raw[];
@@ -597,8 +625,8 @@ __global__ void __launch_bounds__(64, min_blocks<CPL>()) s6_summary_kernel(const
         for (int k = 0; k < NS / 2; k++)
             h[c][k] = make_float2(0.f, 0.f);
     }
-    scan_segment<T, NS, CPL, NPOLY, true, false, false, SOFTPLUS>(a, a.dir[dsel], sm[warp], b, dbase,
-                                                                  active, s0, s1, rev, h, sdt);
+    scan_segment<T, NS, CPL, NPOLY, true, false, false, SOFTPLUS, ORD>(a, a.dir[dsel], sm[warp], b, dbase,
+                                                                       active, s0, s1, rev, h, sdt);
     if (!active)
         return;
 #pragma unroll
@@ -663,7 +691,7 @@ __global__ void s6_carry_kernel(const S6Args a)
 }
 
 // ------------------------------------------------------------------- main
-template <typename T, int NS, int CPL, int NPOLY, bool BIDIR, bool GATE, bool SOFTPLUS>
+template <typename T, int NS, int CPL, int NPOLY, bool BIDIR, bool GATE, bool SOFTPLUS, bool ORD>
 __global__ void __launch_bounds__(64, min_blocks<CPL>()) s6_main_kernel(const S6Args a)
 {
     extern __shared__ __align__(16) char smem_raw[];
@@ -699,8 +727,8 @@ __global__ void __launch_bounds__(64, min_blocks<CPL>()) s6_main_kernel(const S6
             h[c][k].y = (active && src && 2 * k + 1 < a.N) ? src[2 * k + 1] : 0.f;
         }
     }
-    scan_segment<T, NS, CPL, NPOLY, false, BIDIR, GATE, SOFTPLUS>(a, P, sm[warp], b, dbase, active,
-                                                                  s0, s1, rev, h, sdt);
+    scan_segment<T, NS, CPL, NPOLY, false, BIDIR, GATE, SOFTPLUS, ORD>(a, P, sm[warp], b, dbase, active,
+                                                                       s0, s1, rev, h, sdt);
     if (active && P.last_state && last_in_order(seg, a.S, rev)) {
 #pragma unroll
         for (int c = 0; c < CPL; c++) {
@@ -722,14 +750,14 @@ cudaError_t set_smem(KernelT k, int bytes)
     return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
-template <typename T, int NS, int CPL, int NPOLY, bool GATE, bool SOFTPLUS>
+template <typename T, int NS, int CPL, int NPOLY, bool GATE, bool SOFTPLUS, bool ORD>
 cudaError_t launch_typed(const S6Args &a, cudaStream_t st)
 {
     constexpr int smem = smem_bytes<T, NS, CPL>();
     constexpr int kCh = 32 * CPL;
     cudaError_t e;
     if (a.S > 1) {
-        auto ks = s6_summary_kernel<T, NS, CPL, SSM_S6_SUM_NPOLY(NS), SOFTPLUS>;
+        auto ks = s6_summary_kernel<T, NS, CPL, SSM_S6_SUM_NPOLY(NS), SOFTPLUS, ORD>;
         if ((e = set_smem(ks, smem)) != cudaSuccess)
             return e;
         dim3 g1((a.D + kWarps * kCh - 1) / (kWarps * kCh), a.S, a.Bsz * a.ndir);
@@ -738,13 +766,13 @@ cudaError_t launch_typed(const S6Args &a, cudaStream_t st)
         s6_carry_kernel<<<(unsigned)((tot + 255) / 256), 256, 0, st>>>(a);
     }
     if (a.ndir == 2) {
-        auto km = s6_main_kernel<T, NS, CPL, NPOLY, true, GATE, SOFTPLUS>;
+        auto km = s6_main_kernel<T, NS, CPL, NPOLY, true, GATE, SOFTPLUS, ORD>;
         if ((e = set_smem(km, smem)) != cudaSuccess)
             return e;
         dim3 g((a.D + kCh - 1) / kCh, a.S, a.Bsz);
         km<<<g, 64, smem, st>>>(a);
     } else {
-        auto km = s6_main_kernel<T, NS, CPL, NPOLY, false, GATE, SOFTPLUS>;
+        auto km = s6_main_kernel<T, NS, CPL, NPOLY, false, GATE, SOFTPLUS, ORD>;
         if ((e = set_smem(km, smem)) != cudaSuccess)
             return e;
         dim3 g((a.D + kWarps * kCh - 1) / (kWarps * kCh), a.S, a.Bsz);
@@ -756,8 +784,11 @@ cudaError_t launch_typed(const S6Args &a, cudaStream_t st)
 template <typename T, int NS, int NPOLY, bool GATE, bool SOFTPLUS>
 cudaError_t launch_cpl(const S6Args &a, cudaStream_t st)
 {
-    return a.cpl == 1 ? launch_typed<T, NS, 1, NPOLY, GATE, SOFTPLUS>(a, st)
-                      : launch_typed<T, NS, 2, NPOLY, GATE, SOFTPLUS>(a, st);
+    if (a.order || a.mask)
+        return a.cpl == 1 ? launch_typed<T, NS, 1, NPOLY, GATE, SOFTPLUS, true>(a, st)
+                          : launch_typed<T, NS, 2, NPOLY, GATE, SOFTPLUS, true>(a, st);
+    return a.cpl == 1 ? launch_typed<T, NS, 1, NPOLY, GATE, SOFTPLUS, false>(a, st)
+                      : launch_typed<T, NS, 2, NPOLY, GATE, SOFTPLUS, false>(a, st);
 }
 
 #ifndef SSM_S6_NPOLY
@@ -786,6 +817,18 @@ cudaError_t launch_ns(const S6Args &a, cudaStream_t st)
 }
 
 }  // namespace
+
+cudaError_t read_and_clear_s6_error(unsigned *value, cudaStream_t stream)
+{
+    cudaError_t e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess)
+        return e;
+    e = cudaMemcpyFromSymbol(value, g_s6_error, sizeof(unsigned));
+    if (e != cudaSuccess)
+        return e;
+    const unsigned zero = 0;
+    return cudaMemcpyToSymbol(g_s6_error, &zero, sizeof(unsigned));
+}
 
 S6Plan plan_s6(int64_t Bsz, int64_t L, int64_t D, int64_t N, int ndir, int dtype)
 {

@@ -64,7 +64,8 @@ ssm::DirArgs dir_args(const ssm_dir_params &p)
 
 ssm_status run_s6(const ssm_dims *dims, const void *x, const void *delta, int softplus, int ndir,
                   int reverse, const ssm_dir_params *dirs, void *out, void *ws, size_t ws_bytes,
-                  cudaStream_t stream, const float *initial_state = nullptr)
+                  cudaStream_t stream, const float *initial_state = nullptr, const int32_t *order = nullptr,
+                  const unsigned char *mask = nullptr)
 {
     const int dt = dims->dtype == SSM_F32 ? 0 : 1;
     const ssm::S6Plan plan =
@@ -93,6 +94,8 @@ ssm_status run_s6(const ssm_dims *dims, const void *x, const void *delta, int so
     for (int i = 0; i < ndir; i++)
         a.dir[i] = dir_args(dirs[i]);
     a.dir[0].init = initial_state;   // single direction only
+    a.order = order;
+    a.mask = mask;
     a.out = out;
     char *w = static_cast<char *>(ws);
     if (plan.S > 1) {
@@ -141,16 +144,24 @@ ssm_status ssm_scan_plan(const ssm_dims *dims, int bidirectional, int *segments,
     return SSM_OK;
 }
 
-ssm_status ssm_scan_fwd_state(const ssm_dims *dims, const void *x, const void *delta,
-                              const float *delta_bias, int delta_softplus, const float *A,
-                              const void *B, const void *C, const float *D, const void *z,
-                              int reverse, const float *initial_state, void *out, float *last_state,
-                              void *workspace, size_t workspace_bytes, void *stream)
+}  // extern "C"
+
+namespace {
+
+// Single-direction S6 with every option: the entry points below are this
+// with some options off.
+ssm_status scan_single(const ssm_dims *dims, const void *x, const void *delta, const float *delta_bias,
+                       int delta_softplus, const float *A, const void *B, const void *C, const float *D,
+                       const void *z, int reverse, const float *initial_state, const int32_t *order,
+                       const unsigned char *mask, void *out, float *last_state, void *workspace,
+                       size_t workspace_bytes, void *stream)
 {
     ssm_status s = check_s6_dims(dims);
     if (s != SSM_OK)
         return s;
     if ((initial_state && !aligned16(initial_state)) || (last_state && !aligned16(last_state)))
+        return SSM_ERR_MISALIGNED;
+    if (order && (reinterpret_cast<uintptr_t>(order) & 3u))
         return SSM_ERR_MISALIGNED;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (empty_s6(dims)) {
@@ -174,7 +185,75 @@ ssm_status ssm_scan_fwd_state(const ssm_dims *dims, const void *x, const void *d
     if (!aligned16(x) || !aligned16(delta) || !aligned16(out))
         return SSM_ERR_MISALIGNED;
     return run_s6(dims, x, delta, delta_softplus, 1, reverse, &p, out, workspace, workspace_bytes, st,
-                  initial_state);
+                  initial_state, order, mask);
+}
+
+ssm_status scan_bidir(const ssm_dims *dims, const void *x, const void *delta, int delta_softplus,
+                      const ssm_dir_params *fwd, const ssm_dir_params *bwd, const int32_t *order,
+                      const unsigned char *mask, void *out, void *workspace, size_t workspace_bytes,
+                      void *stream)
+{
+    ssm_status s = check_s6_dims(dims);
+    if (s != SSM_OK)
+        return s;
+    if (!fwd || !bwd)
+        return SSM_ERR_INVALID_ARG;
+    if (order && (reinterpret_cast<uintptr_t>(order) & 3u))
+        return SSM_ERR_MISALIGNED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (empty_s6(dims)) {
+        if ((fwd->last_state && !aligned16(fwd->last_state)) ||
+            (bwd->last_state && !aligned16(bwd->last_state)))
+            return SSM_ERR_MISALIGNED;
+        if ((s = zero_state(fwd->last_state, dims, st)) != SSM_OK)
+            return s;
+        return zero_state(bwd->last_state, dims, st);
+    }
+    if (!x || !delta || !out)
+        return SSM_ERR_INVALID_ARG;
+    if ((s = check_dir(fwd)) != SSM_OK || (s = check_dir(bwd)) != SSM_OK)
+        return s;
+    if ((fwd->z == nullptr) != (bwd->z == nullptr))
+        return SSM_ERR_INVALID_ARG;   // both directions gated, or neither
+    if (!aligned16(x) || !aligned16(delta) || !aligned16(out))
+        return SSM_ERR_MISALIGNED;
+    const ssm_dir_params dirs[2] = {*fwd, *bwd};
+    return run_s6(dims, x, delta, delta_softplus, 2, 0, dirs, out, workspace, workspace_bytes, st, nullptr,
+                  order, mask);
+}
+
+}  // namespace
+
+extern "C" {
+
+ssm_status ssm_scan_fwd_state(const ssm_dims *dims, const void *x, const void *delta,
+                              const float *delta_bias, int delta_softplus, const float *A,
+                              const void *B, const void *C, const float *D, const void *z,
+                              int reverse, const float *initial_state, void *out, float *last_state,
+                              void *workspace, size_t workspace_bytes, void *stream)
+{
+    return scan_single(dims, x, delta, delta_bias, delta_softplus, A, B, C, D, z, reverse, initial_state,
+                       nullptr, nullptr, out, last_state, workspace, workspace_bytes, stream);
+}
+
+ssm_status ssm_scan_fwd_ordered(const ssm_dims *dims, const void *x, const void *delta,
+                                const float *delta_bias, int delta_softplus, const float *A,
+                                const void *B, const void *C, const float *D, const void *z,
+                                int reverse, const int32_t *order, const unsigned char *mask, void *out,
+                                float *last_state, void *workspace, size_t workspace_bytes, void *stream)
+{
+    return scan_single(dims, x, delta, delta_bias, delta_softplus, A, B, C, D, z, reverse, nullptr, order,
+                       mask, out, last_state, workspace, workspace_bytes, stream);
+}
+
+ssm_status bidir_scan_fwd_ordered(const ssm_dims *dims, const void *x, const void *delta,
+                                  int delta_softplus, const ssm_dir_params *fwd,
+                                  const ssm_dir_params *bwd, const int32_t *order,
+                                  const unsigned char *mask, void *out, void *workspace,
+                                  size_t workspace_bytes, void *stream)
+{
+    return scan_bidir(dims, x, delta, delta_softplus, fwd, bwd, order, mask, out, workspace,
+                      workspace_bytes, stream);
 }
 
 ssm_status ssm_scan_fwd(const ssm_dims *dims, const void *x, const void *delta,
@@ -228,30 +307,8 @@ ssm_status bidir_scan_fwd(const ssm_dims *dims, const void *x, const void *delta
                           const ssm_dir_params *bwd, void *out, void *workspace,
                           size_t workspace_bytes, void *stream)
 {
-    ssm_status s = check_s6_dims(dims);
-    if (s != SSM_OK)
-        return s;
-    if (!fwd || !bwd)
-        return SSM_ERR_INVALID_ARG;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (empty_s6(dims)) {
-        if ((fwd->last_state && !aligned16(fwd->last_state)) ||
-            (bwd->last_state && !aligned16(bwd->last_state)))
-            return SSM_ERR_MISALIGNED;
-        if ((s = zero_state(fwd->last_state, dims, st)) != SSM_OK)
-            return s;
-        return zero_state(bwd->last_state, dims, st);
-    }
-    if (!x || !delta || !out)
-        return SSM_ERR_INVALID_ARG;
-    if ((s = check_dir(fwd)) != SSM_OK || (s = check_dir(bwd)) != SSM_OK)
-        return s;
-    if ((fwd->z == nullptr) != (bwd->z == nullptr))
-        return SSM_ERR_INVALID_ARG;   // both directions gated, or neither
-    if (!aligned16(x) || !aligned16(delta) || !aligned16(out))
-        return SSM_ERR_MISALIGNED;
-    const ssm_dir_params dirs[2] = {*fwd, *bwd};
-    return run_s6(dims, x, delta, delta_softplus, 2, 0, dirs, out, workspace, workspace_bytes, st);
+    return scan_bidir(dims, x, delta, delta_softplus, fwd, bwd, nullptr, nullptr, out, workspace,
+                      workspace_bytes, stream);
 }
 
 size_t ssd_chunk_workspace_size(const ssd_dims *d)
@@ -330,10 +387,13 @@ ssm_status ssd_chunk_fwd(const ssd_dims *dims, const void *x, const void *delta,
 
 ssm_status ssm_check_device(void *stream)
 {
-    unsigned v = 0;
-    if (ssm::read_and_clear_device_error(&v, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    unsigned v = 0, o = 0;
+    if (ssm::read_and_clear_device_error(&v, static_cast<cudaStream_t>(stream)) != cudaSuccess ||
+        ssm::read_and_clear_s6_error(&o, static_cast<cudaStream_t>(stream)) != cudaSuccess)
         return SSM_ERR_CUDA;
-    return v ? SSM_ERR_DEVICE_TIMEOUT : SSM_OK;
+    if (v)
+        return SSM_ERR_DEVICE_TIMEOUT;
+    return o ? SSM_ERR_INVALID_ARG : SSM_OK;
 }
 
 const char *ssm_status_string(ssm_status s)
