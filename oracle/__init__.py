@@ -168,6 +168,53 @@ def bidir_ordered_arrays(x, delta, fwd: dict, bwd: dict, *, order=None, mask=Non
     return of + ob, lf, lb
 
 
+def conv_u(x, weight, bias=None, silu=True, reverse=False):
+    """The depthwise causal conv1d before the scan (Mamba2 page sec. 4.4
+    listing: groups = channels, padding K-1, the first L outputs kept), with
+    an optional bias and SiLU after it:
+        u[b,t,d] = act(bias[d] + sum_k weight[d,k] x[b, t-(K-1)+k, d]),
+    x taken as 0 outside [0, L).  reverse: the conv of the flipped sequence
+    (a reversed scan's own conv, as each Vim direction has), flipped back --
+    the window then runs over t .. t+K-1."""
+    x = np.asarray(x, dtype=np.float64)
+    w = np.asarray(weight, dtype=np.float64)
+    if reverse:
+        return conv_u(x[:, ::-1], w, bias, silu, False)[:, ::-1].copy()
+    Bsz, L, Dm = x.shape
+    K = w.shape[1]
+    u = np.zeros_like(x)
+    for k in range(K):
+        s = K - 1 - k                      # x[t - s] contributes with weight[:, k]
+        if s < L:
+            u[:, s:, :] += w[None, None, :, k] * x[:, :L - s, :]
+    if bias is not None:
+        u += np.asarray(bias, dtype=np.float64)[None, None, :]
+    if silu:
+        u = u / (1.0 + np.exp(-u))
+    return u
+
+
+def s6_conv_arrays(x_in, conv_weight, delta, A, B, C, *, conv_bias=None, conv_silu=True,
+                   reverse=False, **kw):
+    """S6 whose input is conv_u(x_in): the scan and its D skip both use u."""
+    u = conv_u(x_in, conv_weight, conv_bias, conv_silu, reverse)
+    return s6_arrays(u, delta, A, B, C, reverse=reverse, **kw)
+
+
+def bidir_conv_arrays(x_in, delta, fwd: dict, bwd: dict, conv_f: dict, conv_b: dict, *, softplus=True,
+                      cols=None, nthreads=1):
+    """Bidirectional scan where each direction convolves x_in with its own
+    conv (conv_* dicts: weight, bias, silu) along its scan direction."""
+    uf = conv_u(x_in, conv_f["weight"], conv_f.get("bias"), conv_f.get("silu", True), False)
+    ub = conv_u(x_in, conv_b["weight"], conv_b.get("bias"), conv_b.get("silu", True), True)
+    of, lf = s6_arrays(uf, delta, fwd["A"], fwd["B"], fwd["C"], delta_bias=fwd.get("delta_bias"),
+                       softplus=softplus, D=fwd.get("D"), z=fwd.get("z"), cols=cols, nthreads=nthreads)
+    ob, lb = s6_arrays(ub, delta, bwd["A"], bwd["B"], bwd["C"], delta_bias=bwd.get("delta_bias"),
+                       softplus=softplus, D=bwd.get("D"), z=bwd.get("z"), reverse=True, cols=cols,
+                       nthreads=nthreads)
+    return of + ob, lf, lb
+
+
 def step_arrays(x, delta, A, B, C, state, *, delta_bias=None, softplus=True, D=None, z=None):
     """One time step of S6 for every (b, d) from a stored state -- the
     recurrent (decode) form: x, delta, z (B, D); B, C (B, N); state (B, D, N).

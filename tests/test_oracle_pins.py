@@ -483,3 +483,42 @@ def test_spiral_order_is_a_permutation_from_the_centre():
         o = ssm_gen.order_spiral(H, W)
         assert sorted(o.tolist()) == list(range(H * W))
         assert o[0] == ((H - 1) // 2) * W + (W - 1) // 2
+
+
+# ------------------------------------------------ the conv1d before the scan
+
+@pytest.mark.parametrize("K", [1, 2, 3, 4])
+def test_conv_matches_numpy_convolve(K):
+    """The causal depthwise conv equals numpy's full convolution with the
+    kernel reversed, first L outputs kept, per channel."""
+    rng = np.random.default_rng(500 + K)
+    x = rng.standard_normal((2, 11, 3))
+    w = rng.standard_normal((3, K))
+    bias = rng.standard_normal(3)
+    u = oracle.conv_u(x, w, bias, silu=False)
+    for b in range(2):
+        for d in range(3):
+            ref = np.convolve(x[b, :, d], w[d, ::-1])[:11] + bias[d]
+            _close(u[b, :, d], ref)
+    us = oracle.conv_u(x, w, bias, silu=True)
+    _close(us, _silu(u))
+
+
+def test_conv_reverse_is_flip():
+    rng = np.random.default_rng(510)
+    x = rng.standard_normal((2, 9, 3))
+    w = rng.standard_normal((3, 3))
+    ur = oracle.conv_u(x, w, None, silu=True, reverse=True)
+    _close(ur, oracle.conv_u(x[:, ::-1], w, None, silu=True)[:, ::-1])
+
+
+def test_conv_scan_identity_kernel_is_plain_scan():
+    """Width 1, weight 1, no bias, no SiLU: the conv is the identity and the
+    conv scan is the plain scan of x_in."""
+    rng = np.random.default_rng(520)
+    x, delta, bias, A, B, C, D, z = _rand_case(rng, 2, 10, 3, 4)
+    y, st = oracle.s6_conv_arrays(x, np.ones((3, 1)), delta, A, B, C, conv_silu=False, delta_bias=bias,
+                                  D=D, z=z)
+    y0, st0 = oracle.s6_arrays(x, delta, A, B, C, delta_bias=bias, D=D, z=z)
+    _close(y, y0)
+    _close(st, st0)
