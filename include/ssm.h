@@ -252,6 +252,41 @@ SSM_API ssm_status bidir_scan_fwd_ordered(const ssm_dims *dims, const void *x, c
                                           const unsigned char *mask, void *out, void *workspace,
                                           size_t workspace_bytes, void *stream);
 
+/*
+ * The depthwise causal conv1d that precedes the scan (the Mamba2 page's
+ * block, sec. 4.4 listing: one kernel per channel, padding width-1, the
+ * first L outputs kept; the Vim page, sec. 2: a short kernel before the
+ * scan to mix neighbouring tokens), optionally followed by SiLU:
+ *   u[t, d] = act(bias[d] + sum_{k < width} weight[d, k] x_in[t - (width-1) + k, d])
+ * with t counted along the scan direction (a reversed scan convolves the
+ * flipped sequence) and x_in = 0 before the first step.
+ */
+typedef struct {
+    const float *weight;   /* (D, width) float32, required */
+    const float *bias;     /* (D) float32, or NULL */
+    int32_t width;         /* 1..4 (SSM_ERR_UNSUPPORTED_SHAPE otherwise) */
+    int32_t silu;          /* 1: u = silu(conv), 0: u = conv */
+} ssm_conv_params;
+
+/*
+ * ssm_scan_fwd on u = conv(x_in) computed inside the scan: x_in (B, L, D)
+ * dtype replaces x, and the scan and its D skip both use u.  Other
+ * arguments, workspace and errors as for ssm_scan_fwd.
+ */
+SSM_API ssm_status ssm_scan_fwd_conv(const ssm_dims *dims, const void *x_in, const ssm_conv_params *conv,
+                                     const void *delta, const float *delta_bias, int delta_softplus,
+                                     const float *A, const void *B, const void *C, const float *D,
+                                     const void *z, int reverse, void *out, float *last_state,
+                                     void *workspace, size_t workspace_bytes, void *stream);
+
+/* bidir_scan_fwd on x_in, each direction convolving it with its own conv
+ * along its own scan direction (as each Vim direction has its own conv). */
+SSM_API ssm_status bidir_scan_fwd_conv(const ssm_dims *dims, const void *x_in, const void *delta,
+                                       int delta_softplus, const ssm_dir_params *fwd,
+                                       const ssm_dir_params *bwd, const ssm_conv_params *conv_fwd,
+                                       const ssm_conv_params *conv_bwd, void *out, void *workspace,
+                                       size_t workspace_bytes, void *stream);
+
 /* SSD problem size.  Supported: dtype SSM_BF16, headdim 64, dstate 128,
  * chunk 64, seqlen any value >= 0 (a short last chunk is handled). */
 typedef struct {

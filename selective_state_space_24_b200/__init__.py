@@ -12,6 +12,8 @@ Entry points (names as in include/ssm.h):
 * ``ssm_step(x, delta, A, B, C, state, ...)``  one decode step, state in place
 * ``ssm_scan_fwd_ordered`` / ``bidir_scan_fwd_ordered``  scans along a given
   order of the positions, with an optional token mask
+* ``ssm_scan_fwd_conv`` / ``bidir_scan_fwd_conv``  scans of u = conv1d(x_in),
+  the conv computed inside the scan
 * ``bidir_scan_fwd(x, delta, fwd, bwd, ...)``  Vision-Mamba bidirectional scan
 * ``ssd_chunk_fwd(x, delta, A, B, C, ...)``  Mamba2 SSD chunked scan
 
@@ -59,6 +61,11 @@ class ssm_dir_params(ctypes.Structure):
                 ("last_state", ctypes.c_void_p)]
 
 
+class ssm_conv_params(ctypes.Structure):
+    _fields_ = [("weight", ctypes.c_void_p), ("bias", ctypes.c_void_p), ("width", ctypes.c_int32),
+                ("silu", ctypes.c_int32)]
+
+
 _vp = ctypes.c_void_p
 _sz = ctypes.c_size_t
 _int = ctypes.c_int
@@ -75,6 +82,12 @@ SIGNATURES = {
     "bidir_scan_fwd_ordered": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _int,
                                       ctypes.POINTER(ssm_dir_params), ctypes.POINTER(ssm_dir_params),
                                       _vp, _vp, _vp, _vp, _sz, _vp]),
+    "ssm_scan_fwd_conv": (_int, [ctypes.POINTER(ssm_dims), _vp, ctypes.POINTER(ssm_conv_params), _vp,
+                                 _vp, _int, _vp, _vp, _vp, _vp, _vp, _int, _vp, _vp, _vp, _sz, _vp]),
+    "bidir_scan_fwd_conv": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _int,
+                                   ctypes.POINTER(ssm_dir_params), ctypes.POINTER(ssm_dir_params),
+                                   ctypes.POINTER(ssm_conv_params), ctypes.POINTER(ssm_conv_params),
+                                   _vp, _vp, _sz, _vp]),
     "ssm_step": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp, _vp, _vp,
                         _vp, _vp]),
     "ssm_scan_fwd_noalloc": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp,
@@ -263,6 +276,60 @@ def bidir_scan_fwd_ordered(x, delta, fwd: DirParams, bwd: DirParams, *, order=No
                                     _ptr(out), _ptr(ws), 0 if ws is None else ws.numel(),
                                     _stream_handle(stream))
     _check(st, "bidir_scan_fwd_ordered")
+    return out
+
+
+@dataclass
+class Conv:
+    """The conv1d before the scan (tensors on the device): weight (D, width)
+    float32, bias (D) float32 or None, SiLU after it or not."""
+    weight: object
+    bias: object = None
+    silu: bool = True
+
+    def to_c(self) -> ssm_conv_params:
+        return ssm_conv_params(_ptr(self.weight), _ptr(self.bias), int(self.weight.shape[1]),
+                               int(bool(self.silu)))
+
+
+def ssm_scan_fwd_conv(x_in, conv: Conv, delta, A, B, C, *, delta_bias=None, delta_softplus=True, D=None,
+                      z=None, reverse=False, out=None, last_state=None, ws=None, stream=None):
+    """S6 on u = conv(x_in), computed inside the scan."""
+    torch = _torch()
+    lib = capi()
+    dims = s6_dims(x_in, A.shape[1])
+    if out is None:
+        out = torch.empty_like(x_in)
+    need = lib.ssm_scan_workspace_size(ctypes.byref(dims))
+    if ws is None:
+        ws = workspace(need, x_in.device)
+    cv = conv.to_c()
+    st = lib.ssm_scan_fwd_conv(ctypes.byref(dims), _ptr(x_in), ctypes.byref(cv), _ptr(delta),
+                               _ptr(delta_bias), int(bool(delta_softplus)), _ptr(A), _ptr(B), _ptr(C),
+                               _ptr(D), _ptr(z), int(bool(reverse)), _ptr(out), _ptr(last_state), _ptr(ws),
+                               0 if ws is None else ws.numel(), _stream_handle(stream))
+    _check(st, "ssm_scan_fwd_conv")
+    return out
+
+
+def bidir_scan_fwd_conv(x_in, delta, fwd: DirParams, bwd: DirParams, conv_fwd: Conv, conv_bwd: Conv, *,
+                        delta_softplus=True, out=None, ws=None, stream=None):
+    """bidir_scan_fwd on x_in, each direction with its own conv."""
+    torch = _torch()
+    lib = capi()
+    dims = s6_dims(x_in, fwd.A.shape[1])
+    if out is None:
+        out = torch.empty_like(x_in)
+    need = lib.bidir_scan_workspace_size(ctypes.byref(dims))
+    if ws is None:
+        ws = workspace(need, x_in.device)
+    f, b = fwd.to_c(), bwd.to_c()
+    cf, cb = conv_fwd.to_c(), conv_bwd.to_c()
+    st = lib.bidir_scan_fwd_conv(ctypes.byref(dims), _ptr(x_in), _ptr(delta), int(bool(delta_softplus)),
+                                 ctypes.byref(f), ctypes.byref(b), ctypes.byref(cf), ctypes.byref(cb),
+                                 _ptr(out), _ptr(ws), 0 if ws is None else ws.numel(),
+                                 _stream_handle(stream))
+    _check(st, "bidir_scan_fwd_conv")
     return out
 
 

@@ -18,6 +18,12 @@ struct DirArgs {
     const void *z;       // (Bsz, L, D) or nullptr
     float *last_state;   // (Bsz, D, N) or nullptr
     const float *init;   // (Bsz, D, N) state before the first step, or nullptr (zero)
+    // depthwise causal conv1d applied to x along this direction's scan order
+    // (used by the kernels' conv variant only)
+    const float *conv_w;   // (D, conv_k)
+    const float *conv_b;   // (D) or nullptr
+    int conv_k;            // 1..4
+    int conv_silu;         // 1: SiLU after the conv
 };
 
 // One S6 call (single direction or bidirectional).
@@ -48,6 +54,7 @@ struct S6Args {
                      // when out is fp32)
     const int *order;            // (L) visiting order of the positions, or nullptr (0..L-1)
     const unsigned char *mask;   // (Bsz, L) by position, 0 = bypass the token, or nullptr
+    int conv;                    // 1: x is the conv input x_in, each direction convolves it
 };
 
 struct S6Plan {

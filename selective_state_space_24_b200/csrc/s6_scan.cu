@@ -328,7 +328,7 @@ struct RowCopy {
 //   SUMMARY: local end state from the given h, plus the sum of dt; no output.
 //   otherwise: outputs; BIDIR adds the midpoint exchange with the partner warp.
 template <typename T, int NS, int CPL, int NPOLY, bool SUMMARY, bool BIDIR, bool GATE, bool SOFTPLUS,
-          bool ORD>
+          bool ORD, bool CONV>
 __device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P,
                                              WarpSmem<T, NS, CPL> &sm, int b, int dbase, bool active,
                                              int s0, int s1, bool rev, float2 (&h)[CPL][NS / 2],
@@ -364,6 +364,30 @@ __device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P,
         }
         bias[c] = (active && P.bias) ? P.bias[d + c] : 0.f;
         Dd[c] = (active && P.D) ? P.D[d + c] : 0.f;
+    }
+
+    // CONV: x holds the conv input x_in; u = act(bias + sum_k w[k] x_in) over
+    // this and the previous 3 steps in scan order (weights right-aligned in
+    // cw, zero beyond the conv width).  xh[c][j] is x_in at scan offset
+    // -(3 - j); the window is preloaded from the steps before the segment.
+    float cw[CPL][4], cb[CPL], xh[CPL][3];
+    if (CONV) {
+        const int K = P.conv_k;
+#pragma unroll
+        for (int c = 0; c < CPL; c++) {
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                const int k = K - 4 + j;   // weight index for scan offset -(3 - j)
+                cw[c][j] = (active && k >= 0) ? P.conv_w[(size_t)(d + c) * K + k] : 0.f;
+            }
+            cb[c] = (active && P.conv_b) ? P.conv_b[d + c] : 0.f;
+#pragma unroll
+            for (int j = 0; j < 3; j++) {
+                const int off = 3 - j;   // steps before the segment's first
+                const int t = rev ? s1 - 1 + off : s0 - off;
+                xh[c][j] = (active && t >= 0 && t < a.L) ? ld1<T>(x, (rowbase + t) * a.D + d + c) : 0.f;
+            }
+        }
     }
 
     // midpoint of the pair exchange (see file comment)
@@ -444,6 +468,19 @@ __device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P,
         o.keep = !ORD || !tmask || tmask[rowbase + tpos(i)] != 0;
         float dv[CPL];
         IO<T, CPL>::ld(slot, o.xv);
+        if (CONV) {
+#pragma unroll
+            for (int c = 0; c < CPL; c++) {
+                float u = fmaf(cw[c][3], o.xv[c], cb[c]);
+#pragma unroll
+                for (int j = 0; j < 3; j++)
+                    u = fmaf(cw[c][j], xh[c][j], u);
+                xh[c][0] = xh[c][1];
+                xh[c][1] = xh[c][2];
+                xh[c][2] = o.xv[c];
+                o.xv[c] = P.conv_silu ? silu_f<T>(u) : u;
+            }
+        }
         IO<T, CPL>::ld(slot + WS::kRowB, dv);
         if (!SUMMARY && GATE)
             IO<T, CPL>::ld(slot + 2 * WS::kRowB, o.zv);
@@ -599,7 +636,7 @@ template <typename T, int NS, int CPL>
 constexpr int smem_bytes() { return kWarps * (int)sizeof(WarpSmem<T, NS, CPL>); }
 
 // ---------------------------------------------------------------- summary
-template <typename T, int NS, int CPL, int NPOLY, bool SOFTPLUS, bool ORD>
+template <typename T, int NS, int CPL, int NPOLY, bool SOFTPLUS, bool ORD, bool CONV>
 __global__ void __launch_bounds__(64, min_blocks<CPL>()) s6_summary_kernel(const S6Args a)
 {
     extern __shared__ __align__(16) char smem_raw[];
@@ -625,8 +662,9 @@ __global__ void __launch_bounds__(64, min_blocks<CPL>()) s6_summary_kernel(const
         for (int k = 0; k < NS / 2; k++)
             h[c][k] = make_float2(0.f, 0.f);
     }
-    scan_segment<T, NS, CPL, NPOLY, true, false, false, SOFTPLUS, ORD>(a, a.dir[dsel], sm[warp], b, dbase,
-                                                                       active, s0, s1, rev, h, sdt);
+    scan_segment<T, NS, CPL, NPOLY, true, false, false, SOFTPLUS, ORD, CONV>(a, a.dir[dsel], sm[warp], b,
+                                                                             dbase, active, s0, s1, rev, h,
+                                                                             sdt);
     if (!active)
         return;
 #pragma unroll
@@ -691,7 +729,7 @@ __global__ void s6_carry_kernel(const S6Args a)
 }
 
 // ------------------------------------------------------------------- main
-template <typename T, int NS, int CPL, int NPOLY, bool BIDIR, bool GATE, bool SOFTPLUS, bool ORD>
+template <typename T, int NS, int CPL, int NPOLY, bool BIDIR, bool GATE, bool SOFTPLUS, bool ORD, bool CONV>
 __global__ void __launch_bounds__(64, min_blocks<CPL>()) s6_main_kernel(const S6Args a)
 {
     extern __shared__ __align__(16) char smem_raw[];
@@ -727,8 +765,8 @@ __global__ void __launch_bounds__(64, min_blocks<CPL>()) s6_main_kernel(const S6
             h[c][k].y = (active && src && 2 * k + 1 < a.N) ? src[2 * k + 1] : 0.f;
         }
     }
-    scan_segment<T, NS, CPL, NPOLY, false, BIDIR, GATE, SOFTPLUS, ORD>(a, P, sm[warp], b, dbase, active,
-                                                                       s0, s1, rev, h, sdt);
+    scan_segment<T, NS, CPL, NPOLY, false, BIDIR, GATE, SOFTPLUS, ORD, CONV>(a, P, sm[warp], b, dbase,
+                                                                             active, s0, s1, rev, h, sdt);
     if (active && P.last_state && last_in_order(seg, a.S, rev)) {
 #pragma unroll
         for (int c = 0; c < CPL; c++) {
@@ -750,14 +788,14 @@ cudaError_t set_smem(KernelT k, int bytes)
     return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
-template <typename T, int NS, int CPL, int NPOLY, bool GATE, bool SOFTPLUS, bool ORD>
+template <typename T, int NS, int CPL, int NPOLY, bool GATE, bool SOFTPLUS, bool ORD, bool CONV>
 cudaError_t launch_typed(const S6Args &a, cudaStream_t st)
 {
     constexpr int smem = smem_bytes<T, NS, CPL>();
     constexpr int kCh = 32 * CPL;
     cudaError_t e;
     if (a.S > 1) {
-        auto ks = s6_summary_kernel<T, NS, CPL, SSM_S6_SUM_NPOLY(NS), SOFTPLUS, ORD>;
+        auto ks = s6_summary_kernel<T, NS, CPL, SSM_S6_SUM_NPOLY(NS), SOFTPLUS, ORD, CONV>;
         if ((e = set_smem(ks, smem)) != cudaSuccess)
             return e;
         dim3 g1((a.D + kWarps * kCh - 1) / (kWarps * kCh), a.S, a.Bsz * a.ndir);
@@ -766,13 +804,13 @@ cudaError_t launch_typed(const S6Args &a, cudaStream_t st)
         s6_carry_kernel<<<(unsigned)((tot + 255) / 256), 256, 0, st>>>(a);
     }
     if (a.ndir == 2) {
-        auto km = s6_main_kernel<T, NS, CPL, NPOLY, true, GATE, SOFTPLUS, ORD>;
+        auto km = s6_main_kernel<T, NS, CPL, NPOLY, true, GATE, SOFTPLUS, ORD, CONV>;
         if ((e = set_smem(km, smem)) != cudaSuccess)
             return e;
         dim3 g((a.D + kCh - 1) / kCh, a.S, a.Bsz);
         km<<<g, 64, smem, st>>>(a);
     } else {
-        auto km = s6_main_kernel<T, NS, CPL, NPOLY, false, GATE, SOFTPLUS, ORD>;
+        auto km = s6_main_kernel<T, NS, CPL, NPOLY, false, GATE, SOFTPLUS, ORD, CONV>;
         if ((e = set_smem(km, smem)) != cudaSuccess)
             return e;
         dim3 g((a.D + kWarps * kCh - 1) / (kWarps * kCh), a.S, a.Bsz);
@@ -784,11 +822,15 @@ cudaError_t launch_typed(const S6Args &a, cudaStream_t st)
 template <typename T, int NS, int NPOLY, bool GATE, bool SOFTPLUS>
 cudaError_t launch_cpl(const S6Args &a, cudaStream_t st)
 {
+    // three variants: plain, ordered / masked, conv input (not combined)
     if (a.order || a.mask)
-        return a.cpl == 1 ? launch_typed<T, NS, 1, NPOLY, GATE, SOFTPLUS, true>(a, st)
-                          : launch_typed<T, NS, 2, NPOLY, GATE, SOFTPLUS, true>(a, st);
-    return a.cpl == 1 ? launch_typed<T, NS, 1, NPOLY, GATE, SOFTPLUS, false>(a, st)
-                      : launch_typed<T, NS, 2, NPOLY, GATE, SOFTPLUS, false>(a, st);
+        return a.cpl == 1 ? launch_typed<T, NS, 1, NPOLY, GATE, SOFTPLUS, true, false>(a, st)
+                          : launch_typed<T, NS, 2, NPOLY, GATE, SOFTPLUS, true, false>(a, st);
+    if (a.conv)
+        return a.cpl == 1 ? launch_typed<T, NS, 1, NPOLY, GATE, SOFTPLUS, false, true>(a, st)
+                          : launch_typed<T, NS, 2, NPOLY, GATE, SOFTPLUS, false, true>(a, st);
+    return a.cpl == 1 ? launch_typed<T, NS, 1, NPOLY, GATE, SOFTPLUS, false, false>(a, st)
+                      : launch_typed<T, NS, 2, NPOLY, GATE, SOFTPLUS, false, false>(a, st);
 }
 
 #ifndef SSM_S6_NPOLY

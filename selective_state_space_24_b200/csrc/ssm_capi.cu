@@ -65,7 +65,7 @@ ssm::DirArgs dir_args(const ssm_dir_params &p)
 ssm_status run_s6(const ssm_dims *dims, const void *x, const void *delta, int softplus, int ndir,
                   int reverse, const ssm_dir_params *dirs, void *out, void *ws, size_t ws_bytes,
                   cudaStream_t stream, const float *initial_state = nullptr, const int32_t *order = nullptr,
-                  const unsigned char *mask = nullptr)
+                  const unsigned char *mask = nullptr, const ssm_conv_params *conv = nullptr)
 {
     const int dt = dims->dtype == SSM_F32 ? 0 : 1;
     const ssm::S6Plan plan =
@@ -96,6 +96,15 @@ ssm_status run_s6(const ssm_dims *dims, const void *x, const void *delta, int so
     a.dir[0].init = initial_state;   // single direction only
     a.order = order;
     a.mask = mask;
+    if (conv) {   // one ssm_conv_params per direction
+        a.conv = 1;
+        for (int i = 0; i < ndir; i++) {
+            a.dir[i].conv_w = conv[i].weight;
+            a.dir[i].conv_b = conv[i].bias;
+            a.dir[i].conv_k = conv[i].width;
+            a.dir[i].conv_silu = conv[i].silu ? 1 : 0;
+        }
+    }
     a.out = out;
     char *w = static_cast<char *>(ws);
     if (plan.S > 1) {
@@ -148,16 +157,29 @@ ssm_status ssm_scan_plan(const ssm_dims *dims, int bidirectional, int *segments,
 
 namespace {
 
+ssm_status check_conv(const ssm_conv_params *c)
+{
+    if (!c || !c->weight)
+        return SSM_ERR_INVALID_ARG;
+    if (c->width < 1 || c->width > 4)
+        return SSM_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(c->weight) || (c->bias && !aligned16(c->bias)))
+        return SSM_ERR_MISALIGNED;
+    return SSM_OK;
+}
+
 // Single-direction S6 with every option: the entry points below are this
 // with some options off.
 ssm_status scan_single(const ssm_dims *dims, const void *x, const void *delta, const float *delta_bias,
                        int delta_softplus, const float *A, const void *B, const void *C, const float *D,
                        const void *z, int reverse, const float *initial_state, const int32_t *order,
                        const unsigned char *mask, void *out, float *last_state, void *workspace,
-                       size_t workspace_bytes, void *stream)
+                       size_t workspace_bytes, void *stream, const ssm_conv_params *conv = nullptr)
 {
     ssm_status s = check_s6_dims(dims);
     if (s != SSM_OK)
+        return s;
+    if (conv && (s = check_conv(conv)) != SSM_OK)
         return s;
     if ((initial_state && !aligned16(initial_state)) || (last_state && !aligned16(last_state)))
         return SSM_ERR_MISALIGNED;
@@ -185,16 +207,18 @@ ssm_status scan_single(const ssm_dims *dims, const void *x, const void *delta, c
     if (!aligned16(x) || !aligned16(delta) || !aligned16(out))
         return SSM_ERR_MISALIGNED;
     return run_s6(dims, x, delta, delta_softplus, 1, reverse, &p, out, workspace, workspace_bytes, st,
-                  initial_state, order, mask);
+                  initial_state, order, mask, conv);
 }
 
 ssm_status scan_bidir(const ssm_dims *dims, const void *x, const void *delta, int delta_softplus,
                       const ssm_dir_params *fwd, const ssm_dir_params *bwd, const int32_t *order,
                       const unsigned char *mask, void *out, void *workspace, size_t workspace_bytes,
-                      void *stream)
+                      void *stream, const ssm_conv_params *conv = nullptr)
 {
     ssm_status s = check_s6_dims(dims);
     if (s != SSM_OK)
+        return s;
+    if (conv && ((s = check_conv(&conv[0])) != SSM_OK || (s = check_conv(&conv[1])) != SSM_OK))
         return s;
     if (!fwd || !bwd)
         return SSM_ERR_INVALID_ARG;
@@ -219,7 +243,7 @@ ssm_status scan_bidir(const ssm_dims *dims, const void *x, const void *delta, in
         return SSM_ERR_MISALIGNED;
     const ssm_dir_params dirs[2] = {*fwd, *bwd};
     return run_s6(dims, x, delta, delta_softplus, 2, 0, dirs, out, workspace, workspace_bytes, st, nullptr,
-                  order, mask);
+                  order, mask, conv);
 }
 
 }  // namespace
@@ -244,6 +268,30 @@ ssm_status ssm_scan_fwd_ordered(const ssm_dims *dims, const void *x, const void 
 {
     return scan_single(dims, x, delta, delta_bias, delta_softplus, A, B, C, D, z, reverse, nullptr, order,
                        mask, out, last_state, workspace, workspace_bytes, stream);
+}
+
+ssm_status ssm_scan_fwd_conv(const ssm_dims *dims, const void *x_in, const ssm_conv_params *conv,
+                             const void *delta, const float *delta_bias, int delta_softplus, const float *A,
+                             const void *B, const void *C, const float *D, const void *z, int reverse,
+                             void *out, float *last_state, void *workspace, size_t workspace_bytes,
+                             void *stream)
+{
+    if (!conv)
+        return SSM_ERR_INVALID_ARG;
+    return scan_single(dims, x_in, delta, delta_bias, delta_softplus, A, B, C, D, z, reverse, nullptr,
+                       nullptr, nullptr, out, last_state, workspace, workspace_bytes, stream, conv);
+}
+
+ssm_status bidir_scan_fwd_conv(const ssm_dims *dims, const void *x_in, const void *delta, int delta_softplus,
+                               const ssm_dir_params *fwd, const ssm_dir_params *bwd,
+                               const ssm_conv_params *conv_fwd, const ssm_conv_params *conv_bwd, void *out,
+                               void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (!conv_fwd || !conv_bwd)
+        return SSM_ERR_INVALID_ARG;
+    const ssm_conv_params conv[2] = {*conv_fwd, *conv_bwd};
+    return scan_bidir(dims, x_in, delta, delta_softplus, fwd, bwd, nullptr, nullptr, out, workspace,
+                      workspace_bytes, stream, conv);
 }
 
 ssm_status bidir_scan_fwd_ordered(const ssm_dims *dims, const void *x, const void *delta,

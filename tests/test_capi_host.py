@@ -169,3 +169,18 @@ def test_state_and_step_validation(lib):
     empty = _dims(0, 1, 16, 16)
     assert lib.ssm_step(ctypes.byref(empty), None, None, None, 1, None, None, None, None, None, None,
                         None, None) == 0
+
+
+def test_conv_validation(lib):
+    dims = _dims(2, 8, 16, 16)
+    bad = ssm.ssm_conv_params(FAKE, None, 5, 1)
+    assert lib.ssm_scan_fwd_conv(ctypes.byref(dims), FAKE, ctypes.byref(bad), FAKE, None, 1, FAKE, FAKE,
+                                 FAKE, None, None, 0, FAKE, None, None, 0, None) == 2
+    nul = ssm.ssm_conv_params(None, None, 3, 1)
+    assert lib.ssm_scan_fwd_conv(ctypes.byref(dims), FAKE, ctypes.byref(nul), FAKE, None, 1, FAKE, FAKE,
+                                 FAKE, None, None, 0, FAKE, None, None, 0, None) == 1
+    assert lib.ssm_scan_fwd_conv(ctypes.byref(dims), FAKE, None, FAKE, None, 1, FAKE, FAKE, FAKE, None,
+                                 None, 0, FAKE, None, None, 0, None) == 1
+    mis = ssm.ssm_conv_params(FAKE + 4, None, 3, 1)
+    assert lib.ssm_scan_fwd_conv(ctypes.byref(dims), FAKE, ctypes.byref(mis), FAKE, None, 1, FAKE, FAKE,
+                                 FAKE, None, None, 0, FAKE, None, None, 0, None) == 3
