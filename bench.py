@@ -60,9 +60,12 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
-    p.add_argument("--op", default="scan", choices=["scan", "step"],
-                   help="scan: the workload's scan (default); step: one decode step of a "
-                        "batch-512 x 1536-channel x 16-state fp32 state (ssm_step)")
+    p.add_argument("--op", default="scan", choices=["scan", "ordered", "conv", "step"],
+                   help="scan: the workload's scan (default); ordered: the same bidirectional "
+                        "workload along a random order of the positions with 30%% of the tokens "
+                        "masked; conv: the same with a width-4 conv1d + SiLU per direction computed "
+                        "inside the scan; step: one decode step of a batch-512 x 1536-channel x "
+                        "16-state fp32 state (ssm_step)")
     return p.parse_args()
 
 
@@ -189,11 +192,12 @@ class ClockSampler:
 class DeviceWorkload:
     """Inputs resident in HBM plus the raw C-ABI call of one step."""
 
-    def __init__(self, cfg, seed, device):
+    def __init__(self, cfg, seed, device, op="scan"):
         import torch
         import selective_state_space_24_b200 as ssm
         self.torch, self.ssm, self.dev = torch, ssm, device
         self.cfg = cfg
+        self.op = op
         self.info = workload_info(cfg)
         self.inp = ssm_gen.make_workload(cfg, seed=seed)
         self.lib = ssm.load()
@@ -228,6 +232,19 @@ class DeviceWorkload:
             need = self.lib.ssd_chunk_workspace_size(ctypes.byref(self.dims))
         self.ws = torch.empty(max(int(need), 16), dtype=torch.uint8, device=device)
         self.ws_bytes = int(need)
+        if op != "scan":
+            assert self.info["kind"] == "s6" and self.info["ndir"] == 2, "ordered / conv: bidirectional S6"
+            i = self.inp
+            rng = np.random.default_rng(seed + 1)
+            if op == "ordered":
+                self.order = torch.from_numpy(ssm_gen.order_random(i.seqlen, seed=seed)).to(device)
+                self.mask = torch.from_numpy(ssm_gen.token_mask(i.batch, i.seqlen, 0.7, seed=seed)).to(device)
+            else:
+                mk = lambda: torch.from_numpy((rng.standard_normal((i.dim, 4)) / 2).astype(np.float32)).to(device)
+                self.convw = (mk(), mk())
+                self.convb = torch.zeros(i.dim, device=device)
+                self.conv_f = ssm.ssm_conv_params(self.convw[0].data_ptr(), self.convb.data_ptr(), 4, 1)
+                self.conv_b = ssm.ssm_conv_params(self.convw[1].data_ptr(), self.convb.data_ptr(), 4, 1)
         self.launches_per_step = self._launches()
         self._bind()
 
@@ -251,7 +268,17 @@ class DeviceWorkload:
         """One call of the hot path through the C ABI (inputs resident)."""
         d, lib = self.d, self.lib
         p = lambda t: None if t is None else t.data_ptr()
-        if self.info["kind"] == "s6" and self.info["ndir"] == 2:
+        if self.op == "ordered":
+            st = lib.bidir_scan_fwd_ordered(ctypes.byref(self.dims), p(d["x"]), p(d["delta"]), 1,
+                                            ctypes.byref(self.fwd), ctypes.byref(self.bwd), p(self.order),
+                                            p(self.mask), p(self.out), p(self.ws), self.ws_bytes,
+                                            stream_handle)
+        elif self.op == "conv":
+            st = lib.bidir_scan_fwd_conv(ctypes.byref(self.dims), p(d["x"]), p(d["delta"]), 1,
+                                         ctypes.byref(self.fwd), ctypes.byref(self.bwd),
+                                         ctypes.byref(self.conv_f), ctypes.byref(self.conv_b), p(self.out),
+                                         p(self.ws), self.ws_bytes, stream_handle)
+        elif self.info["kind"] == "s6" and self.info["ndir"] == 2:
             st = lib.bidir_scan_fwd(ctypes.byref(self.dims), p(d["x"]), p(d["delta"]), 1,
                                     ctypes.byref(self.fwd), ctypes.byref(self.bwd), p(self.out),
                                     p(self.ws), self.ws_bytes, stream_handle)
@@ -288,7 +315,7 @@ def run_ours(args, rank, world, local_rank):
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
     info = workload_info(args.config)
-    wl = DeviceWorkload(args.config, seed=rank_seed(rank), device=device)
+    wl = DeviceWorkload(args.config, seed=rank_seed(rank), device=device, op=args.op)
     stream = torch.cuda.current_stream(device)
     sh = stream.cuda_stream
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
@@ -333,13 +360,13 @@ def run_ours(args, rank, world, local_rank):
     t_alu = info["elems"] / alu_peak
     if info["kind"] == "s6" and t_alu > t_hbm:
         roof = {"bound": "alu", "achieved": alu_ach / 1e9, "peak": alu_peak / 1e9,
-                "unit": "Gelem/s", "frac": alu_ach / alu_peak, "traffic": NCU_TRAFFIC.get(args.config),
+                "unit": "Gelem/s", "frac": alu_ach / alu_peak, "traffic": NCU_TRAFFIC.get(args.config) if args.op == "scan" else None,
                 "hbm_achieved_gbs": hbm_ach, "hbm_peak_gbs": peaks["hbm_gbs"],
                 "hbm_frac": hbm_ach / peaks["hbm_gbs"], "peak_source": peak_src,
                 "algorithmic_bytes": info["bytes"], "kernel_ms_median": kern_s * 1e3}
     else:
         roof = {"bound": "hbm", "achieved": hbm_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": hbm_ach / peaks["hbm_gbs"], "traffic": NCU_TRAFFIC.get(args.config),
+                "frac": hbm_ach / peaks["hbm_gbs"], "traffic": NCU_TRAFFIC.get(args.config) if args.op == "scan" else None,
                 "peak_source": peak_src,
                 "algorithmic_bytes": info["bytes"], "kernel_ms_median": kern_s * 1e3}
 
@@ -364,7 +391,7 @@ def run_ours(args, rank, world, local_rank):
                "ms_per_step": ems / ke}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.op == "scan":
         cpu = cpu_baseline(args.config, budget_s=10.0)
 
     res = {
@@ -373,7 +400,8 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32" if info["dtype"] == "f32" else "bf16 storage, f32 compute",
         "data": "synthetic (seeded ssm_gen inputs with the workload's shapes and distributions)",
-        "config": {"workload": info["name"], "config_index": args.config,
+        "config": {"workload": info["name"] + ("" if args.op == "scan" else "_" + args.op),
+                   "config_index": args.config, "op": args.op,
                    **{k: info[k] for k in ("batch", "seqlen", "dim", "dstate", "nheads", "headdim",
                                            "chunk") if k in info},
                    "directions": info["ndir"], "parallelism": f"dp{world} (independent batches)",
