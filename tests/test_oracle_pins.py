@@ -522,3 +522,48 @@ def test_conv_scan_identity_kernel_is_plain_scan():
     y0, st0 = oracle.s6_arrays(x, delta, A, B, C, delta_bias=bias, D=D, z=z)
     _close(y, y0)
     _close(st, st0)
+
+
+# ------------------------------------------------ gradients of the scan
+
+from oracle import grads as ograds  # noqa: E402
+
+
+@pytest.mark.parametrize("reverse", [False, True])
+def test_grad_forward_is_the_scan(reverse):
+    rng = np.random.default_rng(600 + reverse)
+    x, delta, bias, A, B, C, D, z = _rand_case(rng, 2, 7, 3, 4)
+    g = ograds.s6_grads(x, delta, A, B, C, np.ones_like(x), delta_bias=bias, D=D, z=z, reverse=reverse)
+    y, _ = oracle.s6_arrays(x, delta, A, B, C, delta_bias=bias, D=D, z=z, reverse=reverse)
+    _close(g["out"], y)
+
+
+@pytest.mark.parametrize("reverse", [False, True])
+@pytest.mark.parametrize("gate", [False, True])
+def test_grads_match_finite_differences(reverse, gate):
+    """Every gradient against central finite differences of the C oracle's
+    forward (h = 1e-6; agreement to 1e-6 relative to the gradient's size)."""
+    rng = np.random.default_rng(610 + reverse + 2 * gate)
+    x, delta, bias, A, B, C, D, z = _rand_case(rng, 1, 5, 2, 3, gate=gate)
+    dout = rng.standard_normal(x.shape)
+    g = ograds.s6_grads(x, delta, A, B, C, dout, delta_bias=bias, D=D, z=z, reverse=reverse)
+    args = dict(x=x, delta=delta, A=A, B=B, C=C, D=D, z=z, delta_bias=bias)
+
+    def loss(a):
+        y, _ = oracle.s6_arrays(a["x"], a["delta"], a["A"], a["B"], a["C"], delta_bias=a["delta_bias"],
+                                D=a["D"], z=a["z"], reverse=reverse)
+        return float(np.sum(y * dout))
+
+    eps = 1e-6
+    for k, v in args.items():
+        if v is None:
+            continue
+        num = np.zeros_like(v)
+        for idx in np.ndindex(v.shape):
+            a1 = {kk: (vv.copy() if vv is not None else None) for kk, vv in args.items()}
+            a2 = {kk: (vv.copy() if vv is not None else None) for kk, vv in args.items()}
+            a1[k][idx] += eps
+            a2[k][idx] -= eps
+            num[idx] = (loss(a1) - loss(a2)) / (2 * eps)
+        scale = max(np.max(np.abs(num)), 1e-8)
+        assert np.max(np.abs(g[k] - num)) / scale < 1e-6, k
