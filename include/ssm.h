@@ -287,6 +287,32 @@ SSM_API ssm_status bidir_scan_fwd_conv(const ssm_dims *dims, const void *x_in, c
                                        const ssm_conv_params *conv_bwd, void *out, void *workspace,
                                        size_t workspace_bytes, void *stream);
 
+/* Bytes of device workspace ssm_scan_bwd needs for `dims` (0 for invalid dims). */
+SSM_API size_t ssm_scan_bwd_workspace_size(const ssm_dims *dims);
+
+/*
+ * Gradients of ssm_scan_fwd (same dims and inputs, same reverse flag) for
+ * an incoming gradient dout of out -- the training use of the Mamba2 page,
+ * sec. 5.1, which backpropagates through the scan.  The states are
+ * recomputed (a forward pass stores h every 8 steps in the workspace), so
+ * nothing from the forward call is needed.  All gradients are float32:
+ *   dout            (B, L, D) dtype, required
+ *   dx, ddelta      (B, L, D), required, written
+ *   dA (D, N), dB, dC (B, L, N): required, written
+ *   dD (D), dz (B, L, D), ddelta_bias (D): required when D, z, delta_bias
+ *                   are given (else ignored), written
+ * ddelta is the gradient of the raw delta (through the softplus when
+ * delta_softplus is set).  dB, dC sum over the channels, dA, dD and
+ * ddelta_bias over the batch and the sequence.  Workspace:
+ * ssm_scan_bwd_workspace_size(dims) bytes.  Errors as for ssm_scan_fwd.
+ */
+SSM_API ssm_status ssm_scan_bwd(const ssm_dims *dims, const void *x, const void *delta,
+                                const float *delta_bias, int delta_softplus, const float *A,
+                                const void *B, const void *C, const float *D, const void *z,
+                                int reverse, const void *dout, float *dx, float *ddelta, float *dA,
+                                float *dB, float *dC, float *dD, float *dz, float *ddelta_bias,
+                                void *workspace, size_t workspace_bytes, void *stream);
+
 /* SSD problem size.  Supported: dtype SSM_BF16, headdim 64, dstate 128,
  * chunk 64, seqlen any value >= 0 (a short last chunk is handled). */
 typedef struct {

@@ -9,6 +9,7 @@ Entry points (names as in include/ssm.h):
 
 * ``ssm_scan_fwd(x, delta, A, B, C, ...)``  single-direction S6 scan
 * ``ssm_scan_fwd_state(...)``  the same from a given initial state
+* ``ssm_scan_bwd(x, delta, A, B, C, dout, ...)``  gradients of ssm_scan_fwd
 * ``ssm_step(x, delta, A, B, C, state, ...)``  one decode step, state in place
 * ``ssm_scan_fwd_ordered`` / ``bidir_scan_fwd_ordered``  scans along a given
   order of the positions, with an optional token mask
@@ -88,6 +89,9 @@ SIGNATURES = {
                                    ctypes.POINTER(ssm_dir_params), ctypes.POINTER(ssm_dir_params),
                                    ctypes.POINTER(ssm_conv_params), ctypes.POINTER(ssm_conv_params),
                                    _vp, _vp, _sz, _vp]),
+    "ssm_scan_bwd_workspace_size": (_sz, [ctypes.POINTER(ssm_dims)]),
+    "ssm_scan_bwd": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp, _vp, _int,
+                            _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "ssm_step": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp, _vp, _vp,
                         _vp, _vp]),
     "ssm_scan_fwd_noalloc": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp,
@@ -331,6 +335,35 @@ def bidir_scan_fwd_conv(x_in, delta, fwd: DirParams, bwd: DirParams, conv_fwd: C
                                  _stream_handle(stream))
     _check(st, "bidir_scan_fwd_conv")
     return out
+
+
+def ssm_scan_bwd(x, delta, A, B, C, dout, *, delta_bias=None, delta_softplus=True, D=None, z=None,
+                 reverse=False, stream=None):
+    """Gradients of ssm_scan_fwd for the incoming gradient dout: returns a
+    dict of float32 tensors dx, ddelta, dA, dB, dC and, when the input was
+    given, dD, dz, ddelta_bias."""
+    torch = _torch()
+    lib = capi()
+    dims = s6_dims(x, A.shape[1])
+    f32 = dict(dtype=torch.float32, device=x.device)
+    g = {"dx": torch.empty(x.shape, **f32), "ddelta": torch.empty(x.shape, **f32),
+         "dA": torch.empty(A.shape, **f32), "dB": torch.empty(B.shape, **f32),
+         "dC": torch.empty(C.shape, **f32)}
+    if D is not None:
+        g["dD"] = torch.empty(D.shape, **f32)
+    if z is not None:
+        g["dz"] = torch.empty(x.shape, **f32)
+    if delta_bias is not None:
+        g["ddelta_bias"] = torch.empty(delta_bias.shape, **f32)
+    ws = workspace(lib.ssm_scan_bwd_workspace_size(ctypes.byref(dims)), x.device)
+    st = lib.ssm_scan_bwd(ctypes.byref(dims), _ptr(x), _ptr(delta), _ptr(delta_bias),
+                          int(bool(delta_softplus)), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+                          int(bool(reverse)), _ptr(dout), _ptr(g["dx"]), _ptr(g["ddelta"]), _ptr(g["dA"]),
+                          _ptr(g["dB"]), _ptr(g["dC"]), _ptr(g.get("dD")), _ptr(g.get("dz")),
+                          _ptr(g.get("ddelta_bias")), _ptr(ws), 0 if ws is None else ws.numel(),
+                          _stream_handle(stream))
+    _check(st, "ssm_scan_bwd")
+    return g
 
 
 def ssm_step(x, delta, A, B, C, state, *, delta_bias=None, delta_softplus=True, D=None, z=None,

@@ -82,6 +82,24 @@ struct StepArgs {
 };
 cudaError_t launch_step(const StepArgs &a, cudaStream_t stream);
 
+// Gradients of one single-direction S6 call (all float32).  dB, dC, dA, dD,
+// dbias are accumulated with atomics and must be zeroed by the caller;
+// dx, ddelta are written, or added to when accumulate is set (the second
+// direction of a bidirectional backward).
+struct BwdArgs {
+    int Bsz, L, D, N;
+    int dtype;      // 0 = float32, 1 = bf16 (inputs and dout)
+    int softplus;
+    int reverse;
+    int accumulate;
+    const void *x, *delta, *B, *C, *z, *dout;
+    const float *bias, *A, *Dskip;
+    float *dx, *ddelta, *dz, *dA, *dB, *dC, *dD, *dbias;
+    float *ckpt;    // workspace: (Bsz, ceil(L / 8), D, N) states entering each 8-step chunk
+};
+size_t bwd_workspace_bytes(int64_t Bsz, int64_t L, int64_t D, int64_t N);
+cudaError_t launch_bwd(const BwdArgs &a, cudaStream_t stream);
+
 // One SSD call.
 struct SSDArgs {
     int Bsz, L, H, P, N, Q;

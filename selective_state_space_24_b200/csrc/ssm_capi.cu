@@ -314,6 +314,84 @@ ssm_status ssm_scan_fwd(const ssm_dims *dims, const void *x, const void *delta,
                               out, last_state, workspace, workspace_bytes, stream);
 }
 
+size_t ssm_scan_bwd_workspace_size(const ssm_dims *dims)
+{
+    if (check_s6_dims(dims) != SSM_OK || empty_s6(dims))
+        return 0;
+    return ssm::bwd_workspace_bytes(dims->batch, dims->seqlen, dims->dim, dims->dstate);
+}
+
+ssm_status ssm_scan_bwd(const ssm_dims *dims, const void *x, const void *delta, const float *delta_bias,
+                        int delta_softplus, const float *A, const void *B, const void *C, const float *D,
+                        const void *z, int reverse, const void *dout, float *dx, float *ddelta, float *dA,
+                        float *dB, float *dC, float *dD, float *dz, float *ddelta_bias, void *workspace,
+                        size_t workspace_bytes, void *stream)
+{
+    ssm_status s = check_s6_dims(dims);
+    if (s != SSM_OK)
+        return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t nDN = (size_t)dims->dim * dims->dstate;
+    if (empty_s6(dims)) {
+        // no step: every gradient is zero (the ones over (D, N) and (D) too)
+        if (dA && nDN && cudaMemsetAsync(dA, 0, nDN * sizeof(float), st) != cudaSuccess)
+            return SSM_ERR_CUDA;
+        if (D && dD && dims->dim && cudaMemsetAsync(dD, 0, dims->dim * sizeof(float), st) != cudaSuccess)
+            return SSM_ERR_CUDA;
+        if (delta_bias && ddelta_bias && dims->dim &&
+            cudaMemsetAsync(ddelta_bias, 0, dims->dim * sizeof(float), st) != cudaSuccess)
+            return SSM_ERR_CUDA;
+        return SSM_OK;
+    }
+    if (!x || !delta || !A || !B || !C || !dout || !dx || !ddelta || !dA || !dB || !dC)
+        return SSM_ERR_INVALID_ARG;
+    if ((D && !dD) || (z && !dz) || (delta_bias && !ddelta_bias))
+        return SSM_ERR_INVALID_ARG;
+    const void *ptrs[] = {x, delta, delta_bias, A, B, C, D, z, dout, dx, ddelta, dA, dB, dC, dD, dz,
+                          ddelta_bias, workspace};
+    for (const void *q : ptrs)
+        if (q && !aligned16(q))
+            return SSM_ERR_MISALIGNED;
+    const size_t need = ssm::bwd_workspace_bytes(dims->batch, dims->seqlen, dims->dim, dims->dstate);
+    if (!workspace || workspace_bytes < need)
+        return SSM_ERR_WORKSPACE_TOO_SMALL;
+    const size_t nBLN = (size_t)dims->batch * dims->seqlen * dims->dstate;
+    if (cudaMemsetAsync(dA, 0, nDN * sizeof(float), st) != cudaSuccess ||
+        cudaMemsetAsync(dB, 0, nBLN * sizeof(float), st) != cudaSuccess ||
+        cudaMemsetAsync(dC, 0, nBLN * sizeof(float), st) != cudaSuccess ||
+        (D && cudaMemsetAsync(dD, 0, dims->dim * sizeof(float), st) != cudaSuccess) ||
+        (delta_bias && cudaMemsetAsync(ddelta_bias, 0, dims->dim * sizeof(float), st) != cudaSuccess))
+        return SSM_ERR_CUDA;
+    ssm::BwdArgs a;
+    memset(&a, 0, sizeof(a));
+    a.Bsz = (int)dims->batch;
+    a.L = (int)dims->seqlen;
+    a.D = (int)dims->dim;
+    a.N = (int)dims->dstate;
+    a.dtype = dims->dtype == SSM_F32 ? 0 : 1;
+    a.softplus = delta_softplus ? 1 : 0;
+    a.reverse = reverse ? 1 : 0;
+    a.x = x;
+    a.delta = delta;
+    a.B = B;
+    a.C = C;
+    a.z = z;
+    a.dout = dout;
+    a.bias = delta_bias;
+    a.A = A;
+    a.Dskip = D;
+    a.dx = dx;
+    a.ddelta = ddelta;
+    a.dz = z ? dz : nullptr;
+    a.dA = dA;
+    a.dB = dB;
+    a.dC = dC;
+    a.dD = D ? dD : nullptr;
+    a.dbias = delta_bias ? ddelta_bias : nullptr;
+    a.ckpt = static_cast<float *>(workspace);
+    return ssm::launch_bwd(a, st) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
 ssm_status ssm_step(const ssm_dims *dims, const void *x, const void *delta, const float *delta_bias,
                     int delta_softplus, const float *A, const void *B, const void *C, const float *D,
                     const void *z, float *state, void *out, void *stream)

@@ -1,0 +1,74 @@
+"""GPU parity of the S6 backward pass (ssm_scan_bwd) against the float64
+autograd oracle (oracle/grads.py), through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import ssm_gen
+import selective_state_space_24_b200 as ssm
+from oracle import grads as ograds
+from gpu_util import TOL, dev, f32dev, rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib(cuda_device):
+    ssm.load()
+
+
+def _run(inp, dtype, dout, reverse, gate=True, D=True, bias=True, softplus=True):
+    g = ssm.ssm_scan_bwd(dev(inp.x, dtype), dev(inp.delta, dtype), f32dev(inp.A_f), dev(inp.B_f, dtype),
+                         dev(inp.C_f, dtype), dev(dout, dtype),
+                         delta_bias=f32dev(inp.dt_bias_f) if bias else None, delta_softplus=softplus,
+                         D=f32dev(inp.D_f) if D else None, z=dev(inp.z_f, dtype) if gate else None,
+                         reverse=reverse)
+    torch.cuda.synchronize()
+    ref = ograds.s6_grads(inp.x, inp.delta, inp.A_f, inp.B_f, inp.C_f, dout,
+                          delta_bias=inp.dt_bias_f if bias else None, softplus=softplus,
+                          D=inp.D_f if D else None, z=inp.z_f if gate else None, reverse=reverse)
+    return g, ref
+
+
+def _check(g, ref, tol):
+    names = {"dx": "x", "ddelta": "delta", "dA": "A", "dB": "B", "dC": "C", "dD": "D", "dz": "z",
+             "ddelta_bias": "delta_bias"}
+    for k, t in g.items():
+        e = rel_err(t.cpu().numpy(), ref[names[k]])
+        assert e <= tol, f"{k}: rel err {e:.3e}"
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("reverse", [False, True])
+@pytest.mark.parametrize("N", [16, 5])
+def test_bwd_matches_autograd(dtype, reverse, N):
+    """Every gradient; L = 101 leaves a ragged last 8-step chunk, D = 96
+    leaves a CTA of 64 channels half full."""
+    inp = ssm_gen.make_s6_inputs(2, 101, 96, N, dtype=dtype, seed=N + reverse, random_A=True,
+                                 random_D=True)
+    dout = np.random.default_rng(N).standard_normal(inp.x.shape).astype(np.float32)
+    if dtype == "bf16":
+        dout = ssm_gen.round_to_bf16(dout)
+    g, ref = _run(inp, dtype, dout, reverse)
+    _check(g, ref, TOL[dtype])
+
+
+@pytest.mark.parametrize("gate,D,bias,softplus", [(False, True, True, True), (True, False, False, True),
+                                                  (True, True, False, False)])
+def test_bwd_optional_inputs(gate, D, bias, softplus):
+    inp = ssm_gen.make_s6_inputs(1, 64, 32, 16, dtype="f32", seed=3, random_A=True, random_D=True)
+    if not softplus:   # keep dt positive without the softplus
+        inp.delta = np.abs(inp.delta) * 0.1
+    dout = np.random.default_rng(4).standard_normal(inp.x.shape).astype(np.float32)
+    g, ref = _run(inp, "f32", dout, False, gate=gate, D=D, bias=bias, softplus=softplus)
+    assert ("dz" in g) == gate and ("dD" in g) == D and ("ddelta_bias" in g) == bias
+    _check(g, ref, TOL["f32"])
+
+
+def test_bwd_long_sequence():
+    """A longer sequence (many checkpointed chunks), sampled against the
+    oracle on one batch row."""
+    inp = ssm_gen.make_s6_inputs(1, 1000, 64, 16, dtype="f32", seed=8, random_A=True, random_D=True)
+    dout = np.random.default_rng(9).standard_normal(inp.x.shape).astype(np.float32)
+    g, ref = _run(inp, "f32", dout, False)
+    _check(g, ref, TOL["f32"])
