@@ -60,12 +60,13 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
-    p.add_argument("--op", default="scan", choices=["scan", "ordered", "conv", "step"],
+    p.add_argument("--op", default="scan", choices=["scan", "ordered", "conv", "step", "bwd"],
                    help="scan: the workload's scan (default); ordered: the same bidirectional "
                         "workload along a random order of the positions with 30%% of the tokens "
                         "masked; conv: the same with a width-4 conv1d + SiLU per direction computed "
                         "inside the scan; step: one decode step of a batch-512 x 1536-channel x "
-                        "16-state fp32 state (ssm_step)")
+                        "16-state fp32 state (ssm_step); bwd: the gradients (ssm_scan_bwd) of the "
+                        "forward direction of the workload")
     return p.parse_args()
 
 
@@ -490,6 +491,88 @@ def run_step(args):
     }
 
 
+# ---------------------------------------------------------- backward
+
+def run_bwd(args):
+    """Gradients (ssm_scan_bwd) of the forward direction of an S6 workload,
+    inputs and the incoming gradient resident, L2 flushed before every step,
+    CUDA events on the launching stream."""
+    import ctypes
+    import torch
+    from selective_state_space_24_b200 import build as ssm_build
+    import selective_state_space_24_b200 as ssm
+    ssm_build.build()
+    lib = ssm.load()
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    info = workload_info(args.config)
+    assert info["kind"] == "s6", "bwd: an S6 workload"
+    inp = ssm_gen.make_workload(args.config, seed=0)
+    tdt = torch.float32 if inp.dtype == "f32" else torch.bfloat16
+    io = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(tdt).to(device)
+    f32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device)
+    x, delta, z, Bm, Cm = io(inp.x), io(inp.delta), io(inp.z_f), io(inp.B_f), io(inp.C_f)
+    dout = io(np.random.default_rng(1).standard_normal(inp.x.shape))
+    A, bias, Dv = f32(inp.A_f), f32(inp.dt_bias_f), f32(inp.D_f)
+    e = lambda shape: torch.empty(shape, dtype=torch.float32, device=device)
+    g = [e(x.shape), e(x.shape), e(A.shape), e(Bm.shape), e(Cm.shape), e(Dv.shape), e(x.shape),
+         e(bias.shape)]
+    dims = ssm.ssm_dims(inp.batch, inp.seqlen, inp.dim, inp.dstate,
+                        ssm.SSM_F32 if inp.dtype == "f32" else ssm.SSM_BF16)
+    need = int(lib.ssm_scan_bwd_workspace_size(ctypes.byref(dims)))
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=device)
+    p = lambda t: t.data_ptr()
+    stream = torch.cuda.current_stream(device)
+    sh = stream.cuda_stream
+
+    def step():
+        st = lib.ssm_scan_bwd(ctypes.byref(dims), p(x), p(delta), p(bias), 1, p(A), p(Bm), p(Cm), p(Dv),
+                              p(z), 0, p(dout), *[p(t) for t in g], p(ws), need, sh)
+        if st != 0:
+            raise RuntimeError(f"ssm_scan_bwd returned {ssm.STATUS.get(st, st)}")
+
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    for _ in range(max(args.warmup, 3)):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    sampler = ClockSampler(0)
+    sampler.start()
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = [a.elapsed_time(b) for a, b in evs]
+    med = statistics.median(ms)
+    elems = inp.batch * inp.seqlen * inp.dim * inp.dstate
+    es = 4 if inp.dtype == "f32" else 2
+    BL, BLD = inp.batch * inp.seqlen, inp.batch * inp.seqlen * inp.dim
+    # inputs x, delta, z, dout (dtype), B, C; outputs dx, ddelta, dz (fp32), dB, dC (fp32)
+    nbytes = 4 * BLD * es + 2 * BL * inp.dstate * es + 3 * BLD * 4 + 2 * BL * inp.dstate * 4
+    peaks, peak_src = load_peaks()
+    alu_peak = alu_peak_elems(peaks.get("sm_max_mhz", 1965.0))
+    return {
+        "metric": "backward: scan elements/s (B·L·D·N)", "value": elems / (med * 1e-3),
+        "unit": "elements/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": sum(ms) / len(ms), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": info["dtype"], "data": "synthetic (seeded ssm_gen inputs)",
+        "config": {"workload": info["name"] + "_fwd_direction_bwd", "config_index": args.config,
+                   "l2": "flushed before every timed step (512 MB write)",
+                   "algorithmic_bytes_per_step": nbytes, "elements_per_step": elems},
+        "hbm_gbs": nbytes / (med * 1e-3) / 1e9,
+        "roofline": {"bound": "alu", "achieved": elems / (med * 1e-3) / 1e9, "peak": alu_peak / 1e9,
+                     "unit": "Gelem/s", "frac": elems / (med * 1e-3) / alu_peak, "traffic": None,
+                     "peak_source": peak_src, "kernel_ms_median": med,
+                     "note": "three exps per element (checkpoint pass, recompute, adjoint)"},
+        "gpu_launches": 2 * args.steps, "clocks": clocks,
+    }
+
+
 # ------------------------------------------------------------ CPU oracle
 
 def _oracle_sample(cfg, frac_cols):
@@ -587,9 +670,9 @@ def main():
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
         return
-    if args.op == "step":
+    if args.op in ("step", "bwd"):
         if rank == 0:
-            print(json.dumps(run_step(args)), flush=True)
+            print(json.dumps(run_step(args) if args.op == "step" else run_bwd(args)), flush=True)
         return
     if world > 1:
         import datetime
