@@ -47,8 +47,8 @@ L2_FLUSH_BYTES = 512 << 20
 SMS = 148
 # DRAM bytes (read + write) per launch of the dominant kernel, from one ncu
 # capture of the current kernels (profiles/s6_main_vim_small_bidir_fp32.md,
-# profiles/ssd_chunk_mamba2_bf16.md); None where no capture matches them.
-NCU_TRAFFIC = {4: 398.97e6}
+# profiles/ssd_chunk_mamba2_bf16.md); absent where no capture matches them.
+NCU_TRAFFIC = {1: 271.65e6, 4: 398.97e6}
 
 
 def parse():

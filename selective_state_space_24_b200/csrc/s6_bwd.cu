@@ -20,8 +20,10 @@
 // chunks backwards: it recomputes the chunk's states into shared memory
 // from the checkpoint, then sweeps the chunk backwards with lam in
 // registers.  One thread per (b, d); a CTA holds 64 channels of one batch
-// row, and sums dB, dC over them in shared memory before one atomic add
-// per (t, n).  All gradients are float32.
+// row and stages each chunk's B and C rows in shared memory; the per-step
+// inputs of a chunk are loaded together before its work.  dB and dC are
+// summed over a warp's 32 channels with a butterfly of shuffles, then added
+// with one atomic per (warp, t, n).  All gradients are float32.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -45,41 +47,95 @@ template <> __device__ __forceinline__ float ldv<__nv_bfloat16>(const __nv_bfloa
 __device__ __forceinline__ float dt_of(float v, int softplus) { return softplus ? softplus_f(v) : v; }
 __device__ __forceinline__ float sigmoid_f(float v) { return 1.f / (1.f + ex2_mufu(-v * kLog2e)); }
 
+// B (and C) rows of steps [i0, i0 + kKc) in scan order into shared memory:
+// bc[k][n] for B, bc[k][NS + n] for C (zero past L or N).  Whole CTA.
+template <typename T, int NS, bool WITH_C>
+__device__ __forceinline__ void stage_bc(const BwdArgs &a, int b, int i0, float (*bc)[2 * NS])
+{
+    const T *Bm = static_cast<const T *>(a.B), *Cm = static_cast<const T *>(a.C);
+    constexpr int kVals = kKc * (WITH_C ? 2 : 1) * NS;
+    for (int j = threadIdx.x; j < kVals; j += kCta) {
+        const int k = j / ((WITH_C ? 2 : 1) * NS), r = j % ((WITH_C ? 2 : 1) * NS);
+        const int n = r % NS, i = i0 + k;
+        float v = 0.f;
+        if (i < a.L && n < a.N) {
+            const int t = a.reverse ? a.L - 1 - i : i;
+            v = ldv(r < NS ? Bm : Cm, ((size_t)b * a.L + t) * a.N + n);
+        }
+        bc[k][r] = v;
+    }
+}
+
+// Sum v[0..31] over the 32 lanes of the warp: afterwards lane j holds the
+// sum of every lane's v[j] (butterfly: at each stage a lane keeps one half of
+// its values -- the upper half if its lane bit is set -- and adds the
+// partner's copy of that half).
+__device__ __forceinline__ float warp_transpose_sum(float (&v)[32])
+{
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        const bool up = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < o; i++) {
+            const float send = up ? v[i] : v[i + o];
+            const float keep = up ? v[i + o] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+    }
+    return v[0];
+}
+
 template <typename T, int NS>
 __global__ void __launch_bounds__(kCta) s6_bwd_ckpt_kernel(const BwdArgs a)
 {
+    __shared__ float bc[kKc][2 * NS];
     const int d = blockIdx.x * kCta + threadIdx.x;
     const int b = blockIdx.y;
-    if (d >= a.D)
-        return;
+    const bool active = d < a.D;
+    const int dd = active ? d : 0;
     const int N = a.N, L = a.L, nch = (L + kKc - 1) / kKc;
     const T *x = static_cast<const T *>(a.x), *dl = static_cast<const T *>(a.delta);
-    const T *Bm = static_cast<const T *>(a.B);
     float Al[NS], h[NS];
 #pragma unroll
     for (int n = 0; n < NS; n++) {
-        Al[n] = n < N ? a.A[(size_t)d * N + n] * kLog2e : 0.f;
+        Al[n] = (active && n < N) ? a.A[(size_t)dd * N + n] * kLog2e : 0.f;
         h[n] = 0.f;
     }
-    const float bias = a.bias ? a.bias[d] : 0.f;
+    const float bias = (active && a.bias) ? a.bias[dd] : 0.f;
     for (int c = 0; c < nch; c++) {
-        float *ck = a.ckpt + (((size_t)b * nch + c) * a.D + d) * N;
-#pragma unroll
-        for (int n = 0; n < NS; n++)
-            if (n < N)
-                ck[n] = h[n];
-        for (int k = 0; k < kKc; k++) {
-            const int i = c * kKc + k;
-            if (i >= L)
-                break;
-            const int t = a.reverse ? L - 1 - i : i;
-            const size_t row = (size_t)b * L + t;
-            const float dt = dt_of(ldv(dl, row * a.D + d) + bias, a.softplus);
-            const float dtx = dt * ldv(x, row * a.D + d);
+        const int i0 = c * kKc;
+        if (active) {
+            float *ck = a.ckpt + (((size_t)b * nch + c) * a.D + dd) * N;
 #pragma unroll
             for (int n = 0; n < NS; n++)
                 if (n < N)
-                    h[n] = fmaf(ex2_mufu(dt * Al[n]), h[n], dtx * ldv(Bm, row * N + n));
+                    ck[n] = h[n];
+        }
+        // this chunk's per-step scalars, all loads issued together
+        float dtk[kKc], xk[kKc];
+#pragma unroll
+        for (int k = 0; k < kKc; k++) {
+            const int i = i0 + k;
+            dtk[k] = 0.f;
+            xk[k] = 0.f;
+            if (active && i < L) {
+                const int t = a.reverse ? L - 1 - i : i;
+                const size_t io = ((size_t)b * L + t) * a.D + dd;
+                dtk[k] = ldv(dl, io);
+                xk[k] = ldv(x, io);
+            }
+        }
+        __syncthreads();   // the previous chunk is done with bc
+        stage_bc<T, NS, false>(a, b, i0, bc);
+        __syncthreads();
+#pragma unroll
+        for (int k = 0; k < kKc; k++) {
+            const float dt = (i0 + k < L) ? dt_of(dtk[k] + bias, a.softplus) : 0.f;
+            const float dtx = dt * xk[k];
+#pragma unroll
+            for (int n = 0; n < NS; n++)
+                h[n] = fmaf(ex2_mufu(dt * Al[n]), h[n], dtx * bc[k][n]);
         }
     }
 }
@@ -87,17 +143,18 @@ __global__ void __launch_bounds__(kCta) s6_bwd_ckpt_kernel(const BwdArgs a)
 template <typename T, int NS>
 __global__ void __launch_bounds__(kCta) s6_bwd_kernel(const BwdArgs a)
 {
-    // states of the current chunk: hs[k][n][thread]; channel sums: red[thread][2 NS + 1]
+    // states of the current chunk: hs[k][n][thread]; the chunk's B and C
+    // rows; this thread's per-step scalars sc[k][dt, x, dout, z][thread]
     __shared__ float hs[kKc][NS][kCta];
-    __shared__ float red[kCta][2 * NS + 1];
-    const int tid = threadIdx.x;
+    __shared__ float bc[kKc][2 * NS];
+    __shared__ float sc[kKc][5][kCta];
+    const int tid = threadIdx.x, lane = tid & 31;
     const int d = blockIdx.x * kCta + tid;
     const int b = blockIdx.y;
     const bool active = d < a.D;
     const int dd = active ? d : 0;
     const int N = a.N, L = a.L, nch = (L + kKc - 1) / kKc;
     const T *x = static_cast<const T *>(a.x), *dl = static_cast<const T *>(a.delta);
-    const T *Bm = static_cast<const T *>(a.B), *Cm = static_cast<const T *>(a.C);
     const T *zp = static_cast<const T *>(a.z), *go = static_cast<const T *>(a.dout);
     float A[NS], Al[NS], lam[NS], gA[NS];
 #pragma unroll
@@ -113,99 +170,103 @@ __global__ void __launch_bounds__(kCta) s6_bwd_kernel(const BwdArgs a)
 
     for (int c = nch - 1; c >= 0; c--) {
         const int i0 = c * kKc, kn = min(kKc, L - i0);
-        // recompute the chunk's states from the checkpoint
+        __syncthreads();   // the previous chunk is done with bc, hs and sc
+        // this chunk's per-step scalars and the checkpoint, all loads issued together
+#pragma unroll
+        for (int k = 0; k < kKc; k++) {
+            float v = 0.f, xv = 0.f, g = 0.f, zv = 0.f;
+            if (active && k < kn) {
+                const int t = a.reverse ? L - 1 - (i0 + k) : i0 + k;
+                const size_t io = ((size_t)b * L + t) * a.D + dd;
+                v = ldv(dl, io) + bias;
+                xv = ldv(x, io);
+                g = ldv(go, io);
+                if (zp)
+                    zv = ldv(zp, io);
+            }
+            sc[k][0][tid] = v;
+            sc[k][1][tid] = xv;
+            sc[k][2][tid] = g;
+            sc[k][3][tid] = zv;
+        }
         float hp[NS];
         const float *ck = a.ckpt + (((size_t)b * nch + c) * a.D + dd) * N;
 #pragma unroll
         for (int n = 0; n < NS; n++)
             hp[n] = (active && n < N) ? ck[n] : 0.f;
+        stage_bc<T, NS, true>(a, b, i0, bc);
+        __syncthreads();
+        // recompute the chunk's states from the checkpoint
         {
             float h[NS];
 #pragma unroll
             for (int n = 0; n < NS; n++)
                 h[n] = hp[n];
-            for (int k = 0; k < kn; k++) {
-                const int t = a.reverse ? L - 1 - (i0 + k) : i0 + k;
-                const size_t row = (size_t)b * L + t;
-                float dt = 0.f, dtx = 0.f;
-                if (active) {
-                    dt = dt_of(ldv(dl, row * a.D + dd) + bias, a.softplus);
-                    dtx = dt * ldv(x, row * a.D + dd);
-                }
+#pragma unroll
+            for (int k = 0; k < kKc; k++) {
+                const float dt = (k < kn) ? dt_of(sc[k][0][tid], a.softplus) : 0.f;
+                sc[k][4][tid] = dt;
+                const float dtx = dt * sc[k][1][tid];
 #pragma unroll
                 for (int n = 0; n < NS; n++) {
-                    if (n < N)
-                        h[n] = fmaf(ex2_mufu(dt * Al[n]), h[n], dtx * ldv(Bm, row * N + n));
+                    h[n] = fmaf(ex2_mufu(dt * Al[n]), h[n], dtx * bc[k][n]);
                     hs[k][n][tid] = h[n];
                 }
             }
         }
         // backward sweep over the chunk
+#pragma unroll 1
         for (int k = kn - 1; k >= 0; k--) {
             const int t = a.reverse ? L - 1 - (i0 + k) : i0 + k;
             const size_t row = (size_t)b * L + t;
             const size_t io = row * a.D + dd;
-            float dtx = 0.f, dt = 0.f, xv = 0.f, v = 0.f, dy = 0.f;
-            if (active) {
-                v = ldv(dl, io) + bias;
-                dt = dt_of(v, a.softplus);
-                xv = ldv(x, io);
-                dtx = dt * xv;
-                const float g = ldv(go, io);
-                // y_i = C . h_i + D x_i
-                float y = Dv * xv;
+            const float dt = sc[k][4][tid], xv = sc[k][1][tid], dtx = dt * xv;
+            const float gk = sc[k][2][tid], zk = sc[k][3][tid];
+            // y_i = C . h_i + D x_i, then the gate
+            float y = Dv * xv;
 #pragma unroll
-                for (int n = 0; n < NS; n++)
-                    if (n < N)
-                        y = fmaf(ldv(Cm, row * N + n), hs[k][n][tid], y);
-                if (zp) {
-                    const float zv = ldv(zp, io);
-                    const float s = sigmoid_f(zv);
-                    dy = g * zv * s;
-                    if (a.dz)
-                        a.dz[io] = g * y * s * (1.f + zv * (1.f - s));
-                } else {
-                    dy = g;
-                }
+            for (int n = 0; n < NS; n++)
+                y = fmaf(bc[k][NS + n], hs[k][n][tid], y);
+            float dy = gk;
+            if (zp) {
+                const float s = sigmoid_f(zk);
+                dy = gk * zk * s;
+                if (active && a.dz)
+                    a.dz[io] = gk * y * s * (1.f + zk * (1.f - s));
             }
+            if (!active)
+                dy = 0.f;
             float ddt = 0.f, dxs = 0.f;
+            float red[32];
 #pragma unroll
             for (int n = 0; n < NS; n++) {
-                float gB = 0.f, gC = 0.f;
-                if (n < N) {
-                    const float Bn = ldv(Bm, row * N + n), Cn = ldv(Cm, row * N + n);
-                    const float hprev = k > 0 ? hs[k - 1][n][tid] : hp[n];
-                    const float an = ex2_mufu(dt * Al[n]);
-                    const float l = fmaf(dy, Cn, lam[n]);        // lam_i[n]
-                    gC = dy * hs[k][n][tid];
-                    gB = l * dtx;
-                    dxs = fmaf(l, Bn, dxs);
-                    const float ah = an * hprev;
-                    ddt = fmaf(l, fmaf(Bn, xv, A[n] * ah), ddt);
-                    gA[n] = fmaf(l * dt, ah, gA[n]);
-                    lam[n] = an * l;                              // a_i lam_i for step i - 1
-                }
-                red[tid][n] = active ? gB : 0.f;
-                red[tid][NS + n] = active ? gC : 0.f;
+                const float Bn = bc[k][n], Cn = bc[k][NS + n];
+                const float hprev = k > 0 ? hs[k - 1 < 0 ? 0 : k - 1][n][tid] : hp[n];
+                const float an = ex2_mufu(dt * Al[n]);
+                const float l = fmaf(dy, Cn, lam[n]);        // lam_i[n]
+                red[n] = l * dtx;                              // dB contribution
+                red[16 + n] = dy * hs[k][n][tid];              // dC contribution
+                dxs = fmaf(l, Bn, dxs);
+                const float ah = an * hprev;
+                ddt = fmaf(l, fmaf(Bn, xv, A[n] * ah), ddt);
+                gA[n] = fmaf(l * dt, ah, gA[n]);
+                lam[n] = an * l;                               // a_i lam_i for step i - 1
             }
+#pragma unroll
+            for (int n = NS; n < 16; n++)
+                red[n] = red[16 + n] = 0.f;
             if (active) {
                 a.dx[io] = (a.accumulate ? a.dx[io] : 0.f) + fmaf(dy, Dv, dt * dxs);
-                const float dv = a.softplus ? ddt * sigmoid_f(v) : ddt;
+                const float dv = a.softplus ? ddt * sigmoid_f(sc[k][0][tid]) : ddt;
                 a.ddelta[io] = (a.accumulate ? a.ddelta[io] : 0.f) + dv;
                 gbias += dv;
                 gD = fmaf(dy, xv, gD);
             }
-            __syncthreads();
-            // sum dB, dC over the CTA's channels: thread j < 2 NS owns column j
-            if (tid < 2 * NS && (tid % NS) < N) {
-                float s = 0.f;
-#pragma unroll 8
-                for (int r = 0; r < kCta; r++)
-                    s += red[r][tid];
-                float *dst = tid < NS ? a.dB : a.dC;
-                atomicAdd(dst + row * N + (tid % NS), s);
-            }
-            __syncthreads();
+            // dB, dC summed over the warp's 32 channels; lane j holds value j
+            const float s = warp_transpose_sum(red);
+            const int n = lane & 15;
+            if (n < N)
+                atomicAdd((lane < 16 ? a.dB : a.dC) + row * N + n, s);
         }
     }
     if (active) {
