@@ -64,3 +64,23 @@ def s6_grads(x, delta, A, B, C, dout, *, delta_bias=None, softplus=True, D=None,
     res = {k: (None if t is None else t.grad.numpy().copy()) for k, t in ts.items()}
     res["out"] = out.detach().numpy()
     return res
+
+
+def bidir_grads(x, delta, fwd: dict, bwd: dict, dout, *, softplus=True) -> Dict[str, object]:
+    """Gradients of sum(out * dout) for the bidirectional scan (Vim page
+    sec. 3.2: forward scan + reversed scan with its own parameters, summed),
+    by float64 autograd.  Returns {"x", "delta", "out", "fwd": {...},
+    "bwd": {...}} with per-direction keys A, B, C, D, z, delta_bias."""
+    import torch
+    keys = ("A", "B", "C", "D", "z", "delta_bias")
+    tx, td = _t(x, torch, grad=True), _t(delta, torch, grad=True)
+    tf = {k: _t(fwd.get(k), torch, grad=True) for k in keys}
+    tb = {k: _t(bwd.get(k), torch, grad=True) for k in keys}
+    out = (s6_forward_torch(tx, td, tf["A"], tf["B"], tf["C"], delta_bias=tf["delta_bias"], softplus=softplus,
+                            D=tf["D"], z=tf["z"], reverse=False)
+           + s6_forward_torch(tx, td, tb["A"], tb["B"], tb["C"], delta_bias=tb["delta_bias"],
+                              softplus=softplus, D=tb["D"], z=tb["z"], reverse=True))
+    (out * _t(dout, torch)).sum().backward()
+    g = lambda t: None if t is None else t.grad.numpy().copy()
+    return {"x": g(tx), "delta": g(td), "out": out.detach().numpy(),
+            "fwd": {k: g(v) for k, v in tf.items()}, "bwd": {k: g(v) for k, v in tb.items()}}

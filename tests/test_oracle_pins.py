@@ -567,3 +567,41 @@ def test_grads_match_finite_differences(reverse, gate):
             num[idx] = (loss(a1) - loss(a2)) / (2 * eps)
         scale = max(np.max(np.abs(num)), 1e-8)
         assert np.max(np.abs(g[k] - num)) / scale < 1e-6, k
+
+
+def test_bidir_grads_match_finite_differences():
+    """Gradients of the bidirectional scan against central finite
+    differences of the C bidirectional oracle (x, delta and both directions'
+    parameters)."""
+    rng = np.random.default_rng(700)
+    x, delta, bias, A, B, C, D, z = _rand_case(rng, 1, 4, 2, 2)
+    _, _, bias2, A2, B2, C2, D2, z2 = _rand_case(rng, 1, 4, 2, 2)
+    fwd = dict(delta_bias=bias, A=A, B=B, C=C, D=D, z=z)
+    bwd = dict(delta_bias=bias2, A=A2, B=B2, C=C2, D=D2, z=z2)
+    dout = rng.standard_normal(x.shape)
+    g = ograds.bidir_grads(x, delta, fwd, bwd, dout)
+    y0, _, _ = oracle.bidir_arrays(x, delta, fwd, bwd)
+    _close(g["out"], y0)
+
+    def loss(xx, dd, ff, bb):
+        y, _, _ = oracle.bidir_arrays(xx, dd, ff, bb)
+        return float(np.sum(y * dout))
+
+    eps = 1e-6
+    targets = [("x", None), ("delta", None)] + [(k, "fwd") for k in fwd] + [(k, "bwd") for k in bwd]
+    for k, side in targets:
+        base = (x if k == "x" else delta) if side is None else (fwd if side == "fwd" else bwd)[k]
+        ana = g[k] if side is None else g[side][k]
+        num = np.zeros_like(base)
+        for idx in np.ndindex(base.shape):
+            vals = []
+            for sgn in (1, -1):
+                xx, dd = x.copy(), delta.copy()
+                ff = {kk: vv.copy() for kk, vv in fwd.items()}
+                bb = {kk: vv.copy() for kk, vv in bwd.items()}
+                tgt = (xx if k == "x" else dd) if side is None else (ff if side == "fwd" else bb)[k]
+                tgt[idx] += sgn * eps
+                vals.append(loss(xx, dd, ff, bb))
+            num[idx] = (vals[0] - vals[1]) / (2 * eps)
+        scale = max(np.max(np.abs(num)), 1e-8)
+        assert np.max(np.abs(ana - num)) / scale < 1e-6, (k, side)
