@@ -313,6 +313,28 @@ SSM_API ssm_status ssm_scan_bwd(const ssm_dims *dims, const void *x, const void 
                                 float *dB, float *dC, float *dD, float *dz, float *ddelta_bias,
                                 void *workspace, size_t workspace_bytes, void *stream);
 
+/* Gradients of one direction's parameters (bidir_scan_bwd), float32. */
+typedef struct {
+    float *dA;            /* (D, N), required */
+    float *dB, *dC;       /* (B, L, N), required */
+    float *dD;            /* (D): required when the direction has D */
+    float *dz;            /* (B, L, D): required when the direction has z */
+    float *ddelta_bias;   /* (D): required when the direction has delta_bias */
+} ssm_dir_grads;
+
+/*
+ * Gradients of bidir_scan_fwd for an incoming gradient dout (B, L, D) dtype:
+ * dx and ddelta (B, L, D) float32 sum both directions (x and delta are
+ * shared); each direction's parameter gradients go to its ssm_dir_grads.
+ * Same workspace as ssm_scan_bwd (ssm_scan_bwd_workspace_size); errors as
+ * for ssm_scan_bwd.
+ */
+SSM_API ssm_status bidir_scan_bwd(const ssm_dims *dims, const void *x, const void *delta,
+                                  int delta_softplus, const ssm_dir_params *fwd,
+                                  const ssm_dir_params *bwd, const void *dout, float *dx, float *ddelta,
+                                  const ssm_dir_grads *grad_fwd, const ssm_dir_grads *grad_bwd,
+                                  void *workspace, size_t workspace_bytes, void *stream);
+
 /* SSD problem size.  Supported: dtype SSM_BF16, headdim 64, dstate 128,
  * chunk 64, seqlen any value >= 0 (a short last chunk is handled). */
 typedef struct {

@@ -62,6 +62,11 @@ class ssm_dir_params(ctypes.Structure):
                 ("last_state", ctypes.c_void_p)]
 
 
+class ssm_dir_grads(ctypes.Structure):
+    _fields_ = [("dA", ctypes.c_void_p), ("dB", ctypes.c_void_p), ("dC", ctypes.c_void_p),
+                ("dD", ctypes.c_void_p), ("dz", ctypes.c_void_p), ("ddelta_bias", ctypes.c_void_p)]
+
+
 class ssm_conv_params(ctypes.Structure):
     _fields_ = [("weight", ctypes.c_void_p), ("bias", ctypes.c_void_p), ("width", ctypes.c_int32),
                 ("silu", ctypes.c_int32)]
@@ -92,6 +97,9 @@ SIGNATURES = {
     "ssm_scan_bwd_workspace_size": (_sz, [ctypes.POINTER(ssm_dims)]),
     "ssm_scan_bwd": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp, _vp, _int,
                             _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "bidir_scan_bwd": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _int, ctypes.POINTER(ssm_dir_params),
+                              ctypes.POINTER(ssm_dir_params), _vp, _vp, _vp, ctypes.POINTER(ssm_dir_grads),
+                              ctypes.POINTER(ssm_dir_grads), _vp, _sz, _vp]),
     "ssm_step": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp, _vp, _vp,
                         _vp, _vp]),
     "ssm_scan_fwd_noalloc": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp,
@@ -364,6 +372,41 @@ def ssm_scan_bwd(x, delta, A, B, C, dout, *, delta_bias=None, delta_softplus=Tru
                           _stream_handle(stream))
     _check(st, "ssm_scan_bwd")
     return g
+
+
+def bidir_scan_bwd(x, delta, fwd: DirParams, bwd: DirParams, dout, *, delta_softplus=True, stream=None):
+    """Gradients of bidir_scan_fwd: returns (dx, ddelta, grads_fwd, grads_bwd)
+    with float32 tensors; each grads dict holds dA, dB, dC and dD, dz,
+    ddelta_bias for the inputs that direction has."""
+    torch = _torch()
+    lib = capi()
+    dims = s6_dims(x, fwd.A.shape[1])
+    f32 = dict(dtype=torch.float32, device=x.device)
+
+    def mk(p: DirParams):
+        g = {"dA": torch.empty(p.A.shape, **f32), "dB": torch.empty(p.B.shape, **f32),
+             "dC": torch.empty(p.C.shape, **f32)}
+        if p.D is not None:
+            g["dD"] = torch.empty(p.D.shape, **f32)
+        if p.z is not None:
+            g["dz"] = torch.empty(x.shape, **f32)
+        if p.delta_bias is not None:
+            g["ddelta_bias"] = torch.empty(p.delta_bias.shape, **f32)
+        c = ssm_dir_grads(_ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dC"]), _ptr(g.get("dD")), _ptr(g.get("dz")),
+                          _ptr(g.get("ddelta_bias")))
+        return g, c
+
+    gf, cf = mk(fwd)
+    gb, cb = mk(bwd)
+    dx, ddelta = torch.empty(x.shape, **f32), torch.empty(x.shape, **f32)
+    ws = workspace(lib.ssm_scan_bwd_workspace_size(ctypes.byref(dims)), x.device)
+    f, b = fwd.to_c(), bwd.to_c()
+    st = lib.bidir_scan_bwd(ctypes.byref(dims), _ptr(x), _ptr(delta), int(bool(delta_softplus)),
+                            ctypes.byref(f), ctypes.byref(b), _ptr(dout), _ptr(dx), _ptr(ddelta),
+                            ctypes.byref(cf), ctypes.byref(cb), _ptr(ws), 0 if ws is None else ws.numel(),
+                            _stream_handle(stream))
+    _check(st, "bidir_scan_bwd")
+    return dx, ddelta, gf, gb
 
 
 def ssm_step(x, delta, A, B, C, state, *, delta_bias=None, delta_softplus=True, D=None, z=None,

@@ -321,46 +321,37 @@ size_t ssm_scan_bwd_workspace_size(const ssm_dims *dims)
     return ssm::bwd_workspace_bytes(dims->batch, dims->seqlen, dims->dim, dims->dstate);
 }
 
-ssm_status ssm_scan_bwd(const ssm_dims *dims, const void *x, const void *delta, const float *delta_bias,
-                        int delta_softplus, const float *A, const void *B, const void *C, const float *D,
-                        const void *z, int reverse, const void *dout, float *dx, float *ddelta, float *dA,
-                        float *dB, float *dC, float *dD, float *dz, float *ddelta_bias, void *workspace,
-                        size_t workspace_bytes, void *stream)
+}  // extern "C"
+
+namespace {
+
+// One direction's backward launch (ssm_scan_bwd, bidir_scan_bwd): checks,
+// zeroes the accumulated gradients, launches.  accumulate: add into dx and
+// ddelta instead of writing them.
+ssm_status bwd_one(const ssm_dims *dims, const void *x, const void *delta, int delta_softplus,
+                   const ssm_dir_params &p, int reverse, const void *dout, float *dx, float *ddelta,
+                   const ssm_dir_grads &g, void *workspace, size_t workspace_bytes, int accumulate,
+                   cudaStream_t st)
 {
-    ssm_status s = check_s6_dims(dims);
-    if (s != SSM_OK)
-        return s;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const size_t nDN = (size_t)dims->dim * dims->dstate;
-    if (empty_s6(dims)) {
-        // no step: every gradient is zero (the ones over (D, N) and (D) too)
-        if (dA && nDN && cudaMemsetAsync(dA, 0, nDN * sizeof(float), st) != cudaSuccess)
-            return SSM_ERR_CUDA;
-        if (D && dD && dims->dim && cudaMemsetAsync(dD, 0, dims->dim * sizeof(float), st) != cudaSuccess)
-            return SSM_ERR_CUDA;
-        if (delta_bias && ddelta_bias && dims->dim &&
-            cudaMemsetAsync(ddelta_bias, 0, dims->dim * sizeof(float), st) != cudaSuccess)
-            return SSM_ERR_CUDA;
-        return SSM_OK;
-    }
-    if (!x || !delta || !A || !B || !C || !dout || !dx || !ddelta || !dA || !dB || !dC)
+    if (!x || !delta || !p.A || !p.B || !p.C || !dout || !dx || !ddelta || !g.dA || !g.dB || !g.dC)
         return SSM_ERR_INVALID_ARG;
-    if ((D && !dD) || (z && !dz) || (delta_bias && !ddelta_bias))
+    if ((p.D && !g.dD) || (p.z && !g.dz) || (p.delta_bias && !g.ddelta_bias))
         return SSM_ERR_INVALID_ARG;
-    const void *ptrs[] = {x, delta, delta_bias, A, B, C, D, z, dout, dx, ddelta, dA, dB, dC, dD, dz,
-                          ddelta_bias, workspace};
+    const void *ptrs[] = {x, delta, p.delta_bias, p.A, p.B, p.C, p.D, p.z, dout, dx, ddelta, g.dA, g.dB,
+                          g.dC, g.dD, g.dz, g.ddelta_bias, workspace};
     for (const void *q : ptrs)
         if (q && !aligned16(q))
             return SSM_ERR_MISALIGNED;
     const size_t need = ssm::bwd_workspace_bytes(dims->batch, dims->seqlen, dims->dim, dims->dstate);
     if (!workspace || workspace_bytes < need)
         return SSM_ERR_WORKSPACE_TOO_SMALL;
+    const size_t nDN = (size_t)dims->dim * dims->dstate;
     const size_t nBLN = (size_t)dims->batch * dims->seqlen * dims->dstate;
-    if (cudaMemsetAsync(dA, 0, nDN * sizeof(float), st) != cudaSuccess ||
-        cudaMemsetAsync(dB, 0, nBLN * sizeof(float), st) != cudaSuccess ||
-        cudaMemsetAsync(dC, 0, nBLN * sizeof(float), st) != cudaSuccess ||
-        (D && cudaMemsetAsync(dD, 0, dims->dim * sizeof(float), st) != cudaSuccess) ||
-        (delta_bias && cudaMemsetAsync(ddelta_bias, 0, dims->dim * sizeof(float), st) != cudaSuccess))
+    if (cudaMemsetAsync(g.dA, 0, nDN * sizeof(float), st) != cudaSuccess ||
+        cudaMemsetAsync(g.dB, 0, nBLN * sizeof(float), st) != cudaSuccess ||
+        cudaMemsetAsync(g.dC, 0, nBLN * sizeof(float), st) != cudaSuccess ||
+        (p.D && cudaMemsetAsync(g.dD, 0, dims->dim * sizeof(float), st) != cudaSuccess) ||
+        (p.delta_bias && cudaMemsetAsync(g.ddelta_bias, 0, dims->dim * sizeof(float), st) != cudaSuccess))
         return SSM_ERR_CUDA;
     ssm::BwdArgs a;
     memset(&a, 0, sizeof(a));
@@ -371,25 +362,87 @@ ssm_status ssm_scan_bwd(const ssm_dims *dims, const void *x, const void *delta, 
     a.dtype = dims->dtype == SSM_F32 ? 0 : 1;
     a.softplus = delta_softplus ? 1 : 0;
     a.reverse = reverse ? 1 : 0;
+    a.accumulate = accumulate;
     a.x = x;
     a.delta = delta;
-    a.B = B;
-    a.C = C;
-    a.z = z;
+    a.B = p.B;
+    a.C = p.C;
+    a.z = p.z;
     a.dout = dout;
-    a.bias = delta_bias;
-    a.A = A;
-    a.Dskip = D;
+    a.bias = p.delta_bias;
+    a.A = p.A;
+    a.Dskip = p.D;
     a.dx = dx;
     a.ddelta = ddelta;
-    a.dz = z ? dz : nullptr;
-    a.dA = dA;
-    a.dB = dB;
-    a.dC = dC;
-    a.dD = D ? dD : nullptr;
-    a.dbias = delta_bias ? ddelta_bias : nullptr;
+    a.dz = p.z ? g.dz : nullptr;
+    a.dA = g.dA;
+    a.dB = g.dB;
+    a.dC = g.dC;
+    a.dD = p.D ? g.dD : nullptr;
+    a.dbias = p.delta_bias ? g.ddelta_bias : nullptr;
     a.ckpt = static_cast<float *>(workspace);
     return ssm::launch_bwd(a, st) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+// The gradients of an empty problem: zero over (D, N) and (D).
+ssm_status bwd_empty(const ssm_dims *dims, const ssm_dir_params &p, const ssm_dir_grads &g, cudaStream_t st)
+{
+    const size_t nDN = (size_t)dims->dim * dims->dstate;
+    if (g.dA && nDN && cudaMemsetAsync(g.dA, 0, nDN * sizeof(float), st) != cudaSuccess)
+        return SSM_ERR_CUDA;
+    if (p.D && g.dD && dims->dim && cudaMemsetAsync(g.dD, 0, dims->dim * sizeof(float), st) != cudaSuccess)
+        return SSM_ERR_CUDA;
+    if (p.delta_bias && g.ddelta_bias && dims->dim &&
+        cudaMemsetAsync(g.ddelta_bias, 0, dims->dim * sizeof(float), st) != cudaSuccess)
+        return SSM_ERR_CUDA;
+    return SSM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+ssm_status ssm_scan_bwd(const ssm_dims *dims, const void *x, const void *delta, const float *delta_bias,
+                        int delta_softplus, const float *A, const void *B, const void *C, const float *D,
+                        const void *z, int reverse, const void *dout, float *dx, float *ddelta, float *dA,
+                        float *dB, float *dC, float *dD, float *dz, float *ddelta_bias, void *workspace,
+                        size_t workspace_bytes, void *stream)
+{
+    ssm_status s = check_s6_dims(dims);
+    if (s != SSM_OK)
+        return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const ssm_dir_params p{delta_bias, A, B, C, D, z, nullptr};
+    const ssm_dir_grads g{dA, dB, dC, dD, dz, ddelta_bias};
+    if (empty_s6(dims))
+        return bwd_empty(dims, p, g, st);
+    return bwd_one(dims, x, delta, delta_softplus, p, reverse, dout, dx, ddelta, g, workspace, workspace_bytes,
+                   0, st);
+}
+
+ssm_status bidir_scan_bwd(const ssm_dims *dims, const void *x, const void *delta, int delta_softplus,
+                          const ssm_dir_params *fwd, const ssm_dir_params *bwd, const void *dout, float *dx,
+                          float *ddelta, const ssm_dir_grads *grad_fwd, const ssm_dir_grads *grad_bwd,
+                          void *workspace, size_t workspace_bytes, void *stream)
+{
+    ssm_status s = check_s6_dims(dims);
+    if (s != SSM_OK)
+        return s;
+    if (!fwd || !bwd || !grad_fwd || !grad_bwd)
+        return SSM_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (empty_s6(dims)) {
+        if ((s = bwd_empty(dims, *fwd, *grad_fwd, st)) != SSM_OK)
+            return s;
+        return bwd_empty(dims, *bwd, *grad_bwd, st);
+    }
+    // forward direction writes dx, ddelta; the reversed one adds to them (the
+    // two launches share the workspace in stream order)
+    if ((s = bwd_one(dims, x, delta, delta_softplus, *fwd, 0, dout, dx, ddelta, *grad_fwd, workspace,
+                     workspace_bytes, 0, st)) != SSM_OK)
+        return s;
+    return bwd_one(dims, x, delta, delta_softplus, *bwd, 1, dout, dx, ddelta, *grad_bwd, workspace,
+                   workspace_bytes, 1, st);
 }
 
 ssm_status ssm_step(const ssm_dims *dims, const void *x, const void *delta, const float *delta_bias,

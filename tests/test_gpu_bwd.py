@@ -72,3 +72,29 @@ def test_bwd_long_sequence():
     dout = np.random.default_rng(9).standard_normal(inp.x.shape).astype(np.float32)
     g, ref = _run(inp, "f32", dout, False)
     _check(g, ref, TOL["f32"])
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_bidir_bwd_matches_autograd(dtype):
+    """Gradients of the bidirectional scan: dx and ddelta sum both
+    directions, each direction's parameter gradients separately."""
+    from gpu_util import dir_params
+    inp = ssm_gen.make_s6_inputs(2, 77, 96, 16, dtype=dtype, bidir=True, seed=31, random_A=True,
+                                 random_D=True)
+    dout = np.random.default_rng(5).standard_normal(inp.x.shape).astype(np.float32)
+    if dtype == "bf16":
+        dout = ssm_gen.round_to_bf16(dout)
+    f, b = dir_params(inp, "f"), dir_params(inp, "b")
+    dx, ddelta, gf, gb = ssm.bidir_scan_bwd(dev(inp.x, dtype), dev(inp.delta, dtype), f, b, dev(dout, dtype))
+    torch.cuda.synchronize()
+    fw = dict(delta_bias=inp.dt_bias_f, A=inp.A_f, B=inp.B_f, C=inp.C_f, D=inp.D_f, z=inp.z_f)
+    bw = dict(delta_bias=inp.dt_bias_b, A=inp.A_b, B=inp.B_b, C=inp.C_b, D=inp.D_b, z=inp.z_b)
+    ref = ograds.bidir_grads(inp.x, inp.delta, fw, bw, dout)
+    tol = TOL[dtype]
+    assert rel_err(dx.cpu().numpy(), ref["x"]) <= tol
+    assert rel_err(ddelta.cpu().numpy(), ref["delta"]) <= tol
+    names = {"dA": "A", "dB": "B", "dC": "C", "dD": "D", "dz": "z", "ddelta_bias": "delta_bias"}
+    for g, side in ((gf, "fwd"), (gb, "bwd")):
+        for k, t in g.items():
+            e = rel_err(t.cpu().numpy(), ref[side][names[k]])
+            assert e <= tol, f"{side} {k}: rel err {e:.3e}"
