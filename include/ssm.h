@@ -294,7 +294,7 @@ SSM_API size_t ssm_scan_bwd_workspace_size(const ssm_dims *dims);
  * Gradients of ssm_scan_fwd (same dims and inputs, same reverse flag) for
  * an incoming gradient dout of out -- the training use of the Mamba2 page,
  * sec. 5.1, which backpropagates through the scan.  The states are
- * recomputed (a forward pass stores h every 8 steps in the workspace), so
+ * recomputed (a forward pass stores h every 4 steps in the workspace), so
  * nothing from the forward call is needed.  All gradients are float32:
  *   dout            (B, L, D) dtype, required
  *   dx, ddelta      (B, L, D), required, written

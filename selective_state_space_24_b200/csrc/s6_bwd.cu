@@ -34,7 +34,8 @@
 namespace ssm {
 namespace {
 
-constexpr int kKc = 8;         // steps per checkpointed chunk
+constexpr int kKc = 4;         // steps per checkpointed chunk (4: the backward kernel's shared
+                               // memory then allows 6 CTAs per SM, one wave for Vim-Small)
 constexpr int kCta = 64;       // channels (threads) per CTA
 
 template <typename T> __device__ __forceinline__ float ldv(const T *p, size_t i);
@@ -214,7 +215,11 @@ __global__ void __launch_bounds__(kCta) s6_bwd_kernel(const BwdArgs a)
                 }
             }
         }
-        // backward sweep over the chunk
+        // backward sweep over the chunk; hk holds h_k, loaded once per step
+        float hk[NS];
+#pragma unroll
+        for (int n = 0; n < NS; n++)
+            hk[n] = hs[kn - 1][n][tid];
 #pragma unroll 1
         for (int k = kn - 1; k >= 0; k--) {
             const int t = a.reverse ? L - 1 - (i0 + k) : i0 + k;
@@ -226,7 +231,7 @@ __global__ void __launch_bounds__(kCta) s6_bwd_kernel(const BwdArgs a)
             float y = Dv * xv;
 #pragma unroll
             for (int n = 0; n < NS; n++)
-                y = fmaf(bc[k][NS + n], hs[k][n][tid], y);
+                y = fmaf(bc[k][NS + n], hk[n], y);
             float dy = gk;
             if (zp) {
                 const float s = sigmoid_f(zk);
@@ -242,10 +247,12 @@ __global__ void __launch_bounds__(kCta) s6_bwd_kernel(const BwdArgs a)
             for (int n = 0; n < NS; n++) {
                 const float Bn = bc[k][n], Cn = bc[k][NS + n];
                 const float hprev = k > 0 ? hs[k - 1 < 0 ? 0 : k - 1][n][tid] : hp[n];
+                const float hcur = hk[n];
+                hk[n] = hprev;                                  // h_{k-1} for the next step
                 const float an = ex2_mufu(dt * Al[n]);
                 const float l = fmaf(dy, Cn, lam[n]);        // lam_i[n]
                 red[n] = l * dtx;                              // dB contribution
-                red[16 + n] = dy * hs[k][n][tid];              // dC contribution
+                red[16 + n] = dy * hcur;                       // dC contribution
                 dxs = fmaf(l, Bn, dxs);
                 const float ah = an * hprev;
                 ddt = fmaf(l, fmaf(Bn, xv, A[n] * ah), ddt);
