@@ -82,13 +82,28 @@ __global__ void __launch_bounds__(256) s6_step_kernel(const StepArgs a)
                 Av[k] = in ? Ar[k] : 0.f;
             }
         }
+        // this lane's B and C values (one 16-byte load each for fp32, N = 16)
+        float Bv[K], Cv[K];
+        if (VEC && K == 4 && sizeof(T) == 4) {
+            const float4 bv = __ldg(reinterpret_cast<const float4 *>(Bm) + (b * N + part * K) / 4);
+            const float4 cv = __ldg(reinterpret_cast<const float4 *>(Cm) + (b * N + part * K) / 4);
+            Bv[0] = bv.x, Bv[1] = bv.y, Bv[2] = bv.z, Bv[3] = bv.w;
+            Cv[0] = cv.x, Cv[1] = cv.y, Cv[2] = cv.z, Cv[3] = cv.w;
+        } else {
+#pragma unroll
+            for (int k = 0; k < K; k++) {
+                const int n = part * K + k;
+                Bv[k] = (VEC || n < N) ? ldv(Bm, b * N + n) : 0.f;
+                Cv[k] = (VEC || n < N) ? ldv(Cm, b * N + n) : 0.f;
+            }
+        }
 #pragma unroll
         for (int k = 0; k < K; k++) {
             const int n = part * K + k;
             if (VEC || n < N) {
                 const float e = ex2_mufu(dt * (Av[k] * kLog2e));
-                h[k] = fmaf(e, h[k], dtx * ldv(Bm, b * N + n));
-                y = fmaf(ldv(Cm, b * N + n), h[k], y);
+                h[k] = fmaf(e, h[k], dtx * Bv[k]);
+                y = fmaf(Cv[k], h[k], y);
             }
         }
         if (VEC) {
