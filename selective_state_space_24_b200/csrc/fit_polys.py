@@ -1,4 +1,4 @@
-"""Fits the polynomials s6_scan.cu uses:
+"""Fits the polynomials the S6 kernels (s6_scan_impl.cuh) use:
 
 * 2^f for |f| <= 1/2 (ex2_poly2): degree 5, 2.1e-7 relative error in fp32,
   the class of the MUFU ex2.approx instruction;

@@ -70,6 +70,19 @@ S6Plan plan_s6(int64_t Bsz, int64_t L, int64_t D, int64_t N, int ndir, int dtype
 
 cudaError_t launch_s6(const S6Args &a, cudaStream_t stream);
 
+// The S6 kernel parts (s6_part_*.cu): one element type and variant each,
+// and each part's error word (read, and reset if clear).
+#define SSM_S6_PART_DECL(NAME)                                        \
+    cudaError_t launch_s6_##NAME(const S6Args &a, cudaStream_t stream); \
+    cudaError_t s6_error_##NAME(unsigned *value, bool clear);
+SSM_S6_PART_DECL(f32)
+SSM_S6_PART_DECL(f32_ord)
+SSM_S6_PART_DECL(f32_conv)
+SSM_S6_PART_DECL(bf16)
+SSM_S6_PART_DECL(bf16_ord)
+SSM_S6_PART_DECL(bf16_conv)
+#undef SSM_S6_PART_DECL
+
 // One decode step of S6 for every (batch, channel), state updated in place.
 struct StepArgs {
     int Bsz, D, N;
