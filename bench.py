@@ -46,9 +46,10 @@ HBM_FALLBACK_GBS = 6650.0
 L2_FLUSH_BYTES = 512 << 20
 SMS = 148
 # DRAM bytes (read + write) per launch of the dominant kernel, from one ncu
-# capture of the current kernels (profiles/s6_main_vim_small_bidir_fp32.md,
-# profiles/ssd_chunk_mamba2_bf16.md); absent where no capture matches them.
-NCU_TRAFFIC = {1: 271.65e6, 4: 398.97e6}
+# capture of the current kernels (summaries under profiles/); absent where no
+# capture matches them.
+NCU_TRAFFIC = {1: 271.73e6, 4: 398.97e6}
+NCU_TRAFFIC_STEP = 63.05e6
 
 
 def parse():
@@ -485,7 +486,7 @@ def run_step(args):
                    "l2": "flushed before every timed step (512 MB write)",
                    "algorithmic_bytes_per_step": nbytes},
         "roofline": {"bound": "hbm", "achieved": hbm, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": hbm / peaks["hbm_gbs"], "traffic": None, "peak_source": peak_src,
+                     "frac": hbm / peaks["hbm_gbs"], "traffic": NCU_TRAFFIC_STEP, "peak_source": peak_src,
                      "kernel_ms_median": med},
         "gpu_launches": args.steps, "clocks": clocks,
     }
