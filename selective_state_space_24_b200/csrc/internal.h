@@ -108,7 +108,8 @@ struct BwdArgs {
     const void *x, *delta, *B, *C, *z, *dout;
     const float *bias, *A, *Dskip;
     float *dx, *ddelta, *dz, *dA, *dB, *dC, *dD, *dbias;
-    float *ckpt;    // workspace: (Bsz, ceil(L / 4), D, N) states entering each 4-step chunk
+    float *ckpt;    // workspace: (Bsz, ceil(L / 4), D, NS) states entering each 4-step chunk,
+                    // NS = N rounded up to 4, 8 or 16 (16-byte aligned)
 };
 size_t bwd_workspace_bytes(int64_t Bsz, int64_t L, int64_t D, int64_t N);
 cudaError_t launch_bwd(const BwdArgs &a, cudaStream_t stream);

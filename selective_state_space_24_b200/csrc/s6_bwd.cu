@@ -16,7 +16,8 @@
 //   ddelta_i = ddt_i softplus'(v_i) = ddt_i sigmoid(v_i);  dbias += ddelta_i
 //
 // Two kernels.  s6_bwd_ckpt_kernel runs the forward recurrence once and
-// stores h entering every chunk of kKc steps.  s6_bwd_kernel walks the
+// stores h entering every chunk of kKc steps (padded to the template state
+// count, so each channel's checkpoint is whole 16-byte vectors).  s6_bwd_kernel walks the
 // chunks backwards: it recomputes the chunk's states into shared memory
 // from the checkpoint, then sweeps the chunk backwards with lam in
 // registers.  One thread per (b, d); a CTA holds 64 channels of one batch
@@ -37,6 +38,8 @@ namespace {
 constexpr int kKc = 4;         // steps per checkpointed chunk (4: the backward kernel's shared
                                // memory then allows 6 CTAs per SM, one wave for Vim-Small)
 constexpr int kCta = 64;       // channels (threads) per CTA
+constexpr int kStage = 16;     // steps per input stage of the checkpoint pass
+constexpr int kBwdCtasPerSm = 6;   // backward kernel residency: 768 CTAs of Vim-Small in one wave
 
 template <typename T> __device__ __forceinline__ float ldv(const T *p, size_t i);
 template <> __device__ __forceinline__ float ldv<float>(const float *p, size_t i) { return __ldg(p + i); }
@@ -47,25 +50,6 @@ template <> __device__ __forceinline__ float ldv<__nv_bfloat16>(const __nv_bfloa
 
 __device__ __forceinline__ float dt_of(float v, int softplus) { return softplus ? softplus_f(v) : v; }
 __device__ __forceinline__ float sigmoid_f(float v) { return 1.f / (1.f + ex2_mufu(-v * kLog2e)); }
-
-// B (and C) rows of steps [i0, i0 + kKc) in scan order into shared memory:
-// bc[k][n] for B, bc[k][NS + n] for C (zero past L or N).  Whole CTA.
-template <typename T, int NS, bool WITH_C>
-__device__ __forceinline__ void stage_bc(const BwdArgs &a, int b, int i0, float (*bc)[2 * NS])
-{
-    const T *Bm = static_cast<const T *>(a.B), *Cm = static_cast<const T *>(a.C);
-    constexpr int kVals = kKc * (WITH_C ? 2 : 1) * NS;
-    for (int j = threadIdx.x; j < kVals; j += kCta) {
-        const int k = j / ((WITH_C ? 2 : 1) * NS), r = j % ((WITH_C ? 2 : 1) * NS);
-        const int n = r % NS, i = i0 + k;
-        float v = 0.f;
-        if (i < a.L && n < a.N) {
-            const int t = a.reverse ? a.L - 1 - i : i;
-            v = ldv(r < NS ? Bm : Cm, ((size_t)b * a.L + t) * a.N + n);
-        }
-        bc[k][r] = v;
-    }
-}
 
 // Sum v[0..31] over the 32 lanes of the warp: afterwards lane j holds the
 // sum of every lane's v[j] (butterfly: at each stage a lane keeps one half of
@@ -87,16 +71,55 @@ __device__ __forceinline__ float warp_transpose_sum(float (&v)[32])
     return v[0];
 }
 
+// The forward inputs of kStage steps from scan index i0: this thread's
+// delta and x, and its kPer share of the steps' B rows (element e = thread +
+// j kCta of the (step, state) tile).  Zero past L, N or D.
+template <typename T, int NS, int kPer>
+__device__ __forceinline__ void load_stage(const BwdArgs &a, int b, int dd, bool active, int i0,
+                                           float (&v)[kStage], float (&xv)[kStage], float (&bq)[kPer])
+{
+    const T *x = static_cast<const T *>(a.x), *dl = static_cast<const T *>(a.delta);
+    const T *Bm = static_cast<const T *>(a.B);
+#pragma unroll
+    for (int k = 0; k < kStage; k++) {
+        const int i = i0 + k;
+        v[k] = 0.f;
+        xv[k] = 0.f;
+        if (active && i < a.L) {
+            const int t = a.reverse ? a.L - 1 - i : i;
+            const size_t io = ((size_t)b * a.L + t) * a.D + dd;
+            v[k] = ldv(dl, io);
+            xv[k] = ldv(x, io);
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < kPer; j++) {
+        const int e = threadIdx.x + j * kCta, k = e / NS, n = e % NS, i = i0 + k;
+        bq[j] = 0.f;
+        if (i < a.L && n < a.N) {
+            const int t = a.reverse ? a.L - 1 - i : i;
+            bq[j] = ldv(Bm, ((size_t)b * a.L + t) * a.N + n);
+        }
+    }
+}
+
+// Forward recurrence of one (b, d) per thread, storing h entering every
+// kKc-step chunk (NS floats per channel, the padding states stay zero).  The
+// inputs arrive kStage steps at a time, the next stage's loads in flight
+// while the current stage is computed; the stage's B rows sit in a
+// double-buffered shared tile, so one barrier per stage suffices.
 template <typename T, int NS>
 __global__ void __launch_bounds__(kCta) s6_bwd_ckpt_kernel(const BwdArgs a)
 {
-    __shared__ float bc[kKc][2 * NS];
+    constexpr int kPer = kStage * NS / kCta;
+    static_assert(kPer * kCta == kStage * NS, "stage tile must split evenly over the CTA");
+    static_assert(kStage % kKc == 0, "a stage holds whole chunks");
+    __shared__ float bs[2][kStage][NS];
     const int d = blockIdx.x * kCta + threadIdx.x;
     const int b = blockIdx.y;
     const bool active = d < a.D;
     const int dd = active ? d : 0;
-    const int N = a.N, L = a.L, nch = (L + kKc - 1) / kKc;
-    const T *x = static_cast<const T *>(a.x), *dl = static_cast<const T *>(a.delta);
+    const int N = a.N, L = a.L, nch = (L + kKc - 1) / kKc, nst = (L + kStage - 1) / kStage;
     float Al[NS], h[NS];
 #pragma unroll
     for (int n = 0; n < NS; n++) {
@@ -104,136 +127,263 @@ __global__ void __launch_bounds__(kCta) s6_bwd_ckpt_kernel(const BwdArgs a)
         h[n] = 0.f;
     }
     const float bias = (active && a.bias) ? a.bias[dd] : 0.f;
-    for (int c = 0; c < nch; c++) {
-        const int i0 = c * kKc;
-        if (active) {
-            float *ck = a.ckpt + (((size_t)b * nch + c) * a.D + dd) * N;
+    float v[kStage], xv[kStage], bq[kPer];
+    load_stage<T, NS, kPer>(a, b, dd, active, 0, v, xv, bq);
 #pragma unroll
-            for (int n = 0; n < NS; n++)
-                if (n < N)
-                    ck[n] = h[n];
-        }
-        // this chunk's per-step scalars, all loads issued together
-        float dtk[kKc], xk[kKc];
+    for (int j = 0; j < kPer; j++) {
+        const int e = threadIdx.x + j * kCta;
+        bs[0][e / NS][e % NS] = bq[j];
+    }
+    __syncthreads();
+    for (int s = 0; s < nst; s++) {
+        const int i0 = s * kStage;
+        const bool more = s + 1 < nst;
+        float vn[kStage], xn[kStage], bn[kPer];
+        if (more)
+            load_stage<T, NS, kPer>(a, b, dd, active, i0 + kStage, vn, xn, bn);
+        const float(*bc)[NS] = bs[s & 1];
 #pragma unroll
-        for (int k = 0; k < kKc; k++) {
+        for (int k = 0; k < kStage; k++) {
             const int i = i0 + k;
-            dtk[k] = 0.f;
-            xk[k] = 0.f;
-            if (active && i < L) {
-                const int t = a.reverse ? L - 1 - i : i;
-                const size_t io = ((size_t)b * L + t) * a.D + dd;
-                dtk[k] = ldv(dl, io);
-                xk[k] = ldv(x, io);
-            }
-        }
-        __syncthreads();   // the previous chunk is done with bc
-        stage_bc<T, NS, false>(a, b, i0, bc);
-        __syncthreads();
+            if (k % kKc == 0 && active && i < L) {
+                float4 *ck = reinterpret_cast<float4 *>(a.ckpt + (((size_t)b * nch + i / kKc) * a.D + dd) * NS);
 #pragma unroll
-        for (int k = 0; k < kKc; k++) {
-            const float dt = (i0 + k < L) ? dt_of(dtk[k] + bias, a.softplus) : 0.f;
-            const float dtx = dt * xk[k];
+                for (int q = 0; q < NS / 4; q++)
+                    ck[q] = make_float4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
+            }
+            const float dt = i < L ? dt_of(v[k] + bias, a.softplus) : 0.f;
+            const float dtx = dt * xv[k];
 #pragma unroll
             for (int n = 0; n < NS; n++)
                 h[n] = fmaf(ex2_mufu(dt * Al[n]), h[n], dtx * bc[k][n]);
         }
+        if (more) {
+#pragma unroll
+            for (int j = 0; j < kPer; j++) {
+                const int e = threadIdx.x + j * kCta;
+                bs[(s + 1) & 1][e / NS][e % NS] = bn[j];
+            }
+#pragma unroll
+            for (int k = 0; k < kStage; k++) {
+                v[k] = vn[k];
+                xv[k] = xn[k];
+            }
+        }
+        __syncthreads();
     }
 }
 
-template <typename T, int NS>
-__global__ void __launch_bounds__(kCta) s6_bwd_kernel(const BwdArgs a)
+// 16-byte cp.async into shared memory; src_bytes 0 writes zeros (src must
+// still be a valid address, it is not read).
+__device__ __forceinline__ void cp_async16z(void *smem, const void *gmem, bool valid)
 {
-    // states of the current chunk: hs[k][n][thread]; the chunk's B and C
-    // rows; this thread's per-step scalars sc[k][dt, x, dout, z][thread]
-    __shared__ float hs[kKc][NS][kCta];
-    __shared__ float bc[kKc][2 * NS];
-    __shared__ float sc[kKc][5][kCta];
+    const unsigned sa = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+    const int nbytes = valid ? 16 : 0;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(sa), "l"(gmem), "r"(nbytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+template <typename T> __device__ __forceinline__ float tof(T v);
+template <> __device__ __forceinline__ float tof<float>(float v) { return v; }
+template <> __device__ __forceinline__ float tof<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// Shared memory of the backward kernel.
+template <typename T, int NS>
+struct BwdSmem {
+    __align__(16) float hs[kKc][kCta][NS];     // the chunk's recomputed states, a row per thread
+                                               // (16-byte slots swizzled by hs_slot)
+    __align__(16) T raw[2][kKc][4][kCta];      // delta, x, dout, z rows of two chunks
+    __align__(16) float ck[2][kCta][NS + 4];   // checkpoints of two chunks (padded rows: no bank conflicts)
+    __align__(16) float bc[2][kKc][2 * NS];    // B and C rows of two chunks
+    float dt[kKc][kCta];                       // this chunk's dt, a column per thread
+};
+
+// Start the copies of chunk c's delta, x, dout, z rows (16-byte pieces of
+// the CTA's channel range; pieces past L or D, and a missing z, are zero
+// filled) and of this thread's checkpoint into buffer `buf`; one commit group.
+template <typename T, int NS>
+__device__ __forceinline__ void issue_chunk(const BwdArgs &a, BwdSmem<T, NS> &sm, int buf, int b, int d0,
+                                            int c, int nch)
+{
+    constexpr int kPieceCh = 16 / (int)sizeof(T);
+    constexpr int kPiecesRow = kCta / kPieceCh;
+    constexpr int kPieces = kKc * 4 * kPiecesRow;
+    static_assert(kPieces % kCta == 0, "pieces split evenly over the CTA");
+    const int i0 = c * kKc;
+#pragma unroll
+    for (int j = 0; j < kPieces / kCta; j++) {
+        const int p = threadIdx.x + j * kCta, row = p / kPiecesRow, q = p % kPiecesRow;
+        const int k = row >> 2, arr = row & 3, i = i0 + k, ch = d0 + q * kPieceCh;
+        const void *bv = arr == 0 ? a.delta : arr == 1 ? a.x : arr == 2 ? a.dout : a.z;
+        const T *base = static_cast<const T *>(bv);
+        const bool valid = i < a.L && ch < a.D && base != nullptr;
+        const T *g = static_cast<const T *>(a.x);
+        if (valid)
+            g = base + ((size_t)b * a.L + (a.reverse ? a.L - 1 - i : i)) * a.D + ch;
+        cp_async16z(&sm.raw[buf][k][arr][q * kPieceCh], g, valid);
+    }
+    const int d = d0 + threadIdx.x;
+    const bool act = d < a.D;
+    const float *ck = a.ckpt + (((size_t)b * nch + c) * a.D + (act ? d : 0)) * NS;
+#pragma unroll
+    for (int q = 0; q < NS / 4; q++)
+        cp_async16z(&sm.ck[buf][threadIdx.x][4 * q], ck + 4 * q, act);
+    cp_async_commit();
+}
+
+// B and C rows of chunk c into registers (kBq per thread; element e =
+// thread + j kCta of the (step, B | C, state) tile), zero past L or N.
+template <typename T, int NS, int kBq>
+__device__ __forceinline__ void load_bc(const BwdArgs &a, int b, int c, float (&bq)[kBq])
+{
+    const T *Bm = static_cast<const T *>(a.B), *Cm = static_cast<const T *>(a.C);
+#pragma unroll
+    for (int j = 0; j < kBq; j++) {
+        const int e = threadIdx.x + j * kCta, k = e / (2 * NS), r = e % (2 * NS), n = r % NS;
+        const int i = c * kKc + k;
+        bq[j] = 0.f;
+        if (e < kKc * 2 * NS && i < a.L && n < a.N) {
+            const int t = a.reverse ? a.L - 1 - i : i;
+            bq[j] = ldv(r < NS ? Bm : Cm, ((size_t)b * a.L + t) * a.N + n);
+        }
+    }
+}
+
+// Walks the chunks backwards.  Chunk c's inputs were fetched during chunk
+// c + 1 (cp.async for the rows and the checkpoint, registers for B and C),
+// so each chunk waits only for copies that had a whole chunk to land; one
+// barrier per chunk.  hs and dt are per-thread columns (no barrier between
+// the recompute and the sweep).
+// Slot of states [4q, 4q + 4) in a thread's hs row: XOR-swizzled so that
+// the 16-byte accesses of any 8 consecutive threads hit distinct banks.
+template <int NS>
+__device__ __forceinline__ int hs_slot(int tid, int q)
+{
+    constexpr int kQ = NS / 4;
+    return q ^ ((tid / (8 / kQ)) % kQ);
+}
+
+__device__ __forceinline__ float4 lds4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ float f4(const float4 &v, int e) { return e == 0 ? v.x : e == 1 ? v.y : e == 2 ? v.z : v.w; }
+
+// Walks the chunks backwards.  Chunk c's inputs were fetched during chunk
+// c + 1 (cp.async for the rows and the checkpoint, registers for B and C),
+// so each chunk waits only for copies that had a whole chunk to land; one
+// barrier per chunk.  hs and dt are per-thread (no barrier between the
+// recompute and the sweep).
+//
+// In the sweep h_{i-1} is the previous row of hs (the checkpoint for the
+// chunk's first step), and
+//   ddt_i = x_i sum_n lam_i[n] B_i[n] + ln 2 sum_n (lam_i[n] a_i[n] h_{i-1}[n]) A[n] log2(e)
+// reuses the dx sum and the exponent's scaled A.
+template <typename T, int NS>
+__global__ void __launch_bounds__(kCta, kBwdCtasPerSm) s6_bwd_kernel(const BwdArgs a)
+{
+    constexpr int kBq = (kKc * 2 * NS + kCta - 1) / kCta;
+    constexpr float kLn2 = 0.693147180559945309f;
+    __shared__ BwdSmem<T, NS> sm;
     const int tid = threadIdx.x, lane = tid & 31;
-    const int d = blockIdx.x * kCta + tid;
+    const int d0 = blockIdx.x * kCta, d = d0 + tid;
     const int b = blockIdx.y;
     const bool active = d < a.D;
     const int dd = active ? d : 0;
     const int N = a.N, L = a.L, nch = (L + kKc - 1) / kKc;
-    const T *x = static_cast<const T *>(a.x), *dl = static_cast<const T *>(a.delta);
-    const T *zp = static_cast<const T *>(a.z), *go = static_cast<const T *>(a.dout);
-    float A[NS], Al[NS], lam[NS], gA[NS];
+    const bool gate = a.z != nullptr;
+    float Al[NS], lam[NS], gA[NS];
 #pragma unroll
     for (int n = 0; n < NS; n++) {
-        A[n] = (active && n < N) ? a.A[(size_t)dd * N + n] : 0.f;
-        Al[n] = A[n] * kLog2e;
+        Al[n] = (active && n < N) ? a.A[(size_t)dd * N + n] * kLog2e : 0.f;
         lam[n] = 0.f;   // a_{i+1} lam_{i+1}, carried backwards
-        gA[n] = 0.f;
+        gA[n] = 0.f;    // dA[n]: sum over steps of lam_i a_i h_{i-1} dt_i
     }
     const float bias = (active && a.bias) ? a.bias[dd] : 0.f;
     const float Dv = (active && a.Dskip) ? a.Dskip[dd] : 0.f;
     float gD = 0.f, gbias = 0.f;
 
+    float bq[kBq];
+    issue_chunk<T, NS>(a, sm, (nch - 1) & 1, b, d0, nch - 1, nch);
+    load_bc<T, NS, kBq>(a, b, nch - 1, bq);
     for (int c = nch - 1; c >= 0; c--) {
-        const int i0 = c * kKc, kn = min(kKc, L - i0);
-        __syncthreads();   // the previous chunk is done with bc, hs and sc
-        // this chunk's per-step scalars and the checkpoint, all loads issued together
+        const int buf = c & 1, i0 = c * kKc, kn = min(kKc, L - i0);
+        cp_async_wait_all();
 #pragma unroll
-        for (int k = 0; k < kKc; k++) {
-            float v = 0.f, xv = 0.f, g = 0.f, zv = 0.f;
-            if (active && k < kn) {
-                const int t = a.reverse ? L - 1 - (i0 + k) : i0 + k;
-                const size_t io = ((size_t)b * L + t) * a.D + dd;
-                v = ldv(dl, io) + bias;
-                xv = ldv(x, io);
-                g = ldv(go, io);
-                if (zp)
-                    zv = ldv(zp, io);
-            }
-            sc[k][0][tid] = v;
-            sc[k][1][tid] = xv;
-            sc[k][2][tid] = g;
-            sc[k][3][tid] = zv;
+        for (int j = 0; j < kBq; j++) {
+            const int e = tid + j * kCta;
+            if (e < kKc * 2 * NS)
+                sm.bc[buf][e / (2 * NS)][e % (2 * NS)] = bq[j];
         }
-        float hp[NS];
-        const float *ck = a.ckpt + (((size_t)b * nch + c) * a.D + dd) * N;
-#pragma unroll
-        for (int n = 0; n < NS; n++)
-            hp[n] = (active && n < N) ? ck[n] : 0.f;
-        stage_bc<T, NS, true>(a, b, i0, bc);
-        __syncthreads();
+        __syncthreads();   // chunk c's copies visible; every thread is past chunk c + 1
+        if (c > 0) {
+            issue_chunk<T, NS>(a, sm, buf ^ 1, b, d0, c - 1, nch);
+            load_bc<T, NS, kBq>(a, b, c - 1, bq);
+        }
+        const float(*bc)[2 * NS] = sm.bc[buf];
+        const T(*raw)[4][kCta] = sm.raw[buf];
         // recompute the chunk's states from the checkpoint
         {
             float h[NS];
 #pragma unroll
-            for (int n = 0; n < NS; n++)
-                h[n] = hp[n];
+            for (int q = 0; q < NS / 4; q++) {
+                const float4 c4 = lds4(&sm.ck[buf][tid][4 * q]);
+                h[4 * q] = c4.x;
+                h[4 * q + 1] = c4.y;
+                h[4 * q + 2] = c4.z;
+                h[4 * q + 3] = c4.w;
+            }
 #pragma unroll
             for (int k = 0; k < kKc; k++) {
-                const float dt = (k < kn) ? dt_of(sc[k][0][tid], a.softplus) : 0.f;
-                sc[k][4][tid] = dt;
-                const float dtx = dt * sc[k][1][tid];
+                const float dt = (k < kn) ? dt_of(tof(raw[k][0][tid]) + bias, a.softplus) : 0.f;
+                sm.dt[k][tid] = dt;
+                const float dtx = dt * tof(raw[k][1][tid]);
 #pragma unroll
-                for (int n = 0; n < NS; n++) {
-                    h[n] = fmaf(ex2_mufu(dt * Al[n]), h[n], dtx * bc[k][n]);
-                    hs[k][n][tid] = h[n];
+                for (int q = 0; q < NS / 4; q++) {
+                    const float4 Bq = lds4(&bc[k][4 * q]);
+#pragma unroll
+                    for (int e = 0; e < 4; e++) {
+                        const int n = 4 * q + e;
+                        h[n] = fmaf(ex2_mufu(dt * Al[n]), h[n], dtx * f4(Bq, e));
+                    }
+                    *reinterpret_cast<float4 *>(&sm.hs[k][tid][4 * hs_slot<NS>(tid, q)]) =
+                        make_float4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
                 }
             }
         }
-        // backward sweep over the chunk; hk holds h_k, loaded once per step
-        float hk[NS];
-#pragma unroll
-        for (int n = 0; n < NS; n++)
-            hk[n] = hs[kn - 1][n][tid];
+        // backward sweep over the chunk
 #pragma unroll 1
         for (int k = kn - 1; k >= 0; k--) {
             const int t = a.reverse ? L - 1 - (i0 + k) : i0 + k;
             const size_t row = (size_t)b * L + t;
             const size_t io = row * a.D + dd;
-            const float dt = sc[k][4][tid], xv = sc[k][1][tid], dtx = dt * xv;
-            const float gk = sc[k][2][tid], zk = sc[k][3][tid];
+            const float dt = sm.dt[k][tid], xv = tof(raw[k][1][tid]), dtx = dt * xv;
+            const float gk = tof(raw[k][2][tid]);
+            float hk[NS], hm[NS];   // h_i, h_{i-1}
+            const float *prow = k > 0 ? &sm.hs[k > 0 ? k - 1 : 0][tid][0] : &sm.ck[buf][tid][0];
+#pragma unroll
+            for (int q = 0; q < NS / 4; q++) {
+                const float4 h4 = lds4(&sm.hs[k][tid][4 * hs_slot<NS>(tid, q)]);
+                hk[4 * q] = h4.x;
+                hk[4 * q + 1] = h4.y;
+                hk[4 * q + 2] = h4.z;
+                hk[4 * q + 3] = h4.w;
+                const float4 p4 = lds4(prow + 4 * (k > 0 ? hs_slot<NS>(tid, q) : q));
+                hm[4 * q] = p4.x;
+                hm[4 * q + 1] = p4.y;
+                hm[4 * q + 2] = p4.z;
+                hm[4 * q + 3] = p4.w;
+            }
             // y_i = C . h_i + D x_i, then the gate
             float y = Dv * xv;
 #pragma unroll
-            for (int n = 0; n < NS; n++)
-                y = fmaf(bc[k][NS + n], hk[n], y);
+            for (int q = 0; q < NS / 4; q++) {
+                const float4 Cq = lds4(&bc[k][NS + 4 * q]);
+#pragma unroll
+                for (int e = 0; e < 4; e++)
+                    y = fmaf(f4(Cq, e), hk[4 * q + e], y);
+            }
             float dy = gk;
-            if (zp) {
+            if (gate) {
+                const float zk = tof(raw[k][3][tid]);
                 const float s = sigmoid_f(zk);
                 dy = gk * zk * s;
                 if (active && a.dz)
@@ -241,30 +391,34 @@ __global__ void __launch_bounds__(kCta) s6_bwd_kernel(const BwdArgs a)
             }
             if (!active)
                 dy = 0.f;
-            float ddt = 0.f, dxs = 0.f;
+            float dxs = 0.f, dtA = 0.f;
             float red[32];
 #pragma unroll
-            for (int n = 0; n < NS; n++) {
-                const float Bn = bc[k][n], Cn = bc[k][NS + n];
-                const float hprev = k > 0 ? hs[k - 1 < 0 ? 0 : k - 1][n][tid] : hp[n];
-                const float hcur = hk[n];
-                hk[n] = hprev;                                  // h_{k-1} for the next step
-                const float an = ex2_mufu(dt * Al[n]);
-                const float l = fmaf(dy, Cn, lam[n]);        // lam_i[n]
-                red[n] = l * dtx;                              // dB contribution
-                red[16 + n] = dy * hcur;                       // dC contribution
-                dxs = fmaf(l, Bn, dxs);
-                const float ah = an * hprev;
-                ddt = fmaf(l, fmaf(Bn, xv, A[n] * ah), ddt);
-                gA[n] = fmaf(l * dt, ah, gA[n]);
-                lam[n] = an * l;                               // a_i lam_i for step i - 1
+            for (int q = 0; q < NS / 4; q++) {
+                const float4 Bq = lds4(&bc[k][4 * q]), Cq = lds4(&bc[k][NS + 4 * q]);
+#pragma unroll
+                for (int e = 0; e < 4; e++) {
+                    const int n = 4 * q + e;
+                    const float Bn = f4(Bq, e), Cn = f4(Cq, e), hcur = hk[n];
+                    const float an = ex2_mufu(dt * Al[n]);
+                    const float ah = an * hm[n];                 // a_i h_{i-1}
+                    const float l = fmaf(dy, Cn, lam[n]);        // lam_i[n]
+                    red[n] = l * dtx;                            // dB contribution
+                    red[16 + n] = dy * hcur;                     // dC contribution
+                    dxs = fmaf(l, Bn, dxs);
+                    const float lah = l * ah;
+                    dtA = fmaf(lah, Al[n], dtA);
+                    gA[n] = fmaf(dt, lah, gA[n]);
+                    lam[n] = an * l;                             // a_i lam_i for step i - 1
+                }
             }
 #pragma unroll
             for (int n = NS; n < 16; n++)
                 red[n] = red[16 + n] = 0.f;
             if (active) {
+                const float ddt = fmaf(xv, dxs, kLn2 * dtA);
                 a.dx[io] = (a.accumulate ? a.dx[io] : 0.f) + fmaf(dy, Dv, dt * dxs);
-                const float dv = a.softplus ? ddt * sigmoid_f(sc[k][0][tid]) : ddt;
+                const float dv = a.softplus ? ddt * sigmoid_f(tof(raw[k][0][tid]) + bias) : ddt;
                 a.ddelta[io] = (a.accumulate ? a.ddelta[io] : 0.f) + dv;
                 gbias += dv;
                 gD = fmaf(dy, xv, gD);
@@ -292,6 +446,14 @@ template <typename T, int NS>
 cudaError_t launch_ns(const BwdArgs &a, cudaStream_t st)
 {
     dim3 g((a.D + kCta - 1) / kCta, a.Bsz);
+    static bool carveout_set = false;   // ask for the largest shared-memory carveout (6 CTAs per SM)
+    if (!carveout_set) {
+        cudaError_t e = cudaFuncSetAttribute(s6_bwd_kernel<T, NS>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                             (int)cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess)
+            return e;
+        carveout_set = true;
+    }
     s6_bwd_ckpt_kernel<T, NS><<<g, kCta, 0, st>>>(a);
     s6_bwd_kernel<T, NS><<<g, kCta, 0, st>>>(a);
     return cudaGetLastError();
@@ -312,7 +474,8 @@ cudaError_t launch_typed(const BwdArgs &a, cudaStream_t st)
 size_t bwd_workspace_bytes(int64_t Bsz, int64_t L, int64_t D, int64_t N)
 {
     const int64_t nch = (L + kKc - 1) / kKc;
-    return (size_t)Bsz * nch * D * N * sizeof(float);
+    const int64_t ns = N <= 4 ? 4 : N <= 8 ? 8 : 16;   // the kernels' padded state count
+    return (size_t)Bsz * nch * D * ns * sizeof(float);
 }
 
 cudaError_t launch_bwd(const BwdArgs &a, cudaStream_t st)

@@ -40,10 +40,11 @@ def _check(g, ref, tol):
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("reverse", [False, True])
-@pytest.mark.parametrize("N", [16, 5])
+@pytest.mark.parametrize("N", [16, 5, 8, 3])
 def test_bwd_matches_autograd(dtype, reverse, N):
-    """Every gradient; L = 101 leaves a ragged last 8-step chunk, D = 96
-    leaves a CTA of 64 channels half full."""
+    """Every gradient; L = 101 leaves a ragged last 4-step chunk and 16-step
+    input stage, D = 96 leaves a CTA of 64 channels half full; N covers the
+    three padded state counts (4, 8, 16)."""
     inp = ssm_gen.make_s6_inputs(2, 101, 96, N, dtype=dtype, seed=N + reverse, random_A=True,
                                  random_D=True)
     dout = np.random.default_rng(N).standard_normal(inp.x.shape).astype(np.float32)
@@ -62,6 +63,16 @@ def test_bwd_optional_inputs(gate, D, bias, softplus):
     dout = np.random.default_rng(4).standard_normal(inp.x.shape).astype(np.float32)
     g, ref = _run(inp, "f32", dout, False, gate=gate, D=D, bias=bias, softplus=softplus)
     assert ("dz" in g) == gate and ("dD" in g) == D and ("ddelta_bias" in g) == bias
+    _check(g, ref, TOL["f32"])
+
+
+@pytest.mark.parametrize("L", [1, 4, 15, 16, 17, 33])
+def test_bwd_short_sequences(L):
+    """Sequences of one step, one chunk, one input stage and just past
+    stage boundaries."""
+    inp = ssm_gen.make_s6_inputs(2, L, 64, 16, dtype="f32", seed=40 + L, random_A=True, random_D=True)
+    dout = np.random.default_rng(L).standard_normal(inp.x.shape).astype(np.float32)
+    g, ref = _run(inp, "f32", dout, L % 2 == 1)
     _check(g, ref, TOL["f32"])
 
 
