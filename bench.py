@@ -50,6 +50,7 @@ SMS = 148
 # capture matches them.
 NCU_TRAFFIC = {1: 271.73e6, 4: 398.97e6}
 NCU_TRAFFIC_STEP = 63.05e6
+NCU_TRAFFIC_BWD = {1: 410.81e6}
 
 
 def parse():
@@ -111,6 +112,17 @@ def alu_peak_elems(sm_mhz: float) -> float:
     (MUFU 16/clk/SM, FMA 128/clk/SM) finish together -> 64/3 elements per
     clock per SM."""
     return SMS * sm_mhz * 1e6 * (64.0 / 3.0)
+
+
+def bwd_alu_peak_elems(sm_mhz: float) -> float:
+    """Element rate the SM pipes allow for the backward (per element: three
+    exps -- checkpoint pass, recompute, adjoint -- and 19 FMA-pipe operations:
+    3 + 3 for the two forward recurrences, 11 in the adjoint step and about 2
+    adds of the dB / dC warp reduction).  Exps split between the MUFU unit
+    and an 8-operation FMA-pipe polynomial so that both pipes finish
+    together: x / 16 = (19 + 8 (3 - x)) / 128 gives x = 43 / 16, i.e.
+    256 / 43 elements per clock per SM."""
+    return SMS * sm_mhz * 1e6 * (256.0 / 43.0)
 
 
 # ------------------------------------------------------- multi-rank helpers
@@ -556,7 +568,7 @@ def run_bwd(args):
     # inputs x, delta, z, dout (dtype), B, C; outputs dx, ddelta, dz (fp32), dB, dC (fp32)
     nbytes = 4 * BLD * es + 2 * BL * inp.dstate * es + 3 * BLD * 4 + 2 * BL * inp.dstate * 4
     peaks, peak_src = load_peaks()
-    alu_peak = alu_peak_elems(peaks.get("sm_max_mhz", 1965.0))
+    alu_peak = bwd_alu_peak_elems(peaks.get("sm_max_mhz", 1965.0))
     return {
         "metric": "backward: scan elements/s (B·L·D·N)", "value": elems / (med * 1e-3),
         "unit": "elements/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
@@ -567,9 +579,11 @@ def run_bwd(args):
                    "algorithmic_bytes_per_step": nbytes, "elements_per_step": elems},
         "hbm_gbs": nbytes / (med * 1e-3) / 1e9,
         "roofline": {"bound": "alu", "achieved": elems / (med * 1e-3) / 1e9, "peak": alu_peak / 1e9,
-                     "unit": "Gelem/s", "frac": elems / (med * 1e-3) / alu_peak, "traffic": None,
-                     "peak_source": peak_src, "kernel_ms_median": med,
-                     "note": "three exps per element (checkpoint pass, recompute, adjoint)"},
+                     "unit": "Gelem/s", "frac": elems / (med * 1e-3) / alu_peak,
+                     "traffic": NCU_TRAFFIC_BWD.get(args.config), "peak_source": peak_src,
+                     "kernel_ms_median": med,
+                     "note": "achieved over the whole call (checkpoint pass + backward kernel); traffic of "
+                             "the backward kernel, the dominant launch"},
         "gpu_launches": 2 * args.steps, "clocks": clocks,
     }
 
