@@ -114,6 +114,14 @@ def alu_peak_elems(sm_mhz: float) -> float:
     return SMS * sm_mhz * 1e6 * (64.0 / 3.0)
 
 
+def step_stats(ms):
+    """Median, p10 and p90 of the per-step CUDA-event times (ms)."""
+    if len(ms) < 2:
+        return {"median": ms[0], "p10": ms[0], "p90": ms[0]}
+    q = statistics.quantiles(ms, n=10, method="inclusive")
+    return {"median": statistics.median(ms), "p10": q[0], "p90": q[-1]}
+
+
 def bwd_alu_peak_elems(sm_mhz: float) -> float:
     """Element rate the SM pipes allow for the backward (per element: three
     exps -- checkpoint pass, recompute, adjoint -- and 19 FMA-pipe operations:
@@ -411,6 +419,7 @@ def run_ours(args, rank, world, local_rank):
     res = {
         "metric": METRIC, "value": value, "unit": "elements/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step_ms,
+        "step_ms": step_stats(step_ms),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32" if info["dtype"] == "f32" else "bf16 storage, f32 compute",
         "data": "synthetic (seeded ssm_gen inputs with the workload's shapes and distributions)",
@@ -492,7 +501,7 @@ def run_step(args):
     return {
         "metric": "decode step: state elements/s (B·D·N) and HBM GB/s", "value": elems / (med * 1e-3),
         "unit": "elements/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": sum(ms) / len(ms), "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": sum(ms) / len(ms), "step_ms": step_stats(ms), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded ssm_gen inputs)",
         "config": {"workload": "decode_step_b512_d1536_n16_fp32", **STEP_WORKLOAD,
                    "l2": "flushed before every timed step (512 MB write)",
@@ -572,7 +581,7 @@ def run_bwd(args):
     return {
         "metric": "backward: scan elements/s (B·L·D·N)", "value": elems / (med * 1e-3),
         "unit": "elements/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": sum(ms) / len(ms), "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": sum(ms) / len(ms), "step_ms": step_stats(ms), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": info["dtype"], "data": "synthetic (seeded ssm_gen inputs)",
         "config": {"workload": info["name"] + "_fwd_direction_bwd", "config_index": args.config,
                    "l2": "flushed before every timed step (512 MB write)",
@@ -637,9 +646,19 @@ def cpu_baseline(cfg, budget_s=10.0):
     for _ in range(reps):
         _oracle_call(inp, info, sample, threads)
     el = time.perf_counter() - t0
+    # the same oracle on one core, over a sample sized to about budget_s / 2
+    col1_s = per_col_s * threads                      # estimate of one column on one core
+    one = cols[: max(1, min(len(cols), int(budget_s / 2 / col1_s)))]
+    reps1 = max(1, int(budget_s / 2 / (col1_s * len(one))))
+    t0 = time.perf_counter()
+    for _ in range(reps1):
+        _oracle_call(inp, info, one, 1)
+    el1 = time.perf_counter() - t0
     return {"value": len(sample) * reps * per_col / el, "unit": "elements/s", "cores": threads,
             "kind": "oracle", "sample": f"{what}, {el:.1f} s, float64 C oracle, OpenMP",
-            "seconds": el}
+            "seconds": el,
+            "one_core": {"value": len(one) * reps1 * per_col / el1, "unit": "elements/s", "cores": 1,
+                         "sample": f"{len(one)} of {ncols_all} columns x {reps1}, {el1:.1f} s"}}
 
 
 def run_reference(args):
