@@ -238,6 +238,55 @@ __device__ __forceinline__ void cp_async16(void *smem, const void *gmem)
     const unsigned sa = (unsigned)__cvta_generic_to_shared(smem);
     asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
 }
+// L2 eviction priorities for the bidirectional pass.  x and delta are read
+// by both warps of a pair, the first reader in the first half of its scan
+// and the second in the second half: the first read marks the line
+// evict-last (the 77 MB of x and delta of Vim-Small then stay in the 126 MB
+// L2 until the partner reads them), the second read and the read-once
+// streams (z, the final output) evict-first.  The parked half-outputs are
+// written evict-last and read back evict-first.
+#ifndef SSM_S6_L2HINT
+#define SSM_S6_L2HINT 1
+#endif
+__device__ __forceinline__ uint64_t l2_evict_last()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t l2_evict_first()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, uint64_t pol)
+{
+    const unsigned sa = (unsigned)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.ca.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(sa), "l"(gmem), "l"(pol)
+                 : "memory");
+}
+__device__ __forceinline__ void st_hint(float *p, const float (&v)[2], uint64_t pol)
+{
+    asm volatile("st.global.L2::cache_hint.v2.f32 [%0], {%1, %2}, %3;" ::"l"(p), "f"(v[0]), "f"(v[1]), "l"(pol)
+                 : "memory");
+}
+__device__ __forceinline__ void st_hint(float *p, const float (&v)[1], uint64_t pol)
+{
+    asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(p), "f"(v[0]), "l"(pol) : "memory");
+}
+__device__ __forceinline__ void st_hint(__nv_bfloat16 *p, const float (&v)[2], uint64_t pol)
+{
+    const __nv_bfloat162 h = __floats2bfloat162_rn(v[0], v[1]);
+    const uint32_t u = *reinterpret_cast<const uint32_t *>(&h);
+    asm volatile("st.global.L2::cache_hint.b32 [%0], %1, %2;" ::"l"(p), "r"(u), "l"(pol) : "memory");
+}
+__device__ __forceinline__ void st_hint(__nv_bfloat16 *p, const float (&v)[1], uint64_t pol)
+{
+    const __nv_bfloat16 h = __float2bfloat16_rn(v[0]);
+    const unsigned short u = *reinterpret_cast<const unsigned short *>(&h);
+    asm volatile("st.global.L2::cache_hint.b16 [%0], %1, %2;" ::"l"(p), "h"(u), "l"(pol) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int K> __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(K) : "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
@@ -408,11 +457,18 @@ __device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P,
     const bool pc_on = dbase + pc * (16 / (int)sizeof(T)) < a.D;
     const bool spc_on = dbase + spc * 4 < a.D;
     // stash rows of steps [i0, i1)
+    constexpr bool kHint = SSM_S6_L2HINT && BIDIR && !SUMMARY;
+    const uint64_t pol_last = kHint ? l2_evict_last() : 0, pol_first = kHint ? l2_evict_first() : 0;
     auto issue_stash = [&](int i0, int i1) {
         for (int i = i0 + spr; i < i1; i += RS::kRowsPerPass)
-            if (spc_on)
-                cp_async16(slot_of(i) + 3 * WS::kRowB + spc * 16,
-                           stash + (rowbase + tpos(i)) * a.D + dbase + spc * 4);
+            if (spc_on) {
+                char *dst = slot_of(i) + 3 * WS::kRowB + spc * 16;
+                const float *src = stash + (rowbase + tpos(i)) * a.D + dbase + spc * 4;
+                if (kHint)
+                    cp_async16(dst, src, pol_first);
+                else
+                    cp_async16(dst, src);
+            }
     };
     // x / delta / z (and stash when allowed) rows of group c
     auto issue_chunk = [&](int c, bool with_stash) {
@@ -423,10 +479,18 @@ __device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P,
             if (i < i1 && pc_on) {
                 char *slot = slot_of(i) + pc * 16;
                 const size_t ro = (rowbase + tpos(i)) * a.D + dbase + pc * (16 / (int)sizeof(T));
-                cp_async16(slot, x + ro);
-                cp_async16(slot + WS::kRowB, dl + ro);
-                if (!SUMMARY && GATE)
-                    cp_async16(slot + 2 * WS::kRowB, zp + ro);
+                if (kHint) {
+                    const uint64_t pxd = i < M ? pol_last : pol_first;
+                    cp_async16(slot, x + ro, pxd);
+                    cp_async16(slot + WS::kRowB, dl + ro, pxd);
+                    if (GATE)
+                        cp_async16(slot + 2 * WS::kRowB, zp + ro, pol_first);
+                } else {
+                    cp_async16(slot, x + ro);
+                    cp_async16(slot + WS::kRowB, dl + ro);
+                    if (!SUMMARY && GATE)
+                        cp_async16(slot + 2 * WS::kRowB, zp + ro);
+                }
             }
         }
         if (BIDIR && with_stash)
@@ -573,14 +637,20 @@ __device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P,
             if (!BIDIR) {
                 IO<T, CPL>::st(out + io, y);
             } else if (!kPhase2) {
-                IO<float, CPL>::st(stash + io, y);
+                if (kHint)
+                    st_hint(stash + io, y, pol_last);
+                else
+                    IO<float, CPL>::st(stash + io, y);
             } else {
                 float o[CPL];
                 IO<float, CPL>::ld(slot_of(i) + 3 * WS::kRowB + lane * CPL * 4, o);
 #pragma unroll
                 for (int c = 0; c < CPL; c++)
                     y[c] += o[c];
-                IO<T, CPL>::st(out + io, y);
+                if (kHint)
+                    st_hint(out + io, y, pol_first);
+                else
+                    IO<T, CPL>::st(out + io, y);
             }
         }
     };
