@@ -62,13 +62,14 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
-    p.add_argument("--op", default="scan", choices=["scan", "ordered", "conv", "step", "bwd"],
+    p.add_argument("--op", default="scan", choices=["scan", "ordered", "conv", "step", "bwd", "bidir_bwd"],
                    help="scan: the workload's scan (default); ordered: the same bidirectional "
                         "workload along a random order of the positions with 30%% of the tokens "
                         "masked; conv: the same with a width-4 conv1d + SiLU per direction computed "
                         "inside the scan; step: one decode step of a batch-512 x 1536-channel x "
                         "16-state fp32 state (ssm_step); bwd: the gradients (ssm_scan_bwd) of the "
-                        "forward direction of the workload")
+                        "forward direction of the workload; bidir_bwd: the gradients of the whole "
+                        "bidirectional scan (bidir_scan_bwd)")
     return p.parse_args()
 
 
@@ -516,9 +517,10 @@ def run_step(args):
 # ---------------------------------------------------------- backward
 
 def run_bwd(args):
-    """Gradients (ssm_scan_bwd) of the forward direction of an S6 workload,
-    inputs and the incoming gradient resident, L2 flushed before every step,
-    CUDA events on the launching stream."""
+    """Gradients of an S6 workload: of its forward direction (ssm_scan_bwd,
+    --op bwd) or of the whole bidirectional scan (bidir_scan_bwd, --op
+    bidir_bwd); inputs and the incoming gradient resident, L2 flushed before
+    every step, CUDA events on the launching stream."""
     import ctypes
     import torch
     from selective_state_space_24_b200 import build as ssm_build
@@ -546,12 +548,27 @@ def run_bwd(args):
     p = lambda t: t.data_ptr()
     stream = torch.cuda.current_stream(device)
     sh = stream.cuda_stream
+    bidir = args.op == "bidir_bwd"
+    if bidir:
+        assert info["ndir"] == 2, "bidir_bwd: a bidirectional workload"
+        zb, Bb, Cb = io(inp.z_b), io(inp.B_b), io(inp.C_b)
+        Ab, biasb, Db = f32(inp.A_b), f32(inp.dt_bias_b), f32(inp.D_b)
+        pf = ssm.ssm_dir_params(p(bias), p(A), p(Bm), p(Cm), p(Dv), p(z), None)
+        pb = ssm.ssm_dir_params(p(biasb), p(Ab), p(Bb), p(Cb), p(Db), p(zb), None)
+        gb = [e(A.shape), e(Bb.shape), e(Cb.shape), e(Dv.shape), e(x.shape), e(bias.shape)]
+        gf_c = ssm.ssm_dir_grads(*[p(t) for t in (g[2], g[3], g[4], g[5], g[6], g[7])])
+        gb_c = ssm.ssm_dir_grads(*[p(t) for t in gb])
 
     def step():
-        st = lib.ssm_scan_bwd(ctypes.byref(dims), p(x), p(delta), p(bias), 1, p(A), p(Bm), p(Cm), p(Dv),
-                              p(z), 0, p(dout), *[p(t) for t in g], p(ws), need, sh)
+        if bidir:
+            st = lib.bidir_scan_bwd(ctypes.byref(dims), p(x), p(delta), 1, ctypes.byref(pf), ctypes.byref(pb),
+                                    p(dout), p(g[0]), p(g[1]), ctypes.byref(gf_c), ctypes.byref(gb_c), p(ws),
+                                    need, sh)
+        else:
+            st = lib.ssm_scan_bwd(ctypes.byref(dims), p(x), p(delta), p(bias), 1, p(A), p(Bm), p(Cm), p(Dv),
+                                  p(z), 0, p(dout), *[p(t) for t in g], p(ws), need, sh)
         if st != 0:
-            raise RuntimeError(f"ssm_scan_bwd returned {ssm.STATUS.get(st, st)}")
+            raise RuntimeError(f"backward returned {ssm.STATUS.get(st, st)}")
 
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
     for _ in range(max(args.warmup, 3)):
@@ -571,11 +588,14 @@ def run_bwd(args):
     clocks = sampler.stop()
     ms = [a.elapsed_time(b) for a, b in evs]
     med = statistics.median(ms)
-    elems = inp.batch * inp.seqlen * inp.dim * inp.dstate
+    nd = 2 if bidir else 1
+    elems = nd * inp.batch * inp.seqlen * inp.dim * inp.dstate
     es = 4 if inp.dtype == "f32" else 2
     BL, BLD = inp.batch * inp.seqlen, inp.batch * inp.seqlen * inp.dim
-    # inputs x, delta, z, dout (dtype), B, C; outputs dx, ddelta, dz (fp32), dB, dC (fp32)
-    nbytes = 4 * BLD * es + 2 * BL * inp.dstate * es + 3 * BLD * 4 + 2 * BL * inp.dstate * 4
+    # inputs x, delta, dout (dtype) and per direction z, B, C; outputs dx, ddelta (fp32) and per
+    # direction dz, dB, dC (fp32)
+    nbytes = (3 + nd) * BLD * es + 2 * nd * BL * inp.dstate * es + (2 + nd) * BLD * 4 \
+        + 2 * nd * BL * inp.dstate * 4
     peaks, peak_src = load_peaks()
     alu_peak = bwd_alu_peak_elems(peaks.get("sm_max_mhz", 1965.0))
     return {
@@ -583,17 +603,18 @@ def run_bwd(args):
         "unit": "elements/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": sum(ms) / len(ms), "step_ms": step_stats(ms), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": info["dtype"], "data": "synthetic (seeded ssm_gen inputs)",
-        "config": {"workload": info["name"] + "_fwd_direction_bwd", "config_index": args.config,
+        "config": {"workload": info["name"] + ("_bidir_bwd" if bidir else "_fwd_direction_bwd"),
+                   "config_index": args.config,
                    "l2": "flushed before every timed step (512 MB write)",
                    "algorithmic_bytes_per_step": nbytes, "elements_per_step": elems},
         "hbm_gbs": nbytes / (med * 1e-3) / 1e9,
         "roofline": {"bound": "alu", "achieved": elems / (med * 1e-3) / 1e9, "peak": alu_peak / 1e9,
                      "unit": "Gelem/s", "frac": elems / (med * 1e-3) / alu_peak,
-                     "traffic": NCU_TRAFFIC_BWD.get(args.config), "peak_source": peak_src,
+                     "traffic": None if bidir else NCU_TRAFFIC_BWD.get(args.config), "peak_source": peak_src,
                      "kernel_ms_median": med,
-                     "note": "achieved over the whole call (checkpoint pass + backward kernel); traffic of "
-                             "the backward kernel, the dominant launch"},
-        "gpu_launches": 2 * args.steps, "clocks": clocks,
+                     "note": "achieved over the whole call (checkpoint pass + backward kernel per direction); "
+                             "traffic of the backward kernel, the dominant launch"},
+        "gpu_launches": 2 * nd * args.steps, "clocks": clocks,
     }
 
 
@@ -704,7 +725,7 @@ def main():
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
         return
-    if args.op in ("step", "bwd"):
+    if args.op in ("step", "bwd", "bidir_bwd"):
         if rank == 0:
             print(json.dumps(run_step(args) if args.op == "step" else run_bwd(args)), flush=True)
         return

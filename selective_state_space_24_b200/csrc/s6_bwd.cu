@@ -304,6 +304,15 @@ __global__ void __launch_bounds__(kCta, kBwdCtasPerSm) s6_bwd_kernel(const BwdAr
     float bq[kBq];
     issue_chunk<T, NS>(a, sm, (nch - 1) & 1, b, d0, nch - 1, nch);
     load_bc<T, NS, kBq>(a, b, nch - 1, bq);
+    // accumulate: the dx and ddelta already there are loaded one step ahead
+    // of their use (the sweep's order: chunks and steps descending)
+    const bool acc = a.accumulate && active;
+    auto io_of = [&](int i) { return ((size_t)b * L + (a.reverse ? L - 1 - i : i)) * a.D + dd; };
+    float nx_dx = 0.f, nx_dd = 0.f;
+    if (acc) {
+        nx_dx = a.dx[io_of(L - 1)];
+        nx_dd = a.ddelta[io_of(L - 1)];
+    }
     for (int c = nch - 1; c >= 0; c--) {
         const int buf = c & 1, i0 = c * kKc, kn = min(kKc, L - i0);
         cp_async_wait_all();
@@ -357,6 +366,11 @@ __global__ void __launch_bounds__(kCta, kBwdCtasPerSm) s6_bwd_kernel(const BwdAr
             const size_t io = row * a.D + dd;
             const float dt = sm.dt[k][tid], xv = tof(raw[k][1][tid]), dtx = dt * xv;
             const float gk = tof(raw[k][2][tid]);
+            const float old_dx = nx_dx, old_dd = nx_dd;
+            if (acc && i0 + k > 0) {
+                nx_dx = a.dx[io_of(i0 + k - 1)];
+                nx_dd = a.ddelta[io_of(i0 + k - 1)];
+            }
             float hk[NS], hm[NS];   // h_i, h_{i-1}
             const float *prow = k > 0 ? &sm.hs[k > 0 ? k - 1 : 0][tid][0] : &sm.ck[buf][tid][0];
 #pragma unroll
@@ -417,9 +431,9 @@ __global__ void __launch_bounds__(kCta, kBwdCtasPerSm) s6_bwd_kernel(const BwdAr
                 red[n] = red[16 + n] = 0.f;
             if (active) {
                 const float ddt = fmaf(xv, dxs, kLn2 * dtA);
-                a.dx[io] = (a.accumulate ? a.dx[io] : 0.f) + fmaf(dy, Dv, dt * dxs);
+                a.dx[io] = old_dx + fmaf(dy, Dv, dt * dxs);
                 const float dv = a.softplus ? ddt * sigmoid_f(tof(raw[k][0][tid]) + bias) : ddt;
-                a.ddelta[io] = (a.accumulate ? a.ddelta[io] : 0.f) + dv;
+                a.ddelta[io] = old_dd + dv;
                 gbias += dv;
                 gD = fmaf(dy, xv, gD);
             }
