@@ -184,3 +184,29 @@ def test_conv_validation(lib):
     mis = ssm.ssm_conv_params(FAKE + 4, None, 3, 1)
     assert lib.ssm_scan_fwd_conv(ctypes.byref(dims), FAKE, ctypes.byref(mis), FAKE, None, 1, FAKE, FAKE,
                                  FAKE, None, None, 0, FAKE, None, None, 0, None) == 3
+
+
+def test_bwd_workspace_and_validation(lib):
+    """The backward's workspace holds the states entering every 4-step chunk,
+    N padded to 4, 8 or 16 floats per channel; a short or misaligned
+    workspace and missing gradient outputs are rejected before any launch."""
+    for N in range(1, 17):
+        ns = 4 if N <= 4 else 8 if N <= 8 else 16
+        dims = _dims(2, 101, 96, N)
+        assert lib.ssm_scan_bwd_workspace_size(ctypes.byref(dims)) == 2 * 26 * 96 * ns * 4
+    assert lib.ssm_scan_bwd_workspace_size(ctypes.byref(_dims(N=17))) == 0
+    assert lib.ssm_scan_bwd_workspace_size(None) == 0
+
+    dims = _dims(2, 101, 96, 16)
+    need = lib.ssm_scan_bwd_workspace_size(ctypes.byref(dims))
+
+    def bwd(ws=FAKE, wsb=need, dA=FAKE, dD=FAKE):
+        # x, delta, bias, softplus, A, B, C, D, z, reverse, dout, dx, ddelta, dA, dB, dC, dD, dz, dbias
+        return lib.ssm_scan_bwd(ctypes.byref(dims), FAKE, FAKE, None, 1, FAKE, FAKE, FAKE, FAKE, None, 0,
+                                FAKE, FAKE, FAKE, dA, FAKE, FAKE, dD, None, None, ws, wsb, None)
+
+    assert bwd(wsb=need - 1) == 5          # SSM_ERR_WORKSPACE_TOO_SMALL
+    assert bwd(ws=None) == 5
+    assert bwd(ws=FAKE + 4) == 3           # SSM_ERR_MISALIGNED
+    assert bwd(dA=None) == 1               # SSM_ERR_INVALID_ARG
+    assert bwd(dD=None) == 1               # D given without its gradient
