@@ -50,7 +50,7 @@ SMS = 148
 # capture matches them.
 NCU_TRAFFIC = {1: 193.01e6, 4: 398.97e6}
 NCU_TRAFFIC_STEP = 63.05e6
-NCU_TRAFFIC_BWD = {1: 410.81e6}
+NCU_TRAFFIC_BWD = {1: 409.56e6}
 
 
 def parse():

@@ -15,16 +15,17 @@
 //   dA[n] += lam_i[n] dt_i a_i[n] h_{i-1}[n];  dD += dy_i x_i
 //   ddelta_i = ddt_i softplus'(v_i) = ddt_i sigmoid(v_i);  dbias += ddelta_i
 //
-// Two kernels.  s6_bwd_ckpt_kernel runs the forward recurrence once and
-// stores h entering every chunk of kKc steps (padded to the template state
-// count, so each channel's checkpoint is whole 16-byte vectors).  s6_bwd_kernel walks the
-// chunks backwards: it recomputes the chunk's states into shared memory
-// from the checkpoint, then sweeps the chunk backwards with lam in
-// registers.  One thread per (b, d); a CTA holds 64 channels of one batch
-// row and stages each chunk's B and C rows in shared memory; the per-step
-// inputs of a chunk are loaded together before its work.  dB and dC are
-// summed over a warp's 32 channels with a butterfly of shuffles, then added
-// with one atomic per (warp, t, n).  All gradients are float32.
+// Two kernels, one thread per (b, d), a CTA holding 64 channels of one
+// batch row.  s6_bwd_ckpt_kernel runs the forward recurrence once and stores
+// h entering every chunk of kKc steps (padded to the template state count,
+// so each channel's checkpoint is whole 16-byte vectors); its inputs arrive
+// kStage steps at a time, the next stage's in flight during the current one.
+// s6_bwd_kernel walks the chunks backwards: it recomputes the chunk's states
+// into shared memory from the checkpoint, then sweeps the chunk backwards
+// with lam in registers; the next chunk's inputs and checkpoint are copied
+// (cp.async) while the current one is computed.  dB and dC are summed over a
+// warp's 32 channels with a butterfly of shuffles, then added with one
+// atomic per (warp, t, n).  All gradients are float32.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -71,6 +72,31 @@ __device__ __forceinline__ float warp_transpose_sum(float (&v)[32])
     return v[0];
 }
 
+__device__ __forceinline__ float4 lds4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ float2 lo2(const float4 &v) { return make_float2(v.x, v.y); }
+__device__ __forceinline__ float2 hi2(const float4 &v) { return make_float2(v.z, v.w); }
+__device__ __forceinline__ float2 ex2_pair(float2 v) { return make_float2(ex2_mufu(v.x), ex2_mufu(v.y)); }
+
+// One step of the recurrence for NS states held as NS / 2 pairs (packed
+// f32x2 instructions, each lane rounded as the scalar multiply / FMA):
+// h = 2^(dt A log2 e) h + (dt x) B, with Brow 16-byte aligned in shared memory.
+template <int NS>
+__device__ __forceinline__ void recur_pairs(float2 (&h)[NS / 2], const float2 (&Al)[NS / 2], float dt, float dtx,
+                                            const float *Brow)
+{
+    const float2 dt2 = make_float2(dt, dt), dtx2 = make_float2(dtx, dtx);
+#pragma unroll
+    for (int q = 0; q < NS / 4; q++) {
+        const float4 B4 = lds4(Brow + 4 * q);
+#pragma unroll
+        for (int e = 0; e < 2; e++) {
+            const int p = 2 * q + e;
+            const float2 an = ex2_pair(__fmul2_rn(dt2, Al[p]));
+            h[p] = __ffma2_rn(an, h[p], __fmul2_rn(dtx2, e == 0 ? lo2(B4) : hi2(B4)));
+        }
+    }
+}
+
 // The forward inputs of kStage steps from scan index i0: this thread's
 // delta and x, and its kPer share of the steps' B rows (element e = thread +
 // j kCta of the (step, state) tile).  Zero past L, N or D.
@@ -114,17 +140,19 @@ __global__ void __launch_bounds__(kCta) s6_bwd_ckpt_kernel(const BwdArgs a)
     constexpr int kPer = kStage * NS / kCta;
     static_assert(kPer * kCta == kStage * NS, "stage tile must split evenly over the CTA");
     static_assert(kStage % kKc == 0, "a stage holds whole chunks");
-    __shared__ float bs[2][kStage][NS];
+    __shared__ __align__(16) float bs[2][kStage][NS];
     const int d = blockIdx.x * kCta + threadIdx.x;
     const int b = blockIdx.y;
     const bool active = d < a.D;
     const int dd = active ? d : 0;
     const int N = a.N, L = a.L, nch = (L + kKc - 1) / kKc, nst = (L + kStage - 1) / kStage;
-    float Al[NS], h[NS];
+    float2 Al[NS / 2], h[NS / 2];
 #pragma unroll
-    for (int n = 0; n < NS; n++) {
-        Al[n] = (active && n < N) ? a.A[(size_t)dd * N + n] * kLog2e : 0.f;
-        h[n] = 0.f;
+    for (int p = 0; p < NS / 2; p++) {
+        const int n = 2 * p;
+        Al[p] = make_float2((active && n < N) ? a.A[(size_t)dd * N + n] * kLog2e : 0.f,
+                            (active && n + 1 < N) ? a.A[(size_t)dd * N + n + 1] * kLog2e : 0.f);
+        h[p] = make_float2(0.f, 0.f);
     }
     const float bias = (active && a.bias) ? a.bias[dd] : 0.f;
     float v[kStage], xv[kStage], bq[kPer];
@@ -149,13 +177,10 @@ __global__ void __launch_bounds__(kCta) s6_bwd_ckpt_kernel(const BwdArgs a)
                 float4 *ck = reinterpret_cast<float4 *>(a.ckpt + (((size_t)b * nch + i / kKc) * a.D + dd) * NS);
 #pragma unroll
                 for (int q = 0; q < NS / 4; q++)
-                    ck[q] = make_float4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
+                    ck[q] = make_float4(h[2 * q].x, h[2 * q].y, h[2 * q + 1].x, h[2 * q + 1].y);
             }
             const float dt = i < L ? dt_of(v[k] + bias, a.softplus) : 0.f;
-            const float dtx = dt * xv[k];
-#pragma unroll
-            for (int n = 0; n < NS; n++)
-                h[n] = fmaf(ex2_mufu(dt * Al[n]), h[n], dtx * bc[k][n]);
+            recur_pairs<NS>(h, Al, dt, dt * xv[k], bc[k]);
         }
         if (more) {
 #pragma unroll
@@ -264,8 +289,6 @@ __device__ __forceinline__ int hs_slot(int tid, int q)
     return q ^ ((tid / (8 / kQ)) % kQ);
 }
 
-__device__ __forceinline__ float4 lds4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
-__device__ __forceinline__ float f4(const float4 &v, int e) { return e == 0 ? v.x : e == 1 ? v.y : e == 2 ? v.z : v.w; }
 
 // Walks the chunks backwards.  Chunk c's inputs were fetched during chunk
 // c + 1 (cp.async for the rows and the checkpoint, registers for B and C),
@@ -290,12 +313,15 @@ __global__ void __launch_bounds__(kCta, kBwdCtasPerSm) s6_bwd_kernel(const BwdAr
     const int dd = active ? d : 0;
     const int N = a.N, L = a.L, nch = (L + kKc - 1) / kKc;
     const bool gate = a.z != nullptr;
-    float Al[NS], lam[NS], gA[NS];
+    // state pairs (2p, 2p + 1) for the packed f32x2 instructions
+    float2 Al[NS / 2], lam[NS / 2], gA[NS / 2];
 #pragma unroll
-    for (int n = 0; n < NS; n++) {
-        Al[n] = (active && n < N) ? a.A[(size_t)dd * N + n] * kLog2e : 0.f;
-        lam[n] = 0.f;   // a_{i+1} lam_{i+1}, carried backwards
-        gA[n] = 0.f;    // dA[n]: sum over steps of lam_i a_i h_{i-1} dt_i
+    for (int p = 0; p < NS / 2; p++) {
+        const int n = 2 * p;
+        Al[p] = make_float2((active && n < N) ? a.A[(size_t)dd * N + n] * kLog2e : 0.f,
+                            (active && n + 1 < N) ? a.A[(size_t)dd * N + n + 1] * kLog2e : 0.f);
+        lam[p] = make_float2(0.f, 0.f);   // a_{i+1} lam_{i+1}, carried backwards
+        gA[p] = make_float2(0.f, 0.f);    // dA: sum over steps of lam_i a_i h_{i-1} dt_i
     }
     const float bias = (active && a.bias) ? a.bias[dd] : 0.f;
     const float Dv = (active && a.Dskip) ? a.Dskip[dd] : 0.f;
@@ -331,31 +357,22 @@ __global__ void __launch_bounds__(kCta, kBwdCtasPerSm) s6_bwd_kernel(const BwdAr
         const T(*raw)[4][kCta] = sm.raw[buf];
         // recompute the chunk's states from the checkpoint
         {
-            float h[NS];
+            float2 h[NS / 2];
 #pragma unroll
             for (int q = 0; q < NS / 4; q++) {
                 const float4 c4 = lds4(&sm.ck[buf][tid][4 * q]);
-                h[4 * q] = c4.x;
-                h[4 * q + 1] = c4.y;
-                h[4 * q + 2] = c4.z;
-                h[4 * q + 3] = c4.w;
+                h[2 * q] = lo2(c4);
+                h[2 * q + 1] = hi2(c4);
             }
 #pragma unroll
             for (int k = 0; k < kKc; k++) {
                 const float dt = (k < kn) ? dt_of(tof(raw[k][0][tid]) + bias, a.softplus) : 0.f;
                 sm.dt[k][tid] = dt;
-                const float dtx = dt * tof(raw[k][1][tid]);
+                recur_pairs<NS>(h, Al, dt, dt * tof(raw[k][1][tid]), bc[k]);
 #pragma unroll
-                for (int q = 0; q < NS / 4; q++) {
-                    const float4 Bq = lds4(&bc[k][4 * q]);
-#pragma unroll
-                    for (int e = 0; e < 4; e++) {
-                        const int n = 4 * q + e;
-                        h[n] = fmaf(ex2_mufu(dt * Al[n]), h[n], dtx * f4(Bq, e));
-                    }
+                for (int q = 0; q < NS / 4; q++)
                     *reinterpret_cast<float4 *>(&sm.hs[k][tid][4 * hs_slot<NS>(tid, q)]) =
-                        make_float4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
-                }
+                        make_float4(h[2 * q].x, h[2 * q].y, h[2 * q + 1].x, h[2 * q + 1].y);
             }
         }
         // backward sweep over the chunk
@@ -371,30 +388,22 @@ __global__ void __launch_bounds__(kCta, kBwdCtasPerSm) s6_bwd_kernel(const BwdAr
                 nx_dx = a.dx[io_of(i0 + k - 1)];
                 nx_dd = a.ddelta[io_of(i0 + k - 1)];
             }
-            float hk[NS], hm[NS];   // h_i, h_{i-1}
+            float4 hk[NS / 4], hm[NS / 4];   // h_i, h_{i-1}
             const float *prow = k > 0 ? &sm.hs[k > 0 ? k - 1 : 0][tid][0] : &sm.ck[buf][tid][0];
 #pragma unroll
             for (int q = 0; q < NS / 4; q++) {
-                const float4 h4 = lds4(&sm.hs[k][tid][4 * hs_slot<NS>(tid, q)]);
-                hk[4 * q] = h4.x;
-                hk[4 * q + 1] = h4.y;
-                hk[4 * q + 2] = h4.z;
-                hk[4 * q + 3] = h4.w;
-                const float4 p4 = lds4(prow + 4 * (k > 0 ? hs_slot<NS>(tid, q) : q));
-                hm[4 * q] = p4.x;
-                hm[4 * q + 1] = p4.y;
-                hm[4 * q + 2] = p4.z;
-                hm[4 * q + 3] = p4.w;
+                hk[q] = lds4(&sm.hs[k][tid][4 * hs_slot<NS>(tid, q)]);
+                hm[q] = lds4(prow + 4 * (k > 0 ? hs_slot<NS>(tid, q) : q));
             }
             // y_i = C . h_i + D x_i, then the gate
-            float y = Dv * xv;
+            float2 y2 = make_float2(0.f, 0.f);
 #pragma unroll
             for (int q = 0; q < NS / 4; q++) {
-                const float4 Cq = lds4(&bc[k][NS + 4 * q]);
-#pragma unroll
-                for (int e = 0; e < 4; e++)
-                    y = fmaf(f4(Cq, e), hk[4 * q + e], y);
+                const float4 C4 = lds4(&bc[k][NS + 4 * q]);
+                y2 = __ffma2_rn(lo2(C4), lo2(hk[q]), y2);
+                y2 = __ffma2_rn(hi2(C4), hi2(hk[q]), y2);
             }
+            const float y = fmaf(Dv, xv, y2.x + y2.y);
             float dy = gk;
             if (gate) {
                 const float zk = tof(raw[k][3][tid]);
@@ -405,30 +414,36 @@ __global__ void __launch_bounds__(kCta, kBwdCtasPerSm) s6_bwd_kernel(const BwdAr
             }
             if (!active)
                 dy = 0.f;
-            float dxs = 0.f, dtA = 0.f;
+            const float2 dt2 = make_float2(dt, dt), dtx2 = make_float2(dtx, dtx), dy2 = make_float2(dy, dy);
+            float2 dxs2 = make_float2(0.f, 0.f), dtA2 = make_float2(0.f, 0.f);
             float red[32];
 #pragma unroll
             for (int q = 0; q < NS / 4; q++) {
-                const float4 Bq = lds4(&bc[k][4 * q]), Cq = lds4(&bc[k][NS + 4 * q]);
+                const float4 B4 = lds4(&bc[k][4 * q]), C4 = lds4(&bc[k][NS + 4 * q]);
 #pragma unroll
-                for (int e = 0; e < 4; e++) {
-                    const int n = 4 * q + e;
-                    const float Bn = f4(Bq, e), Cn = f4(Cq, e), hcur = hk[n];
-                    const float an = ex2_mufu(dt * Al[n]);
-                    const float ah = an * hm[n];                 // a_i h_{i-1}
-                    const float l = fmaf(dy, Cn, lam[n]);        // lam_i[n]
-                    red[n] = l * dtx;                            // dB contribution
-                    red[16 + n] = dy * hcur;                     // dC contribution
-                    dxs = fmaf(l, Bn, dxs);
-                    const float lah = l * ah;
-                    dtA = fmaf(lah, Al[n], dtA);
-                    gA[n] = fmaf(dt, lah, gA[n]);
-                    lam[n] = an * l;                             // a_i lam_i for step i - 1
+                for (int e = 0; e < 2; e++) {
+                    const int p = 2 * q + e, n = 2 * p;
+                    const float2 Bn = e ? hi2(B4) : lo2(B4), Cn = e ? hi2(C4) : lo2(C4);
+                    const float2 hcur = e ? hi2(hk[q]) : lo2(hk[q]), hprev = e ? hi2(hm[q]) : lo2(hm[q]);
+                    const float2 an = ex2_pair(__fmul2_rn(dt2, Al[p]));
+                    const float2 l = __ffma2_rn(dy2, Cn, lam[p]);       // lam_i
+                    const float2 rb = __fmul2_rn(l, dtx2);              // dB contributions
+                    const float2 rc = __fmul2_rn(dy2, hcur);            // dC contributions
+                    red[n] = rb.x;
+                    red[n + 1] = rb.y;
+                    red[16 + n] = rc.x;
+                    red[16 + n + 1] = rc.y;
+                    dxs2 = __ffma2_rn(l, Bn, dxs2);
+                    const float2 lah = __fmul2_rn(l, __fmul2_rn(an, hprev));   // lam_i a_i h_{i-1}
+                    dtA2 = __ffma2_rn(lah, Al[p], dtA2);
+                    gA[p] = __ffma2_rn(dt2, lah, gA[p]);
+                    lam[p] = __fmul2_rn(an, l);                         // a_i lam_i for step i - 1
                 }
             }
 #pragma unroll
             for (int n = NS; n < 16; n++)
                 red[n] = red[16 + n] = 0.f;
+            const float dxs = dxs2.x + dxs2.y, dtA = dtA2.x + dtA2.y;
             if (active) {
                 const float ddt = fmaf(xv, dxs, kLn2 * dtA);
                 a.dx[io] = old_dx + fmaf(dy, Dv, dt * dxs);
@@ -446,9 +461,12 @@ __global__ void __launch_bounds__(kCta, kBwdCtasPerSm) s6_bwd_kernel(const BwdAr
     }
     if (active) {
 #pragma unroll
-        for (int n = 0; n < NS; n++)
-            if (n < N)
-                atomicAdd(a.dA + (size_t)dd * N + n, gA[n]);
+        for (int p = 0; p < NS / 2; p++) {
+            if (2 * p < N)
+                atomicAdd(a.dA + (size_t)dd * N + 2 * p, gA[p].x);
+            if (2 * p + 1 < N)
+                atomicAdd(a.dA + (size_t)dd * N + 2 * p + 1, gA[p].y);
+        }
         if (a.dD)
             atomicAdd(a.dD + dd, gD);
         if (a.dbias)
