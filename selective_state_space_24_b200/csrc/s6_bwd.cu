@@ -30,6 +30,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "internal.h"
 #include "s6_math.cuh"
 
@@ -478,13 +480,19 @@ template <typename T, int NS>
 cudaError_t launch_ns(const BwdArgs &a, cudaStream_t st)
 {
     dim3 g((a.D + kCta - 1) / kCta, a.Bsz);
-    static bool carveout_set = false;   // ask for the largest shared-memory carveout (6 CTAs per SM)
-    if (!carveout_set) {
-        cudaError_t e = cudaFuncSetAttribute(s6_bwd_kernel<T, NS>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                             (int)cudaSharedmemCarveoutMaxShared);
+    // ask once per device for the largest shared-memory carveout (6 CTAs per SM)
+    static std::atomic<uint64_t> carveout_set{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(carveout_set.load(std::memory_order_relaxed) & bit)) {
+        e = cudaFuncSetAttribute(s6_bwd_kernel<T, NS>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared);
         if (e != cudaSuccess)
             return e;
-        carveout_set = true;
+        carveout_set.fetch_or(bit, std::memory_order_relaxed);
     }
     s6_bwd_ckpt_kernel<T, NS><<<g, kCta, 0, st>>>(a);
     s6_bwd_kernel<T, NS><<<g, kCta, 0, st>>>(a);
