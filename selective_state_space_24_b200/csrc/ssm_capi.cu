@@ -325,13 +325,11 @@ size_t ssm_scan_bwd_workspace_size(const ssm_dims *dims)
 
 namespace {
 
-// One direction's backward launch (ssm_scan_bwd, bidir_scan_bwd): checks,
-// zeroes the accumulated gradients, launches.  accumulate: add into dx and
-// ddelta instead of writing them.
-ssm_status bwd_one(const ssm_dims *dims, const void *x, const void *delta, int delta_softplus,
-                   const ssm_dir_params &p, int reverse, const void *dout, float *dx, float *ddelta,
-                   const ssm_dir_grads &g, void *workspace, size_t workspace_bytes, int accumulate,
-                   cudaStream_t st)
+// The arguments of one direction's backward (ssm_scan_bwd, bidir_scan_bwd),
+// checked before anything is launched.
+ssm_status bwd_check(const ssm_dims *dims, const void *x, const void *delta, const ssm_dir_params &p,
+                     const void *dout, const float *dx, const float *ddelta, const ssm_dir_grads &g,
+                     const void *workspace, size_t workspace_bytes)
 {
     if (!x || !delta || !p.A || !p.B || !p.C || !dout || !dx || !ddelta || !g.dA || !g.dB || !g.dC)
         return SSM_ERR_INVALID_ARG;
@@ -345,6 +343,20 @@ ssm_status bwd_one(const ssm_dims *dims, const void *x, const void *delta, int d
     const size_t need = ssm::bwd_workspace_bytes(dims->batch, dims->seqlen, dims->dim, dims->dstate);
     if (!workspace || workspace_bytes < need)
         return SSM_ERR_WORKSPACE_TOO_SMALL;
+    return SSM_OK;
+}
+
+// One direction's backward launch: checks, zeroes the accumulated
+// gradients, launches.  accumulate: add into dx and ddelta instead of
+// writing them.
+ssm_status bwd_one(const ssm_dims *dims, const void *x, const void *delta, int delta_softplus,
+                   const ssm_dir_params &p, int reverse, const void *dout, float *dx, float *ddelta,
+                   const ssm_dir_grads &g, void *workspace, size_t workspace_bytes, int accumulate,
+                   cudaStream_t st)
+{
+    ssm_status s = bwd_check(dims, x, delta, p, dout, dx, ddelta, g, workspace, workspace_bytes);
+    if (s != SSM_OK)
+        return s;
     const size_t nDN = (size_t)dims->dim * dims->dstate;
     const size_t nBLN = (size_t)dims->batch * dims->seqlen * dims->dstate;
     if (cudaMemsetAsync(g.dA, 0, nDN * sizeof(float), st) != cudaSuccess ||
@@ -436,6 +448,10 @@ ssm_status bidir_scan_bwd(const ssm_dims *dims, const void *x, const void *delta
             return s;
         return bwd_empty(dims, *bwd, *grad_bwd, st);
     }
+    // both directions' arguments first, so that a refused call launches nothing
+    if ((s = bwd_check(dims, x, delta, *fwd, dout, dx, ddelta, *grad_fwd, workspace, workspace_bytes)) != SSM_OK ||
+        (s = bwd_check(dims, x, delta, *bwd, dout, dx, ddelta, *grad_bwd, workspace, workspace_bytes)) != SSM_OK)
+        return s;
     // forward direction writes dx, ddelta; the reversed one adds to them (the
     // two launches share the workspace in stream order)
     if ((s = bwd_one(dims, x, delta, delta_softplus, *fwd, 0, dout, dx, ddelta, *grad_fwd, workspace,

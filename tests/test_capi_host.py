@@ -210,3 +210,29 @@ def test_bwd_workspace_and_validation(lib):
     assert bwd(ws=FAKE + 4) == 3           # SSM_ERR_MISALIGNED
     assert bwd(dA=None) == 1               # SSM_ERR_INVALID_ARG
     assert bwd(dD=None) == 1               # D given without its gradient
+
+
+def test_bidir_bwd_checks_both_directions_first(lib):
+    """bidir_scan_bwd refuses a bad argument of either direction before it
+    launches anything: on a machine without a GPU any launch attempt would
+    end in SSM_ERR_CUDA (6), so a refusal code proves nothing was started."""
+    dims = _dims(2, 33, 64, 16)
+    need = lib.ssm_scan_bwd_workspace_size(ctypes.byref(dims))
+    p = ssm.ssm_dir_params(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None)   # bias, A, B, C, D, z
+    good = ssm.ssm_dir_grads(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE)
+
+    def call(gf=good, gb=good, ws=FAKE, wsb=need, d=dims):
+        return lib.bidir_scan_bwd(ctypes.byref(d), FAKE, FAKE, 1, ctypes.byref(p), ctypes.byref(p), FAKE,
+                                  FAKE, FAKE, None if gf is None else ctypes.byref(gf),
+                                  None if gb is None else ctypes.byref(gb), ws, wsb, None)
+
+    no_dA = ssm.ssm_dir_grads(None, FAKE, FAKE, FAKE, FAKE, FAKE)
+    no_dz = ssm.ssm_dir_grads(FAKE, FAKE, FAKE, FAKE, None, FAKE)
+    misaligned = ssm.ssm_dir_grads(FAKE, FAKE + 8, FAKE, FAKE, FAKE, FAKE)
+    assert call(gb=no_dA) == 1            # the reversed direction's dA missing
+    assert call(gb=no_dz) == 1            # z given without its gradient
+    assert call(gb=misaligned) == 3
+    assert call(gf=no_dA) == 1
+    assert call(gb=None) == 1
+    assert call(wsb=need - 16) == 5
+    assert call(d=_dims(2, 33, 64, 17)) == 2
