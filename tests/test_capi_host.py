@@ -236,3 +236,36 @@ def test_bidir_bwd_checks_both_directions_first(lib):
     assert call(gb=None) == 1
     assert call(wsb=need - 16) == 5
     assert call(d=_dims(2, 33, 64, 17)) == 2
+
+
+def test_binding_signatures_match_the_header():
+    """Every function include/ssm.h declares has a ctypes signature in the
+    binding with the same number of parameters and, per parameter, the same
+    kind: pointer, size_t or integer."""
+    txt = open(os.path.join(ROOT, "include", "ssm.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    decls = re.findall(r"SSM_API\s+([\w\s\*]*?)\b(\w+)\s*\(([^;{]*)\)\s*;", txt)
+    assert len(decls) == len(_declared_functions())
+    ptr_types = (ctypes.c_void_p, ctypes.c_char_p)
+
+    def kind_of_c(decl):
+        if "*" in decl:
+            return "ptr"
+        return "size" if re.search(r"\bsize_t\b", decl) else "int"
+
+    def kind_of_ctypes(t):
+        if t in ptr_types or isinstance(t, type) and issubclass(t, ctypes._Pointer):
+            return "ptr"
+        if t is ctypes.c_size_t:
+            return "size"
+        assert t in (ctypes.c_int, ctypes.c_int32), t
+        return "int"
+
+    for ret, name, args in decls:
+        assert name in ssm.SIGNATURES, name
+        restype, argtypes = ssm.SIGNATURES[name]
+        params = [] if args.strip() in ("", "void") else [a.strip() for a in args.split(",")]
+        assert len(params) == len(argtypes), f"{name}: {len(params)} vs {len(argtypes)}"
+        for i, (c, t) in enumerate(zip(params, argtypes)):
+            assert kind_of_c(c) == kind_of_ctypes(t), f"{name} argument {i}: {c!r} vs {t}"
+        assert kind_of_c(ret) == kind_of_ctypes(restype), f"{name} returns {ret!r} vs {restype}"
