@@ -269,3 +269,34 @@ def test_binding_signatures_match_the_header():
         for i, (c, t) in enumerate(zip(params, argtypes)):
             assert kind_of_c(c) == kind_of_ctypes(t), f"{name} argument {i}: {c!r} vs {t}"
         assert kind_of_c(ret) == kind_of_ctypes(restype), f"{name} returns {ret!r} vs {restype}"
+
+
+def test_struct_layouts_match_the_header(tmp_path):
+    """The ctypes structures have the C structures' field order, offsets and
+    sizes (a plain C program compiled against include/ssm.h prints them)."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    structs = ["ssm_dims", "ssd_dims", "ssm_dir_params", "ssm_dir_grads", "ssm_conv_params"]
+    lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "ssm.h"', "int main(void) {"]
+    for s in structs:
+        lines.append(f'printf("{s} size %zu\\n", sizeof({s}));')
+        for f, _ in getattr(ssm, s)._fields_:
+            lines.append(f'printf("{s} {f} %zu\\n", offsetof({s}, {f}));')
+    lines += ["return 0; }"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)],
+                   check=True)
+    c = {}
+    for line in subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split("\n"):
+        if line:
+            s, f, v = line.split()
+            c[(s, f)] = int(v)
+    for s in structs:
+        cls = getattr(ssm, s)
+        assert ctypes.sizeof(cls) == c[(s, "size")], s
+        for f, _ in cls._fields_:
+            assert getattr(cls, f).offset == c[(s, f)], f"{s}.{f}"
