@@ -524,6 +524,73 @@ def test_conv_scan_identity_kernel_is_plain_scan():
     _close(st, st0)
 
 
+def _delay_kernel(Dm, K, tap):
+    """Weight 1 on tap `tap` of a width-K kernel, 0 elsewhere: u[t] equals
+    x_in[t - (K - 1 - tap)] along the scan direction."""
+    w = np.zeros((Dm, K))
+    w[:, tap] = 1.0
+    return w
+
+
+def _delayed(x, s, toward_end):
+    """x moved s steps along t, zero-filled where nothing moves in: toward_end
+    gives out[t] = x[t - s] (a forward scan's causal window), otherwise
+    out[t] = x[t + s] (the window of a scan that runs from t = L-1 down)."""
+    out = np.zeros_like(x)
+    L = x.shape[1]
+    if s >= L:
+        return out
+    if toward_end:
+        out[:, s:] = x[:, :L - s]
+    else:
+        out[:, :L - s] = x[:, s:]
+    return out
+
+
+@pytest.mark.parametrize("reverse", [False, True])
+@pytest.mark.parametrize("K,tap", [(2, 0), (3, 0), (4, 0), (4, 1), (3, 2)])
+def test_conv_scan_delay_kernel_is_shifted_scan(K, tap, reverse):
+    """A kernel with a single unit tap is a pure delay of K-1-tap steps along
+    the scan's own direction (the conv of the Mamba2 page's listing is causal;
+    a reversed scan convolves the flipped sequence, as each Vim direction has
+    its own branch).  The conv scan must equal the plain scan of x_in shifted
+    by that delay: zero-filled at the front for the forward scan, at the end
+    for the reversed one.  A conv that ignores the direction fails the
+    reversed cases."""
+    rng = np.random.default_rng(530 + 10 * K + tap + 100 * reverse)
+    x, delta, bias, A, B, C, D, z = _rand_case(rng, 2, 11, 3, 4)
+    w = _delay_kernel(3, K, tap)
+    y, st = oracle.s6_conv_arrays(x, w, delta, A, B, C, conv_silu=False, delta_bias=bias, D=D, z=z,
+                                  reverse=reverse)
+    xs = _delayed(x, K - 1 - tap, toward_end=not reverse)
+    y0, st0 = oracle.s6_arrays(xs, delta, A, B, C, delta_bias=bias, D=D, z=z, reverse=reverse)
+    _close(y, y0)
+    _close(st, st0)
+
+
+def test_bidir_conv_delay_kernels_are_shifted_scans():
+    """Bidirectional conv scan with a different delay kernel per direction:
+    the sum of the forward scan of x_in delayed toward the end and the
+    reversed scan of x_in delayed toward the start, each with its own
+    parameters (Vim page sec. 3.2: each direction has its own conv)."""
+    rng = np.random.default_rng(560)
+    x, delta, bias, A, B, C, D, z = _rand_case(rng, 2, 12, 3, 4)
+    _, _, bias2, A2, B2, C2, D2, z2 = _rand_case(rng, 2, 12, 3, 4)
+    fwd = dict(delta_bias=bias, A=A, B=B, C=C, D=D, z=z)
+    bwd = dict(delta_bias=bias2, A=A2, B=B2, C=C2, D=D2, z=z2)
+    cf = dict(weight=_delay_kernel(3, 4, 1), bias=None, silu=False)   # delay 2
+    cb = dict(weight=_delay_kernel(3, 3, 0), bias=None, silu=False)   # delay 2 the other way
+    cb2 = dict(weight=_delay_kernel(3, 4, 0), bias=None, silu=False)  # delay 3
+    for conv_b, sb in ((cb, 2), (cb2, 3)):
+        y, lf, lb = oracle.bidir_conv_arrays(x, delta, fwd, bwd, cf, conv_b)
+        yf, sf = oracle.s6_arrays(_delayed(x, 2, True), delta, A, B, C, delta_bias=bias, D=D, z=z)
+        yb, sbk = oracle.s6_arrays(_delayed(x, sb, False), delta, A2, B2, C2, delta_bias=bias2, D=D2, z=z2,
+                                   reverse=True)
+        _close(y, yf + yb)
+        _close(lf, sf)
+        _close(lb, sbk)
+
+
 # ------------------------------------------------ gradients of the scan
 
 from oracle import grads as ograds  # noqa: E402
