@@ -178,9 +178,12 @@ SSM_API ssm_status ssm_step(const ssm_dims *dims, const void *x, const void *del
  * SSM_NOALLOC_SCRATCH_BYTES) returns SSM_ERR_WORKSPACE_TOO_SMALL before
  * anything runs.  The first call on each device looks up the array's device
  * address with a CUDA runtime call; make that first call before any stream
- * capture.  All calls share the array: nothing in it needs to start at zero,
- * but calls whose kernels overlap on the GPU (other streams, other host
- * threads) race on it.  Allocates nothing.
+ * capture.  The address is kept for the life of the process: after a
+ * cudaDeviceReset (or any teardown of the device's primary context) this
+ * entry point must not be called again in that process.  All calls share the
+ * array: nothing in it needs to start at zero, but calls whose kernels
+ * overlap on the GPU (other streams, other host threads) race on it.
+ * Allocates nothing.
  */
 SSM_API ssm_status ssm_scan_fwd_noalloc(const ssm_dims *dims, const void *x, const void *delta,
                                         const float *delta_bias, int delta_softplus,

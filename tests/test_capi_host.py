@@ -83,6 +83,30 @@ def test_workspace_too_small(lib):
     assert lib.ssm_scan_workspace_size(None) == 0
 
 
+NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024   # SSM_NOALLOC_SCRATCH_BYTES in include/ssm.h
+
+
+def test_noalloc_scratch_covers_every_single_direction_plan(lib):
+    """ssm_scan_fwd_noalloc refuses problems whose workspace exceeds its
+    built-in array.  The segment plan sizes carries to one wave of CTAs, so
+    no accepted single-direction shape should reach the limit: sweep batch,
+    length, channels, states and dtype through ssm_scan_workspace_size."""
+    txt = open(os.path.join(ROOT, "include", "ssm.h")).read()
+    m = re.search(r"#define SSM_NOALLOC_SCRATCH_BYTES \((\d+)u \* (\d+)u \* (\d+)u\)", txt)
+    assert m and int(m.group(1)) * int(m.group(2)) * int(m.group(3)) == NOALLOC_SCRATCH_BYTES
+    worst = 0
+    for dt, dstep in ((ssm.SSM_F32, 4), (ssm.SSM_BF16, 8)):
+        for B in (1, 2, 3, 7, 64, 1000, 100000):
+            for L in (1, 15, 16, 17, 197, 4099, 16384, 1 << 20, 1 << 30):
+                for D in (dstep, 3 * dstep, 64, 192, 200, 768, 2048, 8192, 1 << 16):
+                    for N in (1, 7, 16):
+                        dims = _dims(B=B, L=L, D=D, N=N, dt=dt)
+                        need = lib.ssm_scan_workspace_size(ctypes.byref(dims))
+                        worst = max(worst, need)
+                        assert need <= NOALLOC_SCRATCH_BYTES, (B, L, D, N, dt, need)
+    assert worst > 0
+
+
 def test_bidir_validation(lib):
     dims = _dims()
     good = ssm.ssm_dir_params(None, FAKE, FAKE, FAKE, None, None, None)

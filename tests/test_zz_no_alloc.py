@@ -11,7 +11,7 @@ import torch
 
 import ssm_gen
 import selective_state_space_24_b200 as ssm
-from gpu_util import TOL, dev, f32dev, host, rel_err
+from gpu_util import dev, f32dev
 
 pytestmark = pytest.mark.gpu
 
@@ -41,6 +41,9 @@ def test_noalloc_matches_workspace_path(cuda_device, dtype, reverse):
                         ssm.SSM_F32 if dtype == "f32" else ssm.SSM_BF16)
     assert ssm.capi().ssm_scan_workspace_size(ctypes.byref(dims)) > 0
     ref, ls_ref, outs = _call_both(inp, reverse)
+    # the same kernels on the same plan: the results must be bit-identical
+    # (a stale carry left in the shared array by the first call would show
+    # up in the second)
     for o, ls in outs:
-        assert rel_err(host(o), host(ref)) <= TOL[dtype]
-        assert rel_err(ls.cpu().numpy(), ls_ref.cpu().numpy()) <= TOL[dtype]
+        assert torch.equal(o, ref)
+        assert torch.equal(ls, ls_ref)
