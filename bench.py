@@ -62,6 +62,8 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-per-config", action="store_true",
+                   help="skip timing the other workloads after the headline one")
     p.add_argument("--op", default="scan", choices=["scan", "ordered", "conv", "step", "bwd", "bidir_bwd"],
                    help="scan: the workload's scan (default); ordered: the same bidirectional "
                         "workload along a random order of the positions with 30%% of the tokens "
@@ -115,6 +117,34 @@ def alu_peak_elems(sm_mhz: float) -> float:
     return SMS * sm_mhz * 1e6 * (64.0 / 3.0)
 
 
+def mufu_peak_elems(sm_mhz: float) -> float:
+    """Element rate of the S6 step if every exp ran on the MUFU unit (measured
+    15.9 ex2 per clock per SM on B200; 16 taken) and nothing else limited it:
+    one exp per element -> 16 elements per clock per SM."""
+    return SMS * sm_mhz * 1e6 * 16.0
+
+
+# tcgen05.mma instructions per (chunk, head) in the SSD kernel -- G 8, Yo 8,
+# dS 4, Yd 8 -- and the tensor-pipe cycles one instruction of these shapes
+# occupies (measured on B200 by a one-off probe: ~67 cycles for every
+# M in {64, 128}, N <= 128, K = 16)
+SSD_MMA_PER_CHUNK_HEAD = 28
+SSD_CYCLES_PER_MMA = 67.0
+
+
+def ssd_tensor_pipe_est(info, kern_s: float, sm_mhz: float) -> dict:
+    """Issue-based estimate of the SSD kernel's tensor-pipe utilisation: MMA
+    count x cycles per MMA over (kernel cycles x SMs).  ncu's measured
+    figure is in profiles/; this one is recomputed from every run's time."""
+    chunks = -(-info["seqlen"] // info["chunk"])
+    busy = info["batch"] * info["nheads"] * chunks * SSD_MMA_PER_CHUNK_HEAD * SSD_CYCLES_PER_MMA
+    cyc = kern_s * sm_mhz * 1e6
+    ctas = info["batch"] * info["nheads"]
+    return {"all_sms": busy / (cyc * SMS), "sms_used": min(ctas, SMS),
+            "over_sms_used": busy / (cyc * min(ctas, SMS)),
+            "mma_per_chunk_head": SSD_MMA_PER_CHUNK_HEAD, "cycles_per_mma": SSD_CYCLES_PER_MMA}
+
+
 def step_stats(ms):
     """Median, p10 and p90 of the per-step CUDA-event times (ms)."""
     if len(ms) < 2:
@@ -155,6 +185,45 @@ def max_over_ranks(ms: float, world: int, device=None) -> float:
 def job_throughput(units_per_rank_step: float, world: int, steps: int, job_ms: float) -> float:
     """Units all ranks processed per second of job time."""
     return units_per_rank_step * world * steps / (job_ms * 1e-3)
+
+
+def run_timed(step, flush, steps, world, device, new_event, sync):
+    """The timed region every rank runs: a barrier and a synchronize on both
+    sides, `steps` calls each bracketed by a pair of events (the flush before
+    each call outside them), then the sum of the step times max-reduced over
+    ranks.  new_event() returns an object with record() and
+    elapsed_time(other) in ms (CUDA events on the launching stream on a GPU).
+    Returns (per-step ms of this rank, job ms)."""
+    import torch.distributed as dist
+    evs = [(new_event(), new_event()) for _ in range(steps)]
+    if world > 1:
+        dist.barrier()
+    sync()
+    for i in range(steps):
+        flush(i)
+        evs[i][0].record()
+        step()
+        evs[i][1].record()
+    sync()
+    if world > 1:
+        dist.barrier()
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    return step_ms, max_over_ranks(float(sum(step_ms)), world, device)
+
+
+class StreamEvent:
+    """A timing CUDA event recorded on one stream."""
+
+    def __init__(self, stream):
+        import torch
+        self.stream = stream
+        self.ev = torch.cuda.Event(enable_timing=True)
+
+    def record(self):
+        self.ev.record(self.stream)
+
+    def elapsed_time(self, other):
+        return self.ev.elapsed_time(other.ev)
 
 
 # ----------------------------------------------------------------- clocks
@@ -369,6 +438,151 @@ class DeviceWorkload:
         self._bind()
 
 
+def config_dict(info, cfg, op, world):
+    """The workload a line measures; the same dict in both arms."""
+    return {"workload": info["name"] + ("" if op == "scan" else "_" + op),
+            "config_index": cfg, "op": op,
+            **{k: info[k] for k in ("batch", "seqlen", "dim", "dstate", "nheads", "headdim", "chunk")
+               if k in info},
+            "directions": info["ndir"], "parallelism": f"dp{world} (independent batches)",
+            "l2": "flushed before every timed step (512 MB write)",
+            "algorithmic_bytes_per_step": info["bytes"],
+            "elements_per_step": info["elems"]}
+
+
+def roofline(info, kern_s, traffic):
+    """Roofline of one call: the HBM fraction of the algorithmic bytes (the
+    graded bound for every workload), and beside it, for S6, the two derived
+    on-chip bounds (MUFU-only exp, and exps split between MUFU and the FMA
+    pipe); for SSD the issue-based tensor-pipe estimate."""
+    peaks, peak_src = load_peaks()
+    mhz = peaks.get("sm_max_mhz", 1965.0)
+    hbm_ach = info["bytes"] / kern_s / 1e9
+    r = {"bound": "hbm", "achieved": hbm_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+         "frac": hbm_ach / peaks["hbm_gbs"], "traffic": traffic, "peak_source": peak_src,
+         "algorithmic_bytes": info["bytes"], "kernel_ms_median": kern_s * 1e3}
+    if info["kind"] == "s6":
+        ach = info["elems"] / kern_s
+        mp, ap = mufu_peak_elems(mhz), alu_peak_elems(mhz)
+        r.update({"elements_per_s": ach, "mufu_peak_gelems": mp / 1e9, "mufu_frac": ach / mp,
+                  "alu_peak_gelems": ap / 1e9, "alu_frac": ach / ap,
+                  "derived_bounds": "derived, not measured peaks: mufu = one exp per element on the "
+                                    "MUFU unit (16/clk/SM); alu = exps split between MUFU and an "
+                                    "8-operation FMA-pipe polynomial, 4 FMA-pipe operations per "
+                                    "element (64/3 elements/clk/SM); both at sm_max_mhz"})
+    else:
+        r["tensor_pipe_est"] = ssd_tensor_pipe_est(info, kern_s, mhz)
+    return r
+
+
+def time_steps(wl, stream, flush, warmup, steps):
+    """Per-step CUDA-event times (ms) of `steps` calls after `warmup` untimed
+    ones, the L2 flushed (outside the events) before every call."""
+    import torch
+    sh = stream.cuda_stream
+    for _ in range(max(warmup, 3)):
+        flush.fill_(1.0)
+        wl.step(sh)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for i in range(steps):
+        flush.fill_(float(i))
+        evs[i][0].record(stream)
+        wl.step(sh)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+ERR_SAMPLE_COLS = 256
+
+
+def output_columns(out, info, cols):
+    """Whole-sequence output columns `cols` of one call's output, as (n, L):
+    column b * D + d of an S6 output (B, L, D), (b * H + h) * P + p of an SSD
+    output (B, L, H, P)."""
+    cols = np.asarray(cols)
+    if info["kind"] == "s6":
+        b, d = np.divmod(cols, info["dim"])
+        return out[b, :, d]
+    H, P = info["nheads"], info["headdim"]
+    b, r = np.divmod(cols, H * P)
+    h, p = np.divmod(r, P)
+    return out[b, :, h, p]
+
+
+def sample_columns(wl, cfg):
+    """A seeded sample of whole-sequence output columns of the last call,
+    copied to the host (for the CPU leg's check against the oracle)."""
+    import torch
+    info = wl.info
+    ncols = info["batch"] * (info["dim"] if info["kind"] == "s6" else info["nheads"] * info["headdim"])
+    rng = np.random.default_rng(1000 + cfg)
+    cols = np.sort(rng.choice(ncols, min(ncols, ERR_SAMPLE_COLS), replace=False))
+    g = output_columns(wl.out.float().cpu().numpy(), info, cols)
+    return cols, ncols, np.asarray(g, dtype=np.float64)
+
+
+PER_CONFIG_WARMUP, PER_CONFIG_STEPS = 20, 100
+
+
+def measure_configs(device, stream, flush):
+    """Every workload (0-4) timed the same way -- 20 warm-up and 100 timed
+    calls, L2 flushed before each -- with its roofline; returns the entries
+    and, per workload, a sample of output columns for the oracle check."""
+    import torch
+    entries, samples = [], {}
+    for cfg in sorted(ssm_gen.WORKLOADS):
+        wl = DeviceWorkload(cfg, seed=0, device=device)
+        ms = time_steps(wl, stream, flush, PER_CONFIG_WARMUP, PER_CONFIG_STEPS)
+        info = wl.info
+        st = step_stats(ms)
+        kern_s = st["median"] * 1e-3
+        roof = roofline(info, kern_s, NCU_TRAFFIC.get(cfg))
+        e = {"config_index": cfg, "workload": info["name"], "ms": st,
+             "elements_per_s": info["elems"] / kern_s, "hbm_gbs": roof["achieved"],
+             "hbm_frac": roof["frac"], "launches_per_call": wl.launches_per_step}
+        if info["kind"] == "s6":
+            e.update(mufu_frac=roof["mufu_frac"], alu_frac=roof["alu_frac"])
+        else:
+            e["tensor_pipe_est"] = roof["tensor_pipe_est"]
+        entries.append(e)
+        samples[cfg] = (wl.inp, info, *sample_columns(wl, cfg))
+        del wl
+        torch.cuda.empty_cache()
+    return entries, samples
+
+
+def rel_err(g, o) -> float:
+    """max_i |g_i - o_i| / max(|o_i|, rms(o)): the error measure of the parity
+    tests (a plain ratio is meaningless at gated near-zero outputs)."""
+    rms = float(np.sqrt(np.mean(o * o))) if o.size else 0.0
+    den = np.maximum(np.abs(o), max(rms, 1e-30))
+    return float(np.max(np.abs(g - o) / den)) if o.size else 0.0
+
+
+def oracle_errors(samples, threads):
+    """CPU leg: the float64 oracle on each sampled column set, and the max
+    relative error of the GPU columns against it."""
+    import oracle
+    res = {}
+    for cfg, (inp, info, cols, ncols, g) in samples.items():
+        t0 = time.perf_counter()
+        if info["kind"] == "s6":
+            ref = (oracle.bidir(inp, cols=cols, nthreads=threads)[0] if info["ndir"] == 2
+                   else oracle.s6(inp, cols=cols, nthreads=threads)[0])
+        else:
+            ref = oracle.ssd_seq(inp, cols=cols, nthreads=threads)[0]
+        o = output_columns(ref, info, cols)
+        err = rel_err(g, o)
+        tol = 1e-4 if info["dtype"] == "f32" else 2e-2
+        res[cfg] = {"max_rel_err": err, "tol": tol, "pass": bool(err <= tol),
+                    "sample": f"{len(cols)} of {ncols} columns, whole sequence each",
+                    "oracle_s": time.perf_counter() - t0}
+    return res
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -388,49 +602,20 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     assert torch.isfinite(wl.out.float()).all().item(), "non-finite output"
 
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
     sampler = ClockSampler(local_rank)
     sampler.start()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
     t_wall = time.perf_counter()
-    for i in range(args.steps):
-        flush.fill_(float(i))
-        evs[i][0].record(stream)
-        wl.step(sh)
-        evs[i][1].record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    step_ms, total_ms = run_timed(lambda: wl.step(sh), lambda i: flush.fill_(float(i)), args.steps, world,
+                                  device, lambda: StreamEvent(stream), torch.cuda.synchronize)
     wall = time.perf_counter() - t_wall
     clocks = sampler.stop()
-    step_ms = [a.elapsed_time(b) for a, b in evs]
-    total_ms = max_over_ranks(float(sum(step_ms)), world, device)
     per_step_ms = total_ms / args.steps
     value = job_throughput(info["elems"], world, args.steps, total_ms)
 
-    # roofline of the dominant kernel (the one launch of the step when the
-    # plan has a single segment; else the step is summary + carry + main)
-    peaks, peak_src = load_peaks()
+    # roofline of the call (one launch when the plan has a single segment;
+    # else summary + carry + main, all inside the measured time)
     kern_s = statistics.median(step_ms) * 1e-3
-    hbm_ach = info["bytes"] / kern_s / 1e9
-    alu_peak = alu_peak_elems(peaks.get("sm_max_mhz", 1965.0))
-    alu_ach = info["elems"] / kern_s
-    t_hbm = info["bytes"] / (peaks["hbm_gbs"] * 1e9)
-    t_alu = info["elems"] / alu_peak
-    if info["kind"] == "s6" and t_alu > t_hbm:
-        roof = {"bound": "alu", "achieved": alu_ach / 1e9, "peak": alu_peak / 1e9,
-                "unit": "Gelem/s", "frac": alu_ach / alu_peak, "traffic": NCU_TRAFFIC.get(args.config) if args.op == "scan" else None,
-                "hbm_achieved_gbs": hbm_ach, "hbm_peak_gbs": peaks["hbm_gbs"],
-                "hbm_frac": hbm_ach / peaks["hbm_gbs"], "peak_source": peak_src,
-                "algorithmic_bytes": info["bytes"], "kernel_ms_median": kern_s * 1e3}
-    else:
-        roof = {"bound": "hbm", "achieved": hbm_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": hbm_ach / peaks["hbm_gbs"], "traffic": NCU_TRAFFIC.get(args.config) if args.op == "scan" else None,
-                "peak_source": peak_src,
-                "algorithmic_bytes": info["bytes"], "kernel_ms_median": kern_s * 1e3}
+    roof = roofline(info, kern_s, NCU_TRAFFIC.get(args.config) if args.op == "scan" else None)
 
     e2e = None
     if not args.no_e2e:
@@ -455,10 +640,26 @@ def run_ours(args, rank, world, local_rank):
         e2e = {"value": job_throughput(info["elems"], world, ke, ems), "unit": "elements/s",
                "h2d_bytes_per_step": hb, "d2h_bytes_per_step": db, "steps": ke,
                "ms_per_step": ems / ke}
+    launches = wl.launches_per_step * args.steps
+    del wl
+    torch.cuda.empty_cache()
+
+    # every workload, one GPU only (the per-rank batch sharding of the
+    # headline needs no second pass at N > 1)
+    per_config, samples, pc_clocks = None, None, None
+    if world == 1 and args.op == "scan" and not args.no_per_config:
+        pcs = ClockSampler(local_rank)
+        pcs.start()
+        per_config, samples = measure_configs(device, stream, flush)
+        pc_clocks = pcs.stop()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.op == "scan":
         cpu = cpu_baseline(args.config, budget_s=10.0)
+        if samples:
+            errs = oracle_errors(samples, cpu["cores"])
+            for e in per_config:
+                e["oracle_check"] = errs[e["config_index"]]
 
     res = {
         "metric": METRIC, "value": value, "unit": "elements/s", "n_gpus": world,
@@ -467,19 +668,18 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32" if info["dtype"] == "f32" else "bf16 storage, f32 compute",
         "data": "synthetic (seeded ssm_gen inputs with the workload's shapes and distributions)",
-        "config": {"workload": info["name"] + ("" if args.op == "scan" else "_" + args.op),
-                   "config_index": args.config, "op": args.op,
-                   **{k: info[k] for k in ("batch", "seqlen", "dim", "dstate", "nheads", "headdim",
-                                           "chunk") if k in info},
-                   "directions": info["ndir"], "parallelism": f"dp{world} (independent batches)",
-                   "l2": "flushed before every timed step (512 MB write)",
-                   "algorithmic_bytes_per_step": info["bytes"],
-                   "elements_per_step": info["elems"]},
+        "config": config_dict(info, args.config, args.op, world),
         "hbm_gbs": info["bytes"] / (per_step_ms * 1e-3) / 1e9,
         "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-        "gpu_launches": wl.launches_per_step * args.steps,
+        "gpu_launches": launches,
         "clocks": clocks, "wall_s_timed_region": wall,
     }
+    if per_config is not None:
+        res["per_config"] = per_config
+        res["per_config_protocol"] = (f"{PER_CONFIG_WARMUP} warm-up and {PER_CONFIG_STEPS} timed calls "
+                                      "per workload, L2 flushed before each, CUDA events; oracle_check "
+                                      "from the CPU leg (float64 oracle on sampled columns)")
+        res["per_config_clocks"] = pc_clocks
     return res
 
 
@@ -751,7 +951,7 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": el * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": info["name"], "config_index": args.config},
+        "config": config_dict(info, args.config, "scan", args.gpus),
         "cpu_baseline": {"value": value, "unit": "elements/s", "cores": threads,
                          "kind": "oracle", "sample": samp},
         "e2e": {"value": value, "unit": "elements/s", "h2d_bytes_per_step": 0,

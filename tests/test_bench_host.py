@@ -47,3 +47,49 @@ def test_step_stats_and_throughput():
     # units of every rank over the max-over-ranks job time
     assert bench.job_throughput(1e6, 4, 10, 20.0) == pytest.approx(4e6 * 10 / 0.02)
     assert math.isfinite(bench.job_throughput(1.0, 1, 1, 1e-3))
+
+
+def test_roofline_frac_is_the_hbm_fraction():
+    """Every workload is graded on HBM bytes: frac = algorithmic bytes /
+    time / HBM peak; the derived on-chip bounds sit in their own fields."""
+    peaks, _ = bench.load_peaks()
+    for cfg in range(5):
+        info = bench.workload_info(cfg)
+        r = bench.roofline(info, 1e-4, None)
+        assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+        assert r["achieved"] == pytest.approx(info["bytes"] / 1e-4 / 1e9)
+        assert r["frac"] == pytest.approx(r["achieved"] / peaks["hbm_gbs"])
+        if info["kind"] == "s6":
+            mhz = peaks.get("sm_max_mhz", 1965.0)
+            assert r["mufu_frac"] == pytest.approx(info["elems"] / 1e-4 / (148 * mhz * 1e6 * 16))
+            assert r["alu_frac"] == pytest.approx(r["mufu_frac"] * 16 / (64 / 3))
+        else:
+            t = r["tensor_pipe_est"]
+            assert t["sms_used"] == 128
+            assert t["all_sms"] == pytest.approx(t["over_sms_used"] * 128 / 148)
+
+
+def test_reference_arm_prints_the_same_config():
+    for cfg in range(5):
+        info = bench.workload_info(cfg)
+        a = bench.config_dict(info, cfg, "scan", 1)
+        assert a["config_index"] == cfg and a["algorithmic_bytes_per_step"] == info["bytes"]
+        assert a == bench.config_dict(bench.workload_info(cfg), cfg, "scan", 1)
+
+
+def test_output_columns_and_error_measure():
+    """Column c of an S6 output is (b, d) = divmod(c, D); of an SSD output
+    (b, h, p) with c = (b H + h) P + p; the error measure divides by
+    max(|o|, rms(o))."""
+    import numpy as np
+    s6 = {"kind": "s6", "dim": 5}
+    out = np.arange(2 * 3 * 5).reshape(2, 3, 5)
+    g = bench.output_columns(out, s6, [0, 7])
+    assert (g[0] == out[0, :, 0]).all() and (g[1] == out[1, :, 2]).all()
+    ssd = {"kind": "ssd", "nheads": 3, "headdim": 4}
+    out = np.arange(2 * 6 * 3 * 4).reshape(2, 6, 3, 4)
+    g = bench.output_columns(out, ssd, [(1 * 3 + 2) * 4 + 1])
+    assert (g[0] == out[1, :, 2, 1]).all()
+    o = np.array([1.0, -1.0, 1e-9])
+    assert bench.rel_err(o, o) == 0.0
+    assert bench.rel_err(o + np.array([0.0, 0.0, 1e-3]), o) == pytest.approx(1e-3 / np.sqrt(2 / 3))
