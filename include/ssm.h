@@ -378,6 +378,21 @@ SSM_API ssm_status ssd_chunk_fwd(const ssd_dims *dims, const void *x, const void
  */
 SSM_API ssm_status ssm_check_device(void *stream);
 
+/*
+ * Test hook for the device-timeout path (the pages have no counterpart; it
+ * exists so that a test can make a bounded device wait run out without
+ * faulting or hanging the GPU).  SSD calls enqueued after it, in this
+ * process, run with every pipeline wait limited to `wait_limit` polls
+ * (0 restores the default of 1 << 20) and, if `withhold_chunk` >= 0, with
+ * the producer warp never signalling that chunk's dt, so the consumers' wait
+ * for it runs out: such a call still completes (its outputs are undefined,
+ * every copy and MMA it issued is waited for, its tensor memory is freed)
+ * and the next ssm_check_device returns SSM_ERR_DEVICE_TIMEOUT.
+ * ssm_debug_ssd_stall(-1, 0) restores normal calls.  Process-wide and not
+ * synchronised with calls on other threads: for tests only.
+ */
+SSM_API void ssm_debug_ssd_stall(int withhold_chunk, unsigned wait_limit);
+
 /* Static, human-readable name of a status code. */
 SSM_API const char *ssm_status_string(ssm_status status);
 

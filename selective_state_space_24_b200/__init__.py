@@ -78,6 +78,7 @@ _int = ctypes.c_int
 
 # exported name -> (restype, argtypes)
 SIGNATURES = {
+    "ssm_debug_ssd_stall": (None, [_int, ctypes.c_uint]),
     "ssm_scan_workspace_size": (_sz, [ctypes.POINTER(ssm_dims)]),
     "ssm_scan_fwd": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp, _vp,
                             _int, _vp, _vp, _vp, _sz, _vp]),

@@ -126,6 +126,17 @@ struct SSDArgs {
 };
 
 size_t ssd_workspace_bytes(int64_t Bsz, int64_t L, int64_t H, int64_t P, int64_t N, int64_t Q);
+
+// Test setting of the SSD kernel's bounded waits (process-wide): the poll
+// limit of every pipeline wait (0 = the default) and a chunk whose dt the
+// producer warp never signals (-1 = none), which makes the consumers' wait
+// for it run out.
+struct SSDStall {
+    int withhold_chunk;
+    unsigned wait_limit;
+};
+void ssd_stall_set(int withhold_chunk, unsigned wait_limit);
+SSDStall ssd_stall_get();
 cudaError_t launch_ssd(const SSDArgs &a, cudaStream_t stream);
 
 // Device-side error words: the SSD kernel's (bounded waits that gave up)

@@ -42,6 +42,8 @@
 // core reads (C and B as K-major operands of C B^T, B as an MN-major operand
 // of B^T W, X as an MN-major operand of M X).  Every mbarrier wait is bounded
 // and sets the library's error word if it gives up.
+#include <atomic>
+
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -88,7 +90,8 @@ constexpr int kSmemBytes = kOffVec + 2 * kDtBufs * 64 * 4 + 1024; // + alignment
 // chunk c + 1's first products were issued.
 constexpr uint32_t kColG = 0, kColDS = 64, kColYo = 192, kColYd = 448, kTmemCols = 512;
 
-constexpr long kWaitLimit = 1l << 20;
+constexpr long kWaitLimit = 1l << 20;    // default poll limit of a pipeline wait
+constexpr long kDrainLimit = 1l << 22;   // poll limit of the teardown waits for in-flight copies / MMAs
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
@@ -133,19 +136,21 @@ __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.a
 
 // Bounded wait on an mbarrier phase (with SSM_SSD_SUSPEND_NS > 0 each
 // try_wait may suspend the thread for up to that long; it resumes when the
-// phase completes).  On
-// giving up, a thread flags the library's error word and its CTA's abort
-// word and returns false; every later wait in the CTA then gives up at once,
-// so the kernel still ends promptly (with wrong values, reported by
-// ssm_check_device) and every thread still meets every barrier.
+// phase completes).  On giving up after `limit` polls, a thread flags the
+// library's error word and its CTA's abort word and returns false; every
+// later wait in the CTA then gives up at once.  After a failed wait a role
+// issues no further copies or MMAs and signals no further barriers, so the
+// only asynchronous work left is what was issued before; the teardown waits
+// for it (drain_wait) before TMEM is freed and the CTA exits.  The kernel
+// then ends promptly with wrong values, reported by ssm_check_device.
 #ifndef SSM_SSD_SUSPEND_NS
 #define SSM_SSD_SUSPEND_NS 0
 #endif
 constexpr uint32_t kSuspendNs = SSM_SSD_SUSPEND_NS;
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort)
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, long limit)
 {
     const uint32_t a = smem_u32(bar);
-    for (long it = 0; it < kWaitLimit; it++) {
+    for (long it = 0; it < limit; it++) {
         uint32_t ok;
         if (kSuspendNs)
             asm volatile("{.reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p;}"
@@ -165,6 +170,25 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     *abort = 1;
     atomicExch(&g_device_error, 1u);
     return false;
+}
+
+// Teardown wait for asynchronous work this CTA issued itself (a TMA load
+// landing, a tcgen05.commit arriving): it completes on its own, so the wait
+// ignores the abort word; it is still bounded, and flags the error word if
+// it gives up.
+__device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity)
+{
+    const uint32_t a = smem_u32(bar);
+    for (long it = 0; it < kDrainLimit; it++) {
+        uint32_t ok;
+        asm volatile("{.reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p;}"
+                     : "=r"(ok)
+                     : "r"(a), "r"(parity)
+                     : "memory");
+        if (ok)
+            return;
+    }
+    atomicExch(&g_device_error, 1u);
 }
 
 __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, int c0, int c1, int c2, int c3,
@@ -280,6 +304,8 @@ struct SSDKernelArgs {
     __nv_bfloat16 *out;
     float *last_state;
     int has_z;
+    long wait_limit;      // polls before a pipeline wait gives up
+    int withhold_chunk;   // >= 0: the dt warp never signals that chunk's dt (device-timeout test)
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -299,6 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __shared__ __align__(8) uint64_t bar_dt_full[kDtBufs];    // dt warp: dt / cs of a chunk written
     __shared__ __align__(8) uint64_t bar_free[kDtBufs];       // math threads: done with a chunk's stage and dt
     __shared__ uint32_t tmem_base_sh;
+    __shared__ __align__(8) uint64_t bar_drain;   // tensor core: every MMA this CTA issued is done
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wq = warp & 3;      // TMEM lane quadrant of this warp
@@ -321,6 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bar_g)));
         asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bar_ds)));
         asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bar_mma2)));
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bar_drain)));
         asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(&bar_mready)), "r"(kMath));
         asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(&bar_sready)), "r"(kMath));
         for (int k = 0; k < kDtBufs; k++) {
@@ -344,7 +372,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tb = tmem_base_sh;
     const uint32_t tw = tb + ((uint32_t)(wq * 32) << 16);   // this warp's TMEM lanes
     volatile int *abort = &abort_sh;
-    auto wait = [&](uint64_t *bar, uint32_t parity) { return mbar_wait(bar, parity, abort); };
+    const long limit = args.wait_limit;
+    // every lane of the calling warp waits; the result is the same for the
+    // whole warp (so .sync.aligned instructions after it stay converged)
+    auto wait = [&](uint64_t *bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, limit));
+    };
 
     auto issue_tma = [&](int c) {
         uint8_t *st = sm + (c % kStages) * kStageBytes;
@@ -490,22 +523,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row_i = 16 * wq + (lane & 15);   // M = 64 accumulator row of this thread
     const int c8 = 16 * g + 8 * (lane >> 4);   // first of this thread's 8 columns
 
+    int issued = -1;   // dt warp: the last chunk whose TMA loads were issued
     if (warp == kDtWarp) {
         // ---- the dt warp: for every chunk k, once the math threads are done
         // with chunk k - kStages (its stage and dt buffer), issue chunk k's TMA
-        // loads (lane 0) and compute dt and the cumulative sum of dt A
+        // loads (lane 0) and compute dt and the cumulative sum of dt A.  A
+        // stage is reissued only after the math threads released it, which
+        // they do only after its previous loads landed, so each stage has at
+        // most one load phase in flight.
         float2 draw = load_delta2(0);
         for (int k = 0; k < nch; k++) {
             const float2 dnext = load_delta2(k + 1);
-            if (k >= kStages)
-                wait(&bar_free[k % kStages], ((k / kStages) - 1) & 1);
+            if (k >= kStages && !wait(&bar_free[k % kStages], ((k / kStages) - 1) & 1))
+                break;
+            if (__any_sync(0xffffffffu, *abort))
+                break;
             if (lane == 0)
                 issue_tma(k);
+            issued = k;
             __syncwarp();
             chunk_dt(k, draw);
-            mbar_arrive(&bar_dt_full[k % kDtBufs]);
+            if (k != args.withhold_chunk)
+                mbar_arrive(&bar_dt_full[k % kDtBufs]);
             draw = dnext;
         }
+        // teardown: wait for the loads still in flight (the last phase issued
+        // on each stage)
+        if (lane == 0)
+            for (int k = max(0, issued - kStages + 1); k <= issued; k++)
+                drain_wait(&bar_tma[k % kStages], (k / kStages) & 1);
+        __syncwarp();
     } else if (warp == kMmaWarp) {
         // ---- the MMA warp: lane 0 issues each product once its operands are
         // written and its accumulator read; the warp stays converged.
@@ -519,37 +566,50 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
         };
         bool ok = wait(&bar_sready, 0);   // W(0) written (its TMA landed); S_in(0) is zero
-        lane0([&] {
-            issue_G_Yo(0);
-            issue_dS(0);
-        });
+        if (ok)
+            lane0([&] {
+                issue_G_Yo(0);
+                issue_dS(0);
+            });
         for (int c = 0; c < nch && ok; c++) {
             ok = wait(&bar_mready, c & 1);   // M(c) written, G(c) read
+            if (!ok)
+                break;
             lane0([&] { issue_Yd(c); });
             if (c + 1 < nch) {
-                ok = ok && wait(&bar_sready, (c + 1) & 1);   // W(c + 1), S_in(c + 1) written, dS(c) read
+                ok = wait(&bar_sready, (c + 1) & 1);   // W(c + 1), S_in(c + 1) written, dS(c) read
+                if (!ok)
+                    break;
                 lane0([&] {
                     issue_G_Yo(c + 1);
                     issue_dS(c + 1);
                 });
             }
         }
+        // teardown: one more commit tracks every MMA issued above; wait for it
+        lane0([&] { umma_commit(&bar_drain); });
+        if (lane == 0)
+            drain_wait(&bar_drain, 0);
+        __syncwarp();
     } else {
-        // ---- math threads.  Prologue: W(0)
-        wait(&bar_dt_full[0], 0);
-        wait(&bar_tma[0], 0);
-        w_store(0, w_load(0));
-        fence_async_smem();
-        tc_fence_before();
-        mbar_arrive(&bar_sready);
+        // ---- math threads.  Prologue: W(0).  A failed wait ends this warp's
+        // work (no further signals); the other roles then give up too.
+        bool ok = wait(&bar_dt_full[0], 0) && wait(&bar_tma[0], 0);
+        if (ok) {
+            w_store(0, w_load(0));
+            fence_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bar_sready);
+        }
 
-        for (int c = 0; c < nch; c++) {
+        for (int c = 0; c < nch && ok; c++) {
             const uint8_t *st = sm + (c % kStages) * kStageBytes;
             const float *cs = cs_s + (c % kDtBufs) * 64, *dtv = dt_s + (c % kDtBufs) * 64;
             const int t0 = c * kQ;
             const uint32_t buf = (uint32_t)(c & 1) * 64;
             // ---- 1. masked decay matrix M (bf16 hi + lo, K-major rows i) from G; hand it over
-            wait(&bar_g, c & 1);
+            if (!wait(&bar_g, c & 1))
+                break;
             tc_fence_after();
             {
                 uint32_t gr[8];
@@ -577,13 +637,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(&bar_mready);
             // ---- 2. next chunk's W (the tensor core meanwhile finishes Yo(c), dS(c), Yd(c))
             if (c + 1 < nch) {
-                wait(&bar_dt_full[(c + 1) % kDtBufs], ((c + 1) / kDtBufs) & 1);
-                wait(&bar_tma[(c + 1) % kStages], ((c + 1) / kStages) & 1);
+                if (!wait(&bar_dt_full[(c + 1) % kDtBufs], ((c + 1) / kDtBufs) & 1) ||
+                    !wait(&bar_tma[(c + 1) % kStages], ((c + 1) / kStages) & 1))
+                    break;
                 w_store(c + 1, w_load(c + 1));
             }
             // ---- 3. state update S = exp(cs_end) S + dS; bf16 hi + lo copy S_in(c + 1); hand
             // S_in(c + 1) and W(c + 1) over
-            wait(&bar_ds, c & 1);   // dS(c) done, and Yo(c) before it (S_in(c) is free)
+            if (!wait(&bar_ds, c & 1))   // dS(c) done, and Yo(c) before it (S_in(c) is free)
+                break;
             tc_fence_after();
             {
                 const float decay = ex2f(cs[kQ - 1]);
@@ -620,7 +682,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (args.has_z)
                     zv = *reinterpret_cast<const uint4 *>(st + kStageZ + sw_chunk(row_i, q));
                 const float ei = ex2f(cs[row_i]);
-                wait(&bar_mma2, c & 1);   // Yd(c) done
+                if (!wait(&bar_mma2, c & 1))   // Yd(c) done
+                    break;
                 tc_fence_after();
                 uint32_t yo[8], yl[8], yd[8];
                 tmem_ld_eighth_row(tw + kColYo + 2 * buf + 16 * g, yo);
@@ -704,6 +767,19 @@ bool make_map(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims
 
 size_t ssd_workspace_bytes(int64_t, int64_t, int64_t, int64_t, int64_t, int64_t) { return 0; }
 
+namespace {
+std::atomic<int> g_stall_chunk{-1};
+std::atomic<unsigned> g_stall_limit{0};
+}  // namespace
+
+void ssd_stall_set(int withhold_chunk, unsigned wait_limit)
+{
+    g_stall_chunk.store(withhold_chunk < 0 ? -1 : withhold_chunk);
+    g_stall_limit.store(wait_limit);
+}
+
+SSDStall ssd_stall_get() { return SSDStall{g_stall_chunk.load(), g_stall_limit.load()}; }
+
 cudaError_t launch_ssd(const SSDArgs &a, cudaStream_t stream)
 {
     if (a.P != kP || a.N != kN || a.Q != kQ)
@@ -739,6 +815,9 @@ cudaError_t launch_ssd(const SSDArgs &a, cudaStream_t stream)
     k.out = static_cast<__nv_bfloat16 *>(a.out);
     k.last_state = a.last_state;
     k.has_z = a.z != nullptr;
+    const SSDStall stall = ssd_stall_get();
+    k.wait_limit = stall.wait_limit > 0 ? (long)stall.wait_limit : kWaitLimit;
+    k.withhold_chunk = stall.withhold_chunk;
     cudaError_t e = cudaFuncSetAttribute(ssd_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess)
         return e;

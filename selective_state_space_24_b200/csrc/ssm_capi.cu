@@ -591,6 +591,8 @@ ssm_status ssm_check_device(void *stream)
     return o ? SSM_ERR_INVALID_ARG : SSM_OK;
 }
 
+void ssm_debug_ssd_stall(int withhold_chunk, unsigned wait_limit) { ssm::ssd_stall_set(withhold_chunk, wait_limit); }
+
 const char *ssm_status_string(ssm_status s)
 {
     switch (s) {

@@ -8,12 +8,17 @@ meaningless, so each element's error is divided by max(|o_i|, rms(o)):
 Tolerances: 1e-4 for float32 inputs, 2e-2 for bf16 inputs with float32
 state (the bf16 output rounding alone is 2^-9 relative).
 """
+import os
+
 import numpy as np
 import torch
 
 import selective_state_space_24_b200 as ssm
 
 TOL = {"f32": 1e-4, "bf16": 2e-2}
+
+# the oracle runs on every host core the process may use
+NTHREADS = max(1, len(os.sched_getaffinity(0)))
 
 
 def dev(a, dtype, device="cuda"):

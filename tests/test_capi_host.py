@@ -275,13 +275,21 @@ def test_binding_signatures_match_the_header():
     def kind_of_c(decl):
         if "*" in decl:
             return "ptr"
-        return "size" if re.search(r"\bsize_t\b", decl) else "int"
+        if re.fullmatch(r"\s*void\s*", decl):
+            return "void"
+        if re.search(r"\bsize_t\b", decl):
+            return "size"
+        return "uint" if re.search(r"\bunsigned\b", decl) else "int"
 
     def kind_of_ctypes(t):
+        if t is None:
+            return "void"
         if t in ptr_types or isinstance(t, type) and issubclass(t, ctypes._Pointer):
             return "ptr"
         if t is ctypes.c_size_t:
             return "size"
+        if t is ctypes.c_uint:
+            return "uint"
         assert t in (ctypes.c_int, ctypes.c_int32), t
         return "int"
 

@@ -7,7 +7,7 @@ import torch
 import oracle
 import ssm_gen
 import selective_state_space_24_b200 as ssm
-from gpu_util import TOL, dev, f32dev, host, rel_err, run_bidir, run_s6
+from gpu_util import NTHREADS, TOL, dev, f32dev, host, rel_err, run_bidir, run_s6
 
 pytestmark = pytest.mark.gpu
 
@@ -19,7 +19,7 @@ def _lib(cuda_device):
 
 def _check_s6(inp, reverse):
     out, st = run_s6(inp, reverse=reverse)
-    ref, rst = oracle.s6(inp, reverse=reverse)
+    ref, rst = oracle.s6(inp, reverse=reverse, nthreads=NTHREADS)
     e = rel_err(host(out), ref)
     es = rel_err(st.cpu().numpy(), rst)
     tol = TOL[inp.dtype]
@@ -30,7 +30,7 @@ def _check_s6(inp, reverse):
 
 def _check_bidir(inp, last_state=False, cols=None):
     out, lf, lb = run_bidir(inp, last_state=last_state)
-    ref, rlf, rlb = oracle.bidir(inp, cols=cols)
+    ref, rlf, rlb = oracle.bidir(inp, cols=cols, nthreads=NTHREADS)
     g = host(out)
     tol = TOL[inp.dtype]
     if cols is None:
@@ -63,13 +63,11 @@ def test_vim_small_bidir_reduced_batch_full_compare():
     _check_bidir(inp, last_state=True)
 
 
-def test_vim_small_bidir_full_size_sampled():
+def test_vim_small_bidir_full_size():
     """Vim-Small bidirectional, fp32, B 64 L 197 D 768 -- the bench's launch;
-    96 sampled columns compared over the whole sequence."""
+    every output and both last states against the oracle."""
     inp = ssm_gen.make_workload(1)
-    rng = np.random.default_rng(0)
-    cols = rng.choice(inp.batch * inp.dim, 96, replace=False)
-    _check_bidir(inp, cols=cols)
+    _check_bidir(inp, last_state=True)
 
 
 def test_hires_bidir_bf16_reduced_full_compare():
@@ -77,20 +75,16 @@ def test_hires_bidir_bf16_reduced_full_compare():
     _check_bidir(inp, last_state=True)
 
 
-def test_hires_bidir_bf16_full_size_sampled():
-    """B 8 L 1024 D 768 bf16 with last_state per direction; sampled columns."""
+def test_hires_bidir_bf16_full_size():
+    """B 8 L 1024 D 768 bf16 with last_state per direction; every output."""
     inp = ssm_gen.make_workload(2)
-    rng = np.random.default_rng(1)
-    cols = rng.choice(inp.batch * inp.dim, 96, replace=False)
-    _check_bidir(inp, last_state=True, cols=cols)
+    _check_bidir(inp, last_state=True)
 
 
-def test_long_row_bidir_bf16_full_size_sampled():
-    """Mamba-YOLO stage-1 rows: B 4 L 16384 D 192 bf16; sampled columns."""
+def test_long_row_bidir_bf16_full_size():
+    """Mamba-YOLO stage-1 rows: B 4 L 16384 D 192 bf16; every output."""
     inp = ssm_gen.make_workload(3)
-    rng = np.random.default_rng(2)
-    cols = rng.choice(inp.batch * inp.dim, 48, replace=False)
-    _check_bidir(inp, last_state=True, cols=cols)
+    _check_bidir(inp, last_state=True)
 
 
 # ------------------------------------------------- both lane mappings
@@ -116,13 +110,13 @@ def test_lane_mappings(batch, L, D, bidir, dtype, cpl):
     tol = TOL[dtype]
     if bidir:
         out, lf, lb = run_bidir(inp, last_state=True)
-        ref, rlf, rlb = oracle.bidir(inp, cols=cols, nthreads=8)
+        ref, rlf, rlb = oracle.bidir(inp, cols=cols, nthreads=NTHREADS)
         assert rel_err(host(out)[b, :, d], ref[b, :, d]) <= tol
         assert rel_err(lf.cpu().numpy()[b, d], rlf[b, d]) <= tol
         assert rel_err(lb.cpu().numpy()[b, d], rlb[b, d]) <= tol
     else:
         out, st = run_s6(inp, reverse=True)
-        ref, rst = oracle.s6(inp, reverse=True, cols=cols, nthreads=8)
+        ref, rst = oracle.s6(inp, reverse=True, cols=cols, nthreads=NTHREADS)
         assert rel_err(host(out)[b, :, d], ref[b, :, d]) <= tol
         assert rel_err(st.cpu().numpy()[b, d], rst[b, d]) <= tol
 
