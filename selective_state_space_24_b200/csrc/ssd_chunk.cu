@@ -263,14 +263,9 @@ __device__ __forceinline__ float softplus_f(float v)
     return fmaxf(v, 0.f) + (e < 0.0625f ? s : lg * 0.6931471805599453f);
 }
 
-// silu(z) = z sigmoid(z) = z (1 + tanh(z / 2)) / 2 (tanh.approx: rel. error 2^-11,
-// far below the bf16 output rounding of this path)
-__device__ __forceinline__ float silu_f(float z)
-{
-    float t;
-    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * z));
-    return 0.5f * z * (1.f + t);
-}
+// silu(z) = z sigmoid(z) = h (1 + tanh h) with h = z / 2 is evaluated inline
+// in the epilogue with tanh.approx (relative error 2^-11, far below the bf16
+// output rounding of this path).
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
 {
@@ -282,8 +277,9 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
 __device__ __forceinline__ void split_bf16(float a, float b, uint32_t &hi, uint32_t &lo)
 {
     hi = pack_bf16(a, b);
-    const float ha = __uint_as_float(hi << 16), hb = __uint_as_float(hi & 0xffff0000u);
-    lo = pack_bf16(a - ha, b - hb);
+    const float2 r = __fadd2_rn(make_float2(a, b),
+                                make_float2(-__uint_as_float(hi << 16), -__uint_as_float(hi & 0xffff0000u)));
+    lo = pack_bf16(r.x, r.y);
 }
 
 __device__ __forceinline__ float2 unpack_bf16(uint32_t u)
@@ -326,6 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __shared__ __align__(8) uint64_t bar_free[kDtBufs];       // math threads: done with a chunk's stage and dt
     __shared__ uint32_t tmem_base_sh;
     __shared__ __align__(8) uint64_t bar_drain;   // tensor core: every MMA this CTA issued is done
+    __shared__ float dec_s[kDtBufs];              // per chunk: 2^cs_end, the state's decay over the chunk
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wq = warp & 3;      // TMEM lane quadrant of this warp
@@ -428,9 +425,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane >= o)
                 incl += v;
         }
+        const float c0 = incl - a1, c1 = incl;
         float *cs = cs_s + (c % kDtBufs) * 64, *dtv = dt_s + (c % kDtBufs) * 64;
-        *reinterpret_cast<float2 *>(cs + 2 * lane) = make_float2(incl - a1, incl);
+        *reinterpret_cast<float2 *>(cs + 2 * lane) = make_float2(c0, c1);
         *reinterpret_cast<float2 *>(dtv + 2 * lane) = make_float2(d0, d1);
+        if (lane == 31)   // lane 31 holds cs_end: the chunk's decay, once for every thread
+            dec_s[c % kDtBufs] = ex2f(c1);
     };
 
     // W(c) = exp(cs_end - cs_j) dt_j X[j, :] as bf16 hi + lo, rows j, X's
@@ -455,10 +455,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int j = tid >> 3, q = tid & 7;
         const uint32_t u[4] = {w.xv.x, w.xv.y, w.xv.z, w.xv.w};
         uint32_t o[4], ol[4];
+        const float2 wj2 = make_float2(w.wj, w.wj);
 #pragma unroll
         for (int k = 0; k < 4; k++) {
-            const float2 f = unpack_bf16(u[k]);
-            split_bf16(f.x * w.wj, f.y * w.wj, o[k], ol[k]);
+            const float2 f = __fmul2_rn(unpack_bf16(u[k]), wj2);
+            split_bf16(f.x, f.y, o[k], ol[k]);
         }
         *reinterpret_cast<uint4 *>(wb + sw_chunk(j, q)) = make_uint4(o[0], o[1], o[2], o[3]);
         *reinterpret_cast<uint4 *>(wb + kTileX + sw_chunk(j, q)) = make_uint4(ol[0], ol[1], ol[2], ol[3]);
@@ -611,11 +612,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!wait(&bar_g, c & 1))
                 break;
             tc_fence_after();
+            float e_row;   // 2^cs_i, this thread's row decay for the outputs
             {
                 uint32_t gr[8];
                 tmem_ld_eighth_row(tw + kColG + 16 * g, gr);
                 const float csi = cs[row_i];
                 float e[8];
+                e_row = ex2f(csi);
 #pragma unroll
                 for (int k = 0; k < 8; k++) {
                     const int j = c8 + k;
@@ -624,9 +627,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_wait_ld(gr);
                 uint32_t o[4], ol[4];
 #pragma unroll
-                for (int k = 0; k < 8; k += 2)
-                    split_bf16(__uint_as_float(gr[k]) * e[k], __uint_as_float(gr[k + 1]) * e[k + 1], o[k >> 1],
-                               ol[k >> 1]);
+                for (int k = 0; k < 8; k += 2) {
+                    const float2 m2 = __fmul2_rn(make_float2(__uint_as_float(gr[k]), __uint_as_float(gr[k + 1])),
+                                                 make_float2(e[k], e[k + 1]));
+                    split_bf16(m2.x, m2.y, o[k >> 1], ol[k >> 1]);
+                }
                 const int q = c8 >> 3;
                 *reinterpret_cast<uint4 *>(sm + kOffM + sw_chunk(row_i, q)) = make_uint4(o[0], o[1], o[2], o[3]);
                 *reinterpret_cast<uint4 *>(sm + kOffM + kTileX + sw_chunk(row_i, q)) =
@@ -648,15 +653,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             tc_fence_after();
             {
-                const float decay = ex2f(cs[kQ - 1]);
+                const float decay = dec_s[c % kDtBufs];
                 uint32_t ds[16], dl[16];
                 tmem_ld_row16(tw + kColDS + 16 * g, ds);
                 tmem_ld_row16(tw + kColDS + 64 + 16 * g, dl);
                 tmem_wait_ld(ds);
                 tmem_wait_ld(dl);
+                // S = decay S + (dS_hi + dS_lo), two columns per packed instruction
+                const float2 dec2 = make_float2(decay, decay);
 #pragma unroll
-                for (int k = 0; k < 16; k++)
-                    S[k] = fmaf(decay, S[k], __uint_as_float(ds[k]) + __uint_as_float(dl[k]));
+                for (int k = 0; k < 16; k += 2) {
+                    const float2 d2 = __fadd2_rn(make_float2(__uint_as_float(ds[k]), __uint_as_float(ds[k + 1])),
+                                                 make_float2(__uint_as_float(dl[k]), __uint_as_float(dl[k + 1])));
+                    const float2 s2 = __ffma2_rn(dec2, make_float2(S[k], S[k + 1]), d2);
+                    S[k] = s2.x;
+                    S[k + 1] = s2.y;
+                }
                 if (c + 1 < nch) {
                     uint8_t *sn = sm + kOffS;
 #pragma unroll
@@ -681,7 +693,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint4 zv = make_uint4(0, 0, 0, 0);
                 if (args.has_z)
                     zv = *reinterpret_cast<const uint4 *>(st + kStageZ + sw_chunk(row_i, q));
-                const float ei = ex2f(cs[row_i]);
+                const float ei = e_row;
                 if (!wait(&bar_mma2, c & 1))   // Yd(c) done
                     break;
                 tc_fence_after();
@@ -696,19 +708,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w};
                 const uint32_t zu[4] = {zv.x, zv.y, zv.z, zv.w};
                 uint32_t o[4];
+                // two columns per packed instruction:
+                // y = (Yd + e_i (Yo_hi + Yo_lo) + D x) silu(z), silu(z) = h (1 + tanh h), h = z / 2
+                const float2 ei2 = make_float2(ei, ei), dh2 = make_float2(Dh, Dh);
+#pragma unroll
 #pragma unroll
                 for (int k = 0; k < 4; k++) {
-                    const float2 xf = unpack_bf16(xu[k]);
-                    const float yo0 = __uint_as_float(yo[2 * k]) + __uint_as_float(yl[2 * k]);
-                    const float yo1 = __uint_as_float(yo[2 * k + 1]) + __uint_as_float(yl[2 * k + 1]);
-                    float y0 = fmaf(ei, yo0, __uint_as_float(yd[2 * k])) + Dh * xf.x;
-                    float y1 = fmaf(ei, yo1, __uint_as_float(yd[2 * k + 1])) + Dh * xf.y;
+                    const float2 yo2 = __fadd2_rn(make_float2(__uint_as_float(yo[2 * k]), __uint_as_float(yo[2 * k + 1])),
+                                                  make_float2(__uint_as_float(yl[2 * k]), __uint_as_float(yl[2 * k + 1])));
+                    float2 y2 = __ffma2_rn(ei2, yo2, make_float2(__uint_as_float(yd[2 * k]), __uint_as_float(yd[2 * k + 1])));
+                    y2 = __ffma2_rn(dh2, unpack_bf16(xu[k]), y2);
                     if (args.has_z) {
-                        const float2 zf = unpack_bf16(zu[k]);
-                        y0 *= silu_f(zf.x);
-                        y1 *= silu_f(zf.y);
+                        const float2 h2 = __fmul2_rn(unpack_bf16(zu[k]), make_float2(0.5f, 0.5f));
+                        float2 t2;
+                        asm("tanh.approx.f32 %0, %1;" : "=f"(t2.x) : "f"(h2.x));
+                        asm("tanh.approx.f32 %0, %1;" : "=f"(t2.y) : "f"(h2.y));
+                        y2 = __fmul2_rn(y2, __ffma2_rn(h2, t2, h2));
                     }
-                    o[k] = pack_bf16(y0, y1);
+                    o[k] = pack_bf16(y2.x, y2.y);
                 }
                 if (t < L)
                     *reinterpret_cast<uint4 *>(args.out + (((size_t)b * L + t) * args.H + h) * kP + c8) =
