@@ -48,7 +48,7 @@ SMS = 148
 # DRAM bytes (read + write) per launch of the dominant kernel, from one ncu
 # capture of the current kernels (summaries under profiles/); absent where no
 # capture matches them.
-NCU_TRAFFIC = {1: 193.01e6, 4: 398.97e6}
+NCU_TRAFFIC = {1: 193.01e6}
 NCU_TRAFFIC_STEP = 63.05e6
 NCU_TRAFFIC_BWD = {1: 409.56e6}
 
@@ -64,20 +64,28 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-per-config", action="store_true",
                    help="skip timing the other workloads after the headline one")
-    p.add_argument("--op", default="scan", choices=["scan", "ordered", "conv", "step", "bwd", "bidir_bwd"],
+    p.add_argument("--op", default="scan", choices=["scan", "ordered", "conv", "fwd_ckpt", "step", "bwd", "bidir_bwd",
+                                                    "bwd_ckpt", "bidir_bwd_ckpt"],
                    help="scan: the workload's scan (default); ordered: the same bidirectional "
                         "workload along a random order of the positions with 30%% of the tokens "
                         "masked; conv: the same with a width-4 conv1d + SiLU per direction computed "
                         "inside the scan; step: one decode step of a batch-512 x 1536-channel x "
                         "16-state fp32 state (ssm_step); bwd: the gradients (ssm_scan_bwd) of the "
                         "forward direction of the workload; bidir_bwd: the gradients of the whole "
-                        "bidirectional scan (bidir_scan_bwd)")
+                        "bidirectional scan (bidir_scan_bwd); fwd_ckpt: the bidirectional scan that also "
+                        "stores the checkpoints its backward reads (bidir_scan_fwd_ckpt); bwd_ckpt / "
+                        "bidir_bwd_ckpt: the gradients from those checkpoints (ssm_scan_bwd_ckpt / "
+                        "bidir_scan_bwd_ckpt; the checkpointing forward runs once, untimed, before)")
     return p.parse_args()
 
 
 # --------------------------------------------------------------- workload
 
-def workload_info(cfg: int):
+def workload_info(cfg: int, op: str = "scan"):
+    """Sizes of workload cfg: elements per call and algorithmic bytes (each
+    input and output moved once; with op fwd_ckpt also the checkpoint arrays
+    the checkpointing scan writes -- the state entering every 4-step chunk,
+    16 fp32 per channel and direction)."""
     w = dict(ssm_gen.WORKLOADS[cfg])
     if w["kind"] == "s6":
         ndir = 2 if w["bidir"] else 1
@@ -89,6 +97,9 @@ def workload_info(cfg: int):
         io += ndir * (D * N + 2 * D) * 4              # A, D, delta_bias
         if w.get("last_state"):
             io += ndir * B * D * N * 4
+        if op == "fwd_ckpt":
+            ns = 4 if N <= 4 else 8 if N <= 8 else 16
+            io += ndir * B * ((L + 3) // 4) * D * ns * 4
         w.update(ndir=ndir, elems=elems, bytes=io)
     else:
         B, L, H, P, N = w["batch"], w["seqlen"], w["nheads"], w["headdim"], w["dstate"]
@@ -325,10 +336,15 @@ class DeviceWorkload:
         self.ws = torch.empty(max(int(need), 16), dtype=torch.uint8, device=device)
         self.ws_bytes = int(need)
         if op != "scan":
-            assert self.info["kind"] == "s6" and self.info["ndir"] == 2, "ordered / conv: bidirectional S6"
+            assert self.info["kind"] == "s6" and self.info["ndir"] == 2, \
+                "ordered / conv / fwd_ckpt: bidirectional S6"
             i = self.inp
             rng = np.random.default_rng(seed + 1)
-            if op == "ordered":
+            if op == "fwd_ckpt":
+                nck = int(self.lib.ssm_scan_ckpt_size(ctypes.byref(self.dims))) // 4
+                self.ckpt = (torch.empty(nck, dtype=torch.float32, device=device),
+                             torch.empty(nck, dtype=torch.float32, device=device))
+            elif op == "ordered":
                 self.order = torch.from_numpy(ssm_gen.order_random(i.seqlen, seed=seed)).to(device)
                 self.mask = torch.from_numpy(ssm_gen.token_mask(i.batch, i.seqlen, 0.7, seed=seed)).to(device)
             else:
@@ -365,6 +381,11 @@ class DeviceWorkload:
                                             ctypes.byref(self.fwd), ctypes.byref(self.bwd), p(self.order),
                                             p(self.mask), p(self.out), p(self.ws), self.ws_bytes,
                                             stream_handle)
+        elif self.op == "fwd_ckpt":
+            st = lib.bidir_scan_fwd_ckpt(ctypes.byref(self.dims), p(d["x"]), p(d["delta"]), 1,
+                                         ctypes.byref(self.fwd), ctypes.byref(self.bwd), p(self.out),
+                                         p(self.ckpt[0]), p(self.ckpt[1]), p(self.ws), self.ws_bytes,
+                                         stream_handle)
         elif self.op == "conv":
             st = lib.bidir_scan_fwd_conv(ctypes.byref(self.dims), p(d["x"]), p(d["delta"]), 1,
                                          ctypes.byref(self.fwd), ctypes.byref(self.bwd),
@@ -590,7 +611,7 @@ def run_ours(args, rank, world, local_rank):
     ssm_build.build()
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
-    info = workload_info(args.config)
+    info = workload_info(args.config, args.op)
     wl = DeviceWorkload(args.config, seed=rank_seed(rank), device=device, op=args.op)
     stream = torch.cuda.current_stream(device)
     sh = stream.cuda_stream
@@ -791,7 +812,8 @@ def run_bwd(args):
     p = lambda t: t.data_ptr()
     stream = torch.cuda.current_stream(device)
     sh = stream.cuda_stream
-    bidir = args.op == "bidir_bwd"
+    bidir = args.op in ("bidir_bwd", "bidir_bwd_ckpt")
+    from_ckpt = args.op.endswith("_ckpt")
     if bidir:
         assert info["ndir"] == 2, "bidir_bwd: a bidirectional workload"
         zb, Bb, Cb = io(inp.z_b), io(inp.B_b), io(inp.C_b)
@@ -802,11 +824,34 @@ def run_bwd(args):
         gf_c = ssm.ssm_dir_grads(*[p(t) for t in (g[2], g[3], g[4], g[5], g[6], g[7])])
         gb_c = ssm.ssm_dir_grads(*[p(t) for t in gb])
 
-    def step():
+    if from_ckpt:
+        # the checkpoints of the checkpointing forward, written once (untimed)
+        nck = int(lib.ssm_scan_ckpt_size(ctypes.byref(dims))) // 4
+        ck = [torch.empty(nck, dtype=torch.float32, device=device) for _ in range(2)]
+        out = torch.empty_like(x)
+        wsz = lib.bidir_scan_workspace_size if bidir else lib.ssm_scan_workspace_size
+        fws = torch.empty(max(int(wsz(ctypes.byref(dims))), 16), dtype=torch.uint8, device=device)
         if bidir:
+            st = lib.bidir_scan_fwd_ckpt(ctypes.byref(dims), p(x), p(delta), 1, ctypes.byref(pf), ctypes.byref(pb),
+                                         p(out), p(ck[0]), p(ck[1]), p(fws), fws.numel(), sh)
+        else:
+            st = lib.ssm_scan_fwd_ckpt(ctypes.byref(dims), p(x), p(delta), p(bias), 1, p(A), p(Bm), p(Cm), p(Dv),
+                                       p(z), 0, p(out), None, p(ck[0]), p(fws), fws.numel(), sh)
+        if st != 0:
+            raise RuntimeError(f"checkpointing forward returned {ssm.STATUS.get(st, st)}")
+
+    def step():
+        if bidir and from_ckpt:
+            st = lib.bidir_scan_bwd_ckpt(ctypes.byref(dims), p(x), p(delta), 1, ctypes.byref(pf), ctypes.byref(pb),
+                                         p(dout), p(g[0]), p(g[1]), ctypes.byref(gf_c), ctypes.byref(gb_c),
+                                         p(ck[0]), p(ck[1]), sh)
+        elif bidir:
             st = lib.bidir_scan_bwd(ctypes.byref(dims), p(x), p(delta), 1, ctypes.byref(pf), ctypes.byref(pb),
                                     p(dout), p(g[0]), p(g[1]), ctypes.byref(gf_c), ctypes.byref(gb_c), p(ws),
                                     need, sh)
+        elif from_ckpt:
+            st = lib.ssm_scan_bwd_ckpt(ctypes.byref(dims), p(x), p(delta), p(bias), 1, p(A), p(Bm), p(Cm), p(Dv),
+                                       p(z), 0, p(dout), *[p(t) for t in g], p(ck[0]), sh)
         else:
             st = lib.ssm_scan_bwd(ctypes.byref(dims), p(x), p(delta), p(bias), 1, p(A), p(Bm), p(Cm), p(Dv),
                                   p(z), 0, p(dout), *[p(t) for t in g], p(ws), need, sh)
@@ -846,18 +891,22 @@ def run_bwd(args):
         "unit": "elements/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": sum(ms) / len(ms), "step_ms": step_stats(ms), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": info["dtype"], "data": "synthetic (seeded ssm_gen inputs)",
-        "config": {"workload": info["name"] + ("_bidir_bwd" if bidir else "_fwd_direction_bwd"),
+        "config": {"workload": info["name"] + ("_bidir_bwd" if bidir else "_fwd_direction_bwd")
+                   + ("_from_checkpoints" if from_ckpt else ""),
                    "config_index": args.config,
                    "l2": "flushed before every timed step (512 MB write)",
                    "algorithmic_bytes_per_step": nbytes, "elements_per_step": elems},
         "hbm_gbs": nbytes / (med * 1e-3) / 1e9,
         "roofline": {"bound": "alu", "achieved": elems / (med * 1e-3) / 1e9, "peak": alu_peak / 1e9,
                      "unit": "Gelem/s", "frac": elems / (med * 1e-3) / alu_peak,
-                     "traffic": None if bidir else NCU_TRAFFIC_BWD.get(args.config), "peak_source": peak_src,
+                     "traffic": None if (bidir or from_ckpt) else NCU_TRAFFIC_BWD.get(args.config),
+                     "peak_source": peak_src,
                      "kernel_ms_median": med,
-                     "note": "achieved over the whole call (checkpoint pass + backward kernel per direction); "
-                             "traffic of the backward kernel, the dominant launch"},
-        "gpu_launches": 2 * nd * args.steps, "clocks": clocks,
+                     "note": ("achieved over the whole call (backward kernel per direction, the checkpoints "
+                              "read from the checkpointing forward); " if from_ckpt else
+                              "achieved over the whole call (checkpoint pass + backward kernel per direction); ")
+                             + "traffic of the backward kernel, the dominant launch"},
+        "gpu_launches": (1 if from_ckpt else 2) * nd * args.steps, "clocks": clocks,
     }
 
 
@@ -968,7 +1017,7 @@ def main():
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
         return
-    if args.op in ("step", "bwd", "bidir_bwd"):
+    if args.op in ("step", "bwd", "bidir_bwd", "bwd_ckpt", "bidir_bwd_ckpt"):
         if rank == 0:
             print(json.dumps(run_step(args) if args.op == "step" else run_bwd(args)), flush=True)
         return

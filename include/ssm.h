@@ -338,6 +338,61 @@ SSM_API ssm_status bidir_scan_bwd(const ssm_dims *dims, const void *x, const voi
                                   const ssm_dir_grads *grad_fwd, const ssm_dir_grads *grad_bwd,
                                   void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * Training pair that skips the backward's recompute of the states.  The
+ * backward above rebuilds the state entering every 4-step chunk with a
+ * forward pass of its own (the recompute the Mamba2 page, sec. 5.1, suggests
+ * instead of keeping every step); a training loop runs the forward scan
+ * anyway, so the checkpointing forward below stores those states while it
+ * scans, and the checkpointed backward reads them instead of recomputing.
+ *
+ * Checkpoint array of one direction: the state entering every 4-step chunk
+ * of that direction's scan order (chunk 0's is zero), (B, ceil(L / 4), D, NS)
+ * float32 with NS = N rounded up to 4, 8 or 16 (padding states zero),
+ * ssm_scan_ckpt_size(dims) bytes, caller-owned, 16-byte aligned.  It is only
+ * meaningful for the same dims, inputs and direction; a backward given an
+ * array of another call computes wrong gradients (the library cannot tell).
+ * When the plan cuts the sequence into segments, the entering state of each
+ * segment comes from the carry pass, so the checkpoints (and the gradients
+ * from them) can differ from the recomputed ones in the last bits.
+ */
+SSM_API size_t ssm_scan_ckpt_size(const ssm_dims *dims);
+
+/* ssm_scan_fwd that also writes the checkpoint array `ckpt` (required when
+ * the problem is not empty).  Errors as for ssm_scan_fwd. */
+SSM_API ssm_status ssm_scan_fwd_ckpt(const ssm_dims *dims, const void *x, const void *delta,
+                                     const float *delta_bias, int delta_softplus, const float *A,
+                                     const void *B, const void *C, const float *D, const void *z,
+                                     int reverse, void *out, float *last_state, float *ckpt,
+                                     void *workspace, size_t workspace_bytes, void *stream);
+
+/* bidir_scan_fwd that also writes each direction's checkpoint array
+ * (ckpt_fwd for the forward scan, ckpt_bwd for the reversed one; both
+ * required when the problem is not empty). */
+SSM_API ssm_status bidir_scan_fwd_ckpt(const ssm_dims *dims, const void *x, const void *delta,
+                                       int delta_softplus, const ssm_dir_params *fwd,
+                                       const ssm_dir_params *bwd, void *out, float *ckpt_fwd,
+                                       float *ckpt_bwd, void *workspace, size_t workspace_bytes,
+                                       void *stream);
+
+/* ssm_scan_bwd from the checkpoints of ssm_scan_fwd_ckpt (same dims,
+ * inputs and reverse flag): no workspace, no recompute pass.  Errors as for
+ * ssm_scan_bwd; a NULL ckpt is SSM_ERR_INVALID_ARG. */
+SSM_API ssm_status ssm_scan_bwd_ckpt(const ssm_dims *dims, const void *x, const void *delta,
+                                     const float *delta_bias, int delta_softplus, const float *A,
+                                     const void *B, const void *C, const float *D, const void *z,
+                                     int reverse, const void *dout, float *dx, float *ddelta, float *dA,
+                                     float *dB, float *dC, float *dD, float *dz, float *ddelta_bias,
+                                     const float *ckpt, void *stream);
+
+/* bidir_scan_bwd from the checkpoints of bidir_scan_fwd_ckpt. */
+SSM_API ssm_status bidir_scan_bwd_ckpt(const ssm_dims *dims, const void *x, const void *delta,
+                                       int delta_softplus, const ssm_dir_params *fwd,
+                                       const ssm_dir_params *bwd, const void *dout, float *dx,
+                                       float *ddelta, const ssm_dir_grads *grad_fwd,
+                                       const ssm_dir_grads *grad_bwd, const float *ckpt_fwd,
+                                       const float *ckpt_bwd, void *stream);
+
 /* SSD problem size.  Supported: dtype SSM_BF16, headdim 64, dstate 128,
  * chunk 64, seqlen any value >= 0 (a short last chunk is handled). */
 typedef struct {

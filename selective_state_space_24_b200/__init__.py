@@ -10,6 +10,10 @@ Entry points (names as in include/ssm.h):
 * ``ssm_scan_fwd(x, delta, A, B, C, ...)``  single-direction S6 scan
 * ``ssm_scan_fwd_state(...)``  the same from a given initial state
 * ``ssm_scan_bwd(x, delta, A, B, C, dout, ...)``  gradients of ssm_scan_fwd
+* ``ssm_scan_fwd_ckpt`` / ``bidir_scan_fwd_ckpt``  the forward scans that also
+  store the state entering every 4-step chunk, and ``ssm_scan_bwd_ckpt`` /
+  ``bidir_scan_bwd_ckpt``, the backward passes that read those checkpoints
+  instead of recomputing them
 * ``ssm_step(x, delta, A, B, C, state, ...)``  one decode step, state in place
 * ``ssm_scan_fwd_ordered`` / ``bidir_scan_fwd_ordered``  scans along a given
   order of the positions, with an optional token mask
@@ -101,6 +105,17 @@ SIGNATURES = {
     "bidir_scan_bwd": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _int, ctypes.POINTER(ssm_dir_params),
                               ctypes.POINTER(ssm_dir_params), _vp, _vp, _vp, ctypes.POINTER(ssm_dir_grads),
                               ctypes.POINTER(ssm_dir_grads), _vp, _sz, _vp]),
+    "ssm_scan_ckpt_size": (_sz, [ctypes.POINTER(ssm_dims)]),
+    "ssm_scan_fwd_ckpt": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp, _vp,
+                                 _int, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "bidir_scan_fwd_ckpt": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _int, ctypes.POINTER(ssm_dir_params),
+                                   ctypes.POINTER(ssm_dir_params), _vp, _vp, _vp, _vp, _sz, _vp]),
+    "ssm_scan_bwd_ckpt": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp, _vp,
+                                 _int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "bidir_scan_bwd_ckpt": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _int, ctypes.POINTER(ssm_dir_params),
+                                   ctypes.POINTER(ssm_dir_params), _vp, _vp, _vp,
+                                   ctypes.POINTER(ssm_dir_grads), ctypes.POINTER(ssm_dir_grads), _vp, _vp,
+                                   _vp]),
     "ssm_step": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp, _vp, _vp,
                         _vp, _vp]),
     "ssm_scan_fwd_noalloc": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp,
@@ -407,6 +422,118 @@ def bidir_scan_bwd(x, delta, fwd: DirParams, bwd: DirParams, dout, *, delta_soft
                             ctypes.byref(cf), ctypes.byref(cb), _ptr(ws), 0 if ws is None else ws.numel(),
                             _stream_handle(stream))
     _check(st, "bidir_scan_bwd")
+    return dx, ddelta, gf, gb
+
+
+def _grads(x, p: DirParams):
+    """float32 gradient tensors of one direction's parameters and their
+    ssm_dir_grads."""
+    torch = _torch()
+    f32 = dict(dtype=torch.float32, device=x.device)
+    g = {"dA": torch.empty(p.A.shape, **f32), "dB": torch.empty(p.B.shape, **f32),
+         "dC": torch.empty(p.C.shape, **f32)}
+    if p.D is not None:
+        g["dD"] = torch.empty(p.D.shape, **f32)
+    if p.z is not None:
+        g["dz"] = torch.empty(x.shape, **f32)
+    if p.delta_bias is not None:
+        g["ddelta_bias"] = torch.empty(p.delta_bias.shape, **f32)
+    c = ssm_dir_grads(_ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dC"]), _ptr(g.get("dD")), _ptr(g.get("dz")),
+                      _ptr(g.get("ddelta_bias")))
+    return g, c
+
+
+def ckpt_array(x, N, device=None):
+    """A checkpoint array for the checkpointing scans of x (B, L, D) with N
+    states: float32, ssm_scan_ckpt_size bytes (None for an empty problem)."""
+    torch = _torch()
+    nbytes = capi().ssm_scan_ckpt_size(ctypes.byref(s6_dims(x, N)))
+    if nbytes == 0:
+        return None
+    return torch.empty(nbytes // 4, dtype=torch.float32, device=device or x.device)
+
+
+def ssm_scan_fwd_ckpt(x, delta, A, B, C, *, delta_bias=None, delta_softplus=True, D=None, z=None,
+                      reverse=False, out=None, last_state=None, ckpt=None, ws=None, stream=None):
+    """ssm_scan_fwd that also stores the state entering every 4-step chunk
+    (the checkpoints ssm_scan_bwd_ckpt reads).  Returns (out, ckpt)."""
+    torch = _torch()
+    lib = capi()
+    dims = s6_dims(x, A.shape[1])
+    if out is None:
+        out = torch.empty_like(x)
+    if ckpt is None:
+        ckpt = ckpt_array(x, A.shape[1])
+    need = lib.ssm_scan_workspace_size(ctypes.byref(dims))
+    if ws is None:
+        ws = workspace(need, x.device)
+    st = lib.ssm_scan_fwd_ckpt(ctypes.byref(dims), _ptr(x), _ptr(delta), _ptr(delta_bias),
+                               int(bool(delta_softplus)), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+                               int(bool(reverse)), _ptr(out), _ptr(last_state), _ptr(ckpt), _ptr(ws),
+                               0 if ws is None else ws.numel(), _stream_handle(stream))
+    _check(st, "ssm_scan_fwd_ckpt")
+    return out, ckpt
+
+
+def bidir_scan_fwd_ckpt(x, delta, fwd: DirParams, bwd: DirParams, *, delta_softplus=True, out=None,
+                        ckpt_fwd=None, ckpt_bwd=None, ws=None, stream=None):
+    """bidir_scan_fwd that also stores each direction's checkpoints.
+    Returns (out, ckpt_fwd, ckpt_bwd)."""
+    torch = _torch()
+    lib = capi()
+    dims = s6_dims(x, fwd.A.shape[1])
+    if out is None:
+        out = torch.empty_like(x)
+    if ckpt_fwd is None:
+        ckpt_fwd = ckpt_array(x, fwd.A.shape[1])
+    if ckpt_bwd is None:
+        ckpt_bwd = ckpt_array(x, fwd.A.shape[1])
+    need = lib.bidir_scan_workspace_size(ctypes.byref(dims))
+    if ws is None:
+        ws = workspace(need, x.device)
+    f, b = fwd.to_c(), bwd.to_c()
+    st = lib.bidir_scan_fwd_ckpt(ctypes.byref(dims), _ptr(x), _ptr(delta), int(bool(delta_softplus)),
+                                 ctypes.byref(f), ctypes.byref(b), _ptr(out), _ptr(ckpt_fwd), _ptr(ckpt_bwd),
+                                 _ptr(ws), 0 if ws is None else ws.numel(), _stream_handle(stream))
+    _check(st, "bidir_scan_fwd_ckpt")
+    return out, ckpt_fwd, ckpt_bwd
+
+
+def ssm_scan_bwd_ckpt(x, delta, A, B, C, dout, ckpt, *, delta_bias=None, delta_softplus=True, D=None, z=None,
+                      reverse=False, stream=None):
+    """ssm_scan_bwd from the checkpoints of ssm_scan_fwd_ckpt (same inputs):
+    no recompute pass.  Returns the gradients as ssm_scan_bwd does."""
+    lib = capi()
+    dims = s6_dims(x, A.shape[1])
+    torch = _torch()
+    f32 = dict(dtype=torch.float32, device=x.device)
+    g, c = _grads(x, DirParams(A=A, B=B, C=C, delta_bias=delta_bias, D=D, z=z))
+    g["dx"], g["ddelta"] = torch.empty(x.shape, **f32), torch.empty(x.shape, **f32)
+    st = lib.ssm_scan_bwd_ckpt(ctypes.byref(dims), _ptr(x), _ptr(delta), _ptr(delta_bias),
+                               int(bool(delta_softplus)), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+                               int(bool(reverse)), _ptr(dout), _ptr(g["dx"]), _ptr(g["ddelta"]), c.dA, c.dB,
+                               c.dC, c.dD, c.dz, c.ddelta_bias, _ptr(ckpt), _stream_handle(stream))
+    _check(st, "ssm_scan_bwd_ckpt")
+    return g
+
+
+def bidir_scan_bwd_ckpt(x, delta, fwd: DirParams, bwd: DirParams, dout, ckpt_fwd, ckpt_bwd, *,
+                        delta_softplus=True, stream=None):
+    """bidir_scan_bwd from the checkpoints of bidir_scan_fwd_ckpt.  Returns
+    (dx, ddelta, grads_fwd, grads_bwd) as bidir_scan_bwd does."""
+    torch = _torch()
+    lib = capi()
+    dims = s6_dims(x, fwd.A.shape[1])
+    f32 = dict(dtype=torch.float32, device=x.device)
+    gf, cf = _grads(x, fwd)
+    gb, cb = _grads(x, bwd)
+    dx, ddelta = torch.empty(x.shape, **f32), torch.empty(x.shape, **f32)
+    f, b = fwd.to_c(), bwd.to_c()
+    st = lib.bidir_scan_bwd_ckpt(ctypes.byref(dims), _ptr(x), _ptr(delta), int(bool(delta_softplus)),
+                                 ctypes.byref(f), ctypes.byref(b), _ptr(dout), _ptr(dx), _ptr(ddelta),
+                                 ctypes.byref(cf), ctypes.byref(cb), _ptr(ckpt_fwd), _ptr(ckpt_bwd),
+                                 _stream_handle(stream))
+    _check(st, "bidir_scan_bwd_ckpt")
     return dx, ddelta, gf, gb
 
 

@@ -24,6 +24,10 @@ struct DirArgs {
     const float *conv_b;   // (D) or nullptr
     int conv_k;            // 1..4
     int conv_silu;         // 1: SiLU after the conv
+    // (checkpointing variant only) the state entering every 4-step chunk in
+    // scan order, (Bsz, ceil(L / 4), D, NS) float32, NS = N rounded up to 4,
+    // 8 or 16 -- the array the backward kernel reads
+    float *ckpt;
 };
 
 // One S6 call (single direction or bidirectional).
@@ -55,6 +59,7 @@ struct S6Args {
     const int *order;            // (L) visiting order of the positions, or nullptr (0..L-1)
     const unsigned char *mask;   // (Bsz, L) by position, 0 = bypass the token, or nullptr
     int conv;                    // 1: x is the conv input x_in, each direction convolves it
+    int ckpt;                    // 1: each direction also writes its checkpoints (DirArgs::ckpt)
 };
 
 struct S6Plan {
@@ -81,6 +86,8 @@ SSM_S6_PART_DECL(f32_conv)
 SSM_S6_PART_DECL(bf16)
 SSM_S6_PART_DECL(bf16_ord)
 SSM_S6_PART_DECL(bf16_conv)
+SSM_S6_PART_DECL(f32_ckpt)
+SSM_S6_PART_DECL(bf16_ckpt)
 #undef SSM_S6_PART_DECL
 
 // One decode step of S6 for every (batch, channel), state updated in place.
@@ -110,6 +117,8 @@ struct BwdArgs {
     float *dx, *ddelta, *dz, *dA, *dB, *dC, *dD, *dbias;
     float *ckpt;    // workspace: (Bsz, ceil(L / 4), D, NS) states entering each 4-step chunk,
                     // NS = N rounded up to 4, 8 or 16 (16-byte aligned)
+    int ckpt_given; // 1: ckpt already holds them (written by the checkpointing forward scan),
+                    // so the checkpoint pass is skipped
 };
 size_t bwd_workspace_bytes(int64_t Bsz, int64_t L, int64_t D, int64_t N);
 cudaError_t launch_bwd(const BwdArgs &a, cudaStream_t stream);

@@ -494,7 +494,8 @@ cudaError_t launch_ns(const BwdArgs &a, cudaStream_t st)
             return e;
         carveout_set.fetch_or(bit, std::memory_order_relaxed);
     }
-    s6_bwd_ckpt_kernel<T, NS><<<g, kCta, 0, st>>>(a);
+    if (!a.ckpt_given)
+        s6_bwd_ckpt_kernel<T, NS><<<g, kCta, 0, st>>>(a);
     s6_bwd_kernel<T, NS><<<g, kCta, 0, st>>>(a);
     return cudaGetLastError();
 }

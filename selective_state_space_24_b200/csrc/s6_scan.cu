@@ -59,10 +59,16 @@ S6Plan plan_s6(int64_t Bsz, int64_t L, int64_t D, int64_t N, int ndir, int dtype
 
 cudaError_t launch_s6(const S6Args &a, cudaStream_t st)
 {
-    const int var = (a.order || a.mask) ? 1 : (a.conv ? 2 : 0);
+    const int var = (a.order || a.mask) ? 1 : (a.conv ? 2 : (a.ckpt ? 3 : 0));
     if (a.dtype == 0)
-        return var == 1 ? launch_s6_f32_ord(a, st) : var == 2 ? launch_s6_f32_conv(a, st) : launch_s6_f32(a, st);
-    return var == 1 ? launch_s6_bf16_ord(a, st) : var == 2 ? launch_s6_bf16_conv(a, st) : launch_s6_bf16(a, st);
+        return var == 1 ? launch_s6_f32_ord(a, st)
+               : var == 2 ? launch_s6_f32_conv(a, st)
+               : var == 3 ? launch_s6_f32_ckpt(a, st)
+                          : launch_s6_f32(a, st);
+    return var == 1 ? launch_s6_bf16_ord(a, st)
+           : var == 2 ? launch_s6_bf16_conv(a, st)
+           : var == 3 ? launch_s6_bf16_ckpt(a, st)
+                      : launch_s6_bf16(a, st);
 }
 
 cudaError_t read_and_clear_s6_error(unsigned *value, cudaStream_t stream)
@@ -70,8 +76,9 @@ cudaError_t read_and_clear_s6_error(unsigned *value, cudaStream_t stream)
     cudaError_t e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess)
         return e;
-    cudaError_t (*parts[])(unsigned *, bool) = {s6_error_f32, s6_error_f32_ord, s6_error_f32_conv,
-                                                s6_error_bf16, s6_error_bf16_ord, s6_error_bf16_conv};
+    cudaError_t (*parts[])(unsigned *, bool) = {s6_error_f32,       s6_error_f32_ord,  s6_error_f32_conv,
+                                                s6_error_f32_ckpt,  s6_error_bf16,     s6_error_bf16_ord,
+                                                s6_error_bf16_conv, s6_error_bf16_ckpt};
     *value = 0;
     for (auto f : parts) {
         unsigned v = 0;

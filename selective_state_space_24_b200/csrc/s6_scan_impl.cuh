@@ -287,6 +287,13 @@ __device__ __forceinline__ void st_hint(__nv_bfloat16 *p, const float (&v)[1], u
     const unsigned short u = *reinterpret_cast<const unsigned short *>(&h);
     asm volatile("st.global.L2::cache_hint.b16 [%0], %1, %2;" ::"l"(p), "h"(u), "l"(pol) : "memory");
 }
+// 16-byte store of two state pairs with an L2 eviction policy
+__device__ __forceinline__ void st4_hint(float *p, float2 a, float2 b, uint64_t pol)
+{
+    asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "f"(a.x), "f"(a.y),
+                 "f"(b.x), "f"(b.y), "l"(pol)
+                 : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int K> __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(K) : "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
@@ -380,7 +387,7 @@ struct RowCopy {
 //   SUMMARY: local end state from the given h, plus the sum of dt; no output.
 //   otherwise: outputs; BIDIR adds the midpoint exchange with the partner warp.
 template <typename T, int NS, int CPL, int NPOLY, bool SUMMARY, bool BIDIR, bool GATE, bool SOFTPLUS,
-          bool ORD, bool CONV>
+          bool ORD, bool CONV, bool CKPT = false>
 __device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P,
                                              WarpSmem<T, NS, CPL> &sm, int b, int dbase, bool active,
                                              int s0, int s1, bool rev, float2 (&h)[CPL][NS / 2],
@@ -565,7 +572,25 @@ __device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P,
     struct StepOut {
         float y[CPL];
     };
+    // CKPT: the state entering every 4-step chunk of the direction's scan
+    // order (global scan index g of local step i), stored before step i,
+    // evict-first in L2 (the checkpoints are not read again by this scan and
+    // must not push out the x / delta lines the partner warp re-reads)
+    const int nck = (a.L + 3) / 4;
+    const uint64_t pol_ck = CKPT ? l2_evict_first() : 0;
     auto recur = [&](int i, const StepIn &in) {
+        if (CKPT && !SUMMARY && active) {
+            const int g = rev ? a.L - s1 + i : s0 + i;
+            if ((g & 3) == 0) {
+#pragma unroll
+                for (int c = 0; c < CPL; c++) {
+                    float *ck = P.ckpt + (((size_t)b * nck + (g >> 2)) * a.D + d + c) * NS;
+#pragma unroll
+                    for (int q = 0; q < NS / 4; q++)
+                        st4_hint(ck + 4 * q, h[c][2 * q], h[c][2 * q + 1], pol_ck);
+                }
+            }
+        }
         float2 dtc[CPL], dtx[CPL];
 #pragma unroll
         for (int c = 0; c < CPL; c++) {
@@ -802,7 +827,8 @@ __global__ void s6_carry_kernel(const S6Args a)
 }
 
 // ------------------------------------------------------------------- main
-template <typename T, int NS, int CPL, int NPOLY, bool BIDIR, bool GATE, bool SOFTPLUS, bool ORD, bool CONV>
+template <typename T, int NS, int CPL, int NPOLY, bool BIDIR, bool GATE, bool SOFTPLUS, bool ORD, bool CONV,
+          bool CKPT>
 __global__ void __launch_bounds__(64, min_blocks<CPL>()) s6_main_kernel(const S6Args a)
 {
     extern __shared__ __align__(16) char smem_raw[];
@@ -838,8 +864,8 @@ __global__ void __launch_bounds__(64, min_blocks<CPL>()) s6_main_kernel(const S6
             h[c][k].y = (active && src && 2 * k + 1 < a.N) ? src[2 * k + 1] : 0.f;
         }
     }
-    scan_segment<T, NS, CPL, NPOLY, false, BIDIR, GATE, SOFTPLUS, ORD, CONV>(a, P, sm[warp], b, dbase,
-                                                                             active, s0, s1, rev, h, sdt);
+    scan_segment<T, NS, CPL, NPOLY, false, BIDIR, GATE, SOFTPLUS, ORD, CONV, CKPT>(a, P, sm[warp], b, dbase,
+                                                                                   active, s0, s1, rev, h, sdt);
     if (active && P.last_state && last_in_order(seg, a.S, rev)) {
 #pragma unroll
         for (int c = 0; c < CPL; c++) {
@@ -861,7 +887,7 @@ cudaError_t set_smem(KernelT k, int bytes)
     return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
-template <typename T, int NS, int CPL, int NPOLY, bool GATE, bool SOFTPLUS, bool ORD, bool CONV>
+template <typename T, int NS, int CPL, int NPOLY, bool GATE, bool SOFTPLUS, bool ORD, bool CONV, bool CKPT>
 cudaError_t launch_typed(const S6Args &a, cudaStream_t st)
 {
     constexpr int smem = smem_bytes<T, NS, CPL>();
@@ -877,13 +903,13 @@ cudaError_t launch_typed(const S6Args &a, cudaStream_t st)
         s6_carry_kernel<<<(unsigned)((tot + 255) / 256), 256, 0, st>>>(a);
     }
     if (a.ndir == 2) {
-        auto km = s6_main_kernel<T, NS, CPL, NPOLY, true, GATE, SOFTPLUS, ORD, CONV>;
+        auto km = s6_main_kernel<T, NS, CPL, NPOLY, true, GATE, SOFTPLUS, ORD, CONV, CKPT>;
         if ((e = set_smem(km, smem)) != cudaSuccess)
             return e;
         dim3 g((a.D + kCh - 1) / kCh, a.S, a.Bsz);
         km<<<g, 64, smem, st>>>(a);
     } else {
-        auto km = s6_main_kernel<T, NS, CPL, NPOLY, false, GATE, SOFTPLUS, ORD, CONV>;
+        auto km = s6_main_kernel<T, NS, CPL, NPOLY, false, GATE, SOFTPLUS, ORD, CONV, CKPT>;
         if ((e = set_smem(km, smem)) != cudaSuccess)
             return e;
         dim3 g((a.D + kWarps * kCh - 1) / (kWarps * kCh), a.S, a.Bsz);
@@ -892,12 +918,13 @@ cudaError_t launch_typed(const S6Args &a, cudaStream_t st)
     return cudaGetLastError();
 }
 
-// VAR: 0 plain, 1 ordered / masked, 2 conv input (each a kernel variant)
+// VAR: 0 plain, 1 ordered / masked, 2 conv input, 3 plain with checkpoints
+// (each a kernel variant)
 template <typename T, int NS, int NPOLY, bool GATE, bool SOFTPLUS, int VAR>
 cudaError_t launch_cpl(const S6Args &a, cudaStream_t st)
 {
-    return a.cpl == 1 ? launch_typed<T, NS, 1, NPOLY, GATE, SOFTPLUS, VAR == 1, VAR == 2>(a, st)
-                      : launch_typed<T, NS, 2, NPOLY, GATE, SOFTPLUS, VAR == 1, VAR == 2>(a, st);
+    return a.cpl == 1 ? launch_typed<T, NS, 1, NPOLY, GATE, SOFTPLUS, VAR == 1, VAR == 2, VAR == 3>(a, st)
+                      : launch_typed<T, NS, 2, NPOLY, GATE, SOFTPLUS, VAR == 1, VAR == 2, VAR == 3>(a, st);
 }
 
 #ifndef SSM_S6_NPOLY

@@ -65,7 +65,8 @@ ssm::DirArgs dir_args(const ssm_dir_params &p)
 ssm_status run_s6(const ssm_dims *dims, const void *x, const void *delta, int softplus, int ndir,
                   int reverse, const ssm_dir_params *dirs, void *out, void *ws, size_t ws_bytes,
                   cudaStream_t stream, const float *initial_state = nullptr, const int32_t *order = nullptr,
-                  const unsigned char *mask = nullptr, const ssm_conv_params *conv = nullptr)
+                  const unsigned char *mask = nullptr, const ssm_conv_params *conv = nullptr,
+                  float *const *ckpt = nullptr)
 {
     const int dt = dims->dtype == SSM_F32 ? 0 : 1;
     const ssm::S6Plan plan =
@@ -104,6 +105,11 @@ ssm_status run_s6(const ssm_dims *dims, const void *x, const void *delta, int so
             a.dir[i].conv_k = conv[i].width;
             a.dir[i].conv_silu = conv[i].silu ? 1 : 0;
         }
+    }
+    if (ckpt) {   // one checkpoint array per direction
+        a.ckpt = 1;
+        for (int i = 0; i < ndir; i++)
+            a.dir[i].ckpt = ckpt[i];
     }
     a.out = out;
     char *w = static_cast<char *>(ws);
@@ -174,13 +180,20 @@ ssm_status scan_single(const ssm_dims *dims, const void *x, const void *delta, c
                        int delta_softplus, const float *A, const void *B, const void *C, const float *D,
                        const void *z, int reverse, const float *initial_state, const int32_t *order,
                        const unsigned char *mask, void *out, float *last_state, void *workspace,
-                       size_t workspace_bytes, void *stream, const ssm_conv_params *conv = nullptr)
+                       size_t workspace_bytes, void *stream, const ssm_conv_params *conv = nullptr,
+                       float *ckpt = nullptr, bool want_ckpt = false)
 {
     ssm_status s = check_s6_dims(dims);
     if (s != SSM_OK)
         return s;
     if (conv && (s = check_conv(conv)) != SSM_OK)
         return s;
+    if (want_ckpt && !empty_s6(dims)) {
+        if (!ckpt)
+            return SSM_ERR_INVALID_ARG;
+        if (!aligned16(ckpt))
+            return SSM_ERR_MISALIGNED;
+    }
     if ((initial_state && !aligned16(initial_state)) || (last_state && !aligned16(last_state)))
         return SSM_ERR_MISALIGNED;
     if (order && (reinterpret_cast<uintptr_t>(order) & 3u))
@@ -206,14 +219,15 @@ ssm_status scan_single(const ssm_dims *dims, const void *x, const void *delta, c
         return s;
     if (!aligned16(x) || !aligned16(delta) || !aligned16(out))
         return SSM_ERR_MISALIGNED;
+    float *const ck[1] = {ckpt};
     return run_s6(dims, x, delta, delta_softplus, 1, reverse, &p, out, workspace, workspace_bytes, st,
-                  initial_state, order, mask, conv);
+                  initial_state, order, mask, conv, want_ckpt ? ck : nullptr);
 }
 
 ssm_status scan_bidir(const ssm_dims *dims, const void *x, const void *delta, int delta_softplus,
                       const ssm_dir_params *fwd, const ssm_dir_params *bwd, const int32_t *order,
                       const unsigned char *mask, void *out, void *workspace, size_t workspace_bytes,
-                      void *stream, const ssm_conv_params *conv = nullptr)
+                      void *stream, const ssm_conv_params *conv = nullptr, float *const *ckpt = nullptr)
 {
     ssm_status s = check_s6_dims(dims);
     if (s != SSM_OK)
@@ -222,6 +236,12 @@ ssm_status scan_bidir(const ssm_dims *dims, const void *x, const void *delta, in
         return s;
     if (!fwd || !bwd)
         return SSM_ERR_INVALID_ARG;
+    if (ckpt && !empty_s6(dims)) {
+        if (!ckpt[0] || !ckpt[1])
+            return SSM_ERR_INVALID_ARG;
+        if (!aligned16(ckpt[0]) || !aligned16(ckpt[1]))
+            return SSM_ERR_MISALIGNED;
+    }
     if (order && (reinterpret_cast<uintptr_t>(order) & 3u))
         return SSM_ERR_MISALIGNED;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -243,7 +263,7 @@ ssm_status scan_bidir(const ssm_dims *dims, const void *x, const void *delta, in
         return SSM_ERR_MISALIGNED;
     const ssm_dir_params dirs[2] = {*fwd, *bwd};
     return run_s6(dims, x, delta, delta_softplus, 2, 0, dirs, out, workspace, workspace_bytes, st, nullptr,
-                  order, mask, conv);
+                  order, mask, conv, ckpt);
 }
 
 }  // namespace
@@ -329,7 +349,7 @@ namespace {
 // checked before anything is launched.
 ssm_status bwd_check(const ssm_dims *dims, const void *x, const void *delta, const ssm_dir_params &p,
                      const void *dout, const float *dx, const float *ddelta, const ssm_dir_grads &g,
-                     const void *workspace, size_t workspace_bytes)
+                     const void *workspace, size_t workspace_bytes, bool ckpt_given = false)
 {
     if (!x || !delta || !p.A || !p.B || !p.C || !dout || !dx || !ddelta || !g.dA || !g.dB || !g.dC)
         return SSM_ERR_INVALID_ARG;
@@ -340,6 +360,8 @@ ssm_status bwd_check(const ssm_dims *dims, const void *x, const void *delta, con
     for (const void *q : ptrs)
         if (q && !aligned16(q))
             return SSM_ERR_MISALIGNED;
+    if (ckpt_given)   // the checkpoints of the checkpointing forward scan (their size is the caller's)
+        return workspace ? SSM_OK : SSM_ERR_INVALID_ARG;
     const size_t need = ssm::bwd_workspace_bytes(dims->batch, dims->seqlen, dims->dim, dims->dstate);
     if (!workspace || workspace_bytes < need)
         return SSM_ERR_WORKSPACE_TOO_SMALL;
@@ -352,9 +374,9 @@ ssm_status bwd_check(const ssm_dims *dims, const void *x, const void *delta, con
 ssm_status bwd_one(const ssm_dims *dims, const void *x, const void *delta, int delta_softplus,
                    const ssm_dir_params &p, int reverse, const void *dout, float *dx, float *ddelta,
                    const ssm_dir_grads &g, void *workspace, size_t workspace_bytes, int accumulate,
-                   cudaStream_t st)
+                   cudaStream_t st, bool ckpt_given = false)
 {
-    ssm_status s = bwd_check(dims, x, delta, p, dout, dx, ddelta, g, workspace, workspace_bytes);
+    ssm_status s = bwd_check(dims, x, delta, p, dout, dx, ddelta, g, workspace, workspace_bytes, ckpt_given);
     if (s != SSM_OK)
         return s;
     const size_t nDN = (size_t)dims->dim * dims->dstate;
@@ -393,6 +415,7 @@ ssm_status bwd_one(const ssm_dims *dims, const void *x, const void *delta, int d
     a.dD = p.D ? g.dD : nullptr;
     a.dbias = p.delta_bias ? g.ddelta_bias : nullptr;
     a.ckpt = static_cast<float *>(workspace);
+    a.ckpt_given = ckpt_given ? 1 : 0;
     return ssm::launch_bwd(a, st) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
@@ -459,6 +482,76 @@ ssm_status bidir_scan_bwd(const ssm_dims *dims, const void *x, const void *delta
         return s;
     return bwd_one(dims, x, delta, delta_softplus, *bwd, 1, dout, dx, ddelta, *grad_bwd, workspace,
                    workspace_bytes, 1, st);
+}
+
+size_t ssm_scan_ckpt_size(const ssm_dims *dims)
+{
+    if (check_s6_dims(dims) != SSM_OK || empty_s6(dims))
+        return 0;
+    return ssm::bwd_workspace_bytes(dims->batch, dims->seqlen, dims->dim, dims->dstate);
+}
+
+ssm_status ssm_scan_fwd_ckpt(const ssm_dims *dims, const void *x, const void *delta, const float *delta_bias,
+                             int delta_softplus, const float *A, const void *B, const void *C, const float *D,
+                             const void *z, int reverse, void *out, float *last_state, float *ckpt,
+                             void *workspace, size_t workspace_bytes, void *stream)
+{
+    return scan_single(dims, x, delta, delta_bias, delta_softplus, A, B, C, D, z, reverse, nullptr, nullptr,
+                       nullptr, out, last_state, workspace, workspace_bytes, stream, nullptr, ckpt, true);
+}
+
+ssm_status bidir_scan_fwd_ckpt(const ssm_dims *dims, const void *x, const void *delta, int delta_softplus,
+                               const ssm_dir_params *fwd, const ssm_dir_params *bwd, void *out, float *ckpt_fwd,
+                               float *ckpt_bwd, void *workspace, size_t workspace_bytes, void *stream)
+{
+    float *const ck[2] = {ckpt_fwd, ckpt_bwd};
+    return scan_bidir(dims, x, delta, delta_softplus, fwd, bwd, nullptr, nullptr, out, workspace,
+                      workspace_bytes, stream, nullptr, ck);
+}
+
+ssm_status ssm_scan_bwd_ckpt(const ssm_dims *dims, const void *x, const void *delta, const float *delta_bias,
+                             int delta_softplus, const float *A, const void *B, const void *C, const float *D,
+                             const void *z, int reverse, const void *dout, float *dx, float *ddelta, float *dA,
+                             float *dB, float *dC, float *dD, float *dz, float *ddelta_bias, const float *ckpt,
+                             void *stream)
+{
+    ssm_status s = check_s6_dims(dims);
+    if (s != SSM_OK)
+        return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const ssm_dir_params p{delta_bias, A, B, C, D, z, nullptr};
+    const ssm_dir_grads g{dA, dB, dC, dD, dz, ddelta_bias};
+    if (empty_s6(dims))
+        return bwd_empty(dims, p, g, st);
+    return bwd_one(dims, x, delta, delta_softplus, p, reverse, dout, dx, ddelta, g, const_cast<float *>(ckpt), 0,
+                   0, st, true);
+}
+
+ssm_status bidir_scan_bwd_ckpt(const ssm_dims *dims, const void *x, const void *delta, int delta_softplus,
+                               const ssm_dir_params *fwd, const ssm_dir_params *bwd, const void *dout, float *dx,
+                               float *ddelta, const ssm_dir_grads *grad_fwd, const ssm_dir_grads *grad_bwd,
+                               const float *ckpt_fwd, const float *ckpt_bwd, void *stream)
+{
+    ssm_status s = check_s6_dims(dims);
+    if (s != SSM_OK)
+        return s;
+    if (!fwd || !bwd || !grad_fwd || !grad_bwd)
+        return SSM_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (empty_s6(dims)) {
+        if ((s = bwd_empty(dims, *fwd, *grad_fwd, st)) != SSM_OK)
+            return s;
+        return bwd_empty(dims, *bwd, *grad_bwd, st);
+    }
+    float *cf = const_cast<float *>(ckpt_fwd), *cb = const_cast<float *>(ckpt_bwd);
+    // both directions' arguments first, so that a refused call launches nothing
+    if ((s = bwd_check(dims, x, delta, *fwd, dout, dx, ddelta, *grad_fwd, cf, 0, true)) != SSM_OK ||
+        (s = bwd_check(dims, x, delta, *bwd, dout, dx, ddelta, *grad_bwd, cb, 0, true)) != SSM_OK)
+        return s;
+    if ((s = bwd_one(dims, x, delta, delta_softplus, *fwd, 0, dout, dx, ddelta, *grad_fwd, cf, 0, 0, st, true)) !=
+        SSM_OK)
+        return s;
+    return bwd_one(dims, x, delta, delta_softplus, *bwd, 1, dout, dx, ddelta, *grad_bwd, cb, 0, 1, st, true);
 }
 
 ssm_status ssm_step(const ssm_dims *dims, const void *x, const void *delta, const float *delta_bias,

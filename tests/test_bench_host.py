@@ -93,3 +93,11 @@ def test_output_columns_and_error_measure():
     o = np.array([1.0, -1.0, 1e-9])
     assert bench.rel_err(o, o) == 0.0
     assert bench.rel_err(o + np.array([0.0, 0.0, 1e-3]), o) == pytest.approx(1e-3 / np.sqrt(2 / 3))
+
+
+def test_checkpointing_scan_counts_its_checkpoints():
+    """--op fwd_ckpt also writes each direction's checkpoints: the state
+    entering every 4-step chunk, 16 fp32 per channel."""
+    a, b = bench.workload_info(1), bench.workload_info(1, "fwd_ckpt")
+    assert b["elems"] == a["elems"]
+    assert b["bytes"] - a["bytes"] == 2 * 64 * ((197 + 3) // 4) * 768 * 16 * 4

@@ -332,3 +332,44 @@ def test_struct_layouts_match_the_header(tmp_path):
         assert ctypes.sizeof(cls) == c[(s, "size")], s
         for f, _ in cls._fields_:
             assert getattr(cls, f).offset == c[(s, f)], f"{s}.{f}"
+
+
+def test_checkpointing_pair_validation(lib):
+    """The checkpointing forward / backward pair refuses missing or
+    misaligned checkpoint arrays before launching anything (on this machine
+    any launch would end in SSM_ERR_CUDA = 6); the checkpoint size is the
+    recomputing backward's workspace size."""
+    dims = _dims(2, 101, 96, 16)
+    assert lib.ssm_scan_ckpt_size(ctypes.byref(dims)) == lib.ssm_scan_bwd_workspace_size(ctypes.byref(dims))
+    assert lib.ssm_scan_ckpt_size(ctypes.byref(_dims(L=0))) == 0
+    assert lib.ssm_scan_ckpt_size(None) == 0
+
+    def fwd(ck=FAKE):
+        return lib.ssm_scan_fwd_ckpt(ctypes.byref(dims), FAKE, FAKE, None, 1, FAKE, FAKE, FAKE, None, None, 0,
+                                     FAKE, None, ck, None, 0, None)
+
+    assert fwd(ck=None) == 1
+    assert fwd(ck=FAKE + 8) == 3
+    p = ssm.ssm_dir_params(None, FAKE, FAKE, FAKE, None, None, None)
+    bfw = lambda cf, cb: lib.bidir_scan_fwd_ckpt(ctypes.byref(dims), FAKE, FAKE, 1, ctypes.byref(p),
+                                                 ctypes.byref(p), FAKE, cf, cb, None, 0, None)
+    assert bfw(FAKE, None) == 1
+    assert bfw(FAKE + 4, FAKE) == 3
+    # an empty problem needs no checkpoint array
+    e = _dims(2, 0, 96, 16)
+    assert lib.ssm_scan_fwd_ckpt(ctypes.byref(e), FAKE, FAKE, None, 1, FAKE, FAKE, FAKE, None, None, 0, FAKE,
+                                 None, None, None, 0, None) == 0
+
+    def bwd(ck=FAKE, dA=FAKE):
+        return lib.ssm_scan_bwd_ckpt(ctypes.byref(dims), FAKE, FAKE, None, 1, FAKE, FAKE, FAKE, None, None, 0,
+                                     FAKE, FAKE, FAKE, dA, FAKE, FAKE, None, None, None, ck, None)
+
+    assert bwd(ck=None) == 1
+    assert bwd(ck=FAKE + 4) == 3
+    assert bwd(dA=None) == 1
+    g = ssm.ssm_dir_grads(FAKE, FAKE, FAKE, None, None, None)
+    bbw = lambda cf, cb: lib.bidir_scan_bwd_ckpt(ctypes.byref(dims), FAKE, FAKE, 1, ctypes.byref(p),
+                                                 ctypes.byref(p), FAKE, FAKE, FAKE, ctypes.byref(g),
+                                                 ctypes.byref(g), cf, cb, None)
+    assert bbw(FAKE, None) == 1      # the reversed direction's array missing: refused before any launch
+    assert bbw(None, FAKE) == 1
