@@ -87,10 +87,12 @@ def test_empty_sequence_keeps_initial_state():
     assert torch.equal(last, h0)
 
 
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
-@pytest.mark.parametrize("N", [4, 7, 16])
-def test_step_matches_oracle(dtype, N):
-    batch, D = 3, 96
+@pytest.mark.parametrize("dtype,N,batch,D", [("f32", 4, 3, 96), ("f32", 7, 3, 96), ("f32", 16, 3, 96),
+                                              ("bf16", 4, 3, 96), ("bf16", 7, 3, 96), ("bf16", 16, 3, 96),
+                                              ("bf16", 8, 5, 200), ("f32", 16, 512, 1536)])
+def test_step_matches_oracle(dtype, N, batch, D):
+    """One decode step against the oracle; the last case is the bench's
+    decode workload (B 512, D 1536, N 16, fp32), every row compared."""
     inp = ssm_gen.make_s6_inputs(batch, 1, D, N, dtype=dtype, seed=N, random_A=True, random_D=True)
     state0 = np.random.default_rng(N).standard_normal((batch, D, N)).astype(np.float32)
     p = _params(inp, dtype)
