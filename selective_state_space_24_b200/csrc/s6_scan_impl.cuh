@@ -391,7 +391,7 @@ template <typename T, int NS, int CPL, int NPOLY, bool SUMMARY, bool BIDIR, bool
 __device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P,
                                              WarpSmem<T, NS, CPL> &sm, int b, int dbase, bool active,
                                              int s0, int s1, bool rev, float2 (&h)[CPL][NS / 2],
-                                             float (&sdt)[CPL])
+                                             float (&sdt)[CPL], char *ck_tile = nullptr)
 {
     using WS = WarpSmem<T, NS, CPL>;
     using RC = RowCopy<WS::kRowB>;
@@ -573,22 +573,43 @@ __device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P,
         float y[CPL];
     };
     // CKPT: the state entering every 4-step chunk of the direction's scan
-    // order (global scan index g of local step i), stored before step i,
-    // evict-first in L2 (the checkpoints are not read again by this scan and
-    // must not push out the x / delta lines the partner warp re-reads)
+    // order (global scan index g of local step i), stored before step i.  The
+    // warp's channels are consecutive, so its checkpoint is one contiguous
+    // tile of 32 CPL x NS floats; the lanes first put their rows into a
+    // shared tile (16-byte pieces, XOR-swizzled within each 128-byte line so
+    // that neither the row writes nor the contiguous reads conflict) and
+    // then store it as whole 512-byte warp rows, evict-first in L2 (nothing
+    // in this scan reads them again, and they must not push out the x / delta
+    // lines the partner warp re-reads).
     const int nck = (a.L + 3) / 4;
     const uint64_t pol_ck = CKPT ? l2_evict_first() : 0;
+    constexpr int kCkPieces = 32 * CPL * NS / 4;   // 16-byte pieces of the warp's tile
+    auto ck_slot = [](int piece) {                  // byte offset of a piece in the swizzled tile
+        const int line = piece >> 3;
+        return line * 128 + (((piece & 7) ^ (line & 7)) << 4);
+    };
     auto recur = [&](int i, const StepIn &in) {
-        if (CKPT && !SUMMARY && active) {
+        if (CKPT && !SUMMARY) {
             const int g = rev ? a.L - s1 + i : s0 + i;
             if ((g & 3) == 0) {
 #pragma unroll
-                for (int c = 0; c < CPL; c++) {
-                    float *ck = P.ckpt + (((size_t)b * nck + (g >> 2)) * a.D + d + c) * NS;
+                for (int c = 0; c < CPL; c++)
 #pragma unroll
-                    for (int q = 0; q < NS / 4; q++)
-                        st4_hint(ck + 4 * q, h[c][2 * q], h[c][2 * q + 1], pol_ck);
+                    for (int q = 0; q < NS / 4; q++) {
+                        const int piece = (lane * CPL + c) * (NS / 4) + q;
+                        *reinterpret_cast<float4 *>(ck_tile + ck_slot(piece)) =
+                            make_float4(h[c][2 * q].x, h[c][2 * q].y, h[c][2 * q + 1].x, h[c][2 * q + 1].y);
+                    }
+                __syncwarp();
+                float *ck = P.ckpt + (((size_t)b * nck + (g >> 2)) * a.D + dbase) * NS;
+#pragma unroll
+                for (int k = 0; k < kCkPieces / 32; k++) {
+                    const int piece = k * 32 + lane;
+                    const float4 v = *reinterpret_cast<const float4 *>(ck_tile + ck_slot(piece));
+                    if (dbase + piece / (NS / 4) < a.D)
+                        st4_hint(ck + 4 * piece, make_float2(v.x, v.y), make_float2(v.z, v.w), pol_ck);
                 }
+                __syncwarp();
             }
         }
         float2 dtc[CPL], dtx[CPL];
@@ -732,6 +753,9 @@ __device__ __forceinline__ void scan_segment(const S6Args &a, const DirArgs &P,
 
 template <typename T, int NS, int CPL>
 constexpr int smem_bytes() { return kWarps * (int)sizeof(WarpSmem<T, NS, CPL>); }
+// the checkpointing variant also stages each warp's checkpoint tile
+template <int NS, int CPL>
+constexpr int ck_tile_bytes() { return 32 * CPL * NS * 4; }
 
 // ---------------------------------------------------------------- summary
 template <typename T, int NS, int CPL, int NPOLY, bool SOFTPLUS, bool ORD, bool CONV>
@@ -864,8 +888,10 @@ __global__ void __launch_bounds__(64, min_blocks<CPL>()) s6_main_kernel(const S6
             h[c][k].y = (active && src && 2 * k + 1 < a.N) ? src[2 * k + 1] : 0.f;
         }
     }
+    char *ck_tile = CKPT ? smem_raw + smem_bytes<T, NS, CPL>() + warp * ck_tile_bytes<NS, CPL>() : nullptr;
     scan_segment<T, NS, CPL, NPOLY, false, BIDIR, GATE, SOFTPLUS, ORD, CONV, CKPT>(a, P, sm[warp], b, dbase,
-                                                                                   active, s0, s1, rev, h, sdt);
+                                                                                   active, s0, s1, rev, h, sdt,
+                                                                                   ck_tile);
     if (active && P.last_state && last_in_order(seg, a.S, rev)) {
 #pragma unroll
         for (int c = 0; c < CPL; c++) {
@@ -891,6 +917,7 @@ template <typename T, int NS, int CPL, int NPOLY, bool GATE, bool SOFTPLUS, bool
 cudaError_t launch_typed(const S6Args &a, cudaStream_t st)
 {
     constexpr int smem = smem_bytes<T, NS, CPL>();
+    constexpr int smem_main = smem + (CKPT ? kWarps * ck_tile_bytes<NS, CPL>() : 0);
     constexpr int kCh = 32 * CPL;
     cudaError_t e;
     if (a.S > 1) {
@@ -904,16 +931,16 @@ cudaError_t launch_typed(const S6Args &a, cudaStream_t st)
     }
     if (a.ndir == 2) {
         auto km = s6_main_kernel<T, NS, CPL, NPOLY, true, GATE, SOFTPLUS, ORD, CONV, CKPT>;
-        if ((e = set_smem(km, smem)) != cudaSuccess)
+        if ((e = set_smem(km, smem_main)) != cudaSuccess)
             return e;
         dim3 g((a.D + kCh - 1) / kCh, a.S, a.Bsz);
-        km<<<g, 64, smem, st>>>(a);
+        km<<<g, 64, smem_main, st>>>(a);
     } else {
         auto km = s6_main_kernel<T, NS, CPL, NPOLY, false, GATE, SOFTPLUS, ORD, CONV, CKPT>;
-        if ((e = set_smem(km, smem)) != cudaSuccess)
+        if ((e = set_smem(km, smem_main)) != cudaSuccess)
             return e;
         dim3 g((a.D + kWarps * kCh - 1) / (kWarps * kCh), a.S, a.Bsz);
-        km<<<g, 64, smem, st>>>(a);
+        km<<<g, 64, smem_main, st>>>(a);
     }
     return cudaGetLastError();
 }
