@@ -83,6 +83,7 @@ _int = ctypes.c_int
 # exported name -> (restype, argtypes)
 SIGNATURES = {
     "ssm_debug_ssd_stall": (None, [_int, ctypes.c_uint]),
+    "ssm_debug_s6_mapping": (_int, [_int]),
     "ssm_scan_workspace_size": (_sz, [ctypes.POINTER(ssm_dims)]),
     "ssm_scan_fwd": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp, _vp,
                             _int, _vp, _vp, _vp, _sz, _vp]),
@@ -612,8 +613,29 @@ def ssd_chunk_fwd(x, delta, A, B, C, *, chunk=64, delta_bias=None, delta_softplu
     return out
 
 
+MAPPING_AUTO, MAPPING_WHOLE_CHANNELS, MAPPING_SPLIT_STATES = 0, 1, 2
+
+
+class s6_mapping:
+    """Context manager (tests): plain S6 calls inside it take the given
+    thread layout (ssm_debug_s6_mapping); the cost model decides again on
+    exit."""
+
+    def __init__(self, mode):
+        self.mode = mode
+
+    def __enter__(self):
+        _check(capi().ssm_debug_s6_mapping(int(self.mode)), "ssm_debug_s6_mapping")
+        return self
+
+    def __exit__(self, *exc):
+        capi().ssm_debug_s6_mapping(MAPPING_AUTO)
+        return False
+
+
 def scan_plan(batch, seqlen, dim, dstate, dtype=SSM_F32, bidirectional=False):
-    """(segments, channels_per_lane) the library uses for an S6 problem."""
+    """(segments, channels_per_lane) the library uses for an S6 problem;
+    channels_per_lane 0 means four threads share each channel."""
     lib = capi()
     dims = ssm_dims(batch, seqlen, dim, dstate, dtype)
     seg, cpl = _int(0), _int(0)

@@ -93,7 +93,15 @@ extern "C" SSM_API ssm_status ssm_scan_fwd_noalloc(const ssm_dims *dims, const v
         if (q && !aligned16(q))
             return SSM_ERR_MISALIGNED;
     const int dt = dims->dtype == SSM_F32 ? 0 : 1;
-    const ssm::S6Plan plan = ssm::plan_s6(dims->batch, dims->seqlen, dims->dim, dims->dstate, 1, dt);
+    // the kernel ssm_scan_fwd takes for these sizes; the four-threads-per-
+    // channel one needs no scratch (one pass, single direction)
+    const bool split = ssm::split_eligible(dims->batch, dims->seqlen, dims->dim, dims->dstate, 1);
+    ssm::S6Plan plan = ssm::plan_s6(dims->batch, dims->seqlen, dims->dim, dims->dstate, 1, dt);
+    if (split) {
+        plan.S = 1;
+        plan.T = (int)dims->seqlen;
+        plan.workspace_bytes = 0;
+    }
     if (plan.workspace_bytes > (size_t)SSM_NOALLOC_SCRATCH_BYTES)
         return SSM_ERR_WORKSPACE_TOO_SMALL;   // more scratch than the built-in array holds
 
@@ -118,7 +126,8 @@ extern "C" SSM_API ssm_status ssm_scan_fwd_noalloc(const ssm_dims *dims, const v
     a.delta = delta;
     a.dir[0] = ssm::DirArgs{delta_bias, A, B, C, D, z, last_state};
     a.out = out;
-    if (plan.S > 1) {
+    a.split = split ? 1 : 0;
+    if (a.S > 1) {
         char *w = static_cast<char *>(scratch);
         a.carry_h = reinterpret_cast<float *>(w + plan.carry_h_off);
         a.carry_s = reinterpret_cast<float *>(w + plan.carry_s_off);

@@ -59,6 +59,8 @@ S6Plan plan_s6(int64_t Bsz, int64_t L, int64_t D, int64_t N, int ndir, int dtype
 
 cudaError_t launch_s6(const S6Args &a, cudaStream_t st)
 {
+    if (a.split)
+        return launch_s6_split(a, st);
     const int var = (a.order || a.mask) ? 1 : (a.conv ? 2 : (a.ckpt ? 3 : 0));
     if (a.dtype == 0)
         return var == 1 ? launch_s6_f32_ord(a, st)

@@ -1,0 +1,436 @@
+// s6_split.cu -- the S6 scan (single direction, or the Vision-Mamba pair of
+// directions of "复现Vision Mamba", sec. 3.1 - 3.2) with each channel's 16
+// states split over four threads, for problems with enough channels to
+// keep every SM sub-partition full of warps.
+//
+// Step (Mamba2 page "手写简化版Mamba2", sec. 4.3 - 4.4), per (b, d):
+//     dt = softplus(delta + bias),  h[n] = exp(dt A[n]) h[n] + dt B[n] x,
+//     y  = (C . h + D x) silu(z).
+// Thread (g, q) of a warp -- g = lane / 4 picks one of the warp's 8
+// consecutive channels, q = lane % 4 -- owns states [4q, 4q + 4) of that
+// channel.  Steps go in groups of four, and the per-channel scalar work of
+// a group (softplus, the gate, the skip term, the output store) is spread
+// over the channel's four threads: thread q does it for step q of the
+// group.  A group runs
+//   A  thread q: x, delta, z of step q -> dt, dt x, gate, D x;
+//   B  every thread, steps 0..3 in order: step s's dt and dt x from thread
+//      s of the channel (shuffles), its 4 states' update and their share of
+//      C . h (packed f32x2 multiply / FMA, MUFU exp);
+//   C  the four shares of each step are summed with shuffles so that thread
+//      q ends with y of step q, and stores its output.
+// Each warp streams its rows (x, delta, z: 8 channels; B, C: the whole row
+// of 16) through a cp.async ring of kStages groups, so the copies of the
+// next three groups are in flight during the current one.
+//
+// Bidirectional: a CTA is a pair of warps over the same 8 channels, warp 0
+// scanning t ascending and warp 1 descending.  Each parks the first half of
+// its outputs (in its own scan order) in `stash`, the pair meets at a named
+// barrier, and each then adds the partner's parked value to the second half
+// of its outputs: out is written once and no step is computed twice.  x
+// and delta are read by both warps; the first half's copies ask L2 to keep
+// them for the partner.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+#include <type_traits>
+
+#include "internal.h"
+#include "s6_math.cuh"
+
+namespace ssm {
+namespace {
+
+constexpr int kQ = 4;                  // threads per channel (a quarter of the 16 states each)
+constexpr int kG = 4;                  // steps per group: thread q does step q's scalar work
+constexpr int kChW = 32 / kQ;          // channels per warp
+constexpr int kStages = 4;             // groups in the copy ring (a power of two)
+#ifndef SSM_S6_SPLIT_MINB
+#define SSM_S6_SPLIT_MINB 16
+#endif
+#ifndef SSM_S6_SPLIT_HINTS
+#define SSM_S6_SPLIT_HINTS 1
+#endif
+constexpr int kMinBlocks = SSM_S6_SPLIT_MINB;   // CTAs (warp pairs) per SM: 16 = 32 warps, 64 registers a thread
+static_assert(kG == kQ, "each of a channel's threads takes one step of a group");
+static_assert((kStages & (kStages - 1)) == 0, "ring index by mask");
+// When the plain calls take this kernel (split_eligible).  The one-thread-
+// per-channel kernels give a warp 64 channels (two a thread) and run one step
+// in about 1000 cycles; with fewer than SSM_S6_SPLIT_MAX_WARPS1 warps (under
+// two per SM sub-partition) they are latency-bound, or cut the sequence into
+// segments and scan it twice.  This kernel's warps take about 230 cycles a
+// step but issue about half as many instructions again per element, so past
+// that occupancy the other kernels win.  Below it a cost model, fitted to
+// one-B200 timings of both kernels over batch 1 - 64, L 128 - 1024 and
+// D 192 - 1536, picks the faster (microseconds; E = elements B L D N x
+// directions):
+//   this kernel    max(Tl, Tt) + 0.3 min(Tl, Tt) + 2,  Tl = L x 0.105
+//                  (0.17 for a bidirectional pair), Tt = E / 2.0e6 (1.5e6);
+//   the others     24 + E / 1.2e6.
+#ifndef SSM_S6_SPLIT_MAX_WARPS1
+#define SSM_S6_SPLIT_MAX_WARPS1 1024
+#endif
+
+// One step's slot in the ring: x, delta, (z) for the warp's 8 channels,
+// then the B and C rows.
+template <typename T, bool GATE> struct Slot {
+    static constexpr int kRow = kChW * (int)sizeof(T);
+    static constexpr int kBC = 16 * (int)sizeof(T);
+    static constexpr int kX = 0, kDl = kRow, kZ = 2 * kRow;
+    static constexpr int kB = (GATE ? 3 : 2) * kRow, kC = kB + kBC;
+    static constexpr int kBytes = kC + kBC;
+    static constexpr int kPieces = kBytes / 16;             // 16-byte copies per step
+    static constexpr int kGroupPieces = kG * kPieces;
+    static constexpr int kPerLane = (kGroupPieces + 31) / 32;
+    static constexpr int kGroupBytes = kG * kBytes;
+    static_assert(kBytes % 16 == 0 && kB % 16 == 0 && kRow % 16 == 0, "16-byte pieces");
+};
+
+template <typename T, bool GATE> struct WarpSmem {
+    __align__(16) char ring[kStages][Slot<T, GATE>::kGroupBytes];
+};
+
+__device__ __forceinline__ uint64_t policy_evict_last()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_first()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_normal()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+// 16-byte cp.async with an L2 policy; n = 16 copies, n = 0 writes zeros
+// without reading (src is a valid address all the same)
+__device__ __forceinline__ void cp16(uint32_t dst, const char *src, int n, uint64_t pol)
+{
+    if (!SSM_S6_SPLIT_HINTS) {
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
+        return;
+    }
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;" ::"r"(dst), "l"(src), "r"(n),
+                 "l"(pol)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int K> __device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(K) : "memory"); }
+__device__ __forceinline__ void pair_barrier() { asm volatile("bar.sync 1, 64;" ::: "memory"); }
+
+__device__ __forceinline__ void st_pol(float *p, float v, uint64_t pol)
+{
+    if (!SSM_S6_SPLIT_HINTS) {
+        *p = v;
+        return;
+    }
+    asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(p), "f"(v), "l"(pol) : "memory");
+}
+__device__ __forceinline__ void st_pol(__nv_bfloat16 *p, float v, uint64_t pol)
+{
+    if (!SSM_S6_SPLIT_HINTS) {
+        *p = __float2bfloat16_rn(v);
+        return;
+    }
+    const unsigned short u = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+    asm volatile("st.global.L2::cache_hint.b16 [%0], %1, %2;" ::"l"(p), "h"(u), "l"(pol) : "memory");
+}
+
+template <typename T> __device__ __forceinline__ float lds1(const char *p);
+template <> __device__ __forceinline__ float lds1<float>(const char *p) { return *reinterpret_cast<const float *>(p); }
+template <> __device__ __forceinline__ float lds1<__nv_bfloat16>(const char *p)
+{
+    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(p));
+}
+// four consecutive elements (this thread's quarter of a B or C row) as floats
+template <typename T> __device__ __forceinline__ float4 lds4(const char *p);
+template <> __device__ __forceinline__ float4 lds4<float>(const char *p) { return *reinterpret_cast<const float4 *>(p); }
+template <> __device__ __forceinline__ float4 lds4<__nv_bfloat16>(const char *p)
+{
+    const uint2 u = *reinterpret_cast<const uint2 *>(p);
+    return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u), __uint_as_float(u.y << 16),
+                       __uint_as_float(u.y & 0xffff0000u));
+}
+
+// What a group does with its outputs: store them (one direction); park them
+// (first half of a bidirectional pair); park the steps before the exchange
+// point, meet the partner, then add to the rest (the group holding the
+// exchange point); add the partner's parked values (second half).
+enum Mode { kPlain, kPark, kMixed, kAdd };
+template <Mode M> using ModeTag = std::integral_constant<Mode, M>;
+
+template <typename T, bool BIDIR, bool GATE, bool SOFTPLUS>
+__global__ void __launch_bounds__(64, kMinBlocks) s6_split_kernel(const S6Args a)
+{
+    using S = Slot<T, GATE>;
+    __shared__ WarpSmem<T, GATE> smem[2];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    WarpSmem<T, GATE> &sm = smem[warp];
+    const int g = lane >> 2, q = lane & 3;
+    const int dsel = BIDIR ? warp : 0;
+    const int d0 = (BIDIR ? (int)blockIdx.x : (int)blockIdx.x * 2 + warp) * kChW;   // the warp's first channel
+    const int b = blockIdx.y;
+    const int L = a.L, D = a.D;
+    if (!BIDIR && d0 >= D)
+        return;   // whole warp past the channels (no barrier partner in this mode)
+    const int d = d0 + g;
+    const bool active = d < D;
+    const bool rev = BIDIR ? dsel == 1 : a.reverse != 0;
+    const DirArgs &P = a.dir[dsel];
+
+    // this thread's states [4q, 4q + 4) as two pairs, A scaled by log2(e)
+    float2 A2[2], h2[2];
+    {
+        float4 av = make_float4(0.f, 0.f, 0.f, 0.f), hv = av;
+        if (active) {
+            av = *reinterpret_cast<const float4 *>(P.A + (size_t)d * 16 + 4 * q);
+            if (P.init)
+                hv = *reinterpret_cast<const float4 *>(P.init + ((size_t)b * D + d) * 16 + 4 * q);
+        }
+        A2[0] = make_float2(av.x * kLog2e, av.y * kLog2e);
+        A2[1] = make_float2(av.z * kLog2e, av.w * kLog2e);
+        h2[0] = make_float2(hv.x, hv.y);
+        h2[1] = make_float2(hv.z, hv.w);
+    }
+    const float bias = (active && P.bias) ? P.bias[d] : 0.f;
+    const float Dd = (active && P.D) ? P.D[d] : 0.f;
+
+    // steps before the exchange (bidirectional), in this warp's scan order
+    const int M = BIDIR ? (rev ? L / 2 : (L + 1) / 2) : L;
+    const int G = (L + kG - 1) / kG;
+
+    // --- copies: this lane's 16-byte pieces of a group (piece p = lane + 32 j)
+    const uint64_t pol_last = policy_evict_last(), pol_first = policy_evict_first();
+    const uint64_t pol_normal = policy_evict_normal();
+    const T *x = static_cast<const T *>(a.x), *dl = static_cast<const T *>(a.delta);
+    const T *zp = static_cast<const T *>(P.z);
+    const T *Bm = static_cast<const T *>(P.B), *Cm = static_cast<const T *>(P.C);
+    const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(&sm.ring[0][0]);
+    const char *safe = static_cast<const char *>(a.x);
+    // (piece p of a group lands at byte 16 p of the group's slots: step
+    // p / kPieces, byte 16 (p % kPieces) of that step's slot)
+    const char *cur[S::kPerLane];     // source row of the next group to issue
+    int gstep[S::kPerLane];           // bytes from one group's rows to the next's
+    bool pok[S::kPerLane];            // the piece holds channels below D
+    bool xd[S::kPerLane];             // an x / delta piece: L2 policy by half
+    uint64_t pfix[S::kPerLane];       // the policy of the other pieces
+#pragma unroll
+    for (int j = 0; j < S::kPerLane; j++) {
+        const int p = lane + 32 * j;
+        const bool exists = p < S::kGroupPieces;
+        const int pp = exists ? p : 0;
+        const int s = pp / S::kPieces, off = (pp % S::kPieces) * 16;
+        const int t0 = rev ? L - 1 - s : s;
+        const char *base;
+        long long row;
+        bool ok = exists;
+        if (off < S::kB) {   // x, delta or z of 16 bytes' worth of the warp's channels
+            const int arr = off / S::kRow, jb = off % S::kRow;
+            const T *src = arr == 0 ? x : arr == 1 ? dl : zp;
+            xd[j] = arr < 2;
+            pfix[j] = pol_first;
+            ok = ok && d0 + jb / (int)sizeof(T) < D;
+            row = (long long)D * sizeof(T);
+            base = reinterpret_cast<const char *>(src) + ((long long)b * L + t0) * row + (long long)d0 * sizeof(T) + jb;
+        } else {             // 16 bytes of the B or C row (read by every warp of this batch row)
+            const int o2 = off - S::kB;
+            const T *src = o2 < S::kBC ? Bm : Cm;
+            xd[j] = false;
+            pfix[j] = pol_normal;
+            row = 16 * (long long)sizeof(T);
+            base = reinterpret_cast<const char *>(src) + ((long long)b * L + t0) * row + o2 % S::kBC;
+        }
+        pok[j] = ok;
+        cur[j] = ok ? base : safe;
+        gstep[j] = ok ? (rev ? -1 : 1) * kG * (int)row : 0;
+    }
+    auto issue = [&](int gi) {
+        if (gi < G) {
+            const uint32_t sb = ring_s + (uint32_t)((gi & (kStages - 1)) * S::kGroupBytes) + 16 * lane;
+            const uint64_t pxd = (BIDIR && gi * kG < M) ? pol_last : pol_first;
+            if ((gi + 1) * kG <= L) {
+#pragma unroll
+                for (int j = 0; j < S::kPerLane; j++)
+                    if (lane + 32 * j < S::kGroupPieces)
+                        cp16(sb + 512 * j, cur[j], pok[j] ? 16 : 0, xd[j] ? pxd : pfix[j]);
+            } else {   // the last group is short: steps past L are zero-filled, not read
+#pragma unroll
+                for (int j = 0; j < S::kPerLane; j++)
+                    if (lane + 32 * j < S::kGroupPieces) {
+                        const bool in = pok[j] && gi * kG + (lane + 32 * j) / S::kPieces < L;
+                        cp16(sb + 512 * j, in ? cur[j] : safe, in ? 16 : 0, xd[j] ? pxd : pfix[j]);
+                    }
+            }
+#pragma unroll
+            for (int j = 0; j < S::kPerLane; j++)
+                cur[j] += gstep[j];
+        }
+        cp_commit();
+    };
+
+    // --- outputs: element index of this thread's step of the current group
+    T *out = static_cast<T *>(a.out);
+    float *stash = a.stash;
+    long long oi = ((long long)b * L + (rev ? L - 1 - q : q)) * D + d;
+    const int ostep = (rev ? -1 : 1) * kG * D;
+    float pv = 0.f;   // the partner's parked value for this thread's step (kAdd)
+    auto load_partner = [&](int gi) {
+        if (active && gi * kG + q < L)
+            pv = __ldcg(stash + oi);
+    };
+
+    auto group = [&](int gi, auto mode_tag) {
+        constexpr Mode MODE = decltype(mode_tag)::value;
+        issue(gi + kStages - 1);
+        cp_wait<kStages - 1>();
+        __syncwarp();
+        const char *gs = &sm.ring[gi & (kStages - 1)][0];
+        const int i = gi * kG + q;   // this thread's step
+        const bool valid = i < L;
+        // A: step q's scalars
+        const char *sq = gs + q * S::kBytes + g * (int)sizeof(T);
+        const float xv = lds1<T>(sq + S::kX);
+        float dt = lds1<T>(sq + S::kDl) + bias;
+        if (SOFTPLUS)
+            dt = softplus_f(dt);
+        dt = valid ? dt : 0.f;   // past L: exp(0) = 1 and no input, the state passes through
+        const float dtx = dt * xv;
+        const float gate = GATE ? silu_f<T>(lds1<T>(sq + S::kZ)) : 1.f;
+        const float dxv = Dd * xv;
+        // B: the four steps' state updates and shares of C . h (step s's dt
+        // and dt x come from thread s of the channel)
+        float part[kG];
+#pragma unroll
+        for (int s = 0; s < kG; s++) {
+            const float dts = __shfl_sync(0xffffffffu, dt, (lane & ~3) | s);
+            const float dtxs = __shfl_sync(0xffffffffu, dtx, (lane & ~3) | s);
+            const char *ss = gs + s * S::kBytes + q * 4 * (int)sizeof(T);
+            const float4 B4 = lds4<T>(ss + S::kB), C4 = lds4<T>(ss + S::kC);
+            const float2 dt2 = make_float2(dts, dts), dtx2 = make_float2(dtxs, dtxs);
+            float2 v = __fmul2_rn(dt2, A2[0]);
+            float2 e = make_float2(ex2_mufu(v.x), ex2_mufu(v.y));
+            h2[0] = __ffma2_rn(e, h2[0], __fmul2_rn(dtx2, make_float2(B4.x, B4.y)));
+            v = __fmul2_rn(dt2, A2[1]);
+            e = make_float2(ex2_mufu(v.x), ex2_mufu(v.y));
+            h2[1] = __ffma2_rn(e, h2[1], __fmul2_rn(dtx2, make_float2(B4.z, B4.w)));
+            float2 y2 = __fmul2_rn(make_float2(C4.x, C4.y), h2[0]);
+            y2 = __ffma2_rn(make_float2(C4.z, C4.w), h2[1], y2);
+            part[s] = y2.x + y2.y;
+        }
+        // C: sum the four threads' shares so that thread q holds step q's:
+        // exchange halves across q bit 1 (steps {0, 1} vs {2, 3}), then
+        // across q bit 0
+        const bool hi1 = (q & 2) != 0, hi0 = (q & 1) != 0;
+        float ka = hi1 ? part[2] : part[0], kb = hi1 ? part[3] : part[1];
+        ka += __shfl_xor_sync(0xffffffffu, hi1 ? part[0] : part[2], 2);
+        kb += __shfl_xor_sync(0xffffffffu, hi1 ? part[1] : part[3], 2);
+        const float ysum = (hi0 ? kb : ka) + __shfl_xor_sync(0xffffffffu, hi0 ? ka : kb, 1);
+        const float y = (ysum + dxv) * gate;
+        const bool st = active && valid;
+        if (MODE == kPlain) {
+            if (st)
+                st_pol(out + oi, y, pol_first);
+        } else if (MODE == kPark) {
+            if (st)
+                st_pol(stash + oi, y, pol_last);
+        } else if (MODE == kMixed) {
+            if (st && i < M)
+                st_pol(stash + oi, y, pol_last);
+            pair_barrier();   // both warps' parked halves are written
+            if (st && i >= M)
+                st_pol(out + oi, y + __ldcg(stash + oi), pol_first);
+        } else {
+            if (st)
+                st_pol(out + oi, y + pv, pol_first);
+        }
+        oi += ostep;
+        if (MODE == kAdd)
+            load_partner(gi + 1);   // one group ahead
+        __syncwarp();   // every thread is done with this group's slots and tables
+    };
+
+#pragma unroll
+    for (int k = 0; k < kStages - 1; k++)
+        issue(k);
+    if (!BIDIR) {
+        for (int gi = 0; gi < G; gi++)
+            group(gi, ModeTag<kPlain>{});
+    } else {
+        // groups [0, g1) lie wholly before the exchange point, [g2, G) wholly after
+        const int g1 = M / kG, g2 = (M + kG - 1) / kG;
+        for (int gi = 0; gi < g1; gi++)
+            group(gi, ModeTag<kPark>{});
+        if (g1 < g2)
+            group(g1, ModeTag<kMixed>{});
+        else
+            pair_barrier();
+        load_partner(g2);
+        for (int gi = g2; gi < G; gi++)
+            group(gi, ModeTag<kAdd>{});
+    }
+    cp_wait<0>();
+
+    if (active && P.last_state)
+        *reinterpret_cast<float4 *>(P.last_state + ((size_t)b * D + d) * 16 + 4 * q) =
+            make_float4(h2[0].x, h2[0].y, h2[1].x, h2[1].y);
+}
+
+template <typename T, bool GATE, bool SOFTPLUS>
+cudaError_t launch_t(const S6Args &a, cudaStream_t st)
+{
+    if (a.ndir == 2) {
+        const dim3 grid((unsigned)((a.D + kChW - 1) / kChW), (unsigned)a.Bsz);
+        s6_split_kernel<T, true, GATE, SOFTPLUS><<<grid, 64, 0, st>>>(a);
+    } else {
+        const dim3 grid((unsigned)((a.D + 2 * kChW - 1) / (2 * kChW)), (unsigned)a.Bsz);
+        s6_split_kernel<T, false, GATE, SOFTPLUS><<<grid, 64, 0, st>>>(a);
+    }
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_flags(const S6Args &a, cudaStream_t st)
+{
+    const bool gate = a.dir[0].z != nullptr;
+    if (gate)
+        return a.softplus ? launch_t<T, true, true>(a, st) : launch_t<T, true, false>(a, st);
+    return a.softplus ? launch_t<T, false, true>(a, st) : launch_t<T, false, false>(a, st);
+}
+
+}  // namespace
+
+std::atomic<int> g_split_mode{0};   // 0 cost model, 1 never, 2 whenever supported
+
+bool split_eligible(int64_t Bsz, int64_t L, int64_t D, int64_t N, int ndir)
+{
+    if (N != 16 || L <= 0 || Bsz <= 0 || D <= 0 || Bsz > 65535)
+        return false;
+    const int mode = g_split_mode.load(std::memory_order_relaxed);
+    if (mode != 0)
+        return mode == 2;
+    const int64_t warps1 = (int64_t)ndir * Bsz * ((D + 63) / 64);   // one thread, two channels
+    if (warps1 >= SSM_S6_SPLIT_MAX_WARPS1)
+        return false;
+    const double E = (double)ndir * Bsz * L * D * 16;
+    const double tl = (double)L * (ndir == 2 ? 0.17 : 0.105);
+    const double tt = E / (ndir == 2 ? 1.5e6 : 2.0e6);
+    const double t_split = (tl > tt ? tl + 0.3 * tt : tt + 0.3 * tl) + 2.0;
+    const double t_other = 24.0 + E / 1.2e6;
+    return t_split < t_other;
+}
+
+void split_mode_set(int mode) { g_split_mode.store(mode, std::memory_order_relaxed); }
+
+cudaError_t launch_s6_split(const S6Args &a, cudaStream_t st)
+{
+    return a.dtype == 0 ? launch_flags<float>(a, st) : launch_flags<__nv_bfloat16>(a, st);
+}
+
+}  // namespace ssm

@@ -112,8 +112,14 @@ ssm_status run_s6(const ssm_dims *dims, const void *x, const void *delta, int so
             a.dir[i].ckpt = ckpt[i];
     }
     a.out = out;
+    if (!order && !mask && !conv && !ckpt &&
+        ssm::split_eligible(dims->batch, dims->seqlen, dims->dim, dims->dstate, ndir)) {
+        a.split = 1;   // one pass, four threads per channel
+        a.S = 1;
+        a.T = a.L;
+    }
     char *w = static_cast<char *>(ws);
-    if (plan.S > 1) {
+    if (a.S > 1) {
         a.carry_h = reinterpret_cast<float *>(w + plan.carry_h_off);
         a.carry_s = reinterpret_cast<float *>(w + plan.carry_s_off);
     }
@@ -149,9 +155,15 @@ ssm_status ssm_scan_plan(const ssm_dims *dims, int bidirectional, int *segments,
     if (st != SSM_OK)
         return st;
     ssm::S6Plan plan{1, 0, 2, 0, 0, 0, 0};
-    if (!empty_s6(dims))
-        plan = ssm::plan_s6(dims->batch, dims->seqlen, dims->dim, dims->dstate,
-                            bidirectional ? 2 : 1, dims->dtype == SSM_F32 ? 0 : 1);
+    const int ndir = bidirectional ? 2 : 1;
+    if (!empty_s6(dims)) {
+        plan = ssm::plan_s6(dims->batch, dims->seqlen, dims->dim, dims->dstate, ndir,
+                            dims->dtype == SSM_F32 ? 0 : 1);
+        if (ssm::split_eligible(dims->batch, dims->seqlen, dims->dim, dims->dstate, ndir)) {
+            plan.S = 1;     // one pass
+            plan.cpl = 0;   // four threads share each channel
+        }
+    }
     if (segments)
         *segments = plan.S;
     if (channels_per_lane)
@@ -685,6 +697,14 @@ ssm_status ssm_check_device(void *stream)
 }
 
 void ssm_debug_ssd_stall(int withhold_chunk, unsigned wait_limit) { ssm::ssd_stall_set(withhold_chunk, wait_limit); }
+
+ssm_status ssm_debug_s6_mapping(int mode)
+{
+    if (mode < 0 || mode > 2)
+        return SSM_ERR_INVALID_ARG;
+    ssm::split_mode_set(mode);
+    return SSM_OK;
+}
 
 const char *ssm_status_string(ssm_status s)
 {

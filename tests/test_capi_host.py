@@ -152,6 +152,13 @@ def test_scan_plan(lib):
     workloads' sizes, the bounds the plan keeps, and its argument checks."""
     # Vim-Small bidirectional: enough channels for one pass, two per lane
     assert ssm.scan_plan(64, 197, 768, 16, bidirectional=True) == (1, 2)
+    # fewer channels on a short sequence: four threads per channel, one pass
+    assert ssm.scan_plan(1, 196, 384, 16) == (1, 0)                       # Vim-Tiny
+    assert ssm.scan_plan(16, 197, 768, 16, bidirectional=True) == (1, 0)
+    assert ssm.scan_plan(8, 197, 768, 16, ssm.SSM_BF16) == (1, 0)
+    # ... never with N < 16, never for a long sequence with few channels
+    assert ssm.scan_plan(1, 196, 384, 8)[1] in (1, 2)
+    assert ssm.scan_plan(1, 4096, 384, 16)[1] in (1, 2)
     # the bf16 workloads have few channels: one per lane, several segments
     for b, L, D in ((8, 1024, 768), (4, 16384, 192)):
         seg, cpl = ssm.scan_plan(b, L, D, 16, ssm.SSM_BF16, bidirectional=True)
@@ -171,6 +178,23 @@ def test_scan_plan(lib):
     with pytest.raises(ssm.SSMError):
         ssm.scan_plan(1, 10, 30, 16)                 # D not a multiple of 4
     assert lib.ssm_scan_plan(None, 0, None, None) == 1
+
+
+def test_s6_mapping_hook(lib):
+    """ssm_debug_s6_mapping forces either thread layout (the plan reports
+    it), refuses other modes, and mode 0 gives the cost model back."""
+    try:
+        with ssm.s6_mapping(ssm.MAPPING_SPLIT_STATES):
+            assert ssm.scan_plan(64, 197, 768, 16, bidirectional=True) == (1, 0)
+            assert ssm.scan_plan(1, 4096, 384, 16) == (1, 0)
+            assert ssm.scan_plan(1, 196, 384, 8)[1] in (1, 2)     # N < 16: never
+        with ssm.s6_mapping(ssm.MAPPING_WHOLE_CHANNELS):
+            assert ssm.scan_plan(1, 196, 384, 16)[1] in (1, 2)
+        assert ssm.scan_plan(1, 196, 384, 16) == (1, 0)
+        assert lib.ssm_debug_s6_mapping(3) == 1
+        assert lib.ssm_debug_s6_mapping(-1) == 1
+    finally:
+        lib.ssm_debug_s6_mapping(0)
 
 
 def test_state_and_step_validation(lib):

@@ -14,6 +14,10 @@ import selective_state_space_24_b200 as ssm
 from oracle import grads as ograds
 from gpu_util import TOL, dev, dir_params, f32dev, rel_err
 
+
+def host_f(t):
+    return t.float().cpu().numpy()
+
 pytestmark = pytest.mark.gpu
 
 NAMES = {"dx": "x", "ddelta": "delta", "dA": "A", "dB": "B", "dC": "C", "dD": "D", "dz": "z",
@@ -29,6 +33,13 @@ def _inputs(inp, dtype):
     return dict(x=dev(inp.x, dtype), delta=dev(inp.delta, dtype), A=f32dev(inp.A_f), B=dev(inp.B_f, dtype),
                 C=dev(inp.C_f, dtype), delta_bias=f32dev(inp.dt_bias_f), D=f32dev(inp.D_f),
                 z=dev(inp.z_f, dtype))
+
+
+def _ckpt_segments(B, L, D, dtype):
+    """Segments of the checkpointing forward's plan: it always gives each
+    thread whole channels (the plan of the plain calls under that layout)."""
+    with ssm.s6_mapping(ssm.MAPPING_WHOLE_CHANNELS):
+        return ssm.scan_plan(B, L, D, 16, ssm.SSM_F32 if dtype == "f32" else ssm.SSM_BF16)[0]
 
 
 def _recomputed_ckpt(t, reverse, dout):
@@ -56,26 +67,33 @@ def _recomputed_ckpt(t, reverse, dout):
 @pytest.mark.parametrize("L", [101, 3000])
 def test_fwd_ckpt_outputs_and_checkpoints(dtype, reverse, L):
     """The checkpointing forward writes the plain forward's outputs and last
-    state bit for bit, and the state entering every 4-step chunk: equal bit
-    for bit to the backward's recompute when the plan has one segment, and
-    within rounding of it when the sequence is cut into segments (entering
-    states then come from the carry pass)."""
+    state: bit for bit when the plain forward takes the same thread layout
+    (one or two channels per thread), to rounding when it splits the
+    channels' states over four threads.  It also writes the state entering
+    every 4-step chunk: equal bit for bit to the backward's recompute when
+    the plan has one segment, and within rounding of it when the sequence is
+    cut into segments (entering states then come from the carry pass)."""
     inp = ssm_gen.make_s6_inputs(2, L, 96, 16, dtype=dtype, seed=L + reverse, random_A=True, random_D=True)
     t = _inputs(inp, dtype)
     ls0 = torch.zeros((2, 96, 16), device="cuda")
     ls1 = torch.zeros((2, 96, 16), device="cuda")
+    ls2 = torch.zeros((2, 96, 16), device="cuda")
     kw = dict(delta_bias=t["delta_bias"], D=t["D"], z=t["z"], reverse=reverse)
-    out0 = ssm.ssm_scan_fwd(t["x"], t["delta"], t["A"], t["B"], t["C"], last_state=ls0, **kw)
+    with ssm.s6_mapping(ssm.MAPPING_WHOLE_CHANNELS):
+        out0 = ssm.ssm_scan_fwd(t["x"], t["delta"], t["A"], t["B"], t["C"], last_state=ls0, **kw)
+    with ssm.s6_mapping(ssm.MAPPING_SPLIT_STATES):
+        out2 = ssm.ssm_scan_fwd(t["x"], t["delta"], t["A"], t["B"], t["C"], last_state=ls2, **kw)
     out1, ck = ssm.ssm_scan_fwd_ckpt(t["x"], t["delta"], t["A"], t["B"], t["C"], last_state=ls1, **kw)
     torch.cuda.synchronize()
     assert torch.equal(out0, out1) and torch.equal(ls0, ls1)
+    assert rel_err(host_f(out2), host_f(out1)) <= TOL[dtype] and rel_err(host_f(ls2), host_f(ls1)) <= TOL["f32"]
     dout = dev(np.ones(inp.x.shape, np.float32), dtype)
     ref = _recomputed_ckpt(t, reverse, dout)
     assert ck.shape == ref.shape
     nck = (L + 3) // 4
     c4 = ck.view(2, nck, 96, 16)
     assert torch.count_nonzero(c4[:, 0]).item() == 0          # chunk 0 enters from zero
-    seg, _ = ssm.scan_plan(2, L, 96, 16, ssm.SSM_F32 if dtype == "f32" else ssm.SSM_BF16)
+    seg = _ckpt_segments(2, L, 96, dtype)
     if seg == 1:
         assert torch.equal(ck, ref)
     else:
@@ -111,7 +129,7 @@ def test_bwd_ckpt_matches_autograd(dtype, reverse, B, L, D):
     for k, v in g.items():
         e = rel_err(v.cpu().numpy(), ref[NAMES[k]])
         assert e <= TOL[dtype], f"{k}: rel err {e:.3e}"
-    seg, _ = ssm.scan_plan(B, L, D, 16, ssm.SSM_F32 if dtype == "f32" else ssm.SSM_BF16)
+    seg = _ckpt_segments(B, L, D, dtype)
     for k in (("dx", "ddelta", "dz") if seg == 1 else ("dx",)):
         assert torch.equal(g[k], g0[k]), k
 
@@ -129,7 +147,8 @@ def test_bidir_ckpt_pair_matches_autograd(dtype, L):
         dout = ssm_gen.round_to_bf16(dout)
     f, b = dir_params(inp, "f"), dir_params(inp, "b")
     x, delta, dd = dev(inp.x, dtype), dev(inp.delta, dtype), dev(dout, dtype)
-    out0 = ssm.bidir_scan_fwd(x, delta, f, b)
+    with ssm.s6_mapping(ssm.MAPPING_WHOLE_CHANNELS):   # the layout the checkpointing forward takes
+        out0 = ssm.bidir_scan_fwd(x, delta, f, b)
     out1, ckf, ckb = ssm.bidir_scan_fwd_ckpt(x, delta, f, b)
     dx, ddelta, gf, gb = ssm.bidir_scan_bwd_ckpt(x, delta, f, b, dd, ckf, ckb)
     torch.cuda.synchronize()

@@ -98,7 +98,8 @@ def test_identity_order_is_bitwise_plain():
     inp = ssm_gen.make_s6_inputs(2, 300, 64, 16, dtype="f32", bidir=True, seed=12)
     f, b = dir_params(inp, "f"), dir_params(inp, "b")
     x, delta = dev(inp.x, "f32"), dev(inp.delta, "f32")
-    plain = ssm.bidir_scan_fwd(x, delta, f, b)
+    with ssm.s6_mapping(ssm.MAPPING_WHOLE_CHANNELS):   # the layout the ordered scan takes
+        plain = ssm.bidir_scan_fwd(x, delta, f, b)
     ordered = ssm.bidir_scan_fwd_ordered(x, delta, f, b, order=_i32(np.arange(300)),
                                          mask=_u8(np.ones((2, 300))))
     torch.cuda.synchronize()

@@ -100,6 +100,11 @@ def test_lane_mappings(batch, L, D, bidir, dtype, cpl):
     segments, against the oracle on sampled columns (reversed for the
     single-direction cases)."""
     code = ssm.SSM_F32 if dtype == "f32" else ssm.SSM_BF16
+    with ssm.s6_mapping(ssm.MAPPING_WHOLE_CHANNELS):
+        _lane_mapping_case(batch, L, D, bidir, dtype, cpl, code)
+
+
+def _lane_mapping_case(batch, L, D, bidir, dtype, cpl, code):
     seg, got = ssm.scan_plan(batch, L, D, 16, code, bidirectional=bidir)
     assert got == cpl and seg > 1
     inp = ssm_gen.make_s6_inputs(batch, L, D, 16, dtype=dtype, bidir=bidir, seed=L + D,

@@ -1,0 +1,163 @@
+"""GPU parity of the four-threads-per-channel layout of the plain S6 scans
+(s6_split.cu) against the float64 oracle.  The layout is forced with the
+library's test hook, so shapes the cost model would give to the other
+layout are covered too: sequence lengths whose last 4-step group is short,
+the bidirectional exchange point falling inside a group or on its edge, a
+warp only partly inside D, absent optional inputs, initial and last states,
+and agreement with the one-or-two-channels-per-thread layout at full
+sizes."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import ssm_gen
+import selective_state_space_24_b200 as ssm
+from gpu_util import NTHREADS, TOL, dev, f32dev, host, rel_err, run_bidir, run_s6
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib(cuda_device):
+    ssm.load()
+
+
+@pytest.fixture(autouse=True)
+def _split_layout():
+    with ssm.s6_mapping(ssm.MAPPING_SPLIT_STATES):
+        yield
+
+
+def _plan_is_split(inp, bidir):
+    code = ssm.SSM_F32 if inp.dtype == "f32" else ssm.SSM_BF16
+    return ssm.scan_plan(inp.batch, inp.seqlen, inp.dim, 16, code, bidirectional=bidir) == (1, 0)
+
+
+# L % 4 covers every length of the last group; for the pair, ceil(L / 2) and
+# floor(L / 2) put the exchange point at every offset inside a group
+@pytest.mark.parametrize("L", [1, 2, 3, 4, 5, 6, 7, 8, 9, 13, 64, 197])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_bidir_every_exchange_offset(L, dtype):
+    inp = ssm_gen.make_s6_inputs(2, L, 24, 16, dtype=dtype, bidir=True, seed=100 + L, random_A=True,
+                                 random_D=True)
+    assert _plan_is_split(inp, True)
+    out, lf, lb = run_bidir(inp, last_state=True)
+    ref, rlf, rlb = oracle.bidir(inp, nthreads=NTHREADS)
+    tol = TOL[dtype]
+    assert rel_err(host(out), ref) <= tol
+    assert rel_err(lf.cpu().numpy(), rlf) <= tol
+    assert rel_err(lb.cpu().numpy(), rlb) <= tol
+
+
+@pytest.mark.parametrize("L", [1, 3, 4, 5, 31, 197])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("reverse", [False, True])
+def test_single_direction_ragged(L, dtype, reverse):
+    inp = ssm_gen.make_s6_inputs(3, L, 40, 16, dtype=dtype, seed=200 + L, random_A=True, random_D=True)
+    assert _plan_is_split(inp, False)
+    out, st = run_s6(inp, reverse=reverse)
+    ref, rst = oracle.s6(inp, reverse=reverse, nthreads=NTHREADS)
+    tol = TOL[dtype]
+    assert rel_err(host(out), ref) <= tol
+    assert rel_err(st.cpu().numpy(), rst) <= tol
+
+
+@pytest.mark.parametrize("bidir", [False, True])
+def test_warp_partly_inside_d(bidir):
+    """fp32 with D = 12: the second block of 8 channels holds 4, so its copies
+    of x / delta / z are half zero-filled and half its threads idle."""
+    inp = ssm_gen.make_s6_inputs(2, 37, 12, 16, dtype="f32", bidir=bidir, seed=7, random_A=True,
+                                 random_D=True)
+    tol = TOL["f32"]
+    if bidir:
+        out, lf, lb = run_bidir(inp, last_state=True)
+        ref, rlf, rlb = oracle.bidir(inp, nthreads=NTHREADS)
+        assert rel_err(lf.cpu().numpy(), rlf) <= tol and rel_err(lb.cpu().numpy(), rlb) <= tol
+    else:
+        out, st = run_s6(inp, reverse=True)
+        ref, rst = oracle.s6(inp, reverse=True, nthreads=NTHREADS)
+        assert rel_err(st.cpu().numpy(), rst) <= tol
+    assert rel_err(host(out), ref) <= tol
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_optional_inputs_absent(dtype):
+    """No gate, no skip, no bias, softplus off (both directions)."""
+    inp = ssm_gen.make_s6_inputs(2, 50, 16, 16, dtype=dtype, bidir=True, seed=9, gate=False)
+    delta = np.abs(inp.delta)
+    x, dl = dev(inp.x, dtype), dev(delta, dtype)
+    mk = lambda s: ssm.DirParams(A=f32dev(getattr(inp, "A" + s)), B=dev(getattr(inp, "B" + s), dtype),
+                                 C=dev(getattr(inp, "C" + s), dtype))
+    out = ssm.bidir_scan_fwd(x, dl, mk("_f"), mk("_b"), delta_softplus=False)
+    one = ssm.ssm_scan_fwd(x, dl, f32dev(inp.A_f), dev(inp.B_f, dtype), dev(inp.C_f, dtype),
+                           delta_softplus=False)
+    torch.cuda.synchronize()
+    xr = host(x).astype(np.float64) if dtype == "bf16" else inp.x
+    dr = host(dl).astype(np.float64) if dtype == "bf16" else delta
+    ref, _, _ = oracle.bidir_arrays(xr, dr, dict(A=inp.A_f, B=inp.B_f, C=inp.C_f),
+                                    dict(A=inp.A_b, B=inp.B_b, C=inp.C_b), softplus=False)
+    ref1, _ = oracle.s6_arrays(xr, dr, inp.A_f, inp.B_f, inp.C_f, softplus=False)
+    assert rel_err(host(out), ref) <= TOL[dtype]
+    assert rel_err(host(one), ref1) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("reverse", [False, True])
+def test_initial_state_and_chained_pieces(reverse):
+    """A scan from a given state, and a sequence scanned as three pieces with
+    the state handed on in place, both against one oracle scan."""
+    Bsz, L, D = 2, 90, 32
+    inp = ssm_gen.make_s6_inputs(Bsz, L, D, 16, dtype="f32", seed=11 + reverse, random_A=True, random_D=True)
+    h0 = np.random.default_rng(3).standard_normal((Bsz, D, 16)).astype(np.float32)
+    A, B, C = f32dev(inp.A_f), dev(inp.B_f, "f32"), dev(inp.C_f, "f32")
+    kw = dict(delta_bias=f32dev(inp.dt_bias_f), D=f32dev(inp.D_f), reverse=reverse)
+    x, delta, z = dev(inp.x, "f32"), dev(inp.delta, "f32"), dev(inp.z_f, "f32")
+    last = torch.empty((Bsz, D, 16), device="cuda")
+    out = ssm.ssm_scan_fwd_state(x, delta, A, B, C, z=z, initial_state=f32dev(h0), last_state=last, **kw)
+    torch.cuda.synchronize()
+    ref, rst = oracle.s6_arrays(inp.x, inp.delta, inp.A_f, inp.B_f, inp.C_f, delta_bias=inp.dt_bias_f,
+                                D=inp.D_f, z=inp.z_f, reverse=reverse, initial_state=h0)
+    assert rel_err(host(out), ref) <= TOL["f32"] and rel_err(last.cpu().numpy(), rst) <= TOL["f32"]
+    # three pieces in scan order, the state carried in place
+    state = f32dev(h0)
+    pieces = [slice(0, 37), slice(37, 38), slice(38, L)]
+    out2 = torch.empty_like(out)
+    for sl in (reversed(pieces) if reverse else pieces):
+        o = ssm.ssm_scan_fwd_state(x[:, sl].contiguous(), delta[:, sl].contiguous(), A, B[:, sl].contiguous(),
+                                   C[:, sl].contiguous(), z=z[:, sl].contiguous(), initial_state=state,
+                                   last_state=state, **kw)
+        out2[:, sl] = o
+    torch.cuda.synchronize()
+    assert rel_err(host(out2), ref) <= TOL["f32"] and rel_err(state.cpu().numpy(), rst) <= TOL["f32"]
+
+
+@pytest.mark.parametrize("dtype,bidir,batch,L,D", [("f32", True, 64, 197, 768), ("bf16", True, 8, 1024, 768),
+                                                   ("f32", False, 16, 197, 768), ("bf16", False, 4, 300, 1536)])
+def test_layouts_agree_at_full_size(dtype, bidir, batch, L, D):
+    """Every output of the two layouts on the same inputs (the cost model
+    picks either for such sizes), and sampled columns against the oracle."""
+    inp = ssm_gen.make_s6_inputs(batch, L, D, 16, dtype=dtype, bidir=bidir, seed=batch + L)
+    run = (lambda: run_bidir(inp, last_state=True)) if bidir else (lambda: run_s6(inp))
+    split = run()
+    with ssm.s6_mapping(ssm.MAPPING_WHOLE_CHANNELS):
+        whole = run()
+    tol = TOL[dtype]
+    for a, b in zip(split, whole):
+        assert rel_err(host(a), host(b)) <= tol
+    cols = np.random.default_rng(0).choice(batch * D, 24, replace=False)
+    bb, dd = np.divmod(cols, D)
+    ref = (oracle.bidir(inp, cols=cols, nthreads=NTHREADS) if bidir
+           else oracle.s6(inp, cols=cols, nthreads=NTHREADS))[0]
+    assert rel_err(host(split[0])[bb, :, dd], ref[bb, :, dd]) <= tol
+
+
+def test_noalloc_takes_the_same_layout():
+    """ssm_scan_fwd_noalloc takes the layout ssm_scan_fwd takes: bit for bit."""
+    inp = ssm_gen.make_s6_inputs(4, 120, 256, 16, dtype="f32", seed=5, random_A=True, random_D=True)
+    x, delta = dev(inp.x, "f32"), dev(inp.delta, "f32")
+    A, B, C = f32dev(inp.A_f), dev(inp.B_f, "f32"), dev(inp.C_f, "f32")
+    kw = dict(delta_bias=f32dev(inp.dt_bias_f), D=f32dev(inp.D_f), z=dev(inp.z_f, "f32"))
+    ref = ssm.ssm_scan_fwd(x, delta, A, B, C, **kw)
+    out = ssm.ssm_scan_fwd_noalloc(x, delta, A, B, C, **kw)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
