@@ -357,9 +357,26 @@ class DeviceWorkload:
         self._bind()
 
     def _launches(self):
-        if self.info["kind"] == "s6":
-            return 3 if self.ws_bytes > 0 else 1
-        return 1
+        """Kernel launches of one call: the S6 plan's segment count decides
+        (summary, carry and main passes, or the main pass alone).  The plain
+        scan reports its own plan; the ordered / conv / checkpointing
+        variants always give each thread whole channels, so their plan is
+        read under that layout."""
+        if self.info["kind"] != "s6":
+            return 1
+        seg, cpl = ctypes.c_int(0), ctypes.c_int(0)
+        query = lambda: self.lib.ssm_scan_plan(ctypes.byref(self.dims), int(self.info["ndir"] == 2),
+                                               ctypes.byref(seg), ctypes.byref(cpl))
+        if self.op == "scan":
+            st = query()
+        else:
+            self.lib.ssm_debug_s6_mapping(1)
+            try:
+                st = query()
+            finally:
+                self.lib.ssm_debug_s6_mapping(0)
+        assert st == 0, st
+        return 3 if seg.value > 1 else 1
 
     def _bind(self):
         d = self.d

@@ -101,3 +101,25 @@ def test_checkpointing_scan_counts_its_checkpoints():
     a, b = bench.workload_info(1), bench.workload_info(1, "fwd_ckpt")
     assert b["elems"] == a["elems"]
     assert b["bytes"] - a["bytes"] == 2 * 64 * ((197 + 3) // 4) * 768 * 16 * 4
+
+
+def test_launch_count_follows_the_plan():
+    """The launches a call makes, as bench.py counts them from the library's
+    plan (host-only query): one pass for Vim-Tiny (four threads per channel)
+    and Vim-Small, summary + carry + main for the long bf16 rows, and the
+    whole-channel plan for the checkpointing variant; SSD one launch."""
+    import types
+    import selective_state_space_24_b200 as ssm
+    lib = ssm.capi()
+    expect = {(0, "scan"): 1, (1, "scan"): 1, (2, "scan"): 3, (3, "scan"): 3, (1, "fwd_ckpt"): 1,
+              (1, "ordered"): 1, (4, "scan"): 1}
+    for (cfg, op), n in expect.items():
+        w = bench.workload_info(cfg, op)
+        dims = None
+        if w["kind"] == "s6":
+            dims = ssm.ssm_dims(w["batch"], w["seqlen"], w["dim"], w["dstate"],
+                                ssm.SSM_F32 if w["dtype"] == "f32" else ssm.SSM_BF16)
+        ns = types.SimpleNamespace(info=w, op=op, lib=lib, dims=dims)
+        assert bench.DeviceWorkload._launches(ns) == n, (cfg, op)
+    # the query leaves the layout choice to the cost model again
+    assert ssm.scan_plan(1, 196, 384, 16) == (1, 0)
