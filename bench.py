@@ -49,7 +49,7 @@ SMS = 148
 # capture of the current kernels (summaries under profiles/); absent where no
 # capture matches them.
 NCU_TRAFFIC = {1: 193.01e6, 4: 397.22e6}
-NCU_TRAFFIC_STEP = 63.05e6
+NCU_TRAFFIC_STEP = 62.01e6
 NCU_TRAFFIC_BWD = {1: 409.56e6}
 
 

@@ -7,8 +7,8 @@
 //     y  = (C h + D x) silu(z).
 //
 // The state is the only large operand (B D N float32 read and written
-// once), so the kernel is HBM-bound; four lanes share one (b, d) row, each
-// holding a quarter of its N <= 16 states in registers.
+// once); one or two lanes share one (b, d) row, each holding its share of
+// the row's N <= 16 states in registers.
 // The transcendentals take the same forms as in the scan kernels
 // (s6_math.cuh), with A scaled by log2(e) before the product with dt.
 #include <cuda_bf16.h>
@@ -30,65 +30,86 @@ template <> __device__ __forceinline__ float ldv<__nv_bfloat16>(const __nv_bfloa
 __device__ __forceinline__ void stv(float *p, size_t i, float v) { p[i] = v; }
 __device__ __forceinline__ void stv(__nv_bfloat16 *p, size_t i, float v) { p[i] = __float2bfloat16_rn(v); }
 
-// Four lanes share one (b, d) row: lane part p owns states [p K, p K + K),
-// K = NS / 4, so a warp's state loads and stores cover 8 whole rows
-// (8 x 4 N bytes) contiguously.  The readout is summed over the four lanes
-// with two shuffles.
-template <typename T, int NS, bool VEC>
+// LANES lanes (1, 2 or 4) share one (b, d) row: lane part p owns states
+// [p K, p K + K), K = NS / LANES, so a warp covers 32 / LANES consecutive
+// rows and each of its state loads spans them contiguously.  All of a
+// row's loads are issued before its arithmetic.  The readout is summed over
+// a row's lanes with log2(LANES) shuffles.  The per-row scalar work
+// (softplus, the gate, the index arithmetic) is done by every lane of the
+// row, so fewer lanes per row issue fewer instructions per state; more
+// states per lane hold more registers and keep fewer rows in flight.
+// Measured on B200 (L2 flushed before each step): N = 16 fp32 (B 512,
+// D 1536) 28.7 us with two lanes per row, 32.8 with four, 34.8 with one;
+// N = 8 bf16 (B 256, D 1000) 10.7 us with one lane, 12.3 with two or four.
+// SSM_STEP_LANES = 0 takes those (two lanes for 16 states, else one).
+#ifndef SSM_STEP_LANES
+#define SSM_STEP_LANES 0
+#endif
+template <typename T, int NS, bool VEC, int LANES>
 __global__ void __launch_bounds__(256) s6_step_kernel(const StepArgs a)
 {
-    constexpr int K = NS / 4;
+    constexpr int K = NS / LANES;
+    static_assert(K >= 1 && NS % LANES == 0, "states split evenly over the lanes");
     const size_t tid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const size_t row = tid >> 2;   // b * D + d
-    const int part = (int)(tid & 3);
-    const bool live = row < (size_t)a.Bsz * a.D;   // whole groups of 4 agree
+    const size_t row = tid / LANES;   // b * D + d
+    const int part = (int)(tid % LANES);
+    const size_t nrows = (size_t)a.Bsz * a.D;
+    const bool live = row < nrows;    // whole groups of LANES lanes agree
     const int N = a.N;
-    const int d = live ? (int)(row % a.D) : 0;
-    const size_t b = live ? row / a.D : 0;
+    size_t b = 0;
+    int d = 0;
+    if (live) {
+        if (nrows <= 0xffffffffu)
+            b = (unsigned)row / (unsigned)a.D;
+        else
+            b = row / (size_t)a.D;
+        d = (int)(row - b * (size_t)a.D);
+    }
     const T *x = static_cast<const T *>(a.x), *dl = static_cast<const T *>(a.delta);
     const T *Bm = static_cast<const T *>(a.B), *Cm = static_cast<const T *>(a.C);
     const T *z = static_cast<const T *>(a.z);
 
-    float y = 0.f, xv = 0.f;
+    float y = 0.f, xv = 0.f, zv = 0.f, Dk = 0.f;
     if (live) {
+        float h[K], Av[K], Bv[K], Cv[K];
         xv = ldv(x, row);
-        float dt = ldv(dl, row) + (a.bias ? a.bias[d] : 0.f);
-        if (a.softplus)
-            dt = softplus_f(dt);
-        const float dtx = dt * xv;
-        float h[K], Av[K];
+        const float dv = ldv(dl, row);
+        if (z)
+            zv = ldv(z, row);
+        const float bias = a.bias ? a.bias[d] : 0.f;
+        Dk = a.Dskip ? a.Dskip[d] : 0.f;   // with the row's other loads, not after the shuffles
         float *st = a.state + row * N + part * K;
         const float *Ar = a.A + (size_t)d * N + part * K;
-        if (VEC) {   // N == NS: this lane's K states are one aligned vector
-            if (K == 4) {
-                const float4 hv = *reinterpret_cast<const float4 *>(st);
-                const float4 av = __ldg(reinterpret_cast<const float4 *>(Ar));
-                h[0] = hv.x, h[1] = hv.y, h[2] = hv.z, h[3] = hv.w;
-                Av[0] = av.x, Av[1] = av.y, Av[2] = av.z, Av[3] = av.w;
-            } else if (K == 2) {
-                const float2 hv = *reinterpret_cast<const float2 *>(st);
-                const float2 av = __ldg(reinterpret_cast<const float2 *>(Ar));
-                h[0] = hv.x, h[1] = hv.y;
-                Av[0] = av.x, Av[1] = av.y;
-            } else {
-                h[0] = st[0];
-                Av[0] = __ldg(Ar);
+        if (VEC && K % 4 == 0) {   // N == NS: this lane's K states are K / 4 aligned vectors
+#pragma unroll
+            for (int v = 0; v < K / 4; v++) {
+                const float4 hv = reinterpret_cast<const float4 *>(st)[v];
+                const float4 av = __ldg(reinterpret_cast<const float4 *>(Ar) + v);
+                h[4 * v] = hv.x, h[4 * v + 1] = hv.y, h[4 * v + 2] = hv.z, h[4 * v + 3] = hv.w;
+                Av[4 * v] = av.x, Av[4 * v + 1] = av.y, Av[4 * v + 2] = av.z, Av[4 * v + 3] = av.w;
             }
+        } else if (VEC && K == 2) {
+            const float2 hv = *reinterpret_cast<const float2 *>(st);
+            const float2 av = __ldg(reinterpret_cast<const float2 *>(Ar));
+            h[0] = hv.x, h[1] = hv.y;
+            Av[0] = av.x, Av[1] = av.y;
         } else {
 #pragma unroll
             for (int k = 0; k < K; k++) {
-                const bool in = part * K + k < N;
+                const bool in = VEC || part * K + k < N;
                 h[k] = in ? st[k] : 0.f;
                 Av[k] = in ? Ar[k] : 0.f;
             }
         }
-        // this lane's B and C values (one 16-byte load each for fp32, N = 16)
-        float Bv[K], Cv[K];
-        if (VEC && K == 4 && sizeof(T) == 4) {
-            const float4 bv = __ldg(reinterpret_cast<const float4 *>(Bm) + (b * N + part * K) / 4);
-            const float4 cv = __ldg(reinterpret_cast<const float4 *>(Cm) + (b * N + part * K) / 4);
-            Bv[0] = bv.x, Bv[1] = bv.y, Bv[2] = bv.z, Bv[3] = bv.w;
-            Cv[0] = cv.x, Cv[1] = cv.y, Cv[2] = cv.z, Cv[3] = cv.w;
+        // this lane's B and C values (16-byte loads for fp32 and N = NS)
+        if (VEC && K % 4 == 0 && sizeof(T) == 4) {
+#pragma unroll
+            for (int v = 0; v < K / 4; v++) {
+                const float4 bv = __ldg(reinterpret_cast<const float4 *>(Bm) + (b * N + part * K) / 4 + v);
+                const float4 cv = __ldg(reinterpret_cast<const float4 *>(Cm) + (b * N + part * K) / 4 + v);
+                Bv[4 * v] = bv.x, Bv[4 * v + 1] = bv.y, Bv[4 * v + 2] = bv.z, Bv[4 * v + 3] = bv.w;
+                Cv[4 * v] = cv.x, Cv[4 * v + 1] = cv.y, Cv[4 * v + 2] = cv.z, Cv[4 * v + 3] = cv.w;
+            }
         } else {
 #pragma unroll
             for (int k = 0; k < K; k++) {
@@ -97,6 +118,10 @@ __global__ void __launch_bounds__(256) s6_step_kernel(const StepArgs a)
                 Cv[k] = (VEC || n < N) ? ldv(Cm, b * N + n) : 0.f;
             }
         }
+        float dt = dv + bias;
+        if (a.softplus)
+            dt = softplus_f(dt);
+        const float dtx = dt * xv;
 #pragma unroll
         for (int k = 0; k < K; k++) {
             const int n = part * K + k;
@@ -106,27 +131,26 @@ __global__ void __launch_bounds__(256) s6_step_kernel(const StepArgs a)
                 y = fmaf(Cv[k], h[k], y);
             }
         }
-        if (VEC) {
-            if (K == 4)
-                *reinterpret_cast<float4 *>(st) = make_float4(h[0], h[1], h[2], h[3]);
-            else if (K == 2)
-                *reinterpret_cast<float2 *>(st) = make_float2(h[0], h[1]);
-            else
-                st[0] = h[0];
+        if (VEC && K % 4 == 0) {
+#pragma unroll
+            for (int v = 0; v < K / 4; v++)
+                reinterpret_cast<float4 *>(st)[v] = make_float4(h[4 * v], h[4 * v + 1], h[4 * v + 2], h[4 * v + 3]);
+        } else if (VEC && K == 2) {
+            *reinterpret_cast<float2 *>(st) = make_float2(h[0], h[1]);
         } else {
 #pragma unroll
             for (int k = 0; k < K; k++)
-                if (part * K + k < N)
+                if (VEC || part * K + k < N)
                     st[k] = h[k];
         }
     }
-    y += __shfl_xor_sync(0xffffffffu, y, 1);
-    y += __shfl_xor_sync(0xffffffffu, y, 2);
+#pragma unroll
+    for (int o = 1; o < LANES; o <<= 1)
+        y += __shfl_xor_sync(0xffffffffu, y, o);
     if (live && part == 0) {
-        if (a.Dskip)
-            y = fmaf(a.Dskip[d], xv, y);
+        y = fmaf(Dk, xv, y);
         if (z)
-            y *= silu_f<T>(ldv(z, row));
+            y *= silu_f<T>(zv);
         stv(static_cast<T *>(a.out), row, y);
     }
 }
@@ -134,12 +158,14 @@ __global__ void __launch_bounds__(256) s6_step_kernel(const StepArgs a)
 template <typename T, int NS>
 cudaError_t launch_ns(const StepArgs &a, cudaStream_t st)
 {
-    const size_t threads = (size_t)a.Bsz * a.D * 4;
+    constexpr int LANES = SSM_STEP_LANES == 0 ? (NS == 16 ? 2 : 1)
+                                              : (NS >= SSM_STEP_LANES ? SSM_STEP_LANES : NS);
+    const size_t threads = (size_t)a.Bsz * a.D * LANES;
     const unsigned grid = (unsigned)((threads + 255) / 256);
     if (a.N == NS)
-        s6_step_kernel<T, NS, true><<<grid, 256, 0, st>>>(a);
+        s6_step_kernel<T, NS, true, LANES><<<grid, 256, 0, st>>>(a);
     else
-        s6_step_kernel<T, NS, false><<<grid, 256, 0, st>>>(a);
+        s6_step_kernel<T, NS, false, LANES><<<grid, 256, 0, st>>>(a);
     return cudaGetLastError();
 }
 
