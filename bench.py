@@ -50,7 +50,7 @@ SMS = 148
 # capture matches them.
 NCU_TRAFFIC = {1: 193.01e6, 4: 397.22e6}
 NCU_TRAFFIC_STEP = 62.01e6
-NCU_TRAFFIC_BWD = {1: 409.56e6}
+NCU_TRAFFIC_BWD = {1: 407.23e6}
 
 
 def parse():
