@@ -46,40 +46,50 @@ constexpr int kQ = 4;                  // threads per channel (a quarter of the 
 constexpr int kG = 4;                  // steps per group: thread q does step q's scalar work
 constexpr int kChW = 32 / kQ;          // channels per warp
 constexpr int kStages = 4;             // groups in the copy ring (a power of two)
+// CTAs (warp pairs) per SM the registers are sized for, and whether the
+// copies and stores carry L2 eviction priorities.  Measured with this
+// layout forced (one B200, µs): 12 CTAs (80 registers) without priorities
+// -- bidirectional B 8, L 1024, D 768 bf16 135, B 32 / 64, L 197 fp32 90 /
+// 164 -- against 16 CTAs (64 registers, spilling in the bidirectional
+// variants) with them 164 / 96 / 168; the problems this layout takes fit
+// in L2, so the priorities only cost registers.
 #ifndef SSM_S6_SPLIT_MINB
-#define SSM_S6_SPLIT_MINB 16
+#define SSM_S6_SPLIT_MINB 12
 #endif
 #ifndef SSM_S6_SPLIT_HINTS
-#define SSM_S6_SPLIT_HINTS 1
+#define SSM_S6_SPLIT_HINTS 0
 #endif
-constexpr int kMinBlocks = SSM_S6_SPLIT_MINB;   // CTAs (warp pairs) per SM: 16 = 32 warps, 64 registers a thread
+constexpr int kMinBlocks = SSM_S6_SPLIT_MINB;
 static_assert(kG == kQ, "each of a channel's threads takes one step of a group");
 static_assert((kStages & (kStages - 1)) == 0, "ring index by mask");
 // When the plain calls take this kernel (split_eligible).  The one-thread-
 // per-channel kernels give a warp 64 channels (two a thread) and run one step
 // in about 1000 cycles; with fewer than SSM_S6_SPLIT_MAX_WARPS1 warps (under
 // two per SM sub-partition) they are latency-bound, or cut the sequence into
-// segments and scan it twice.  This kernel's warps take about 230 cycles a
-// step but issue about half as many instructions again per element, so past
-// that occupancy the other kernels win.  Below it a cost model, fitted to
-// one-B200 timings of both kernels over batch 1 - 64, L 128 - 1024 and
-// D 192 - 1536, picks the faster (microseconds; E = elements B L D N x
-// directions):
-//   this kernel    max(Tl, Tt) + 0.3 min(Tl, Tt) + 2,  Tl = L x 0.105
-//                  (0.17 for a bidirectional pair), Tt = E / 2.0e6 (1.5e6);
-//   the others     24 + E / 1.2e6.
+// segments and scan it twice.  This kernel's warps take a step in a few
+// hundred cycles but issue about half as many instructions again per
+// element, so past that occupancy the other kernels win.  Below it a cost
+// model, fitted to one-B200 timings of both kernels over 47 sizes (batch
+// 1 - 128, L 197 - 16384, D 192 - 1536, both dtypes, one and two
+// directions; it picks the faster in all 47), decides (microseconds;
+// E = elements B L D N x directions):
+//   this kernel    max(Tl, Tt) + 0.3 min(Tl, Tt) + 6 (9 for a pair),
+//                  Tl = L x 0.067 (0.082), Tt = E / 2.15e6 (1.9e6);
+//   the others     22 + 0.01 L + E / 1.333e6.
 #ifndef SSM_S6_SPLIT_MAX_WARPS1
 #define SSM_S6_SPLIT_MAX_WARPS1 1024
 #endif
 
 // One step's slot in the ring: x, delta, (z) for the warp's 8 channels,
-// then the B and C rows.
-template <typename T, bool GATE> struct Slot {
+// then the B and C rows, then (bidirectional) the partner's 8 parked fp32
+// outputs of that step, which are copied only once the pair has met.
+template <typename T, bool GATE, bool BIDIR> struct Slot {
     static constexpr int kRow = kChW * (int)sizeof(T);
     static constexpr int kBC = 16 * (int)sizeof(T);
     static constexpr int kX = 0, kDl = kRow, kZ = 2 * kRow;
     static constexpr int kB = (GATE ? 3 : 2) * kRow, kC = kB + kBC;
-    static constexpr int kBytes = kC + kBC;
+    static constexpr int kPk = kC + kBC;                    // parked row (bidirectional)
+    static constexpr int kBytes = kPk + (BIDIR ? kChW * 4 : 0);
     static constexpr int kPieces = kBytes / 16;             // 16-byte copies per step
     static constexpr int kGroupPieces = kG * kPieces;
     static constexpr int kPerLane = (kGroupPieces + 31) / 32;
@@ -87,24 +97,30 @@ template <typename T, bool GATE> struct Slot {
     static_assert(kBytes % 16 == 0 && kB % 16 == 0 && kRow % 16 == 0, "16-byte pieces");
 };
 
-template <typename T, bool GATE> struct WarpSmem {
-    __align__(16) char ring[kStages][Slot<T, GATE>::kGroupBytes];
+template <typename T, bool GATE, bool BIDIR> struct WarpSmem {
+    __align__(16) char ring[kStages][Slot<T, GATE, BIDIR>::kGroupBytes];
 };
 
 __device__ __forceinline__ uint64_t policy_evict_last()
 {
+    if (!SSM_S6_SPLIT_HINTS)
+        return 0;
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
     return p;
 }
 __device__ __forceinline__ uint64_t policy_evict_first()
 {
+    if (!SSM_S6_SPLIT_HINTS)
+        return 0;
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
     return p;
 }
 __device__ __forceinline__ uint64_t policy_evict_normal()
 {
+    if (!SSM_S6_SPLIT_HINTS)
+        return 0;
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
     return p;
@@ -169,10 +185,10 @@ template <Mode M> using ModeTag = std::integral_constant<Mode, M>;
 template <typename T, bool BIDIR, bool GATE, bool SOFTPLUS>
 __global__ void __launch_bounds__(64, kMinBlocks) s6_split_kernel(const S6Args a)
 {
-    using S = Slot<T, GATE>;
-    __shared__ WarpSmem<T, GATE> smem[2];
+    using S = Slot<T, GATE, BIDIR>;
+    __shared__ WarpSmem<T, GATE, BIDIR> smem[2];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    WarpSmem<T, GATE> &sm = smem[warp];
+    WarpSmem<T, GATE, BIDIR> &sm = smem[warp];
     const int g = lane >> 2, q = lane & 3;
     const int dsel = BIDIR ? warp : 0;
     const int d0 = (BIDIR ? (int)blockIdx.x : (int)blockIdx.x * 2 + warp) * kChW;   // the warp's first channel
@@ -220,6 +236,7 @@ __global__ void __launch_bounds__(64, kMinBlocks) s6_split_kernel(const S6Args a
     int gstep[S::kPerLane];           // bytes from one group's rows to the next's
     bool pok[S::kPerLane];            // the piece holds channels below D
     bool xd[S::kPerLane];             // an x / delta piece: L2 policy by half
+    bool pk[S::kPerLane];             // a piece of the partner's parked row
     uint64_t pfix[S::kPerLane];       // the policy of the other pieces
 #pragma unroll
     for (int j = 0; j < S::kPerLane; j++) {
@@ -231,7 +248,16 @@ __global__ void __launch_bounds__(64, kMinBlocks) s6_split_kernel(const S6Args a
         const char *base;
         long long row;
         bool ok = exists;
-        if (off < S::kB) {   // x, delta or z of 16 bytes' worth of the warp's channels
+        pk[j] = false;
+        if (off >= S::kPk) {   // 4 of the partner's parked fp32 outputs (bidirectional)
+            const int jb = off - S::kPk;
+            xd[j] = false;
+            pk[j] = true;
+            pfix[j] = pol_first;
+            ok = ok && d0 + jb / 4 < D;
+            row = (long long)D * 4;
+            base = reinterpret_cast<const char *>(a.stash) + ((long long)b * L + t0) * row + (long long)d0 * 4 + jb;
+        } else if (off < S::kB) {   // x, delta or z of 16 bytes' worth of the warp's channels
             const int arr = off / S::kRow, jb = off % S::kRow;
             const T *src = arr == 0 ? x : arr == 1 ? dl : zp;
             xd[j] = arr < 2;
@@ -251,6 +277,10 @@ __global__ void __launch_bounds__(64, kMinBlocks) s6_split_kernel(const S6Args a
         cur[j] = ok ? base : safe;
         gstep[j] = ok ? (rev ? -1 : 1) * kG * (int)row : 0;
     }
+    // parked rows are copied only after the pair has met (parked_live), for
+    // the groups wholly after the exchange point
+    bool parked_live = false;
+    int next_gi = 0;   // groups [0, next_gi) have been copied (next_gi <= G)
     auto issue = [&](int gi) {
         if (gi < G) {
             const uint32_t sb = ring_s + (uint32_t)((gi & (kStages - 1)) * S::kGroupBytes) + 16 * lane;
@@ -258,12 +288,12 @@ __global__ void __launch_bounds__(64, kMinBlocks) s6_split_kernel(const S6Args a
             if ((gi + 1) * kG <= L) {
 #pragma unroll
                 for (int j = 0; j < S::kPerLane; j++)
-                    if (lane + 32 * j < S::kGroupPieces)
+                    if (lane + 32 * j < S::kGroupPieces && (!BIDIR || !pk[j] || parked_live))
                         cp16(sb + 512 * j, cur[j], pok[j] ? 16 : 0, xd[j] ? pxd : pfix[j]);
             } else {   // the last group is short: steps past L are zero-filled, not read
 #pragma unroll
                 for (int j = 0; j < S::kPerLane; j++)
-                    if (lane + 32 * j < S::kGroupPieces) {
+                    if (lane + 32 * j < S::kGroupPieces && (!BIDIR || !pk[j] || parked_live)) {
                         const bool in = pok[j] && gi * kG + (lane + 32 * j) / S::kPieces < L;
                         cp16(sb + 512 * j, in ? cur[j] : safe, in ? 16 : 0, xd[j] ? pxd : pfix[j]);
                     }
@@ -271,8 +301,27 @@ __global__ void __launch_bounds__(64, kMinBlocks) s6_split_kernel(const S6Args a
 #pragma unroll
             for (int j = 0; j < S::kPerLane; j++)
                 cur[j] += gstep[j];
+            next_gi = gi + 1;   // cur[] now points at group next_gi's rows
         }
         cp_commit();
+    };
+    // after the pair has met: the parked rows of the groups from g0 on that
+    // were copied before it, then every copy in flight drained (so the
+    // group counting of the waits stays exact)
+    auto catch_up = [&](int g0) {
+        for (int gj = g0; gj < next_gi && gj < G; gj++) {
+            const uint32_t sb = ring_s + (uint32_t)((gj & (kStages - 1)) * S::kGroupBytes) + 16 * lane;
+#pragma unroll
+            for (int j = 0; j < S::kPerLane; j++)
+                if (lane + 32 * j < S::kGroupPieces && pk[j]) {
+                    const bool in = pok[j] && gj * kG + (lane + 32 * j) / S::kPieces < L;
+                    const char *src = cur[j] - (long long)(next_gi - gj) * gstep[j];
+                    cp16(sb + 512 * j, in ? src : safe, in ? 16 : 0, pfix[j]);
+                }
+        }
+        cp_commit();
+        cp_wait<0>();
+        __syncwarp();
     };
 
     // --- outputs: element index of this thread's step of the current group
@@ -280,11 +329,6 @@ __global__ void __launch_bounds__(64, kMinBlocks) s6_split_kernel(const S6Args a
     float *stash = a.stash;
     long long oi = ((long long)b * L + (rev ? L - 1 - q : q)) * D + d;
     const int ostep = (rev ? -1 : 1) * kG * D;
-    float pv = 0.f;   // the partner's parked value for this thread's step (kAdd)
-    auto load_partner = [&](int gi) {
-        if (active && gi * kG + q < L)
-            pv = __ldcg(stash + oi);
-    };
 
     auto group = [&](int gi, auto mode_tag) {
         constexpr Mode MODE = decltype(mode_tag)::value;
@@ -347,12 +391,11 @@ __global__ void __launch_bounds__(64, kMinBlocks) s6_split_kernel(const S6Args a
             if (st && i >= M)
                 st_pol(out + oi, y + __ldcg(stash + oi), pol_first);
         } else {
-            if (st)
-                st_pol(out + oi, y + pv, pol_first);
+            if (st)   // the partner's parked value, copied with this group's rows
+                st_pol(out + oi, y + *reinterpret_cast<const float *>(gs + q * S::kBytes + S::kPk + 4 * g),
+                       pol_first);
         }
         oi += ostep;
-        if (MODE == kAdd)
-            load_partner(gi + 1);   // one group ahead
         __syncwarp();   // every thread is done with this group's slots and tables
     };
 
@@ -371,7 +414,8 @@ __global__ void __launch_bounds__(64, kMinBlocks) s6_split_kernel(const S6Args a
             group(g1, ModeTag<kMixed>{});
         else
             pair_barrier();
-        load_partner(g2);
+        parked_live = true;
+        catch_up(g2);
         for (int gi = g2; gi < G; gi++)
             group(gi, ModeTag<kAdd>{});
     }
@@ -419,10 +463,10 @@ bool split_eligible(int64_t Bsz, int64_t L, int64_t D, int64_t N, int ndir)
     if (warps1 >= SSM_S6_SPLIT_MAX_WARPS1)
         return false;
     const double E = (double)ndir * Bsz * L * D * 16;
-    const double tl = (double)L * (ndir == 2 ? 0.17 : 0.105);
-    const double tt = E / (ndir == 2 ? 1.5e6 : 2.0e6);
-    const double t_split = (tl > tt ? tl + 0.3 * tt : tt + 0.3 * tl) + 2.0;
-    const double t_other = 24.0 + E / 1.2e6;
+    const double tl = (double)L * (ndir == 2 ? 0.082 : 0.067);
+    const double tt = E / (ndir == 2 ? 1.9e6 : 2.15e6);
+    const double t_split = (tl > tt ? tl + 0.3 * tt : tt + 0.3 * tl) + (ndir == 2 ? 9.0 : 6.0);
+    const double t_other = 22.0 + 0.01 * (double)L + E / 1.333e6;
     return t_split < t_other;
 }
 

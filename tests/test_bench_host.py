@@ -105,13 +105,14 @@ def test_checkpointing_scan_counts_its_checkpoints():
 
 def test_launch_count_follows_the_plan():
     """The launches a call makes, as bench.py counts them from the library's
-    plan (host-only query): one pass for Vim-Tiny (four threads per channel)
-    and Vim-Small, summary + carry + main for the long bf16 rows, and the
-    whole-channel plan for the checkpointing variant; SSD one launch."""
+    plan (host-only query): one pass for Vim-Tiny and the hi-res bf16 scan
+    (four threads per channel) and Vim-Small, summary + carry + main for the
+    long bf16 rows, and the whole-channel plan for the checkpointing
+    variant; SSD one launch."""
     import types
     import selective_state_space_24_b200 as ssm
     lib = ssm.capi()
-    expect = {(0, "scan"): 1, (1, "scan"): 1, (2, "scan"): 3, (3, "scan"): 3, (1, "fwd_ckpt"): 1,
+    expect = {(0, "scan"): 1, (1, "scan"): 1, (2, "scan"): 1, (3, "scan"): 3, (1, "fwd_ckpt"): 1,
               (1, "ordered"): 1, (4, "scan"): 1}
     for (cfg, op), n in expect.items():
         w = bench.workload_info(cfg, op)

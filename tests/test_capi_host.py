@@ -159,10 +159,13 @@ def test_scan_plan(lib):
     # ... never with N < 16, never for a long sequence with few channels
     assert ssm.scan_plan(1, 196, 384, 8)[1] in (1, 2)
     assert ssm.scan_plan(1, 4096, 384, 16)[1] in (1, 2)
-    # the bf16 workloads have few channels: one per lane, several segments
-    for b, L, D in ((8, 1024, 768), (4, 16384, 192)):
-        seg, cpl = ssm.scan_plan(b, L, D, 16, ssm.SSM_BF16, bidirectional=True)
-        assert cpl == 1 and 1 < seg <= (L + 15) // 16
+    assert ssm.scan_plan(2, 1024, 768, 16, bidirectional=True)[1] in (1, 2)
+    # the long-row bf16 workload has few channels and a long row: one per
+    # lane, several segments; the hi-res one splits each channel over four
+    # threads in one pass
+    seg, cpl = ssm.scan_plan(4, 16384, 192, 16, ssm.SSM_BF16, bidirectional=True)
+    assert cpl == 1 and 1 < seg <= (16384 + 15) // 16
+    assert ssm.scan_plan(8, 1024, 768, 16, ssm.SSM_BF16, bidirectional=True) == (1, 0)
     # segments never shorter than 16 steps, never more than the steps
     for L in (1, 15, 16, 17, 100):
         seg, _ = ssm.scan_plan(1, L, 32, 16)
