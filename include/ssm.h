@@ -217,8 +217,9 @@ SSM_API ssm_status bidir_scan_fwd(const ssm_dims *dims, const void *x, const voi
  *                      chunked scan with state hand-off of the Mamba2 page,
  *                      sec. 3.2, run as summary, carry and main passes)
  *   channels_per_lane  (out, may be NULL) 1 or 2: channels one GPU thread owns;
- *                      0: four threads share each channel, a quarter of its
- *                      16 states each (one pass, no segments; N = 16 only)
+ *                      -2 or -4: that many threads share each channel, each
+ *                      holding an equal share of its 16 states (one pass, no
+ *                      segments; N = 16 only)
  * Host-only, makes no CUDA call.  Returns the status the scan entry points
  * give for invalid dims; an empty problem reports 1 segment.
  */
@@ -455,11 +456,12 @@ SSM_API void ssm_debug_ssd_stall(int withhold_chunk, unsigned wait_limit);
  * scans (ssm_scan_fwd, ssm_scan_fwd_state, ssm_scan_fwd_noalloc,
  * bidir_scan_fwd; the pages have no counterpart).  With N = 16 those calls
  * either give each GPU thread one or two whole channels (cutting long
- * sequences into segments), or split each channel's 16 states over four
- * threads in one pass; a cost model fitted to measured B200 timings picks
- * the faster for the sizes (mode 0, the default).  Mode 1 makes calls
- * enqueued after it, in this process, always take the first layout, mode 2
- * the second whenever N = 16; ssm_scan_plan reports what the calls take.
+ * sequences into segments), or split each channel's 16 states over four or
+ * over two threads in one pass; a cost model fitted to measured B200
+ * timings picks the fastest for the sizes (mode 0, the default).  Mode 1
+ * makes calls enqueued after it, in this process, always take the first
+ * layout, mode 2 four threads per channel and mode 3 two whenever N = 16;
+ * ssm_scan_plan reports what the calls take.
  * The two layouts sum the readout in different orders, so results agree to
  * rounding, not bit for bit.  Returns SSM_ERR_INVALID_ARG for another mode.
  * Process-wide and not synchronised with calls on other threads: for tests.

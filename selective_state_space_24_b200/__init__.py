@@ -613,7 +613,7 @@ def ssd_chunk_fwd(x, delta, A, B, C, *, chunk=64, delta_bias=None, delta_softplu
     return out
 
 
-MAPPING_AUTO, MAPPING_WHOLE_CHANNELS, MAPPING_SPLIT_STATES = 0, 1, 2
+MAPPING_AUTO, MAPPING_WHOLE_CHANNELS, MAPPING_SPLIT_STATES, MAPPING_SPLIT_STATES_2 = 0, 1, 2, 3
 
 
 class s6_mapping:
@@ -635,7 +635,7 @@ class s6_mapping:
 
 def scan_plan(batch, seqlen, dim, dstate, dtype=SSM_F32, bidirectional=False):
     """(segments, channels_per_lane) the library uses for an S6 problem;
-    channels_per_lane 0 means four threads share each channel."""
+    channels_per_lane -2 or -4 means that many threads share each channel."""
     lib = capi()
     dims = ssm_dims(batch, seqlen, dim, dstate, dtype)
     seg, cpl = _int(0), _int(0)

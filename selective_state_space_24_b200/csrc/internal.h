@@ -60,8 +60,8 @@ struct S6Args {
     const unsigned char *mask;   // (Bsz, L) by position, 0 = bypass the token, or nullptr
     int conv;                    // 1: x is the conv input x_in, each direction convolves it
     int ckpt;                    // 1: each direction also writes its checkpoints (DirArgs::ckpt)
-    int split;                   // 1: four threads per channel (s6_split.cu); needs N == 16, S == 1,
-                                 // and none of order / mask / conv / ckpt
+    int split;                   // 2 or 4: that many threads per channel (s6_split.cu); needs
+                                 // N == 16, S == 1, and none of order / mask / conv / ckpt
 };
 
 struct S6Plan {
@@ -77,13 +77,15 @@ S6Plan plan_s6(int64_t Bsz, int64_t L, int64_t D, int64_t N, int ndir, int dtype
 
 cudaError_t launch_s6(const S6Args &a, cudaStream_t stream);
 
-// The four-threads-per-channel kernel: whether a plain call (no order,
-// mask, conv or checkpoints) of these sizes takes it, and its launcher.
-// It needs no workspace beyond the bidirectional bf16 stash of plan_s6.
-bool split_eligible(int64_t Bsz, int64_t L, int64_t D, int64_t N, int ndir);
+// The kernel that splits each channel's states over two or four threads:
+// how many threads per channel a plain call (no order, mask, conv or
+// checkpoints) of these sizes takes (0: the one-or-two-channels-per-thread
+// kernels), and its launcher.  It needs no workspace beyond the
+// bidirectional bf16 stash of plan_s6.
+int split_threads(int64_t Bsz, int64_t L, int64_t D, int64_t N, int ndir);
 cudaError_t launch_s6_split(const S6Args &a, cudaStream_t stream);
-// Test setting (process-wide): 0 the cost model decides, 1 never this
-// kernel, 2 this kernel whenever it supports the call.
+// Test setting (process-wide): 0 the cost model decides, 1 never the split
+// layouts, 2 four threads per channel, 3 two, whenever supported.
 void split_mode_set(int mode);
 
 // The S6 kernel parts (s6_part_*.cu): one element type and variant each,

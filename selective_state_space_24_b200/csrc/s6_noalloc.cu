@@ -95,7 +95,7 @@ extern "C" SSM_API ssm_status ssm_scan_fwd_noalloc(const ssm_dims *dims, const v
     const int dt = dims->dtype == SSM_F32 ? 0 : 1;
     // the kernel ssm_scan_fwd takes for these sizes; the four-threads-per-
     // channel one needs no scratch (one pass, single direction)
-    const bool split = ssm::split_eligible(dims->batch, dims->seqlen, dims->dim, dims->dstate, 1);
+    const int split = ssm::split_threads(dims->batch, dims->seqlen, dims->dim, dims->dstate, 1);
     ssm::S6Plan plan = ssm::plan_s6(dims->batch, dims->seqlen, dims->dim, dims->dstate, 1, dt);
     if (split) {
         plan.S = 1;
@@ -126,7 +126,7 @@ extern "C" SSM_API ssm_status ssm_scan_fwd_noalloc(const ssm_dims *dims, const v
     a.delta = delta;
     a.dir[0] = ssm::DirArgs{delta_bias, A, B, C, D, z, last_state};
     a.out = out;
-    a.split = split ? 1 : 0;
+    a.split = split;
     if (a.S > 1) {
         char *w = static_cast<char *>(scratch);
         a.carry_h = reinterpret_cast<float *>(w + plan.carry_h_off);

@@ -42,9 +42,7 @@
 namespace ssm {
 namespace {
 
-constexpr int kQ = 4;                  // threads per channel (a quarter of the 16 states each)
-constexpr int kG = 4;                  // steps per group: thread q does step q's scalar work
-constexpr int kChW = 32 / kQ;          // channels per warp
+constexpr int kG = 4;                  // steps per group
 constexpr int kStages = 4;             // groups in the copy ring (a power of two)
 // CTAs (warp pairs) per SM the registers are sized for, and whether the
 // copies and stores carry L2 eviction priorities.  Measured with this
@@ -59,31 +57,52 @@ constexpr int kStages = 4;             // groups in the copy ring (a power of tw
 #ifndef SSM_S6_SPLIT_HINTS
 #define SSM_S6_SPLIT_HINTS 0
 #endif
-constexpr int kMinBlocks = SSM_S6_SPLIT_MINB;
-static_assert(kG == kQ, "each of a channel's threads takes one step of a group");
+#ifndef SSM_S6_SPLIT_MINB2
+#define SSM_S6_SPLIT_MINB2 10
+#endif
+// CTAs per SM by threads per channel (two threads per channel hold 8
+// states each and need more registers)
+template <int Q> constexpr int min_blocks() { return Q == 2 ? SSM_S6_SPLIT_MINB2 : SSM_S6_SPLIT_MINB; }
 static_assert((kStages & (kStages - 1)) == 0, "ring index by mask");
-// When the plain calls take this kernel (split_eligible).  The one-thread-
-// per-channel kernels give a warp 64 channels (two a thread) and run one step
-// in about 1000 cycles; with fewer than SSM_S6_SPLIT_MAX_WARPS1 warps (under
-// two per SM sub-partition) they are latency-bound, or cut the sequence into
-// segments and scan it twice.  This kernel's warps take a step in a few
-// hundred cycles but issue about half as many instructions again per
-// element, so past that occupancy the other kernels win.  Below it a cost
-// model, fitted to one-B200 timings of both kernels over 47 sizes (batch
-// 1 - 128, L 197 - 16384, D 192 - 1536, both dtypes, one and two
-// directions; it picks the faster in all 47), decides (microseconds;
-// E = elements B L D N x directions):
-//   this kernel    max(Tl, Tt) + 0.3 min(Tl, Tt) + 6 (9 for a pair),
-//                  Tl = L x 0.067 (0.082), Tt = E / 2.15e6 (1.9e6);
-//   the others     22 + 0.01 L + E / 1.333e6.
+// Which layout the plain calls take (split_threads).  The one-thread-per-
+// channel kernels give a warp 64 channels (two a thread); with fewer than
+// SSM_S6_SPLIT_MAX_WARPS1 warps (under two per SM sub-partition) they are
+// latency-bound, or cut the sequence into segments and scan it twice.  Two
+// threads per channel (8 states each) issue fewer instructions per element
+// than four and run 4x the warps of the one-channel kernel: measured on
+// B200 it is the fastest layout for every problem that gives the
+// one-channel kernel at least that many warps (Vim-Small bidirectional
+// fp32: 134 against 140 us; B 128: 239 against 261).  Below it a cost model
+// fitted to the timings of all three layouts over 62 sizes (batch 1 - 256,
+// L 196 - 16384, D 192 - 1536, both dtypes, one and two directions; it
+// picks the fastest in 61, the miss costs 1.9%) decides, in microseconds,
+// with E = elements B L D N x directions and (single direction / pair):
+//   q threads per channel   max(Tl, Tt) + 0.3 min(Tl, Tt) + c,
+//        q = 4: Tl = L x 0.067 / 0.082, Tt = E / 2.15e6 / 1.9e6, c = 6 / 9;
+//        q = 2: Tl = L x 0.087 / 0.105, Tt = E / 2.9e6 / 2.65e6, c = 11 / 12;
+//   the one-channel kernels 22 + 0.01 L + E / 1.333e6.
 #ifndef SSM_S6_SPLIT_MAX_WARPS1
 #define SSM_S6_SPLIT_MAX_WARPS1 1024
 #endif
 
+#ifndef SSM_S6_SPLIT_SKEW
+#define SSM_S6_SPLIT_SKEW 1
+#endif
+// Smallest stride >= bytes (16-byte steps) whose word offset mod 32 is an
+// odd multiple of w (w = 4, 8 or 16 words).
+constexpr int skew_stride(int bytes, int w)
+{
+    int s = bytes;
+    while (!(((s / 4) % 32) % w == 0 && (((s / 4) % 32) / w) % 2 == 1))
+        s += 16;
+    return s;
+}
+
 // One step's slot in the ring: x, delta, (z) for the warp's 8 channels,
 // then the B and C rows, then (bidirectional) the partner's 8 parked fp32
 // outputs of that step, which are copied only once the pair has met.
-template <typename T, bool GATE, bool BIDIR> struct Slot {
+template <typename T, bool GATE, bool BIDIR, int Q> struct Slot {
+    static constexpr int kChW = 32 / Q;                     // channels per warp
     static constexpr int kRow = kChW * (int)sizeof(T);
     static constexpr int kBC = 16 * (int)sizeof(T);
     static constexpr int kX = 0, kDl = kRow, kZ = 2 * kRow;
@@ -93,12 +112,19 @@ template <typename T, bool GATE, bool BIDIR> struct Slot {
     static constexpr int kPieces = kBytes / 16;             // 16-byte copies per step
     static constexpr int kGroupPieces = kG * kPieces;
     static constexpr int kPerLane = (kGroupPieces + 31) / 32;
-    static constexpr int kGroupBytes = kG * kBytes;
+    // Step slots are kStride bytes apart: the Q threads of a channel read
+    // the x, delta, z (and parked) values of Q consecutive steps at once, so
+    // consecutive slots are skewed by an odd multiple of one step's widest
+    // channel block in banks (kRow / 4 words, or kChW for the fp32 parked
+    // row) -- a stride that is a multiple of 128 bytes would put every one
+    // of those steps on the same banks.
+    static constexpr int kStride = SSM_S6_SPLIT_SKEW ? skew_stride(kBytes, BIDIR ? kChW : kRow / 4) : kBytes;
+    static constexpr int kGroupBytes = kG * kStride;
     static_assert(kBytes % 16 == 0 && kB % 16 == 0 && kRow % 16 == 0, "16-byte pieces");
 };
 
-template <typename T, bool GATE, bool BIDIR> struct WarpSmem {
-    __align__(16) char ring[kStages][Slot<T, GATE, BIDIR>::kGroupBytes];
+template <typename T, bool GATE, bool BIDIR, int Q> struct WarpSmem {
+    __align__(16) char ring[kStages][Slot<T, GATE, BIDIR, Q>::kGroupBytes];
 };
 
 __device__ __forceinline__ uint64_t policy_evict_last()
@@ -182,14 +208,19 @@ template <> __device__ __forceinline__ float4 lds4<__nv_bfloat16>(const char *p)
 enum Mode { kPlain, kPark, kMixed, kAdd };
 template <Mode M> using ModeTag = std::integral_constant<Mode, M>;
 
-template <typename T, bool BIDIR, bool GATE, bool SOFTPLUS>
-__global__ void __launch_bounds__(64, kMinBlocks) s6_split_kernel(const S6Args a)
+template <typename T, int Q, bool BIDIR, bool GATE, bool SOFTPLUS>
+__global__ void __launch_bounds__(64, min_blocks<Q>()) s6_split_kernel(const S6Args a)
 {
-    using S = Slot<T, GATE, BIDIR>;
-    __shared__ WarpSmem<T, GATE, BIDIR> smem[2];
+    static_assert(Q == 2 || Q == 4, "two or four threads per channel");
+    using S = Slot<T, GATE, BIDIR, Q>;
+    constexpr int kChW = S::kChW;
+    constexpr int NQ = 16 / Q;          // states per thread
+    constexpr int NP = NQ / 2;          // state pairs per thread
+    constexpr int SPL = kG / Q;         // steps of a group whose scalars a thread computes
+    __shared__ WarpSmem<T, GATE, BIDIR, Q> smem[2];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    WarpSmem<T, GATE, BIDIR> &sm = smem[warp];
-    const int g = lane >> 2, q = lane & 3;
+    WarpSmem<T, GATE, BIDIR, Q> &sm = smem[warp];
+    const int g = lane / Q, q = lane % Q;
     const int dsel = BIDIR ? warp : 0;
     const int d0 = (BIDIR ? (int)blockIdx.x : (int)blockIdx.x * 2 + warp) * kChW;   // the warp's first channel
     const int b = blockIdx.y;
@@ -201,19 +232,20 @@ __global__ void __launch_bounds__(64, kMinBlocks) s6_split_kernel(const S6Args a
     const bool rev = BIDIR ? dsel == 1 : a.reverse != 0;
     const DirArgs &P = a.dir[dsel];
 
-    // this thread's states [4q, 4q + 4) as two pairs, A scaled by log2(e)
-    float2 A2[2], h2[2];
-    {
+    // this thread's states [NQ q, NQ q + NQ) as pairs, A scaled by log2(e)
+    float2 A2[NP], h2[NP];
+#pragma unroll
+    for (int v = 0; v < NQ / 4; v++) {
         float4 av = make_float4(0.f, 0.f, 0.f, 0.f), hv = av;
         if (active) {
-            av = *reinterpret_cast<const float4 *>(P.A + (size_t)d * 16 + 4 * q);
+            av = *reinterpret_cast<const float4 *>(P.A + (size_t)d * 16 + NQ * q + 4 * v);
             if (P.init)
-                hv = *reinterpret_cast<const float4 *>(P.init + ((size_t)b * D + d) * 16 + 4 * q);
+                hv = *reinterpret_cast<const float4 *>(P.init + ((size_t)b * D + d) * 16 + NQ * q + 4 * v);
         }
-        A2[0] = make_float2(av.x * kLog2e, av.y * kLog2e);
-        A2[1] = make_float2(av.z * kLog2e, av.w * kLog2e);
-        h2[0] = make_float2(hv.x, hv.y);
-        h2[1] = make_float2(hv.z, hv.w);
+        A2[2 * v] = make_float2(av.x * kLog2e, av.y * kLog2e);
+        A2[2 * v + 1] = make_float2(av.z * kLog2e, av.w * kLog2e);
+        h2[2 * v] = make_float2(hv.x, hv.y);
+        h2[2 * v + 1] = make_float2(hv.z, hv.w);
     }
     const float bias = (active && P.bias) ? P.bias[d] : 0.f;
     const float Dd = (active && P.D) ? P.D[d] : 0.f;
@@ -230,9 +262,9 @@ __global__ void __launch_bounds__(64, kMinBlocks) s6_split_kernel(const S6Args a
     const T *Bm = static_cast<const T *>(P.B), *Cm = static_cast<const T *>(P.C);
     const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(&sm.ring[0][0]);
     const char *safe = static_cast<const char *>(a.x);
-    // (piece p of a group lands at byte 16 p of the group's slots: step
-    // p / kPieces, byte 16 (p % kPieces) of that step's slot)
+    // (piece p of a group is byte 16 (p % kPieces) of step p / kPieces's slot)
     const char *cur[S::kPerLane];     // source row of the next group to issue
+    uint32_t dst[S::kPerLane];        // its offset in a group's slots
     int gstep[S::kPerLane];           // bytes from one group's rows to the next's
     bool pok[S::kPerLane];            // the piece holds channels below D
     bool xd[S::kPerLane];             // an x / delta piece: L2 policy by half
@@ -245,6 +277,7 @@ __global__ void __launch_bounds__(64, kMinBlocks) s6_split_kernel(const S6Args a
         const int pp = exists ? p : 0;
         const int s = pp / S::kPieces, off = (pp % S::kPieces) * 16;
         const int t0 = rev ? L - 1 - s : s;
+        dst[j] = (uint32_t)(s * S::kStride + off);
         const char *base;
         long long row;
         bool ok = exists;
@@ -283,19 +316,19 @@ __global__ void __launch_bounds__(64, kMinBlocks) s6_split_kernel(const S6Args a
     int next_gi = 0;   // groups [0, next_gi) have been copied (next_gi <= G)
     auto issue = [&](int gi) {
         if (gi < G) {
-            const uint32_t sb = ring_s + (uint32_t)((gi & (kStages - 1)) * S::kGroupBytes) + 16 * lane;
+            const uint32_t sb = ring_s + (uint32_t)((gi & (kStages - 1)) * S::kGroupBytes);
             const uint64_t pxd = (BIDIR && gi * kG < M) ? pol_last : pol_first;
             if ((gi + 1) * kG <= L) {
 #pragma unroll
                 for (int j = 0; j < S::kPerLane; j++)
                     if (lane + 32 * j < S::kGroupPieces && (!BIDIR || !pk[j] || parked_live))
-                        cp16(sb + 512 * j, cur[j], pok[j] ? 16 : 0, xd[j] ? pxd : pfix[j]);
+                        cp16(sb + dst[j], cur[j], pok[j] ? 16 : 0, xd[j] ? pxd : pfix[j]);
             } else {   // the last group is short: steps past L are zero-filled, not read
 #pragma unroll
                 for (int j = 0; j < S::kPerLane; j++)
                     if (lane + 32 * j < S::kGroupPieces && (!BIDIR || !pk[j] || parked_live)) {
                         const bool in = pok[j] && gi * kG + (lane + 32 * j) / S::kPieces < L;
-                        cp16(sb + 512 * j, in ? cur[j] : safe, in ? 16 : 0, xd[j] ? pxd : pfix[j]);
+                        cp16(sb + dst[j], in ? cur[j] : safe, in ? 16 : 0, xd[j] ? pxd : pfix[j]);
                     }
             }
 #pragma unroll
@@ -310,13 +343,13 @@ __global__ void __launch_bounds__(64, kMinBlocks) s6_split_kernel(const S6Args a
     // group counting of the waits stays exact)
     auto catch_up = [&](int g0) {
         for (int gj = g0; gj < next_gi && gj < G; gj++) {
-            const uint32_t sb = ring_s + (uint32_t)((gj & (kStages - 1)) * S::kGroupBytes) + 16 * lane;
+            const uint32_t sb = ring_s + (uint32_t)((gj & (kStages - 1)) * S::kGroupBytes);
 #pragma unroll
             for (int j = 0; j < S::kPerLane; j++)
                 if (lane + 32 * j < S::kGroupPieces && pk[j]) {
                     const bool in = pok[j] && gj * kG + (lane + 32 * j) / S::kPieces < L;
                     const char *src = cur[j] - (long long)(next_gi - gj) * gstep[j];
-                    cp16(sb + 512 * j, in ? src : safe, in ? 16 : 0, pfix[j]);
+                    cp16(sb + dst[j], in ? src : safe, in ? 16 : 0, pfix[j]);
                 }
         }
         cp_commit();
@@ -324,11 +357,13 @@ __global__ void __launch_bounds__(64, kMinBlocks) s6_split_kernel(const S6Args a
         __syncwarp();
     };
 
-    // --- outputs: element index of this thread's step of the current group
+    // --- outputs: element index of this thread's first step (q) of the
+    // current group; its step q + Q r is r Q rows further in scan order
     T *out = static_cast<T *>(a.out);
     float *stash = a.stash;
     long long oi = ((long long)b * L + (rev ? L - 1 - q : q)) * D + d;
     const int ostep = (rev ? -1 : 1) * kG * D;
+    const int rstep = (rev ? -1 : 1) * Q * D;
 
     auto group = [&](int gi, auto mode_tag) {
         constexpr Mode MODE = decltype(mode_tag)::value;
@@ -336,64 +371,102 @@ __global__ void __launch_bounds__(64, kMinBlocks) s6_split_kernel(const S6Args a
         cp_wait<kStages - 1>();
         __syncwarp();
         const char *gs = &sm.ring[gi & (kStages - 1)][0];
-        const int i = gi * kG + q;   // this thread's step
-        const bool valid = i < L;
-        // A: step q's scalars
-        const char *sq = gs + q * S::kBytes + g * (int)sizeof(T);
-        const float xv = lds1<T>(sq + S::kX);
-        float dt = lds1<T>(sq + S::kDl) + bias;
-        if (SOFTPLUS)
-            dt = softplus_f(dt);
-        dt = valid ? dt : 0.f;   // past L: exp(0) = 1 and no input, the state passes through
-        const float dtx = dt * xv;
-        const float gate = GATE ? silu_f<T>(lds1<T>(sq + S::kZ)) : 1.f;
-        const float dxv = Dd * xv;
+        // A: the scalars of this thread's steps q + Q r of the group
+        float dt[SPL], dtx[SPL], gate[SPL], dxv[SPL];
+        bool valid[SPL];
+#pragma unroll
+        for (int r = 0; r < SPL; r++) {
+            const int i = gi * kG + q + Q * r;
+            valid[r] = i < L;
+            const char *sq = gs + (q + Q * r) * S::kStride + g * (int)sizeof(T);
+            const float xv = lds1<T>(sq + S::kX);
+            float t = lds1<T>(sq + S::kDl) + bias;
+            if (SOFTPLUS)
+                t = softplus_f(t);
+            dt[r] = valid[r] ? t : 0.f;   // past L: exp(0) = 1 and no input, the state passes through
+            dtx[r] = dt[r] * xv;
+            gate[r] = GATE ? silu_f<T>(lds1<T>(sq + S::kZ)) : 1.f;
+            dxv[r] = Dd * xv;
+        }
         // B: the four steps' state updates and shares of C . h (step s's dt
-        // and dt x come from thread s of the channel)
+        // and dt x come from thread s % Q of the channel)
         float part[kG];
 #pragma unroll
         for (int s = 0; s < kG; s++) {
-            const float dts = __shfl_sync(0xffffffffu, dt, (lane & ~3) | s);
-            const float dtxs = __shfl_sync(0xffffffffu, dtx, (lane & ~3) | s);
-            const char *ss = gs + s * S::kBytes + q * 4 * (int)sizeof(T);
-            const float4 B4 = lds4<T>(ss + S::kB), C4 = lds4<T>(ss + S::kC);
+            const int src = (lane & ~(Q - 1)) | (s % Q);
+            const float dts = __shfl_sync(0xffffffffu, dt[s / Q], src);
+            const float dtxs = __shfl_sync(0xffffffffu, dtx[s / Q], src);
+            const char *ss = gs + s * S::kStride + q * NQ * (int)sizeof(T);
             const float2 dt2 = make_float2(dts, dts), dtx2 = make_float2(dtxs, dtxs);
-            float2 v = __fmul2_rn(dt2, A2[0]);
-            float2 e = make_float2(ex2_mufu(v.x), ex2_mufu(v.y));
-            h2[0] = __ffma2_rn(e, h2[0], __fmul2_rn(dtx2, make_float2(B4.x, B4.y)));
-            v = __fmul2_rn(dt2, A2[1]);
-            e = make_float2(ex2_mufu(v.x), ex2_mufu(v.y));
-            h2[1] = __ffma2_rn(e, h2[1], __fmul2_rn(dtx2, make_float2(B4.z, B4.w)));
-            float2 y2 = __fmul2_rn(make_float2(C4.x, C4.y), h2[0]);
-            y2 = __ffma2_rn(make_float2(C4.z, C4.w), h2[1], y2);
+            float2 y2 = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int v = 0; v < NQ / 4; v++) {
+                const float4 B4 = lds4<T>(ss + S::kB + 4 * v * (int)sizeof(T));
+                const float4 C4 = lds4<T>(ss + S::kC + 4 * v * (int)sizeof(T));
+                float2 w = __fmul2_rn(dt2, A2[2 * v]);
+                float2 e = make_float2(ex2_mufu(w.x), ex2_mufu(w.y));
+                h2[2 * v] = __ffma2_rn(e, h2[2 * v], __fmul2_rn(dtx2, make_float2(B4.x, B4.y)));
+                w = __fmul2_rn(dt2, A2[2 * v + 1]);
+                e = make_float2(ex2_mufu(w.x), ex2_mufu(w.y));
+                h2[2 * v + 1] = __ffma2_rn(e, h2[2 * v + 1], __fmul2_rn(dtx2, make_float2(B4.z, B4.w)));
+                y2 = __ffma2_rn(make_float2(C4.x, C4.y), h2[2 * v], y2);
+                y2 = __ffma2_rn(make_float2(C4.z, C4.w), h2[2 * v + 1], y2);
+            }
             part[s] = y2.x + y2.y;
         }
-        // C: sum the four threads' shares so that thread q holds step q's:
-        // exchange halves across q bit 1 (steps {0, 1} vs {2, 3}), then
-        // across q bit 0
-        const bool hi1 = (q & 2) != 0, hi0 = (q & 1) != 0;
-        float ka = hi1 ? part[2] : part[0], kb = hi1 ? part[3] : part[1];
-        ka += __shfl_xor_sync(0xffffffffu, hi1 ? part[0] : part[2], 2);
-        kb += __shfl_xor_sync(0xffffffffu, hi1 ? part[1] : part[3], 2);
-        const float ysum = (hi0 ? kb : ka) + __shfl_xor_sync(0xffffffffu, hi0 ? ka : kb, 1);
-        const float y = (ysum + dxv) * gate;
-        const bool st = active && valid;
-        if (MODE == kPlain) {
-            if (st)
-                st_pol(out + oi, y, pol_first);
-        } else if (MODE == kPark) {
-            if (st)
-                st_pol(stash + oi, y, pol_last);
-        } else if (MODE == kMixed) {
-            if (st && i < M)
-                st_pol(stash + oi, y, pol_last);
-            pair_barrier();   // both warps' parked halves are written
-            if (st && i >= M)
-                st_pol(out + oi, y + __ldcg(stash + oi), pol_first);
+        // C: sum the channel's Q shares of each step so that thread q holds
+        // those of its steps q + Q r
+        float ysum[SPL];
+        if (Q == 4) {
+            // exchange halves across q bit 1 (steps {0, 1} vs {2, 3}), then
+            // across q bit 0
+            const bool hi1 = (q & 2) != 0, hi0 = (q & 1) != 0;
+            float ka = hi1 ? part[2] : part[0], kb = hi1 ? part[3] : part[1];
+            ka += __shfl_xor_sync(0xffffffffu, hi1 ? part[0] : part[2], 2);
+            kb += __shfl_xor_sync(0xffffffffu, hi1 ? part[1] : part[3], 2);
+            ysum[0] = (hi0 ? kb : ka) + __shfl_xor_sync(0xffffffffu, hi0 ? ka : kb, 1);
         } else {
-            if (st)   // the partner's parked value, copied with this group's rows
-                st_pol(out + oi, y + *reinterpret_cast<const float *>(gs + q * S::kBytes + S::kPk + 4 * g),
-                       pol_first);
+            // thread q keeps steps q and q + 2 and sends the other two
+            const bool hi = q != 0;
+#pragma unroll
+            for (int r = 0; r < SPL; r++)
+                ysum[r] = (hi ? part[2 * r + 1] : part[2 * r]) +
+                          __shfl_xor_sync(0xffffffffu, hi ? part[2 * r] : part[2 * r + 1], 1);
+        }
+        float y[SPL];
+        bool st[SPL];
+#pragma unroll
+        for (int r = 0; r < SPL; r++) {
+            y[r] = (ysum[r] + dxv[r]) * gate[r];
+            st[r] = active && valid[r];
+        }
+        if (MODE == kPlain) {
+#pragma unroll
+            for (int r = 0; r < SPL; r++)
+                if (st[r])
+                    st_pol(out + oi + r * rstep, y[r], pol_first);
+        } else if (MODE == kPark) {
+#pragma unroll
+            for (int r = 0; r < SPL; r++)
+                if (st[r])
+                    st_pol(stash + oi + r * rstep, y[r], pol_last);
+        } else if (MODE == kMixed) {
+#pragma unroll
+            for (int r = 0; r < SPL; r++)
+                if (st[r] && gi * kG + q + Q * r < M)
+                    st_pol(stash + oi + r * rstep, y[r], pol_last);
+            pair_barrier();   // both warps' parked halves are written
+#pragma unroll
+            for (int r = 0; r < SPL; r++)
+                if (st[r] && gi * kG + q + Q * r >= M)
+                    st_pol(out + oi + r * rstep, y[r] + __ldcg(stash + oi + r * rstep), pol_first);
+        } else {
+#pragma unroll
+            for (int r = 0; r < SPL; r++)
+                if (st[r])   // the partner's parked value, copied with this group's rows
+                    st_pol(out + oi + r * rstep,
+                           y[r] + *reinterpret_cast<const float *>(gs + (q + Q * r) * S::kStride + S::kPk + 4 * g),
+                           pol_first);
         }
         oi += ostep;
         __syncwarp();   // every thread is done with this group's slots and tables
@@ -421,22 +494,32 @@ __global__ void __launch_bounds__(64, kMinBlocks) s6_split_kernel(const S6Args a
     }
     cp_wait<0>();
 
-    if (active && P.last_state)
-        *reinterpret_cast<float4 *>(P.last_state + ((size_t)b * D + d) * 16 + 4 * q) =
-            make_float4(h2[0].x, h2[0].y, h2[1].x, h2[1].y);
+    if (active && P.last_state) {
+#pragma unroll
+        for (int v = 0; v < NQ / 4; v++)
+            *reinterpret_cast<float4 *>(P.last_state + ((size_t)b * D + d) * 16 + NQ * q + 4 * v) =
+                make_float4(h2[2 * v].x, h2[2 * v].y, h2[2 * v + 1].x, h2[2 * v + 1].y);
+    }
+}
+
+template <typename T, int Q, bool GATE, bool SOFTPLUS>
+cudaError_t launch_q(const S6Args &a, cudaStream_t st)
+{
+    constexpr int kChW = 32 / Q;
+    if (a.ndir == 2) {
+        const dim3 grid((unsigned)((a.D + kChW - 1) / kChW), (unsigned)a.Bsz);
+        s6_split_kernel<T, Q, true, GATE, SOFTPLUS><<<grid, 64, 0, st>>>(a);
+    } else {
+        const dim3 grid((unsigned)((a.D + 2 * kChW - 1) / (2 * kChW)), (unsigned)a.Bsz);
+        s6_split_kernel<T, Q, false, GATE, SOFTPLUS><<<grid, 64, 0, st>>>(a);
+    }
+    return cudaGetLastError();
 }
 
 template <typename T, bool GATE, bool SOFTPLUS>
 cudaError_t launch_t(const S6Args &a, cudaStream_t st)
 {
-    if (a.ndir == 2) {
-        const dim3 grid((unsigned)((a.D + kChW - 1) / kChW), (unsigned)a.Bsz);
-        s6_split_kernel<T, true, GATE, SOFTPLUS><<<grid, 64, 0, st>>>(a);
-    } else {
-        const dim3 grid((unsigned)((a.D + 2 * kChW - 1) / (2 * kChW)), (unsigned)a.Bsz);
-        s6_split_kernel<T, false, GATE, SOFTPLUS><<<grid, 64, 0, st>>>(a);
-    }
-    return cudaGetLastError();
+    return a.split == 2 ? launch_q<T, 2, GATE, SOFTPLUS>(a, st) : launch_q<T, 4, GATE, SOFTPLUS>(a, st);
 }
 
 template <typename T>
@@ -450,24 +533,32 @@ cudaError_t launch_flags(const S6Args &a, cudaStream_t st)
 
 }  // namespace
 
-std::atomic<int> g_split_mode{0};   // 0 cost model, 1 never, 2 whenever supported
+// 0 cost model, 1 never these layouts, 2 four threads per channel whenever
+// supported, 3 two threads per channel whenever supported
+std::atomic<int> g_split_mode{0};
 
-bool split_eligible(int64_t Bsz, int64_t L, int64_t D, int64_t N, int ndir)
+int split_threads(int64_t Bsz, int64_t L, int64_t D, int64_t N, int ndir)
 {
     if (N != 16 || L <= 0 || Bsz <= 0 || D <= 0 || Bsz > 65535)
-        return false;
+        return 0;
     const int mode = g_split_mode.load(std::memory_order_relaxed);
     if (mode != 0)
-        return mode == 2;
+        return mode == 2 ? 4 : mode == 3 ? 2 : 0;
     const int64_t warps1 = (int64_t)ndir * Bsz * ((D + 63) / 64);   // one thread, two channels
     if (warps1 >= SSM_S6_SPLIT_MAX_WARPS1)
-        return false;
+        return 2;
+    const bool pair = ndir == 2;
     const double E = (double)ndir * Bsz * L * D * 16;
-    const double tl = (double)L * (ndir == 2 ? 0.082 : 0.067);
-    const double tt = E / (ndir == 2 ? 1.9e6 : 2.15e6);
-    const double t_split = (tl > tt ? tl + 0.3 * tt : tt + 0.3 * tl) + (ndir == 2 ? 9.0 : 6.0);
-    const double t_other = 22.0 + 0.01 * (double)L + E / 1.333e6;
-    return t_split < t_other;
+    auto t_split = [&](double lat, double thr, double c) {
+        const double tl = (double)L * lat, tt = E / thr;
+        return (tl > tt ? tl + 0.3 * tt : tt + 0.3 * tl) + c;
+    };
+    const double t4 = t_split(pair ? 0.082 : 0.067, pair ? 1.9e6 : 2.15e6, pair ? 9.0 : 6.0);
+    const double t2 = t_split(pair ? 0.105 : 0.087, pair ? 2.65e6 : 2.9e6, pair ? 12.0 : 11.0);
+    const double t1 = 22.0 + 0.01 * (double)L + E / 1.333e6;
+    if (t1 <= t4 && t1 <= t2)
+        return 0;
+    return t2 < t4 ? 2 : 4;
 }
 
 void split_mode_set(int mode) { g_split_mode.store(mode, std::memory_order_relaxed); }

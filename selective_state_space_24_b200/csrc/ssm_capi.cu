@@ -112,9 +112,11 @@ ssm_status run_s6(const ssm_dims *dims, const void *x, const void *delta, int so
             a.dir[i].ckpt = ckpt[i];
     }
     a.out = out;
-    if (!order && !mask && !conv && !ckpt &&
-        ssm::split_eligible(dims->batch, dims->seqlen, dims->dim, dims->dstate, ndir)) {
-        a.split = 1;   // one pass, four threads per channel
+    const int q = (order || mask || conv || ckpt)
+                      ? 0
+                      : ssm::split_threads(dims->batch, dims->seqlen, dims->dim, dims->dstate, ndir);
+    if (q) {
+        a.split = q;   // one pass, q threads per channel
         a.S = 1;
         a.T = a.L;
     }
@@ -159,9 +161,10 @@ ssm_status ssm_scan_plan(const ssm_dims *dims, int bidirectional, int *segments,
     if (!empty_s6(dims)) {
         plan = ssm::plan_s6(dims->batch, dims->seqlen, dims->dim, dims->dstate, ndir,
                             dims->dtype == SSM_F32 ? 0 : 1);
-        if (ssm::split_eligible(dims->batch, dims->seqlen, dims->dim, dims->dstate, ndir)) {
-            plan.S = 1;     // one pass
-            plan.cpl = 0;   // four threads share each channel
+        const int q = ssm::split_threads(dims->batch, dims->seqlen, dims->dim, dims->dstate, ndir);
+        if (q) {
+            plan.S = 1;      // one pass
+            plan.cpl = -q;   // q threads share each channel
         }
     }
     if (segments)
@@ -700,7 +703,7 @@ void ssm_debug_ssd_stall(int withhold_chunk, unsigned wait_limit) { ssm::ssd_sta
 
 ssm_status ssm_debug_s6_mapping(int mode)
 {
-    if (mode < 0 || mode > 2)
+    if (mode < 0 || mode > 3)
         return SSM_ERR_INVALID_ARG;
     ssm::split_mode_set(mode);
     return SSM_OK;

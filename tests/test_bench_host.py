@@ -123,4 +123,4 @@ def test_launch_count_follows_the_plan():
         ns = types.SimpleNamespace(info=w, op=op, lib=lib, dims=dims)
         assert bench.DeviceWorkload._launches(ns) == n, (cfg, op)
     # the query leaves the layout choice to the cost model again
-    assert ssm.scan_plan(1, 196, 384, 16) == (1, 0)
+    assert ssm.scan_plan(1, 196, 384, 16) == (1, -4)

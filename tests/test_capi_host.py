@@ -150,12 +150,13 @@ def test_plan_is_deterministic(lib):
 def test_scan_plan(lib):
     """The launch-plan query: segment count and channels per lane for the
     workloads' sizes, the bounds the plan keeps, and its argument checks."""
-    # Vim-Small bidirectional: enough channels for one pass, two per lane
-    assert ssm.scan_plan(64, 197, 768, 16, bidirectional=True) == (1, 2)
-    # fewer channels on a short sequence: four threads per channel, one pass
-    assert ssm.scan_plan(1, 196, 384, 16) == (1, 0)                       # Vim-Tiny
-    assert ssm.scan_plan(16, 197, 768, 16, bidirectional=True) == (1, 0)
-    assert ssm.scan_plan(8, 197, 768, 16, ssm.SSM_BF16) == (1, 0)
+    # Vim-Small bidirectional: two threads per channel, one pass
+    assert ssm.scan_plan(64, 197, 768, 16, bidirectional=True) == (1, -2)
+    # fewer channels on a short sequence: four or two threads per channel, one pass
+    assert ssm.scan_plan(1, 196, 384, 16) == (1, -4)                       # Vim-Tiny
+    assert ssm.scan_plan(16, 197, 768, 16, bidirectional=True) == (1, -2)
+    assert ssm.scan_plan(8, 197, 768, 16, ssm.SSM_BF16) == (1, -4)
+    assert ssm.scan_plan(256, 1024, 768, 16) == (1, -2)
     # ... never with N < 16, never for a long sequence with few channels
     assert ssm.scan_plan(1, 196, 384, 8)[1] in (1, 2)
     assert ssm.scan_plan(1, 4096, 384, 16)[1] in (1, 2)
@@ -165,7 +166,7 @@ def test_scan_plan(lib):
     # threads in one pass
     seg, cpl = ssm.scan_plan(4, 16384, 192, 16, ssm.SSM_BF16, bidirectional=True)
     assert cpl == 1 and 1 < seg <= (16384 + 15) // 16
-    assert ssm.scan_plan(8, 1024, 768, 16, ssm.SSM_BF16, bidirectional=True) == (1, 0)
+    assert ssm.scan_plan(8, 1024, 768, 16, ssm.SSM_BF16, bidirectional=True) == (1, -4)
     # segments never shorter than 16 steps, never more than the steps
     for L in (1, 15, 16, 17, 100):
         seg, _ = ssm.scan_plan(1, L, 32, 16)
@@ -188,13 +189,15 @@ def test_s6_mapping_hook(lib):
     it), refuses other modes, and mode 0 gives the cost model back."""
     try:
         with ssm.s6_mapping(ssm.MAPPING_SPLIT_STATES):
-            assert ssm.scan_plan(64, 197, 768, 16, bidirectional=True) == (1, 0)
-            assert ssm.scan_plan(1, 4096, 384, 16) == (1, 0)
+            assert ssm.scan_plan(64, 197, 768, 16, bidirectional=True) == (1, -4)
+            assert ssm.scan_plan(1, 4096, 384, 16) == (1, -4)
             assert ssm.scan_plan(1, 196, 384, 8)[1] in (1, 2)     # N < 16: never
         with ssm.s6_mapping(ssm.MAPPING_WHOLE_CHANNELS):
             assert ssm.scan_plan(1, 196, 384, 16)[1] in (1, 2)
-        assert ssm.scan_plan(1, 196, 384, 16) == (1, 0)
-        assert lib.ssm_debug_s6_mapping(3) == 1
+        assert ssm.scan_plan(1, 196, 384, 16) == (1, -4)
+        with ssm.s6_mapping(ssm.MAPPING_SPLIT_STATES_2):
+            assert ssm.scan_plan(64, 197, 768, 16, bidirectional=True) == (1, -2)
+        assert lib.ssm_debug_s6_mapping(4) == 1
         assert lib.ssm_debug_s6_mapping(-1) == 1
     finally:
         lib.ssm_debug_s6_mapping(0)

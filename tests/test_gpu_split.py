@@ -1,5 +1,5 @@
-"""GPU parity of the four-threads-per-channel layout of the plain S6 scans
-(s6_split.cu) against the float64 oracle.  The layout is forced with the
+"""GPU parity of the split-state layouts of the plain S6 scans (s6_split.cu:
+four or two threads per channel) against the float64 oracle.  The layout is forced with the
 library's test hook, so shapes the cost model would give to the other
 layout are covered too: sequence lengths whose last 4-step group is short,
 the bidirectional exchange point falling inside a group or on its edge, a
@@ -23,25 +23,31 @@ def _lib(cuda_device):
     ssm.load()
 
 
-@pytest.fixture(autouse=True)
-def _split_layout():
-    with ssm.s6_mapping(ssm.MAPPING_SPLIT_STATES):
-        yield
+# every test runs with four and with two threads per channel
+@pytest.fixture(autouse=True, params=[ssm.MAPPING_SPLIT_STATES, ssm.MAPPING_SPLIT_STATES_2], ids=["q4", "q2"])
+def _split_layout(request):
+    with ssm.s6_mapping(request.param):
+        yield request.param
 
 
-def _plan_is_split(inp, bidir):
+@pytest.fixture
+def threads(_split_layout):
+    return 4 if _split_layout == ssm.MAPPING_SPLIT_STATES else 2
+
+
+def _plan_is_split(inp, bidir, threads):
     code = ssm.SSM_F32 if inp.dtype == "f32" else ssm.SSM_BF16
-    return ssm.scan_plan(inp.batch, inp.seqlen, inp.dim, 16, code, bidirectional=bidir) == (1, 0)
+    return ssm.scan_plan(inp.batch, inp.seqlen, inp.dim, 16, code, bidirectional=bidir) == (1, -threads)
 
 
 # L % 4 covers every length of the last group; for the pair, ceil(L / 2) and
 # floor(L / 2) put the exchange point at every offset inside a group
 @pytest.mark.parametrize("L", [1, 2, 3, 4, 5, 6, 7, 8, 9, 13, 64, 197])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_bidir_every_exchange_offset(L, dtype):
+def test_bidir_every_exchange_offset(L, dtype, threads):
     inp = ssm_gen.make_s6_inputs(2, L, 24, 16, dtype=dtype, bidir=True, seed=100 + L, random_A=True,
                                  random_D=True)
-    assert _plan_is_split(inp, True)
+    assert _plan_is_split(inp, True, threads)
     out, lf, lb = run_bidir(inp, last_state=True)
     ref, rlf, rlb = oracle.bidir(inp, nthreads=NTHREADS)
     tol = TOL[dtype]
@@ -53,9 +59,9 @@ def test_bidir_every_exchange_offset(L, dtype):
 @pytest.mark.parametrize("L", [1, 3, 4, 5, 31, 197])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("reverse", [False, True])
-def test_single_direction_ragged(L, dtype, reverse):
+def test_single_direction_ragged(L, dtype, reverse, threads):
     inp = ssm_gen.make_s6_inputs(3, L, 40, 16, dtype=dtype, seed=200 + L, random_A=True, random_D=True)
-    assert _plan_is_split(inp, False)
+    assert _plan_is_split(inp, False, threads)
     out, st = run_s6(inp, reverse=reverse)
     ref, rst = oracle.s6(inp, reverse=reverse, nthreads=NTHREADS)
     tol = TOL[dtype]
@@ -65,8 +71,9 @@ def test_single_direction_ragged(L, dtype, reverse):
 
 @pytest.mark.parametrize("bidir", [False, True])
 def test_warp_partly_inside_d(bidir):
-    """fp32 with D = 12: the second block of 8 channels holds 4, so its copies
-    of x / delta / z are half zero-filled and half its threads idle."""
+    """fp32 with D = 12: the last block of channels (8 a warp with four
+    threads per channel, 16 with two) reaches past D, so part of its copies
+    of x / delta / z are zero-filled and part of its threads idle."""
     inp = ssm_gen.make_s6_inputs(2, 37, 12, 16, dtype="f32", bidir=bidir, seed=7, random_A=True,
                                  random_D=True)
     tol = TOL["f32"]
