@@ -359,7 +359,7 @@ class DeviceWorkload:
     def _launches(self):
         """Kernel launches of one call: the S6 plan's segment count decides
         (summary, carry and main passes, or the main pass alone).  The plain
-        scan reports its own plan; the ordered / conv / checkpointing
+        and checkpointing scans take the reported plan; the ordered / conv
         variants always give each thread whole channels, so their plan is
         read under that layout."""
         if self.info["kind"] != "s6":
@@ -367,7 +367,7 @@ class DeviceWorkload:
         seg, cpl = ctypes.c_int(0), ctypes.c_int(0)
         query = lambda: self.lib.ssm_scan_plan(ctypes.byref(self.dims), int(self.info["ndir"] == 2),
                                                ctypes.byref(seg), ctypes.byref(cpl))
-        if self.op == "scan":
+        if self.op in ("scan", "fwd_ckpt"):
             st = query()
         else:
             self.lib.ssm_debug_s6_mapping(1)

@@ -452,9 +452,9 @@ SSM_API ssm_status ssm_check_device(void *stream);
 SSM_API void ssm_debug_ssd_stall(int withhold_chunk, unsigned wait_limit);
 
 /*
- * Test hook for the choice between the two thread layouts of the plain S6
- * scans (ssm_scan_fwd, ssm_scan_fwd_state, ssm_scan_fwd_noalloc,
- * bidir_scan_fwd; the pages have no counterpart).  With N = 16 those calls
+ * Test hook for the choice between the thread layouts of the plain S6 scans
+ * (ssm_scan_fwd, ssm_scan_fwd_state, ssm_scan_fwd_noalloc, bidir_scan_fwd and
+ * the checkpointing forwards; the pages have no counterpart).  With N = 16 those calls
  * either give each GPU thread one or two whole channels (cutting long
  * sequences into segments), or split each channel's 16 states over four or
  * over two threads in one pass; a cost model fitted to measured B200

@@ -61,7 +61,7 @@ struct S6Args {
     int conv;                    // 1: x is the conv input x_in, each direction convolves it
     int ckpt;                    // 1: each direction also writes its checkpoints (DirArgs::ckpt)
     int split;                   // 2 or 4: that many threads per channel (s6_split.cu); needs
-                                 // N == 16, S == 1, and none of order / mask / conv / ckpt
+                                 // N == 16, S == 1, and none of order / mask / conv
 };
 
 struct S6Plan {

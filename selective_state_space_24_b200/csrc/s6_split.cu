@@ -388,6 +388,16 @@ __global__ void __launch_bounds__(64, min_blocks<Q>()) s6_split_kernel(const S6A
             gate[r] = GATE ? silu_f<T>(lds1<T>(sq + S::kZ)) : 1.f;
             dxv[r] = Dd * xv;
         }
+        // checkpointing calls: the state entering this group is the
+        // checkpoint of 4-step chunk gi of the scan order; each thread's
+        // share of its channel's 16 states is contiguous, so the warp's
+        // stores cover its channels' rows in one run
+        if (P.ckpt && active) {
+            float4 *ck = reinterpret_cast<float4 *>(P.ckpt + (((size_t)b * G + gi) * D + d) * 16 + NQ * q);
+#pragma unroll
+            for (int v = 0; v < NQ / 4; v++)
+                ck[v] = make_float4(h2[2 * v].x, h2[2 * v].y, h2[2 * v + 1].x, h2[2 * v + 1].y);
+        }
         // B: the four steps' state updates and shares of C . h (step s's dt
         // and dt x come from thread s % Q of the channel)
         float part[kG];

@@ -112,7 +112,10 @@ ssm_status run_s6(const ssm_dims *dims, const void *x, const void *delta, int so
             a.dir[i].ckpt = ckpt[i];
     }
     a.out = out;
-    const int q = (order || mask || conv || ckpt)
+    // the split-state layouts also serve the checkpointing calls (their 4-step
+    // groups are the checkpoint chunks); ordered and conv calls keep the
+    // one-channel kernels
+    const int q = (order || mask || conv)
                       ? 0
                       : ssm::split_threads(dims->batch, dims->seqlen, dims->dim, dims->dstate, ndir);
     if (q) {

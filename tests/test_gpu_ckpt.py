@@ -36,10 +36,9 @@ def _inputs(inp, dtype):
 
 
 def _ckpt_segments(B, L, D, dtype):
-    """Segments of the checkpointing forward's plan: it always gives each
-    thread whole channels (the plan of the plain calls under that layout)."""
-    with ssm.s6_mapping(ssm.MAPPING_WHOLE_CHANNELS):
-        return ssm.scan_plan(B, L, D, 16, ssm.SSM_F32 if dtype == "f32" else ssm.SSM_BF16)[0]
+    """Segments of the checkpointing forward's plan (the plain call's plan:
+    one for the split-state layouts)."""
+    return ssm.scan_plan(B, L, D, 16, ssm.SSM_F32 if dtype == "f32" else ssm.SSM_BF16)[0]
 
 
 def _recomputed_ckpt(t, reverse, dout):
@@ -67,21 +66,20 @@ def _recomputed_ckpt(t, reverse, dout):
 @pytest.mark.parametrize("L", [101, 3000])
 def test_fwd_ckpt_outputs_and_checkpoints(dtype, reverse, L):
     """The checkpointing forward writes the plain forward's outputs and last
-    state: bit for bit when the plain forward takes the same thread layout
-    (one or two channels per thread), to rounding when it splits the
-    channels' states over four threads.  It also writes the state entering
-    every 4-step chunk: equal bit for bit to the backward's recompute when
-    the plan has one segment, and within rounding of it when the sequence is
-    cut into segments (entering states then come from the carry pass)."""
+    state bit for bit (both take the plan's layout), and to rounding those
+    of the one-channel layout when the plan splits the states over threads.
+    It also writes the state entering every 4-step chunk: equal bit for bit
+    to the backward's recompute when the plan has one segment, and within
+    rounding of it when the sequence is cut into segments (entering states
+    then come from the carry pass)."""
     inp = ssm_gen.make_s6_inputs(2, L, 96, 16, dtype=dtype, seed=L + reverse, random_A=True, random_D=True)
     t = _inputs(inp, dtype)
     ls0 = torch.zeros((2, 96, 16), device="cuda")
     ls1 = torch.zeros((2, 96, 16), device="cuda")
     ls2 = torch.zeros((2, 96, 16), device="cuda")
     kw = dict(delta_bias=t["delta_bias"], D=t["D"], z=t["z"], reverse=reverse)
+    out0 = ssm.ssm_scan_fwd(t["x"], t["delta"], t["A"], t["B"], t["C"], last_state=ls0, **kw)
     with ssm.s6_mapping(ssm.MAPPING_WHOLE_CHANNELS):
-        out0 = ssm.ssm_scan_fwd(t["x"], t["delta"], t["A"], t["B"], t["C"], last_state=ls0, **kw)
-    with ssm.s6_mapping(ssm.MAPPING_SPLIT_STATES):
         out2 = ssm.ssm_scan_fwd(t["x"], t["delta"], t["A"], t["B"], t["C"], last_state=ls2, **kw)
     out1, ck = ssm.ssm_scan_fwd_ckpt(t["x"], t["delta"], t["A"], t["B"], t["C"], last_state=ls1, **kw)
     torch.cuda.synchronize()
@@ -147,8 +145,7 @@ def test_bidir_ckpt_pair_matches_autograd(dtype, L):
         dout = ssm_gen.round_to_bf16(dout)
     f, b = dir_params(inp, "f"), dir_params(inp, "b")
     x, delta, dd = dev(inp.x, dtype), dev(inp.delta, dtype), dev(dout, dtype)
-    with ssm.s6_mapping(ssm.MAPPING_WHOLE_CHANNELS):   # the layout the checkpointing forward takes
-        out0 = ssm.bidir_scan_fwd(x, delta, f, b)
+    out0 = ssm.bidir_scan_fwd(x, delta, f, b)
     out1, ckf, ckb = ssm.bidir_scan_fwd_ckpt(x, delta, f, b)
     dx, ddelta, gf, gb = ssm.bidir_scan_bwd_ckpt(x, delta, f, b, dd, ckf, ckb)
     torch.cuda.synchronize()
