@@ -461,7 +461,9 @@ SSM_API void ssm_debug_ssd_stall(int withhold_chunk, unsigned wait_limit);
  * timings picks the fastest for the sizes (mode 0, the default).  Mode 1
  * makes calls enqueued after it, in this process, always take the first
  * layout, mode 2 four threads per channel and mode 3 two whenever N = 16;
- * ssm_scan_plan reports what the calls take.
+ * ssm_scan_plan reports what the calls take.  The backward passes with
+ * N = 16 split each channel's states over four threads unless mode 1 is
+ * set (then one thread per channel).
  * The two layouts sum the readout in different orders, so results agree to
  * rounding, not bit for bit.  Returns SSM_ERR_INVALID_ARG for another mode.
  * Process-wide and not synchronised with calls on other threads: for tests.

@@ -135,6 +135,12 @@ struct BwdArgs {
 };
 size_t bwd_workspace_bytes(int64_t Bsz, int64_t L, int64_t D, int64_t N);
 cudaError_t launch_bwd(const BwdArgs &a, cudaStream_t stream);
+// The backward sweep with each channel's 16 states over four threads
+// (s6_bwd_split.cu; N == 16), from the checkpoints in a.ckpt.
+cudaError_t launch_bwd_split(const BwdArgs &a, cudaStream_t stream);
+// Whether the N = 16 backward takes it: not under layout mode 1 of the
+// test setting (split_mode_set).
+bool bwd_split_enabled();
 
 // One SSD call.
 struct SSDArgs {

@@ -502,6 +502,11 @@ cudaError_t launch_ns(const BwdArgs &a, cudaStream_t st)
     }
     if (!a.ckpt_given)
         s6_bwd_ckpt_kernel<T, NS><<<g, kCta, 0, st>>>(a);
+    if (NS == 16 && a.N == 16 && bwd_split_enabled()) {
+        if ((e = cudaGetLastError()) != cudaSuccess)
+            return e;
+        return launch_bwd_split(a, st);
+    }
     s6_bwd_kernel<T, NS><<<g, kCta, 0, st>>>(a);
     return cudaGetLastError();
 }

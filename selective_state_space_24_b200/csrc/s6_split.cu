@@ -84,6 +84,9 @@ static_assert((kStages & (kStages - 1)) == 0, "ring index by mask");
 #ifndef SSM_S6_SPLIT_MAX_WARPS1
 #define SSM_S6_SPLIT_MAX_WARPS1 1024
 #endif
+#ifndef SSM_BWD_SPLIT
+#define SSM_BWD_SPLIT 1
+#endif
 
 #ifndef SSM_S6_SPLIT_SKEW
 #define SSM_S6_SPLIT_SKEW 1
@@ -572,6 +575,8 @@ int split_threads(int64_t Bsz, int64_t L, int64_t D, int64_t N, int ndir)
 }
 
 void split_mode_set(int mode) { g_split_mode.store(mode, std::memory_order_relaxed); }
+
+bool bwd_split_enabled() { return SSM_BWD_SPLIT && g_split_mode.load(std::memory_order_relaxed) != 1; }
 
 cudaError_t launch_s6_split(const S6Args &a, cudaStream_t st)
 {
