@@ -103,6 +103,9 @@ template <typename T, bool GATE> struct BwdSplitSmem {
 #ifndef SSM_BWD_SPLIT_MINB
 #define SSM_BWD_SPLIT_MINB 4
 #endif
+#ifndef SSM_BWD_SPLIT_KEEP_A
+#define SSM_BWD_SPLIT_KEEP_A 1
+#endif
 template <typename T, bool GATE>
 __global__ void __launch_bounds__(32 * kWarpsB, SSM_BWD_SPLIT_MINB) s6_bwd_split_kernel(const BwdArgs a)
 {
@@ -133,9 +136,8 @@ __global__ void __launch_bounds__(32 * kWarpsB, SSM_BWD_SPLIT_MINB) s6_bwd_split
     const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(&sm.ring[warp][0][0]);
     const char *safe = static_cast<const char *>(a.x);
     const char *cur[S::kPerLane];
-    long long cstep[S::kPerLane];   // bytes from one chunk's source to the previous chunk's
+    int cstep[S::kPerLane];         // bytes from one chunk's source to the previous chunk's
     uint32_t dst[S::kPerLane];
-    int pstep[S::kPerLane];         // the piece's step in the chunk (kKc: checkpoint)
     bool pok[S::kPerLane];
     const int c0 = nch - 1;         // the first chunk processed
 #pragma unroll
@@ -148,7 +150,6 @@ __global__ void __launch_bounds__(32 * kWarpsB, SSM_BWD_SPLIT_MINB) s6_bwd_split
         long long step;
         if (pp < kKc * S::kStepPieces) {
             const int s = pp / S::kStepPieces, off = (pp % S::kStepPieces) * 16;
-            pstep[j] = s;
             dst[j] = (uint32_t)(s * S::kStride + off);
             const int i0 = c0 * kKc + s;
             const long long t0 = rev ? (long long)L - 1 - i0 : i0;   // may lie outside [0, L) only for a
@@ -170,7 +171,6 @@ __global__ void __launch_bounds__(32 * kWarpsB, SSM_BWD_SPLIT_MINB) s6_bwd_split
             step = (rev ? 1 : -1) * (long long)kKc * row;   // chunks descend: t descends (ascends reversed)
         } else {
             const int cp = pp - kKc * S::kStepPieces;   // 16 bytes of the checkpoint rows
-            pstep[j] = kKc;
             dst[j] = (uint32_t)(S::kCk + cp * 16);
             ok = ok && d0w + cp / 4 < D;
             base = reinterpret_cast<const char *>(a.ckpt) + (((long long)b * nch + c0) * D + d0w) * 64 + cp * 16;
@@ -178,18 +178,28 @@ __global__ void __launch_bounds__(32 * kWarpsB, SSM_BWD_SPLIT_MINB) s6_bwd_split
         }
         pok[j] = ok;
         cur[j] = ok ? base : safe;
-        cstep[j] = ok ? step : 0;
+        cstep[j] = ok ? (int)step : 0;
     }
     auto issue = [&](int jj) {   // processed index jj: chunk nch - 1 - jj
         if (jj < nch) {
             const int c = nch - 1 - jj;
             const uint32_t sb = ring_s + (uint32_t)((jj % kStages) * S::kChunkBytes);
+            if ((c + 1) * kKc <= L) {
 #pragma unroll
-            for (int j = 0; j < S::kPerLane; j++)
-                if (lane + 32 * j < S::kPieces) {
-                    const bool in = pok[j] && (pstep[j] == kKc || c * kKc + pstep[j] < L);
-                    cp16(sb + dst[j], in ? cur[j] : safe, in ? 16 : 0);
+                for (int j = 0; j < S::kPerLane; j++)
+                    if (lane + 32 * j < S::kPieces)
+                        cp16(sb + dst[j], cur[j], pok[j] ? 16 : 0);
+            } else {   // the short last chunk: steps past L are zero-filled, not read
+#pragma unroll
+                for (int j = 0; j < S::kPerLane; j++) {
+                    const int p = lane + 32 * j;
+                    if (p < S::kPieces) {
+                        const bool ck = p >= kKc * S::kStepPieces;
+                        const bool in = pok[j] && (ck || c * kKc + p / S::kStepPieces < L);
+                        cp16(sb + dst[j], in ? cur[j] : safe, in ? 16 : 0);
+                    }
                 }
+            }
 #pragma unroll
             for (int j = 0; j < S::kPerLane; j++)
                 cur[j] += cstep[j];
@@ -274,7 +284,8 @@ __global__ void __launch_bounds__(32 * kWarpsB, SSM_BWD_SPLIT_MINB) s6_bwd_split
             if (GATE && a.dz && vq && active)
                 a.dz[ioq] = gq * fmaf(Dv, xq, ys) * sgq * (1.f + zq * (1.f - sgq));
         }
-        // C: the sweep, steps descending
+        // C: the sweep, steps descending (a = exp(dt A) kept from the
+        // recompute, or recomputed here when registers are short)
         float dxs[kKc], dta[kKc];
         float (*red)[kWarpsB][32] = sm.red[jj & 1];
 #pragma unroll
@@ -297,10 +308,17 @@ __global__ void __launch_bounds__(32 * kWarpsB, SSM_BWD_SPLIT_MINB) s6_bwd_split
                 v[4 + 2 * e] = rc.x;
                 v[4 + 2 * e + 1] = rc.y;
                 dxs2 = __ffma2_rn(l, Bn, dxs2);
-                const float2 lah = __fmul2_rn(l, __fmul2_rn(an[k][e], h[k][e]));   // lam_i a_i h_{i-1}
+                float2 ak;
+                if (SSM_BWD_SPLIT_KEEP_A) {
+                    ak = an[k][e];
+                } else {
+                    const float2 w = __fmul2_rn(dt2, Al[e]);
+                    ak = make_float2(ex2_mufu(w.x), ex2_mufu(w.y));
+                }
+                const float2 lah = __fmul2_rn(l, __fmul2_rn(ak, h[k][e]));   // lam_i a_i h_{i-1}
                 dta2 = __ffma2_rn(lah, Al[e], dta2);
                 gA[e] = __ffma2_rn(dt2, lah, gA[e]);
-                lam[e] = __fmul2_rn(an[k][e], l);
+                lam[e] = __fmul2_rn(ak, l);
             }
             dxs[k] = dxs2.x + dxs2.y;
             dta[k] = dta2.x + dta2.y;
