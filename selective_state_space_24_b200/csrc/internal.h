@@ -84,6 +84,10 @@ cudaError_t launch_s6(const S6Args &a, cudaStream_t stream);
 // bidirectional bf16 stash of plan_s6.
 int split_threads(int64_t Bsz, int64_t L, int64_t D, int64_t N, int ndir);
 cudaError_t launch_s6_split(const S6Args &a, cudaStream_t stream);
+// The same kernel as the backward's checkpoint pass: one direction (a.dir[0],
+// a.reverse), a.split threads per channel, only dir[0].ckpt written (the
+// state entering every 4-step chunk; no outputs, gate or skip).
+cudaError_t launch_s6_split_ckpt_only(const S6Args &a, cudaStream_t stream);
 // Test setting (process-wide): 0 the cost model decides, 1 never the split
 // layouts, 2 four threads per channel, 3 two, whenever supported.
 void split_mode_set(int mode);

@@ -31,6 +31,7 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <string.h>
 
 #include "internal.h"
 #include "s6_math.cuh"
@@ -500,9 +501,26 @@ cudaError_t launch_ns(const BwdArgs &a, cudaStream_t st)
             return e;
         carveout_set.fetch_or(bit, std::memory_order_relaxed);
     }
-    if (!a.ckpt_given)
-        s6_bwd_ckpt_kernel<T, NS><<<g, kCta, 0, st>>>(a);
-    if (NS == 16 && a.N == 16 && bwd_split_enabled()) {
+    const bool split = NS == 16 && a.N == 16 && bwd_split_enabled();
+    if (!a.ckpt_given) {
+        // the checkpoint pass: the split-state forward kernel when the plan
+        // gives these sizes a split layout, else one thread per channel
+        const int q = split ? split_threads(a.Bsz, a.L, a.D, a.N, 1) : 0;
+        if (q) {
+            S6Args f;
+            memset(&f, 0, sizeof(f));
+            f.Bsz = a.Bsz, f.L = a.L, f.D = a.D, f.N = a.N, f.S = 1, f.T = a.L;
+            f.dtype = a.dtype, f.softplus = a.softplus, f.ndir = 1, f.reverse = a.reverse;
+            f.x = a.x, f.delta = a.delta, f.split = q;
+            f.dir[0].bias = a.bias, f.dir[0].A = a.A, f.dir[0].B = a.B, f.dir[0].C = a.C;
+            f.dir[0].ckpt = a.ckpt;
+            if ((e = launch_s6_split_ckpt_only(f, st)) != cudaSuccess)
+                return e;
+        } else {
+            s6_bwd_ckpt_kernel<T, NS><<<g, kCta, 0, st>>>(a);
+        }
+    }
+    if (split) {
         if ((e = cudaGetLastError()) != cudaSuccess)
             return e;
         return launch_bwd_split(a, st);

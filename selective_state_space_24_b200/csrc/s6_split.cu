@@ -211,7 +211,9 @@ template <> __device__ __forceinline__ float4 lds4<__nv_bfloat16>(const char *p)
 enum Mode { kPlain, kPark, kMixed, kAdd };
 template <Mode M> using ModeTag = std::integral_constant<Mode, M>;
 
-template <typename T, int Q, bool BIDIR, bool GATE, bool SOFTPLUS>
+// OUT = false: the checkpoint pass of the backward (single direction, no
+// gate): only the states entering each 4-step group are stored.
+template <typename T, int Q, bool BIDIR, bool GATE, bool SOFTPLUS, bool OUT = true>
 __global__ void __launch_bounds__(64, min_blocks<Q>()) s6_split_kernel(const S6Args a)
 {
     static_assert(Q == 2 || Q == 4, "two or four threads per channel");
@@ -272,6 +274,7 @@ __global__ void __launch_bounds__(64, min_blocks<Q>()) s6_split_kernel(const S6A
     bool pok[S::kPerLane];            // the piece holds channels below D
     bool xd[S::kPerLane];             // an x / delta piece: L2 policy by half
     bool pk[S::kPerLane];             // a piece of the partner's parked row
+    bool use[S::kPerLane];            // copied at all (no C rows without outputs)
     uint64_t pfix[S::kPerLane];       // the policy of the other pieces
 #pragma unroll
     for (int j = 0; j < S::kPerLane; j++) {
@@ -285,6 +288,7 @@ __global__ void __launch_bounds__(64, min_blocks<Q>()) s6_split_kernel(const S6A
         long long row;
         bool ok = exists;
         pk[j] = false;
+        use[j] = exists;
         if (off >= S::kPk) {   // 4 of the partner's parked fp32 outputs (bidirectional)
             const int jb = off - S::kPk;
             xd[j] = false;
@@ -304,6 +308,7 @@ __global__ void __launch_bounds__(64, min_blocks<Q>()) s6_split_kernel(const S6A
         } else {             // 16 bytes of the B or C row (read by every warp of this batch row)
             const int o2 = off - S::kB;
             const T *src = o2 < S::kBC ? Bm : Cm;
+            use[j] = exists && (OUT || o2 < S::kBC);
             xd[j] = false;
             pfix[j] = pol_normal;
             row = 16 * (long long)sizeof(T);
@@ -324,12 +329,12 @@ __global__ void __launch_bounds__(64, min_blocks<Q>()) s6_split_kernel(const S6A
             if ((gi + 1) * kG <= L) {
 #pragma unroll
                 for (int j = 0; j < S::kPerLane; j++)
-                    if (lane + 32 * j < S::kGroupPieces && (!BIDIR || !pk[j] || parked_live))
+                    if ((OUT ? lane + 32 * j < S::kGroupPieces : use[j]) && (!BIDIR || !pk[j] || parked_live))
                         cp16(sb + dst[j], cur[j], pok[j] ? 16 : 0, xd[j] ? pxd : pfix[j]);
             } else {   // the last group is short: steps past L are zero-filled, not read
 #pragma unroll
                 for (int j = 0; j < S::kPerLane; j++)
-                    if (lane + 32 * j < S::kGroupPieces && (!BIDIR || !pk[j] || parked_live)) {
+                    if ((OUT ? lane + 32 * j < S::kGroupPieces : use[j]) && (!BIDIR || !pk[j] || parked_live)) {
                         const bool in = pok[j] && gi * kG + (lane + 32 * j) / S::kPieces < L;
                         cp16(sb + dst[j], in ? cur[j] : safe, in ? 16 : 0, xd[j] ? pxd : pfix[j]);
                     }
@@ -415,17 +420,23 @@ __global__ void __launch_bounds__(64, min_blocks<Q>()) s6_split_kernel(const S6A
 #pragma unroll
             for (int v = 0; v < NQ / 4; v++) {
                 const float4 B4 = lds4<T>(ss + S::kB + 4 * v * (int)sizeof(T));
-                const float4 C4 = lds4<T>(ss + S::kC + 4 * v * (int)sizeof(T));
                 float2 w = __fmul2_rn(dt2, A2[2 * v]);
                 float2 e = make_float2(ex2_mufu(w.x), ex2_mufu(w.y));
                 h2[2 * v] = __ffma2_rn(e, h2[2 * v], __fmul2_rn(dtx2, make_float2(B4.x, B4.y)));
                 w = __fmul2_rn(dt2, A2[2 * v + 1]);
                 e = make_float2(ex2_mufu(w.x), ex2_mufu(w.y));
                 h2[2 * v + 1] = __ffma2_rn(e, h2[2 * v + 1], __fmul2_rn(dtx2, make_float2(B4.z, B4.w)));
-                y2 = __ffma2_rn(make_float2(C4.x, C4.y), h2[2 * v], y2);
-                y2 = __ffma2_rn(make_float2(C4.z, C4.w), h2[2 * v + 1], y2);
+                if (OUT) {
+                    const float4 C4 = lds4<T>(ss + S::kC + 4 * v * (int)sizeof(T));
+                    y2 = __ffma2_rn(make_float2(C4.x, C4.y), h2[2 * v], y2);
+                    y2 = __ffma2_rn(make_float2(C4.z, C4.w), h2[2 * v + 1], y2);
+                }
             }
             part[s] = y2.x + y2.y;
+        }
+        if (!OUT) {   // checkpoint pass: nothing else to write
+            __syncwarp();
+            return;
         }
         // C: sum the channel's Q shares of each step so that thread q holds
         // those of its steps q + Q r
@@ -507,7 +518,7 @@ __global__ void __launch_bounds__(64, min_blocks<Q>()) s6_split_kernel(const S6A
     }
     cp_wait<0>();
 
-    if (active && P.last_state) {
+    if (OUT && active && P.last_state) {
 #pragma unroll
         for (int v = 0; v < NQ / 4; v++)
             *reinterpret_cast<float4 *>(P.last_state + ((size_t)b * D + d) * 16 + NQ * q + 4 * v) =
@@ -533,6 +544,23 @@ template <typename T, bool GATE, bool SOFTPLUS>
 cudaError_t launch_t(const S6Args &a, cudaStream_t st)
 {
     return a.split == 2 ? launch_q<T, 2, GATE, SOFTPLUS>(a, st) : launch_q<T, 4, GATE, SOFTPLUS>(a, st);
+}
+
+// the backward's checkpoint pass: one direction, no gate, no outputs
+template <typename T, int Q, bool SOFTPLUS>
+cudaError_t launch_ckpt_q(const S6Args &a, cudaStream_t st)
+{
+    constexpr int kChW = 32 / Q;
+    const dim3 grid((unsigned)((a.D + 2 * kChW - 1) / (2 * kChW)), (unsigned)a.Bsz);
+    s6_split_kernel<T, Q, false, false, SOFTPLUS, false><<<grid, 64, 0, st>>>(a);
+    return cudaGetLastError();
+}
+template <typename T>
+cudaError_t launch_ckpt_t(const S6Args &a, cudaStream_t st)
+{
+    if (a.split == 2)
+        return a.softplus ? launch_ckpt_q<T, 2, true>(a, st) : launch_ckpt_q<T, 2, false>(a, st);
+    return a.softplus ? launch_ckpt_q<T, 4, true>(a, st) : launch_ckpt_q<T, 4, false>(a, st);
 }
 
 template <typename T>
@@ -577,6 +605,11 @@ int split_threads(int64_t Bsz, int64_t L, int64_t D, int64_t N, int ndir)
 void split_mode_set(int mode) { g_split_mode.store(mode, std::memory_order_relaxed); }
 
 bool bwd_split_enabled() { return SSM_BWD_SPLIT && g_split_mode.load(std::memory_order_relaxed) != 1; }
+
+cudaError_t launch_s6_split_ckpt_only(const S6Args &a, cudaStream_t st)
+{
+    return a.dtype == 0 ? launch_ckpt_t<float>(a, st) : launch_ckpt_t<__nv_bfloat16>(a, st);
+}
 
 cudaError_t launch_s6_split(const S6Args &a, cudaStream_t st)
 {
