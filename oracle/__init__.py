@@ -11,6 +11,9 @@ Functions (all return float64 numpy arrays):
   with skip term and SiLU gate)
 * ``bidir(inp, ...)``                  -- forward + reversed with separate
   parameters, summed
+* ``s6_arrays(..., zoh=True)`` / ``bidir_arrays(..., zoh=True)`` -- the
+  same scans with the exact zero-order-hold input coefficient instead of
+  dt B
 * ``ssd_seq(inp, ...)``                -- Mamba2 SSD as the sequential scan
   with a scalar A per head
 * ``ssd_chunked(inp, chunk, ...)``     -- Mamba2 SSD in the chunked form
@@ -61,6 +64,8 @@ def _load():
                                           ctypes.c_int])
         lib.oracle_bidir.argtypes = ([_i64] * 4 + [_dp, _dp, ctypes.c_int] + [_dp] * 7 + [_dp] * 7
                                      + [_dp, _ip, _i64, ctypes.c_int])
+        lib.oracle_s6_zoh.argtypes = lib.oracle_s6_state.argtypes
+        lib.oracle_bidir_zoh.argtypes = lib.oracle_bidir.argtypes
         lib.oracle_ssd_seq.argtypes = [_i64] * 5 + [_dp, _dp, _dp, ctypes.c_int, _dp, _dp, _dp, _dp,
                                                     _dp, _dp, _dp, _ip, _i64, ctypes.c_int]
         lib.oracle_ssd_chunked.argtypes = [_i64] * 6 + [_dp, _dp, _dp, ctypes.c_int, _dp, _dp, _dp,
@@ -92,11 +97,13 @@ def _cols(cols):
 
 
 def s6_arrays(x, delta, A, B, C, *, delta_bias=None, softplus=True, D=None, z=None,
-              reverse=False, cols=None, want_state=True, nthreads=1, initial_state=None
+              reverse=False, cols=None, want_state=True, nthreads=1, initial_state=None, zoh=False
               ) -> Tuple[np.ndarray, Optional[np.ndarray]]:
     """Single-direction S6 on raw arrays: returns (out (B,L,D), last_state (B,D,N)).
 
-    initial_state (B, D, N): the state before the first step (None = zero)."""
+    initial_state (B, D, N): the state before the first step (None = zero).
+    zoh: the exact zero-order-hold input coefficient (exp(dt a) - 1) / a of
+    the Mamba2 page, sec. 2.2, instead of its dt B approximation."""
     x, delta, A, B, C = map(_f64, (x, delta, A, B, C))
     delta_bias, D, z, h0 = map(_f64, (delta_bias, D, z, initial_state))
     Bsz, L, Dm = x.shape
@@ -104,7 +111,13 @@ def s6_arrays(x, delta, A, B, C, *, delta_bias=None, softplus=True, D=None, z=No
     out = np.zeros((Bsz, L, Dm))
     st = np.zeros((Bsz, Dm, N)) if want_state else None
     keep, cp, nc = _cols(cols)
-    if h0 is None:
+    if zoh:
+        if h0 is not None:
+            assert h0.shape == (Bsz, Dm, N)
+        _load().oracle_s6_zoh(Bsz, L, Dm, N, _ptr(x), _ptr(delta), _ptr(delta_bias),
+                              int(softplus), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+                              int(reverse), _ptr(h0), _ptr(out), _ptr(st), cp, nc, int(nthreads))
+    elif h0 is None:
         _load().oracle_s6(Bsz, L, Dm, N, _ptr(x), _ptr(delta), _ptr(delta_bias), int(softplus),
                           _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), int(reverse), _ptr(out),
                           _ptr(st), cp, nc, int(nthreads))
@@ -233,11 +246,12 @@ def s6(inp, reverse=False, cols=None, softplus=True, nthreads=1):
                      nthreads=nthreads)
 
 
-def bidir_arrays(x, delta, fwd: dict, bwd: dict, *, softplus=True, cols=None, nthreads=1):
+def bidir_arrays(x, delta, fwd: dict, bwd: dict, *, softplus=True, cols=None, nthreads=1, zoh=False):
     """Bidirectional scan on raw arrays.
 
     fwd / bwd: dicts with keys delta_bias, A, B, C, D, z (delta_bias, D, z may
-    be None).  Returns (out, last_state_f, last_state_b).
+    be None).  zoh: the exact zero-order-hold coefficient (see s6_arrays) in
+    both directions.  Returns (out, last_state_f, last_state_b).
     """
     x, delta = _f64(x), _f64(delta)
     Bsz, L, Dm = x.shape
@@ -248,12 +262,11 @@ def bidir_arrays(x, delta, fwd: dict, bwd: dict, *, softplus=True, cols=None, nt
     f = {k: _f64(fwd.get(k)) for k in ("delta_bias", "A", "B", "C", "D", "z")}
     b = {k: _f64(bwd.get(k)) for k in ("delta_bias", "A", "B", "C", "D", "z")}
     keep, cp, nc = _cols(cols)
-    _load().oracle_bidir(Bsz, L, Dm, N, _ptr(x), _ptr(delta), int(softplus),
-                         _ptr(f["delta_bias"]), _ptr(f["A"]), _ptr(f["B"]), _ptr(f["C"]),
-                         _ptr(f["D"]), _ptr(f["z"]), _ptr(lf),
-                         _ptr(b["delta_bias"]), _ptr(b["A"]), _ptr(b["B"]), _ptr(b["C"]),
-                         _ptr(b["D"]), _ptr(b["z"]), _ptr(lb),
-                         _ptr(out), cp, nc, int(nthreads))
+    fn = _load().oracle_bidir_zoh if zoh else _load().oracle_bidir
+    fn(Bsz, L, Dm, N, _ptr(x), _ptr(delta), int(softplus),
+       _ptr(f["delta_bias"]), _ptr(f["A"]), _ptr(f["B"]), _ptr(f["C"]), _ptr(f["D"]), _ptr(f["z"]), _ptr(lf),
+       _ptr(b["delta_bias"]), _ptr(b["A"]), _ptr(b["B"]), _ptr(b["C"]), _ptr(b["D"]), _ptr(b["z"]), _ptr(lb),
+       _ptr(out), cp, nc, int(nthreads))
     return out, lf, lb
 
 

@@ -11,7 +11,8 @@
  *  - "手写简化版Mamba2：状态空间模型如何突破Transformer长序列瓶颈"
  *    (intelliparadigm.com), sec. 2.2: discrete recurrence
  *    h_t = Abar h_{t-1} + Bbar x_t, y_t = C h_t + D x_t with Abar = exp(dt A)
- *    and the Bbar ~= dt B approximation that Mamba uses;
+ *    and the Bbar ~= dt B approximation that Mamba uses (the exact
+ *    zero-order-hold Bbar of the same section in the *_zoh functions);
  *    sec. 4.2: dt = softplus(...), A negative;
  *    sec. 4.3: the per-time-step reference scan (state zero-initialised,
  *    elementwise decay over the N states, readout summed over N);
@@ -60,9 +61,29 @@ static double dt_of(double delta, const double *bias, int64_t d, int softplus)
 }
 
 /*
+ * The input coefficient of one state for one step.  The Mamba2 page,
+ * sec. 2.2, discretises h' = A h + B x by zero-order hold (x held constant
+ * over the step, the equation integrated exactly):
+ *   Abar = exp(dt A),   Bbar = (dt A)^-1 (exp(dt A) - I) dt B,
+ * and the scans of sec. 4.3 use the approximation Bbar = dt B.  A is
+ * diagonal here, so per state the exact coefficient of B is
+ * (exp(dt a) - 1) / a, written with expm1 so that small dt a does not
+ * cancel; its limit at a = 0 is dt.
+ */
+static double bbar_coef(double dt, double a, int zoh)
+{
+    if (!zoh)
+        return dt;
+    if (a == 0.0)
+        return dt;
+    return expm1(dt * a) / a;
+}
+
+/*
  * One S6 column (batch b, channel d): the recurrence of sec. 4.3 with the
- * skip term and gate of sec. 4.4.  The state starts at h0 (N values) or, if
- * h0 is NULL, at zero as in sec. 4.3.  mask (Bsz, L) or NULL: a token with
+ * skip term and gate of sec. 4.4 (zoh: the exact zero-order-hold Bbar of
+ * sec. 2.2 instead of dt B; see bbar_coef).  The state starts at h0 (N
+ * values) or, if h0 is NULL, at zero as in sec. 4.3.  mask (Bsz, L) or NULL: a token with
  * mask 0 is bypassed (Samba page, sec. 2: the state is not updated and the
  * computation is skipped) -- h passes through unchanged and y[t] = 0.
  * Writes y[t] for t in [0, L) and the final state (N values) to hlast if
@@ -72,7 +93,7 @@ static void s6_column(int64_t b, int64_t d, int64_t L, int64_t D, int64_t N,
                       const double *x, const double *delta, const double *bias, int softplus,
                       const double *A, const double *Bm, const double *Cm, const double *Dv,
                       const double *z, int reverse, double *y, double *hlast, double *h,
-                      const double *h0, const unsigned char *mask)
+                      const double *h0, const unsigned char *mask, int zoh)
 {
     for (int64_t n = 0; n < N; n++)
         h[n] = h0 ? h0[n] : 0.0;
@@ -87,7 +108,8 @@ static void s6_column(int64_t b, int64_t d, int64_t L, int64_t D, int64_t N,
         double acc = 0.0;
         for (int64_t n = 0; n < N; n++) {
             double dA = exp(dt * A[d * N + n]);              /* Abar = exp(dt A) */
-            double dBx = dt * Bm[(b * L + t) * N + n] * x[i]; /* Bbar x = dt B x  */
+            double dBx = bbar_coef(dt, A[d * N + n], zoh) * Bm[(b * L + t) * N + n] * x[i];
+                                                              /* Bbar x (dt B x unless zoh) */
             h[n] = dA * h[n] + dBx;
             acc += Cm[(b * L + t) * N + n] * h[n];
         }
@@ -117,7 +139,7 @@ static void s6_run(int64_t Bsz, int64_t L, int64_t D, int64_t N,
                    const double *A, const double *Bm, const double *Cm, const double *Dv,
                    const double *z, int reverse, double *out, double *last_state,
                    const double *initial_state, const unsigned char *mask, const int64_t *cols,
-                   int64_t ncols, int nthreads, int accumulate)
+                   int64_t ncols, int nthreads, int accumulate, int zoh)
 {
     int64_t total = cols ? ncols : Bsz * D;
 #ifdef _OPENMP
@@ -137,7 +159,7 @@ static void s6_run(int64_t Bsz, int64_t L, int64_t D, int64_t N,
             double *hl = last_state ? last_state + (b * D + d) * N : NULL;
             const double *h0 = initial_state ? initial_state + (b * D + d) * N : NULL;
             s6_column(b, d, L, D, N, x, delta, delta_bias, softplus, A, Bm, Cm, Dv, z,
-                      reverse, y, hl, h, h0, mask);
+                      reverse, y, hl, h, h0, mask, zoh);
             for (int64_t t = 0; t < L; t++) {
                 int64_t i = (b * L + t) * D + d;
                 out[i] = accumulate ? out[i] + y[t] : y[t];
@@ -155,7 +177,7 @@ void oracle_s6(int64_t Bsz, int64_t L, int64_t D, int64_t N,
                const int64_t *cols, int64_t ncols, int nthreads)
 {
     s6_run(Bsz, L, D, N, x, delta, delta_bias, softplus, A, Bm, Cm, Dv, z, reverse, out,
-           last_state, NULL, NULL, cols, ncols, nthreads, 0);
+           last_state, NULL, NULL, cols, ncols, nthreads, 0, 0);
 }
 
 /*
@@ -172,7 +194,7 @@ void oracle_s6_state(int64_t Bsz, int64_t L, int64_t D, int64_t N,
                      double *last_state, const int64_t *cols, int64_t ncols, int nthreads)
 {
     s6_run(Bsz, L, D, N, x, delta, delta_bias, softplus, A, Bm, Cm, Dv, z, reverse, out,
-           last_state, initial_state, NULL, cols, ncols, nthreads, 0);
+           last_state, initial_state, NULL, cols, ncols, nthreads, 0, 0);
 }
 
 /*
@@ -189,7 +211,7 @@ void oracle_s6_masked(int64_t Bsz, int64_t L, int64_t D, int64_t N,
                       double *last_state, const int64_t *cols, int64_t ncols, int nthreads)
 {
     s6_run(Bsz, L, D, N, x, delta, delta_bias, softplus, A, Bm, Cm, Dv, z, reverse, out,
-           last_state, NULL, mask, cols, ncols, nthreads, 0);
+           last_state, NULL, mask, cols, ncols, nthreads, 0, 0);
 }
 
 /*
@@ -207,9 +229,39 @@ void oracle_bidir(int64_t Bsz, int64_t L, int64_t D, int64_t N,
                   double *out, const int64_t *cols, int64_t ncols, int nthreads)
 {
     s6_run(Bsz, L, D, N, x, delta, bias_f, softplus, A_f, B_f, C_f, D_f, z_f, 0, out, last_f,
-           NULL, NULL, cols, ncols, nthreads, 0);
+           NULL, NULL, cols, ncols, nthreads, 0, 0);
     s6_run(Bsz, L, D, N, x, delta, bias_b, softplus, A_b, B_b, C_b, D_b, z_b, 1, out, last_b,
-           NULL, NULL, cols, ncols, nthreads, 1);
+           NULL, NULL, cols, ncols, nthreads, 1, 0);
+}
+
+/*
+ * oracle_s6_state with the exact zero-order-hold input coefficient of the
+ * Mamba2 page, sec. 2.2 (bbar_coef) in place of dt B.  initial_state may be
+ * NULL (zero).
+ */
+void oracle_s6_zoh(int64_t Bsz, int64_t L, int64_t D, int64_t N,
+                   const double *x, const double *delta, const double *delta_bias, int softplus,
+                   const double *A, const double *Bm, const double *Cm, const double *Dv,
+                   const double *z, int reverse, const double *initial_state, double *out,
+                   double *last_state, const int64_t *cols, int64_t ncols, int nthreads)
+{
+    s6_run(Bsz, L, D, N, x, delta, delta_bias, softplus, A, Bm, Cm, Dv, z, reverse, out,
+           last_state, initial_state, NULL, cols, ncols, nthreads, 0, 1);
+}
+
+/* oracle_bidir with the zero-order-hold coefficient in both directions. */
+void oracle_bidir_zoh(int64_t Bsz, int64_t L, int64_t D, int64_t N,
+                      const double *x, const double *delta, int softplus,
+                      const double *bias_f, const double *A_f, const double *B_f, const double *C_f,
+                      const double *D_f, const double *z_f, double *last_f,
+                      const double *bias_b, const double *A_b, const double *B_b, const double *C_b,
+                      const double *D_b, const double *z_b, double *last_b,
+                      double *out, const int64_t *cols, int64_t ncols, int nthreads)
+{
+    s6_run(Bsz, L, D, N, x, delta, bias_f, softplus, A_f, B_f, C_f, D_f, z_f, 0, out, last_f,
+           NULL, NULL, cols, ncols, nthreads, 0, 1);
+    s6_run(Bsz, L, D, N, x, delta, bias_b, softplus, A_b, B_b, C_b, D_b, z_b, 1, out, last_b,
+           NULL, NULL, cols, ncols, nthreads, 1, 1);
 }
 
 /*

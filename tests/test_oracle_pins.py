@@ -672,3 +672,113 @@ def test_bidir_grads_match_finite_differences():
             num[idx] = (vals[0] - vals[1]) / (2 * eps)
         scale = max(np.max(np.abs(num)), 1e-8)
         assert np.max(np.abs(ana - num)) / scale < 1e-6, (k, side)
+
+
+# ---------------------------------------------------- exact zero-order hold
+# The Mamba2 page, sec. 2.2: zero-order hold keeps x constant over each
+# step and integrates h' = A h + B x exactly, which gives Abar = exp(dt A)
+# and Bbar = (dt A)^-1 (exp(dt A) - I) dt B; the scans use dt B instead.
+# The pins below check the oracle's exact form against a numerical ODE
+# integration and against scipy's matrix-exponential discretisation.
+
+
+def test_zoh_is_the_exact_integral_of_the_continuous_system():
+    """Each step integrates h' = a h + B_t x_t (x_t, B_t held over the step
+    of length dt_t) with an adaptive Runge-Kutta solver; the readout
+    y_t = C_t . h_t + D x_t is then compared with the oracle's outputs, and
+    the final state with its last state.  Includes a zero and a positive
+    entry of A."""
+    from scipy.integrate import solve_ivp
+    rng = np.random.default_rng(91)
+    L, Dm, N = 9, 2, 3
+    x = rng.standard_normal((1, L, Dm))
+    dt = rng.uniform(0.05, 0.8, (1, L, Dm))
+    A = np.array([[-1.5, 0.0, 0.4], [-6.0, -0.02, -0.7]])
+    B = rng.standard_normal((1, L, N))
+    C = rng.standard_normal((1, L, N))
+    Dv = rng.uniform(0.5, 1.5, Dm)
+    h0 = rng.standard_normal((1, Dm, N))
+    y, st = oracle.s6_arrays(x, dt, A, B, C, softplus=False, D=Dv, initial_state=h0, zoh=True)
+    for d in range(Dm):
+        h = h0[0, d].copy()
+        for t in range(L):
+            u = B[0, t] * x[0, t, d]
+            sol = solve_ivp(lambda _s, hh: A[d] * hh + u, (0.0, dt[0, t, d]), h, method="DOP853",
+                            rtol=1e-12, atol=1e-14)
+            h = sol.y[:, -1]
+            _close(y[0, t, d], np.dot(C[0, t], h) + Dv[d] * x[0, t, d], 1e-9)
+        _close(st[0, d], h, 1e-9)
+
+
+@pytest.mark.parametrize("reverse", [False, True])
+def test_zoh_lti_matches_scipy_discretisation(reverse):
+    """Constant dt, B and C per channel make each channel an LTI system;
+    scipy.signal.cont2discrete(method='zoh') discretises it through the
+    exponential of the augmented matrix [[A, B], [0, 0]] dt, and dlsim runs
+    it.  The reversed scan is the forward one on the flipped input."""
+    from scipy import signal
+    rng = np.random.default_rng(92)
+    L, Dm, N = 40, 3, 4
+    x = rng.standard_normal((1, L, Dm))
+    dtc = rng.uniform(0.02, 0.6, Dm)
+    delta = np.broadcast_to(dtc, (1, L, Dm)).copy()
+    A = -np.exp(rng.uniform(-1.0, 1.5, (Dm, N)))
+    A[1, 2] = 0.0
+    Bv, Cv = rng.standard_normal(N), rng.standard_normal(N)
+    B = np.broadcast_to(Bv, (1, L, N)).copy()
+    C = np.broadcast_to(Cv, (1, L, N)).copy()
+    Dv = rng.uniform(0.5, 1.5, Dm)
+    y, _ = oracle.s6_arrays(x, delta, A, B, C, softplus=False, D=Dv, reverse=reverse, zoh=True)
+    for d in range(Dm):
+        Ad, Bd, Cd, Dd, _ = signal.cont2discrete((np.diag(A[d]), Bv[:, None], Cv[None, :], [[Dv[d]]]),
+                                                 dtc[d], method="zoh")
+        u = x[0, ::-1, d] if reverse else x[0, :, d]
+        # dlsim's y_t uses the state before step t; the scan reads out after
+        # it, i.e. C (Ad h + Bd u_t) + D u_t: the same system with C Ad, C Bd + D
+        _, yd, _ = signal.dlsim((Ad, Bd, Cd @ Ad, Cd @ Bd + Dd, dtc[d]), u)
+        ref = yd[:, 0][::-1] if reverse else yd[:, 0]
+        _close(y[0, :, d], ref, 1e-11)
+
+
+def test_zoh_with_zero_A_is_the_dt_B_scan():
+    """With A = 0 the exact coefficient's limit is dt, so both forms agree
+    bit for bit (exp(0) = 1 in both)."""
+    rng = np.random.default_rng(93)
+    x, delta, bias, A, B, C, D, z = _rand_case(rng, 2, 13, 3, 4)
+    A = np.zeros_like(A)
+    kw = dict(delta_bias=bias, D=D, z=z)
+    y0, s0 = oracle.s6_arrays(x, delta, A, B, C, **kw)
+    y1, s1 = oracle.s6_arrays(x, delta, A, B, C, zoh=True, **kw)
+    assert np.array_equal(y0, y1) and np.array_equal(s0, s1)
+
+
+def test_zoh_approaches_dt_B_for_small_steps():
+    """The two forms differ by a factor expm1(w) / w = 1 + w / 2 + ... per
+    state (w = dt a), so for a single step from zero the ratio of the states
+    is that factor, and for small dt the outputs agree to O(dt a)."""
+    rng = np.random.default_rng(94)
+    x, delta, bias, A, B, C, D, z = _rand_case(rng, 1, 1, 2, 3, gate=False)
+    dt = np.full((1, 1, 2), 0.3)
+    _, s_e = oracle.s6_arrays(x, dt, A, B, C, softplus=False)
+    _, s_z = oracle.s6_arrays(x, dt, A, B, C, softplus=False, zoh=True)
+    w = 0.3 * A
+    _close(s_z[0] / s_e[0], np.expm1(w) / w, 1e-13)
+    x, delta, bias, A, B, C, D, z = _rand_case(rng, 1, 50, 2, 3, gate=False)
+    small = np.full_like(x, 1e-5)
+    y_e, _ = oracle.s6_arrays(x, small, A, B, C, softplus=False)
+    y_z, _ = oracle.s6_arrays(x, small, A, B, C, softplus=False, zoh=True)
+    gap = np.max(np.abs(y_z - y_e)) / np.max(np.abs(y_e))
+    assert 0.0 < gap <= 1e-5 * np.max(np.abs(A))
+
+
+def test_zoh_bidir_is_sum_of_directions():
+    rng = np.random.default_rng(95)
+    x, delta, bias, A, B, C, D, z = _rand_case(rng, 2, 11, 3, 4)
+    _, _, bias2, A2, B2, C2, D2, z2 = _rand_case(rng, 2, 11, 3, 4)
+    fwd = dict(delta_bias=bias, A=A, B=B, C=C, D=D, z=z)
+    bwd = dict(delta_bias=bias2, A=A2, B=B2, C=C2, D=D2, z=z2)
+    out, lf, lb = oracle.bidir_arrays(x, delta, fwd, bwd, zoh=True)
+    yf, sf = oracle.s6_arrays(x, delta, A, B, C, delta_bias=bias, D=D, z=z, zoh=True)
+    yb, sb = oracle.s6_arrays(x, delta, A2, B2, C2, delta_bias=bias2, D=D2, z=z2, reverse=True, zoh=True)
+    _close(out, yf + yb)
+    assert np.array_equal(lf, sf) and np.array_equal(lb, sb)
