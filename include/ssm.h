@@ -208,6 +208,36 @@ SSM_API ssm_status bidir_scan_fwd(const ssm_dims *dims, const void *x, const voi
                           size_t workspace_bytes, void *stream);
 
 /*
+ * ssm_scan_fwd_state and bidir_scan_fwd with the exact zero-order-hold
+ * discretisation of the Mamba2 page, sec. 2.2, in place of its dt B
+ * approximation: x is held constant over each step and h' = A h + B x is
+ * integrated exactly, so per state
+ *   h_t = exp(dt a) h_{t-1} + ((exp(dt a) - 1) / a) B_t x_t
+ * (the limit dt B_t x_t where a = 0).  On the GPU the coefficient is
+ * (e - 1) / a from the step's own exponential e where |dt a| >= 1/16, and
+ * the series dt (1 + u/2 + u^2/6 + u^3/24), u = dt a, below that (where
+ * e - 1 would cancel).
+ * Arguments, layouts, workspace (ssm_scan_workspace_size /
+ * bidir_scan_workspace_size of the same dims) and errors as for
+ * ssm_scan_fwd_state and bidir_scan_fwd, and:
+ *   dims->dstate must be 16 and dims->batch at most 65535
+ *   (SSM_ERR_UNSUPPORTED_SHAPE otherwise): these run only on the layout
+ *   that splits each channel's 16 states over two or four threads.
+ * Forward scans only: the backward, checkpointing, ordered, conv and decode
+ * entry points use dt B.
+ */
+SSM_API ssm_status ssm_scan_fwd_zoh(const ssm_dims *dims, const void *x, const void *delta,
+                                   const float *delta_bias, int delta_softplus, const float *A,
+                                   const void *B, const void *C, const float *D, const void *z,
+                                   int reverse, const float *initial_state, void *out,
+                                   float *last_state, void *workspace, size_t workspace_bytes,
+                                   void *stream);
+SSM_API ssm_status bidir_scan_fwd_zoh(const ssm_dims *dims, const void *x, const void *delta,
+                                     int delta_softplus, const ssm_dir_params *fwd,
+                                     const ssm_dir_params *bwd, void *out, void *workspace,
+                                     size_t workspace_bytes, void *stream);
+
+/*
  * How ssm_scan_fwd (bidirectional = 0) or bidir_scan_fwd (bidirectional = 1)
  * runs a problem of these sizes.  The pages have no counterpart: this is a
  * query of the library's own launch plan, for callers sizing work and for

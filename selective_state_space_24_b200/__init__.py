@@ -9,6 +9,8 @@ Entry points (names as in include/ssm.h):
 
 * ``ssm_scan_fwd(x, delta, A, B, C, ...)``  single-direction S6 scan
 * ``ssm_scan_fwd_state(...)``  the same from a given initial state
+* ``ssm_scan_fwd_zoh`` / ``bidir_scan_fwd_zoh``  the forward scans with the
+  exact zero-order-hold input coefficient instead of dt B (N = 16)
 * ``ssm_scan_bwd(x, delta, A, B, C, dout, ...)``  gradients of ssm_scan_fwd
 * ``ssm_scan_fwd_ckpt`` / ``bidir_scan_fwd_ckpt``  the forward scans that also
   store the state entering every 4-step chunk, and ``ssm_scan_bwd_ckpt`` /
@@ -89,6 +91,11 @@ SIGNATURES = {
                             _int, _vp, _vp, _vp, _sz, _vp]),
     "ssm_scan_fwd_state": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp,
                                   _vp, _int, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "ssm_scan_fwd_zoh": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp,
+                                _vp, _int, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "bidir_scan_fwd_zoh": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _int,
+                                  ctypes.POINTER(ssm_dir_params), ctypes.POINTER(ssm_dir_params), _vp,
+                                  _vp, _sz, _vp]),
     "ssm_scan_fwd_ordered": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp,
                                     _vp, _int, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "bidir_scan_fwd_ordered": (_int, [ctypes.POINTER(ssm_dims), _vp, _vp, _int,
@@ -263,6 +270,26 @@ def ssm_scan_fwd_state(x, delta, A, B, C, *, initial_state=None, delta_bias=None
                                 _ptr(last_state), _ptr(ws), 0 if ws is None else ws.numel(),
                                 _stream_handle(stream))
     _check(st, "ssm_scan_fwd_state")
+    return out
+
+
+def ssm_scan_fwd_zoh(x, delta, A, B, C, *, initial_state=None, delta_bias=None, delta_softplus=True,
+                     D=None, z=None, reverse=False, out=None, last_state=None, ws=None, stream=None):
+    """ssm_scan_fwd_state with the exact zero-order-hold input coefficient
+    (exp(dt a) - 1) / a in place of dt (N = 16)."""
+    torch = _torch()
+    lib = capi()
+    dims = s6_dims(x, A.shape[1])
+    if out is None:
+        out = torch.empty_like(x)
+    need = lib.ssm_scan_workspace_size(ctypes.byref(dims))
+    if ws is None:
+        ws = workspace(need, x.device)
+    st = lib.ssm_scan_fwd_zoh(ctypes.byref(dims), _ptr(x), _ptr(delta), _ptr(delta_bias),
+                              int(bool(delta_softplus)), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+                              int(bool(reverse)), _ptr(initial_state), _ptr(out), _ptr(last_state),
+                              _ptr(ws), 0 if ws is None else ws.numel(), _stream_handle(stream))
+    _check(st, "ssm_scan_fwd_zoh")
     return out
 
 
@@ -590,6 +617,26 @@ def bidir_scan_fwd(x, delta, fwd: DirParams, bwd: DirParams, *, delta_softplus=T
                             ctypes.byref(f), ctypes.byref(b), _ptr(out), _ptr(ws),
                             0 if ws is None else ws.numel(), _stream_handle(stream))
     _check(st, "bidir_scan_fwd")
+    return out
+
+
+def bidir_scan_fwd_zoh(x, delta, fwd: DirParams, bwd: DirParams, *, delta_softplus=True, out=None,
+                       ws=None, stream=None):
+    """bidir_scan_fwd with the exact zero-order-hold input coefficient in
+    both directions (N = 16)."""
+    torch = _torch()
+    lib = capi()
+    dims = s6_dims(x, fwd.A.shape[1])
+    if out is None:
+        out = torch.empty_like(x)
+    need = lib.bidir_scan_workspace_size(ctypes.byref(dims))
+    if ws is None:
+        ws = workspace(need, x.device)
+    f, b = fwd.to_c(), bwd.to_c()
+    st = lib.bidir_scan_fwd_zoh(ctypes.byref(dims), _ptr(x), _ptr(delta), int(bool(delta_softplus)),
+                                ctypes.byref(f), ctypes.byref(b), _ptr(out), _ptr(ws),
+                                0 if ws is None else ws.numel(), _stream_handle(stream))
+    _check(st, "bidir_scan_fwd_zoh")
     return out
 
 

@@ -62,6 +62,7 @@ struct S6Args {
     int ckpt;                    // 1: each direction also writes its checkpoints (DirArgs::ckpt)
     int split;                   // 2 or 4: that many threads per channel (s6_split.cu); needs
                                  // N == 16, S == 1, and none of order / mask / conv
+    int zoh;                     // 1: the exact zero-order-hold input coefficient (needs split)
 };
 
 struct S6Plan {

@@ -61,8 +61,12 @@ constexpr int kStages = 4;             // groups in the copy ring (a power of tw
 #define SSM_S6_SPLIT_MINB2 10
 #endif
 // CTAs per SM by threads per channel (two threads per channel hold 8
-// states each and need more registers)
-template <int Q> constexpr int min_blocks() { return Q == 2 ? SSM_S6_SPLIT_MINB2 : SSM_S6_SPLIT_MINB; }
+// states each and need more registers); the zero-order-hold variants keep
+// 1 / A of their states as well
+template <int Q, bool ZOH = false> constexpr int min_blocks()
+{
+    return ZOH ? (Q == 2 ? 8 : 10) : (Q == 2 ? SSM_S6_SPLIT_MINB2 : SSM_S6_SPLIT_MINB);
+}
 static_assert((kStages & (kStages - 1)) == 0, "ring index by mask");
 // Which layout the plain calls take (split_threads).  The one-thread-per-
 // channel kernels give a warp 64 channels (two a thread); with fewer than
@@ -209,12 +213,39 @@ template <> __device__ __forceinline__ float4 lds4<__nv_bfloat16>(const char *p)
 // point, meet the partner, then add to the rest (the group holding the
 // exchange point); add the partner's parked values (second half).
 enum Mode { kPlain, kPark, kMixed, kAdd };
+
+// The factor of B in a state pair's update: dt x (Bbar = dt B), or for the
+// exact zero-order hold (xv = x) x (e - 1) / a, with e = exp(dt a) and
+// w = dt a log2(e), taken as x dt (1 + u / 2 + u^2 / 6 + u^3 / 24) with
+// u = dt a where |u| < 1/16
+template <bool ZOH>
+__device__ __forceinline__ float2 in_coef(float2 dt2, float2 xv2, float2 w, float2 e, float2 iA)
+{
+    if (!ZOH)
+        return xv2;   // dt x
+    constexpr float kLn2 = 0.693147180559945309f;
+    constexpr float c1 = kLn2 / 2.f, c2 = kLn2 * kLn2 / 6.f, c3 = kLn2 * kLn2 * kLn2 / 24.f;
+    constexpr float kSeries = 0.0625f / kLn2;   // |u| < 1/16 in units of w
+    float2 p = __ffma2_rn(w, make_float2(c3, c3), make_float2(c2, c2));
+    p = __ffma2_rn(w, p, make_float2(c1, c1));
+    p = __ffma2_rn(w, p, make_float2(1.f, 1.f));
+    const float2 series = __fmul2_rn(dt2, p);
+    const float2 direct = __fmul2_rn(__fadd2_rn(e, make_float2(-1.f, -1.f)), iA);
+    const float2 c = make_float2(fabsf(w.x) < kSeries ? series.x : direct.x, fabsf(w.y) < kSeries ? series.y : direct.y);
+    return __fmul2_rn(c, xv2);
+}
 template <Mode M> using ModeTag = std::integral_constant<Mode, M>;
 
 // OUT = false: the checkpoint pass of the backward (single direction, no
 // gate): only the states entering each 4-step group are stored.
-template <typename T, int Q, bool BIDIR, bool GATE, bool SOFTPLUS, bool OUT = true>
-__global__ void __launch_bounds__(64, min_blocks<Q>()) s6_split_kernel(const S6Args a)
+// ZOH: the exact zero-order-hold input coefficient of the Mamba2 page,
+// sec. 2.2 -- Bbar = (dt A)^-1 (exp(dt A) - I) dt B, per state
+// (exp(dt a) - 1) / a -- instead of dt B.  e - 1 from the exponential the
+// step computes anyway would lose its leading digits for small dt a, so
+// there (|dt a| < 1/16) the coefficient is dt (1 + w / 2 + w^2 / 6 +
+// w^3 / 24), w = dt a, whose truncation error is below 1.3e-7 relative.
+template <typename T, int Q, bool BIDIR, bool GATE, bool SOFTPLUS, bool OUT = true, bool ZOH = false>
+__global__ void __launch_bounds__(64, min_blocks<Q, ZOH>()) s6_split_kernel(const S6Args a)
 {
     static_assert(Q == 2 || Q == 4, "two or four threads per channel");
     using S = Slot<T, GATE, BIDIR, Q>;
@@ -239,6 +270,7 @@ __global__ void __launch_bounds__(64, min_blocks<Q>()) s6_split_kernel(const S6A
 
     // this thread's states [NQ q, NQ q + NQ) as pairs, A scaled by log2(e)
     float2 A2[NP], h2[NP];
+    float2 iA2[ZOH ? NP : 1] = {};   // zero-order hold: 1 / A (natural units)
 #pragma unroll
     for (int v = 0; v < NQ / 4; v++) {
         float4 av = make_float4(0.f, 0.f, 0.f, 0.f), hv = av;
@@ -249,6 +281,10 @@ __global__ void __launch_bounds__(64, min_blocks<Q>()) s6_split_kernel(const S6A
         }
         A2[2 * v] = make_float2(av.x * kLog2e, av.y * kLog2e);
         A2[2 * v + 1] = make_float2(av.z * kLog2e, av.w * kLog2e);
+        if (ZOH) {   // (a = 0 only ever takes the series branch)
+            iA2[2 * v] = make_float2(1.f / av.x, 1.f / av.y);
+            iA2[2 * v + 1] = make_float2(1.f / av.z, 1.f / av.w);
+        }
         h2[2 * v] = make_float2(hv.x, hv.y);
         h2[2 * v + 1] = make_float2(hv.z, hv.w);
     }
@@ -392,7 +428,7 @@ __global__ void __launch_bounds__(64, min_blocks<Q>()) s6_split_kernel(const S6A
             if (SOFTPLUS)
                 t = softplus_f(t);
             dt[r] = valid[r] ? t : 0.f;   // past L: exp(0) = 1 and no input, the state passes through
-            dtx[r] = dt[r] * xv;
+            dtx[r] = ZOH ? xv : dt[r] * xv;   // zero-order hold: x (its coefficient carries dt)
             gate[r] = GATE ? silu_f<T>(lds1<T>(sq + S::kZ)) : 1.f;
             dxv[r] = Dd * xv;
         }
@@ -422,10 +458,13 @@ __global__ void __launch_bounds__(64, min_blocks<Q>()) s6_split_kernel(const S6A
                 const float4 B4 = lds4<T>(ss + S::kB + 4 * v * (int)sizeof(T));
                 float2 w = __fmul2_rn(dt2, A2[2 * v]);
                 float2 e = make_float2(ex2_mufu(w.x), ex2_mufu(w.y));
-                h2[2 * v] = __ffma2_rn(e, h2[2 * v], __fmul2_rn(dtx2, make_float2(B4.x, B4.y)));
+                h2[2 * v] = __ffma2_rn(e, h2[2 * v], __fmul2_rn(in_coef<ZOH>(dt2, dtx2, w, e, iA2[ZOH ? 2 * v : 0]),
+                                                                make_float2(B4.x, B4.y)));
                 w = __fmul2_rn(dt2, A2[2 * v + 1]);
                 e = make_float2(ex2_mufu(w.x), ex2_mufu(w.y));
-                h2[2 * v + 1] = __ffma2_rn(e, h2[2 * v + 1], __fmul2_rn(dtx2, make_float2(B4.z, B4.w)));
+                h2[2 * v + 1] = __ffma2_rn(
+                    e, h2[2 * v + 1],
+                    __fmul2_rn(in_coef<ZOH>(dt2, dtx2, w, e, iA2[ZOH ? 2 * v + 1 : 0]), make_float2(B4.z, B4.w)));
                 if (OUT) {
                     const float4 C4 = lds4<T>(ss + S::kC + 4 * v * (int)sizeof(T));
                     y2 = __ffma2_rn(make_float2(C4.x, C4.y), h2[2 * v], y2);
@@ -526,24 +565,24 @@ __global__ void __launch_bounds__(64, min_blocks<Q>()) s6_split_kernel(const S6A
     }
 }
 
-template <typename T, int Q, bool GATE, bool SOFTPLUS>
+template <typename T, int Q, bool GATE, bool SOFTPLUS, bool ZOH>
 cudaError_t launch_q(const S6Args &a, cudaStream_t st)
 {
     constexpr int kChW = 32 / Q;
     if (a.ndir == 2) {
         const dim3 grid((unsigned)((a.D + kChW - 1) / kChW), (unsigned)a.Bsz);
-        s6_split_kernel<T, Q, true, GATE, SOFTPLUS><<<grid, 64, 0, st>>>(a);
+        s6_split_kernel<T, Q, true, GATE, SOFTPLUS, true, ZOH><<<grid, 64, 0, st>>>(a);
     } else {
         const dim3 grid((unsigned)((a.D + 2 * kChW - 1) / (2 * kChW)), (unsigned)a.Bsz);
-        s6_split_kernel<T, Q, false, GATE, SOFTPLUS><<<grid, 64, 0, st>>>(a);
+        s6_split_kernel<T, Q, false, GATE, SOFTPLUS, true, ZOH><<<grid, 64, 0, st>>>(a);
     }
     return cudaGetLastError();
 }
 
-template <typename T, bool GATE, bool SOFTPLUS>
+template <typename T, bool GATE, bool SOFTPLUS, bool ZOH>
 cudaError_t launch_t(const S6Args &a, cudaStream_t st)
 {
-    return a.split == 2 ? launch_q<T, 2, GATE, SOFTPLUS>(a, st) : launch_q<T, 4, GATE, SOFTPLUS>(a, st);
+    return a.split == 2 ? launch_q<T, 2, GATE, SOFTPLUS, ZOH>(a, st) : launch_q<T, 4, GATE, SOFTPLUS, ZOH>(a, st);
 }
 
 // the backward's checkpoint pass: one direction, no gate, no outputs
@@ -563,13 +602,13 @@ cudaError_t launch_ckpt_t(const S6Args &a, cudaStream_t st)
     return a.softplus ? launch_ckpt_q<T, 4, true>(a, st) : launch_ckpt_q<T, 4, false>(a, st);
 }
 
-template <typename T>
+template <typename T, bool ZOH>
 cudaError_t launch_flags(const S6Args &a, cudaStream_t st)
 {
     const bool gate = a.dir[0].z != nullptr;
     if (gate)
-        return a.softplus ? launch_t<T, true, true>(a, st) : launch_t<T, true, false>(a, st);
-    return a.softplus ? launch_t<T, false, true>(a, st) : launch_t<T, false, false>(a, st);
+        return a.softplus ? launch_t<T, true, true, ZOH>(a, st) : launch_t<T, true, false, ZOH>(a, st);
+    return a.softplus ? launch_t<T, false, true, ZOH>(a, st) : launch_t<T, false, false, ZOH>(a, st);
 }
 
 }  // namespace
@@ -613,7 +652,9 @@ cudaError_t launch_s6_split_ckpt_only(const S6Args &a, cudaStream_t st)
 
 cudaError_t launch_s6_split(const S6Args &a, cudaStream_t st)
 {
-    return a.dtype == 0 ? launch_flags<float>(a, st) : launch_flags<__nv_bfloat16>(a, st);
+    if (a.zoh)
+        return a.dtype == 0 ? launch_flags<float, true>(a, st) : launch_flags<__nv_bfloat16, true>(a, st);
+    return a.dtype == 0 ? launch_flags<float, false>(a, st) : launch_flags<__nv_bfloat16, false>(a, st);
 }
 
 }  // namespace ssm

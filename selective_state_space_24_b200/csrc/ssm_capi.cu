@@ -66,8 +66,11 @@ ssm_status run_s6(const ssm_dims *dims, const void *x, const void *delta, int so
                   int reverse, const ssm_dir_params *dirs, void *out, void *ws, size_t ws_bytes,
                   cudaStream_t stream, const float *initial_state = nullptr, const int32_t *order = nullptr,
                   const unsigned char *mask = nullptr, const ssm_conv_params *conv = nullptr,
-                  float *const *ckpt = nullptr)
+                  float *const *ckpt = nullptr, bool zoh = false)
 {
+    // the exact zero-order hold runs on the split-state kernel only
+    if (zoh && (dims->dstate != 16 || dims->batch > 65535))
+        return SSM_ERR_UNSUPPORTED_SHAPE;
     const int dt = dims->dtype == SSM_F32 ? 0 : 1;
     const ssm::S6Plan plan =
         ssm::plan_s6(dims->batch, dims->seqlen, dims->dim, dims->dstate, ndir, dt);
@@ -115,9 +118,13 @@ ssm_status run_s6(const ssm_dims *dims, const void *x, const void *delta, int so
     // the split-state layouts also serve the checkpointing calls (their 4-step
     // groups are the checkpoint chunks); ordered and conv calls keep the
     // one-channel kernels
-    const int q = (order || mask || conv)
-                      ? 0
-                      : ssm::split_threads(dims->batch, dims->seqlen, dims->dim, dims->dstate, ndir);
+    int q = (order || mask || conv)
+                ? 0
+                : ssm::split_threads(dims->batch, dims->seqlen, dims->dim, dims->dstate, ndir);
+    if (zoh) {   // the plan's split layout, else four threads per channel
+        a.zoh = 1;
+        q = q ? q : 4;
+    }
     if (q) {
         a.split = q;   // one pass, q threads per channel
         a.S = 1;
@@ -199,7 +206,7 @@ ssm_status scan_single(const ssm_dims *dims, const void *x, const void *delta, c
                        const void *z, int reverse, const float *initial_state, const int32_t *order,
                        const unsigned char *mask, void *out, float *last_state, void *workspace,
                        size_t workspace_bytes, void *stream, const ssm_conv_params *conv = nullptr,
-                       float *ckpt = nullptr, bool want_ckpt = false)
+                       float *ckpt = nullptr, bool want_ckpt = false, bool zoh = false)
 {
     ssm_status s = check_s6_dims(dims);
     if (s != SSM_OK)
@@ -239,13 +246,14 @@ ssm_status scan_single(const ssm_dims *dims, const void *x, const void *delta, c
         return SSM_ERR_MISALIGNED;
     float *const ck[1] = {ckpt};
     return run_s6(dims, x, delta, delta_softplus, 1, reverse, &p, out, workspace, workspace_bytes, st,
-                  initial_state, order, mask, conv, want_ckpt ? ck : nullptr);
+                  initial_state, order, mask, conv, want_ckpt ? ck : nullptr, zoh);
 }
 
 ssm_status scan_bidir(const ssm_dims *dims, const void *x, const void *delta, int delta_softplus,
                       const ssm_dir_params *fwd, const ssm_dir_params *bwd, const int32_t *order,
                       const unsigned char *mask, void *out, void *workspace, size_t workspace_bytes,
-                      void *stream, const ssm_conv_params *conv = nullptr, float *const *ckpt = nullptr)
+                      void *stream, const ssm_conv_params *conv = nullptr, float *const *ckpt = nullptr,
+                      bool zoh = false)
 {
     ssm_status s = check_s6_dims(dims);
     if (s != SSM_OK)
@@ -281,7 +289,7 @@ ssm_status scan_bidir(const ssm_dims *dims, const void *x, const void *delta, in
         return SSM_ERR_MISALIGNED;
     const ssm_dir_params dirs[2] = {*fwd, *bwd};
     return run_s6(dims, x, delta, delta_softplus, 2, 0, dirs, out, workspace, workspace_bytes, st, nullptr,
-                  order, mask, conv, ckpt);
+                  order, mask, conv, ckpt, zoh);
 }
 
 }  // namespace
@@ -296,6 +304,16 @@ ssm_status ssm_scan_fwd_state(const ssm_dims *dims, const void *x, const void *d
 {
     return scan_single(dims, x, delta, delta_bias, delta_softplus, A, B, C, D, z, reverse, initial_state,
                        nullptr, nullptr, out, last_state, workspace, workspace_bytes, stream);
+}
+
+ssm_status ssm_scan_fwd_zoh(const ssm_dims *dims, const void *x, const void *delta, const float *delta_bias,
+                            int delta_softplus, const float *A, const void *B, const void *C, const float *D,
+                            const void *z, int reverse, const float *initial_state, void *out,
+                            float *last_state, void *workspace, size_t workspace_bytes, void *stream)
+{
+    return scan_single(dims, x, delta, delta_bias, delta_softplus, A, B, C, D, z, reverse, initial_state,
+                       nullptr, nullptr, out, last_state, workspace, workspace_bytes, stream, nullptr, nullptr,
+                       false, true);
 }
 
 ssm_status ssm_scan_fwd_ordered(const ssm_dims *dims, const void *x, const void *delta,
@@ -615,6 +633,14 @@ ssm_status bidir_scan_fwd(const ssm_dims *dims, const void *x, const void *delta
 {
     return scan_bidir(dims, x, delta, delta_softplus, fwd, bwd, nullptr, nullptr, out, workspace,
                       workspace_bytes, stream);
+}
+
+ssm_status bidir_scan_fwd_zoh(const ssm_dims *dims, const void *x, const void *delta, int delta_softplus,
+                              const ssm_dir_params *fwd, const ssm_dir_params *bwd, void *out,
+                              void *workspace, size_t workspace_bytes, void *stream)
+{
+    return scan_bidir(dims, x, delta, delta_softplus, fwd, bwd, nullptr, nullptr, out, workspace,
+                      workspace_bytes, stream, nullptr, nullptr, true);
 }
 
 size_t ssd_chunk_workspace_size(const ssd_dims *d)
