@@ -50,7 +50,7 @@ SMS = 148
 # capture matches them.
 NCU_TRAFFIC = {1: 208.71e6, 4: 397.22e6}
 NCU_TRAFFIC_STEP = 62.01e6
-NCU_TRAFFIC_BWD = {1: 415.96e6}
+NCU_TRAFFIC_BWD = {1: 408.07e6}
 
 
 def parse():
