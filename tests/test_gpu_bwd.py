@@ -109,3 +109,23 @@ def test_bidir_bwd_matches_autograd(dtype):
         for k, t in g.items():
             e = rel_err(t.cpu().numpy(), ref[side][names[k]])
             assert e <= tol, f"{side} {k}: rel err {e:.3e}"
+
+
+@pytest.mark.parametrize("layout", [ssm.MAPPING_WHOLE_CHANNELS, ssm.MAPPING_SPLIT_STATES, ssm.MAPPING_SPLIT_STATES_2],
+                         ids=["whole", "q4", "q2"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("reverse", [False, True])
+def test_bwd_checkpoint_pass_in_every_layout(layout, dtype, reverse):
+    """The plain backward's recompute pass runs on the forward layout the
+    plan gives the sizes (here forced): the split-state kernel without
+    outputs with two or four threads per channel, or the one-thread-per-
+    channel checkpoint kernel (which mode also selects the one-thread
+    backward sweep).  L = 70 leaves a short last chunk; D = 40 leaves warps
+    partly past D in every layout."""
+    inp = ssm_gen.make_s6_inputs(3, 70, 40, 16, dtype=dtype, seed=60 + reverse, random_A=True, random_D=True)
+    dout = np.random.default_rng(61).standard_normal(inp.x.shape).astype(np.float32)
+    if dtype == "bf16":
+        dout = ssm_gen.round_to_bf16(dout)
+    with ssm.s6_mapping(layout):
+        g, ref = _run(inp, dtype, dout, reverse)
+    _check(g, ref, TOL[dtype])

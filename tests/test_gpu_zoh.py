@@ -127,3 +127,14 @@ def test_state_sizes_other_than_16_are_refused():
     x, delta = dev(inp.x, "f32"), dev(inp.delta, "f32")
     with pytest.raises(ssm.SSMError, match="UNSUPPORTED_SHAPE"):
         ssm.ssm_scan_fwd_zoh(x, delta, f32dev(inp.A_f), dev(inp.B_f, "f32"), dev(inp.C_f, "f32"))
+
+
+def test_hires_bidirectional_bf16_full_size():
+    """B 8 L 1024 D 768 bf16 with the exact zero-order hold: every output
+    and both last states."""
+    inp = ssm_gen.make_workload(2)
+    out, lf, lb = _bidir(inp)
+    ref, rlf, rlb = _ref_bidir(inp)
+    assert rel_err(host(out), ref) <= TOL["bf16"]
+    assert rel_err(lf.cpu().numpy(), rlf) <= TOL["bf16"]
+    assert rel_err(lb.cpu().numpy(), rlb) <= TOL["bf16"]
