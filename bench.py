@@ -64,12 +64,13 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-per-config", action="store_true",
                    help="skip timing the other workloads after the headline one")
-    p.add_argument("--op", default="scan", choices=["scan", "ordered", "conv", "fwd_ckpt", "step", "bwd", "bidir_bwd",
-                                                    "bwd_ckpt", "bidir_bwd_ckpt"],
+    p.add_argument("--op", default="scan", choices=["scan", "ordered", "conv", "fwd_ckpt", "zoh", "step", "bwd",
+                                                    "bidir_bwd", "bwd_ckpt", "bidir_bwd_ckpt"],
                    help="scan: the workload's scan (default); ordered: the same bidirectional "
                         "workload along a random order of the positions with 30%% of the tokens "
                         "masked; conv: the same with a width-4 conv1d + SiLU per direction computed "
-                        "inside the scan; step: one decode step of a batch-512 x 1536-channel x "
+                        "inside the scan; zoh: the same with the exact zero-order-hold input coefficient "
+                        "(bidir_scan_fwd_zoh); step: one decode step of a batch-512 x 1536-channel x "
                         "16-state fp32 state (ssm_step); bwd: the gradients (ssm_scan_bwd) of the "
                         "forward direction of the workload; bidir_bwd: the gradients of the whole "
                         "bidirectional scan (bidir_scan_bwd); fwd_ckpt: the bidirectional scan that also "
@@ -337,13 +338,15 @@ class DeviceWorkload:
         self.ws_bytes = int(need)
         if op != "scan":
             assert self.info["kind"] == "s6" and self.info["ndir"] == 2, \
-                "ordered / conv / fwd_ckpt: bidirectional S6"
+                "ordered / conv / fwd_ckpt / zoh: bidirectional S6"
             i = self.inp
             rng = np.random.default_rng(seed + 1)
             if op == "fwd_ckpt":
                 nck = int(self.lib.ssm_scan_ckpt_size(ctypes.byref(self.dims))) // 4
                 self.ckpt = (torch.empty(nck, dtype=torch.float32, device=device),
                              torch.empty(nck, dtype=torch.float32, device=device))
+            elif op == "zoh":
+                pass
             elif op == "ordered":
                 self.order = torch.from_numpy(ssm_gen.order_random(i.seqlen, seed=seed)).to(device)
                 self.mask = torch.from_numpy(ssm_gen.token_mask(i.batch, i.seqlen, 0.7, seed=seed)).to(device)
@@ -362,8 +365,8 @@ class DeviceWorkload:
         and checkpointing scans take the reported plan; the ordered / conv
         variants always give each thread whole channels, so their plan is
         read under that layout."""
-        if self.info["kind"] != "s6":
-            return 1
+        if self.info["kind"] != "s6" or self.op == "zoh":
+            return 1   # (the zero-order-hold scans always run as one split-state pass)
         seg, cpl = ctypes.c_int(0), ctypes.c_int(0)
         query = lambda: self.lib.ssm_scan_plan(ctypes.byref(self.dims), int(self.info["ndir"] == 2),
                                                ctypes.byref(seg), ctypes.byref(cpl))
@@ -403,6 +406,10 @@ class DeviceWorkload:
                                          ctypes.byref(self.fwd), ctypes.byref(self.bwd), p(self.out),
                                          p(self.ckpt[0]), p(self.ckpt[1]), p(self.ws), self.ws_bytes,
                                          stream_handle)
+        elif self.op == "zoh":
+            st = lib.bidir_scan_fwd_zoh(ctypes.byref(self.dims), p(d["x"]), p(d["delta"]), 1,
+                                        ctypes.byref(self.fwd), ctypes.byref(self.bwd), p(self.out),
+                                        p(self.ws), self.ws_bytes, stream_handle)
         elif self.op == "conv":
             st = lib.bidir_scan_fwd_conv(ctypes.byref(self.dims), p(d["x"]), p(d["delta"]), 1,
                                          ctypes.byref(self.fwd), ctypes.byref(self.bwd),

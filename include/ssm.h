@@ -222,7 +222,9 @@ SSM_API ssm_status bidir_scan_fwd(const ssm_dims *dims, const void *x, const voi
  * ssm_scan_fwd_state and bidir_scan_fwd, and:
  *   dims->dstate must be 16 and dims->batch at most 65535
  *   (SSM_ERR_UNSUPPORTED_SHAPE otherwise): these run only on the layout
- *   that splits each channel's 16 states over two or four threads.
+ *   that splits each channel's 16 states over two or four threads, in one
+ *   pass without segments, so long sequences over few channels (where the
+ *   dt B scans cut the sequence into segments) run several times slower.
  * Forward scans only: the backward, checkpointing, ordered, conv and decode
  * entry points use dt B.
  */

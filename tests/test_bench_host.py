@@ -113,7 +113,7 @@ def test_launch_count_follows_the_plan():
     import selective_state_space_24_b200 as ssm
     lib = ssm.capi()
     expect = {(0, "scan"): 1, (1, "scan"): 1, (2, "scan"): 1, (3, "scan"): 3, (1, "fwd_ckpt"): 1,
-              (1, "ordered"): 1, (4, "scan"): 1}
+              (1, "ordered"): 1, (3, "zoh"): 1, (4, "scan"): 1}
     for (cfg, op), n in expect.items():
         w = bench.workload_info(cfg, op)
         dims = None
