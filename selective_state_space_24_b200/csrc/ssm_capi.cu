@@ -68,9 +68,6 @@ ssm_status run_s6(const ssm_dims *dims, const void *x, const void *delta, int so
                   const unsigned char *mask = nullptr, const ssm_conv_params *conv = nullptr,
                   float *const *ckpt = nullptr, bool zoh = false)
 {
-    // the exact zero-order hold runs on the split-state kernel only
-    if (zoh && (dims->dstate != 16 || dims->batch > 65535))
-        return SSM_ERR_UNSUPPORTED_SHAPE;
     const int dt = dims->dtype == SSM_F32 ? 0 : 1;
     const ssm::S6Plan plan =
         ssm::plan_s6(dims->batch, dims->seqlen, dims->dim, dims->dstate, ndir, dt);
@@ -249,6 +246,16 @@ ssm_status scan_single(const ssm_dims *dims, const void *x, const void *delta, c
                   initial_state, order, mask, conv, want_ckpt ? ck : nullptr, zoh);
 }
 
+// the zero-order-hold scans: N = 16 and a batch that fits the grid, also
+// for empty problems, so that the refusal does not depend on L
+ssm_status zoh_dims(const ssm_dims *dims)
+{
+    const ssm_status s = check_s6_dims(dims);
+    if (s != SSM_OK)
+        return s;
+    return dims->dstate != 16 || dims->batch > 65535 ? SSM_ERR_UNSUPPORTED_SHAPE : SSM_OK;
+}
+
 ssm_status scan_bidir(const ssm_dims *dims, const void *x, const void *delta, int delta_softplus,
                       const ssm_dir_params *fwd, const ssm_dir_params *bwd, const int32_t *order,
                       const unsigned char *mask, void *out, void *workspace, size_t workspace_bytes,
@@ -311,6 +318,9 @@ ssm_status ssm_scan_fwd_zoh(const ssm_dims *dims, const void *x, const void *del
                             const void *z, int reverse, const float *initial_state, void *out,
                             float *last_state, void *workspace, size_t workspace_bytes, void *stream)
 {
+    const ssm_status s = zoh_dims(dims);
+    if (s != SSM_OK)
+        return s;
     return scan_single(dims, x, delta, delta_bias, delta_softplus, A, B, C, D, z, reverse, initial_state,
                        nullptr, nullptr, out, last_state, workspace, workspace_bytes, stream, nullptr, nullptr,
                        false, true);
@@ -639,6 +649,9 @@ ssm_status bidir_scan_fwd_zoh(const ssm_dims *dims, const void *x, const void *d
                               const ssm_dir_params *fwd, const ssm_dir_params *bwd, void *out,
                               void *workspace, size_t workspace_bytes, void *stream)
 {
+    const ssm_status s = zoh_dims(dims);
+    if (s != SSM_OK)
+        return s;
     return scan_bidir(dims, x, delta, delta_softplus, fwd, bwd, nullptr, nullptr, out, workspace,
                       workspace_bytes, stream, nullptr, nullptr, true);
 }

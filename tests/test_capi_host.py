@@ -403,3 +403,23 @@ def test_checkpointing_pair_validation(lib):
                                                  ctypes.byref(g), cf, cb, None)
     assert bbw(FAKE, None) == 1      # the reversed direction's array missing: refused before any launch
     assert bbw(None, FAKE) == 1
+
+
+def test_zero_order_hold_validation(lib):
+    """ssm_scan_fwd_zoh / bidir_scan_fwd_zoh: N must be 16 and the batch fit
+    the grid, refused before anything runs (also for empty problems); other
+    arguments as for the dt B scans; an empty problem with N = 16 is a
+    no-op."""
+    def single(dims, x=FAKE, init=None):
+        return lib.ssm_scan_fwd_zoh(ctypes.byref(dims), x, FAKE, None, 1, FAKE, FAKE, FAKE, None, None, 0,
+                                    init, FAKE, None, None, 0, None)
+    good = ssm.ssm_dir_params(None, FAKE, FAKE, FAKE, None, None, None)
+    bidir = lambda dims: lib.bidir_scan_fwd_zoh(ctypes.byref(dims), FAKE, FAKE, 1, ctypes.byref(good),
+                                                ctypes.byref(good), FAKE, None, 0, None)
+    for d in (_dims(2, 8, 16, 8), _dims(2, 0, 16, 4), _dims(70000, 4, 16, 16)):
+        assert single(d) == 2 and bidir(d) == 2
+    assert single(_dims(2, 8, 16, 16), x=None) == 1
+    assert single(_dims(2, 8, 16, 16), init=FAKE + 4) == 3
+    assert lib.ssm_scan_fwd_zoh(None, FAKE, FAKE, None, 1, FAKE, FAKE, FAKE, None, None, 0, None, FAKE, None,
+                                None, 0, None) == 1
+    assert single(_dims(2, 0, 16, 16)) == 0 and bidir(_dims(0, 8, 16, 16)) == 0

@@ -138,3 +138,26 @@ def test_hires_bidirectional_bf16_full_size():
     assert rel_err(host(out), ref) <= TOL["bf16"]
     assert rel_err(lf.cpu().numpy(), rlf) <= TOL["bf16"]
     assert rel_err(lb.cpu().numpy(), rlb) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("layout", [ssm.MAPPING_SPLIT_STATES, ssm.MAPPING_SPLIT_STATES_2], ids=["q4", "q2"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_optional_inputs_absent(layout, dtype):
+    """No gate, no skip, no bias, softplus off, in both entry points."""
+    inp = _inputs(2, 37, 24, dtype, seed=13, bidir=True)
+    delta = np.abs(inp.delta)
+    if dtype == "bf16":
+        delta = ssm_gen.round_to_bf16(delta)
+    x, dl = dev(inp.x, dtype), dev(delta, dtype)
+    mk = lambda s: ssm.DirParams(A=f32dev(getattr(inp, "A_" + s)), B=dev(getattr(inp, "B_" + s), dtype),
+                                 C=dev(getattr(inp, "C_" + s), dtype))
+    with ssm.s6_mapping(layout):
+        out = ssm.bidir_scan_fwd_zoh(x, dl, mk("f"), mk("b"), delta_softplus=False)
+        one = ssm.ssm_scan_fwd_zoh(x, dl, f32dev(inp.A_f), dev(inp.B_f, dtype), dev(inp.C_f, dtype),
+                                   delta_softplus=False, reverse=True)
+    torch.cuda.synchronize()
+    ref, _, _ = oracle.bidir_arrays(inp.x, delta, dict(A=inp.A_f, B=inp.B_f, C=inp.C_f),
+                                    dict(A=inp.A_b, B=inp.B_b, C=inp.C_b), softplus=False, zoh=True)
+    ref1, _ = oracle.s6_arrays(inp.x, delta, inp.A_f, inp.B_f, inp.C_f, softplus=False, reverse=True, zoh=True)
+    assert rel_err(host(out), ref) <= TOL[dtype]
+    assert rel_err(host(one), ref1) <= TOL[dtype]
