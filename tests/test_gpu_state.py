@@ -89,10 +89,14 @@ def test_empty_sequence_keeps_initial_state():
 
 @pytest.mark.parametrize("dtype,N,batch,D", [("f32", 4, 3, 96), ("f32", 7, 3, 96), ("f32", 16, 3, 96),
                                               ("bf16", 4, 3, 96), ("bf16", 7, 3, 96), ("bf16", 16, 3, 96),
-                                              ("bf16", 8, 5, 200), ("f32", 16, 512, 1536)])
+                                              ("bf16", 8, 5, 200), ("f32", 16, 512, 1536),
+                                              ("bf16", 16, 512, 1536), ("f32", 16, 700, 136),
+                                              ("bf16", 16, 3, 8)])
 def test_step_matches_oracle(dtype, N, batch, D):
-    """One decode step against the oracle; the last case is the bench's
-    decode workload (B 512, D 1536, N 16, fp32), every row compared."""
+    """One decode step against the oracle; (512, 1536) is the bench's decode
+    workload (several 128-row tiles per CTA of the N = 16 kernel), every row
+    compared; (700, 136) gives some CTAs a second tile and a 96-row last
+    tile; (3, 8) bf16 a single 24-row tile."""
     inp = ssm_gen.make_s6_inputs(batch, 1, D, N, dtype=dtype, seed=N, random_A=True, random_D=True)
     state0 = np.random.default_rng(N).standard_normal((batch, D, N)).astype(np.float32)
     p = _params(inp, dtype)
@@ -124,3 +128,21 @@ def test_decode_loop_equals_scan():
     ref, rst = _oracle_scan(inp, None, False)
     assert rel_err(torch.stack(ys, 1).cpu().numpy(), ref) <= TOL["f32"]
     assert rel_err(state.cpu().numpy(), rst) <= TOL["f32"]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_step_optional_inputs_absent(dtype):
+    """N = 16 decode step with no gate, skip or bias and softplus off."""
+    batch, D = 40, 64
+    inp = ssm_gen.make_s6_inputs(batch, 1, D, 16, dtype=dtype, seed=5, random_A=True)
+    delta = np.abs(inp.delta[:, 0])
+    state0 = np.random.default_rng(6).standard_normal((batch, D, 16)).astype(np.float32)
+    state = f32dev(state0)
+    y = ssm.ssm_step(dev(inp.x[:, 0], dtype), dev(delta, dtype), f32dev(inp.A_f),
+                     dev(inp.B_f[:, 0], dtype), dev(inp.C_f[:, 0], dtype), state, delta_softplus=False)
+    torch.cuda.synchronize()
+    ry, rst = oracle.step_arrays(inp.x[:, 0], delta, inp.A_f, inp.B_f[:, 0], inp.C_f[:, 0], state0,
+                                 softplus=False)
+    assert rel_err(host(y), ry) <= TOL[dtype]
+    assert rel_err(state.cpu().numpy(), rst) <= TOL[dtype]
+    ssm.check_device()   # no device-side error word set
