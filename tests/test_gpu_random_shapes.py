@@ -7,7 +7,10 @@ four threads per channel) is exercised at sizes no hand-written case
 picks; every output and last state is compared in full.  Twenty-five more
 draw backward problems and compare every gradient with the autograd
 oracle, and fifteen draw Mamba2 SSD problems (batch, length, heads,
-optional inputs) against the sequential oracle."""
+optional inputs) against the sequential oracle.  Further draws cover the
+ordered scans with a random permutation and token mask, the conv prologue
+with random widths, the checkpointing training pair, the exact
+zero-order-hold scans and the decode step."""
 import numpy as np
 import pytest
 import torch
@@ -130,3 +133,159 @@ def test_ssd(seed):
                                      D=inp.D if skip else None, z=inp.z if gate else None, nthreads=NTHREADS)
     assert rel_err(host(out), ref) <= TOL["bf16"], (Bz, L, H, N, gate, skip, bias)
     assert rel_err(ls.cpu().numpy(), rls) <= TOL["bf16"]
+
+
+def _dirparams(inp, s, dtype, f, Bz, D, N):
+    return ssm.DirParams(A=f32dev(getattr(inp, "A_" + s)), B=dev(getattr(inp, "B_" + s), dtype),
+                         C=dev(getattr(inp, "C_" + s), dtype),
+                         D=f32dev(getattr(inp, "D_" + s)) if f["skip"] else None,
+                         z=dev(getattr(inp, "z_" + s), dtype) if f["gate"] else None,
+                         delta_bias=f32dev(getattr(inp, "dt_bias_" + s)))
+
+
+def _oracle_dir(inp, s, f):
+    return dict(A=getattr(inp, "A_" + s), B=getattr(inp, "B_" + s), C=getattr(inp, "C_" + s),
+                D=getattr(inp, "D_" + s) if f["skip"] else None, z=getattr(inp, "z_" + s) if f["gate"] else None,
+                delta_bias=getattr(inp, "dt_bias_" + s))
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_ordered_with_mask(seed):
+    """Scans along a random order of the positions with a random token mask
+    (keep rate drawn too), one direction or both."""
+    dtype, Bz, L, D, N, f = _draw(4000 + seed, max_elems=1_500_000)
+    rng = np.random.default_rng(seed)
+    inp = ssm_gen.make_s6_inputs(Bz, L, D, N, dtype=dtype, bidir=True, seed=seed, gate=f["gate"],
+                                 random_A=True, random_D=True)
+    order = rng.permutation(L).astype(np.int32)
+    mask = (rng.random((Bz, L)) < rng.uniform(0.3, 1.0)).astype(np.uint8)
+    x, dl = dev(inp.x, dtype), dev(inp.delta, dtype)
+    o_d, m_d = torch.from_numpy(order).cuda(), torch.from_numpy(mask).cuda()
+    if f["bidir"]:
+        out = ssm.bidir_scan_fwd_ordered(x, dl, _dirparams(inp, "f", dtype, f, Bz, D, N),
+                                         _dirparams(inp, "b", dtype, f, Bz, D, N), order=o_d, mask=m_d)
+        torch.cuda.synchronize()
+        ref = oracle.bidir_ordered_arrays(inp.x, inp.delta, _oracle_dir(inp, "f", f), _oracle_dir(inp, "b", f),
+                                          order=order, mask=mask, nthreads=NTHREADS)[0]
+    else:
+        p = _dirparams(inp, "f", dtype, f, Bz, D, N)
+        out = ssm.ssm_scan_fwd_ordered(x, dl, p.A, p.B, p.C, order=o_d, mask=m_d, delta_bias=p.delta_bias,
+                                       D=p.D, z=p.z, reverse=f["reverse"])
+        torch.cuda.synchronize()
+        q = _oracle_dir(inp, "f", f)
+        ref = oracle.s6_ordered_arrays(inp.x, inp.delta, q["A"], q["B"], q["C"], order=order, mask=mask,
+                                       delta_bias=q["delta_bias"], D=q["D"], z=q["z"], reverse=f["reverse"],
+                                       nthreads=NTHREADS)[0]
+    ssm.check_device()
+    assert rel_err(host(out), ref) <= TOL[dtype], (dtype, Bz, L, D, N, f)
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_conv_prologue(seed):
+    """Scans of u = act(conv1d(x_in)) with a random width (1-4), bias and
+    SiLU flag per direction."""
+    dtype, Bz, L, D, N, f = _draw(5000 + seed, max_elems=1_500_000)
+    rng = np.random.default_rng(seed)
+    inp = ssm_gen.make_s6_inputs(Bz, L, D, N, dtype=dtype, bidir=True, seed=seed, gate=f["gate"],
+                                 random_A=True, random_D=True)
+
+    def conv():
+        K = int(rng.integers(1, 5))
+        w = (rng.standard_normal((D, K)) / 2).astype(np.float32)
+        b = rng.standard_normal(D).astype(np.float32) if rng.random() < 0.5 else None
+        silu = bool(rng.random() < 0.7)
+        return dict(weight=w, bias=b, silu=silu), ssm.Conv(weight=f32dev(w), bias=f32dev(b), silu=silu)
+
+    cf, cf_d = conv()
+    cb, cb_d = conv()
+    x, dl = dev(inp.x, dtype), dev(inp.delta, dtype)
+    if f["bidir"]:
+        out = ssm.bidir_scan_fwd_conv(x, dl, _dirparams(inp, "f", dtype, f, Bz, D, N),
+                                      _dirparams(inp, "b", dtype, f, Bz, D, N), cf_d, cb_d)
+        torch.cuda.synchronize()
+        ref = oracle.bidir_conv_arrays(inp.x, inp.delta, _oracle_dir(inp, "f", f), _oracle_dir(inp, "b", f),
+                                       cf, cb, nthreads=NTHREADS)[0]
+    else:
+        p = _dirparams(inp, "f", dtype, f, Bz, D, N)
+        out = ssm.ssm_scan_fwd_conv(x, cf_d, dl, p.A, p.B, p.C, delta_bias=p.delta_bias, D=p.D, z=p.z,
+                                    reverse=f["reverse"])
+        torch.cuda.synchronize()
+        q = _oracle_dir(inp, "f", f)
+        ref = oracle.s6_conv_arrays(inp.x, cf["weight"], inp.delta, q["A"], q["B"], q["C"], conv_bias=cf["bias"],
+                                    conv_silu=cf["silu"], reverse=f["reverse"], delta_bias=q["delta_bias"],
+                                    D=q["D"], z=q["z"], nthreads=NTHREADS)[0]
+    assert rel_err(host(out), ref) <= TOL[dtype], (dtype, Bz, L, D, N, f)
+
+
+@pytest.mark.parametrize("seed", range(10))
+def test_checkpointing_training_pair(seed):
+    """bidir_scan_fwd_ckpt's output against the oracle, then
+    bidir_scan_bwd_ckpt from its checkpoints against the autograd oracle."""
+    dtype, Bz, L, D, N, f = _draw(6000 + seed, max_elems=600_000)
+    inp = ssm_gen.make_s6_inputs(Bz, L, D, N, dtype=dtype, bidir=True, seed=seed, gate=f["gate"],
+                                 random_A=True, random_D=True)
+    dout = np.random.default_rng(seed).standard_normal(inp.x.shape).astype(np.float32)
+    if dtype == "bf16":
+        dout = ssm_gen.round_to_bf16(dout)
+    x, dl = dev(inp.x, dtype), dev(inp.delta, dtype)
+    pf, pb = _dirparams(inp, "f", dtype, f, Bz, D, N), _dirparams(inp, "b", dtype, f, Bz, D, N)
+    out, ckf, ckb = ssm.bidir_scan_fwd_ckpt(x, dl, pf, pb)
+    dx, ddelta, gf, gb = ssm.bidir_scan_bwd_ckpt(x, dl, pf, pb, dev(dout, dtype), ckf, ckb)
+    torch.cuda.synchronize()
+    fw, bw = _oracle_dir(inp, "f", f), _oracle_dir(inp, "b", f)
+    ref = oracle.bidir_arrays(inp.x, inp.delta, fw, bw, nthreads=NTHREADS)[0]
+    tol = TOL[dtype]
+    assert rel_err(host(out), ref) <= tol
+    rg = ograds.bidir_grads(inp.x, inp.delta, fw, bw, dout)
+    assert rel_err(dx.cpu().numpy(), rg["x"]) <= tol
+    assert rel_err(ddelta.cpu().numpy(), rg["delta"]) <= tol
+    names = {"dA": "A", "dB": "B", "dC": "C", "dD": "D", "dz": "z", "ddelta_bias": "delta_bias"}
+    for g, side in ((gf, "fwd"), (gb, "bwd")):
+        for k, t in g.items():
+            assert rel_err(t.cpu().numpy(), rg[side][names[k]]) <= tol, (side, k)
+
+
+@pytest.mark.parametrize("seed", range(10))
+def test_zero_order_hold(seed):
+    dtype, Bz, L, D, N, f = _draw(7000 + seed, max_elems=1_500_000)
+    N = 16
+    inp = ssm_gen.make_s6_inputs(Bz, L, D, N, dtype=dtype, bidir=True, seed=seed, gate=f["gate"],
+                                 random_A=True, random_D=True)
+    x, dl = dev(inp.x, dtype), dev(inp.delta, dtype)
+    if f["bidir"]:
+        out = ssm.bidir_scan_fwd_zoh(x, dl, _dirparams(inp, "f", dtype, f, Bz, D, N),
+                                     _dirparams(inp, "b", dtype, f, Bz, D, N))
+        torch.cuda.synchronize()
+        ref = oracle.bidir_arrays(inp.x, inp.delta, _oracle_dir(inp, "f", f), _oracle_dir(inp, "b", f), zoh=True,
+                                  nthreads=NTHREADS)[0]
+    else:
+        h0 = np.random.default_rng(seed).standard_normal((Bz, D, N)).astype(np.float32)
+        p = _dirparams(inp, "f", dtype, f, Bz, D, N)
+        out = ssm.ssm_scan_fwd_zoh(x, dl, p.A, p.B, p.C, delta_bias=p.delta_bias, D=p.D, z=p.z,
+                                   reverse=f["reverse"], initial_state=f32dev(h0))
+        torch.cuda.synchronize()
+        q = _oracle_dir(inp, "f", f)
+        ref = oracle.s6_arrays(inp.x, inp.delta, q["A"], q["B"], q["C"], delta_bias=q["delta_bias"], D=q["D"],
+                               z=q["z"], reverse=f["reverse"], initial_state=h0, zoh=True, nthreads=NTHREADS)[0]
+    assert rel_err(host(out), ref) <= TOL[dtype], (dtype, Bz, L, D, N, f)
+
+
+@pytest.mark.parametrize("seed", range(10))
+def test_decode_step(seed):
+    rng = np.random.default_rng(8000 + seed)
+    dtype = "f32" if rng.random() < 0.5 else "bf16"
+    vec = 4 if dtype == "f32" else 8
+    Bz, D, N = int(rng.integers(1, 300)), vec * int(rng.integers(1, 200)), int(rng.integers(1, 17))
+    gate, skip = bool(rng.random() < 0.7), bool(rng.random() < 0.7)
+    inp = ssm_gen.make_s6_inputs(Bz, 1, D, N, dtype=dtype, seed=seed, gate=gate, random_A=True, random_D=True)
+    state0 = rng.standard_normal((Bz, D, N)).astype(np.float32)
+    state = f32dev(state0)
+    y = ssm.ssm_step(dev(inp.x[:, 0], dtype), dev(inp.delta[:, 0], dtype), f32dev(inp.A_f),
+                     dev(inp.B_f[:, 0], dtype), dev(inp.C_f[:, 0], dtype), state, delta_bias=f32dev(inp.dt_bias_f),
+                     D=f32dev(inp.D_f) if skip else None, z=dev(inp.z_f[:, 0], dtype) if gate else None)
+    torch.cuda.synchronize()
+    ry, rst = oracle.step_arrays(inp.x[:, 0], inp.delta[:, 0], inp.A_f, inp.B_f[:, 0], inp.C_f[:, 0], state0,
+                                 delta_bias=inp.dt_bias_f, D=inp.D_f if skip else None,
+                                 z=inp.z_f[:, 0] if gate else None)
+    assert rel_err(host(y), ry) <= TOL[dtype], (dtype, Bz, D, N, gate, skip)
+    assert rel_err(state.cpu().numpy(), rst) <= TOL[dtype]
