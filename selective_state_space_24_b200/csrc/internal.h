@@ -63,6 +63,8 @@ struct S6Args {
     int split;                   // 2 or 4: that many threads per channel (s6_split.cu); needs
                                  // N == 16, S == 1, and none of order / mask / conv
     int zoh;                     // 1: the exact zero-order-hold input coefficient (needs split)
+    int mix_rows2;               // split == 2 and 0 < mix_rows2 < Bsz: rows [mix_rows2, Bsz) take
+                                 // four threads per channel in the same launch
 };
 
 struct S6Plan {
@@ -84,6 +86,9 @@ cudaError_t launch_s6(const S6Args &a, cudaStream_t stream);
 // kernels), and its launcher.  It needs no workspace beyond the
 // bidirectional bf16 stash of plan_s6.
 int split_threads(int64_t Bsz, int64_t L, int64_t D, int64_t N, int ndir);
+// With two threads per channel: how many leading batch rows keep it when
+// the rest take four threads per channel in the same launch (0: all keep it).
+int split_mix_rows(int64_t Bsz, int64_t D, int ndir);
 cudaError_t launch_s6_split(const S6Args &a, cudaStream_t stream);
 // The same kernel as the backward's checkpoint pass: one direction (a.dir[0],
 // a.reverse), a.split threads per channel, only dir[0].ckpt written (the

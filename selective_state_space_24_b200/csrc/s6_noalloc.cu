@@ -127,6 +127,8 @@ extern "C" SSM_API ssm_status ssm_scan_fwd_noalloc(const ssm_dims *dims, const v
     a.dir[0] = ssm::DirArgs{delta_bias, A, B, C, D, z, last_state};
     a.out = out;
     a.split = split;
+    if (split == 2)   // the same launch ssm_scan_fwd makes
+        a.mix_rows2 = ssm::split_mix_rows(dims->batch, dims->dim, 1);
     if (a.S > 1) {
         char *w = static_cast<char *>(scratch);
         a.carry_h = reinterpret_cast<float *>(w + plan.carry_h_off);

@@ -244,8 +244,10 @@ template <Mode M> using ModeTag = std::integral_constant<Mode, M>;
 // step computes anyway would lose its leading digits for small dt a, so
 // there (|dt a| < 1/16) the coefficient is dt (1 + w / 2 + w^2 / 6 +
 // w^3 / 24), w = dt a, whose truncation error is below 1.3e-7 relative.
-template <typename T, int Q, bool BIDIR, bool GATE, bool SOFTPLUS, bool OUT = true, bool ZOH = false>
-__global__ void __launch_bounds__(64, min_blocks<Q, ZOH>()) s6_split_kernel(const S6Args a)
+// The body of one CTA: channel block bx (its warp pair's channels) of
+// batch row b.
+template <typename T, int Q, bool BIDIR, bool GATE, bool SOFTPLUS, bool OUT, bool ZOH>
+__device__ __forceinline__ void split_body(const S6Args &a, WarpSmem<T, GATE, BIDIR, Q> *smem, int bx, int b)
 {
     static_assert(Q == 2 || Q == 4, "two or four threads per channel");
     using S = Slot<T, GATE, BIDIR, Q>;
@@ -253,13 +255,11 @@ __global__ void __launch_bounds__(64, min_blocks<Q, ZOH>()) s6_split_kernel(cons
     constexpr int NQ = 16 / Q;          // states per thread
     constexpr int NP = NQ / 2;          // state pairs per thread
     constexpr int SPL = kG / Q;         // steps of a group whose scalars a thread computes
-    __shared__ WarpSmem<T, GATE, BIDIR, Q> smem[2];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     WarpSmem<T, GATE, BIDIR, Q> &sm = smem[warp];
     const int g = lane / Q, q = lane % Q;
     const int dsel = BIDIR ? warp : 0;
-    const int d0 = (BIDIR ? (int)blockIdx.x : (int)blockIdx.x * 2 + warp) * kChW;   // the warp's first channel
-    const int b = blockIdx.y;
+    const int d0 = (BIDIR ? bx : bx * 2 + warp) * kChW;   // the warp's first channel
     const int L = a.L, D = a.D;
     if (!BIDIR && d0 >= D)
         return;   // whole warp past the channels (no barrier partner in this mode)
@@ -565,6 +565,35 @@ __global__ void __launch_bounds__(64, min_blocks<Q, ZOH>()) s6_split_kernel(cons
     }
 }
 
+template <typename T, int Q, bool BIDIR, bool GATE, bool SOFTPLUS, bool OUT = true, bool ZOH = false>
+__global__ void __launch_bounds__(64, min_blocks<Q, ZOH>()) s6_split_kernel(const S6Args a)
+{
+    __shared__ WarpSmem<T, GATE, BIDIR, Q> smem[2];
+    split_body<T, Q, BIDIR, GATE, SOFTPLUS, OUT, ZOH>(a, smem, (int)blockIdx.x, (int)blockIdx.y);
+}
+
+// Two threads per channel for batch rows [0, a.mix_rows2), four for the
+// rest, in one launch (1-D grid, the two-thread CTAs first): the
+// half-width four-thread CTAs dispatched last even out the work left on
+// the SM sub-partitions at the end of the launch.
+template <typename T, bool BIDIR, bool GATE, bool SOFTPLUS>
+__global__ void __launch_bounds__(64, min_blocks<2>()) s6_split_mixed_kernel(const S6Args a)
+{
+    using W2 = WarpSmem<T, GATE, BIDIR, 2>;
+    using W4 = WarpSmem<T, GATE, BIDIR, 4>;
+    __shared__ __align__(16) char smem[sizeof(W2) > sizeof(W4) ? 2 * sizeof(W2) : 2 * sizeof(W4)];
+    const int nx2 = BIDIR ? (a.D + 15) / 16 : (a.D + 31) / 32, nx4 = BIDIR ? (a.D + 7) / 8 : (a.D + 15) / 16;
+    const long long n2 = (long long)a.mix_rows2 * nx2, bid = blockIdx.x;
+    if (bid < n2) {
+        split_body<T, 2, BIDIR, GATE, SOFTPLUS, true, false>(a, reinterpret_cast<W2 *>(smem), (int)(bid % nx2),
+                                                           (int)(bid / nx2));
+    } else {
+        const long long r = bid - n2;
+        split_body<T, 4, BIDIR, GATE, SOFTPLUS, true, false>(a, reinterpret_cast<W4 *>(smem), (int)(r % nx4),
+                                                           a.mix_rows2 + (int)(r / nx4));
+    }
+}
+
 template <typename T, int Q, bool GATE, bool SOFTPLUS, bool ZOH>
 cudaError_t launch_q(const S6Args &a, cudaStream_t st)
 {
@@ -582,6 +611,16 @@ cudaError_t launch_q(const S6Args &a, cudaStream_t st)
 template <typename T, bool GATE, bool SOFTPLUS, bool ZOH>
 cudaError_t launch_t(const S6Args &a, cudaStream_t st)
 {
+    if (!ZOH && a.split == 2 && a.mix_rows2 > 0 && a.mix_rows2 < a.Bsz) {
+        const bool bidir = a.ndir == 2;
+        const long long nx2 = bidir ? (a.D + 15) / 16 : (a.D + 31) / 32, nx4 = bidir ? (a.D + 7) / 8 : (a.D + 15) / 16;
+        const unsigned grid = (unsigned)(a.mix_rows2 * nx2 + (long long)(a.Bsz - a.mix_rows2) * nx4);
+        if (bidir)
+            s6_split_mixed_kernel<T, true, GATE, SOFTPLUS><<<grid, 64, 0, st>>>(a);
+        else
+            s6_split_mixed_kernel<T, false, GATE, SOFTPLUS><<<grid, 64, 0, st>>>(a);
+        return cudaGetLastError();
+    }
     return a.split == 2 ? launch_q<T, 2, GATE, SOFTPLUS, ZOH>(a, st) : launch_q<T, 4, GATE, SOFTPLUS, ZOH>(a, st);
 }
 
@@ -639,6 +678,33 @@ int split_threads(int64_t Bsz, int64_t L, int64_t D, int64_t N, int ndir)
     if (t1 <= t4 && t1 <= t2)
         return 0;
     return t2 < t4 ? 2 : 4;
+}
+
+#ifndef SSM_S6_SPLIT_MIX
+#define SSM_S6_SPLIT_MIX 1
+#endif
+int split_mix_rows(int64_t Bsz, int64_t D, int ndir)
+{
+    if (!SSM_S6_SPLIT_MIX)
+        return 0;
+    // The launch takes about as long as its busiest SM sub-partition's
+    // warps (each CTA is 2 warps): ceil(warps / 592) of them.  Rows moved
+    // to four threads per channel become twice the warps at about 0.57 of
+    // the cost each, and being dispatched last they fill the sub-partitions
+    // left short; mix only when the mean load then ends well below that
+    // ceiling.
+    constexpr int64_t kSubPartitions = 148 * 4;
+    constexpr double kQ4Warp = 0.57, kSlack = 0.3;
+    const int64_t nx2 = ndir == 2 ? (D + 15) / 16 : (D + 31) / 32;   // CTAs (2 warps each) per batch row
+    const int64_t nx4 = ndir == 2 ? (D + 7) / 8 : (D + 15) / 16;
+    const int64_t warps = 2 * Bsz * nx2, levels = warps / kSubPartitions;
+    if (levels == 0 || warps % kSubPartitions == 0)
+        return 0;
+    const int64_t rows2 = levels * kSubPartitions / (2 * nx2);   // these fill `levels` exactly or less
+    if (rows2 <= 0 || rows2 >= Bsz)
+        return 0;
+    const double mean = (2.0 * rows2 * nx2 + kQ4Warp * 2.0 * (Bsz - rows2) * nx4) / kSubPartitions;
+    return mean + kSlack < (double)(levels + 1) ? (int)rows2 : 0;
 }
 
 void split_mode_set(int mode) { g_split_mode.store(mode, std::memory_order_relaxed); }

@@ -158,9 +158,10 @@ def test_layouts_agree_at_full_size(dtype, bidir, batch, L, D):
     assert rel_err(host(split[0])[bb, :, dd], ref[bb, :, dd]) <= tol
 
 
-def test_noalloc_takes_the_same_layout():
+@pytest.mark.parametrize("batch,L,D", [(4, 120, 256), (100, 40, 768)])   # the second mixes rows
+def test_noalloc_takes_the_same_layout(batch, L, D):
     """ssm_scan_fwd_noalloc takes the layout ssm_scan_fwd takes: bit for bit."""
-    inp = ssm_gen.make_s6_inputs(4, 120, 256, 16, dtype="f32", seed=5, random_A=True, random_D=True)
+    inp = ssm_gen.make_s6_inputs(batch, L, D, 16, dtype="f32", seed=5, random_A=True, random_D=True)
     x, delta = dev(inp.x, "f32"), dev(inp.delta, "f32")
     A, B, C = f32dev(inp.A_f), dev(inp.B_f, "f32"), dev(inp.C_f, "f32")
     kw = dict(delta_bias=f32dev(inp.dt_bias_f), D=f32dev(inp.D_f), z=dev(inp.z_f, "f32"))
@@ -168,3 +169,25 @@ def test_noalloc_takes_the_same_layout():
     out = ssm.ssm_scan_fwd_noalloc(x, delta, A, B, C, **kw)
     torch.cuda.synchronize()
     assert torch.equal(out, ref)
+
+
+@pytest.mark.parametrize("dtype,bidir,batch,L,D", [("f32", True, 64, 60, 768), ("bf16", True, 62, 33, 768),
+                                                   ("f32", False, 13, 57, 768), ("bf16", False, 26, 41, 384)])
+def test_mixed_rows_in_one_launch(dtype, bidir, batch, L, D, threads):
+    """With two threads per channel, sizes whose warps overfill the last
+    round of the SM sub-partitions run their trailing batch rows with four
+    threads per channel in the same launch; every output and last state
+    against the oracle (under the four-thread setting these sizes run
+    unmixed)."""
+    inp = ssm_gen.make_s6_inputs(batch, L, D, 16, dtype=dtype, bidir=bidir, seed=batch + L, random_A=True,
+                                 random_D=True)
+    tol = TOL[dtype]
+    if bidir:
+        out, lf, lb = run_bidir(inp, last_state=True)
+        ref, rlf, rlb = oracle.bidir(inp, nthreads=NTHREADS)
+        assert rel_err(lf.cpu().numpy(), rlf) <= tol and rel_err(lb.cpu().numpy(), rlb) <= tol
+    else:
+        out, st = run_s6(inp, reverse=True)
+        ref, rst = oracle.s6(inp, reverse=True, nthreads=NTHREADS)
+        assert rel_err(st.cpu().numpy(), rst) <= tol
+    assert rel_err(host(out), ref) <= tol
