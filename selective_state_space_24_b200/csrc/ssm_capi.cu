@@ -124,7 +124,7 @@ ssm_status run_s6(const ssm_dims *dims, const void *x, const void *delta, int so
     }
     if (q) {
         a.split = q;   // one pass, q threads per channel
-        if (q == 2 && !zoh && !ckpt)
+        if (q == 2 && !zoh)   // (checkpoints are the same in either layout)
             a.mix_rows2 = ssm::split_mix_rows(dims->batch, dims->dim, ndir);
         a.S = 1;
         a.T = a.L;
