@@ -251,7 +251,9 @@ SSM_API ssm_status bidir_scan_fwd_zoh(const ssm_dims *dims, const void *x, const
  *   channels_per_lane  (out, may be NULL) 1 or 2: channels one GPU thread owns;
  *                      -2 or -4: that many threads share each channel, each
  *                      holding an equal share of its 16 states (one pass, no
- *                      segments; N = 16 only)
+ *                      segments; N = 16 only).  With -2 the last batch rows
+ *                      may take four threads per channel in the same launch,
+ *                      where that evens out the launch's last round of warps.
  * Host-only, makes no CUDA call.  Returns the status the scan entry points
  * give for invalid dims; an empty problem reports 1 segment.
  */
