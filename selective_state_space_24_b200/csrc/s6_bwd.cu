@@ -512,6 +512,8 @@ cudaError_t launch_ns(const BwdArgs &a, cudaStream_t st)
             f.Bsz = a.Bsz, f.L = a.L, f.D = a.D, f.N = a.N, f.S = 1, f.T = a.L;
             f.dtype = a.dtype, f.softplus = a.softplus, f.ndir = 1, f.reverse = a.reverse;
             f.x = a.x, f.delta = a.delta, f.split = q;
+            if (q == 2)
+                f.mix_rows2 = split_mix_rows(a.Bsz, a.D, 1);
             f.dir[0].bias = a.bias, f.dir[0].A = a.A, f.dir[0].B = a.B, f.dir[0].C = a.C;
             f.dir[0].ckpt = a.ckpt;
             if ((e = launch_s6_split_ckpt_only(f, st)) != cudaSuccess)

@@ -576,7 +576,7 @@ __global__ void __launch_bounds__(64, min_blocks<Q, ZOH>()) s6_split_kernel(cons
 // rest, in one launch (1-D grid, the two-thread CTAs first): the
 // half-width four-thread CTAs dispatched last even out the work left on
 // the SM sub-partitions at the end of the launch.
-template <typename T, bool BIDIR, bool GATE, bool SOFTPLUS>
+template <typename T, bool BIDIR, bool GATE, bool SOFTPLUS, bool OUT = true>
 __global__ void __launch_bounds__(64, min_blocks<2>()) s6_split_mixed_kernel(const S6Args a)
 {
     using W2 = WarpSmem<T, GATE, BIDIR, 2>;
@@ -585,12 +585,12 @@ __global__ void __launch_bounds__(64, min_blocks<2>()) s6_split_mixed_kernel(con
     const int nx2 = BIDIR ? (a.D + 15) / 16 : (a.D + 31) / 32, nx4 = BIDIR ? (a.D + 7) / 8 : (a.D + 15) / 16;
     const long long n2 = (long long)a.mix_rows2 * nx2, bid = blockIdx.x;
     if (bid < n2) {
-        split_body<T, 2, BIDIR, GATE, SOFTPLUS, true, false>(a, reinterpret_cast<W2 *>(smem), (int)(bid % nx2),
-                                                           (int)(bid / nx2));
+        split_body<T, 2, BIDIR, GATE, SOFTPLUS, OUT, false>(a, reinterpret_cast<W2 *>(smem), (int)(bid % nx2),
+                                                          (int)(bid / nx2));
     } else {
         const long long r = bid - n2;
-        split_body<T, 4, BIDIR, GATE, SOFTPLUS, true, false>(a, reinterpret_cast<W4 *>(smem), (int)(r % nx4),
-                                                           a.mix_rows2 + (int)(r / nx4));
+        split_body<T, 4, BIDIR, GATE, SOFTPLUS, OUT, false>(a, reinterpret_cast<W4 *>(smem), (int)(r % nx4),
+                                                          a.mix_rows2 + (int)(r / nx4));
     }
 }
 
@@ -636,6 +636,15 @@ cudaError_t launch_ckpt_q(const S6Args &a, cudaStream_t st)
 template <typename T>
 cudaError_t launch_ckpt_t(const S6Args &a, cudaStream_t st)
 {
+    if (a.split == 2 && a.mix_rows2 > 0 && a.mix_rows2 < a.Bsz) {   // the mixed launch, as for the scans
+        const unsigned grid = (unsigned)((long long)a.mix_rows2 * ((a.D + 31) / 32) +
+                                         (long long)(a.Bsz - a.mix_rows2) * ((a.D + 15) / 16));
+        if (a.softplus)
+            s6_split_mixed_kernel<T, false, false, true, false><<<grid, 64, 0, st>>>(a);
+        else
+            s6_split_mixed_kernel<T, false, false, false, false><<<grid, 64, 0, st>>>(a);
+        return cudaGetLastError();
+    }
     if (a.split == 2)
         return a.softplus ? launch_ckpt_q<T, 2, true>(a, st) : launch_ckpt_q<T, 2, false>(a, st);
     return a.softplus ? launch_ckpt_q<T, 4, true>(a, st) : launch_ckpt_q<T, 4, false>(a, st);
