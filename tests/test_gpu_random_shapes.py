@@ -289,3 +289,27 @@ def test_decode_step(seed):
                                  z=inp.z_f[:, 0] if gate else None)
     assert rel_err(host(y), ry) <= TOL[dtype], (dtype, Bz, D, N, gate, skip)
     assert rel_err(state.cpu().numpy(), rst) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_many_warp_sizes(seed):
+    """Batches large enough that the plan gives two threads per channel and
+    often mixes in four-thread rows at the end of the launch (short
+    sequences keep the oracle quick); every output against the oracle."""
+    rng = np.random.default_rng(9000 + seed)
+    dtype = "f32" if rng.random() < 0.5 else "bf16"
+    Bz, L = int(rng.integers(40, 130)), int(rng.integers(1, 50))
+    D = int(rng.choice([384, 512, 768]))
+    bidir = bool(rng.random() < 0.6)
+    inp = ssm_gen.make_s6_inputs(Bz, L, D, 16, dtype=dtype, bidir=bidir, seed=seed, random_A=True, random_D=True)
+    from gpu_util import run_bidir, run_s6
+    tol = TOL[dtype]
+    if bidir:
+        out, lf, lb = run_bidir(inp, last_state=True)
+        ref, rlf, rlb = oracle.bidir(inp, nthreads=NTHREADS)
+        assert rel_err(lf.cpu().numpy(), rlf) <= tol and rel_err(lb.cpu().numpy(), rlb) <= tol
+    else:
+        out, st = run_s6(inp, reverse=bool(seed % 2))
+        ref, rst = oracle.s6(inp, reverse=bool(seed % 2), nthreads=NTHREADS)
+        assert rel_err(st.cpu().numpy(), rst) <= tol
+    assert rel_err(host(out), ref) <= tol, (dtype, Bz, L, D, bidir)
