@@ -60,12 +60,20 @@ constexpr int kStages = 4;             // groups in the copy ring (a power of tw
 #ifndef SSM_S6_SPLIT_MINB2
 #define SSM_S6_SPLIT_MINB2 10
 #endif
+#ifndef SSM_S6_SPLIT_MINB2_PAIR
+#define SSM_S6_SPLIT_MINB2_PAIR 8
+#endif
 // CTAs per SM by threads per channel (two threads per channel hold 8
-// states each and need more registers); the zero-order-hold variants keep
-// 1 / A of their states as well
-template <int Q, bool ZOH = false> constexpr int min_blocks()
+// states each and need more registers: single direction 10 CTAs of 96
+// registers; the pair's exchange adds more, and its 8 CTAs of up to 128
+// registers measured 3-9% faster -- Vim-Small 131.1 -> 125.0 us, its
+// checkpointing forward 149.6 -> 136.3, B 48 bf16 107.5 -> 102.4 -- while
+// a single direction at 8 lost 2%); the zero-order-hold variants keep 1 / A
+// of their states as well
+template <int Q, bool ZOH = false, bool BIDIR = false> constexpr int min_blocks()
 {
-    return ZOH ? (Q == 2 ? 8 : 10) : (Q == 2 ? SSM_S6_SPLIT_MINB2 : SSM_S6_SPLIT_MINB);
+    return ZOH ? (Q == 2 ? 8 : 10)
+               : (Q == 2 ? (BIDIR ? SSM_S6_SPLIT_MINB2_PAIR : SSM_S6_SPLIT_MINB2) : SSM_S6_SPLIT_MINB);
 }
 static_assert((kStages & (kStages - 1)) == 0, "ring index by mask");
 // Which layout the plain calls take (split_threads).  The one-thread-per-
@@ -566,7 +574,7 @@ __device__ __forceinline__ void split_body(const S6Args &a, WarpSmem<T, GATE, BI
 }
 
 template <typename T, int Q, bool BIDIR, bool GATE, bool SOFTPLUS, bool OUT = true, bool ZOH = false>
-__global__ void __launch_bounds__(64, min_blocks<Q, ZOH>()) s6_split_kernel(const S6Args a)
+__global__ void __launch_bounds__(64, min_blocks<Q, ZOH, BIDIR>()) s6_split_kernel(const S6Args a)
 {
     __shared__ WarpSmem<T, GATE, BIDIR, Q> smem[2];
     split_body<T, Q, BIDIR, GATE, SOFTPLUS, OUT, ZOH>(a, smem, (int)blockIdx.x, (int)blockIdx.y);
@@ -577,7 +585,7 @@ __global__ void __launch_bounds__(64, min_blocks<Q, ZOH>()) s6_split_kernel(cons
 // half-width four-thread CTAs dispatched last even out the work left on
 // the SM sub-partitions at the end of the launch.
 template <typename T, bool BIDIR, bool GATE, bool SOFTPLUS, bool OUT = true>
-__global__ void __launch_bounds__(64, min_blocks<2>()) s6_split_mixed_kernel(const S6Args a)
+__global__ void __launch_bounds__(64, min_blocks<2, false, BIDIR>()) s6_split_mixed_kernel(const S6Args a)
 {
     using W2 = WarpSmem<T, GATE, BIDIR, 2>;
     using W4 = WarpSmem<T, GATE, BIDIR, 4>;
