@@ -48,7 +48,7 @@ SMS = 148
 # DRAM bytes (read + write) per launch of the dominant kernel, from one ncu
 # capture of the current kernels (summaries under profiles/); absent where no
 # capture matches them.
-NCU_TRAFFIC = {1: 221.53e6, 4: 397.22e6}
+NCU_TRAFFIC = {1: 193.52e6, 4: 397.22e6}
 NCU_TRAFFIC_STEP = 62.01e6
 NCU_TRAFFIC_BWD = {1: 408.07e6}
 
