@@ -63,17 +63,23 @@ constexpr int kStages = 4;             // groups in the copy ring (a power of tw
 #ifndef SSM_S6_SPLIT_MINB2_PAIR
 #define SSM_S6_SPLIT_MINB2_PAIR 8
 #endif
-// CTAs per SM by threads per channel (two threads per channel hold 8
-// states each and need more registers: single direction 10 CTAs of 96
-// registers; the pair's exchange adds more, and its 8 CTAs of up to 128
-// registers measured 3-9% faster -- Vim-Small 131.1 -> 125.0 us, its
-// checkpointing forward 149.6 -> 136.3, B 48 bf16 107.5 -> 102.4 -- while
-// a single direction at 8 lost 2%); the zero-order-hold variants keep 1 / A
-// of their states as well
+#ifndef SSM_S6_SPLIT_MINB_PAIR
+#define SSM_S6_SPLIT_MINB_PAIR 8
+#endif
+// CTAs per SM by threads per channel and direction.  Two threads per
+// channel hold 8 states each and need more registers: a single direction
+// at 10 CTAs (96 registers); the pair's exchange adds more, and its 8 CTAs
+// of up to 128 registers measured 3-9% faster -- Vim-Small 131.1 -> 125.0
+// us, its checkpointing forward 149.6 -> 136.3, B 48 bf16 107.5 -> 102.4 --
+// while a single direction at 8 lost 2%.  Four threads per channel: a
+// single direction at 12 (80 registers; 8 lost 7%), the pair at 8 (B 8,
+// L 1024, D 768 bf16 144 -> 133 us; B 4, L 512 fp32 61.4 -> 55.3).  The
+// zero-order-hold variants keep 1 / A of their states as well.
 template <int Q, bool ZOH = false, bool BIDIR = false> constexpr int min_blocks()
 {
     return ZOH ? (Q == 2 ? 8 : 10)
-               : (Q == 2 ? (BIDIR ? SSM_S6_SPLIT_MINB2_PAIR : SSM_S6_SPLIT_MINB2) : SSM_S6_SPLIT_MINB);
+               : (Q == 2 ? (BIDIR ? SSM_S6_SPLIT_MINB2_PAIR : SSM_S6_SPLIT_MINB2)
+                         : (BIDIR ? SSM_S6_SPLIT_MINB_PAIR : SSM_S6_SPLIT_MINB));
 }
 static_assert((kStages & (kStages - 1)) == 0, "ring index by mask");
 // Which layout the plain calls take (split_threads).  The one-thread-per-
