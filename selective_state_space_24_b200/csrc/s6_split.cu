@@ -1,7 +1,13 @@
 // s6_split.cu -- the S6 scan (single direction, or the Vision-Mamba pair of
 // directions of "复现Vision Mamba", sec. 3.1 - 3.2) with each channel's 16
-// states split over four threads, for problems with enough channels to
-// keep every SM sub-partition full of warps.
+// states split over Q = 4 threads (described below) or Q = 2 threads (8
+// channels a warp becomes 16, 8 states a thread; thread q then does the
+// scalar work of steps q and q + 2).  The plan (split_threads) picks Q or
+// the one-or-two-channels-per-thread kernels by size; with Q = 2 the last
+// batch rows may run with Q = 4 in the same launch (split_mix_rows), which
+// evens out the launch's last round of warps.  The same kernel body also
+// serves the checkpointing forwards, the backward's checkpoint pass (no
+// outputs) and the exact zero-order-hold scans.
 //
 // Step (Mamba2 page "手写简化版Mamba2", sec. 4.3 - 4.4), per (b, d):
 //     dt = softplus(delta + bias),  h[n] = exp(dt A[n]) h[n] + dt B[n] x,
@@ -27,8 +33,8 @@
 // its outputs (in its own scan order) in `stash`, the pair meets at a named
 // barrier, and each then adds the partner's parked value to the second half
 // of its outputs: out is written once and no step is computed twice.  x
-// and delta are read by both warps; the first half's copies ask L2 to keep
-// them for the partner.
+// and delta are read by both warps (and stay in L2 for the partner: the
+// problems these layouts take fit in it).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
