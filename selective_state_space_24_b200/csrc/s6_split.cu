@@ -83,7 +83,7 @@ constexpr int kStages = 4;             // groups in the copy ring (a power of tw
 // zero-order-hold variants keep 1 / A of their states as well.
 template <int Q, bool ZOH = false, bool BIDIR = false> constexpr int min_blocks()
 {
-    return ZOH ? (Q == 2 ? 8 : 10)
+    return ZOH ? (Q == 2 || BIDIR ? 8 : 10)
                : (Q == 2 ? (BIDIR ? SSM_S6_SPLIT_MINB2_PAIR : SSM_S6_SPLIT_MINB2)
                          : (BIDIR ? SSM_S6_SPLIT_MINB_PAIR : SSM_S6_SPLIT_MINB));
 }
