@@ -730,8 +730,8 @@ int split_mix_rows(int64_t Bsz, int64_t D, int ndir)
     if (levels == 0 || warps % kSubPartitions == 0)
         return 0;
     const int64_t rows2 = levels * kSubPartitions / (2 * nx2);   // these fill `levels` exactly or less
-    if (rows2 <= 0 || rows2 >= Bsz)
-        return 0;
+    if (rows2 <= 0 || rows2 >= Bsz || rows2 * nx2 + (Bsz - rows2) * nx4 > 0x7fffffff)
+        return 0;   // (the mixed launch's grid is one-dimensional)
     const double mean = (2.0 * rows2 * nx2 + kQ4Warp * 2.0 * (Bsz - rows2) * nx4) / kSubPartitions;
     return mean + kSlack < (double)(levels + 1) ? (int)rows2 : 0;
 }
